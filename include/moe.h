@@ -1,0 +1,164 @@
+/*
+ * moe.h -- C ABI of libmoe.so, a B200 (sm_100a) implementation of the sparse
+ * Mixture-of-Experts block of the Qwen3.x hybrid models.
+ *
+ * The block (one per layer; "Vue d'ensemble" page of the Qwen3.8-Max report,
+ * section "Le motif": every layer ends in a MoE block), per token x of width d:
+ *   1. a linear router scores the E experts            (Qwen3.6 explainer page,
+ *   2. softmax over the E scores, keep the k largest    router paragraphs)
+ *   3. renormalise the k kept probabilities to sum to 1
+ *   4. each kept expert is a SwiGLU MLP                 ("Architecture" page,
+ *        E_e(x) = W_down[e] (SiLU(W_gate[e] x) * (W_up[e] x))   config.json keys
+ *      with intermediate width I                        hidden_act = silu,
+ *                                                       moe_intermediate_size)
+ *   5. one shared SwiGLU expert of width I_s is always  (Qwen3.6 explainer: one
+ *      added with weight 1                              "shared" expert always on;
+ *                                                       shared_expert_intermediate_size)
+ *   y = sum_{e kept} w_e E_e(x) + S(x).
+ *
+ * Conventions for every entry point
+ *   - All tensor pointers are DEVICE pointers into contiguous row-major
+ *     buffers that the caller allocates and owns.  The library never
+ *     allocates or frees device memory and never synchronises the stream.
+ *   - Work is enqueued asynchronously on `stream` (a cudaStream_t; NULL is the
+ *     legacy default stream).  A return of MOE_OK means the work was enqueued.
+ *   - Errors the host can see (bad sizes, NULL or misaligned pointers, a
+ *     workspace that is too small) are returned before anything is launched;
+ *     MOE_ERR_CUDA reports a launch error.  Faults the device sees (an expert
+ *     id out of range in moe_permute's input, a pipeline wait that timed out)
+ *     are recorded in a device status word that moe_device_status() reads.
+ *   - moe_last_error_string() describes the last non-OK status returned on
+ *     the calling thread.
+ *   - Weight layout is the linear-layer convention (out x in, row-major):
+ *       w_router [E, d] (activation type), w_gate [E, I, d], w_up [E, I, d],
+ *       w_down [E, d, I]; shared: ws_gate [I_s, d], ws_up [I_s, d],
+ *       ws_down [d, I_s].  I_s == 0 means no shared expert (ws_* ignored).
+ *   - Types: activations (x, x_perm, y_perm, y) are MOE_F32 or MOE_BF16;
+ *     weights are MOE_F32 (with F32 activations), MOE_BF16, or
+ *     MOE_FP8_E4M3_B128 (bf16 activations; E4M3 codes with one fp32 scale per
+ *     128 x 128 block: value = decode(q) * scale[row/128][col/128]).
+ *   - FP8 `scales` packs, in this order: gate [E][I/128][d/128], up (same),
+ *     down [E][d/128][I/128], shared gate [I_s/128][d/128], shared up (same),
+ *     shared down [d/128][I_s/128].  NULL for non-FP8 weights.
+ *   - Limits: 1 <= k <= min(E, 16); E <= 512; d, I, I_s multiples of 8
+ *     (multiples of 128 for FP8 weights); T >= 0 with T * (k + 1) < 2^31;
+ *     every pointer 16-byte aligned.
+ */
+#ifndef MOE_H
+#define MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,          /* a size, pointer or type is not allowed */
+  MOE_ERR_UNSUPPORTED = 2,          /* a valid combination this build does not implement */
+  MOE_ERR_ALIGNMENT = 3,            /* a pointer or a row stride is not 16-byte aligned */
+  MOE_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes below the *_workspace_size() figure */
+  MOE_ERR_CUDA = 5,                 /* a CUDA runtime call or a launch failed */
+  MOE_ERR_DEVICE_CHECK = 6,         /* device status: a kernel rejected its input */
+  MOE_ERR_TIMEOUT = 7               /* device status: a pipeline wait gave up */
+} moe_status;
+
+typedef enum { MOE_F32 = 0, MOE_BF16 = 1, MOE_FP8_E4M3_B128 = 2 } moe_dtype;
+
+/* Shapes of one block invocation.  R = T*k routed rows; R' = R + T (I_s > 0)
+ * or R (I_s == 0) dispatched rows. */
+typedef struct {
+  int64_t T;         /* tokens */
+  int32_t d;         /* hidden width */
+  int32_t E;         /* routed experts */
+  int32_t k;         /* experts kept per token */
+  int32_t I;         /* routed expert intermediate width */
+  int32_t I_s;       /* shared expert intermediate width, 0 = none */
+  int32_t act_dtype; /* moe_dtype of activations and of w_router */
+  int32_t w_dtype;   /* moe_dtype of expert weights */
+} moe_problem;
+
+/* Validate a problem on the host (no CUDA call).  MOE_OK or the reason. */
+MOE_API moe_status moe_check_problem(const moe_problem* p);
+
+/* Bytes of device workspace the calls below need (0 for an invalid problem).
+ * moe_workspace_size covers moe_layer_forward; moe_stage_workspace_size
+ * covers moe_permute and moe_expert_ffn.  Pure host functions. */
+MOE_API size_t moe_workspace_size(const moe_problem* p);
+MOE_API size_t moe_stage_workspace_size(const moe_problem* p);
+
+/* Router stage (steps 1-3).  x [T, d]; w_router [E, d]; router_bias [E] fp32
+ * or NULL (added to the logits before the softmax).  Writes topk_ids
+ * int32 [T, k] (descending probability, equal values -> lower index) and
+ * topk_w fp32 [T, k] (renormalised, each row sums to 1). */
+MOE_API moe_status moe_router_topk(const moe_problem* p, const void* x, const void* w_router,
+                           const float* router_bias, int32_t* topk_ids, float* topk_w,
+                           void* stream);
+
+/* Dispatch stage (the token is "sent to" its experts, Qwen3.6 explainer,
+ * router paragraph): a stable sort of the T*k (token, slot) pairs by expert.
+ * Outputs: offs int32 [E+2] (group e = rows offs[e]..offs[e+1]-1, ordered by
+ * (token, slot); group E = the shared expert, every token in order);
+ * row_tok int32 [R'] (source token of each row); row_w fp32 [R'] (routing
+ * weight; 1 for shared rows); pos int32 [T, k] (row of pair (t, j));
+ * x_perm [R', d] = x[row_tok].  ws: moe_stage_workspace_size() bytes.
+ * An expert id outside [0, E) sets MOE_ERR_DEVICE_CHECK in the device status
+ * and the affected pairs are dropped. */
+MOE_API moe_status moe_permute(const moe_problem* p, const void* x, const int32_t* topk_ids,
+                       const float* topk_w, void* x_perm, int32_t* row_tok, float* row_w,
+                       int32_t* pos, int32_t* offs, void* ws, size_t ws_bytes, void* stream);
+
+/* Expert stage (step 4 and the shared expert of step 5, unweighted):
+ * y_perm[r] = E_g(x_perm[r]) for every row r of group g (g == E: shared).
+ * x_perm, y_perm [R', d] in the activation type; offs as moe_permute writes
+ * it.  ws: moe_stage_workspace_size() bytes. */
+MOE_API moe_status moe_expert_ffn(const moe_problem* p, const void* x_perm, const int32_t* offs,
+                          const void* w_gate, const void* w_up, const void* w_down,
+                          const void* ws_gate, const void* ws_up, const void* ws_down,
+                          const float* scales, void* y_perm, void* ws, size_t ws_bytes,
+                          void* stream);
+
+/* Combine stage: y[t] = sum_j topk_w[t, j] * y_perm[pos[t, j]] + y_perm[offs[E] + t]
+ * (the last term when I_s > 0).  y [T, d] in the activation type. */
+MOE_API moe_status moe_combine(const moe_problem* p, const void* y_perm, const int32_t* pos,
+                       const float* topk_w, const int32_t* offs, void* y, void* stream);
+
+/* The whole block, fused: router + top-k, dispatch, gate/up GEMM with SwiGLU,
+ * down GEMM whose epilogue applies the routing weight and adds into y, plus
+ * the shared expert.  y [T, d] in the activation type.  topk_ids_out and
+ * topk_w_out ([T, k]) may be NULL.  ws: moe_workspace_size() bytes. */
+MOE_API moe_status moe_layer_forward(const moe_problem* p, const void* x, const void* w_router,
+                             const float* router_bias, const void* w_gate, const void* w_up,
+                             const void* w_down, const void* ws_gate, const void* ws_up,
+                             const void* ws_down, const float* scales, void* y,
+                             int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/* Kernel-path selection for the calls above on the calling process:
+ * 0 = automatic (tensor-core kernels where the shapes allow), 1 = SIMT CUDA
+ * kernels only (fp32 FMA; the path of fp32 problems), 2 = tensor-core kernels
+ * required (MOE_ERR_UNSUPPORTED when a shape does not allow them). */
+MOE_API moe_status moe_set_path(int path);
+
+/* Synchronously read and clear the device status word of the current device
+ * (MOE_OK, MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT); *detail receives the
+ * raw code (which kernel and which wait), or 0.  Synchronises the device. */
+MOE_API moe_status moe_device_status(int32_t* detail);
+
+/* Number of kernels the last successful call on this thread launched. */
+MOE_API int moe_last_launch_count(void);
+
+MOE_API const char* moe_last_error_string(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_H */

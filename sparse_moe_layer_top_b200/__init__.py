@@ -1,0 +1,237 @@
+"""Python binding of libmoe.so -- the sparse MoE block on B200 (sm_100a).
+
+Argument marshalling only: every step of the block runs in the library's CUDA
+kernels.  Tensors are CUDA torch tensors (contiguous, row-major); the calls
+enqueue on the current torch stream and never synchronise.  The library is
+built in-tree (``python -m sparse_moe_layer_top_b200.build``); importing this
+package without it raises at once -- there is no fallback.
+
+Entry points mirror ``include/moe.h``: ``router_topk``, ``permute``,
+``expert_ffn``, ``combine``, ``layer_forward``; ``MoELayer`` keeps a
+layer's weights and workspace together.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = ["MoEError", "Problem", "router_topk", "permute", "expert_ffn", "combine", "layer_forward",
+           "workspace_size", "stage_workspace_size", "set_path", "device_status", "last_launch_count",
+           "MoELayer", "lib_path", "F32", "BF16", "FP8_E4M3_B128"]
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+lib_path = os.path.join(HERE, "libmoe.so")
+
+F32, BF16, FP8_E4M3_B128 = 0, 1, 2
+_STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_ALIGNMENT",
+           4: "MOE_ERR_WORKSPACE_TOO_SMALL", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_DEVICE_CHECK", 7: "MOE_ERR_TIMEOUT"}
+EXPORTS = ("moe_check_problem", "moe_workspace_size", "moe_stage_workspace_size", "moe_router_topk",
+           "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_set_path",
+           "moe_device_status", "moe_last_launch_count", "moe_last_error_string")
+
+
+class MoEError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__("%s: %s" % (_STATUS.get(status, status), msg))
+        self.status = status
+
+
+class Problem(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int32), ("E", ctypes.c_int32), ("k", ctypes.c_int32),
+                ("I", ctypes.c_int32), ("I_s", ctypes.c_int32), ("act_dtype", ctypes.c_int32),
+                ("w_dtype", ctypes.c_int32)]
+
+    @classmethod
+    def make(cls, T, d, E, k, I, I_s, act="bf16", w="bf16"):
+        codes = {"f32": F32, "bf16": BF16, "fp8": FP8_E4M3_B128}
+        return cls(int(T), int(d), int(E), int(k), int(I), int(I_s), codes[act], codes[w])
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        if not os.path.exists(lib_path):
+            raise ImportError("libmoe.so is not built (run python -m sparse_moe_layer_top_b200.build)")
+        L = ctypes.CDLL(lib_path)
+        P, PP = ctypes.c_void_p, ctypes.POINTER(Problem)
+        S = ctypes.c_int
+        L.moe_check_problem.argtypes = [PP]
+        L.moe_workspace_size.argtypes = [PP]
+        L.moe_workspace_size.restype = ctypes.c_size_t
+        L.moe_stage_workspace_size.argtypes = [PP]
+        L.moe_stage_workspace_size.restype = ctypes.c_size_t
+        L.moe_router_topk.argtypes = [PP, P, P, P, P, P, P]
+        L.moe_permute.argtypes = [PP, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.moe_expert_ffn.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.moe_combine.argtypes = [PP, P, P, P, P, P, P]
+        L.moe_layer_forward.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.moe_set_path.argtypes = [ctypes.c_int]
+        L.moe_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32)]
+        L.moe_last_launch_count.restype = ctypes.c_int
+        L.moe_last_error_string.restype = ctypes.c_char_p
+        for f in ("moe_check_problem", "moe_router_topk", "moe_permute", "moe_expert_ffn", "moe_combine",
+                  "moe_layer_forward", "moe_set_path", "moe_device_status"):
+            getattr(L, f).restype = S
+        _lib = L
+    return _lib
+
+
+def _check(status):
+    if status != 0:
+        raise MoEError(status, lib().moe_last_error_string().decode())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _act(prob):
+    return torch.float32 if prob.act_dtype == F32 else torch.bfloat16
+
+
+def workspace_size(prob):
+    return lib().moe_workspace_size(ctypes.byref(prob))
+
+
+def stage_workspace_size(prob):
+    return lib().moe_stage_workspace_size(ctypes.byref(prob))
+
+
+def check_problem(prob):
+    _check(lib().moe_check_problem(ctypes.byref(prob)))
+
+
+def set_path(path):
+    """0 automatic, 1 SIMT kernels only, 2 tensor-core kernels required."""
+    _check(lib().moe_set_path(int(path)))
+
+
+def device_status():
+    """(status, detail) of the device status word, which is then cleared (synchronises)."""
+    d = ctypes.c_int32(0)
+    s = lib().moe_device_status(ctypes.byref(d))
+    return s, d.value
+
+
+def last_launch_count():
+    return lib().moe_last_launch_count()
+
+
+def _ws(nbytes, device, ws):
+    if ws is None:
+        ws = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
+    return ws
+
+
+def router_topk(prob, x, w_router, bias=None, topk_ids=None, topk_w=None, stream=None):
+    T, k = prob.T, prob.k
+    if topk_ids is None:
+        topk_ids = torch.empty((T, k), dtype=torch.int32, device=x.device)
+    if topk_w is None:
+        topk_w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    _check(lib().moe_router_topk(ctypes.byref(prob), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(topk_ids),
+                                 _ptr(topk_w), _stream(stream)))
+    return topk_ids, topk_w
+
+
+def rows_total(prob):
+    return prob.T * prob.k + (prob.T if prob.I_s > 0 else 0)
+
+
+def permute(prob, x, topk_ids, topk_w, ws=None, stream=None):
+    """-> dict(x_perm, row_tok, row_w, pos, offs)."""
+    dev = x.device
+    Rp = rows_total(prob)
+    out = dict(x_perm=torch.empty((Rp, prob.d), dtype=_act(prob), device=dev),
+               row_tok=torch.empty(Rp, dtype=torch.int32, device=dev),
+               row_w=torch.empty(Rp, dtype=torch.float32, device=dev),
+               pos=torch.empty((prob.T, prob.k), dtype=torch.int32, device=dev),
+               offs=torch.empty(prob.E + 2, dtype=torch.int32, device=dev))
+    nbytes = stage_workspace_size(prob)
+    ws = _ws(nbytes, dev, ws)
+    _check(lib().moe_permute(ctypes.byref(prob), _ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(out["x_perm"]),
+                             _ptr(out["row_tok"]), _ptr(out["row_w"]), _ptr(out["pos"]), _ptr(out["offs"]),
+                             _ptr(ws), ws.numel(), _stream(stream)))
+    return out
+
+
+def expert_ffn(prob, x_perm, offs, wg, wu, wd, s_wg=None, s_wu=None, s_wd=None, scales=None, y_perm=None,
+               ws=None, stream=None):
+    dev = x_perm.device
+    if y_perm is None:
+        y_perm = torch.empty((x_perm.shape[0], prob.d), dtype=_act(prob), device=dev)
+    ws = _ws(stage_workspace_size(prob), dev, ws)
+    _check(lib().moe_expert_ffn(ctypes.byref(prob), _ptr(x_perm), _ptr(offs), _ptr(wg), _ptr(wu), _ptr(wd),
+                                _ptr(s_wg), _ptr(s_wu), _ptr(s_wd), _ptr(scales), _ptr(y_perm), _ptr(ws), ws.numel(),
+                                _stream(stream)))
+    return y_perm
+
+
+def combine(prob, y_perm, pos, topk_w, offs, y=None, stream=None):
+    if y is None:
+        y = torch.empty((prob.T, prob.d), dtype=_act(prob), device=y_perm.device)
+    _check(lib().moe_combine(ctypes.byref(prob), _ptr(y_perm), _ptr(pos), _ptr(topk_w), _ptr(offs), _ptr(y),
+                             _stream(stream)))
+    return y
+
+
+def layer_forward(prob, x, w_router, bias, wg, wu, wd, s_wg=None, s_wu=None, s_wd=None, scales=None, y=None,
+                  topk_ids=None, topk_w=None, ws=None, stream=None):
+    if y is None:
+        y = torch.empty((prob.T, prob.d), dtype=_act(prob), device=x.device)
+    ws = _ws(workspace_size(prob), x.device, ws)
+    _check(lib().moe_layer_forward(ctypes.byref(prob), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(wg), _ptr(wu),
+                                   _ptr(wd), _ptr(s_wg), _ptr(s_wu), _ptr(s_wd), _ptr(scales), _ptr(y),
+                                   _ptr(topk_ids), _ptr(topk_w), _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+class MoELayer:
+    """One block's weights plus a workspace sized for up to `max_tokens` tokens."""
+
+    def __init__(self, d, E, k, I, I_s, w_router, wg, wu, wd, s_wg=None, s_wu=None, s_wd=None, bias=None,
+                 scales=None, act="bf16", w="bf16", max_tokens=0):
+        self.shape = (d, E, k, I, I_s, act, w)
+        self.w = (w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales)
+        self.device = wg.device
+        self.ws = None
+        if max_tokens:
+            self._reserve(max_tokens)
+
+    def problem(self, T):
+        d, E, k, I, I_s, act, w = self.shape
+        return Problem.make(T, d, E, k, I, I_s, act, w)
+
+    def _reserve(self, T):
+        n = workspace_size(self.problem(T))
+        if self.ws is None or self.ws.numel() < n:
+            self.ws = torch.empty(n, dtype=torch.uint8, device=self.device)
+
+    def __call__(self, x, y=None, topk_ids=None, topk_w=None, stream=None):
+        prob = self.problem(x.shape[0])
+        self._reserve(x.shape[0])
+        w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales = self.w
+        return layer_forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, y=y,
+                             topk_ids=topk_ids, topk_w=topk_w, ws=self.ws, stream=stream)
+
+    @classmethod
+    def from_inputs(cls, inp, max_tokens=0):
+        return cls(inp.d, inp.E, inp.k, inp.I, inp.I_s, inp.w_r, inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu,
+                   inp.s_wd, bias=inp.bias, scales=inp.scales, act=inp.act, w=inp.w, max_tokens=max_tokens)
+
+
+lib()

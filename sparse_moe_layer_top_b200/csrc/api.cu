@@ -1,0 +1,700 @@
+// api.cu -- host side of libmoe.so: argument checks, workspace carving, TMA
+// tensor-map encoding and the launch sequence of every entry point of moe.h.
+// One translation unit: the kernels are included from the headers beside it.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/moe.h"
+#include "common.cuh"
+#include "permute.cuh"
+#include "simt.cuh"
+#include "tc_gemm.cuh"
+
+using namespace moe;
+
+// ============================================================== errors
+static thread_local char g_err[512] = "no error";
+static thread_local int g_launches = 0;
+static thread_local int g_launches_pending = 0;
+
+static moe_status fail(moe_status s, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof g_err, fmt, ap);
+  va_end(ap);
+  return s;
+}
+
+#define CUDA_TRY(call)                                                                      \
+  do {                                                                                      \
+    cudaError_t e_ = (call);                                                                \
+    if (e_ != cudaSuccess) return fail(MOE_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+#define LAUNCH_CHECK(name)                                                                   \
+  do {                                                                                       \
+    cudaError_t e_ = cudaGetLastError();                                                     \
+    if (e_ != cudaSuccess) return fail(MOE_ERR_CUDA, "launch %s: %s", name, cudaGetErrorString(e_)); \
+    ++g_launches_pending;                                                                    \
+  } while (0)
+
+// ============================================================== device state
+// The device status word: kernels record a rejected input or a wait that gave
+// up; moe_device_status() reads and clears it.
+static __device__ unsigned g_status;
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  bool ready = false;
+  unsigned* status = nullptr;
+  int sms = 0;
+  bool attr_set = false;
+};
+static DeviceInfo g_dev[kMaxDevices];
+static std::mutex g_dev_mu;
+static int g_path = 0;
+
+template <typename K>
+static cudaError_t allow_smem(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+}
+
+// GEMM instantiations used by the library.
+using Gemm1Cfg = TcGemmCfg<128, true, 4>;
+using Gemm2Cfg = TcGemmCfg<256, false, 4>;
+static constexpr int kRouterSmem = 227 * 1024;
+
+static moe_status device_info(DeviceInfo** out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& d = g_dev[dev];
+  if (!d.ready) {
+    void* p = nullptr;
+    CUDA_TRY(cudaGetSymbolAddress(&p, g_status));
+    d.status = static_cast<unsigned*>(p);
+    CUDA_TRY(cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev));
+    int major = 0, minor = 0;
+    CUDA_TRY(cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev));
+    CUDA_TRY(cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev));
+    if (major != 10 || minor != 0)
+      return fail(MOE_ERR_UNSUPPORTED, "libmoe is built for sm_100a; device %d is sm_%d%d", dev, major, minor);
+    CUDA_TRY(allow_smem(k_gemm_tc<128, true, 4, kTcSwiGLU>, Gemm1Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcCombine>, Gemm2Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcStore>, Gemm2Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_router_tc, kRouterSmem));
+    d.ready = true;
+  }
+  *out = &d;
+  return MOE_OK;
+}
+
+// ============================================================== tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static moe_status encode_fn(EncodeTiledFn* out) {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    err = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q);
+    if (err == cudaSuccess && q == cudaDriverEntryPointSuccess) fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  if (!fn) return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled unavailable (%s)", cudaGetErrorString(err));
+  *out = fn;
+  return MOE_OK;
+}
+
+// bf16 tensor, 128-byte swizzle, box {64, box_rows} (x {1}); out-of-range reads give zeros.
+static moe_status map_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                           const uint64_t* strides_bytes, uint32_t box_rows) {
+  EncodeTiledFn enc;
+  moe_status s = encode_fn(&enc);
+  if (s != MOE_OK) return s;
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t box[3] = {(cuuint32_t)kBK, box_rows, 1}, es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) gd[i] = dims[i] ? dims[i] : 1;
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, box, es,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) rank %d dims %llu x %llu", (int)r, rank,
+                (unsigned long long)gd[0], (unsigned long long)gd[1]);
+  return MOE_OK;
+}
+static moe_status map2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t stride_elems,
+                        uint32_t box_rows) {
+  uint64_t dims[2] = {inner, outer}, st[1] = {stride_elems * 2};
+  return map_bf16(m, base, 2, dims, st, box_rows);
+}
+static moe_status map3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
+                        uint32_t box_rows) {
+  uint64_t dims[3] = {inner, mid, outer}, st[2] = {inner * 2, inner * mid * 2};
+  return map_bf16(m, base, 3, dims, st, box_rows);
+}
+
+// ============================================================== checks
+static size_t esize(int dt) { return dt == MOE_F32 ? 4 : dt == MOE_BF16 ? 2 : 1; }
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+static moe_status check(const moe_problem* p) {
+  if (!p) return fail(MOE_ERR_INVALID_ARG, "problem is NULL");
+  if (p->T < 0) return fail(MOE_ERR_INVALID_ARG, "T = %lld < 0", (long long)p->T);
+  if (p->d <= 0 || p->E <= 0 || p->k <= 0 || p->I <= 0 || p->I_s < 0)
+    return fail(MOE_ERR_INVALID_ARG, "sizes must be positive (d=%d E=%d k=%d I=%d I_s=%d)", p->d, p->E, p->k, p->I,
+                p->I_s);
+  if (p->E > kMaxE) return fail(MOE_ERR_UNSUPPORTED, "E = %d > %d", p->E, kMaxE);
+  if (p->k > p->E || p->k > kMaxK) return fail(MOE_ERR_INVALID_ARG, "k = %d must be <= min(E, %d)", p->k, kMaxK);
+  if (p->act_dtype != MOE_F32 && p->act_dtype != MOE_BF16)
+    return fail(MOE_ERR_INVALID_ARG, "activation type %d is not F32 or BF16", p->act_dtype);
+  if (p->w_dtype != MOE_F32 && p->w_dtype != MOE_BF16 && p->w_dtype != MOE_FP8_E4M3_B128)
+    return fail(MOE_ERR_INVALID_ARG, "weight type %d unknown", p->w_dtype);
+  if (p->act_dtype == MOE_F32 && p->w_dtype != MOE_F32)
+    return fail(MOE_ERR_UNSUPPORTED, "F32 activations need F32 weights");
+  if (p->act_dtype == MOE_BF16 && p->w_dtype == MOE_F32)
+    return fail(MOE_ERR_UNSUPPORTED, "BF16 activations take BF16 or FP8 weights");
+  if (p->d % 8 || p->I % 8 || p->I_s % 8)
+    return fail(MOE_ERR_ALIGNMENT, "d, I, I_s must be multiples of 8 (16-byte rows)");
+  if (p->w_dtype == MOE_FP8_E4M3_B128 && (p->d % 128 || p->I % 128 || p->I_s % 128))
+    return fail(MOE_ERR_INVALID_ARG, "FP8 block scales need d, I, I_s multiples of 128");
+  if (p->T * (int64_t)(p->k + 1) >= (int64_t)1 << 31) return fail(MOE_ERR_UNSUPPORTED, "T*(k+1) >= 2^31");
+  return MOE_OK;
+}
+
+static bool misaligned(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15u) != 0; }
+
+#define NEED(ptr)                                                                              \
+  do {                                                                                         \
+    if (!(ptr)) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", #ptr);                          \
+    if (misaligned(ptr)) return fail(MOE_ERR_ALIGNMENT, "%s is not 16-byte aligned", #ptr);    \
+  } while (0)
+#define MAYBE(ptr)                                                                             \
+  do {                                                                                         \
+    if ((ptr) && misaligned(ptr)) return fail(MOE_ERR_ALIGNMENT, "%s is not 16-byte aligned", #ptr); \
+  } while (0)
+
+// Tensor-core kernels: bf16 activations and bf16 weights.
+static bool tc_shapes(const moe_problem& p) { return p.act_dtype == MOE_BF16 && p.w_dtype == MOE_BF16; }
+static bool tc_router_shapes(const moe_problem& p) { return p.act_dtype == MOE_BF16; }
+
+static moe_status choose(bool tc_possible, bool* use_tc) {
+  if (g_path == 1) {
+    *use_tc = false;
+  } else if (g_path == 2) {
+    if (!tc_possible) return fail(MOE_ERR_UNSUPPORTED, "tensor-core path required but the types do not allow it");
+    *use_tc = true;
+  } else {
+    *use_tc = tc_possible;
+  }
+  return MOE_OK;
+}
+
+// ============================================================== workspace
+struct Layout {
+  size_t counts = 0, pre_a = 0, pre_b = 0, ids = 0, tw = 0, offs = 0, row_tok = 0, row_w = 0, pos = 0, xp = 0,
+         h = 0, y32 = 0, total = 0;
+};
+
+static int64_t rows_total(const moe_problem& p) { return p.T * p.k + (p.I_s > 0 ? p.T : 0); }
+static int64_t n_chunks(const moe_problem& p) { return std::max<int64_t>(1, cdiv(p.T * p.k, kChunk)); }
+static int64_t ldh_of(const moe_problem& p) { return std::max(p.I, p.I_s); }
+
+static Layout layout(const moe_problem& p, bool forward) {
+  Layout L;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    size_t r = o;
+    o += align_up(std::max<size_t>(bytes, 1), 256);
+    return r;
+  };
+  const int64_t n = p.T * p.k, Rp = rows_total(p);
+  const size_t ab = esize(p.act_dtype);
+  L.counts = take(n_chunks(p) * p.E * 4);
+  L.pre_a = take((p.E + 2) * 4);
+  L.pre_b = take((p.E + 2) * 4);
+  if (forward) {
+    L.ids = take(n * 4);
+    L.tw = take(n * 4);
+    L.offs = take((p.E + 2) * 4);
+    L.row_tok = take(Rp * 4);
+    L.row_w = take(Rp * 4);
+    L.pos = take(n * 4);
+    L.xp = take(Rp * p.d * ab);
+  }
+  L.h = take(Rp * ldh_of(p) * ab);
+  if (forward && p.act_dtype == MOE_BF16) L.y32 = take(p.T * p.d * 4);
+  L.total = o;
+  return L;
+}
+
+// ============================================================== launch pieces
+static Schedule sched_simt(int n_r, int n_s) { return Schedule{64, 64, n_r, n_s, 0}; }
+static Schedule sched_tc(int bn, int n_r, int n_s) { return Schedule{kBM, bn, n_r, n_s, 0}; }
+
+static moe_status launch_router(const moe_problem& p, const void* x, const void* wr, const float* bias,
+                                int32_t* ids, float* tw, cudaStream_t st, DeviceInfo* dev) {
+  if (p.T == 0) return MOE_OK;
+  bool tc;
+  moe_status s = choose(tc_router_shapes(p), &tc);
+  if (s != MOE_OK) return s;
+  if (!tc) {
+    dim3 grid((unsigned)cdiv(p.T, 8));
+    if (p.act_dtype == MOE_F32)
+      k_router_simt<float><<<grid, 256, 0, st>>>((const float*)x, (const float*)wr, bias, p.T, p.d, p.E, p.k, ids, tw);
+    else
+      k_router_simt<bf16><<<grid, 256, 0, st>>>((const bf16*)x, (const bf16*)wr, bias, p.T, p.d, p.E, p.k, ids, tw);
+    LAUNCH_CHECK("router_simt");
+    return MOE_OK;
+  }
+  TcRouterArgs a;
+  a.T = p.T;
+  a.E = p.E;
+  a.E_pad = (int)align_up(p.E, 16);
+  a.k = p.k;
+  a.kblocks = (int)cdiv(p.d, kBK);
+  a.n1 = std::min(a.E_pad, 256);
+  a.n2 = a.E_pad > 256 ? a.E_pad - 256 : 0;
+  a.tmem_cols = 32;
+  while (a.tmem_cols < a.E_pad) a.tmem_cols <<= 1;
+  const int stage_bytes = kBM * kBK * 2 + (a.n2 ? 512 : a.E_pad) * kBK * 2;
+  a.stages = std::min(4, (kRouterSmem - 1024 - 256) / stage_bytes);
+  a.bias = bias;
+  a.ids = ids;
+  a.tw = tw;
+  a.status = dev->status;
+  CUtensorMap tx, tw_map;
+  s = map2d(&tx, x, p.d, p.T, p.d, kBM);
+  if (s != MOE_OK) return s;
+  s = map2d(&tw_map, wr, p.d, p.E, p.d, a.n2 ? 256 : a.E_pad);
+  if (s != MOE_OK) return s;
+  const int smem = 1024 + a.stages * stage_bytes + 256;
+  k_router_tc<<<(unsigned)cdiv(p.T, kBM), 192, smem, st>>>(tx, tw_map, a);
+  LAUNCH_CHECK("router_tc");
+  return MOE_OK;
+}
+
+// Count, scan and scatter: offs, row_tok, row_w, pos; optionally the tile prefixes.
+static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, const float* tw, int32_t* offs,
+                                  int32_t* row_tok, float* row_w, int32_t* pos, int32_t* counts, Schedule sa,
+                                  int32_t* pre_a, Schedule sb, int32_t* pre_b, cudaStream_t st, DeviceInfo* dev) {
+  const int64_t n = p.T * p.k;
+  const int nch = (int)n_chunks(p);
+  if (n > 0) {
+    k_count<<<nch, 256, 0, st>>>(ids, n, p.E, counts, dev->status);
+    LAUNCH_CHECK("count");
+  } else {
+    CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)p.E * 4, st));
+  }
+  k_scan<<<1, 1024, 0, st>>>(counts, nch, p.E, p.T, p.k, p.I_s > 0, offs, sa, pre_a, sb, pre_b);
+  LAUNCH_CHECK("scan");
+  if (n > 0) {
+    k_scatter<<<nch, kScatterWarps * 32, 0, st>>>(ids, tw, n, p.k, p.E, counts, row_tok, row_w, pos);
+    LAUNCH_CHECK("scatter");
+  }
+  if (p.I_s > 0 && p.T > 0) {
+    k_shared_rows<<<(unsigned)cdiv(p.T, 256), 256, 0, st>>>(p.T, offs, p.E, row_tok, row_w);
+    LAUNCH_CHECK("shared_rows");
+  }
+  return MOE_OK;
+}
+
+static moe_status launch_gather(const moe_problem& p, const void* x, const int32_t* row_tok, const int32_t* offs,
+                                void* xp, cudaStream_t st, DeviceInfo* dev) {
+  const int vec = (int)(p.d * esize(p.act_dtype) / 16);
+  const int64_t rows = rows_total(p);
+  if (rows == 0) return MOE_OK;
+  unsigned grid = (unsigned)std::min<int64_t>(cdiv(rows, 8), (int64_t)dev->sms * 8);
+  k_gather<<<grid, 256, 0, st>>>((const uint4*)x, row_tok, offs, p.E, p.T, vec, (uint4*)xp);
+  LAUNCH_CHECK("gather");
+  return MOE_OK;
+}
+
+struct ExpertWeights {
+  const void *wg, *wu, *wd, *sg, *su, *sd;
+  const float* scales;
+};
+
+// FP8 scale sub-buffers (see moe.h).
+static void scale_parts(const moe_problem& p, const float* sc, const float* part[6]) {
+  const int64_t gd = p.d / 128, gi = p.I / 128, gs = p.I_s / 128;
+  const int64_t off[6] = {0,
+                          (int64_t)p.E * gi * gd,
+                          2 * (int64_t)p.E * gi * gd,
+                          3 * (int64_t)p.E * gi * gd,
+                          3 * (int64_t)p.E * gi * gd + gs * gd,
+                          3 * (int64_t)p.E * gi * gd + 2 * gs * gd};
+  for (int i = 0; i < 6; ++i) part[i] = sc ? sc + off[i] : nullptr;
+}
+
+template <typename TA, typename TW>
+static moe_status simt_gemms(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
+                             int32_t* pre_a, int32_t* pre_b, void* H, bool combine, float* y32,
+                             const int32_t* row_tok, const float* row_w, void* out, cudaStream_t st,
+                             DeviceInfo* dev) {
+  const float* sp[6];
+  scale_parts(p, w.scales, sp);
+  const unsigned grid = (unsigned)dev->sms * 4;
+  SimtGemmArgs<TA, TW> a{};
+  a.offs = offs;
+  a.E = p.E;
+  a.rows_cap = rows_total(p);
+  // gate/up: A = dispatched rows [R', d], N = I (I_s), K = d
+  a.A = (const TA*)xp;
+  a.lda = p.d;
+  a.prefix = pre_a;
+  a.N_r = p.I;
+  a.N_s = p.I_s;
+  a.K_r = p.d;
+  a.K_s = p.d;
+  a.b1 = WeightSet<TW>{(const TW*)w.wg, (const TW*)w.sg, sp[0], sp[3]};
+  a.b2 = WeightSet<TW>{(const TW*)w.wu, (const TW*)w.su, sp[1], sp[4]};
+  a.H = (TA*)H;
+  a.ldh = ldh_of(p);
+  k_gemm_simt<TA, TW, kEpiSwiGLU><<<grid, 256, 0, st>>>(a);
+  LAUNCH_CHECK("gemm_simt_swiglu");
+  // down: A = H [R', ldh], N = d, K = I (I_s)
+  SimtGemmArgs<TA, TW> b{};
+  b.offs = offs;
+  b.E = p.E;
+  b.rows_cap = rows_total(p);
+  b.A = (const TA*)H;
+  b.lda = ldh_of(p);
+  b.prefix = pre_b;
+  b.N_r = p.d;
+  b.N_s = p.d;
+  b.K_r = p.I;
+  b.K_s = p.I_s;
+  b.b1 = WeightSet<TW>{(const TW*)w.wd, (const TW*)w.sd, sp[2], sp[5]};
+  b.b2 = b.b1;
+  if (combine) {
+    b.y32 = y32;
+    b.ldy = p.d;
+    b.T = p.T;
+    b.row_tok = row_tok;
+    b.row_w = row_w;
+    k_gemm_simt<TA, TW, kEpiCombine><<<grid, 256, 0, st>>>(b);
+    LAUNCH_CHECK("gemm_simt_combine");
+  } else {
+    b.out = (TA*)out;
+    b.ldo = p.d;
+    k_gemm_simt<TA, TW, kEpiStore><<<grid, 256, 0, st>>>(b);
+    LAUNCH_CHECK("gemm_simt_store");
+  }
+  return MOE_OK;
+}
+
+static moe_status tc_gemms(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
+                           int32_t* pre_a, int32_t* pre_b, void* H, bool combine, float* y32,
+                           const int32_t* row_tok, const float* row_w, void* out, cudaStream_t st,
+                           DeviceInfo* dev) {
+  const int64_t Rp = rows_total(p), ldh = ldh_of(p);
+  const bool sh = p.I_s > 0;
+  moe_status s;
+  CUtensorMap aR, aS, bR, bS, cR, cS;
+  // gate/up + SwiGLU
+  if ((s = map2d(&aR, xp, p.d, Rp, p.d, kBM)) != MOE_OK) return s;
+  if ((s = map3d(&bR, w.wg, p.d, p.I, p.E, 128)) != MOE_OK) return s;
+  if ((s = map3d(&cR, w.wu, p.d, p.I, p.E, 128)) != MOE_OK) return s;
+  bS = bR;
+  cS = cR;
+  if (sh) {
+    if ((s = map2d(&bS, w.sg, p.d, p.I_s, p.d, 128)) != MOE_OK) return s;
+    if ((s = map2d(&cS, w.su, p.d, p.I_s, p.d, 128)) != MOE_OK) return s;
+  }
+  TcGemmArgs a{};
+  a.offs = offs;
+  a.prefix = pre_a;
+  a.E = p.E;
+  a.rows_cap = Rp;
+  a.N_r = p.I;
+  a.N_s = p.I_s;
+  a.K_r = p.d;
+  a.K_s = p.d;
+  a.H = (bf16*)H;
+  a.ldh = ldh;
+  a.status = dev->status;
+  k_gemm_tc<128, true, 4, kTcSwiGLU><<<dev->sms, 192, Gemm1Cfg::SMEM_BYTES, st>>>(aR, aR, bR, bS, cR, cS, a);
+  LAUNCH_CHECK("gemm_tc_swiglu");
+  // down
+  if ((s = map2d(&aR, H, p.I, Rp, ldh, kBM)) != MOE_OK) return s;
+  aS = aR;
+  if (sh && (s = map2d(&aS, H, p.I_s, Rp, ldh, kBM)) != MOE_OK) return s;
+  if ((s = map3d(&bR, w.wd, p.I, p.d, p.E, 256)) != MOE_OK) return s;
+  bS = bR;
+  if (sh && (s = map2d(&bS, w.sd, p.I_s, p.d, p.I_s, 256)) != MOE_OK) return s;
+  TcGemmArgs b{};
+  b.offs = offs;
+  b.prefix = pre_b;
+  b.E = p.E;
+  b.rows_cap = Rp;
+  b.N_r = p.d;
+  b.N_s = p.d;
+  b.K_r = p.I;
+  b.K_s = p.I_s;
+  b.status = dev->status;
+  if (combine) {
+    b.y32 = y32;
+    b.ldy = p.d;
+    b.T = p.T;
+    b.row_tok = row_tok;
+    b.row_w = row_w;
+    k_gemm_tc<256, false, 4, kTcCombine><<<dev->sms, 192, Gemm2Cfg::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
+    LAUNCH_CHECK("gemm_tc_combine");
+  } else {
+    b.out = (bf16*)out;
+    b.ldo = p.d;
+    k_gemm_tc<256, false, 4, kTcStore><<<dev->sms, 192, Gemm2Cfg::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
+    LAUNCH_CHECK("gemm_tc_store");
+  }
+  return MOE_OK;
+}
+
+static moe_status expert_gemms(const moe_problem& p, bool tc, const void* xp, const int32_t* offs,
+                               const ExpertWeights& w, int32_t* pre_a, int32_t* pre_b, void* H, bool combine,
+                               float* y32, const int32_t* row_tok, const float* row_w, void* out, cudaStream_t st,
+                               DeviceInfo* dev) {
+  if (tc) return tc_gemms(p, xp, offs, w, pre_a, pre_b, H, combine, y32, row_tok, row_w, out, st, dev);
+  if (p.act_dtype == MOE_F32)
+    return simt_gemms<float, float>(p, xp, offs, w, pre_a, pre_b, H, combine, y32, row_tok, row_w, out, st, dev);
+  if (p.w_dtype == MOE_BF16)
+    return simt_gemms<bf16, bf16>(p, xp, offs, w, pre_a, pre_b, H, combine, y32, row_tok, row_w, out, st, dev);
+  return simt_gemms<bf16, uint8_t>(p, xp, offs, w, pre_a, pre_b, H, combine, y32, row_tok, row_w, out, st, dev);
+}
+
+static void schedules(const moe_problem& p, bool tc, Schedule* sa, Schedule* sb) {
+  if (tc) {
+    *sa = sched_tc(128, p.I, p.I_s);
+    *sb = sched_tc(256, p.d, p.d);
+  } else {
+    *sa = sched_simt(p.I, p.I_s);
+    *sb = sched_simt(p.d, p.d);
+  }
+}
+
+static moe_status check_weights(const moe_problem& p, const ExpertWeights& w) {
+  NEED(w.wg);
+  NEED(w.wu);
+  NEED(w.wd);
+  if (p.I_s > 0) {
+    NEED(w.sg);
+    NEED(w.su);
+    NEED(w.sd);
+  }
+  if (p.w_dtype == MOE_FP8_E4M3_B128) NEED(w.scales);
+  return MOE_OK;
+}
+
+// ============================================================== C ABI
+extern "C" {
+
+moe_status moe_check_problem(const moe_problem* p) { return check(p); }
+
+size_t moe_workspace_size(const moe_problem* p) { return check(p) == MOE_OK ? layout(*p, true).total : 0; }
+size_t moe_stage_workspace_size(const moe_problem* p) { return check(p) == MOE_OK ? layout(*p, false).total : 0; }
+
+moe_status moe_set_path(int path) {
+  if (path < 0 || path > 2) return fail(MOE_ERR_INVALID_ARG, "path %d is not 0, 1 or 2", path);
+  g_path = path;
+  return MOE_OK;
+}
+
+int moe_last_launch_count(void) { return g_launches; }
+const char* moe_last_error_string(void) { return g_err; }
+
+moe_status moe_device_status(int32_t* detail) {
+  DeviceInfo* dev;
+  moe_status s = device_info(&dev);
+  if (s != MOE_OK) return s;
+  CUDA_TRY(cudaDeviceSynchronize());
+  unsigned v = 0, zero = 0;
+  CUDA_TRY(cudaMemcpyFromSymbol(&v, g_status, sizeof v));
+  CUDA_TRY(cudaMemcpyToSymbol(g_status, &zero, sizeof zero));
+  if (detail) *detail = (int32_t)v;
+  if (v == 0) return MOE_OK;
+  if ((v >> 24) == 0x07) return fail(MOE_ERR_TIMEOUT, "device wait timed out (code 0x%08x)", v);
+  return fail(MOE_ERR_DEVICE_CHECK, "device check failed (code 0x%08x)", v);
+}
+
+moe_status moe_router_topk(const moe_problem* p, const void* x, const void* w_router, const float* router_bias,
+                           int32_t* topk_ids, float* topk_w, void* stream) {
+  moe_status s = check(p);
+  if (s != MOE_OK) return s;
+  if (p->T > 0) {
+    NEED(x);
+    NEED(w_router);
+    MAYBE(router_bias);
+    NEED(topk_ids);
+    NEED(topk_w);
+  }
+  DeviceInfo* dev;
+  if ((s = device_info(&dev)) != MOE_OK) return s;
+  g_launches_pending = 0;
+  s = launch_router(*p, x, w_router, router_bias, topk_ids, topk_w, (cudaStream_t)stream, dev);
+  if (s == MOE_OK) g_launches = g_launches_pending;
+  return s;
+}
+
+moe_status moe_permute(const moe_problem* p, const void* x, const int32_t* topk_ids, const float* topk_w,
+                       void* x_perm, int32_t* row_tok, float* row_w, int32_t* pos, int32_t* offs, void* ws,
+                       size_t ws_bytes, void* stream) {
+  moe_status s = check(p);
+  if (s != MOE_OK) return s;
+  NEED(offs);
+  NEED(ws);
+  if (p->T > 0) {
+    NEED(x);
+    NEED(topk_ids);
+    NEED(topk_w);
+    NEED(x_perm);
+    NEED(row_tok);
+    NEED(row_w);
+    NEED(pos);
+  }
+  const Layout L = layout(*p, false);
+  if (ws_bytes < L.total)
+    return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
+  DeviceInfo* dev;
+  if ((s = device_info(&dev)) != MOE_OK) return s;
+  g_launches_pending = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* w = (char*)ws;
+  s = launch_dispatch(*p, topk_ids, topk_w, offs, row_tok, row_w, pos, (int32_t*)(w + L.counts), Schedule{},
+                      nullptr, Schedule{}, nullptr, st, dev);
+  if (s != MOE_OK) return s;
+  s = launch_gather(*p, x, row_tok, offs, x_perm, st, dev);
+  if (s == MOE_OK) g_launches = g_launches_pending;
+  return s;
+}
+
+moe_status moe_expert_ffn(const moe_problem* p, const void* x_perm, const int32_t* offs, const void* w_gate,
+                          const void* w_up, const void* w_down, const void* ws_gate, const void* ws_up,
+                          const void* ws_down, const float* scales, void* y_perm, void* ws, size_t ws_bytes,
+                          void* stream) {
+  moe_status s = check(p);
+  if (s != MOE_OK) return s;
+  if (p->T == 0) return MOE_OK;
+  NEED(x_perm);
+  NEED(offs);
+  NEED(y_perm);
+  NEED(ws);
+  ExpertWeights w{w_gate, w_up, w_down, ws_gate, ws_up, ws_down, scales};
+  if ((s = check_weights(*p, w)) != MOE_OK) return s;
+  const Layout L = layout(*p, false);
+  if (ws_bytes < L.total)
+    return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
+  bool tc;
+  if ((s = choose(tc_shapes(*p), &tc)) != MOE_OK) return s;
+  DeviceInfo* dev;
+  if ((s = device_info(&dev)) != MOE_OK) return s;
+  g_launches_pending = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* wsp = (char*)ws;
+  Schedule sa, sb;
+  schedules(*p, tc, &sa, &sb);
+  int32_t* pre_a = (int32_t*)(wsp + L.pre_a);
+  int32_t* pre_b = (int32_t*)(wsp + L.pre_b);
+  k_tile_prefix<<<1, 1024, 0, st>>>(offs, p->E, sa, pre_a, sb, pre_b);
+  LAUNCH_CHECK("tile_prefix");
+  s = expert_gemms(*p, tc, x_perm, offs, w, pre_a, pre_b, wsp + L.h, false, nullptr, nullptr, nullptr, y_perm, st,
+                   dev);
+  if (s == MOE_OK) g_launches = g_launches_pending;
+  return s;
+}
+
+moe_status moe_combine(const moe_problem* p, const void* y_perm, const int32_t* pos, const float* topk_w,
+                       const int32_t* offs, void* y, void* stream) {
+  moe_status s = check(p);
+  if (s != MOE_OK) return s;
+  if (p->T == 0) return MOE_OK;
+  NEED(y_perm);
+  NEED(pos);
+  NEED(topk_w);
+  NEED(offs);
+  NEED(y);
+  DeviceInfo* dev;
+  if ((s = device_info(&dev)) != MOE_OK) return s;
+  g_launches_pending = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (p->act_dtype == MOE_F32)
+    k_combine<float><<<(unsigned)p->T, 256, 0, st>>>((const float*)y_perm, pos, topk_w, offs, p->E, p->k, p->d, p->T,
+                                                     (float*)y);
+  else
+    k_combine<bf16><<<(unsigned)p->T, 256, 0, st>>>((const bf16*)y_perm, pos, topk_w, offs, p->E, p->k, p->d, p->T,
+                                                    (bf16*)y);
+  LAUNCH_CHECK("combine");
+  g_launches = g_launches_pending;
+  return MOE_OK;
+}
+
+moe_status moe_layer_forward(const moe_problem* p, const void* x, const void* w_router, const float* router_bias,
+                             const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
+                             const void* ws_up, const void* ws_down, const float* scales, void* y,
+                             int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  moe_status s = check(p);
+  if (s != MOE_OK) return s;
+  if (p->T == 0) {
+    g_launches = 0;
+    return MOE_OK;
+  }
+  NEED(x);
+  NEED(w_router);
+  MAYBE(router_bias);
+  NEED(y);
+  MAYBE(topk_ids_out);
+  MAYBE(topk_w_out);
+  NEED(ws);
+  ExpertWeights w{w_gate, w_up, w_down, ws_gate, ws_up, ws_down, scales};
+  if ((s = check_weights(*p, w)) != MOE_OK) return s;
+  const Layout L = layout(*p, true);
+  if (ws_bytes < L.total)
+    return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
+  bool tc;
+  if ((s = choose(tc_shapes(*p), &tc)) != MOE_OK) return s;
+  DeviceInfo* dev;
+  if ((s = device_info(&dev)) != MOE_OK) return s;
+  g_launches_pending = 0;
+  cudaStream_t st = (cudaStream_t)stream;
+  char* wsp = (char*)ws;
+  int32_t* ids = topk_ids_out ? topk_ids_out : (int32_t*)(wsp + L.ids);
+  float* tw = topk_w_out ? topk_w_out : (float*)(wsp + L.tw);
+  int32_t* offs = (int32_t*)(wsp + L.offs);
+  int32_t* row_tok = (int32_t*)(wsp + L.row_tok);
+  float* row_w = (float*)(wsp + L.row_w);
+  int32_t* pos = (int32_t*)(wsp + L.pos);
+  int32_t* pre_a = (int32_t*)(wsp + L.pre_a);
+  int32_t* pre_b = (int32_t*)(wsp + L.pre_b);
+  float* y32 = p->act_dtype == MOE_BF16 ? (float*)(wsp + L.y32) : (float*)y;
+  CUDA_TRY(cudaMemsetAsync(y32, 0, (size_t)p->T * p->d * 4, st));
+  if ((s = launch_router(*p, x, w_router, router_bias, ids, tw, st, dev)) != MOE_OK) return s;
+  Schedule sa, sb;
+  schedules(*p, tc, &sa, &sb);
+  s = launch_dispatch(*p, ids, tw, offs, row_tok, row_w, pos, (int32_t*)(wsp + L.counts), sa, pre_a, sb, pre_b, st,
+                      dev);
+  if (s != MOE_OK) return s;
+  if ((s = launch_gather(*p, x, row_tok, offs, wsp + L.xp, st, dev)) != MOE_OK) return s;
+  s = expert_gemms(*p, tc, wsp + L.xp, offs, w, pre_a, pre_b, wsp + L.h, true, y32, row_tok, row_w, nullptr, st,
+                   dev);
+  if (s != MOE_OK) return s;
+  if (p->act_dtype == MOE_BF16) {
+    const int64_t n8 = p->T * p->d / 8;
+    unsigned grid = (unsigned)std::min<int64_t>(cdiv(n8, 256), (int64_t)dev->sms * 16);
+    k_finalize_bf16<<<grid, 256, 0, st>>>((const float4*)y32, (uint4*)y, n8);
+    LAUNCH_CHECK("finalize");
+  }
+  g_launches = g_launches_pending;
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+// common.cuh -- element types, conversions and small device helpers shared by
+// the kernels of libmoe.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+namespace moe {
+
+using bf16 = __nv_bfloat16;
+using fp8 = __nv_fp8_storage_t;  // raw E4M3 code
+
+// Device status codes: high byte = which check, low bits = where.
+enum : unsigned {
+  kStatusBadExpertId = 0x06000001u,  // a routing id outside [0, E)
+  kStatusTimeoutBase = 0x07000000u,  // | (kernel id << 8) | wait site
+};
+enum : unsigned { kKernRouterTc = 1, kKernGemmTc = 2, kKernGemmSwap = 3 };
+
+__device__ __forceinline__ float to_f32(float v) { return v; }
+__device__ __forceinline__ float to_f32(bf16 v) { return __bfloat162float(v); }
+__device__ __forceinline__ void from_f32(float v, float* dst) { *dst = v; }
+__device__ __forceinline__ void from_f32(float v, bf16* dst) { *dst = __float2bfloat16_rn(v); }
+
+// E4M3 code -> float through the hardware conversion.
+__device__ __forceinline__ float e4m3_to_f32(uint8_t q) {
+  __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(q), __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+__device__ __forceinline__ float silu_f32(float z) { return z / (1.0f + __expf(-z)); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__host__ __device__ __forceinline__ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Locate the group whose tile range holds `tile`: prefix[g] <= tile < prefix[g+1].
+__device__ __forceinline__ int find_group(const int32_t* prefix, int ngroups, int tile) {
+  int lo = 0, hi = ngroups;  // invariant prefix[lo] <= tile < prefix[hi]
+  while (hi - lo > 1) {
+    int mid = (lo + hi) >> 1;
+    if (__ldg(prefix + mid) <= tile) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// One GEMM's tile schedule over the E+1 groups (group E = shared expert):
+// tiles of group g = m_tiles(rows_g) * ceil(N_g / bn), with
+// m_tiles = ceil(rows / bm) for the row-tiled kernels, and 0 or 1 for the
+// weight-row (swap) kernels whose N covers every row of a group.
+struct Schedule {
+  int bm, bn, n_routed, n_shared, swap;
+};
+
+__device__ __forceinline__ int sched_tiles(const Schedule& s, int g, int E, int rows) {
+  int n = g < E ? s.n_routed : s.n_shared;
+  if (rows <= 0 || n <= 0) return 0;
+  int mt = s.swap ? 1 : (int)cdiv(rows, s.bm);
+  return mt * (int)cdiv(n, s.bn);
+}
+
+}  // namespace moe

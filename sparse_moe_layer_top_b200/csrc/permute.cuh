@@ -1,0 +1,196 @@
+// permute.cuh -- dispatch of (token, slot) pairs to expert-contiguous rows.
+//
+// The token "is sent to" its k experts (Qwen3.6 explainer, router paragraph).
+// Here that is a stable counting sort by expert in three passes over the
+// flattened T*k routing ids, cut into chunks of kChunk pairs:
+//   k_count    per-chunk histogram over the E experts;
+//   k_scan     per-expert exclusive scan over chunks, then over experts ->
+//              group offsets offs[E+2] and each chunk's base row per expert;
+//              also the tile prefix sums of the GEMM schedules;
+//   k_scatter  within a chunk, warps take consecutive sub-ranges; ranks come
+//              from warp match masks, so row order = (token, slot) order;
+//   k_gather   copies x rows into the dispatched buffer (16-byte vectors).
+// Group E (the shared expert) is every token in order at rows T*k .. T*k+T-1.
+#pragma once
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kChunk = 2048;       // pairs per chunk
+constexpr int kScatterWarps = 8;   // warps of k_scatter (256 threads)
+constexpr int kMaxE = 512;
+
+__global__ void __launch_bounds__(256) k_count(const int32_t* __restrict__ ids, int64_t n, int E,
+                                               int32_t* __restrict__ counts, unsigned* status) {
+  __shared__ int32_t h[kMaxE];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+  __syncthreads();
+  int64_t c0 = (int64_t)blockIdx.x * kChunk;
+  int64_t c1 = c0 + kChunk < n ? c0 + kChunk : n;
+  for (int64_t i = c0 + threadIdx.x; i < c1; i += blockDim.x) {
+    int e = __ldg(ids + i);
+    if ((unsigned)e < (unsigned)E) atomicAdd(&h[e], 1);
+    else atomicCAS(status, 0u, (unsigned)kStatusBadExpertId);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) counts[(int64_t)blockIdx.x * E + e] = h[e];
+}
+
+// Inclusive block-wide scan of one int per thread (blockDim.x == 1024).
+__device__ __forceinline__ int block_incl_scan(int v, int* sm_warp) {
+  int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  if (lane == 31) sm_warp[w] = v;
+  __syncthreads();
+  if (w == 0) {
+    int s = sm_warp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int t = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += t;
+    }
+    sm_warp[lane] = s;
+  }
+  __syncthreads();
+  if (w > 0) v += sm_warp[w - 1];
+  __syncthreads();
+  return v;
+}
+
+// Tile prefix of one schedule from the group offsets (E+1 groups, one thread each).
+__device__ __forceinline__ void write_tile_prefix(const Schedule& s, int E, int rows_g, int32_t* prefix,
+                                                  int* sm_warp) {
+  int g = threadIdx.x;
+  int tiles = (g <= E) ? sched_tiles(s, g, E, rows_g) : 0;
+  int incl = block_incl_scan(tiles, sm_warp);
+  if (g <= E) prefix[g] = incl - tiles;
+  if (g == E) prefix[E + 1] = incl;
+}
+
+// One block of 1024 threads.  counts[c*E+e] (chunk histograms) becomes the
+// absolute first row of expert e's pairs in chunk c.
+__global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ counts, int nchunks, int E, int64_t T, int k,
+                                               int has_shared, int32_t* __restrict__ offs, Schedule sa,
+                                               int32_t* __restrict__ prefix_a, Schedule sb,
+                                               int32_t* __restrict__ prefix_b) {
+  __shared__ int sm_warp[32];
+  int e = threadIdx.x;
+  int total = 0;
+  if (e < E)
+    for (int c = 0; c < nchunks; ++c) total += counts[(int64_t)c * E + e];
+  int incl = block_incl_scan(e < E ? total : 0, sm_warp);
+  int start = incl - (e < E ? total : 0);
+  if (e < E) {
+    offs[e] = start;
+    int run = start;
+    for (int c = 0; c < nchunks; ++c) {
+      int v = counts[(int64_t)c * E + e];
+      counts[(int64_t)c * E + e] = run;
+      run += v;
+    }
+  }
+  // pairs with an invalid id were not counted: the routed rows stay contiguous
+  if (e == E) {
+    offs[E] = start;
+    offs[E + 1] = start + (has_shared ? (int)T : 0);
+  }
+  int rows = e < E ? total : (e == E ? (has_shared ? (int)T : 0) : 0);
+  if (prefix_a) write_tile_prefix(sa, E, rows, prefix_a, sm_warp);
+  if (prefix_b) write_tile_prefix(sb, E, rows, prefix_b, sm_warp);
+}
+
+// Tile prefixes from caller-supplied group offsets (the expert stage alone).
+__global__ void __launch_bounds__(1024) k_tile_prefix(const int32_t* __restrict__ offs, int E, Schedule sa,
+                                                      int32_t* __restrict__ prefix_a, Schedule sb,
+                                                      int32_t* __restrict__ prefix_b) {
+  __shared__ int sm_warp[32];
+  int g = threadIdx.x;
+  int rows = g <= E ? offs[g + 1] - offs[g] : 0;
+  if (prefix_a) write_tile_prefix(sa, E, rows, prefix_a, sm_warp);
+  if (prefix_b) write_tile_prefix(sb, E, rows, prefix_b, sm_warp);
+}
+
+__global__ void __launch_bounds__(kScatterWarps * 32) k_scatter(const int32_t* __restrict__ ids,
+                                                                const float* __restrict__ topk_w, int64_t n, int k,
+                                                                int E, const int32_t* __restrict__ base,
+                                                                int32_t* __restrict__ row_tok,
+                                                                float* __restrict__ row_w,
+                                                                int32_t* __restrict__ pos) {
+  __shared__ int32_t wb[kScatterWarps][kMaxE];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int sub = kChunk / kScatterWarps;
+  const int64_t c0 = (int64_t)blockIdx.x * kChunk;
+  const int64_t s0 = c0 + (int64_t)warp * sub;
+  for (int e = lane; e < E; e += 32) wb[warp][e] = 0;
+  __syncwarp();
+  // pass 1: per-warp histogram of its sub-range
+  for (int64_t i = s0 + lane; i < s0 + sub && i < n; i += 32) {
+    int e = __ldg(ids + i);
+    if ((unsigned)e < (unsigned)E) atomicAdd(&wb[warp][e], 1);
+  }
+  __syncthreads();
+  // exclusive scan across the warps of the chunk, per expert
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = base[(int64_t)blockIdx.x * E + e];
+    for (int w = 0; w < kScatterWarps; ++w) {
+      int v = wb[w][e];
+      wb[w][e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  // pass 2: in order, 32 pairs at a time; equal experts rank by lane order
+  const unsigned lt = (1u << lane) - 1u;
+  for (int64_t b = s0; b < s0 + sub && b < n; b += 32) {
+    int64_t i = b + lane;
+    bool act = i < n && i < s0 + sub;
+    int e = act ? __ldg(ids + i) : -1;
+    bool ok = act && (unsigned)e < (unsigned)E;
+    unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+    int r = 0;
+    if (ok) r = wb[warp][e] + __popc(peers & lt);
+    __syncwarp();
+    if (ok && (peers & lt) == 0) wb[warp][e] += __popc(peers);  // lowest peer advances the cursor
+    __syncwarp();
+    if (ok) {
+      row_tok[r] = (int32_t)(i / k);
+      row_w[r] = __ldg(topk_w + i);
+      pos[i] = r;
+    } else if (act) {
+      pos[i] = -1;
+    }
+  }
+}
+
+// Shared-expert rows: row offs[E] + t is token t with weight 1.
+__global__ void k_shared_rows(int64_t T, const int32_t* __restrict__ offs, int E, int32_t* __restrict__ row_tok,
+                              float* __restrict__ row_w) {
+  int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  int64_t R = offs[E];
+  if (t < T) {
+    row_tok[R + t] = (int32_t)t;
+    row_w[R + t] = 1.0f;
+  }
+}
+
+// x_perm[r] = x[row_tok[r]], one warp per row, 16-byte vectors (row bytes % 16 == 0).
+__global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ x, const int32_t* __restrict__ row_tok,
+                                                const int32_t* __restrict__ offs, int E, int64_t T,
+                                                int vec_per_row, uint4* __restrict__ xp) {
+  const int64_t rows = offs[E + 1];
+  const int lane = threadIdx.x & 31;
+  for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
+       r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
+    int t = __ldg(row_tok + r);
+    if ((uint64_t)t >= (uint64_t)T) t = 0;  // cannot happen for valid routing
+    const uint4* src = x + (int64_t)t * vec_per_row;
+    uint4* dst = xp + r * vec_per_row;
+    for (int v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,534 @@
+// tc_gemm.cuh -- tensor-core (tcgen05) kernels for sm_100a: the grouped expert
+// GEMMs and the router GEMM with its fused top-k.
+//
+// Grouped GEMM (row-tiled form).  For every group g (expert g, or g == E the
+// shared expert) with rows r0 .. r0+rows-1 of the activation matrix A:
+//     D[r, n] = sum_c A[r, c] * B_g[n, c],  n < N_g,  c < K_g,
+// with B_g K-major (the weights' own out x in layout).  One persistent CTA per
+// SM walks a device-built tile list (group, 128-row block, BN-column block);
+// tiles of one column block of a group are adjacent, so the CTAs that share a
+// weight tile run together and the second read comes from L2.
+//
+// Warp roles (6 warps):
+//   warp 0      TMA producer: A tile 128 x 64 and B tile(s) BN x 64 per stage,
+//               128-byte swizzled, into a STAGES-deep shared-memory ring;
+//   warp 1      TMEM owner and MMA issuer: tcgen05.mma M=128, N=BN, K=16,
+//               fp32 accumulators in TMEM, double-buffered across tiles;
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (warp w reads TMEM
+//               lanes 32*(w%4) ..), then one of
+//                 SwiGLU   H[r, n] = SiLU(gate) * up  -> bf16   (DUAL: two B)
+//                 Combine  y32[tok(r), n] += w(r) * D  (fp32 vector reductions)
+//                 Store    out[r, n] = D -> bf16.
+// Rows of a tile past the end of its group are computed and discarded; rows
+// never mix in a GEMM, so those rows cannot disturb the kept ones.
+#pragma once
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;  // 64 bf16 = one 128-byte swizzle row
+
+enum { kTcSwiGLU = 0, kTcCombine = 1, kTcStore = 2 };
+
+struct TcGemmArgs {
+  const int32_t* offs;    // [E+2] group row starts
+  const int32_t* prefix;  // [E+2] tile prefix of this schedule
+  int E;
+  int N_r, N_s, K_r, K_s;
+  int64_t rows_cap;       // rows of the activation/output buffers; no row at or past it is written
+  bf16* H;                // SwiGLU output [rows, ldh]
+  int64_t ldh;
+  float* y32;             // Combine output [T, ldy]
+  int64_t ldy, T;
+  const int32_t* row_tok;
+  const float* row_w;
+  bf16* out;              // Store output [rows, ldo]
+  int64_t ldo;
+  unsigned* status;
+};
+
+struct TileInfo {
+  int g, rows, m0, n0, kblocks, N;
+  int64_t row0;
+};
+
+template <int BN>
+__device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, int tile) {
+  TileInfo t;
+  t.g = find_group(p.prefix, p.E + 1, tile);
+  const int r0 = __ldg(p.offs + t.g);
+  t.rows = __ldg(p.offs + t.g + 1) - r0;
+  const int mtc = (t.rows + kBM - 1) / kBM;
+  const int local = tile - __ldg(p.prefix + t.g);
+  const int mb = local % mtc, nb = local / mtc;
+  t.m0 = mb * kBM;
+  t.row0 = (int64_t)r0 + t.m0;
+  t.n0 = nb * BN;
+  const bool sh = t.g == p.E;
+  t.N = sh ? p.N_s : p.N_r;
+  t.kblocks = ((sh ? p.K_s : p.K_r) + kBK - 1) / kBK;
+  return t;
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Wait (bounded, ignoring the abort flag) for a TMA copy already issued.
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+}
+
+template <int BN, bool DUAL, int STAGES>
+struct TcGemmCfg {
+  static constexpr int A_BYTES = kBM * kBK * 2;
+  static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES * (DUAL ? 2 : 1);
+  static constexpr int ACC_COLS = DUAL ? 2 * BN : BN;
+  static constexpr int TMEM_COLS = 2 * ACC_COLS;
+  static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8 + 16;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static_assert(TMEM_COLS == 64 || TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  static_assert(SMEM_BYTES <= 232448, "shared memory");
+};
+
+template <int BN, bool DUAL, int STAGES, int EPI>
+__global__ void __launch_bounds__(192, 1)
+    k_gemm_tc(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
+              const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
+              const __grid_constant__ CUtensorMap tmC_r, const __grid_constant__ CUtensorMap tmC_s, TcGemmArgs p) {
+  using Cfg = TcGemmCfg<BN, DUAL, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned tcode = kStatusTimeoutBase | (kKernGemmTc << 8);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull + b, 1);
+      mbar_init(tempty + b, 4);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tmap(&tmA_r);
+    prefetch_tmap(&tmA_s);
+    prefetch_tmap(&tmB_r);
+    prefetch_tmap(&tmB_s);
+    if (DUAL) {
+      prefetch_tmap(&tmC_r);
+      prefetch_tmap(&tmC_s);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = __ldg(p.prefix + p.E + 1);
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------ TMA producer
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_a = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, last_par = 0;
+      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        const TileInfo t = decode_tile<BN>(p, tile);
+        const bool sh = t.g == p.E;
+        bool ok = true;
+        for (int kb = 0; kb < t.kblocks; ++kb) {
+          if (!mbar_wait(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 1)) {
+            ok = false;
+            break;
+          }
+          uint8_t* sa = smem + stage * Cfg::STAGE_BYTES;
+          uint8_t* sb = sa + Cfg::A_BYTES;
+          mbar_arrive_expect_tx(full + stage, Cfg::STAGE_BYTES);
+          tma_load_2d(sa, sh ? &tmA_s : &tmA_r, full + stage, kb * kBK, (int)t.row0, pol_a);
+          if (sh) tma_load_2d(sb, &tmB_s, full + stage, kb * kBK, t.n0, pol_w);
+          else tma_load_3d(sb, &tmB_r, full + stage, kb * kBK, t.n0, t.g, pol_w);
+          if (DUAL) {
+            uint8_t* sc = sb + Cfg::B_BYTES;
+            if (sh) tma_load_2d(sc, &tmC_s, full + stage, kb * kBK, t.n0, pol_w);
+            else tma_load_3d(sc, &tmC_r, full + stage, kb * kBK, t.n0, t.g, pol_w);
+          }
+          issued |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+      if (*abort_flag)  // copies in flight must land before the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (issued >> s & 1u) drain_wait(full + s, last_par >> s & 1u);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------ MMA issuer
+      constexpr uint32_t idesc = idesc_bf16(kBM, BN);
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileInfo t = decode_tile<BN>(p, tile);
+        if (!mbar_wait(tempty + acc, acc_phase ^ 1, abort_flag, p.status, tcode | 2)) break;
+        tc_fence_after();
+        const uint32_t d0 = tmem_base + acc * Cfg::ACC_COLS;
+        for (int kb = 0; kb < t.kblocks; ++kb) {
+          if (!mbar_wait(full + stage, phase, abort_flag, p.status, tcode | 3)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(smem + stage * Cfg::STAGE_BYTES);
+          const uint32_t sb = sa + Cfg::A_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(sa + kk * 32);
+            const uint32_t accum = (kb | kk) != 0;
+            umma_f16(d0, ad, sdesc_sw128(sb + kk * 32), idesc, accum);
+            if (DUAL) umma_f16(d0 + BN, ad, sdesc_sw128(sb + Cfg::B_BYTES + kk * 32), idesc, accum);
+          }
+          umma_commit(empty + stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        umma_commit(tfull + acc);
+        if (++acc == 2) {
+          acc = 0;
+          acc_phase ^= 1;
+        }
+      }
+      // every MMA issued must finish before TMEM is released
+      umma_commit(drain);
+      drain_wait(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const TileInfo t = decode_tile<BN>(p, tile);
+      if (!mbar_wait(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)) break;
+      tc_fence_after();
+      const uint32_t tb = tmem_base + acc * Cfg::ACC_COLS + ((uint32_t)(q * 32) << 16);
+      const int64_t grow = t.row0 + row;
+      const bool valid = t.m0 + row < t.rows && grow < p.rows_cap;
+      if (EPI == kTcSwiGLU) {
+        bf16* dst = p.H + grow * p.ldh;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t g[32], u[32];
+          tmem_ld32(tb + c * 32, g);
+          tmem_ld32(tb + BN + c * 32, u);
+          tmem_wait_regs(g);
+          tmem_wait_regs(u);
+          if (valid) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int n = t.n0 + c * 32 + v * 8;
+              if (n < t.N) {
+                uint4 o;
+                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const float g0 = __uint_as_float(g[v * 8 + 2 * e]), g1 = __uint_as_float(g[v * 8 + 2 * e + 1]);
+                  const float u0 = __uint_as_float(u[v * 8 + 2 * e]), u1 = __uint_as_float(u[v * 8 + 2 * e + 1]);
+                  ow[e] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
+                }
+                *reinterpret_cast<uint4*>(dst + n) = o;
+              }
+            }
+          }
+        }
+      } else if (EPI == kTcCombine) {
+        int tok = 0;
+        float w = 0.f;
+        if (valid) {
+          tok = __ldg(p.row_tok + grow);
+          w = __ldg(p.row_w + grow);
+        }
+        const bool ok = valid && (uint64_t)tok < (uint64_t)p.T;
+        float* dst = p.y32 + (int64_t)tok * p.ldy;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t a[32];
+          tmem_ld32(tb + c * 32, a);
+          tmem_wait_regs(a);
+          if (ok) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const int n = t.n0 + c * 32 + v * 4;
+              if (n < t.N)
+                atomicAdd(reinterpret_cast<float4*>(dst + n),
+                          make_float4(w * __uint_as_float(a[4 * v]), w * __uint_as_float(a[4 * v + 1]),
+                                      w * __uint_as_float(a[4 * v + 2]), w * __uint_as_float(a[4 * v + 3])));
+            }
+          }
+        }
+      } else {
+        bf16* dst = p.out + grow * p.ldo;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t a[32];
+          tmem_ld32(tb + c * 32, a);
+          tmem_wait_regs(a);
+          if (valid) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int n = t.n0 + c * 32 + v * 8;
+              if (n < t.N) {
+                uint4 o;
+                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  ow[e] = pack_bf16x2(__uint_as_float(a[v * 8 + 2 * e]), __uint_as_float(a[v * 8 + 2 * e + 1]));
+                *reinterpret_cast<uint4*>(dst + n) = o;
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(tempty + acc);
+      if (++acc == 2) {
+        acc = 0;
+        acc_phase ^= 1;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------- router
+// One CTA per 128 tokens: logits[128, E] = x_blk . W_r^T accumulate in TMEM
+// (E padded to a multiple of 16; up to two MMAs of N <= 256 side by side),
+// then each epilogue thread scans its token's row of logits in TMEM, keeps
+// the k largest (equal values -> lower expert index) in registers, and
+// writes the ids and the softmax over the kept logits (= the full softmax
+// renormalised over the kept experts).
+constexpr int kMaxK = 16;
+
+struct TcRouterArgs {
+  int64_t T;
+  int E, E_pad, k, kblocks, stages;
+  int n1, n2;          // MMA widths of the two halves (n2 == 0: one)
+  int tmem_cols;
+  const float* bias;
+  int32_t* ids;
+  float* tw;
+  unsigned* status;
+};
+
+__global__ void __launch_bounds__(192, 1)
+    k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcRouterArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = align1024(smem_raw);
+  const int A_BYTES = kBM * kBK * 2;
+  const int B_BYTES = (p.n2 ? 512 : p.E_pad) * kBK * 2;
+  const int STAGE_BYTES = A_BYTES + B_BYTES;
+  const int S = p.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * STAGE_BYTES);
+  uint64_t* empty = full + S;
+  uint64_t* tfull = empty + S;
+  uint64_t* drain = tfull + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned tcode = kStatusTimeoutBase | (kKernRouterTc << 8);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(full + s, 1);
+      mbar_init(empty + s, 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, p.tmem_cols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int row0 = blockIdx.x * kBM;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      const uint64_t pol = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, last_par = 0;
+      for (int kb = 0; kb < p.kblocks; ++kb) {
+        if (!mbar_wait(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 1)) break;
+        uint8_t* sa = smem + stage * STAGE_BYTES;
+        uint8_t* sb = sa + A_BYTES;
+        mbar_arrive_expect_tx(full + stage, STAGE_BYTES);
+        tma_load_2d(sa, &tmX, full + stage, kb * kBK, row0, pol);
+        tma_load_2d(sb, &tmW, full + stage, kb * kBK, 0, pol);
+        if (p.n2) tma_load_2d(sb + 256 * kBK * 2, &tmW, full + stage, kb * kBK, 256, pol);
+        issued |= 1u << stage;
+        last_par = (last_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (*abort_flag)
+        for (int s = 0; s < S; ++s)
+          if (issued >> s & 1u) drain_wait(full + s, last_par >> s & 1u);
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t id1 = idesc_bf16(kBM, p.n1);
+      const uint32_t id2 = idesc_bf16(kBM, p.n2 ? p.n2 : 16);
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int kb = 0; kb < p.kblocks; ++kb) {
+        if (!mbar_wait(full + stage, phase, abort_flag, p.status, tcode | 3)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
+        const uint32_t sb = sa + A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(sa + kk * 32);
+          const uint32_t accum = (kb | kk) != 0;
+          umma_f16(tmem_base, ad, sdesc_sw128(sb + kk * 32), id1, accum);
+          if (p.n2) umma_f16(tmem_base + 256, ad, sdesc_sw128(sb + 256 * kBK * 2 + kk * 32), id2, accum);
+        }
+        umma_commit(empty + stage);
+        if (++stage == S) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      if (ok) umma_commit(tfull);
+      umma_commit(drain);
+      drain_wait(drain, 0);
+    }
+    __syncwarp();
+  } else {
+    const int q = warp & 3;
+    const int row = q * 32 + lane;
+    const int64_t t = (int64_t)row0 + row;
+    if (mbar_wait(tfull, 0, abort_flag, p.status, tcode | 4)) {
+      tc_fence_after();
+      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16);
+      float tv[kMaxK];
+      int te[kMaxK];
+#pragma unroll
+      for (int i = 0; i < kMaxK; ++i) {
+        tv[i] = -INFINITY;
+        te[i] = -1;
+      }
+      float kth = -INFINITY;
+      const int k = p.k;
+      for (int c = 0; c < p.E_pad; c += 32) {
+        uint32_t a[32];
+        tmem_ld32(tb + c, a);
+        tmem_wait_regs(a);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const int e = c + j;
+          if (e < p.E) {
+            float v = __uint_as_float(a[j]);
+            if (p.bias) v += __ldg(p.bias + e);
+            if (v > kth) {
+#pragma unroll
+              for (int i = kMaxK - 1; i > 0; --i) {
+                if (i < k) {
+                  if (tv[i - 1] < v) {
+                    tv[i] = tv[i - 1];
+                    te[i] = te[i - 1];
+                  } else if (tv[i] < v) {
+                    tv[i] = v;
+                    te[i] = e;
+                  }
+                }
+              }
+              if (tv[0] < v) {
+                tv[0] = v;
+                te[0] = e;
+              }
+#pragma unroll
+              for (int i = 0; i < kMaxK; ++i)
+                if (i == k - 1) kth = tv[i];
+            }
+          }
+        }
+      }
+      if (t < p.T) {
+        float den = 0.f;
+#pragma unroll
+        for (int i = 0; i < kMaxK; ++i)
+          if (i < k) den += __expf(tv[i] - tv[0]);
+        const float inv = 1.0f / den;
+#pragma unroll
+        for (int i = 0; i < kMaxK; ++i)
+          if (i < k) {
+            p.ids[t * k + i] = te[i];
+            p.tw[t * k + i] = __expf(tv[i] - tv[0]) * inv;
+          }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem_base, p.tmem_cols);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,92 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/moe.h declares, and rejects bad arguments on the host before it
+touches CUDA (null or misaligned pointers, bad sizes, a short workspace)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import sparse_moe_layer_top_b200 as moe
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return sorted(set(re.findall(r"MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for f in ("moe_router_topk", "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward"):
+        assert f in names
+
+
+def test_library_exports_every_declared_symbol():
+    L = ctypes.CDLL(moe.lib_path)
+    for name in _declared():
+        assert hasattr(L, name), name
+    assert set(_declared()) == set(moe.EXPORTS)
+
+
+def P(**kw):
+    base = dict(T=64, d=256, E=16, k=2, I=128, I_s=64, act="bf16", w="bf16")
+    base.update(kw)
+    return moe.Problem.make(**base)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(), 0),
+    (dict(T=0), 0),
+    (dict(act="f32", w="f32"), 0),
+    (dict(w="fp8", d=256, I=128, I_s=128), 0),
+    (dict(T=-1), 1),
+    (dict(k=0), 1),
+    (dict(k=17, E=32), 1),
+    (dict(k=5, E=4), 1),
+    (dict(E=513), 2),
+    (dict(d=100), 3),
+    (dict(I=12), 3),
+    (dict(act="f32", w="bf16"), 2),
+    (dict(w="fp8", d=192), 1),
+    (dict(I_s=0), 0),
+])
+def test_check_problem(kw, status):
+    assert moe.lib().moe_check_problem(ctypes.byref(P(**kw))) == status
+
+
+def test_workspace_sizes_grow_with_tokens():
+    a = moe.workspace_size(P(T=64))
+    b = moe.workspace_size(P(T=4096))
+    assert 0 < a < b
+    assert moe.workspace_size(P(k=0)) == 0
+    # forward workspace holds at least the dispatched rows, H and the fp32 output
+    p = P(T=4096)
+    Rp = 4096 * 3
+    assert b >= Rp * 256 * 2 + Rp * 128 * 2 + 4096 * 256 * 4
+    assert moe.stage_workspace_size(p) < b
+
+
+def _call_forward(prob, x=16, wr=16, y=16, ws=16, ws_bytes=None, wg=16):
+    L = moe.lib()
+    v = lambda a: None if a is None else ctypes.c_void_p(a)
+    n = moe.workspace_size(prob) if ws_bytes is None else ws_bytes
+    return L.moe_layer_forward(ctypes.byref(prob), v(x), v(wr), None, v(wg), v(16), v(16), v(16), v(16), v(16),
+                               None, v(y), None, None, v(ws), n, None)
+
+
+def test_host_rejects_before_any_launch():
+    prob = P()
+    # fake (never dereferenced) 16-byte aligned addresses; every case fails on the host
+    assert _call_forward(prob, x=None) == 1
+    assert _call_forward(prob, wg=None) == 1
+    assert _call_forward(prob, y=0x1008) == 3
+    assert _call_forward(prob, ws_bytes=moe.workspace_size(prob) - 1) == 4
+    assert b"workspace" in moe.lib().moe_last_error_string()
+    assert _call_forward(P(E=600)) == 2
+
+
+def test_set_path_validates():
+    assert moe.lib().moe_set_path(3) == 1
+    assert moe.lib().moe_set_path(0) == 0

@@ -1,0 +1,243 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle.
+
+Inputs come from moe_inputs (seeded), drawn on the CPU and copied to the GPU,
+so both sides see the same values.  Sizes span several tiles and ragged tails
+while the oracle still finishes in seconds.
+"""
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs
+import oracle
+from parity import TOL, TOL_W, check_routing, precision_key, rel_l2, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def moe():
+    import sparse_moe_layer_top_b200 as m
+    yield m
+    m.set_path(0)
+
+
+def _prob(moe, inp):
+    return moe.Problem.make(inp.T, inp.d, inp.E, inp.k, inp.I, inp.I_s, inp.act, inp.w)
+
+
+def _no_device_errors(moe):
+    s, detail = moe.device_status()
+    assert s == 0, "device status %d detail 0x%08x" % (s, detail & 0xffffffff)
+
+
+# (T, d, E, k, I, I_s, act, w, bias)
+FORWARD_CASES = {
+    "tiny_fp32": (32, 128, 16, 2, 64, 64, "f32", "f32", None),
+    "fp32_ragged": (77, 96, 24, 3, 40, 24, "f32", "f32", None),
+    "bf16_multi_tile": (300, 256, 20, 4, 192, 128, "bf16", "bf16", None),
+    "bf16_35b_shape_T256": (256, 2048, 256, 8, 512, 512, "bf16", "bf16", None),
+    "bf16_E512_k10": (130, 512, 512, 10, 256, 256, "bf16", "bf16", None),
+    "bf16_zipf": (200, 256, 64, 6, 128, 128, "bf16", "bf16", "zipf"),
+    "bf16_no_shared": (150, 192, 12, 2, 96, 0, "bf16", "bf16", None),
+    "bf16_T1": (1, 256, 40, 5, 128, 64, "bf16", "bf16", None),
+    "bf16_I_ne_Is": (129, 256, 16, 3, 136, 264, "bf16", "bf16", None),
+    "fp8_small": (64, 256, 8, 2, 256, 128, "bf16", "fp8", None),
+}
+
+
+def _make(case, seed=0):
+    T, d, E, k, I, I_s, act, w, bias = FORWARD_CASES[case]
+    return moe_inputs.make_inputs(T, d, E, k, I, I_s, act=act, w=w, bias=bias, seed=seed,
+                                  shared=I_s > 0)
+
+
+def _oracle_forward(inp, force_ids=None):
+    return oracle.moe_forward(inp.x, inp.w_r, inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu, inp.s_wd, inp.k,
+                              bias=inp.bias, scales=inp.scales, force_ids=force_ids)
+
+
+def _gpu_forward(moe, g):
+    prob = _prob(moe, g)
+    ids = torch.empty((g.T, g.k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((g.T, g.k), dtype=torch.float32, device="cuda")
+    y = moe.layer_forward(prob, g.x, g.w_r, g.bias, g.wg, g.wu, g.wd, g.s_wg, g.s_wu, g.s_wd, g.scales,
+                          topk_ids=ids, topk_w=tw)
+    torch.cuda.synchronize()
+    return y.float().cpu().numpy(), ids.cpu().numpy(), tw.cpu().numpy()
+
+
+@pytest.mark.parametrize("path", [0, 1])
+@pytest.mark.parametrize("case", list(FORWARD_CASES))
+def test_forward_matches_oracle(moe, case, path):
+    inp = _make(case)
+    if path == 1 and inp.act == "bf16" and inp.d * inp.I > 1 << 20:
+        pytest.skip("SIMT path at this size is covered by the smaller cases")
+    moe.set_path(path)
+    g = to_device(inp, "cuda")
+    y, ids, tw = _gpu_forward(moe, g)
+    _no_device_errors(moe)
+    key = precision_key(inp)
+    y_or, ids_or, w_or, probs = _oracle_forward(inp)
+    use, differ = check_routing(ids, tw, probs, ids_or, TOL_W[key])
+    if differ:
+        y_or, *_ = _oracle_forward(inp, force_ids=use)
+    err = rel_l2(y, y_or)
+    assert err <= TOL[key], "rel-L2 %.3g > %.3g (near-tie tokens with another set: %d)" % (err, TOL[key], differ)
+
+
+@pytest.mark.parametrize("case", ["tiny_fp32", "bf16_multi_tile", "bf16_E512_k10", "bf16_zipf", "bf16_T1"])
+def test_router_matches_oracle(moe, case):
+    inp = _make(case)
+    g = to_device(inp, "cuda")
+    ids, tw = moe.router_topk(_prob(moe, g), g.x, g.w_r, g.bias)
+    torch.cuda.synchronize()
+    _no_device_errors(moe)
+    probs, ids_or, _ = oracle.router(inp.x, inp.w_r, inp.k, bias=inp.bias)
+    check_routing(ids.cpu().numpy(), tw.cpu().numpy(), probs, ids_or, TOL_W[precision_key(inp)])
+
+
+@pytest.mark.parametrize("T,E,k,act", [(37, 9, 3, "f32"), (1000, 64, 8, "bf16"), (5000, 512, 10, "bf16"),
+                                       (3, 600 // 2, 16, "bf16"), (1, 4, 4, "f32")])
+def test_permute_is_the_oracles_stable_sort(moe, T, E, k, act):
+    d = 64
+    inp = moe_inputs.make_inputs(T, d, E, k, 16, 16, act=act, w=act, seed=T)
+    ids, tw = moe_inputs.random_routing(T, E, k, seed=T + 1)
+    prob = moe.Problem.make(T, d, E, k, 16, 16, act, act)
+    out = moe.permute(prob, inp.x.cuda(), ids.cuda(), tw.cuda())
+    torch.cuda.synchronize()
+    _no_device_errors(moe)
+    offs, row_tok, _, pos = oracle.permute(ids.numpy(), E)
+    assert np.array_equal(out["offs"].cpu().numpy(), offs)
+    assert np.array_equal(out["row_tok"].cpu().numpy(), row_tok)
+    assert np.array_equal(out["pos"].cpu().numpy(), pos)
+    rw = out["row_w"].cpu().numpy()
+    R = T * k
+    assert np.array_equal(rw[:R], tw.numpy().reshape(-1)[np.argsort(pos.reshape(-1))])
+    assert (rw[R:] == 1.0).all()
+    assert torch.equal(out["x_perm"].cpu(), inp.x[torch.from_numpy(row_tok).long()])
+
+
+def test_permute_single_hot_expert_and_empty_experts(moe):
+    T, E, k, d = 700, 33, 1, 32
+    ids = torch.full((T, k), 17, dtype=torch.int32)
+    tw = torch.ones((T, k))
+    x = torch.randn(T, d)
+    prob = moe.Problem.make(T, d, E, k, 8, 8, "f32", "f32")
+    out = moe.permute(prob, x.cuda(), ids.cuda(), tw.cuda())
+    torch.cuda.synchronize()
+    offs = out["offs"].cpu().numpy()
+    assert (offs[:18] == 0).all() and (offs[18:E + 1] == T).all() and offs[E + 1] == 2 * T
+    assert np.array_equal(out["row_tok"].cpu().numpy()[:T], np.arange(T))
+
+
+def _random_dispatch(E, sizes, d, act, seed):
+    """Dispatched rows for the expert stage alone: groups of the given sizes
+    (the last one the shared expert) in a buffer of R' = T*k + T rows with
+    k = 1 and T large enough, as the stage's contract has it."""
+    g = torch.Generator().manual_seed(seed)
+    R = sum(sizes)
+    T = max(sum(sizes[:E]), sizes[E], 1)
+    dt = torch.float32 if act == "f32" else torch.bfloat16
+    x_perm = torch.zeros((2 * T, d), dtype=dt)
+    x_perm[:R] = torch.randn((R, d), generator=g).to(dt)
+    offs = moe_inputs.random_groups(E, sizes)
+    return x_perm, offs, T, R
+
+
+@pytest.mark.parametrize("path", [0, 1])
+@pytest.mark.parametrize("sizes_kind", ["ragged", "one_hot_expert", "empty_shared"])
+def test_expert_ffn_matches_oracle(moe, sizes_kind, path):
+    E, d, I, I_s = 12, 256, 192, 128
+    if sizes_kind == "ragged":
+        sizes = [0, 5, 130, 1, 0, 257, 64, 3, 0, 128, 127, 9] + [150]
+    elif sizes_kind == "one_hot_expert":
+        sizes = [0] * 7 + [400] + [0] * 4 + [100]
+    else:
+        sizes = [3, 0, 70, 0, 0, 1, 2, 140, 0, 0, 0, 5] + [0]
+    inp = moe_inputs.make_inputs(1, d, E, 1, I, I_s, act="bf16", w="bf16", seed=7)
+    x_perm, offs, T, R = _random_dispatch(E, sizes, d, "bf16", 11)
+    moe.set_path(path)
+    prob = moe.Problem.make(T, d, E, 1, I, I_s, "bf16", "bf16")
+    yp = moe.expert_ffn(prob, x_perm.cuda(), offs.cuda(), inp.wg.cuda(), inp.wu.cuda(), inp.wd.cuda(),
+                        inp.s_wg.cuda(), inp.s_wu.cuda(), inp.s_wd.cuda())
+    torch.cuda.synchronize()
+    _no_device_errors(moe)
+    ref = oracle.expert_ffn(x_perm[:R], offs.numpy(), inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu, inp.s_wd)
+    got = yp[:R].float().cpu().numpy()
+    assert rel_l2(got, ref) <= TOL["bf16"]
+    # per group as well, so that a wrong group offset cannot hide in the total
+    o = offs.numpy()
+    for gi in range(E + 1):
+        if o[gi + 1] > o[gi]:
+            assert rel_l2(got[o[gi]:o[gi + 1]], ref[o[gi]:o[gi + 1]]) <= TOL["bf16"], "group %d" % gi
+
+
+@pytest.mark.parametrize("act", ["f32", "bf16"])
+def test_combine_matches_oracle(moe, act):
+    T, E, k, d = 93, 10, 3, 136
+    ids, tw = moe_inputs.random_routing(T, E, k, seed=5)
+    offs, row_tok, _, pos = oracle.permute(ids.numpy(), E)
+    R = T * (k + 1)
+    dt = torch.float32 if act == "f32" else torch.bfloat16
+    y_perm = torch.randn((R, d), generator=torch.Generator().manual_seed(3)).to(dt)
+    prob = moe.Problem.make(T, d, E, k, 8, 8, act, act)
+    y = moe.combine(prob, y_perm.cuda(), torch.from_numpy(pos).cuda(), tw.cuda(), torch.from_numpy(offs).cuda())
+    torch.cuda.synchronize()
+    ref = oracle.combine(y_perm, pos, tw, offs, E)
+    assert rel_l2(y.float().cpu().numpy(), ref) <= (1e-6 if act == "f32" else 5e-3)
+
+
+def test_stages_chain_to_the_forward(moe):
+    inp = _make("bf16_multi_tile", seed=3)
+    g = to_device(inp, "cuda")
+    prob = _prob(moe, g)
+    ids, tw = moe.router_topk(prob, g.x, g.w_r, g.bias)
+    pm = moe.permute(prob, g.x, ids, tw)
+    yp = moe.expert_ffn(prob, pm["x_perm"], pm["offs"], g.wg, g.wu, g.wd, g.s_wg, g.s_wu, g.s_wd)
+    y_stage = moe.combine(prob, yp, pm["pos"], tw, pm["offs"])
+    y_fused = moe.layer_forward(prob, g.x, g.w_r, g.bias, g.wg, g.wu, g.wd, g.s_wg, g.s_wu, g.s_wd)
+    torch.cuda.synchronize()
+    _no_device_errors(moe)
+    assert rel_l2(y_stage.float().cpu().numpy(), y_fused.float().cpu().numpy()) <= 1e-2
+
+
+def test_paths_agree_bf16(moe):
+    inp = _make("bf16_35b_shape_T256", seed=1)
+    g = to_device(inp, "cuda")
+    out = []
+    for path in (1, 2):
+        moe.set_path(path)
+        y, ids, tw = _gpu_forward(moe, g)
+        out.append((y, ids))
+    moe.set_path(0)
+    assert rel_l2(out[1][0], out[0][0]) <= 1e-2
+
+
+def test_out_of_range_expert_id_sets_device_status(moe):
+    T, E, k, d = 64, 8, 2, 32
+    ids, tw = moe_inputs.random_routing(T, E, k, seed=2)
+    ids[5, 1] = E  # not a valid expert
+    prob = moe.Problem.make(T, d, E, k, 8, 8, "f32", "f32")
+    out = moe.permute(prob, torch.randn(T, d).cuda(), ids.cuda(), tw.cuda())
+    s, detail = moe.device_status()
+    assert s == 6 and detail == 0x06000001
+    assert int(out["pos"][5, 1]) == -1
+    assert moe.device_status()[0] == 0  # reading clears it
+
+
+def test_repeat_calls_are_deterministic_in_routing_and_close_in_output(moe):
+    inp = _make("bf16_multi_tile", seed=4)
+    g = to_device(inp, "cuda")
+    y1, ids1, tw1 = _gpu_forward(moe, g)
+    y2, ids2, tw2 = _gpu_forward(moe, g)
+    assert np.array_equal(ids1, ids2) and np.array_equal(tw1, tw2)
+    assert rel_l2(y1, y2) <= 1e-3  # only the order of the fp32 reductions may differ
+
+
+def test_launch_count_reported(moe):
+    inp = _make("bf16_multi_tile")
+    g = to_device(inp, "cuda")
+    moe.set_path(0)
+    _gpu_forward(moe, g)
+    assert moe.last_launch_count() >= 7
