@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Throughput of the sparse MoE block on B200 (tokens/s), one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+A step is one full forward of the block (router + top-k, dispatch, gate/up
+GEMM with SwiGLU, down GEMM with the weighted combine, shared expert) over one
+batch of T synthetic tokens resident in HBM.  With N > 1 (torchrun, one
+process per GPU) every rank runs its own batch against its own copy of the
+weights -- the block needs no exchange between batches -- so the scaling is
+weak and no collective touches the data path; the step time is the maximum
+over ranks.
+
+`--impl reference` times the float64 CPU oracle on this machine's cores
+instead (the reference arm): same workload, metric and unit, each step a
+bounded sample of the batch's tokens.
+"""
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer tokens/s at 1 B200; % HBM roofline (decode) / % bf16 TC peak (prefill)"
+UNIT = "tokens/s"
+DEFAULT_CONFIG = "qwen36_35b_a3b_bf16"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLUSH_BYTES = 256 << 20
+KERNEL_SOURCES = ("api.cu", "common.cuh", "permute.cuh", "ptx.cuh", "router.cuh", "simt.cuh", "tc_gemm.cuh")
+
+
+# ---------------------------------------------------------------- helpers
+def kernel_source_sha():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "sparse_moe_layer_top_b200", "csrc")
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(d, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, if it still matches the kernel source."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        for e in d.get("entries", []):
+            if e["kernel"] == kernel and e["workload"] == workload and e["source_sha"] == kernel_source_sha():
+                return float(e["dram_bytes_per_launch"])
+    except Exception:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="moe_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), "--query-gpu=" + self.Q,
+                                          "--format=csv,noheader,nounits", "-lms", "200", "-f", self.path],
+                                         stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    c = [x.strip() for x in line.split(",")]
+                    if len(c) >= 9:
+                        rows.append(c)
+            os.unlink(self.path)
+        except Exception:
+            pass
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [s for s in sm if s > 0.5 * (max(mx) if mx else 1)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def routing_counts(moe, layer, x):
+    """Rows per group from the block's own router (outside the timed region)."""
+    import torch
+    prob = layer.problem(x.shape[0])
+    w_router, bias = layer.w[0], layer.w[1]
+    ids, _ = moe.router_topk(prob, x, w_router, bias)
+    cnt = torch.bincount(ids.reshape(-1).long(), minlength=prob.E).cpu().tolist()
+    return cnt
+
+
+def work_model(c, counts, T):
+    """Algorithmic bytes and flops of the block and of its two expert GEMMs.
+
+    Weights are counted for the experts that received at least one row (and
+    the shared expert); each kernel's activations once in and once out (the
+    gate/up GEMM reads the dispatched rows and writes H; the down GEMM reads H
+    and writes the weighted (token, slot) rows).  For the whole block only the
+    weights, W_r, x and y count: the dispatch copy, H and the slot rows are
+    overheads."""
+    d, E, k, I, I_s = c["d"], c["E"], c["k"], c["I"], c["I_s"]
+    ab = 4 if c["act"] == "f32" else 2
+    wb = {"f32": 4, "bf16": 2, "fp8": 1}[c["w"]]
+    active = sum(1 for n in counts if n > 0)
+    R = sum(counts)
+    sh = 1 if I_s > 0 else 0
+    w_gu = (active * 2 * d * I + sh * 2 * d * I_s) * wb
+    w_dn = (active * d * I + sh * d * I_s) * wb
+    h_bytes = (R * I + sh * T * I_s) * ab
+    g1 = {"bytes": w_gu + (R + sh * T) * d * ab + h_bytes, "flops": 4 * d * (R * I + sh * T * I_s)}
+    g2 = {"bytes": w_dn + h_bytes + (R + sh * T) * d * ab, "flops": 2 * d * (R * I + sh * T * I_s)}
+    layer = {"bytes": w_gu + w_dn + E * d * ab + 2 * T * d * ab,
+             "flops": 2 * T * d * E + 6 * d * (R * I + sh * T * I_s)}
+    if c["w"] == "fp8":
+        n_sc = (E * 3 * (I // 128) * (d // 128) + sh * 3 * (I_s // 128) * (d // 128)) * 4
+        layer["bytes"] += n_sc * active // max(E, 1)
+    return {"active_experts": active, "rows": R, "gemm_gate_up": g1, "gemm_down": g2, "layer": layer}
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+def oracle_sample_time(inp_cpu_fn, n_tokens):
+    """Seconds the oracle takes for the first n tokens (full weights on the host)."""
+    import oracle
+    c = inp_cpu_fn()
+    x = c["x"][:n_tokens]
+    t0 = time.perf_counter()
+    oracle.moe_forward(x, c["w_r"], c["wg"], c["wu"], c["wd"], c["s_wg"], c["s_wu"], c["s_wd"], c["k"],
+                       bias=c["bias"], scales=c["scales"], want_probs=False)
+    return time.perf_counter() - t0
+
+
+def host_copy(inp):
+    out = {}
+    for n in ("x", "w_r", "bias", "wg", "wu", "wd", "s_wg", "s_wu", "s_wd", "scales"):
+        t = getattr(inp, n)
+        out[n] = None if t is None else t.detach().cpu()
+    out["k"] = inp.k
+    return out
+
+
+def cpu_baseline(inp, target_s=15.0):
+    """The oracle, as it stands, on a bounded token sample of the batch."""
+    import oracle
+    wbytes = sum(getattr(inp, n).numel() * getattr(inp, n).element_size()
+                 for n in ("wg", "wu", "wd") if getattr(inp, n) is not None)
+    if wbytes > (8 << 30):
+        return {"value": None, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                "sample": "not run: weights too large to copy to the host here"}
+    host = host_copy(inp)
+    probe = 16
+    t_probe = oracle_sample_time(lambda: host, probe)
+    n = int(max(probe, min(inp.T, target_s * probe / max(t_probe, 1e-6))))
+    n = max(probe, n - n % 8)
+    t = oracle_sample_time(lambda: host, n)
+    return {"value": n / t, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "first %d of %d tokens of the batch, full block in float64 (%.1f s)" % (n, inp.T, t)}
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def aggregate(step_ms, tokens, world, device=None):
+    """(max step ms over ranks, total tokens over ranks); plain values when alone."""
+    if world <= 1:
+        return step_ms, tokens
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([step_ms], dtype=torch.float64, device=device)
+    n = torch.tensor([float(tokens)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dist.all_reduce(n, op=dist.ReduceOp.SUM)
+    return float(t.item()), int(n.item())
+
+
+def barrier(world, device=None):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+
+    import moe_inputs
+    import sparse_moe_layer_top_b200 as moe
+
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", device_id=dev, timeout=datetime.timedelta(seconds=300))
+
+    cfg = dict(moe_inputs.CONFIGS[args.config])
+    inp = moe_inputs.make_config(args.config, seed=0, device=dev, x_seed=rank)
+    T = inp.T
+    layer = moe.MoELayer.from_inputs(inp, max_tokens=T)
+    x = inp.x
+    y = torch.empty((T, inp.d), dtype=x.dtype, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    counts = routing_counts(moe, layer, x)
+    work = work_model(cfg, counts, T)
+
+    for _ in range(args.warmup):
+        layer(x, y)
+    torch.cuda.synchronize()
+    s, detail = moe.device_status()
+    if s != 0:
+        raise RuntimeError("device status %d (0x%08x) after warm-up" % (s, detail & 0xffffffff))
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    clocks = ClockSampler(local)
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    clocks.start()
+    moe.profile_enable(2)  # events around the tensor-core GEMMs only
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record()
+        layer(x, y)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    launches_per_step = moe.last_launch_count()
+    prof = moe.profile_read()
+    moe.profile_enable(0)
+    clk = clocks.stop()
+    step_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    ms_max, tokens_all = aggregate(step_ms, T, world, dev)
+
+    # per-kernel durations of the GEMMs (CUDA events on the launching stream, timed region)
+    per = {}
+    for name, ms in prof:
+        per.setdefault(name, []).append(ms)
+    kern = {n: statistics.mean(v) for n, v in per.items()}
+
+    # end to end through the public API: pinned host x in, pinned host y out
+    xh = x.cpu().pin_memory()
+    yh = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+    xd = torch.empty_like(x)
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for _ in range(2):
+        xd.copy_(xh, non_blocking=True)
+        layer(xd, y)
+        yh.copy_(y, non_blocking=True)
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    for i in range(K):
+        flush.zero_()
+        e2e_ev[i][0].record()
+        xd.copy_(xh, non_blocking=True)
+        layer(xd, y)
+        yh.copy_(y, non_blocking=True)
+        e2e_ev[i][1].record()
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    e2e_ms = statistics.mean(a.elapsed_time(b) for a, b in e2e_ev)
+    e2e_max, _ = aggregate(e2e_ms, T, world, dev)
+    s, detail = moe.device_status()
+    if s != 0:
+        raise RuntimeError("device status %d (0x%08x) after the timed steps" % (s, detail & 0xffffffff))
+
+    peaks, peak_src = load_peaks()
+    line = None
+    if rank == 0:
+        gemms = {"gemm_tc_swiglu": work["gemm_gate_up"], "gemm_tc_down": work["gemm_down"]}
+        dom = max((n for n in gemms if n in kern), key=lambda n: kern[n], default=None)
+        roof = None
+        if dom is not None:
+            wk = gemms[dom]
+            t_s = kern[dom] / 1e3
+            hbm_t = wk["bytes"] / (peaks["hbm_gbs"] * 1e9)
+            tc_t = wk["flops"] / (peaks["bf16_tflops"] * 1e12)
+            if hbm_t >= tc_t:
+                roof = {"bound": "hbm", "achieved": wk["bytes"] / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+            else:
+                roof = {"bound": "tensor", "achieved": wk["flops"] / t_s / 1e12, "peak": peaks["bf16_tflops"],
+                        "unit": "TFLOP/s"}
+            roof["frac"] = roof["achieved"] / roof["peak"]
+            roof["traffic"] = load_traffic(dom, args.config)
+            roof.update({"kernel": dom, "kernel_ms": kern[dom], "algorithmic_bytes": wk["bytes"],
+                         "algorithmic_flops": wk["flops"], "peak_source": peak_src + " (burst)"})
+        lw = work["layer"]
+        st = step_ms / 1e3
+        layer_roof = {"bytes": lw["bytes"], "flops": lw["flops"],
+                      "hbm_frac": lw["bytes"] / st / 1e9 / peaks["hbm_gbs"],
+                      "tc_frac": lw["flops"] / st / 1e12 / peaks["bf16_tflops"],
+                      "achieved_gbs": lw["bytes"] / st / 1e9, "achieved_tflops": lw["flops"] / st / 1e12,
+                      "active_experts": work["active_experts"], "peak_source": peak_src}
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            cpu = cpu_baseline(inp, args.cpu_seconds)
+        line = {
+            "metric": METRIC, "value": tokens_all / (ms_max / 1e3), "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": cfg["act"], "data": "synthetic (seeded N(0,1) tokens, N(0,0.02^2) weights)",
+            "config": {"workload": args.config, "T": T, "d": cfg["d"], "E": cfg["E"], "k": cfg["k"], "I": cfg["I"],
+                       "I_s": cfg["I_s"], "act": cfg["act"], "weights": cfg["w"],
+                       "router_bias": cfg["bias"], "global_tokens": tokens_all,
+                       "parallelism": "dp%d (independent token batches per GPU, weights replicated)" % world,
+                       "l2": "flushed between timed steps (256 MiB write outside the events)"},
+            "roofline": roof, "layer_roofline": layer_roof, "cpu_baseline": cpu,
+            "e2e": {"value": tokens_all / (e2e_max / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": x.numel() * x.element_size(),
+                    "d2h_bytes_per_step": y.numel() * y.element_size()},
+            "gpu_launches": launches_per_step * K, "launches_per_step": launches_per_step,
+            "kernel_ms": kern, "clocks": clk, "impl": "ours",
+        }
+    if world > 1:
+        dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args):
+    """The float64 oracle on the host cores, on a bounded sample per step."""
+    world, rank, local = dist_env()
+    if rank != 0:
+        return
+    import torch
+
+    import moe_inputs
+    import oracle
+
+    cfg = dict(moe_inputs.CONFIGS[args.config])
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    inp = moe_inputs.make_config(args.config, seed=0, device=dev)
+    wbytes = sum(getattr(inp, n).numel() * getattr(inp, n).element_size() for n in ("wg", "wu", "wd"))
+    if wbytes > (8 << 30):
+        print(json.dumps({"impl": "reference", "unavailable": "the float64 oracle needs the full weights on the "
+                          "host; %.1f GB is beyond this arm's host-memory budget" % (wbytes / 1e9)}))
+        return
+    host = host_copy(inp)
+    per_step = args.ref_tokens
+    samples = []
+    for i in range(args.warmup + args.steps):
+        lo = (i * per_step) % max(inp.T - per_step + 1, 1)
+        x = host["x"][lo:lo + per_step]
+        t0 = time.perf_counter()
+        oracle.moe_forward(x, host["w_r"], host["wg"], host["wu"], host["wd"], host["s_wg"], host["s_wu"],
+                           host["s_wd"], host["k"], bias=host["bias"], scales=host["scales"], want_probs=False)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            samples.append(dt)
+    ms = statistics.mean(samples) * 1e3
+    value = per_step / (ms / 1e3)
+    sample = "%d tokens of the %d-token batch per step, full block in float64" % (per_step, inp.T)
+    print(json.dumps({
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) tokens, N(0,0.02^2) weights)",
+        "config": {"workload": args.config, "T": inp.T, "d": cfg["d"], "E": cfg["E"], "k": cfg["k"],
+                   "I": cfg["I"], "I_s": cfg["I_s"], "act": cfg["act"], "weights": cfg["w"],
+                   "tokens_per_step": per_step},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    import moe_inputs
+    ap.add_argument("--config", choices=sorted(moe_inputs.CONFIGS), default=DEFAULT_CONFIG)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-tokens", type=int, default=32)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    world, _, _ = dist_env()
+    if world != args.gpus and not (world == 1 and args.gpus == 1):
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus %d needs torchrun with %d processes" % (args.gpus, args.gpus))
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

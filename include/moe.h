@@ -98,10 +98,12 @@ MOE_API size_t moe_stage_workspace_size(const moe_problem* p);
 /* Router stage (steps 1-3).  x [T, d]; w_router [E, d]; router_bias [E] fp32
  * or NULL (added to the logits before the softmax).  Writes topk_ids
  * int32 [T, k] (descending probability, equal values -> lower index) and
- * topk_w fp32 [T, k] (renormalised, each row sums to 1). */
+ * topk_w fp32 [T, k] (renormalised, each row sums to 1).  ws:
+ * moe_stage_workspace_size() bytes (holds the logits; may be NULL for F32
+ * problems). */
 MOE_API moe_status moe_router_topk(const moe_problem* p, const void* x, const void* w_router,
                            const float* router_bias, int32_t* topk_ids, float* topk_w,
-                           void* stream);
+                           void* ws, size_t ws_bytes, void* stream);
 
 /* Dispatch stage (the token is "sent to" its experts, Qwen3.6 explainer,
  * router paragraph): a stable sort of the T*k (token, slot) pairs by expert.
@@ -155,6 +157,19 @@ MOE_API moe_status moe_device_status(int32_t* detail);
 
 /* Number of kernels the last successful call on this thread launched. */
 MOE_API int moe_last_launch_count(void);
+
+/* Per-launch timing for profiling.  on = 1: every kernel the calling thread
+ * launches through this library is bracketed by two CUDA events recorded on
+ * its stream; on = 2: only the tensor-core GEMM launches; on = 0: off.
+ * Events are created once and reused; at most 4096 launches are recorded
+ * until the next read.  Every call clears the record. */
+MOE_API moe_status moe_profile_enable(int on);
+
+/* Copy up to `max` recorded launches, in launch order, into ms[] (device
+ * milliseconds, -1 if unavailable) and names[] (static strings owned by the
+ * library; either array may be NULL), waiting for each launch's end event.
+ * Returns the number copied and clears the record. */
+MOE_API int moe_profile_read(int max, float* ms, const char** names);
 
 MOE_API const char* moe_last_error_string(void);
 

@@ -3,8 +3,8 @@
 Argument marshalling only: every step of the block runs in the library's CUDA
 kernels.  Tensors are CUDA torch tensors (contiguous, row-major); the calls
 enqueue on the current torch stream and never synchronise.  The library is
-built in-tree (``python -m sparse_moe_layer_top_b200.build``); importing this
-package without it raises at once -- there is no fallback.
+built in-tree (``python -m sparse_moe_layer_top_b200.build``) and loaded on
+first use; every call raises if it is missing -- there is no fallback.
 
 Entry points mirror ``include/moe.h``: ``router_topk``, ``permute``,
 ``expert_ffn``, ``combine``, ``layer_forward``; ``MoELayer`` keeps a
@@ -17,6 +17,7 @@ import torch
 
 __all__ = ["MoEError", "Problem", "router_topk", "permute", "expert_ffn", "combine", "layer_forward",
            "workspace_size", "stage_workspace_size", "set_path", "device_status", "last_launch_count",
+           "profile_enable", "profile_read",
            "MoELayer", "lib_path", "F32", "BF16", "FP8_E4M3_B128"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -27,7 +28,8 @@ _STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "
            4: "MOE_ERR_WORKSPACE_TOO_SMALL", 5: "MOE_ERR_CUDA", 6: "MOE_ERR_DEVICE_CHECK", 7: "MOE_ERR_TIMEOUT"}
 EXPORTS = ("moe_check_problem", "moe_workspace_size", "moe_stage_workspace_size", "moe_router_topk",
            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_set_path",
-           "moe_device_status", "moe_last_launch_count", "moe_last_error_string")
+           "moe_device_status", "moe_last_launch_count", "moe_profile_enable", "moe_profile_read",
+           "moe_last_error_string")
 
 
 class MoEError(RuntimeError):
@@ -63,7 +65,7 @@ def lib():
         L.moe_workspace_size.restype = ctypes.c_size_t
         L.moe_stage_workspace_size.argtypes = [PP]
         L.moe_stage_workspace_size.restype = ctypes.c_size_t
-        L.moe_router_topk.argtypes = [PP, P, P, P, P, P, P]
+        L.moe_router_topk.argtypes = [PP, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_permute.argtypes = [PP, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_expert_ffn.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_combine.argtypes = [PP, P, P, P, P, P, P]
@@ -71,6 +73,11 @@ def lib():
         L.moe_set_path.argtypes = [ctypes.c_int]
         L.moe_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32)]
         L.moe_last_launch_count.restype = ctypes.c_int
+        L.moe_profile_enable.argtypes = [ctypes.c_int]
+        L.moe_profile_enable.restype = ctypes.c_int
+        L.moe_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_float),
+                                       ctypes.POINTER(ctypes.c_char_p)]
+        L.moe_profile_read.restype = ctypes.c_int
         L.moe_last_error_string.restype = ctypes.c_char_p
         for f in ("moe_check_problem", "moe_router_topk", "moe_permute", "moe_expert_ffn", "moe_combine",
                   "moe_layer_forward", "moe_set_path", "moe_device_status"):
@@ -131,20 +138,36 @@ def last_launch_count():
     return lib().moe_last_launch_count()
 
 
+def profile_enable(mode=1):
+    """1: bracket every library kernel launch of this thread with CUDA events;
+    2: only the tensor-core GEMM launches; 0: off."""
+    _check(lib().moe_profile_enable(int(mode)))
+
+
+def profile_read(max_launches=4096):
+    """[(kernel name, device ms), ...] of the launches recorded since the last
+    read (waits for them), in launch order."""
+    ms = (ctypes.c_float * max_launches)()
+    names = (ctypes.c_char_p * max_launches)()
+    n = lib().moe_profile_read(max_launches, ms, names)
+    return [(names[i].decode(), float(ms[i])) for i in range(n)]
+
+
 def _ws(nbytes, device, ws):
     if ws is None:
         ws = torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device)
     return ws
 
 
-def router_topk(prob, x, w_router, bias=None, topk_ids=None, topk_w=None, stream=None):
+def router_topk(prob, x, w_router, bias=None, topk_ids=None, topk_w=None, ws=None, stream=None):
     T, k = prob.T, prob.k
     if topk_ids is None:
         topk_ids = torch.empty((T, k), dtype=torch.int32, device=x.device)
     if topk_w is None:
         topk_w = torch.empty((T, k), dtype=torch.float32, device=x.device)
+    ws = _ws(stage_workspace_size(prob), x.device, ws)
     _check(lib().moe_router_topk(ctypes.byref(prob), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(topk_ids),
-                                 _ptr(topk_w), _stream(stream)))
+                                 _ptr(topk_w), _ptr(ws), ws.numel(), _stream(stream)))
     return topk_ids, topk_w
 
 
@@ -232,6 +255,3 @@ class MoELayer:
     def from_inputs(cls, inp, max_tokens=0):
         return cls(inp.d, inp.E, inp.k, inp.I, inp.I_s, inp.w_r, inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu,
                    inp.s_wd, bias=inp.bias, scales=inp.scales, act=inp.act, w=inp.w, max_tokens=max_tokens)
-
-
-lib()

@@ -13,6 +13,7 @@
 #include "../../include/moe.h"
 #include "common.cuh"
 #include "permute.cuh"
+#include "router.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
 
@@ -22,6 +23,7 @@ using namespace moe;
 static thread_local char g_err[512] = "no error";
 static thread_local int g_launches = 0;
 static thread_local int g_launches_pending = 0;
+constexpr int kProfileCapacity = 4096;
 
 static moe_status fail(moe_status s, const char* fmt, ...) {
   va_list ap;
@@ -37,10 +39,52 @@ static moe_status fail(moe_status s, const char* fmt, ...) {
     if (e_ != cudaSuccess) return fail(MOE_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
   } while (0)
 
-#define LAUNCH_CHECK(name)                                                                   \
+// Optional per-launch timing: when enabled, every kernel launch of the
+// calling thread is bracketed by two CUDA events recorded on its stream.
+struct LaunchEvent {
+  const char* name;
+  cudaEvent_t begin, end;
+};
+struct Profiler {
+  bool on = false, pending = false;
+  int mode = 0;
+  int used = 0;
+  LaunchEvent ev[kProfileCapacity];
+  int created = 0;
+};
+static thread_local Profiler g_prof;
+
+// Mode 2 records only the tensor-core GEMM launches (names "gemm_tc_*").
+static bool prof_wants(const char* name) {
+  return g_prof.mode == 1 || (g_prof.mode == 2 && strncmp(name, "gemm_tc", 7) == 0);
+}
+static void prof_begin(const char* name, cudaStream_t st) {
+  Profiler& P = g_prof;
+  P.pending = false;
+  if (!P.on || P.used >= kProfileCapacity || !prof_wants(name)) return;
+  if (P.used == P.created) {
+    if (cudaEventCreate(&P.ev[P.used].begin) != cudaSuccess) return;
+    if (cudaEventCreate(&P.ev[P.used].end) != cudaSuccess) return;
+    ++P.created;
+  }
+  cudaEventRecord(P.ev[P.used].begin, st);
+  P.pending = true;
+}
+static void prof_end(const char* name, cudaStream_t st) {
+  Profiler& P = g_prof;
+  if (!P.on || !P.pending || P.used >= P.created) return;
+  P.pending = false;
+  P.ev[P.used].name = name;
+  cudaEventRecord(P.ev[P.used].end, st);
+  ++P.used;
+}
+
+#define PROF_BEGIN(name, st) prof_begin(name, st)
+#define LAUNCH_CHECK(name, st)                                                               \
   do {                                                                                       \
     cudaError_t e_ = cudaGetLastError();                                                     \
     if (e_ != cudaSuccess) return fail(MOE_ERR_CUDA, "launch %s: %s", name, cudaGetErrorString(e_)); \
+    prof_end(name, st);                                                                      \
     ++g_launches_pending;                                                                    \
   } while (0)
 
@@ -68,7 +112,6 @@ static cudaError_t allow_smem(K kernel, int bytes) {
 // GEMM instantiations used by the library.
 using Gemm1Cfg = TcGemmCfg<128, true, 4>;
 using Gemm2Cfg = TcGemmCfg<256, false, 4>;
-static constexpr int kRouterSmem = 227 * 1024;
 
 static moe_status device_info(DeviceInfo** out) {
   int dev = 0;
@@ -87,9 +130,9 @@ static moe_status device_info(DeviceInfo** out) {
     if (major != 10 || minor != 0)
       return fail(MOE_ERR_UNSUPPORTED, "libmoe is built for sm_100a; device %d is sm_%d%d", dev, major, minor);
     CUDA_TRY(allow_smem(k_gemm_tc<128, true, 4, kTcSwiGLU>, Gemm1Cfg::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcCombine>, Gemm2Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcSlotStore>, Gemm2Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcStore>, Gemm2Cfg::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_router_tc, kRouterSmem));
+    CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcLogits>, Gemm2Cfg::SMEM_BYTES));
     d.ready = true;
   }
   *out = &d;
@@ -185,9 +228,8 @@ static bool misaligned(const void* ptr) { return (reinterpret_cast<uintptr_t>(pt
     if ((ptr) && misaligned(ptr)) return fail(MOE_ERR_ALIGNMENT, "%s is not 16-byte aligned", #ptr); \
   } while (0)
 
-// Tensor-core kernels: bf16 activations and bf16 weights.
+// Tensor-core expert kernels: bf16 activations and bf16 weights.
 static bool tc_shapes(const moe_problem& p) { return p.act_dtype == MOE_BF16 && p.w_dtype == MOE_BF16; }
-static bool tc_router_shapes(const moe_problem& p) { return p.act_dtype == MOE_BF16; }
 
 static moe_status choose(bool tc_possible, bool* use_tc) {
   if (g_path == 1) {
@@ -202,15 +244,42 @@ static moe_status choose(bool tc_possible, bool* use_tc) {
 }
 
 // ============================================================== workspace
+// Router split along d: enough (row block, expert block, split) tiles to cover
+// the GPU, each split at least 4 K-blocks deep.  A fixed target keeps the
+// workspace size a pure function of the problem.
+constexpr int kRouterBN = 256;
+constexpr int kTargetTiles = 148;
+
+struct RouterSplit {
+  int ksplit, kb_per, tiles;
+  int64_t ldp;  // row stride of the logit partials (floats)
+};
+static RouterSplit router_split(const moe_problem& p) {
+  RouterSplit r;
+  const int kblocks = (int)cdiv(p.d, kBK);
+  const int mn = (int)(cdiv(std::max<int64_t>(p.T, 1), kBM) * cdiv(p.E, kRouterBN));
+  int ks = (int)std::min<int64_t>(cdiv(kTargetTiles, mn), std::max(1, kblocks / 4));
+  ks = std::max(ks, 1);
+  r.kb_per = (int)cdiv(kblocks, ks);
+  r.ksplit = (int)cdiv(kblocks, r.kb_per);
+  r.tiles = mn * r.ksplit;
+  r.ldp = (int64_t)align_up(p.E, 32);
+  return r;
+}
+
 struct Layout {
-  size_t counts = 0, pre_a = 0, pre_b = 0, ids = 0, tw = 0, offs = 0, row_tok = 0, row_w = 0, pos = 0, xp = 0,
-         h = 0, y32 = 0, total = 0;
+  size_t counts = 0, pre_a = 0, pre_b = 0, part = 0, ids = 0, tw = 0, offs = 0, row_tok = 0, row_w = 0, pos = 0,
+         row_dst = 0, xp = 0, h = 0, total = 0;
 };
 
 static int64_t rows_total(const moe_problem& p) { return p.T * p.k + (p.I_s > 0 ? p.T : 0); }
-static int64_t n_chunks(const moe_problem& p) { return std::max<int64_t>(1, cdiv(p.T * p.k, kChunk)); }
+static int64_t n_chunks(const moe_problem& p) { return std::max<int64_t>(1, cdiv(p.T, kChunkTokens)); }
 static int64_t ldh_of(const moe_problem& p) { return std::max(p.I, p.I_s); }
 
+// Workspace of moe_layer_forward (forward) or of the stage calls.  In the
+// forward, the dispatched rows x_perm and the weighted (token, slot) rows of
+// the down projection share one buffer: the gate/up GEMM has consumed the
+// former before the down GEMM writes the latter.
 static Layout layout(const moe_problem& p, bool forward) {
   Layout L;
   size_t o = 0;
@@ -224,6 +293,10 @@ static Layout layout(const moe_problem& p, bool forward) {
   L.counts = take(n_chunks(p) * p.E * 4);
   L.pre_a = take((p.E + 2) * 4);
   L.pre_b = take((p.E + 2) * 4);
+  if (p.act_dtype == MOE_BF16) {
+    const RouterSplit rs = router_split(p);
+    L.part = take((size_t)rs.ksplit * p.T * rs.ldp * 4);
+  }
   if (forward) {
     L.ids = take(n * 4);
     L.tw = take(n * 4);
@@ -231,10 +304,10 @@ static Layout layout(const moe_problem& p, bool forward) {
     L.row_tok = take(Rp * 4);
     L.row_w = take(Rp * 4);
     L.pos = take(n * 4);
-    L.xp = take(Rp * p.d * ab);
+    L.row_dst = take(Rp * 4);
+    L.xp = take(std::max(Rp, p.T * (p.k + 1)) * p.d * ab);
   }
   L.h = take(Rp * ldh_of(p) * ab);
-  if (forward && p.act_dtype == MOE_BF16) L.y32 = take(p.T * p.d * 4);
   L.total = o;
   return L;
 }
@@ -243,69 +316,78 @@ static Layout layout(const moe_problem& p, bool forward) {
 static Schedule sched_simt(int n_r, int n_s) { return Schedule{64, 64, n_r, n_s, 0}; }
 static Schedule sched_tc(int bn, int n_r, int n_s) { return Schedule{kBM, bn, n_r, n_s, 0}; }
 
+// Router and top-k.  `counts` (may be NULL) receives the per-chunk histograms
+// for the dispatch when the tensor-core path is taken; *counted says so.
 static moe_status launch_router(const moe_problem& p, const void* x, const void* wr, const float* bias,
-                                int32_t* ids, float* tw, cudaStream_t st, DeviceInfo* dev) {
+                                int32_t* ids, float* tw, float* part, int32_t* counts, bool* counted,
+                                cudaStream_t st, DeviceInfo* dev) {
+  *counted = false;
   if (p.T == 0) return MOE_OK;
   bool tc;
-  moe_status s = choose(tc_router_shapes(p), &tc);
+  moe_status s = choose(p.act_dtype == MOE_BF16, &tc);
   if (s != MOE_OK) return s;
   if (!tc) {
     dim3 grid((unsigned)cdiv(p.T, 8));
+    PROF_BEGIN("router_simt", st);
     if (p.act_dtype == MOE_F32)
       k_router_simt<float><<<grid, 256, 0, st>>>((const float*)x, (const float*)wr, bias, p.T, p.d, p.E, p.k, ids, tw);
     else
       k_router_simt<bf16><<<grid, 256, 0, st>>>((const bf16*)x, (const bf16*)wr, bias, p.T, p.d, p.E, p.k, ids, tw);
-    LAUNCH_CHECK("router_simt");
+    LAUNCH_CHECK("router_simt", st);
     return MOE_OK;
   }
-  TcRouterArgs a;
-  a.T = p.T;
-  a.E = p.E;
-  a.E_pad = (int)align_up(p.E, 16);
-  a.k = p.k;
-  a.kblocks = (int)cdiv(p.d, kBK);
-  a.n1 = std::min(a.E_pad, 256);
-  a.n2 = a.E_pad > 256 ? a.E_pad - 256 : 0;
-  a.tmem_cols = 32;
-  while (a.tmem_cols < a.E_pad) a.tmem_cols <<= 1;
-  const int stage_bytes = kBM * kBK * 2 + (a.n2 ? 512 : a.E_pad) * kBK * 2;
-  a.stages = std::min(4, (kRouterSmem - 1024 - 256) / stage_bytes);
-  a.bias = bias;
-  a.ids = ids;
-  a.tw = tw;
+  const RouterSplit rs = router_split(p);
+  CUtensorMap ax, bw;
+  if ((s = map2d(&ax, x, p.d, p.T, p.d, kBM)) != MOE_OK) return s;
+  if ((s = map2d(&bw, wr, p.d, p.E, p.d, kRouterBN)) != MOE_OK) return s;
+  TcGemmArgs a{};
+  a.E = 0;
+  a.N_s = p.E;
+  a.K_s = p.d;
+  a.rows_cap = p.T;
+  a.single_rows = (int)p.T;
+  a.single_tiles = rs.tiles;
+  a.ksplit = rs.ksplit;
+  a.kb_per_split = rs.kb_per;
+  a.part = part;
+  a.ldp = rs.ldp;
+  a.part_stride = p.T * rs.ldp;
   a.status = dev->status;
-  CUtensorMap tx, tw_map;
-  s = map2d(&tx, x, p.d, p.T, p.d, kBM);
-  if (s != MOE_OK) return s;
-  s = map2d(&tw_map, wr, p.d, p.E, p.d, a.n2 ? 256 : a.E_pad);
-  if (s != MOE_OK) return s;
-  const int smem = 1024 + a.stages * stage_bytes + 256;
-  k_router_tc<<<(unsigned)cdiv(p.T, kBM), 192, smem, st>>>(tx, tw_map, a);
-  LAUNCH_CHECK("router_tc");
+  PROF_BEGIN("gemm_tc_router", st);
+  k_gemm_tc<kRouterBN, false, 4, kTcLogits>
+      <<<std::min(rs.tiles, dev->sms), 192, Gemm2Cfg::SMEM_BYTES, st>>>(ax, ax, bw, bw, bw, bw, a);
+  LAUNCH_CHECK("gemm_tc_router", st);
+  if (counts) CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * p.E * 4, st));
+  PROF_BEGIN("topk", st);
+  k_topk<<<(unsigned)cdiv(p.T, 8), 256, 0, st>>>(part, rs.ksplit, p.T * rs.ldp, rs.ldp, bias, p.T, p.E, p.k, ids, tw,
+                                                 counts);
+  LAUNCH_CHECK("topk", st);
+  *counted = counts != nullptr;
   return MOE_OK;
 }
 
-// Count, scan and scatter: offs, row_tok, row_w, pos; optionally the tile prefixes.
-static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, const float* tw, int32_t* offs,
-                                  int32_t* row_tok, float* row_w, int32_t* pos, int32_t* counts, Schedule sa,
-                                  int32_t* pre_a, Schedule sb, int32_t* pre_b, cudaStream_t st, DeviceInfo* dev) {
-  const int64_t n = p.T * p.k;
+// Histogram (unless the router wrote it), scan and scatter: offs, row_tok,
+// row_w, pos, row_dst (may be NULL), the shared rows; optionally the tile prefixes.
+static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, const float* tw, bool counted,
+                                  int32_t* offs, int32_t* row_tok, float* row_w, int32_t* pos, int32_t* row_dst,
+                                  int32_t* counts, Schedule sa, int32_t* pre_a, Schedule sb, int32_t* pre_b,
+                                  cudaStream_t st, DeviceInfo* dev) {
   const int nch = (int)n_chunks(p);
-  if (n > 0) {
-    k_count<<<nch, 256, 0, st>>>(ids, n, p.E, counts, dev->status);
-    LAUNCH_CHECK("count");
-  } else {
+  if (p.T == 0) {
     CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)p.E * 4, st));
+  } else if (!counted) {
+    PROF_BEGIN("count", st);
+    k_count<<<nch, 256, 0, st>>>(ids, p.T, p.k, p.E, counts, dev->status);
+    LAUNCH_CHECK("count", st);
   }
-  k_scan<<<1, 1024, 0, st>>>(counts, nch, p.E, p.T, p.k, p.I_s > 0, offs, sa, pre_a, sb, pre_b);
-  LAUNCH_CHECK("scan");
-  if (n > 0) {
-    k_scatter<<<nch, kScatterWarps * 32, 0, st>>>(ids, tw, n, p.k, p.E, counts, row_tok, row_w, pos);
-    LAUNCH_CHECK("scatter");
-  }
-  if (p.I_s > 0 && p.T > 0) {
-    k_shared_rows<<<(unsigned)cdiv(p.T, 256), 256, 0, st>>>(p.T, offs, p.E, row_tok, row_w);
-    LAUNCH_CHECK("shared_rows");
+  PROF_BEGIN("scan", st);
+  k_scan<<<1, 1024, 0, st>>>(counts, nch, p.E, p.T, p.I_s > 0, offs, sa, pre_a, sb, pre_b);
+  LAUNCH_CHECK("scan", st);
+  if (p.T > 0) {
+    PROF_BEGIN("scatter", st);
+    k_scatter<<<nch, kScatterWarps * 32, 0, st>>>(ids, tw, p.T, p.k, p.E, counts, offs, p.I_s > 0, row_tok, row_w,
+                                                  pos, row_dst);
+    LAUNCH_CHECK("scatter", st);
   }
   return MOE_OK;
 }
@@ -316,8 +398,9 @@ static moe_status launch_gather(const moe_problem& p, const void* x, const int32
   const int64_t rows = rows_total(p);
   if (rows == 0) return MOE_OK;
   unsigned grid = (unsigned)std::min<int64_t>(cdiv(rows, 8), (int64_t)dev->sms * 8);
+  PROF_BEGIN("gather", st);
   k_gather<<<grid, 256, 0, st>>>((const uint4*)x, row_tok, offs, p.E, p.T, vec, (uint4*)xp);
-  LAUNCH_CHECK("gather");
+  LAUNCH_CHECK("gather", st);
   return MOE_OK;
 }
 
@@ -338,10 +421,19 @@ static void scale_parts(const moe_problem& p, const float* sc, const float* part
   for (int i = 0; i < 6; ++i) part[i] = sc ? sc + off[i] : nullptr;
 }
 
+// Output of the down projection: either the weighted rows in (token, slot)
+// order (the fused forward) or the unweighted rows in dispatch order (the
+// expert stage alone).
+struct DownOut {
+  void* ys;               // slot layout [T*(k+1), d], or NULL
+  const int32_t* row_dst;
+  const float* row_w;
+  void* out;              // dispatch layout [R', d], or NULL
+};
+
 template <typename TA, typename TW>
 static moe_status simt_gemms(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
-                             int32_t* pre_a, int32_t* pre_b, void* H, bool combine, float* y32,
-                             const int32_t* row_tok, const float* row_w, void* out, cudaStream_t st,
+                             int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
                              DeviceInfo* dev) {
   const float* sp[6];
   scale_parts(p, w.scales, sp);
@@ -362,8 +454,9 @@ static moe_status simt_gemms(const moe_problem& p, const void* xp, const int32_t
   a.b2 = WeightSet<TW>{(const TW*)w.wu, (const TW*)w.su, sp[1], sp[4]};
   a.H = (TA*)H;
   a.ldh = ldh_of(p);
+  PROF_BEGIN("gemm_simt_swiglu", st);
   k_gemm_simt<TA, TW, kEpiSwiGLU><<<grid, 256, 0, st>>>(a);
-  LAUNCH_CHECK("gemm_simt_swiglu");
+  LAUNCH_CHECK("gemm_simt_swiglu", st);
   // down: A = H [R', ldh], N = d, K = I (I_s)
   SimtGemmArgs<TA, TW> b{};
   b.offs = offs;
@@ -378,26 +471,26 @@ static moe_status simt_gemms(const moe_problem& p, const void* xp, const int32_t
   b.K_s = p.I_s;
   b.b1 = WeightSet<TW>{(const TW*)w.wd, (const TW*)w.sd, sp[2], sp[5]};
   b.b2 = b.b1;
-  if (combine) {
-    b.y32 = y32;
+  if (o.ys) {
+    b.ys = (TA*)o.ys;
     b.ldy = p.d;
-    b.T = p.T;
-    b.row_tok = row_tok;
-    b.row_w = row_w;
-    k_gemm_simt<TA, TW, kEpiCombine><<<grid, 256, 0, st>>>(b);
-    LAUNCH_CHECK("gemm_simt_combine");
+    b.row_dst = o.row_dst;
+    b.row_w = o.row_w;
+    PROF_BEGIN("gemm_simt_slot", st);
+    k_gemm_simt<TA, TW, kEpiSlotStore><<<grid, 256, 0, st>>>(b);
+    LAUNCH_CHECK("gemm_simt_slot", st);
   } else {
-    b.out = (TA*)out;
+    b.out = (TA*)o.out;
     b.ldo = p.d;
+    PROF_BEGIN("gemm_simt_store", st);
     k_gemm_simt<TA, TW, kEpiStore><<<grid, 256, 0, st>>>(b);
-    LAUNCH_CHECK("gemm_simt_store");
+    LAUNCH_CHECK("gemm_simt_store", st);
   }
   return MOE_OK;
 }
 
 static moe_status tc_gemms(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
-                           int32_t* pre_a, int32_t* pre_b, void* H, bool combine, float* y32,
-                           const int32_t* row_tok, const float* row_w, void* out, cudaStream_t st,
+                           int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
                            DeviceInfo* dev) {
   const int64_t Rp = rows_total(p), ldh = ldh_of(p);
   const bool sh = p.I_s > 0;
@@ -418,6 +511,7 @@ static moe_status tc_gemms(const moe_problem& p, const void* xp, const int32_t* 
   a.prefix = pre_a;
   a.E = p.E;
   a.rows_cap = Rp;
+  a.single_rows = -1;
   a.N_r = p.I;
   a.N_s = p.I_s;
   a.K_r = p.d;
@@ -425,8 +519,9 @@ static moe_status tc_gemms(const moe_problem& p, const void* xp, const int32_t* 
   a.H = (bf16*)H;
   a.ldh = ldh;
   a.status = dev->status;
+  PROF_BEGIN("gemm_tc_swiglu", st);
   k_gemm_tc<128, true, 4, kTcSwiGLU><<<dev->sms, 192, Gemm1Cfg::SMEM_BYTES, st>>>(aR, aR, bR, bS, cR, cS, a);
-  LAUNCH_CHECK("gemm_tc_swiglu");
+  LAUNCH_CHECK("gemm_tc_swiglu", st);
   // down
   if ((s = map2d(&aR, H, p.I, Rp, ldh, kBM)) != MOE_OK) return s;
   aS = aR;
@@ -439,38 +534,37 @@ static moe_status tc_gemms(const moe_problem& p, const void* xp, const int32_t* 
   b.prefix = pre_b;
   b.E = p.E;
   b.rows_cap = Rp;
+  b.single_rows = -1;
   b.N_r = p.d;
   b.N_s = p.d;
   b.K_r = p.I;
   b.K_s = p.I_s;
   b.status = dev->status;
-  if (combine) {
-    b.y32 = y32;
+  if (o.ys) {
+    b.ys = (bf16*)o.ys;
     b.ldy = p.d;
-    b.T = p.T;
-    b.row_tok = row_tok;
-    b.row_w = row_w;
-    k_gemm_tc<256, false, 4, kTcCombine><<<dev->sms, 192, Gemm2Cfg::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
-    LAUNCH_CHECK("gemm_tc_combine");
+    b.row_dst = o.row_dst;
+    b.row_w = o.row_w;
+    PROF_BEGIN("gemm_tc_down", st);
+    k_gemm_tc<256, false, 4, kTcSlotStore><<<dev->sms, 192, Gemm2Cfg::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
+    LAUNCH_CHECK("gemm_tc_down", st);
   } else {
-    b.out = (bf16*)out;
+    b.out = (bf16*)o.out;
     b.ldo = p.d;
+    PROF_BEGIN("gemm_tc_store", st);
     k_gemm_tc<256, false, 4, kTcStore><<<dev->sms, 192, Gemm2Cfg::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
-    LAUNCH_CHECK("gemm_tc_store");
+    LAUNCH_CHECK("gemm_tc_store", st);
   }
   return MOE_OK;
 }
 
 static moe_status expert_gemms(const moe_problem& p, bool tc, const void* xp, const int32_t* offs,
-                               const ExpertWeights& w, int32_t* pre_a, int32_t* pre_b, void* H, bool combine,
-                               float* y32, const int32_t* row_tok, const float* row_w, void* out, cudaStream_t st,
-                               DeviceInfo* dev) {
-  if (tc) return tc_gemms(p, xp, offs, w, pre_a, pre_b, H, combine, y32, row_tok, row_w, out, st, dev);
-  if (p.act_dtype == MOE_F32)
-    return simt_gemms<float, float>(p, xp, offs, w, pre_a, pre_b, H, combine, y32, row_tok, row_w, out, st, dev);
-  if (p.w_dtype == MOE_BF16)
-    return simt_gemms<bf16, bf16>(p, xp, offs, w, pre_a, pre_b, H, combine, y32, row_tok, row_w, out, st, dev);
-  return simt_gemms<bf16, uint8_t>(p, xp, offs, w, pre_a, pre_b, H, combine, y32, row_tok, row_w, out, st, dev);
+                               const ExpertWeights& w, int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o,
+                               cudaStream_t st, DeviceInfo* dev) {
+  if (tc) return tc_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
+  if (p.act_dtype == MOE_F32) return simt_gemms<float, float>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
+  if (p.w_dtype == MOE_BF16) return simt_gemms<bf16, bf16>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
+  return simt_gemms<bf16, uint8_t>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
 }
 
 static void schedules(const moe_problem& p, bool tc, Schedule* sa, Schedule* sb) {
@@ -511,6 +605,30 @@ moe_status moe_set_path(int path) {
 }
 
 int moe_last_launch_count(void) { return g_launches; }
+
+moe_status moe_profile_enable(int on) {
+  if (on < 0 || on > 2) return fail(MOE_ERR_INVALID_ARG, "profile mode %d is not 0, 1 or 2", on);
+  g_prof.on = on != 0;
+  g_prof.mode = on;
+  g_prof.used = 0;
+  return MOE_OK;
+}
+
+int moe_profile_read(int max, float* ms, const char** names) {
+  Profiler& P = g_prof;
+  int n = std::min(max, P.used);
+  for (int i = 0; i < n; ++i) {
+    float t = -1.f;
+    if (cudaEventSynchronize(P.ev[i].end) != cudaSuccess ||
+        cudaEventElapsedTime(&t, P.ev[i].begin, P.ev[i].end) != cudaSuccess)
+      t = -1.f;
+    if (ms) ms[i] = t;
+    if (names) names[i] = P.ev[i].name;
+  }
+  P.used = 0;
+  return n;
+}
+
 const char* moe_last_error_string(void) { return g_err; }
 
 moe_status moe_device_status(int32_t* detail) {
@@ -528,20 +646,31 @@ moe_status moe_device_status(int32_t* detail) {
 }
 
 moe_status moe_router_topk(const moe_problem* p, const void* x, const void* w_router, const float* router_bias,
-                           int32_t* topk_ids, float* topk_w, void* stream) {
+                           int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes, void* stream) {
   moe_status s = check(p);
   if (s != MOE_OK) return s;
-  if (p->T > 0) {
-    NEED(x);
-    NEED(w_router);
-    MAYBE(router_bias);
-    NEED(topk_ids);
-    NEED(topk_w);
+  if (p->T == 0) {
+    g_launches = 0;
+    return MOE_OK;
+  }
+  NEED(x);
+  NEED(w_router);
+  MAYBE(router_bias);
+  NEED(topk_ids);
+  NEED(topk_w);
+  const Layout L = layout(*p, false);
+  if (p->act_dtype == MOE_BF16) {
+    NEED(ws);
+    if (ws_bytes < L.total)
+      return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
   }
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != MOE_OK) return s;
   g_launches_pending = 0;
-  s = launch_router(*p, x, w_router, router_bias, topk_ids, topk_w, (cudaStream_t)stream, dev);
+  bool counted;
+  float* part = ws ? (float*)((char*)ws + L.part) : nullptr;
+  s = launch_router(*p, x, w_router, router_bias, topk_ids, topk_w, part, nullptr, &counted, (cudaStream_t)stream,
+                    dev);
   if (s == MOE_OK) g_launches = g_launches_pending;
   return s;
 }
@@ -570,8 +699,8 @@ moe_status moe_permute(const moe_problem* p, const void* x, const int32_t* topk_
   g_launches_pending = 0;
   cudaStream_t st = (cudaStream_t)stream;
   char* w = (char*)ws;
-  s = launch_dispatch(*p, topk_ids, topk_w, offs, row_tok, row_w, pos, (int32_t*)(w + L.counts), Schedule{},
-                      nullptr, Schedule{}, nullptr, st, dev);
+  s = launch_dispatch(*p, topk_ids, topk_w, false, offs, row_tok, row_w, pos, nullptr, (int32_t*)(w + L.counts),
+                      Schedule{}, nullptr, Schedule{}, nullptr, st, dev);
   if (s != MOE_OK) return s;
   s = launch_gather(*p, x, row_tok, offs, x_perm, st, dev);
   if (s == MOE_OK) g_launches = g_launches_pending;
@@ -584,7 +713,10 @@ moe_status moe_expert_ffn(const moe_problem* p, const void* x_perm, const int32_
                           void* stream) {
   moe_status s = check(p);
   if (s != MOE_OK) return s;
-  if (p->T == 0) return MOE_OK;
+  if (p->T == 0) {
+    g_launches = 0;
+    return MOE_OK;
+  }
   NEED(x_perm);
   NEED(offs);
   NEED(y_perm);
@@ -605,10 +737,11 @@ moe_status moe_expert_ffn(const moe_problem* p, const void* x_perm, const int32_
   schedules(*p, tc, &sa, &sb);
   int32_t* pre_a = (int32_t*)(wsp + L.pre_a);
   int32_t* pre_b = (int32_t*)(wsp + L.pre_b);
+  PROF_BEGIN("tile_prefix", st);
   k_tile_prefix<<<1, 1024, 0, st>>>(offs, p->E, sa, pre_a, sb, pre_b);
-  LAUNCH_CHECK("tile_prefix");
-  s = expert_gemms(*p, tc, x_perm, offs, w, pre_a, pre_b, wsp + L.h, false, nullptr, nullptr, nullptr, y_perm, st,
-                   dev);
+  LAUNCH_CHECK("tile_prefix", st);
+  DownOut o{nullptr, nullptr, nullptr, y_perm};
+  s = expert_gemms(*p, tc, x_perm, offs, w, pre_a, pre_b, wsp + L.h, o, st, dev);
   if (s == MOE_OK) g_launches = g_launches_pending;
   return s;
 }
@@ -617,7 +750,10 @@ moe_status moe_combine(const moe_problem* p, const void* y_perm, const int32_t* 
                        const int32_t* offs, void* y, void* stream) {
   moe_status s = check(p);
   if (s != MOE_OK) return s;
-  if (p->T == 0) return MOE_OK;
+  if (p->T == 0) {
+    g_launches = 0;
+    return MOE_OK;
+  }
   NEED(y_perm);
   NEED(pos);
   NEED(topk_w);
@@ -627,13 +763,14 @@ moe_status moe_combine(const moe_problem* p, const void* y_perm, const int32_t* 
   if ((s = device_info(&dev)) != MOE_OK) return s;
   g_launches_pending = 0;
   cudaStream_t st = (cudaStream_t)stream;
+  PROF_BEGIN("combine", st);
   if (p->act_dtype == MOE_F32)
     k_combine<float><<<(unsigned)p->T, 256, 0, st>>>((const float*)y_perm, pos, topk_w, offs, p->E, p->k, p->d, p->T,
                                                      (float*)y);
   else
     k_combine<bf16><<<(unsigned)p->T, 256, 0, st>>>((const bf16*)y_perm, pos, topk_w, offs, p->E, p->k, p->d, p->T,
                                                     (bf16*)y);
-  LAUNCH_CHECK("combine");
+  LAUNCH_CHECK("combine", st);
   g_launches = g_launches_pending;
   return MOE_OK;
 }
@@ -669,30 +806,32 @@ moe_status moe_layer_forward(const moe_problem* p, const void* x, const void* w_
   char* wsp = (char*)ws;
   int32_t* ids = topk_ids_out ? topk_ids_out : (int32_t*)(wsp + L.ids);
   float* tw = topk_w_out ? topk_w_out : (float*)(wsp + L.tw);
+  int32_t* counts = (int32_t*)(wsp + L.counts);
   int32_t* offs = (int32_t*)(wsp + L.offs);
   int32_t* row_tok = (int32_t*)(wsp + L.row_tok);
   float* row_w = (float*)(wsp + L.row_w);
   int32_t* pos = (int32_t*)(wsp + L.pos);
+  int32_t* row_dst = (int32_t*)(wsp + L.row_dst);
   int32_t* pre_a = (int32_t*)(wsp + L.pre_a);
   int32_t* pre_b = (int32_t*)(wsp + L.pre_b);
-  float* y32 = p->act_dtype == MOE_BF16 ? (float*)(wsp + L.y32) : (float*)y;
-  CUDA_TRY(cudaMemsetAsync(y32, 0, (size_t)p->T * p->d * 4, st));
-  if ((s = launch_router(*p, x, w_router, router_bias, ids, tw, st, dev)) != MOE_OK) return s;
+  void* xp = wsp + L.xp;
+  bool counted;
+  s = launch_router(*p, x, w_router, router_bias, ids, tw, (float*)(wsp + L.part), counts, &counted, st, dev);
+  if (s != MOE_OK) return s;
   Schedule sa, sb;
   schedules(*p, tc, &sa, &sb);
-  s = launch_dispatch(*p, ids, tw, offs, row_tok, row_w, pos, (int32_t*)(wsp + L.counts), sa, pre_a, sb, pre_b, st,
-                      dev);
+  s = launch_dispatch(*p, ids, tw, counted, offs, row_tok, row_w, pos, row_dst, counts, sa, pre_a, sb, pre_b, st, dev);
   if (s != MOE_OK) return s;
-  if ((s = launch_gather(*p, x, row_tok, offs, wsp + L.xp, st, dev)) != MOE_OK) return s;
-  s = expert_gemms(*p, tc, wsp + L.xp, offs, w, pre_a, pre_b, wsp + L.h, true, y32, row_tok, row_w, nullptr, st,
-                   dev);
+  if ((s = launch_gather(*p, x, row_tok, offs, xp, st, dev)) != MOE_OK) return s;
+  DownOut o{xp, row_dst, row_w, nullptr};  // the slot rows reuse the dispatched-row buffer
+  s = expert_gemms(*p, tc, xp, offs, w, pre_a, pre_b, wsp + L.h, o, st, dev);
   if (s != MOE_OK) return s;
-  if (p->act_dtype == MOE_BF16) {
-    const int64_t n8 = p->T * p->d / 8;
-    unsigned grid = (unsigned)std::min<int64_t>(cdiv(n8, 256), (int64_t)dev->sms * 16);
-    k_finalize_bf16<<<grid, 256, 0, st>>>((const float4*)y32, (uint4*)y, n8);
-    LAUNCH_CHECK("finalize");
-  }
+  PROF_BEGIN("slot_sum", st);
+  if (p->act_dtype == MOE_F32)
+    k_slot_sum<float><<<(unsigned)p->T, 256, 0, st>>>((const float*)xp, pos, p->k, p->I_s > 0, p->d, (float*)y);
+  else
+    k_slot_sum<bf16><<<(unsigned)p->T, 256, 0, st>>>((const bf16*)xp, pos, p->k, p->I_s > 0, p->d, (bf16*)y);
+  LAUNCH_CHECK("slot_sum", st);
   g_launches = g_launches_pending;
   return MOE_OK;
 }

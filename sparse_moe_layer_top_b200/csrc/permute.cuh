@@ -1,32 +1,35 @@
 // permute.cuh -- dispatch of (token, slot) pairs to expert-contiguous rows.
 //
 // The token "is sent to" its k experts (Qwen3.6 explainer, router paragraph).
-// Here that is a stable counting sort by expert in three passes over the
-// flattened T*k routing ids, cut into chunks of kChunk pairs:
-//   k_count    per-chunk histogram over the E experts;
+// Here that is a stable counting sort by expert over chunks of kChunkTokens
+// tokens (chunk c = the pairs of tokens c*kChunkTokens ...):
+//   counts     per-chunk histogram over the E experts (written by k_topk, or
+//              by k_count when the routing comes from elsewhere);
 //   k_scan     per-expert exclusive scan over chunks, then over experts ->
-//              group offsets offs[E+2] and each chunk's base row per expert;
+//              group offsets offs[E+2] and each chunk's first row per expert;
 //              also the tile prefix sums of the GEMM schedules;
-//   k_scatter  within a chunk, warps take consecutive sub-ranges; ranks come
-//              from warp match masks, so row order = (token, slot) order;
+//   k_scatter  within a chunk, warps take consecutive token ranges; ranks come
+//              from warp match masks, so row order = (token, slot) order; the
+//              chunk's shared-expert rows are written too;
 //   k_gather   copies x rows into the dispatched buffer (16-byte vectors).
-// Group E (the shared expert) is every token in order at rows T*k .. T*k+T-1.
+// Group E (the shared expert) is every token in order at rows offs[E] + t.
 #pragma once
 #include "common.cuh"
+#include "router.cuh"
 
 namespace moe {
 
-constexpr int kChunk = 2048;       // pairs per chunk
 constexpr int kScatterWarps = 8;   // warps of k_scatter (256 threads)
 constexpr int kMaxE = 512;
 
-__global__ void __launch_bounds__(256) k_count(const int32_t* __restrict__ ids, int64_t n, int E,
+__global__ void __launch_bounds__(256) k_count(const int32_t* __restrict__ ids, int64_t T, int k, int E,
                                                int32_t* __restrict__ counts, unsigned* status) {
   __shared__ int32_t h[kMaxE];
   for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
   __syncthreads();
-  int64_t c0 = (int64_t)blockIdx.x * kChunk;
-  int64_t c1 = c0 + kChunk < n ? c0 + kChunk : n;
+  const int64_t n = T * k;
+  const int64_t c0 = (int64_t)blockIdx.x * kChunkTokens * k;
+  const int64_t c1 = min(n, c0 + (int64_t)kChunkTokens * k);
   for (int64_t i = c0 + threadIdx.x; i < c1; i += blockDim.x) {
     int e = __ldg(ids + i);
     if ((unsigned)e < (unsigned)E) atomicAdd(&h[e], 1);
@@ -61,7 +64,7 @@ __device__ __forceinline__ int block_incl_scan(int v, int* sm_warp) {
   return v;
 }
 
-// Tile prefix of one schedule from the group offsets (E+1 groups, one thread each).
+// Tile prefix of one schedule from the group sizes (E+1 groups, one thread each).
 __device__ __forceinline__ void write_tile_prefix(const Schedule& s, int E, int rows_g, int32_t* prefix,
                                                   int* sm_warp) {
   int g = threadIdx.x;
@@ -73,15 +76,17 @@ __device__ __forceinline__ void write_tile_prefix(const Schedule& s, int E, int 
 
 // One block of 1024 threads.  counts[c*E+e] (chunk histograms) becomes the
 // absolute first row of expert e's pairs in chunk c.
-__global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ counts, int nchunks, int E, int64_t T, int k,
+__global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ counts, int nchunks, int E, int64_t T,
                                                int has_shared, int32_t* __restrict__ offs, Schedule sa,
                                                int32_t* __restrict__ prefix_a, Schedule sb,
                                                int32_t* __restrict__ prefix_b) {
   __shared__ int sm_warp[32];
   int e = threadIdx.x;
   int total = 0;
-  if (e < E)
+  if (e < E) {
+#pragma unroll 8
     for (int c = 0; c < nchunks; ++c) total += counts[(int64_t)c * E + e];
+  }
   int incl = block_incl_scan(e < E ? total : 0, sm_warp);
   int start = incl - (e < E ? total : 0);
   if (e < E) {
@@ -114,21 +119,25 @@ __global__ void __launch_bounds__(1024) k_tile_prefix(const int32_t* __restrict_
   if (prefix_b) write_tile_prefix(sb, E, rows, prefix_b, sm_warp);
 }
 
-__global__ void __launch_bounds__(kScatterWarps * 32) k_scatter(const int32_t* __restrict__ ids,
-                                                                const float* __restrict__ topk_w, int64_t n, int k,
-                                                                int E, const int32_t* __restrict__ base,
-                                                                int32_t* __restrict__ row_tok,
-                                                                float* __restrict__ row_w,
-                                                                int32_t* __restrict__ pos) {
+// One block per chunk.  Writes, for every routed pair (t, j) with a valid id:
+// row r, row_tok[r] = t, row_w[r] = topk_w[t,j], pos[t*k+j] = r and (if
+// row_dst is given) row_dst[r] = t*(k+1) + j; invalid pairs get pos = -1.
+// With has_shared, also the chunk's shared-expert rows offs[E] + t.
+__global__ void __launch_bounds__(kScatterWarps * 32) k_scatter(
+    const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int64_t T, int k, int E,
+    const int32_t* __restrict__ base, const int32_t* __restrict__ offs, int has_shared,
+    int32_t* __restrict__ row_tok, float* __restrict__ row_w, int32_t* __restrict__ pos,
+    int32_t* __restrict__ row_dst) {
   __shared__ int32_t wb[kScatterWarps][kMaxE];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int sub = kChunk / kScatterWarps;
-  const int64_t c0 = (int64_t)blockIdx.x * kChunk;
-  const int64_t s0 = c0 + (int64_t)warp * sub;
+  constexpr int kTokPerWarp = kChunkTokens / kScatterWarps;
+  const int64_t n = T * k;
+  const int64_t s0 = ((int64_t)blockIdx.x * kChunkTokens + (int64_t)warp * kTokPerWarp) * k;
+  const int64_t s1 = min(n, s0 + (int64_t)kTokPerWarp * k);
   for (int e = lane; e < E; e += 32) wb[warp][e] = 0;
   __syncwarp();
-  // pass 1: per-warp histogram of its sub-range
-  for (int64_t i = s0 + lane; i < s0 + sub && i < n; i += 32) {
+  // pass 1: per-warp histogram of its pairs
+  for (int64_t i = s0 + lane; i < s1; i += 32) {
     int e = __ldg(ids + i);
     if ((unsigned)e < (unsigned)E) atomicAdd(&wb[warp][e], 1);
   }
@@ -145,35 +154,35 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_scatter(const int32_t* _
   __syncthreads();
   // pass 2: in order, 32 pairs at a time; equal experts rank by lane order
   const unsigned lt = (1u << lane) - 1u;
-  for (int64_t b = s0; b < s0 + sub && b < n; b += 32) {
-    int64_t i = b + lane;
-    bool act = i < n && i < s0 + sub;
-    int e = act ? __ldg(ids + i) : -1;
-    bool ok = act && (unsigned)e < (unsigned)E;
-    unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+  for (int64_t b = s0; b < s1; b += 32) {
+    const int64_t i = b + lane;
+    const bool act = i < s1;
+    const int e = act ? __ldg(ids + i) : -1;
+    const bool ok = act && (unsigned)e < (unsigned)E;
+    const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
     int r = 0;
     if (ok) r = wb[warp][e] + __popc(peers & lt);
     __syncwarp();
     if (ok && (peers & lt) == 0) wb[warp][e] += __popc(peers);  // lowest peer advances the cursor
     __syncwarp();
     if (ok) {
-      row_tok[r] = (int32_t)(i / k);
+      const int64_t t = i / k;
+      row_tok[r] = (int32_t)t;
       row_w[r] = __ldg(topk_w + i);
       pos[i] = r;
+      if (row_dst) row_dst[r] = (int32_t)(t * (k + 1) + (i - t * k));
     } else if (act) {
       pos[i] = -1;
     }
   }
-}
-
-// Shared-expert rows: row offs[E] + t is token t with weight 1.
-__global__ void k_shared_rows(int64_t T, const int32_t* __restrict__ offs, int E, int32_t* __restrict__ row_tok,
-                              float* __restrict__ row_w) {
-  int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  int64_t R = offs[E];
-  if (t < T) {
-    row_tok[R + t] = (int32_t)t;
-    row_w[R + t] = 1.0f;
+  if (has_shared) {
+    const int64_t R = __ldg(offs + E);
+    for (int64_t t = (int64_t)blockIdx.x * kChunkTokens + threadIdx.x;
+         t < min(T, (int64_t)(blockIdx.x + 1) * kChunkTokens); t += blockDim.x) {
+      row_tok[R + t] = (int32_t)t;
+      row_w[R + t] = 1.0f;
+      if (row_dst) row_dst[R + t] = (int32_t)(t * (k + 1) + k);
+    }
   }
 }
 

@@ -7,77 +7,12 @@
 
 namespace moe {
 
-// ---------------------------------------------------------------- router
-// One warp per token.  Lane l owns experts l, l+32, ... (E <= 512 -> <= 16).
-// Logit = x . W_r[e] (+ bias[e]); the k largest logits are taken by repeated
-// warp arg-max (equal values -> lower expert index); the weights are the
-// softmax over the kept logits, which equals the full softmax renormalised
-// over the kept experts.
-template <typename TA>
-__global__ void __launch_bounds__(256) k_router_simt(const TA* __restrict__ x, const TA* __restrict__ wr,
-                                                     const float* __restrict__ bias, int64_t T, int d, int E, int k,
-                                                     int32_t* __restrict__ ids, float* __restrict__ tw) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t t = (int64_t)blockIdx.x * 8 + warp;
-  if (t >= T) return;
-  const TA* xt = x + t * d;
-  float l[16];
-#pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    int e = lane + 32 * i;
-    float acc = -INFINITY;
-    if (e < E) {
-      const TA* w = wr + (int64_t)e * d;
-      acc = 0.f;
-      for (int j = 0; j < d; ++j) acc = fmaf(to_f32(xt[j]), to_f32(w[j]), acc);
-      if (bias) acc += bias[e];
-    }
-    l[i] = acc;
-  }
-  unsigned taken = 0;
-  float v0 = 0.f, den = 0.f;
-  float sel_v[16];
-  int sel_e[16];
-  for (int s = 0; s < k; ++s) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      int e = lane + 32 * i;
-      if (e < E && !(taken >> i & 1u) && (l[i] > bv || be == 0x7fffffff)) {
-        bv = l[i];
-        be = e;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      int oe = __shfl_xor_sync(0xffffffffu, be, o);
-      if (ov > bv || (ov == bv && oe < be)) {
-        bv = ov;
-        be = oe;
-      }
-    }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
-    if (s == 0) v0 = bv;
-    sel_v[s & 15] = bv;
-    sel_e[s & 15] = be;
-    den += __expf(bv - v0);
-  }
-  if (lane == 0) {
-    for (int s = 0; s < k; ++s) {
-      ids[t * k + s] = sel_e[s];
-      tw[t * k + s] = __expf(sel_v[s] - v0) / den;
-    }
-  }
-}
-
 // ---------------------------------------------------------------- grouped GEMM
 // C[r, n] = sum_c A[r, c] * B_g[n, c] over the rows r of group g (rows
 // offs[g] .. offs[g+1]-1 of A) and n < N_g, for every group g (g == E: the
 // shared expert).  64 x 64 tiles, 16-deep K steps, 256 threads x (4 x 4)
 // outputs; a persistent grid walks the device-built tile prefix.
-enum { kEpiSwiGLU = 0, kEpiCombine = 1, kEpiStore = 2 };
+enum { kEpiSwiGLU = 0, kEpiSlotStore = 1, kEpiStore = 2 };
 
 template <typename TW>
 struct WeightSet {
@@ -99,9 +34,9 @@ struct SimtGemmArgs {
   WeightSet<TW> b1, b2;   // b2: the up projection of the SwiGLU epilogue
   TA* H;                  // kEpiSwiGLU: [rows, ldh]
   int64_t ldh;
-  float* y32;             // kEpiCombine: [T, ldy] fp32, accumulated
-  int64_t ldy, T;
-  const int32_t* row_tok;
+  TA* ys;                 // kEpiSlotStore: [T*(k+1), ldy], row_w-weighted, (token, slot) order
+  int64_t ldy;
+  const int32_t* row_dst;
   const float* row_w;
   TA* out;                // kEpiStore: [rows, ldo]
   int64_t ldo;
@@ -186,9 +121,9 @@ __global__ void __launch_bounds__(256) k_gemm_simt(SimtGemmArgs<TA, TW> p) {
         if (n >= N) continue;
         if (EPI == kEpiSwiGLU) {
           from_f32(silu_f32(acc[i][j]) * acc2[i][j], p.H + r * p.ldh + n);
-        } else if (EPI == kEpiCombine) {
-          int tok = __ldg(p.row_tok + r);
-          if ((uint64_t)tok < (uint64_t)p.T) atomicAdd(p.y32 + (int64_t)tok * p.ldy + n, __ldg(p.row_w + r) * acc[i][j]);
+        } else if (EPI == kEpiSlotStore) {
+          int64_t dr = __ldg(p.row_dst + r);
+          if (dr >= 0) from_f32(__ldg(p.row_w + r) * acc[i][j], p.ys + dr * p.ldy + n);
         } else {
           from_f32(acc[i][j], p.out + r * p.ldo + n);
         }
@@ -218,16 +153,45 @@ __global__ void __launch_bounds__(256) k_combine(const TA* __restrict__ yp, cons
   }
 }
 
-// y (bf16) = y32 (fp32), 8 elements per thread.
-__global__ void k_finalize_bf16(const float4* __restrict__ y32, uint4* __restrict__ y, int64_t n8) {
-  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
-    float4 a = y32[2 * i], b = y32[2 * i + 1];
-    uint4 o;
-    o.x = pack_bf16x2(a.x, a.y);
-    o.y = pack_bf16x2(a.z, a.w);
-    o.z = pack_bf16x2(b.x, b.y);
-    o.w = pack_bf16x2(b.z, b.w);
-    y[i] = o;
+// y[t] = sum over the token's k+1 slots of ys[t*(k+1) + j] (routed slots with
+// a dropped pair are skipped; slot k is the shared expert).  The slots already
+// carry their routing weights; the sum runs in fp32 in slot order, so the
+// result does not depend on scheduling.  One block per token, 8 elements per
+// thread and step.
+template <typename TA>
+__global__ void __launch_bounds__(256) k_slot_sum(const TA* __restrict__ ys, const int32_t* __restrict__ pos, int k,
+                                                  int has_shared, int d, TA* __restrict__ y) {
+  const int64_t t = blockIdx.x;
+  const TA* src = ys + t * (int64_t)(k + 1) * d;
+  unsigned ok = 0;
+  for (int j = 0; j < k; ++j) ok |= (__ldg(pos + t * k + j) >= 0 ? 1u : 0u) << j;
+  if (has_shared) ok |= 1u << k;
+  for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j <= k; ++j) {
+      if (!(ok >> j & 1u)) continue;
+      const TA* row = src + (int64_t)j * d + c;
+      if (sizeof(TA) == 2) {
+        uint4 v = *reinterpret_cast<const uint4*>(row);
+        const bf16* h = reinterpret_cast<const bf16*>(&v);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += to_f32(h[e]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += to_f32(row[e]);
+      }
+    }
+    if (sizeof(TA) == 2) {
+      uint4 o;
+      o.x = pack_bf16x2(acc[0], acc[1]);
+      o.y = pack_bf16x2(acc[2], acc[3]);
+      o.z = pack_bf16x2(acc[4], acc[5]);
+      o.w = pack_bf16x2(acc[6], acc[7]);
+      *reinterpret_cast<uint4*>(y + t * d + c) = o;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) from_f32(acc[e], y + t * d + c + e);
+    }
   }
 }
 

@@ -1,13 +1,15 @@
-// tc_gemm.cuh -- tensor-core (tcgen05) kernels for sm_100a: the grouped expert
-// GEMMs and the router GEMM with its fused top-k.
+// tc_gemm.cuh -- tensor-core (tcgen05) GEMM kernel for sm_100a, shared by the
+// router and the two expert projections.
 //
 // Grouped GEMM (row-tiled form).  For every group g (expert g, or g == E the
 // shared expert) with rows r0 .. r0+rows-1 of the activation matrix A:
 //     D[r, n] = sum_c A[r, c] * B_g[n, c],  n < N_g,  c < K_g,
 // with B_g K-major (the weights' own out x in layout).  One persistent CTA per
-// SM walks a device-built tile list (group, 128-row block, BN-column block);
-// tiles of one column block of a group are adjacent, so the CTAs that share a
-// weight tile run together and the second read comes from L2.
+// SM walks a tile list (group, 128-row block, BN-column block, K split); the
+// list comes from a device-built prefix sum over groups, or -- in the
+// single-group mode the router uses -- from the kernel's arguments.  Tiles of
+// one column block of a group are adjacent, so the CTAs that share a weight
+// tile run together and the second read of it comes from L2.
 //
 // Warp roles (6 warps):
 //   warp 0      TMA producer: A tile 128 x 64 and B tile(s) BN x 64 per stage,
@@ -16,9 +18,11 @@
 //               fp32 accumulators in TMEM, double-buffered across tiles;
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (warp w reads TMEM
 //               lanes 32*(w%4) ..), then one of
-//                 SwiGLU   H[r, n] = SiLU(gate) * up  -> bf16   (DUAL: two B)
-//                 Combine  y32[tok(r), n] += w(r) * D  (fp32 vector reductions)
-//                 Store    out[r, n] = D -> bf16.
+//                 SwiGLU    H[r, n] = SiLU(gate) * up -> bf16      (DUAL: two B)
+//                 SlotStore Y[dst(r), n] = w(r) * D -> bf16: the routing weight
+//                           applied and the row put back in (token, slot) order
+//                 Store     out[r, n] = D -> bf16
+//                 Logits    part[split][r, n] = D (+ nothing) -> fp32
 // Rows of a tile past the end of its group are computed and discarded; rows
 // never mix in a GEMM, so those rows cannot disturb the kept ones.
 #pragma once
@@ -30,45 +34,77 @@ namespace moe {
 constexpr int kBM = 128;
 constexpr int kBK = 64;  // 64 bf16 = one 128-byte swizzle row
 
-enum { kTcSwiGLU = 0, kTcCombine = 1, kTcStore = 2 };
+enum { kTcSwiGLU = 0, kTcSlotStore = 1, kTcStore = 2, kTcLogits = 3 };
 
 struct TcGemmArgs {
-  const int32_t* offs;    // [E+2] group row starts
-  const int32_t* prefix;  // [E+2] tile prefix of this schedule
+  const int32_t* offs;    // [E+2] group row starts (grouped mode)
+  const int32_t* prefix;  // [E+2] tile prefix of this schedule (grouped mode)
   int E;
   int N_r, N_s, K_r, K_s;
   int64_t rows_cap;       // rows of the activation/output buffers; no row at or past it is written
+  // single-group mode (single_rows >= 0): one group of single_rows rows that
+  // uses the "shared" maps, split along K into ksplit parts
+  int single_rows, single_tiles, ksplit, kb_per_split;
   bf16* H;                // SwiGLU output [rows, ldh]
   int64_t ldh;
-  float* y32;             // Combine output [T, ldy]
-  int64_t ldy, T;
-  const int32_t* row_tok;
-  const float* row_w;
+  bf16* ys;               // SlotStore output [T*(k+1), ldy]
+  int64_t ldy;
+  const int32_t* row_dst; // SlotStore: destination row of each dispatched row
+  const float* row_w;     // SlotStore: routing weight of each dispatched row
   bf16* out;              // Store output [rows, ldo]
   int64_t ldo;
+  float* part;            // Logits output [ksplit][rows, ldp]
+  int64_t ldp, part_stride;
   unsigned* status;
 };
 
 struct TileInfo {
-  int g, rows, m0, n0, kblocks, N;
+  int g, rows, m0, n0, kb0, kb1, N, split;
   int64_t row0;
 };
 
+// s_pre / s_offs: the schedule's tile prefix and group offsets, cached in
+// shared memory at kernel start (grouped mode).
 template <int BN>
-__device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, int tile) {
+__device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, const int32_t* s_pre, const int32_t* s_offs,
+                                                int tile) {
   TileInfo t;
-  t.g = find_group(p.prefix, p.E + 1, tile);
-  const int r0 = __ldg(p.offs + t.g);
-  t.rows = __ldg(p.offs + t.g + 1) - r0;
+  if (p.single_rows >= 0) {
+    t.g = p.E;
+    t.rows = p.single_rows;
+    const int mtc = (t.rows + kBM - 1) / kBM, ntc = (p.N_s + BN - 1) / BN;
+    t.split = tile / (mtc * ntc);
+    const int local = tile - t.split * mtc * ntc;
+    t.m0 = (local % mtc) * kBM;
+    t.n0 = (local / mtc) * BN;
+    t.row0 = t.m0;
+    t.N = p.N_s;
+    const int kbt = (p.K_s + kBK - 1) / kBK;
+    t.kb0 = t.split * p.kb_per_split;
+    t.kb1 = min(kbt, t.kb0 + p.kb_per_split);
+    return t;
+  }
+  {
+    int lo = 0, hi = p.E + 1;  // s_pre[lo] <= tile < s_pre[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_pre[mid] <= tile) lo = mid; else hi = mid;
+    }
+    t.g = lo;
+  }
+  const int r0 = s_offs[t.g];
+  t.rows = s_offs[t.g + 1] - r0;
   const int mtc = (t.rows + kBM - 1) / kBM;
-  const int local = tile - __ldg(p.prefix + t.g);
+  const int local = tile - s_pre[t.g];
   const int mb = local % mtc, nb = local / mtc;
   t.m0 = mb * kBM;
   t.row0 = (int64_t)r0 + t.m0;
   t.n0 = nb * BN;
   const bool sh = t.g == p.E;
   t.N = sh ? p.N_s : p.N_r;
-  t.kblocks = ((sh ? p.K_s : p.K_r) + kBK - 1) / kBK;
+  t.kb0 = 0;
+  t.kb1 = ((sh ? p.K_s : p.K_r) + kBK - 1) / kBK;
+  t.split = 0;
   return t;
 }
 
@@ -91,7 +127,8 @@ struct TcGemmCfg {
   static constexpr int ACC_COLS = DUAL ? 2 * BN : BN;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
   static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8 + 16;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int SCHED_INTS = 2 * (512 + 2);  // tile prefix + group offsets, E <= 512
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + SCHED_INTS * 4;
   static_assert(TMEM_COLS == 64 || TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -112,9 +149,16 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* s_pre = reinterpret_cast<int32_t*>(smem + STAGES * Cfg::STAGE_BYTES + Cfg::BAR_BYTES);
+  int32_t* s_offs = s_pre + 514;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned tcode = kStatusTimeoutBase | (kKernGemmTc << 8);
+  if (p.single_rows < 0)
+    for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) {
+      s_pre[i] = __ldg(p.prefix + i);
+      s_offs[i] = __ldg(p.offs + i);
+    }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -147,7 +191,7 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = __ldg(p.prefix + p.E + 1);
+  const int total = p.single_rows >= 0 ? p.single_tiles : s_pre[p.E + 1];
 
   if (warp == 0) {
     if (lane == 0) {
@@ -157,10 +201,10 @@ __global__ void __launch_bounds__(192, 1)
       int stage = 0;
       uint32_t phase = 0, issued = 0, last_par = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-        const TileInfo t = decode_tile<BN>(p, tile);
+        const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
         const bool sh = t.g == p.E;
         bool ok = true;
-        for (int kb = 0; kb < t.kblocks; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 1)) {
             ok = false;
             break;
@@ -198,11 +242,11 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const TileInfo t = decode_tile<BN>(p, tile);
+        const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
         if (!mbar_wait(tempty + acc, acc_phase ^ 1, abort_flag, p.status, tcode | 2)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + acc * Cfg::ACC_COLS;
-        for (int kb = 0; kb < t.kblocks; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(full + stage, phase, abort_flag, p.status, tcode | 3)) {
             ok = false;
             break;
@@ -213,7 +257,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t ad = sdesc_sw128(sa + kk * 32);
-            const uint32_t accum = (kb | kk) != 0;
+            const uint32_t accum = (kb != t.kb0 || kk != 0);
             umma_f16(d0, ad, sdesc_sw128(sb + kk * 32), idesc, accum);
             if (DUAL) umma_f16(d0 + BN, ad, sdesc_sw128(sb + Cfg::B_BYTES + kk * 32), idesc, accum);
           }
@@ -242,7 +286,7 @@ __global__ void __launch_bounds__(192, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const TileInfo t = decode_tile<BN>(p, tile);
+      const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
       if (!mbar_wait(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + acc * Cfg::ACC_COLS + ((uint32_t)(q * 32) << 16);
@@ -275,28 +319,49 @@ __global__ void __launch_bounds__(192, 1)
             }
           }
         }
-      } else if (EPI == kTcCombine) {
-        int tok = 0;
+      } else if (EPI == kTcSlotStore) {
+        int64_t dr = 0;
         float w = 0.f;
         if (valid) {
-          tok = __ldg(p.row_tok + grow);
+          dr = __ldg(p.row_dst + grow);
           w = __ldg(p.row_w + grow);
         }
-        const bool ok = valid && (uint64_t)tok < (uint64_t)p.T;
-        float* dst = p.y32 + (int64_t)tok * p.ldy;
+        bf16* dst = p.ys + dr * p.ldy;
 #pragma unroll 1
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t a[32];
           tmem_ld32(tb + c * 32, a);
           tmem_wait_regs(a);
-          if (ok) {
+          if (valid && dr >= 0) {
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              const int n = t.n0 + c * 32 + v * 8;
+              if (n < t.N) {
+                uint4 o;
+                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  ow[e] = pack_bf16x2(w * __uint_as_float(a[v * 8 + 2 * e]), w * __uint_as_float(a[v * 8 + 2 * e + 1]));
+                *reinterpret_cast<uint4*>(dst + n) = o;
+              }
+            }
+          }
+        }
+      } else if (EPI == kTcLogits) {
+        float* dst = p.part + (int64_t)t.split * p.part_stride + grow * p.ldp;
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t a[32];
+          tmem_ld32(tb + c * 32, a);
+          tmem_wait_regs(a);
+          if (valid) {
 #pragma unroll
             for (int v = 0; v < 8; ++v) {
               const int n = t.n0 + c * 32 + v * 4;
               if (n < t.N)
-                atomicAdd(reinterpret_cast<float4*>(dst + n),
-                          make_float4(w * __uint_as_float(a[4 * v]), w * __uint_as_float(a[4 * v + 1]),
-                                      w * __uint_as_float(a[4 * v + 2]), w * __uint_as_float(a[4 * v + 3])));
+                *reinterpret_cast<float4*>(dst + n) =
+                    make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
+                                __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
             }
           }
         }
@@ -339,195 +404,6 @@ __global__ void __launch_bounds__(192, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
-  }
-}
-
-// ---------------------------------------------------------------- router
-// One CTA per 128 tokens: logits[128, E] = x_blk . W_r^T accumulate in TMEM
-// (E padded to a multiple of 16; up to two MMAs of N <= 256 side by side),
-// then each epilogue thread scans its token's row of logits in TMEM, keeps
-// the k largest (equal values -> lower expert index) in registers, and
-// writes the ids and the softmax over the kept logits (= the full softmax
-// renormalised over the kept experts).
-constexpr int kMaxK = 16;
-
-struct TcRouterArgs {
-  int64_t T;
-  int E, E_pad, k, kblocks, stages;
-  int n1, n2;          // MMA widths of the two halves (n2 == 0: one)
-  int tmem_cols;
-  const float* bias;
-  int32_t* ids;
-  float* tw;
-  unsigned* status;
-};
-
-__global__ void __launch_bounds__(192, 1)
-    k_router_tc(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW, TcRouterArgs p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = align1024(smem_raw);
-  const int A_BYTES = kBM * kBK * 2;
-  const int B_BYTES = (p.n2 ? 512 : p.E_pad) * kBK * 2;
-  const int STAGE_BYTES = A_BYTES + B_BYTES;
-  const int S = p.stages;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * STAGE_BYTES);
-  uint64_t* empty = full + S;
-  uint64_t* tfull = empty + S;
-  uint64_t* drain = tfull + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const unsigned tcode = kStatusTimeoutBase | (kKernRouterTc << 8);
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < S; ++s) {
-      mbar_init(full + s, 1);
-      mbar_init(empty + s, 1);
-    }
-    mbar_init(tfull, 1);
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_barrier_init();
-  }
-  if (warp == 1) {
-    tmem_alloc(tmem_slot, p.tmem_cols);
-    tmem_relinquish();
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  const int row0 = blockIdx.x * kBM;
-
-  if (warp == 0) {
-    if (lane == 0) {
-      const uint64_t pol = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0, issued = 0, last_par = 0;
-      for (int kb = 0; kb < p.kblocks; ++kb) {
-        if (!mbar_wait(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 1)) break;
-        uint8_t* sa = smem + stage * STAGE_BYTES;
-        uint8_t* sb = sa + A_BYTES;
-        mbar_arrive_expect_tx(full + stage, STAGE_BYTES);
-        tma_load_2d(sa, &tmX, full + stage, kb * kBK, row0, pol);
-        tma_load_2d(sb, &tmW, full + stage, kb * kBK, 0, pol);
-        if (p.n2) tma_load_2d(sb + 256 * kBK * 2, &tmW, full + stage, kb * kBK, 256, pol);
-        issued |= 1u << stage;
-        last_par = (last_par & ~(1u << stage)) | (phase << stage);
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-      if (*abort_flag)
-        for (int s = 0; s < S; ++s)
-          if (issued >> s & 1u) drain_wait(full + s, last_par >> s & 1u);
-    }
-    __syncwarp();
-  } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t id1 = idesc_bf16(kBM, p.n1);
-      const uint32_t id2 = idesc_bf16(kBM, p.n2 ? p.n2 : 16);
-      int stage = 0;
-      uint32_t phase = 0;
-      bool ok = true;
-      for (int kb = 0; kb < p.kblocks; ++kb) {
-        if (!mbar_wait(full + stage, phase, abort_flag, p.status, tcode | 3)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t sa = smem_u32(smem + stage * STAGE_BYTES);
-        const uint32_t sb = sa + A_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(sa + kk * 32);
-          const uint32_t accum = (kb | kk) != 0;
-          umma_f16(tmem_base, ad, sdesc_sw128(sb + kk * 32), id1, accum);
-          if (p.n2) umma_f16(tmem_base + 256, ad, sdesc_sw128(sb + 256 * kBK * 2 + kk * 32), id2, accum);
-        }
-        umma_commit(empty + stage);
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1;
-        }
-      }
-      if (ok) umma_commit(tfull);
-      umma_commit(drain);
-      drain_wait(drain, 0);
-    }
-    __syncwarp();
-  } else {
-    const int q = warp & 3;
-    const int row = q * 32 + lane;
-    const int64_t t = (int64_t)row0 + row;
-    if (mbar_wait(tfull, 0, abort_flag, p.status, tcode | 4)) {
-      tc_fence_after();
-      const uint32_t tb = tmem_base + ((uint32_t)(q * 32) << 16);
-      float tv[kMaxK];
-      int te[kMaxK];
-#pragma unroll
-      for (int i = 0; i < kMaxK; ++i) {
-        tv[i] = -INFINITY;
-        te[i] = -1;
-      }
-      float kth = -INFINITY;
-      const int k = p.k;
-      for (int c = 0; c < p.E_pad; c += 32) {
-        uint32_t a[32];
-        tmem_ld32(tb + c, a);
-        tmem_wait_regs(a);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int e = c + j;
-          if (e < p.E) {
-            float v = __uint_as_float(a[j]);
-            if (p.bias) v += __ldg(p.bias + e);
-            if (v > kth) {
-#pragma unroll
-              for (int i = kMaxK - 1; i > 0; --i) {
-                if (i < k) {
-                  if (tv[i - 1] < v) {
-                    tv[i] = tv[i - 1];
-                    te[i] = te[i - 1];
-                  } else if (tv[i] < v) {
-                    tv[i] = v;
-                    te[i] = e;
-                  }
-                }
-              }
-              if (tv[0] < v) {
-                tv[0] = v;
-                te[0] = e;
-              }
-#pragma unroll
-              for (int i = 0; i < kMaxK; ++i)
-                if (i == k - 1) kth = tv[i];
-            }
-          }
-        }
-      }
-      if (t < p.T) {
-        float den = 0.f;
-#pragma unroll
-        for (int i = 0; i < kMaxK; ++i)
-          if (i < k) den += __expf(tv[i] - tv[0]);
-        const float inv = 1.0f / den;
-#pragma unroll
-        for (int i = 0; i < kMaxK; ++i)
-          if (i < k) {
-            p.ids[t * k + i] = te[i];
-            p.tw[t * k + i] = __expf(tv[i] - tv[0]) * inv;
-          }
-      }
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 1) {
-    __syncwarp();
-    tc_fence_after();
-    tmem_dealloc(tmem_base, p.tmem_cols);
   }
 }
 

@@ -61,10 +61,11 @@ def test_workspace_sizes_grow_with_tokens():
     b = moe.workspace_size(P(T=4096))
     assert 0 < a < b
     assert moe.workspace_size(P(k=0)) == 0
-    # forward workspace holds at least the dispatched rows, H and the fp32 output
+    # forward workspace holds at least the dispatched rows (shared with the
+    # weighted slot rows of the down projection) and the SwiGLU activations H
     p = P(T=4096)
     Rp = 4096 * 3
-    assert b >= Rp * 256 * 2 + Rp * 128 * 2 + 4096 * 256 * 4
+    assert b >= Rp * 256 * 2 + Rp * 128 * 2
     assert moe.stage_workspace_size(p) < b
 
 
