@@ -144,6 +144,28 @@ MOE_API moe_status moe_layer_forward(const moe_problem* p, const void* x, const 
                              int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes,
                              void* stream);
 
+/* moe_router_topk for callers that cannot allocate device memory: code that
+ * runs where cudaMalloc is off limits (inside a host framework that owns every
+ * device allocation, or on a latency-critical thread that must not enter an
+ * allocator) and so cannot hand the router a workspace.  The block's pages
+ * have no counterpart of this entry point; it is a property of the library.
+ * Same arguments and results as moe_router_topk minus the workspace: the
+ * router's logit partials go to a file-scope __device__ array of
+ * MOE_ROUTER_STATIC_SCRATCH_BYTES that every device that loads the library
+ * keeps until the process exits.  Nothing is allocated or freed.
+ *   - Problems whose partials need more than that (about
+ *     splits * T * roundup(E, 32) * 4 bytes; e.g. T = 8192 with E = 512) are
+ *     rejected with MOE_ERR_UNSUPPORTED before anything is launched.
+ *   - The first call on a device looks up that device's copy of the array
+ *     (a one-time set-up); make it before any stream capture.
+ *   - Every call uses the same array and leaves its contents behind; calls
+ *     that overlap on the GPU (other streams, other threads) race on it and
+ *     must be serialised by the caller. */
+#define MOE_ROUTER_STATIC_SCRATCH_BYTES (32u << 20)
+MOE_API moe_status moe_router_topk_static(const moe_problem* p, const void* x, const void* w_router,
+                                  const float* router_bias, int32_t* topk_ids, float* topk_w,
+                                  void* stream);
+
 /* Kernel-path selection for the calls above on the calling process:
  * 0 = automatic (tensor-core kernels where the shapes allow), 1 = SIMT CUDA
  * kernels only (fp32 FMA; the path of fp32 problems), 2 = tensor-core kernels

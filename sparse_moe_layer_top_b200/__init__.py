@@ -29,7 +29,7 @@ _STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "
 EXPORTS = ("moe_check_problem", "moe_workspace_size", "moe_stage_workspace_size", "moe_router_topk",
            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_set_path",
            "moe_device_status", "moe_last_launch_count", "moe_profile_enable", "moe_profile_read",
-           "moe_last_error_string")
+           "moe_last_error_string", "moe_router_topk_static")
 
 
 class MoEError(RuntimeError):
@@ -66,6 +66,7 @@ def lib():
         L.moe_stage_workspace_size.argtypes = [PP]
         L.moe_stage_workspace_size.restype = ctypes.c_size_t
         L.moe_router_topk.argtypes = [PP, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.moe_router_topk_static.argtypes = [PP, P, P, P, P, P, P]
         L.moe_permute.argtypes = [PP, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_expert_ffn.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_combine.argtypes = [PP, P, P, P, P, P, P]
@@ -79,7 +80,7 @@ def lib():
                                        ctypes.POINTER(ctypes.c_char_p)]
         L.moe_profile_read.restype = ctypes.c_int
         L.moe_last_error_string.restype = ctypes.c_char_p
-        for f in ("moe_check_problem", "moe_router_topk", "moe_permute", "moe_expert_ffn", "moe_combine",
+        for f in ("moe_check_problem", "moe_router_topk", "moe_router_topk_static", "moe_permute", "moe_expert_ffn", "moe_combine",
                   "moe_layer_forward", "moe_set_path", "moe_device_status"):
             getattr(L, f).restype = S
         _lib = L

@@ -837,3 +837,63 @@ moe_status moe_layer_forward(const moe_problem* p, const void* x, const void* w_
 }
 
 }  // extern "C"
+
+// ============================================================== router without a workspace
+// For callers that cannot allocate device memory themselves (see
+// moe_router_topk_static in moe.h): the logit partials go to a fixed array
+// that every device holding this library keeps for the life of the process.
+static __device__ __align__(256) unsigned char g_router_scratch[MOE_ROUTER_STATIC_SCRATCH_BYTES];
+static void* g_router_scratch_ptr[kMaxDevices];
+static std::mutex g_router_scratch_mu;
+
+// Device address of this device's copy of the array (host code may not use
+// the symbol itself: on the host it names a stand-in, not device memory).
+static moe_status router_scratch(void** out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_CUDA, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_router_scratch_mu);
+  if (!g_router_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&ptr, g_router_scratch);
+    if (e != cudaSuccess || !ptr)
+      return fail(MOE_ERR_CUDA, "cudaGetSymbolAddress(router scratch): %s", cudaGetErrorString(e));
+    g_router_scratch_ptr[dev] = ptr;
+  }
+  *out = g_router_scratch_ptr[dev];
+  return MOE_OK;
+}
+
+extern "C" moe_status moe_router_topk_static(const moe_problem* p, const void* x, const void* w_router,
+                                             const float* router_bias, int32_t* topk_ids, float* topk_w,
+                                             void* stream) {
+  moe_status s = check(p);
+  if (s != MOE_OK) return s;
+  if (p->T == 0) {
+    g_launches = 0;
+    return MOE_OK;
+  }
+  NEED(x);
+  NEED(w_router);
+  MAYBE(router_bias);
+  NEED(topk_ids);
+  NEED(topk_w);
+  size_t need = 0;
+  if (p->act_dtype == MOE_BF16) {
+    const RouterSplit rs = router_split(*p);
+    need = (size_t)rs.ksplit * p->T * rs.ldp * 4;
+  }
+  if (need > (size_t)MOE_ROUTER_STATIC_SCRATCH_BYTES)
+    return fail(MOE_ERR_UNSUPPORTED, "router needs %zu bytes of scratch; the built-in array holds %zu (use moe_router_topk with a workspace)",
+                need, (size_t)MOE_ROUTER_STATIC_SCRATCH_BYTES);
+  DeviceInfo* dev;
+  if ((s = device_info(&dev)) != MOE_OK) return s;
+  void* scratch = nullptr;
+  if ((s = router_scratch(&scratch)) != MOE_OK) return s;
+  g_launches_pending = 0;
+  bool counted;
+  s = launch_router(*p, x, w_router, router_bias, topk_ids, topk_w, (float*)scratch, nullptr, &counted,
+                    (cudaStream_t)stream, dev);
+  if (s == MOE_OK) g_launches = g_launches_pending;
+  return s;
+}

@@ -1,0 +1,74 @@
+"""moe_router_topk_static: the router stage for callers that cannot allocate
+device memory and so have no workspace to give it.
+
+It is called through the C ABI and must reproduce moe_router_topk (the same
+kernels, with the logit partials in the library's built-in array instead of
+a caller workspace), on two calls in a row, since the array keeps whatever the
+previous call left in it.  This file is collected last on purpose.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import moe_inputs
+from parity import TOL_W
+
+pytestmark = pytest.mark.gpu
+
+
+def _p(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+@pytest.mark.parametrize("shape", [(300, 256, 20, 4, "bf16"), (4096, 2048, 256, 8, "bf16"),
+                                   (64, 8192, 512, 10, "bf16"), (77, 96, 24, 3, "f32")])
+def test_static_router_matches_workspace_router_twice(shape):
+    import sparse_moe_layer_top_b200 as moe
+    T, d, E, k, act = shape
+    torch.cuda.set_device(0)
+    x = moe_inputs.randn((T, d), "cuda", 5, moe_inputs.X, 1.0, torch.float32 if act == "f32" else torch.bfloat16)
+    w_r = moe_inputs.randn((E, d), "cuda", 5, moe_inputs.W_R, 0.02, x.dtype)
+    bias = moe_inputs.zipf_bias(E, "cuda")
+    prob = moe.Problem.make(T, d, E, k, 64, 64, act, act)
+    L = moe.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+    ws = torch.empty(max(moe.stage_workspace_size(prob), 1), dtype=torch.uint8, device="cuda")
+    ids_ref = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    w_ref = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    assert L.moe_router_topk(ctypes.byref(prob), _p(x), _p(w_r), _p(bias), _p(ids_ref), _p(w_ref), _p(ws),
+                             ws.numel(), stream) == 0
+    torch.cuda.synchronize()
+
+    for call in range(2):
+        ids = torch.full((T, k), -7, dtype=torch.int32, device="cuda")
+        tw = torch.full((T, k), -1.0, dtype=torch.float32, device="cuda")
+        rc = L.moe_router_topk_static(ctypes.byref(prob), _p(x), _p(w_r), _p(bias), _p(ids), _p(tw), stream)
+        assert rc == 0, L.moe_last_error_string()
+        torch.cuda.synchronize()
+        assert moe.device_status()[0] == 0
+        assert torch.equal(ids, ids_ref), "call %d: expert ids differ" % call
+        err = (tw - w_ref).abs().max().item()
+        assert err <= TOL_W[act], "call %d: weight error %.3g" % (call, err)
+
+
+def test_static_router_rejects_what_does_not_fit():
+    import sparse_moe_layer_top_b200 as moe
+    # 157 x 2 (row block, expert block) tiles already cover the GPU, so the
+    # router takes one split: 20000 x 512 fp32 logits = 41 MB > the 32 MiB
+    # array.  Real buffers all the same, so that nothing could go wrong even
+    # if the check let the call through.
+    T, d, E, k = 20000, 8192, 512, 10
+    x = torch.zeros((T, d), dtype=torch.bfloat16, device="cuda")
+    w_r = torch.zeros((E, d), dtype=torch.bfloat16, device="cuda")
+    ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    prob = moe.Problem.make(T, d, E, k, 2048, 2048, "bf16", "bf16")
+    L = moe.lib()
+    rc = L.moe_router_topk_static(ctypes.byref(prob), _p(x), _p(w_r), None, _p(ids), _p(tw),
+                                  ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert rc == 2
+    assert b"scratch" in L.moe_last_error_string()
