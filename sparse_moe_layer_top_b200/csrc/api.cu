@@ -133,6 +133,9 @@ static moe_status device_info(DeviceInfo** out) {
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcSlotStore>, Gemm2Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcStore>, Gemm2Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcLogits>, Gemm2Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_tc<128, true, 4, kTcSwiGLU, true>, Gemm1Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcSlotStore, true>, Gemm2Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcStore, true>, Gemm2Cfg::SMEM_BYTES));
     d.ready = true;
   }
   *out = &d;
@@ -159,8 +162,10 @@ static moe_status encode_fn(EncodeTiledFn* out) {
   return MOE_OK;
 }
 
-// bf16 tensor, 128-byte swizzle, box {64, box_rows} (x {1}); out-of-range reads give zeros.
-static moe_status map_bf16(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+// Box {64 elements, box_rows} (x {1}); bf16 tiles are 128-byte swizzled for the
+// MMA, 1-byte E4M3 tiles are loaded plain for the converter warps.
+// Out-of-range reads give zeros.
+static moe_status map_tile(CUtensorMap* m, const void* base, bool bytes, int rank, const uint64_t* dims,
                            const uint64_t* strides_bytes, uint32_t box_rows) {
   EncodeTiledFn enc;
   moe_status s = encode_fn(&enc);
@@ -169,23 +174,26 @@ static moe_status map_bf16(CUtensorMap* m, const void* base, int rank, const uin
   cuuint32_t box[3] = {(cuuint32_t)kBK, box_rows, 1}, es[3] = {1, 1, 1};
   for (int i = 0; i < rank; ++i) gd[i] = dims[i] ? dims[i] : 1;
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
-  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), gd, gs, box, es,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  CUresult r = enc(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
+                   const_cast<void*>(base), gd, gs, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   bytes ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) rank %d dims %llu x %llu", (int)r, rank,
                 (unsigned long long)gd[0], (unsigned long long)gd[1]);
   return MOE_OK;
 }
 static moe_status map2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t stride_elems,
-                        uint32_t box_rows) {
-  uint64_t dims[2] = {inner, outer}, st[1] = {stride_elems * 2};
-  return map_bf16(m, base, 2, dims, st, box_rows);
+                        uint32_t box_rows, bool bytes = false) {
+  const uint64_t eb = bytes ? 1 : 2;
+  uint64_t dims[2] = {inner, outer}, st[1] = {stride_elems * eb};
+  return map_tile(m, base, bytes, 2, dims, st, box_rows);
 }
 static moe_status map3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
-                        uint32_t box_rows) {
-  uint64_t dims[3] = {inner, mid, outer}, st[2] = {inner * 2, inner * mid * 2};
-  return map_bf16(m, base, 3, dims, st, box_rows);
+                        uint32_t box_rows, bool bytes = false) {
+  const uint64_t eb = bytes ? 1 : 2;
+  uint64_t dims[3] = {inner, mid, outer}, st[2] = {inner * eb, inner * mid * eb};
+  return map_tile(m, base, bytes, 3, dims, st, box_rows);
 }
 
 // ============================================================== checks
@@ -228,8 +236,10 @@ static bool misaligned(const void* ptr) { return (reinterpret_cast<uintptr_t>(pt
     if ((ptr) && misaligned(ptr)) return fail(MOE_ERR_ALIGNMENT, "%s is not 16-byte aligned", #ptr); \
   } while (0)
 
-// Tensor-core expert kernels: bf16 activations and bf16 weights.
-static bool tc_shapes(const moe_problem& p) { return p.act_dtype == MOE_BF16 && p.w_dtype == MOE_BF16; }
+// Tensor-core expert kernels: bf16 activations; bf16 or E4M3 weights.
+static bool tc_shapes(const moe_problem& p) {
+  return p.act_dtype == MOE_BF16 && (p.w_dtype == MOE_BF16 || p.w_dtype == MOE_FP8_E4M3_B128);
+}
 
 static moe_status choose(bool tc_possible, bool* use_tc) {
   if (g_path == 1) {
@@ -489,22 +499,26 @@ static moe_status simt_gemms(const moe_problem& p, const void* xp, const int32_t
   return MOE_OK;
 }
 
-static moe_status tc_gemms(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
-                           int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
-                           DeviceInfo* dev) {
+template <bool FP8>
+static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
+                             int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
+                             DeviceInfo* dev) {
   const int64_t Rp = rows_total(p), ldh = ldh_of(p);
   const bool sh = p.I_s > 0;
+  const unsigned threads = FP8 ? 320 : 192;
+  const float* sp[6];
+  scale_parts(p, w.scales, sp);
   moe_status s;
   CUtensorMap aR, aS, bR, bS, cR, cS;
   // gate/up + SwiGLU
   if ((s = map2d(&aR, xp, p.d, Rp, p.d, kBM)) != MOE_OK) return s;
-  if ((s = map3d(&bR, w.wg, p.d, p.I, p.E, 128)) != MOE_OK) return s;
-  if ((s = map3d(&cR, w.wu, p.d, p.I, p.E, 128)) != MOE_OK) return s;
+  if ((s = map3d(&bR, w.wg, p.d, p.I, p.E, 128, FP8)) != MOE_OK) return s;
+  if ((s = map3d(&cR, w.wu, p.d, p.I, p.E, 128, FP8)) != MOE_OK) return s;
   bS = bR;
   cS = cR;
   if (sh) {
-    if ((s = map2d(&bS, w.sg, p.d, p.I_s, p.d, 128)) != MOE_OK) return s;
-    if ((s = map2d(&cS, w.su, p.d, p.I_s, p.d, 128)) != MOE_OK) return s;
+    if ((s = map2d(&bS, w.sg, p.d, p.I_s, p.d, 128, FP8)) != MOE_OK) return s;
+    if ((s = map2d(&cS, w.su, p.d, p.I_s, p.d, 128, FP8)) != MOE_OK) return s;
   }
   TcGemmArgs a{};
   a.offs = offs;
@@ -518,17 +532,21 @@ static moe_status tc_gemms(const moe_problem& p, const void* xp, const int32_t* 
   a.K_s = p.d;
   a.H = (bf16*)H;
   a.ldh = ldh;
+  a.sc_b_r = sp[0];
+  a.sc_b_s = sp[3];
+  a.sc_c_r = sp[1];
+  a.sc_c_s = sp[4];
   a.status = dev->status;
   PROF_BEGIN("gemm_tc_swiglu", st);
-  k_gemm_tc<128, true, 4, kTcSwiGLU><<<dev->sms, 192, Gemm1Cfg::SMEM_BYTES, st>>>(aR, aR, bR, bS, cR, cS, a);
+  k_gemm_tc<128, true, 4, kTcSwiGLU, FP8><<<dev->sms, threads, Gemm1Cfg::SMEM_BYTES, st>>>(aR, aR, bR, bS, cR, cS, a);
   LAUNCH_CHECK("gemm_tc_swiglu", st);
   // down
   if ((s = map2d(&aR, H, p.I, Rp, ldh, kBM)) != MOE_OK) return s;
   aS = aR;
   if (sh && (s = map2d(&aS, H, p.I_s, Rp, ldh, kBM)) != MOE_OK) return s;
-  if ((s = map3d(&bR, w.wd, p.I, p.d, p.E, 256)) != MOE_OK) return s;
+  if ((s = map3d(&bR, w.wd, p.I, p.d, p.E, 256, FP8)) != MOE_OK) return s;
   bS = bR;
-  if (sh && (s = map2d(&bS, w.sd, p.I_s, p.d, p.I_s, 256)) != MOE_OK) return s;
+  if (sh && (s = map2d(&bS, w.sd, p.I_s, p.d, p.I_s, 256, FP8)) != MOE_OK) return s;
   TcGemmArgs b{};
   b.offs = offs;
   b.prefix = pre_b;
@@ -539,6 +557,8 @@ static moe_status tc_gemms(const moe_problem& p, const void* xp, const int32_t* 
   b.N_s = p.d;
   b.K_r = p.I;
   b.K_s = p.I_s;
+  b.sc_b_r = sp[2];
+  b.sc_b_s = sp[5];
   b.status = dev->status;
   if (o.ys) {
     b.ys = (bf16*)o.ys;
@@ -546,16 +566,24 @@ static moe_status tc_gemms(const moe_problem& p, const void* xp, const int32_t* 
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
     PROF_BEGIN("gemm_tc_down", st);
-    k_gemm_tc<256, false, 4, kTcSlotStore><<<dev->sms, 192, Gemm2Cfg::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
+    k_gemm_tc<256, false, 4, kTcSlotStore, FP8>
+        <<<dev->sms, threads, Gemm2Cfg::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
     LAUNCH_CHECK("gemm_tc_down", st);
   } else {
     b.out = (bf16*)o.out;
     b.ldo = p.d;
     PROF_BEGIN("gemm_tc_store", st);
-    k_gemm_tc<256, false, 4, kTcStore><<<dev->sms, 192, Gemm2Cfg::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
+    k_gemm_tc<256, false, 4, kTcStore, FP8><<<dev->sms, threads, Gemm2Cfg::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
     LAUNCH_CHECK("gemm_tc_store", st);
   }
   return MOE_OK;
+}
+
+static moe_status tc_gemms(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
+                           int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
+                           DeviceInfo* dev) {
+  if (p.w_dtype == MOE_FP8_E4M3_B128) return tc_gemms_t<true>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
+  return tc_gemms_t<false>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
 }
 
 static moe_status expert_gemms(const moe_problem& p, bool tc, const void* xp, const int32_t* offs,

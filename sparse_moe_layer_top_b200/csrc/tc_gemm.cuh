@@ -25,6 +25,12 @@
 //                 Logits    part[split][r, n] = D (+ nothing) -> fp32
 // Rows of a tile past the end of its group are computed and discarded; rows
 // never mix in a GEMM, so those rows cannot disturb the kept ones.
+//
+// E4M3 weights (FP8 = true, 10 warps): the TMA brings the raw 1-byte weight
+// tile (64 bytes per row, unswizzled) into the upper half of the stage's bf16
+// B buffer; warps 6..9 read it, multiply by the tile's 128 x 128 block scale,
+// write bf16 in the 128-byte-swizzled layout the MMA expects, fence the async
+// proxy and release the stage to the MMA warp.  The MMA itself stays bf16.
 #pragma once
 #include "common.cuh"
 #include "ptx.cuh"
@@ -55,6 +61,9 @@ struct TcGemmArgs {
   int64_t ldo;
   float* part;            // Logits output [ksplit][rows, ldp]
   int64_t ldp, part_stride;
+  // E4M3 weights: fp32 scales per 128 x 128 block, [E][N/128][K/128] routed,
+  // [N/128][K/128] shared; B = gate (or the single operand), C = up
+  const float *sc_b_r, *sc_b_s, *sc_c_r, *sc_c_s;
   unsigned* status;
 };
 
@@ -126,16 +135,46 @@ struct TcGemmCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES * (DUAL ? 2 : 1);
   static constexpr int ACC_COLS = DUAL ? 2 * BN : BN;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
-  static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8 + 16;
+  static constexpr int BAR_BYTES = (3 * STAGES + 5) * 8 + 16;
   static constexpr int SCHED_INTS = 2 * (512 + 2);  // tile prefix + group offsets, E <= 512
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + SCHED_INTS * 4;
   static_assert(TMEM_COLS == 64 || TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
-  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128");
+  static_assert(BN % 16 == 0 && BN >= 16 && (DUAL ? 2 * BN : BN) <= 256, "UMMA N for M=128");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-template <int BN, bool DUAL, int STAGES, int EPI>
-__global__ void __launch_bounds__(192, 1)
+// Named barrier 1 among the 128 converter threads.
+__device__ __forceinline__ void conv_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// Barrier 1 with an AND over the converters' flags: all of them see the same answer.
+__device__ __forceinline__ bool conv_all(bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)ok)
+      : "memory");
+  return r != 0;
+}
+// Generic-proxy shared-memory writes made visible to the async proxy (tensor core).
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Four E4M3 codes (one 32-bit word, element 0 in the low byte) times a scale -> four bf16.
+__device__ __forceinline__ uint2 e4m3x4_scaled_bf16(uint32_t w, float sc) {
+  const __half2_raw lo = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w & 0xffffu), __NV_E4M3);
+  const __half2_raw hi = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w >> 16), __NV_E4M3);
+  const float2 a = __half22float2(__half2(lo));
+  const float2 b = __half22float2(__half2(hi));
+  uint2 r;
+  r.x = pack_bf16x2(a.x * sc, a.y * sc);
+  r.y = pack_bf16x2(b.x * sc, b.y * sc);
+  return r;
+}
+
+template <int BN, bool DUAL, int STAGES, int EPI, bool FP8 = false>
+__global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
               const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
               const __grid_constant__ CUtensorMap tmC_r, const __grid_constant__ CUtensorMap tmC_s, TcGemmArgs p) {
@@ -147,7 +186,8 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* full8 = drain + 1;  // FP8: TMA landed (A + raw weights); `full` then means converted
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full8 + STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* s_pre = reinterpret_cast<int32_t*>(smem + STAGES * Cfg::STAGE_BYTES + Cfg::BAR_BYTES);
   int32_t* s_offs = s_pre + 514;
@@ -162,8 +202,9 @@ __global__ void __launch_bounds__(192, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full + s, 1);
+      mbar_init(full + s, FP8 ? 128 : 1);
       mbar_init(empty + s, 1);
+      mbar_init(full8 + s, 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull + b, 1);
@@ -211,14 +252,18 @@ __global__ void __launch_bounds__(192, 1)
           }
           uint8_t* sa = smem + stage * Cfg::STAGE_BYTES;
           uint8_t* sb = sa + Cfg::A_BYTES;
-          mbar_arrive_expect_tx(full + stage, Cfg::STAGE_BYTES);
-          tma_load_2d(sa, sh ? &tmA_s : &tmA_r, full + stage, kb * kBK, (int)t.row0, pol_a);
-          if (sh) tma_load_2d(sb, &tmB_s, full + stage, kb * kBK, t.n0, pol_w);
-          else tma_load_3d(sb, &tmB_r, full + stage, kb * kBK, t.n0, t.g, pol_w);
+          uint64_t* land = (FP8 ? full8 : full) + stage;
+          // FP8: raw 1-byte rows packed in the upper half of the bf16 B buffer
+          constexpr int NB = DUAL ? 2 * BN : BN;
+          uint8_t* sbw = FP8 ? sb + NB * 64 : sb;
+          uint8_t* scw = FP8 ? sbw + BN * 64 : sb + Cfg::B_BYTES;
+          mbar_arrive_expect_tx(land, FP8 ? Cfg::A_BYTES + NB * 64 : Cfg::STAGE_BYTES);
+          tma_load_2d(sa, sh ? &tmA_s : &tmA_r, land, kb * kBK, (int)t.row0, pol_a);
+          if (sh) tma_load_2d(sbw, &tmB_s, land, kb * kBK, t.n0, pol_w);
+          else tma_load_3d(sbw, &tmB_r, land, kb * kBK, t.n0, t.g, pol_w);
           if (DUAL) {
-            uint8_t* sc = sb + Cfg::B_BYTES;
-            if (sh) tma_load_2d(sc, &tmC_s, full + stage, kb * kBK, t.n0, pol_w);
-            else tma_load_3d(sc, &tmC_r, full + stage, kb * kBK, t.n0, t.g, pol_w);
+            if (sh) tma_load_2d(scw, &tmC_s, land, kb * kBK, t.n0, pol_w);
+            else tma_load_3d(scw, &tmC_r, land, kb * kBK, t.n0, t.g, pol_w);
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
@@ -231,13 +276,16 @@ __global__ void __launch_bounds__(192, 1)
       }
       if (*abort_flag)  // copies in flight must land before the CTA exits
         for (int s = 0; s < STAGES; ++s)
-          if (issued >> s & 1u) drain_wait(full + s, last_par >> s & 1u);
+          if (issued >> s & 1u) drain_wait((FP8 ? full8 : full) + s, last_par >> s & 1u);
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = idesc_bf16(kBM, BN);
+      // DUAL: the gate and up tiles sit back to back in shared memory, so one
+      // MMA of N = 2*BN fills both accumulators (gate at d0, up at d0 + BN) and
+      // reads the A tile once instead of twice.
+      constexpr uint32_t idesc = idesc_bf16(kBM, DUAL ? 2 * BN : BN);
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
@@ -259,7 +307,6 @@ __global__ void __launch_bounds__(192, 1)
             const uint64_t ad = sdesc_sw128(sa + kk * 32);
             const uint32_t accum = (kb != t.kb0 || kk != 0);
             umma_f16(d0, ad, sdesc_sw128(sb + kk * 32), idesc, accum);
-            if (DUAL) umma_f16(d0 + BN, ad, sdesc_sw128(sb + Cfg::B_BYTES + kk * 32), idesc, accum);
           }
           umma_commit(empty + stage);
           if (++stage == STAGES) {
@@ -279,7 +326,7 @@ __global__ void __launch_bounds__(192, 1)
       drain_wait(drain, 0);
     }
     __syncwarp();
-  } else {
+  } else if (warp < 6) {
     // ------------------------------------------------ epilogue (warps 2..5)
     const int q = warp & 3;
     const int row = q * 32 + lane;
@@ -394,6 +441,64 @@ __global__ void __launch_bounds__(192, 1)
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
+      }
+    }
+  } else if (FP8) {
+    // ------------------------------------------------ E4M3 -> bf16 converters (warps 6..9)
+    constexpr int NB = DUAL ? 2 * BN : BN;  // bf16 rows of a B stage: gate rows, then up rows
+    static_assert(!FP8 || NB == 256, "converter mapping: two rows per thread");
+    const int ct = threadIdx.x - 192;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
+      const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
+      const bool sh = t.g == p.E;
+      const int kb128 = ((sh ? p.K_s : p.K_r) + 127) / 128, nb128 = (t.N + 127) / 128;
+      const int64_t eoff = (int64_t)t.g * nb128 * kb128;
+      const float* s1 = sh ? p.sc_b_s : p.sc_b_r + eoff;
+      const float* s2 = DUAL ? (sh ? p.sc_c_s : p.sc_c_r + eoff) : s1;
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        const bool ok = mbar_wait(full8 + stage, phase, abort_flag, p.status, tcode | 5);
+        if (!conv_all(ok)) {
+          stop = true;
+          break;
+        }
+        uint8_t* sb = smem + stage * Cfg::STAGE_BYTES + Cfg::A_BYTES;
+        const uint8_t* raw = sb + NB * 64;
+        uint4 q[2][4];
+        float sc[2];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int r = ct + 128 * h;
+          const uint4* src = reinterpret_cast<const uint4*>(raw + r * 64);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) q[h][v] = src[v];
+          const bool up = DUAL && r >= BN;
+          const int n = t.n0 + (up ? r - BN : r);
+          sc[h] = n < t.N ? __ldg((up ? s2 : s1) + (n / 128) * kb128 + (kb * kBK) / 128) : 0.f;
+        }
+        conv_sync();  // every raw byte read before any bf16 byte overwrites it
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int r = ct + 128 * h;
+          uint8_t* dst = sb + r * 128;
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const uint2 a = e4m3x4_scaled_bf16(q[h][v].x, sc[h]);
+            const uint2 b = e4m3x4_scaled_bf16(q[h][v].y, sc[h]);
+            const uint2 c = e4m3x4_scaled_bf16(q[h][v].z, sc[h]);
+            const uint2 d = e4m3x4_scaled_bf16(q[h][v].w, sc[h]);
+            *reinterpret_cast<uint4*>(dst + (((2 * v) ^ (r & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+            *reinterpret_cast<uint4*>(dst + (((2 * v + 1) ^ (r & 7)) << 4)) = make_uint4(c.x, c.y, d.x, d.y);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(full + stage);
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
       }
     }
   }

@@ -43,6 +43,7 @@ FORWARD_CASES = {
     "bf16_T1": (1, 256, 40, 5, 128, 64, "bf16", "bf16", None),
     "bf16_I_ne_Is": (129, 256, 16, 3, 136, 264, "bf16", "bf16", None),
     "fp8_small": (64, 256, 8, 2, 256, 128, "bf16", "fp8", None),
+    "fp8_multi_tile": (300, 384, 12, 3, 384, 256, "bf16", "fp8", None),
 }
 
 
@@ -211,6 +212,19 @@ def test_paths_agree_bf16(moe):
         y, ids, tw = _gpu_forward(moe, g)
         out.append((y, ids))
     moe.set_path(0)
+    assert rel_l2(out[1][0], out[0][0]) <= 1e-2
+
+
+def test_paths_agree_fp8(moe):
+    inp = moe_inputs.make_inputs(200, 512, 24, 4, 256, 256, act="bf16", w="fp8", seed=2)
+    g = to_device(inp, "cuda")
+    out = []
+    for path in (1, 2):
+        moe.set_path(path)
+        y, ids, tw = _gpu_forward(moe, g)
+        out.append((y, ids))
+    moe.set_path(0)
+    assert np.array_equal(out[0][1], out[1][1])
     assert rel_l2(out[1][0], out[0][0]) <= 1e-2
 
 
