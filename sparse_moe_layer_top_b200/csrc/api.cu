@@ -112,6 +112,9 @@ static cudaError_t allow_smem(K kernel, int bytes) {
 // GEMM instantiations used by the library.
 using Gemm1Cfg = TcGemmCfg<128, true, 4>;
 using Gemm2Cfg = TcGemmCfg<256, false, 4>;
+constexpr int kFp8Stages = 2;
+using Gemm1F8Cfg = TcGemmCfg<128, true, kFp8Stages, true>;
+using Gemm2F8Cfg = TcGemmCfg<256, false, kFp8Stages, true>;
 
 static moe_status device_info(DeviceInfo** out) {
   int dev = 0;
@@ -133,9 +136,9 @@ static moe_status device_info(DeviceInfo** out) {
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcSlotStore>, Gemm2Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcStore>, Gemm2Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcLogits>, Gemm2Cfg::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_tc<128, true, 4, kTcSwiGLU, true>, Gemm1Cfg::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcSlotStore, true>, Gemm2Cfg::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcStore, true>, Gemm2Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_tc<128, true, kFp8Stages, kTcSwiGLU, true>, Gemm1F8Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_tc<256, false, kFp8Stages, kTcSlotStore, true>, Gemm2F8Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_tc<256, false, kFp8Stages, kTcStore, true>, Gemm2F8Cfg::SMEM_BYTES));
     d.ready = true;
   }
   *out = &d;
@@ -505,7 +508,9 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
                              DeviceInfo* dev) {
   const int64_t Rp = rows_total(p), ldh = ldh_of(p);
   const bool sh = p.I_s > 0;
-  const unsigned threads = FP8 ? 320 : 192;
+  constexpr int S = FP8 ? kFp8Stages : 4;
+  using C1 = TcGemmCfg<128, true, S, FP8>;
+  using C2 = TcGemmCfg<256, false, S, FP8>;
   const float* sp[6];
   scale_parts(p, w.scales, sp);
   moe_status s;
@@ -538,7 +543,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   a.sc_c_s = sp[4];
   a.status = dev->status;
   PROF_BEGIN("gemm_tc_swiglu", st);
-  k_gemm_tc<128, true, 4, kTcSwiGLU, FP8><<<dev->sms, threads, Gemm1Cfg::SMEM_BYTES, st>>>(aR, aR, bR, bS, cR, cS, a);
+  k_gemm_tc<128, true, S, kTcSwiGLU, FP8><<<dev->sms, C1::THREADS, C1::SMEM_BYTES, st>>>(aR, aR, bR, bS, cR, cS, a);
   LAUNCH_CHECK("gemm_tc_swiglu", st);
   // down
   if ((s = map2d(&aR, H, p.I, Rp, ldh, kBM)) != MOE_OK) return s;
@@ -566,14 +571,14 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
     PROF_BEGIN("gemm_tc_down", st);
-    k_gemm_tc<256, false, 4, kTcSlotStore, FP8>
-        <<<dev->sms, threads, Gemm2Cfg::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
+    k_gemm_tc<256, false, S, kTcSlotStore, FP8>
+        <<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
     LAUNCH_CHECK("gemm_tc_down", st);
   } else {
     b.out = (bf16*)o.out;
     b.ldo = p.d;
     PROF_BEGIN("gemm_tc_store", st);
-    k_gemm_tc<256, false, 4, kTcStore, FP8><<<dev->sms, threads, Gemm2Cfg::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
+    k_gemm_tc<256, false, S, kTcStore, FP8><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
     LAUNCH_CHECK("gemm_tc_store", st);
   }
   return MOE_OK;

@@ -93,6 +93,13 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* m, uin
       : "memory");
 }
 
+// Bring a tensor tile into L2 ahead of its load (no shared-memory destination).
+__device__ __forceinline__ void tma_prefetch_2d(const CUtensorMap* m, int c0, int c1) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(
+                   reinterpret_cast<uint64_t>(m)), "r"(c0), "r"(c1)
+               : "memory");
+}
+
 // L2 eviction-priority policies for the cache hint.
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;

@@ -26,11 +26,14 @@
 // Rows of a tile past the end of its group are computed and discarded; rows
 // never mix in a GEMM, so those rows cannot disturb the kept ones.
 //
-// E4M3 weights (FP8 = true, 10 warps): the TMA brings the raw 1-byte weight
-// tile (64 bytes per row, unswizzled) into the upper half of the stage's bf16
-// B buffer; warps 6..9 read it, multiply by the tile's 128 x 128 block scale,
-// write bf16 in the 128-byte-swizzled layout the MMA expects, fence the async
-// proxy and release the stage to the MMA warp.  The MMA itself stays bf16.
+// E4M3 weights (FP8 = true, 15 warps): warp 0 streams raw 1-byte weight
+// tiles (64 bytes per row, unswizzled) into a ring of their own, deeper than
+// the stage ring so that more weight bytes are in flight, and prefetches the
+// matching A tile into L2; warp 14 loads the A tiles into the stage ring;
+// warps 6..13 -- one thread per weight row -- multiply the raw tile by its
+// 128 x 128 block scale, write bf16 in the 128-byte-swizzled layout the MMA
+// expects, fence the async proxy and release the stage to the MMA warp.  The
+// MMA itself stays bf16.
 #pragma once
 #include "common.cuh"
 #include "ptx.cuh"
@@ -128,36 +131,28 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     if (globaltimer_ns() - t0 > kWaitLimitNs) break;
 }
 
-template <int BN, bool DUAL, int STAGES>
+template <int BN, bool DUAL, int STAGES, bool FP8 = false>
 struct TcGemmCfg {
   static constexpr int A_BYTES = kBM * kBK * 2;
   static constexpr int B_BYTES = BN * kBK * 2;
+  static constexpr int NB = DUAL ? 2 * BN : BN;          // B rows per stage (gate rows, then up rows)
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES * (DUAL ? 2 : 1);
+  // FP8: a separate, deeper ring of raw E4M3 weight tiles (64 bytes per row)
+  static constexpr int RAW_BYTES = FP8 ? NB * kBK : 0;
+  static constexpr int RAW_STAGES = FP8 ? 6 : 0;
+  static constexpr int RING_BYTES = STAGES * STAGE_BYTES + RAW_STAGES * RAW_BYTES;
+  // FP8: + one converter thread per B row, + one warp issuing the A tiles
+  static constexpr int THREADS = FP8 ? 192 + NB + 32 : 192;
   static constexpr int ACC_COLS = DUAL ? 2 * BN : BN;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
-  static constexpr int BAR_BYTES = (3 * STAGES + 5) * 8 + 16;
+  static constexpr int BAR_BYTES = (3 * STAGES + 2 * RAW_STAGES + 5) * 8 + 16;
   static constexpr int SCHED_INTS = 2 * (512 + 2);  // tile prefix + group offsets, E <= 512
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES + SCHED_INTS * 4;
+  static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + SCHED_INTS * 4;
   static_assert(TMEM_COLS == 64 || TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
   static_assert(BN % 16 == 0 && BN >= 16 && (DUAL ? 2 * BN : BN) <= 256, "UMMA N for M=128");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-// Named barrier 1 among the 128 converter threads.
-__device__ __forceinline__ void conv_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
-// Barrier 1 with an AND over the converters' flags: all of them see the same answer.
-__device__ __forceinline__ bool conv_all(bool ok) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.and.pred q, 1, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)ok)
-      : "memory");
-  return r != 0;
-}
 // Generic-proxy shared-memory writes made visible to the async proxy (tensor core).
 __device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
@@ -174,22 +169,25 @@ __device__ __forceinline__ uint2 e4m3x4_scaled_bf16(uint32_t w, float sc) {
 }
 
 template <int BN, bool DUAL, int STAGES, int EPI, bool FP8 = false>
-__global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
+__global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
               const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
               const __grid_constant__ CUtensorMap tmC_r, const __grid_constant__ CUtensorMap tmC_s, TcGemmArgs p) {
-  using Cfg = TcGemmCfg<BN, DUAL, STAGES>;
+  using Cfg = TcGemmCfg<BN, DUAL, STAGES, FP8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * Cfg::STAGE_BYTES);
+  uint8_t* raw_ring = smem + STAGES * Cfg::STAGE_BYTES;       // FP8 only
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::RING_BYTES);
   uint64_t* empty = full + STAGES;
-  uint64_t* tfull = empty + STAGES;
+  uint64_t* a_full = empty + STAGES;     // FP8: the stage's A tile has landed
+  uint64_t* tfull = a_full + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint64_t* full8 = drain + 1;  // FP8: TMA landed (A + raw weights); `full` then means converted
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full8 + STAGES);
+  uint64_t* raw_full = drain + 1;        // FP8: raw weight tile landed
+  uint64_t* raw_empty = raw_full + Cfg::RAW_STAGES;  // FP8: raw tile converted
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(raw_empty + Cfg::RAW_STAGES);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int32_t* s_pre = reinterpret_cast<int32_t*>(smem + STAGES * Cfg::STAGE_BYTES + Cfg::BAR_BYTES);
+  int32_t* s_pre = reinterpret_cast<int32_t*>(smem + Cfg::RING_BYTES + Cfg::BAR_BYTES);
   int32_t* s_offs = s_pre + 514;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -202,9 +200,13 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full + s, FP8 ? 128 : 1);
+      mbar_init(full + s, FP8 ? Cfg::NB : 1);  // FP8: the converters' arrivals
       mbar_init(empty + s, 1);
-      mbar_init(full8 + s, 1);
+      mbar_init(a_full + s, 1);
+    }
+    for (int s = 0; s < Cfg::RAW_STAGES; ++s) {
+      mbar_init(raw_full + s, 1);
+      mbar_init(raw_empty + s, Cfg::NB);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull + b, 1);
@@ -237,8 +239,14 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer
+      // bf16: A and B tiles into the stage ring.  FP8: raw weight tiles into
+      // the raw ring, running ahead of the stage ring, plus an L2 prefetch of
+      // the A tile that the A warp will load for the same K-block.
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_a = policy_evict_last();
+      constexpr int RING = FP8 ? Cfg::RAW_STAGES : STAGES;
+      uint64_t* land0 = FP8 ? raw_full : full;
+      uint64_t* free0 = FP8 ? raw_empty : empty;
       int stage = 0;
       uint32_t phase = 0, issued = 0, last_par = 0;
       for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
@@ -246,28 +254,38 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
         const bool sh = t.g == p.E;
         bool ok = true;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 1)) {
+          if (!mbar_wait(free0 + stage, phase ^ 1, abort_flag, p.status, tcode | 1)) {
             ok = false;
             break;
           }
-          uint8_t* sa = smem + stage * Cfg::STAGE_BYTES;
-          uint8_t* sb = sa + Cfg::A_BYTES;
-          uint64_t* land = (FP8 ? full8 : full) + stage;
-          // FP8: raw 1-byte rows packed in the upper half of the bf16 B buffer
-          constexpr int NB = DUAL ? 2 * BN : BN;
-          uint8_t* sbw = FP8 ? sb + NB * 64 : sb;
-          uint8_t* scw = FP8 ? sbw + BN * 64 : sb + Cfg::B_BYTES;
-          mbar_arrive_expect_tx(land, FP8 ? Cfg::A_BYTES + NB * 64 : Cfg::STAGE_BYTES);
-          tma_load_2d(sa, sh ? &tmA_s : &tmA_r, land, kb * kBK, (int)t.row0, pol_a);
-          if (sh) tma_load_2d(sbw, &tmB_s, land, kb * kBK, t.n0, pol_w);
-          else tma_load_3d(sbw, &tmB_r, land, kb * kBK, t.n0, t.g, pol_w);
-          if (DUAL) {
-            if (sh) tma_load_2d(scw, &tmC_s, land, kb * kBK, t.n0, pol_w);
-            else tma_load_3d(scw, &tmC_r, land, kb * kBK, t.n0, t.g, pol_w);
+          uint64_t* land = land0 + stage;
+          if (FP8) {
+            uint8_t* sbw = raw_ring + stage * Cfg::RAW_BYTES;
+            uint8_t* scw = sbw + BN * kBK;
+            mbar_arrive_expect_tx(land, Cfg::RAW_BYTES);
+            if (sh) tma_load_2d(sbw, &tmB_s, land, kb * kBK, t.n0, pol_w);
+            else tma_load_3d(sbw, &tmB_r, land, kb * kBK, t.n0, t.g, pol_w);
+            if (DUAL) {
+              if (sh) tma_load_2d(scw, &tmC_s, land, kb * kBK, t.n0, pol_w);
+              else tma_load_3d(scw, &tmC_r, land, kb * kBK, t.n0, t.g, pol_w);
+            }
+            tma_prefetch_2d(sh ? &tmA_s : &tmA_r, kb * kBK, (int)t.row0);
+          } else {
+            uint8_t* sa = smem + stage * Cfg::STAGE_BYTES;
+            uint8_t* sb = sa + Cfg::A_BYTES;
+            mbar_arrive_expect_tx(land, Cfg::STAGE_BYTES);
+            tma_load_2d(sa, sh ? &tmA_s : &tmA_r, land, kb * kBK, (int)t.row0, pol_a);
+            if (sh) tma_load_2d(sb, &tmB_s, land, kb * kBK, t.n0, pol_w);
+            else tma_load_3d(sb, &tmB_r, land, kb * kBK, t.n0, t.g, pol_w);
+            if (DUAL) {
+              uint8_t* sc = sb + Cfg::B_BYTES;
+              if (sh) tma_load_2d(sc, &tmC_s, land, kb * kBK, t.n0, pol_w);
+              else tma_load_3d(sc, &tmC_r, land, kb * kBK, t.n0, t.g, pol_w);
+            }
           }
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == RING) {
             stage = 0;
             phase ^= 1;
           }
@@ -275,8 +293,8 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
         if (!ok) break;
       }
       if (*abort_flag)  // copies in flight must land before the CTA exits
-        for (int s = 0; s < STAGES; ++s)
-          if (issued >> s & 1u) drain_wait((FP8 ? full8 : full) + s, last_par >> s & 1u);
+        for (int s = 0; s < RING; ++s)
+          if (issued >> s & 1u) drain_wait(land0 + s, last_par >> s & 1u);
     }
     __syncwarp();
   } else if (warp == 1) {
@@ -295,7 +313,8 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
         tc_fence_after();
         const uint32_t d0 = tmem_base + acc * Cfg::ACC_COLS;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
-          if (!mbar_wait(full + stage, phase, abort_flag, p.status, tcode | 3)) {
+          if ((FP8 && !mbar_wait(a_full + stage, phase, abort_flag, p.status, tcode | 6)) ||
+              !mbar_wait(full + stage, phase, abort_flag, p.status, tcode | 3)) {
             ok = false;
             break;
           }
@@ -443,64 +462,123 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
         acc_phase ^= 1;
       }
     }
-  } else if (FP8) {
-    // ------------------------------------------------ E4M3 -> bf16 converters (warps 6..9)
-    constexpr int NB = DUAL ? 2 * BN : BN;  // bf16 rows of a B stage: gate rows, then up rows
-    static_assert(!FP8 || NB == 256, "converter mapping: two rows per thread");
+  } else if (FP8 && warp < 6 + Cfg::NB / 32) {
+    // ------------------------------------------------ E4M3 -> bf16 converters
+    // Four threads per 64-byte raw row (one 16-byte chunk each, so a quarter
+    // warp reads 128 consecutive bytes), four passes over the 256 rows.  Rows
+    // 0..127 and 128..255 each sit in one 128-row scale block, so a thread
+    // follows two scale streams, prefetched one 128-wide K block ahead.
+    static_assert(!FP8 || Cfg::NB == 256, "converter mapping covers 256 rows");
     const int ct = threadIdx.x - 192;
-    int stage = 0;
-    uint32_t phase = 0;
+    const int sub = ct & 3, rbase = ct >> 2;  // chunk of the row, row within a pass
+    int stage = 0, rstage = 0;
+    uint32_t phase = 0, rphase = 0;
     bool stop = false;
     for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
       const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
       const bool sh = t.g == p.E;
       const int kb128 = ((sh ? p.K_s : p.K_r) + 127) / 128, nb128 = (t.N + 127) / 128;
       const int64_t eoff = (int64_t)t.g * nb128 * kb128;
-      const float* s1 = sh ? p.sc_b_s : p.sc_b_r + eoff;
-      const float* s2 = DUAL ? (sh ? p.sc_c_s : p.sc_c_r + eoff) : s1;
+      // scale rows of the two halves (NULL where the half lies past N)
+      const float* srow[2];
+      if (DUAL) {
+        const int nb = t.n0 / 128;
+        const bool in = t.n0 < t.N;
+        srow[0] = in ? (sh ? p.sc_b_s : p.sc_b_r + eoff) + (int64_t)nb * kb128 : nullptr;
+        srow[1] = in ? (sh ? p.sc_c_s : p.sc_c_r + eoff) + (int64_t)nb * kb128 : nullptr;
+      } else {
+        const float* base = sh ? p.sc_b_s : p.sc_b_r + eoff;
+        srow[0] = t.n0 < t.N ? base + (int64_t)(t.n0 / 128) * kb128 : nullptr;
+        srow[1] = t.n0 + 128 < t.N ? base + (int64_t)(t.n0 / 128 + 1) * kb128 : nullptr;
+      }
+      float cur[2], nxt[2];
+      {
+        const int j = t.kb0 / 2;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          cur[h] = srow[h] ? __ldg(srow[h] + j) : 0.f;
+          nxt[h] = (srow[h] && j + 1 < kb128) ? __ldg(srow[h] + j + 1) : 0.f;
+        }
+      }
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
-        const bool ok = mbar_wait(full8 + stage, phase, abort_flag, p.status, tcode | 5);
-        if (!conv_all(ok)) {
+        if (kb > t.kb0 && (kb & 1) == 0) {  // a new 128-wide K block: rotate, prefetch the next
+          const int j = kb / 2;
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            cur[h] = nxt[h];
+            nxt[h] = (srow[h] && j + 1 < kb128) ? __ldg(srow[h] + j + 1) : 0.f;
+          }
+        }
+        if (!mbar_wait(raw_full + rstage, rphase, abort_flag, p.status, tcode | 5) ||
+            !mbar_wait(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 7)) {
           stop = true;
           break;
         }
-        uint8_t* sb = smem + stage * Cfg::STAGE_BYTES + Cfg::A_BYTES;
-        const uint8_t* raw = sb + NB * 64;
-        uint4 q[2][4];
-        float sc[2];
+        const uint8_t* raw = raw_ring + rstage * Cfg::RAW_BYTES;
+        uint8_t* bst = smem + stage * Cfg::STAGE_BYTES + Cfg::A_BYTES;
+        uint4 q[4];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int r = ct + 128 * h;
-          const uint4* src = reinterpret_cast<const uint4*>(raw + r * 64);
+        for (int ps = 0; ps < 4; ++ps)
+          q[ps] = *reinterpret_cast<const uint4*>(raw + (rbase + 64 * ps) * kBK + sub * 16);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) q[h][v] = src[v];
-          const bool up = DUAL && r >= BN;
-          const int n = t.n0 + (up ? r - BN : r);
-          sc[h] = n < t.N ? __ldg((up ? s2 : s1) + (n / 128) * kb128 + (kb * kBK) / 128) : 0.f;
+        for (int ps = 0; ps < 4; ++ps) {
+          const int r = rbase + 64 * ps;
+          const float sc = cur[ps >> 1];
+          const uint2 a = e4m3x4_scaled_bf16(q[ps].x, sc);
+          const uint2 b = e4m3x4_scaled_bf16(q[ps].y, sc);
+          const uint2 c = e4m3x4_scaled_bf16(q[ps].z, sc);
+          const uint2 d = e4m3x4_scaled_bf16(q[ps].w, sc);
+          uint8_t* dst = bst + r * 128;
+          *reinterpret_cast<uint4*>(dst + (((2 * sub) ^ (r & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+          *reinterpret_cast<uint4*>(dst + (((2 * sub + 1) ^ (r & 7)) << 4)) = make_uint4(c.x, c.y, d.x, d.y);
         }
-        conv_sync();  // every raw byte read before any bf16 byte overwrites it
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int r = ct + 128 * h;
-          uint8_t* dst = sb + r * 128;
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const uint2 a = e4m3x4_scaled_bf16(q[h][v].x, sc[h]);
-            const uint2 b = e4m3x4_scaled_bf16(q[h][v].y, sc[h]);
-            const uint2 c = e4m3x4_scaled_bf16(q[h][v].z, sc[h]);
-            const uint2 d = e4m3x4_scaled_bf16(q[h][v].w, sc[h]);
-            *reinterpret_cast<uint4*>(dst + (((2 * v) ^ (r & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
-            *reinterpret_cast<uint4*>(dst + (((2 * v + 1) ^ (r & 7)) << 4)) = make_uint4(c.x, c.y, d.x, d.y);
-          }
-        }
+        // The raw slot goes back to the TMA only now: its bytes have been
+        // consumed, and the proxy fence orders these generic-proxy reads before
+        // the async-proxy write that will refill the slot.
         fence_proxy_async_smem();
         mbar_arrive(full + stage);
+        mbar_arrive(raw_empty + rstage);
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;
         }
+        if (++rstage == Cfg::RAW_STAGES) {
+          rstage = 0;
+          rphase ^= 1;
+        }
       }
     }
+  } else if (FP8) {
+    // ------------------------------------------------ A tiles into the stage ring (FP8 mode)
+    if (lane == 0) {
+      const uint64_t pol_a = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, last_par = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
+        const bool sh = t.g == p.E;
+        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+          if (!mbar_wait(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 8)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(a_full + stage, Cfg::A_BYTES);
+          tma_load_2d(smem + stage * Cfg::STAGE_BYTES, sh ? &tmA_s : &tmA_r, a_full + stage, kb * kBK, (int)t.row0,
+                      pol_a);
+          issued |= 1u << stage;
+          last_par = (last_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (*abort_flag)
+        for (int s = 0; s < STAGES; ++s)
+          if (issued >> s & 1u) drain_wait(a_full + s, last_par >> s & 1u);
+    }
+    __syncwarp();
   }
 
   tc_fence_before();
