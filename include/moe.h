@@ -167,9 +167,13 @@ MOE_API moe_status moe_router_topk_static(const moe_problem* p, const void* x, c
                                   void* stream);
 
 /* Kernel-path selection for the calls above on the calling process:
- * 0 = automatic (tensor-core kernels where the shapes allow), 1 = SIMT CUDA
- * kernels only (fp32 FMA; the path of fp32 problems), 2 = tensor-core kernels
- * required (MOE_ERR_UNSUPPORTED when a shape does not allow them). */
+ * 0 = automatic (tensor-core kernels where the types allow; for the expert
+ *     GEMMs the weight-row form when T*k <= 64*E, i.e. when an expert sees at
+ *     most one 64-token chunk on average, else the row-tiled form);
+ * 1 = SIMT CUDA kernels only (fp32 FMA; the path of fp32 problems);
+ * 2 = tensor-core kernels required, row-tiled expert GEMMs;
+ * 3 = tensor-core kernels required, weight-row expert GEMMs.
+ * 2 and 3 return MOE_ERR_UNSUPPORTED when the types do not allow them. */
 MOE_API moe_status moe_set_path(int path);
 
 /* Synchronously read and clear the device status word of the current device

@@ -124,7 +124,8 @@ def check_problem(prob):
 
 
 def set_path(path):
-    """0 automatic, 1 SIMT kernels only, 2 tensor-core kernels required."""
+    """0 automatic, 1 SIMT kernels only, 2 row-tiled tensor-core expert GEMMs,
+    3 weight-row tensor-core expert GEMMs."""
     _check(lib().moe_set_path(int(path)))
 
 

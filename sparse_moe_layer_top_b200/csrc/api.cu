@@ -16,6 +16,7 @@
 #include "router.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
+#include "tc_swap.cuh"
 
 using namespace moe;
 
@@ -139,6 +140,12 @@ static moe_status device_info(DeviceInfo** out) {
     CUDA_TRY(allow_smem(k_gemm_tc<128, true, kFp8Stages, kTcSwiGLU, true>, Gemm1F8Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, kFp8Stages, kTcSlotStore, true>, Gemm2F8Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, kFp8Stages, kTcStore, true>, Gemm2F8Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap<true, kTcSwiGLU, false>, SwapCfg<true, false>::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap<false, kTcSlotStore, false>, SwapCfg<false, false>::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap<false, kTcStore, false>, SwapCfg<false, false>::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap<true, kTcSwiGLU, true>, SwapCfg<true, true>::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap<false, kTcSlotStore, true>, SwapCfg<false, true>::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap<false, kTcStore, true>, SwapCfg<false, true>::SMEM_BYTES));
     d.ready = true;
   }
   *out = &d;
@@ -247,12 +254,28 @@ static bool tc_shapes(const moe_problem& p) {
 static moe_status choose(bool tc_possible, bool* use_tc) {
   if (g_path == 1) {
     *use_tc = false;
-  } else if (g_path == 2) {
+  } else if (g_path >= 2) {
     if (!tc_possible) return fail(MOE_ERR_UNSUPPORTED, "tensor-core path required but the types do not allow it");
     *use_tc = true;
   } else {
     *use_tc = tc_possible;
   }
+  return MOE_OK;
+}
+
+// Expert GEMM form: 0 SIMT, 1 row-tiled tensor core, 2 weight-row (swap)
+// tensor core.  Automatic choice: the weight-row form when an expert sees at
+// most one token chunk on average (T*k <= 64*E), where a 128-row activation
+// tile would be mostly empty.
+enum { kFormSimt = 0, kFormRows = 1, kFormSwap = 2 };
+static moe_status choose_form(const moe_problem& p, int* form) {
+  bool tc;
+  moe_status s = choose(tc_shapes(p), &tc);
+  if (s != MOE_OK) return s;
+  if (!tc) *form = kFormSimt;
+  else if (g_path == 2) *form = kFormRows;
+  else if (g_path == 3) *form = kFormSwap;
+  else *form = p.T * (int64_t)p.k <= (int64_t)kNCH * p.E ? kFormSwap : kFormRows;
   return MOE_OK;
 }
 
@@ -591,19 +614,106 @@ static moe_status tc_gemms(const moe_problem& p, const void* xp, const int32_t* 
   return tc_gemms_t<false>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
 }
 
-static moe_status expert_gemms(const moe_problem& p, bool tc, const void* xp, const int32_t* offs,
+template <bool FP8>
+static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
+                               int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
+                               DeviceInfo* dev) {
+  using C1 = SwapCfg<true, FP8>;
+  using C2 = SwapCfg<false, FP8>;
+  const int64_t Rp = rows_total(p), ldh = ldh_of(p);
+  const bool sh = p.I_s > 0;
+  const float* sp[6];
+  scale_parts(p, w.scales, sp);
+  moe_status s;
+  CUtensorMap xR, xS, bR, bS, cR, cS;
+  // gate/up + SwiGLU: weights [E, I, d] are the M operand, token rows the N operand
+  if ((s = map2d(&xR, xp, p.d, Rp, p.d, kNCH)) != MOE_OK) return s;
+  if ((s = map3d(&bR, w.wg, p.d, p.I, p.E, 128, FP8)) != MOE_OK) return s;
+  if ((s = map3d(&cR, w.wu, p.d, p.I, p.E, 128, FP8)) != MOE_OK) return s;
+  bS = bR;
+  cS = cR;
+  if (sh) {
+    if ((s = map2d(&bS, w.sg, p.d, p.I_s, p.d, 128, FP8)) != MOE_OK) return s;
+    if ((s = map2d(&cS, w.su, p.d, p.I_s, p.d, 128, FP8)) != MOE_OK) return s;
+  }
+  TcGemmArgs a{};
+  a.offs = offs;
+  a.prefix = pre_a;
+  a.E = p.E;
+  a.rows_cap = Rp;
+  a.single_rows = -1;
+  a.N_r = p.I;
+  a.N_s = p.I_s;
+  a.K_r = p.d;
+  a.K_s = p.d;
+  a.H = (bf16*)H;
+  a.ldh = ldh;
+  a.sc_b_r = sp[0];
+  a.sc_b_s = sp[3];
+  a.sc_c_r = sp[1];
+  a.sc_c_s = sp[4];
+  a.status = dev->status;
+  PROF_BEGIN("gemm_tc_swiglu", st);
+  k_gemm_swap<true, kTcSwiGLU, FP8><<<dev->sms, C1::THREADS, C1::SMEM_BYTES, st>>>(xR, xR, bR, bS, cR, cS, a);
+  LAUNCH_CHECK("gemm_tc_swiglu", st);
+  // down: W_down [E, d, I] is the M operand, H rows the N operand
+  if ((s = map2d(&xR, H, p.I, Rp, ldh, kNCH)) != MOE_OK) return s;
+  xS = xR;
+  if (sh && (s = map2d(&xS, H, p.I_s, Rp, ldh, kNCH)) != MOE_OK) return s;
+  if ((s = map3d(&bR, w.wd, p.I, p.d, p.E, 128, FP8)) != MOE_OK) return s;
+  bS = bR;
+  if (sh && (s = map2d(&bS, w.sd, p.I_s, p.d, p.I_s, 128, FP8)) != MOE_OK) return s;
+  TcGemmArgs b{};
+  b.offs = offs;
+  b.prefix = pre_b;
+  b.E = p.E;
+  b.rows_cap = Rp;
+  b.single_rows = -1;
+  b.N_r = p.d;
+  b.N_s = p.d;
+  b.K_r = p.I;
+  b.K_s = p.I_s;
+  b.sc_b_r = sp[2];
+  b.sc_b_s = sp[5];
+  b.status = dev->status;
+  if (o.ys) {
+    b.ys = (bf16*)o.ys;
+    b.ldy = p.d;
+    b.row_dst = o.row_dst;
+    b.row_w = o.row_w;
+    PROF_BEGIN("gemm_tc_down", st);
+    k_gemm_swap<false, kTcSlotStore, FP8><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(xR, xS, bR, bS, bR, bS, b);
+    LAUNCH_CHECK("gemm_tc_down", st);
+  } else {
+    b.out = (bf16*)o.out;
+    b.ldo = p.d;
+    PROF_BEGIN("gemm_tc_store", st);
+    k_gemm_swap<false, kTcStore, FP8><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(xR, xS, bR, bS, bR, bS, b);
+    LAUNCH_CHECK("gemm_tc_store", st);
+  }
+  return MOE_OK;
+}
+
+static moe_status expert_gemms(const moe_problem& p, int form, const void* xp, const int32_t* offs,
                                const ExpertWeights& w, int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o,
                                cudaStream_t st, DeviceInfo* dev) {
-  if (tc) return tc_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
+  if (form == kFormSwap) {
+    if (p.w_dtype == MOE_FP8_E4M3_B128) return swap_gemms_t<true>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
+    return swap_gemms_t<false>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
+  }
+  if (form == kFormRows) return tc_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
   if (p.act_dtype == MOE_F32) return simt_gemms<float, float>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
   if (p.w_dtype == MOE_BF16) return simt_gemms<bf16, bf16>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
   return simt_gemms<bf16, uint8_t>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
 }
 
-static void schedules(const moe_problem& p, bool tc, Schedule* sa, Schedule* sb) {
-  if (tc) {
+static void schedules(const moe_problem& p, int form, Schedule* sa, Schedule* sb) {
+  if (form == kFormRows) {
     *sa = sched_tc(128, p.I, p.I_s);
     *sb = sched_tc(256, p.d, p.d);
+  } else if (form == kFormSwap) {  // (token chunk, 128 weight rows) tiles
+    *sa = Schedule{kNCH, 128, p.I, p.I_s, 0};
+    *sb = Schedule{kNCH, 128, p.d, p.d, 0};
   } else {
     *sa = sched_simt(p.I, p.I_s);
     *sb = sched_simt(p.d, p.d);
@@ -632,7 +742,7 @@ size_t moe_workspace_size(const moe_problem* p) { return check(p) == MOE_OK ? la
 size_t moe_stage_workspace_size(const moe_problem* p) { return check(p) == MOE_OK ? layout(*p, false).total : 0; }
 
 moe_status moe_set_path(int path) {
-  if (path < 0 || path > 2) return fail(MOE_ERR_INVALID_ARG, "path %d is not 0, 1 or 2", path);
+  if (path < 0 || path > 3) return fail(MOE_ERR_INVALID_ARG, "path %d is not 0, 1, 2 or 3", path);
   g_path = path;
   return MOE_OK;
 }
@@ -759,22 +869,22 @@ moe_status moe_expert_ffn(const moe_problem* p, const void* x_perm, const int32_
   const Layout L = layout(*p, false);
   if (ws_bytes < L.total)
     return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
-  bool tc;
-  if ((s = choose(tc_shapes(*p), &tc)) != MOE_OK) return s;
+  int form;
+  if ((s = choose_form(*p, &form)) != MOE_OK) return s;
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != MOE_OK) return s;
   g_launches_pending = 0;
   cudaStream_t st = (cudaStream_t)stream;
   char* wsp = (char*)ws;
   Schedule sa, sb;
-  schedules(*p, tc, &sa, &sb);
+  schedules(*p, form, &sa, &sb);
   int32_t* pre_a = (int32_t*)(wsp + L.pre_a);
   int32_t* pre_b = (int32_t*)(wsp + L.pre_b);
   PROF_BEGIN("tile_prefix", st);
   k_tile_prefix<<<1, 1024, 0, st>>>(offs, p->E, sa, pre_a, sb, pre_b);
   LAUNCH_CHECK("tile_prefix", st);
   DownOut o{nullptr, nullptr, nullptr, y_perm};
-  s = expert_gemms(*p, tc, x_perm, offs, w, pre_a, pre_b, wsp + L.h, o, st, dev);
+  s = expert_gemms(*p, form, x_perm, offs, w, pre_a, pre_b, wsp + L.h, o, st, dev);
   if (s == MOE_OK) g_launches = g_launches_pending;
   return s;
 }
@@ -830,8 +940,8 @@ moe_status moe_layer_forward(const moe_problem* p, const void* x, const void* w_
   const Layout L = layout(*p, true);
   if (ws_bytes < L.total)
     return fail(MOE_ERR_WORKSPACE_TOO_SMALL, "workspace %zu bytes < %zu needed", ws_bytes, L.total);
-  bool tc;
-  if ((s = choose(tc_shapes(*p), &tc)) != MOE_OK) return s;
+  int form;
+  if ((s = choose_form(*p, &form)) != MOE_OK) return s;
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != MOE_OK) return s;
   g_launches_pending = 0;
@@ -852,12 +962,12 @@ moe_status moe_layer_forward(const moe_problem* p, const void* x, const void* w_
   s = launch_router(*p, x, w_router, router_bias, ids, tw, (float*)(wsp + L.part), counts, &counted, st, dev);
   if (s != MOE_OK) return s;
   Schedule sa, sb;
-  schedules(*p, tc, &sa, &sb);
+  schedules(*p, form, &sa, &sb);
   s = launch_dispatch(*p, ids, tw, counted, offs, row_tok, row_w, pos, row_dst, counts, sa, pre_a, sb, pre_b, st, dev);
   if (s != MOE_OK) return s;
   if ((s = launch_gather(*p, x, row_tok, offs, xp, st, dev)) != MOE_OK) return s;
   DownOut o{xp, row_dst, row_w, nullptr};  // the slot rows reuse the dispatched-row buffer
-  s = expert_gemms(*p, tc, xp, offs, w, pre_a, pre_b, wsp + L.h, o, st, dev);
+  s = expert_gemms(*p, form, xp, offs, w, pre_a, pre_b, wsp + L.h, o, st, dev);
   if (s != MOE_OK) return s;
   PROF_BEGIN("slot_sum", st);
   if (p->act_dtype == MOE_F32)

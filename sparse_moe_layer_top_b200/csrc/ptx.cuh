@@ -47,22 +47,25 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Every wait in the library is bounded: after kWaitLimitNs without progress
-// the waiter records `where` in the device status word, raises the CTA's
-// abort flag and returns false; any other waiter of the CTA that sees the
-// abort flag returns false at once.  Kernels then skip their remaining work,
-// drain what they issued and release TMEM before exiting.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+// Every wait in the library is bounded: after about kWaitLimitCycles SM
+// cycles without progress (about 2 s at B200 clocks; longer at lower clocks,
+// bounded all the same) the waiter records `where` in the device status word,
+// raises the CTA's abort flag and returns false; any other waiter of the CTA
+// that sees the abort flag returns false at once.  Kernels then skip their
+// remaining work, drain what they issued and release TMEM before exiting.
+// The bound is kept off the fast path: the cycle counter and the abort flag
+// are read once every 256 polls.
+constexpr long long kWaitLimitCycles = 4000000000ll;
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned* status, unsigned where) {
   if (mbar_try_wait(bar, parity)) return true;
-  uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 63u) == 0) {
+    if ((i & 255u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (clock64() - t0 > kWaitLimitCycles) {
         *abort_flag = 1;
         atomicCAS(status, 0u, where);
         return false;

@@ -126,9 +126,9 @@ __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
 
 // Wait (bounded, ignoring the abort flag) for a TMA copy already issued.
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
-  uint64_t t0 = globaltimer_ns();
+  const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity))
-    if (globaltimer_ns() - t0 > kWaitLimitNs) break;
+    if (clock64() - t0 > kWaitLimitCycles) break;
 }
 
 template <int BN, bool DUAL, int STAGES, bool FP8 = false>
@@ -168,6 +168,81 @@ __device__ __forceinline__ uint2 e4m3x4_scaled_bf16(uint32_t w, float sc) {
   return r;
 }
 
+// The two 128-row halves of a converter stage (gate and up rows, or the two
+// 128-row blocks of a 256-row weight tile) each read one row of 128 x 128
+// block scales along K.  cur[] holds the scales of the current 128-wide K
+// block, nxt[] the next one, loaded one block ahead.
+struct ScaleStreams {
+  const float* row[2];  // NULL: the half lies past the end of the weight matrix
+  int kb128;
+  float cur[2], nxt[2];
+  __device__ __forceinline__ void start(int kb0) {
+    const int j = kb0 / 2;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      cur[h] = row[h] ? __ldg(row[h] + j) : 0.f;
+      nxt[h] = (row[h] && j + 1 < kb128) ? __ldg(row[h] + j + 1) : 0.f;
+    }
+  }
+  // call before converting K-block kb (kb0 <= kb; K-blocks are 64 wide)
+  __device__ __forceinline__ void at(int kb, int kb0) {
+    if (kb > kb0 && (kb & 1) == 0) {
+      const int j = kb / 2;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        cur[h] = nxt[h];
+        nxt[h] = (row[h] && j + 1 < kb128) ? __ldg(row[h] + j + 1) : 0.f;
+      }
+    }
+  }
+};
+
+// One converter thread's share of a stage: NB raw E4M3 rows of 64 bytes at
+// `raw` become NB bf16 rows of 128 bytes at `dst`, 128-byte swizzled.  NB
+// threads take four passes; in each, four threads share a row (one 16-byte
+// chunk each), so a quarter warp reads 128 consecutive bytes.  Rows 0..127
+// use scale stream 0, rows 128..255 stream 1.
+template <int NB>
+__device__ __forceinline__ void convert_e4m3_rows(const uint8_t* raw, uint8_t* dst, int ct, const float (&cur)[2]) {
+  constexpr int RPP = NB / 4;  // rows per pass
+  const int sub = ct & 3, rbase = ct >> 2;
+  uint4 q[4];
+#pragma unroll
+  for (int ps = 0; ps < 4; ++ps) q[ps] = *reinterpret_cast<const uint4*>(raw + (rbase + RPP * ps) * kBK + sub * 16);
+#pragma unroll
+  for (int ps = 0; ps < 4; ++ps) {
+    const int r = rbase + RPP * ps;
+    const float sc = cur[r >= 128 ? 1 : 0];
+    const uint2 a = e4m3x4_scaled_bf16(q[ps].x, sc);
+    const uint2 b = e4m3x4_scaled_bf16(q[ps].y, sc);
+    const uint2 c = e4m3x4_scaled_bf16(q[ps].z, sc);
+    const uint2 d = e4m3x4_scaled_bf16(q[ps].w, sc);
+    uint8_t* o = dst + r * 128;
+    *reinterpret_cast<uint4*>(o + (((2 * sub) ^ (r & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
+    *reinterpret_cast<uint4*>(o + (((2 * sub + 1) ^ (r & 7)) << 4)) = make_uint4(c.x, c.y, d.x, d.y);
+  }
+}
+
+// Scale rows of a converter stage for weight rows n0 .. n0+NB-1 of group g.
+// dual: rows 0..127 gate (sb), 128..255 up (sc); else 1 or 2 row blocks of sb.
+__device__ __forceinline__ void scale_rows(ScaleStreams& ss, bool dual, bool sh, int g, int n0, int N, int K,
+                                           const float* sb_r, const float* sb_s, const float* sc_r,
+                                           const float* sc_s, int nrows) {
+  ss.kb128 = (K + 127) / 128;
+  const int nb128 = (N + 127) / 128;
+  const int64_t eoff = (int64_t)g * nb128 * ss.kb128;
+  const float* base_b = sh ? sb_s : sb_r + eoff;
+  if (dual) {
+    const bool in = n0 < N;
+    const float* base_c = sh ? sc_s : sc_r + eoff;
+    ss.row[0] = in ? base_b + (int64_t)(n0 / 128) * ss.kb128 : nullptr;
+    ss.row[1] = in ? base_c + (int64_t)(n0 / 128) * ss.kb128 : nullptr;
+  } else {
+    ss.row[0] = n0 < N ? base_b + (int64_t)(n0 / 128) * ss.kb128 : nullptr;
+    ss.row[1] = (nrows > 128 && n0 + 128 < N) ? base_b + (int64_t)(n0 / 128 + 1) * ss.kb128 : nullptr;
+  }
+}
+
 template <int BN, bool DUAL, int STAGES, int EPI, bool FP8 = false>
 __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
@@ -200,13 +275,13 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full + s, FP8 ? Cfg::NB : 1);  // FP8: the converters' arrivals
+      mbar_init(full + s, FP8 ? Cfg::NB / 32 : 1);  // FP8: one arrival per converter warp
       mbar_init(empty + s, 1);
       mbar_init(a_full + s, 1);
     }
     for (int s = 0; s < Cfg::RAW_STAGES; ++s) {
       mbar_init(raw_full + s, 1);
-      mbar_init(raw_empty + s, Cfg::NB);
+      mbar_init(raw_empty + s, Cfg::NB / 32);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull + b, 1);
@@ -464,80 +539,37 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
     }
   } else if (FP8 && warp < 6 + Cfg::NB / 32) {
     // ------------------------------------------------ E4M3 -> bf16 converters
-    // Four threads per 64-byte raw row (one 16-byte chunk each, so a quarter
-    // warp reads 128 consecutive bytes), four passes over the 256 rows.  Rows
-    // 0..127 and 128..255 each sit in one 128-row scale block, so a thread
-    // follows two scale streams, prefetched one 128-wide K block ahead.
     static_assert(!FP8 || Cfg::NB == 256, "converter mapping covers 256 rows");
     const int ct = threadIdx.x - 192;
-    const int sub = ct & 3, rbase = ct >> 2;  // chunk of the row, row within a pass
     int stage = 0, rstage = 0;
     uint32_t phase = 0, rphase = 0;
     bool stop = false;
     for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
       const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
       const bool sh = t.g == p.E;
-      const int kb128 = ((sh ? p.K_s : p.K_r) + 127) / 128, nb128 = (t.N + 127) / 128;
-      const int64_t eoff = (int64_t)t.g * nb128 * kb128;
-      // scale rows of the two halves (NULL where the half lies past N)
-      const float* srow[2];
-      if (DUAL) {
-        const int nb = t.n0 / 128;
-        const bool in = t.n0 < t.N;
-        srow[0] = in ? (sh ? p.sc_b_s : p.sc_b_r + eoff) + (int64_t)nb * kb128 : nullptr;
-        srow[1] = in ? (sh ? p.sc_c_s : p.sc_c_r + eoff) + (int64_t)nb * kb128 : nullptr;
-      } else {
-        const float* base = sh ? p.sc_b_s : p.sc_b_r + eoff;
-        srow[0] = t.n0 < t.N ? base + (int64_t)(t.n0 / 128) * kb128 : nullptr;
-        srow[1] = t.n0 + 128 < t.N ? base + (int64_t)(t.n0 / 128 + 1) * kb128 : nullptr;
-      }
-      float cur[2], nxt[2];
-      {
-        const int j = t.kb0 / 2;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          cur[h] = srow[h] ? __ldg(srow[h] + j) : 0.f;
-          nxt[h] = (srow[h] && j + 1 < kb128) ? __ldg(srow[h] + j + 1) : 0.f;
-        }
-      }
+      ScaleStreams ss;
+      scale_rows(ss, DUAL, sh, t.g, t.n0, t.N, sh ? p.K_s : p.K_r, p.sc_b_r, p.sc_b_s, p.sc_c_r, p.sc_c_s,
+                 Cfg::NB);
+      ss.start(t.kb0);
       for (int kb = t.kb0; kb < t.kb1; ++kb) {
-        if (kb > t.kb0 && (kb & 1) == 0) {  // a new 128-wide K block: rotate, prefetch the next
-          const int j = kb / 2;
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            cur[h] = nxt[h];
-            nxt[h] = (srow[h] && j + 1 < kb128) ? __ldg(srow[h] + j + 1) : 0.f;
-          }
-        }
-        if (!mbar_wait(raw_full + rstage, rphase, abort_flag, p.status, tcode | 5) ||
-            !mbar_wait(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 7)) {
+        ss.at(kb, t.kb0);
+        const bool ok = mbar_wait(raw_full + rstage, rphase, abort_flag, p.status, tcode | 5) &&
+                        mbar_wait(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 7);
+        if (!__all_sync(0xffffffffu, ok)) {  // the warp goes on, or stops, as one
           stop = true;
           break;
         }
-        const uint8_t* raw = raw_ring + rstage * Cfg::RAW_BYTES;
-        uint8_t* bst = smem + stage * Cfg::STAGE_BYTES + Cfg::A_BYTES;
-        uint4 q[4];
-#pragma unroll
-        for (int ps = 0; ps < 4; ++ps)
-          q[ps] = *reinterpret_cast<const uint4*>(raw + (rbase + 64 * ps) * kBK + sub * 16);
-#pragma unroll
-        for (int ps = 0; ps < 4; ++ps) {
-          const int r = rbase + 64 * ps;
-          const float sc = cur[ps >> 1];
-          const uint2 a = e4m3x4_scaled_bf16(q[ps].x, sc);
-          const uint2 b = e4m3x4_scaled_bf16(q[ps].y, sc);
-          const uint2 c = e4m3x4_scaled_bf16(q[ps].z, sc);
-          const uint2 d = e4m3x4_scaled_bf16(q[ps].w, sc);
-          uint8_t* dst = bst + r * 128;
-          *reinterpret_cast<uint4*>(dst + (((2 * sub) ^ (r & 7)) << 4)) = make_uint4(a.x, a.y, b.x, b.y);
-          *reinterpret_cast<uint4*>(dst + (((2 * sub + 1) ^ (r & 7)) << 4)) = make_uint4(c.x, c.y, d.x, d.y);
-        }
+        convert_e4m3_rows<Cfg::NB>(raw_ring + rstage * Cfg::RAW_BYTES,
+                                   smem + stage * Cfg::STAGE_BYTES + Cfg::A_BYTES, ct, ss.cur);
         // The raw slot goes back to the TMA only now: its bytes have been
         // consumed, and the proxy fence orders these generic-proxy reads before
         // the async-proxy write that will refill the slot.
         fence_proxy_async_smem();
-        mbar_arrive(full + stage);
-        mbar_arrive(raw_empty + rstage);
+        __syncwarp();  // the warp's writes and proxy fences, then one arrival per warp
+        if (lane == 0) {
+          mbar_arrive(full + stage);
+          mbar_arrive(raw_empty + rstage);
+        }
         if (++stage == STAGES) {
           stage = 0;
           phase ^= 1;

@@ -22,6 +22,13 @@ def moe():
     m.set_path(0)
 
 
+@pytest.fixture(autouse=True)
+def _automatic_path_after_each_test():
+    yield
+    import sparse_moe_layer_top_b200 as m
+    m.set_path(0)
+
+
 def _prob(moe, inp):
     return moe.Problem.make(inp.T, inp.d, inp.E, inp.k, inp.I, inp.I_s, inp.act, inp.w)
 
@@ -68,12 +75,15 @@ def _gpu_forward(moe, g):
     return y.float().cpu().numpy(), ids.cpu().numpy(), tw.cpu().numpy()
 
 
-@pytest.mark.parametrize("path", [0, 1])
+# 0 automatic, 1 SIMT kernels, 2 row-tiled tensor-core GEMMs, 3 weight-row tensor-core GEMMs
+@pytest.mark.parametrize("path", [0, 1, 2, 3])
 @pytest.mark.parametrize("case", list(FORWARD_CASES))
 def test_forward_matches_oracle(moe, case, path):
     inp = _make(case)
     if path == 1 and inp.act == "bf16" and inp.d * inp.I > 1 << 20:
         pytest.skip("SIMT path at this size is covered by the smaller cases")
+    if path >= 2 and inp.act == "f32":
+        pytest.skip("fp32 problems run on the SIMT kernels only")
     moe.set_path(path)
     g = to_device(inp, "cuda")
     y, ids, tw = _gpu_forward(moe, g)
@@ -146,7 +156,7 @@ def _random_dispatch(E, sizes, d, act, seed):
     return x_perm, offs, T, R
 
 
-@pytest.mark.parametrize("path", [0, 1])
+@pytest.mark.parametrize("path", [0, 1, 2, 3])
 @pytest.mark.parametrize("sizes_kind", ["ragged", "one_hot_expert", "empty_shared"])
 def test_expert_ffn_matches_oracle(moe, sizes_kind, path):
     E, d, I, I_s = 12, 256, 192, 128
@@ -203,29 +213,34 @@ def test_stages_chain_to_the_forward(moe):
     assert rel_l2(y_stage.float().cpu().numpy(), y_fused.float().cpu().numpy()) <= 1e-2
 
 
-def test_paths_agree_bf16(moe):
+@pytest.mark.parametrize("w", ["bf16", "fp8"])
+def test_paths_agree(moe, w):
+    # SIMT, row-tiled and weight-row GEMMs on one problem whose groups span
+    # one to several 64-row chunks (and a shared group of 200 rows)
+    inp = moe_inputs.make_inputs(200, 512, 24, 4, 256, 256, act="bf16", w=w, seed=2)
+    g = to_device(inp, "cuda")
+    out = []
+    for path in (1, 2, 3):
+        moe.set_path(path)
+        y, ids, tw = _gpu_forward(moe, g)
+        out.append((y, ids))
+    moe.set_path(0)
+    _no_device_errors(moe)
+    for y, ids in out[1:]:
+        assert np.array_equal(out[0][1], ids)
+        assert rel_l2(y, out[0][0]) <= 1e-2
+
+
+def test_paths_agree_35b_shape(moe):
     inp = _make("bf16_35b_shape_T256", seed=1)
     g = to_device(inp, "cuda")
     out = []
-    for path in (1, 2):
+    for path in (1, 2, 3):
         moe.set_path(path)
         y, ids, tw = _gpu_forward(moe, g)
-        out.append((y, ids))
+        out.append(y)
     moe.set_path(0)
-    assert rel_l2(out[1][0], out[0][0]) <= 1e-2
-
-
-def test_paths_agree_fp8(moe):
-    inp = moe_inputs.make_inputs(200, 512, 24, 4, 256, 256, act="bf16", w="fp8", seed=2)
-    g = to_device(inp, "cuda")
-    out = []
-    for path in (1, 2):
-        moe.set_path(path)
-        y, ids, tw = _gpu_forward(moe, g)
-        out.append((y, ids))
-    moe.set_path(0)
-    assert np.array_equal(out[0][1], out[1][1])
-    assert rel_l2(out[1][0], out[0][0]) <= 1e-2
+    assert rel_l2(out[1], out[0]) <= 1e-2 and rel_l2(out[2], out[0]) <= 1e-2
 
 
 def test_out_of_range_expert_id_sets_device_status(moe):
