@@ -1,0 +1,85 @@
+"""bench.py's host-side logic without a GPU: the multi-rank aggregation (two
+gloo ranks on CPU), the algorithmic work model, and the reference arm's JSON
+line on the tiny workload."""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank(rank, world, port, q):
+    import datetime
+    import torch.distributed as dist
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    ms, tokens = bench.aggregate(step_ms=1.5 + rank, tokens=100 * (rank + 1), world=world)
+    bench.barrier(world)
+    dist.destroy_process_group()
+    q.put((rank, ms, tokens))
+
+
+def test_aggregate_takes_the_slowest_rank_and_sums_tokens():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    got = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert got == [(0, 2.5, 300), (1, 2.5, 300)]
+
+
+def test_aggregate_alone_is_identity():
+    assert bench.aggregate(3.0, 7, 1) == (3.0, 7)
+
+
+def test_work_model_counts_active_experts_and_rows():
+    c = dict(d=2048, E=256, k=8, I=512, I_s=512, act="bf16", w="bf16")
+    counts = [128] * 255 + [0]
+    w = bench.work_model(c, counts, 4096 * 8 // 8)
+    assert w["active_experts"] == 255 and w["rows"] == 128 * 255
+    # gate+up weights of 255 experts and the shared expert, bf16
+    g1 = w["gemm_gate_up"]
+    weights = (255 * 2 * 2048 * 512 + 2 * 2048 * 512) * 2
+    assert g1["bytes"] >= weights
+    assert g1["flops"] == 4 * 2048 * (128 * 255 * 512 + 4096 * 512)
+    lw = w["layer"]
+    assert lw["flops"] == 2 * 4096 * 2048 * 256 + 6 * 2048 * (128 * 255 * 512 + 4096 * 512)
+
+
+def test_reference_arm_prints_one_json_line():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config",
+                          "tiny_fp32", "--steps", "3", "--warmup", "3"], capture_output=True, text=True,
+                         timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["unit"] == "tokens/s" and d["value"] > 0
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["e2e"]["h2d_bytes_per_step"] == 0
+    assert d["metric"] == bench.METRIC
+
+
+def test_warmup_below_three_is_refused():
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--warmup", "2"], capture_output=True,
+                         text=True, timeout=300, cwd=ROOT)
+    assert out.returncode != 0 and "warmup" in out.stderr
