@@ -402,8 +402,9 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
   return MOE_OK;
 }
 
-// Histogram (unless the router wrote it), scan and scatter: offs, row_tok,
-// row_w, pos, row_dst (may be NULL), the shared rows; optionally the tile prefixes.
+// Histogram (unless the router wrote it), then one kernel that scans it and
+// scatters: offs, row_tok, row_w, pos, row_dst (may be NULL), the shared rows,
+// and optionally the tile prefixes.
 static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, const float* tw, bool counted,
                                   int32_t* offs, int32_t* row_tok, float* row_w, int32_t* pos, int32_t* row_dst,
                                   int32_t* counts, Schedule sa, int32_t* pre_a, Schedule sb, int32_t* pre_b,
@@ -416,15 +417,10 @@ static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, cons
     k_count<<<nch, 256, 0, st>>>(ids, p.T, p.k, p.E, counts, dev->status);
     LAUNCH_CHECK("count", st);
   }
-  PROF_BEGIN("scan", st);
-  k_scan<<<1, 1024, 0, st>>>(counts, nch, p.E, p.T, p.I_s > 0, offs, sa, pre_a, sb, pre_b);
-  LAUNCH_CHECK("scan", st);
-  if (p.T > 0) {
-    PROF_BEGIN("scatter", st);
-    k_scatter<<<nch, kScatterWarps * 32, 0, st>>>(ids, tw, p.T, p.k, p.E, counts, offs, p.I_s > 0, row_tok, row_w,
-                                                  pos, row_dst);
-    LAUNCH_CHECK("scatter", st);
-  }
+  PROF_BEGIN("dispatch", st);
+  k_dispatch<<<nch, kScatterWarps * 32, 0, st>>>(ids, tw, p.T, p.k, p.E, counts, nch, p.I_s > 0, offs, sa, pre_a, sb,
+                                                 pre_b, row_tok, row_w, pos, row_dst);
+  LAUNCH_CHECK("dispatch", st);
   return MOE_OK;
 }
 

@@ -3,15 +3,16 @@
 // The token "is sent to" its k experts (Qwen3.6 explainer, router paragraph).
 // Here that is a stable counting sort by expert over chunks of kChunkTokens
 // tokens (chunk c = the pairs of tokens c*kChunkTokens ...):
-//   counts     per-chunk histogram over the E experts (written by k_topk, or
-//              by k_count when the routing comes from elsewhere);
-//   k_scan     per-expert exclusive scan over chunks, then over experts ->
-//              group offsets offs[E+2] and each chunk's first row per expert;
-//              also the tile prefix sums of the GEMM schedules;
-//   k_scatter  within a chunk, warps take consecutive token ranges; ranks come
-//              from warp match masks, so row order = (token, slot) order; the
-//              chunk's shared-expert rows are written too;
-//   k_gather   copies x rows into the dispatched buffer (16-byte vectors).
+//   counts      per-chunk histogram over the E experts (written by k_topk, or
+//               by k_count when the routing comes from elsewhere);
+//   k_dispatch  one block per chunk: column sums of the histograms give the
+//               group offsets offs[E+2] and the chunk's first row per expert
+//               (block 0 also writes the tile prefix sums of the GEMM
+//               schedules); within the chunk, warps take consecutive token
+//               ranges and rank equal experts by warp match masks, so row
+//               order = (token, slot) order; the chunk's shared-expert rows
+//               are written too;
+//   k_gather    copies x rows into the dispatched buffer (16-byte vectors).
 // Group E (the shared expert) is every token in order at rows offs[E] + t.
 #pragma once
 #include "common.cuh"
@@ -19,7 +20,7 @@
 
 namespace moe {
 
-constexpr int kScatterWarps = 8;   // warps of k_scatter (256 threads)
+constexpr int kScatterWarps = 8;   // warps of k_dispatch (256 threads)
 constexpr int kMaxE = 512;
 
 __global__ void __launch_bounds__(256) k_count(const int32_t* __restrict__ ids, int64_t T, int k, int E,
@@ -74,40 +75,6 @@ __device__ __forceinline__ void write_tile_prefix(const Schedule& s, int E, int 
   if (g == E) prefix[E + 1] = incl;
 }
 
-// One block of 1024 threads.  counts[c*E+e] (chunk histograms) becomes the
-// absolute first row of expert e's pairs in chunk c.
-__global__ void __launch_bounds__(1024) k_scan(int32_t* __restrict__ counts, int nchunks, int E, int64_t T,
-                                               int has_shared, int32_t* __restrict__ offs, Schedule sa,
-                                               int32_t* __restrict__ prefix_a, Schedule sb,
-                                               int32_t* __restrict__ prefix_b) {
-  __shared__ int sm_warp[32];
-  int e = threadIdx.x;
-  int total = 0;
-  if (e < E) {
-#pragma unroll 8
-    for (int c = 0; c < nchunks; ++c) total += counts[(int64_t)c * E + e];
-  }
-  int incl = block_incl_scan(e < E ? total : 0, sm_warp);
-  int start = incl - (e < E ? total : 0);
-  if (e < E) {
-    offs[e] = start;
-    int run = start;
-    for (int c = 0; c < nchunks; ++c) {
-      int v = counts[(int64_t)c * E + e];
-      counts[(int64_t)c * E + e] = run;
-      run += v;
-    }
-  }
-  // pairs with an invalid id were not counted: the routed rows stay contiguous
-  if (e == E) {
-    offs[E] = start;
-    offs[E + 1] = start + (has_shared ? (int)T : 0);
-  }
-  int rows = e < E ? total : (e == E ? (has_shared ? (int)T : 0) : 0);
-  if (prefix_a) write_tile_prefix(sa, E, rows, prefix_a, sm_warp);
-  if (prefix_b) write_tile_prefix(sb, E, rows, prefix_b, sm_warp);
-}
-
 // Tile prefixes from caller-supplied group offsets (the expert stage alone).
 __global__ void __launch_bounds__(1024) k_tile_prefix(const int32_t* __restrict__ offs, int E, Schedule sa,
                                                       int32_t* __restrict__ prefix_a, Schedule sb,
@@ -119,40 +86,120 @@ __global__ void __launch_bounds__(1024) k_tile_prefix(const int32_t* __restrict_
   if (prefix_b) write_tile_prefix(sb, E, rows, prefix_b, sm_warp);
 }
 
-// One block per chunk.  Writes, for every routed pair (t, j) with a valid id:
-// row r, row_tok[r] = t, row_w[r] = topk_w[t,j], pos[t*k+j] = r and (if
-// row_dst is given) row_dst[r] = t*(k+1) + j; invalid pairs get pos = -1.
-// With has_shared, also the chunk's shared-expert rows offs[E] + t.
-__global__ void __launch_bounds__(kScatterWarps * 32) k_scatter(
+// Inclusive scan over a block of 256 threads, each holding two consecutive
+// values (v0, v1) of a 512-entry sequence; returns the inclusive sums.
+__device__ __forceinline__ int2 block256_scan2(int v0, int v1, int* sm_warp) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  int v = v0 + v1;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += t;
+  }
+  if (lane == 31) sm_warp[w] = v;
+  __syncthreads();
+  int before = 0;
+  for (int i = 0; i < w; ++i) before += sm_warp[i];
+  __syncthreads();
+  const int incl1 = before + v;  // through v1
+  return make_int2(incl1 - v1, incl1);
+}
+
+// Scan and scatter in one kernel: block c (one chunk of kChunkTokens tokens)
+// sums the chunk histograms of every expert over all chunks and over the
+// chunks before its own, scans the totals into the group offsets, and then
+// places its own pairs in (token, slot) order.  Block 0 also writes offs and the
+// tile prefixes of the two GEMM schedules.  256 threads, E <= 512.
+__global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
     const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int64_t T, int k, int E,
-    const int32_t* __restrict__ base, const int32_t* __restrict__ offs, int has_shared,
-    int32_t* __restrict__ row_tok, float* __restrict__ row_w, int32_t* __restrict__ pos,
-    int32_t* __restrict__ row_dst) {
+    const int32_t* __restrict__ counts, int nchunks, int has_shared, int32_t* __restrict__ offs, Schedule sa,
+    int32_t* __restrict__ prefix_a, Schedule sb, int32_t* __restrict__ prefix_b, int32_t* __restrict__ row_tok,
+    float* __restrict__ row_w, int32_t* __restrict__ pos, int32_t* __restrict__ row_dst) {
   __shared__ int32_t wb[kScatterWarps][kMaxE];
+  __shared__ int32_t s_base[kMaxE];
+  __shared__ int sm_warp[32];
+  __shared__ int s_R, s_tot;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
+  // 1. per expert: total over all chunks, and over the chunks before this one
+  int tot[2] = {0, 0}, pre[2] = {0, 0};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int e = 2 * threadIdx.x + h;
+    if (e < E) {
+#pragma unroll 8
+      for (int cc = 0; cc < nchunks; ++cc) {
+        const int v = __ldg(counts + (int64_t)cc * E + e);
+        tot[h] += v;
+        pre[h] += cc < c ? v : 0;
+      }
+    }
+  }
+  // 2. group offsets
+  const int2 inc = block256_scan2(tot[0], tot[1], sm_warp);
+  const int start0 = inc.x - tot[0], start1 = inc.y - tot[1];
+  if (threadIdx.x == blockDim.x - 1) s_R = inc.y;  // routed rows = sum of all totals
+  if (2 * threadIdx.x < E) s_base[2 * threadIdx.x] = start0 + pre[0];
+  if (2 * threadIdx.x + 1 < E) s_base[2 * threadIdx.x + 1] = start1 + pre[1];
+  __syncthreads();
+  const int R = s_R;
+  if (c == 0) {
+    if (2 * threadIdx.x < E) offs[2 * threadIdx.x] = start0;
+    if (2 * threadIdx.x + 1 < E) offs[2 * threadIdx.x + 1] = start1;
+    if (threadIdx.x == 0) {
+      offs[E] = R;
+      offs[E + 1] = R + (has_shared ? (int)T : 0);
+    }
+    // tile prefixes over the E+1 groups (group E: the shared expert); with
+    // E == 512 the shared group is one past the 512 the block scans
+    for (int which = 0; which < 2; ++which) {
+      const Schedule& sc = which ? sb : sa;
+      int32_t* pf = which ? prefix_b : prefix_a;
+      if (!pf) continue;
+      int tl[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int g = 2 * threadIdx.x + h;
+        const int rows = g < E ? tot[h] : (has_shared ? (int)T : 0);
+        tl[h] = g <= E ? sched_tiles(sc, g, E, rows) : 0;
+      }
+      const int2 ti = block256_scan2(tl[0], tl[1], sm_warp);
+      if (2 * threadIdx.x <= E) pf[2 * threadIdx.x] = ti.x - tl[0];
+      if (2 * threadIdx.x + 1 <= E) pf[2 * threadIdx.x + 1] = ti.y - tl[1];
+      if (threadIdx.x == blockDim.x - 1) s_tot = ti.y;
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        if (E < kMaxE) {
+          pf[E + 1] = s_tot;
+        } else {
+          pf[E] = s_tot;
+          pf[E + 1] = s_tot + sched_tiles(sc, E, E, has_shared ? (int)T : 0);
+        }
+      }
+      __syncthreads();
+    }
+  }
+  // 3. the chunk's pairs: per-warp histograms, their scan, then ranks by match masks
   constexpr int kTokPerWarp = kChunkTokens / kScatterWarps;
   const int64_t n = T * k;
-  const int64_t s0 = ((int64_t)blockIdx.x * kChunkTokens + (int64_t)warp * kTokPerWarp) * k;
+  const int64_t s0 = ((int64_t)c * kChunkTokens + (int64_t)warp * kTokPerWarp) * k;
   const int64_t s1 = min(n, s0 + (int64_t)kTokPerWarp * k);
   for (int e = lane; e < E; e += 32) wb[warp][e] = 0;
   __syncwarp();
-  // pass 1: per-warp histogram of its pairs
   for (int64_t i = s0 + lane; i < s1; i += 32) {
-    int e = __ldg(ids + i);
+    const int e = __ldg(ids + i);
     if ((unsigned)e < (unsigned)E) atomicAdd(&wb[warp][e], 1);
   }
   __syncthreads();
-  // exclusive scan across the warps of the chunk, per expert
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = base[(int64_t)blockIdx.x * E + e];
+    int run = s_base[e];
     for (int w = 0; w < kScatterWarps; ++w) {
-      int v = wb[w][e];
+      const int v = wb[w][e];
       wb[w][e] = run;
       run += v;
     }
   }
   __syncthreads();
-  // pass 2: in order, 32 pairs at a time; equal experts rank by lane order
   const unsigned lt = (1u << lane) - 1u;
   for (int64_t b = s0; b < s1; b += 32) {
     const int64_t i = b + lane;
@@ -163,7 +210,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_scatter(
     int r = 0;
     if (ok) r = wb[warp][e] + __popc(peers & lt);
     __syncwarp();
-    if (ok && (peers & lt) == 0) wb[warp][e] += __popc(peers);  // lowest peer advances the cursor
+    if (ok && (peers & lt) == 0) wb[warp][e] += __popc(peers);
     __syncwarp();
     if (ok) {
       const int64_t t = i / k;
@@ -176,9 +223,8 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_scatter(
     }
   }
   if (has_shared) {
-    const int64_t R = __ldg(offs + E);
-    for (int64_t t = (int64_t)blockIdx.x * kChunkTokens + threadIdx.x;
-         t < min(T, (int64_t)(blockIdx.x + 1) * kChunkTokens); t += blockDim.x) {
+    for (int64_t t = (int64_t)c * kChunkTokens + threadIdx.x; t < min(T, (int64_t)(c + 1) * kChunkTokens);
+         t += blockDim.x) {
       row_tok[R + t] = (int32_t)t;
       row_w[R + t] = 1.0f;
       if (row_dst) row_dst[R + t] = (int32_t)(t * (k + 1) + k);

@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ part, in
 #pragma unroll
   for (int i = 0; i < 16; ++i) l[i] = (lane + 32 * i < E) ? (bias ? __ldg(bias + lane + 32 * i) : 0.f) : -INFINITY;
   const float* row = part + t * ldp;
-#pragma unroll 2
+#pragma unroll 4
   for (int s = 0; s < nsplit; ++s) {
 #pragma unroll
     for (int i = 0; i < 16; ++i)
