@@ -391,7 +391,7 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
   a.status = dev->status;
   PROF_BEGIN("gemm_tc_router", st);
   k_gemm_tc<kRouterBN, false, 4, kTcLogits>
-      <<<std::min(rs.tiles, dev->sms), 192, Gemm2Cfg::SMEM_BYTES, st>>>(ax, ax, bw, bw, bw, bw, a);
+      <<<std::min(rs.tiles, dev->sms), Gemm2Cfg::THREADS, Gemm2Cfg::SMEM_BYTES, st>>>(ax, ax, bw, bw, bw, bw, a);
   LAUNCH_CHECK("gemm_tc_router", st);
   if (counts) CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * p.E * 4, st));
   PROF_BEGIN("topk", st);

@@ -142,12 +142,17 @@ struct TcGemmCfg {
   static constexpr int RAW_STAGES = FP8 ? 6 : 0;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES + RAW_STAGES * RAW_BYTES;
   // FP8: + one converter thread per B row, + one warp issuing the A tiles
-  static constexpr int THREADS = FP8 ? 192 + NB + 32 : 192;
+  // epilogue warps: 4 (one per TMEM lane quarter) with E4M3 weights, else 8
+  // (two per quarter, splitting the accumulator columns) so stores drain faster
+  static constexpr int EPI_WARPS = FP8 ? 4 : 8;
+  static constexpr int THREADS = FP8 ? 192 + NB + 32 : 64 + 32 * EPI_WARPS;
   static constexpr int ACC_COLS = DUAL ? 2 * BN : BN;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
   static constexpr int BAR_BYTES = (3 * STAGES + 2 * RAW_STAGES + 5) * 8 + 16;
   static constexpr int SCHED_INTS = 2 * (512 + 2);  // tile prefix + group offsets, E <= 512
-  static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + SCHED_INTS * 4;
+  // epilogue staging: 32 rows x 64 bytes per epilogue warp
+  static constexpr int EPI_OFF = (RING_BYTES + BAR_BYTES + SCHED_INTS * 4 + 127) / 128 * 128;
+  static constexpr int SMEM_BYTES = 1024 + EPI_OFF + EPI_WARPS * 2048;
   static_assert(TMEM_COLS == 64 || TMEM_COLS == 128 || TMEM_COLS == 256 || TMEM_COLS == 512, "TMEM columns");
   static_assert(BN % 16 == 0 && BN >= 16 && (DUAL ? 2 * BN : BN) <= 256, "UMMA N for M=128");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
@@ -166,6 +171,32 @@ __device__ __forceinline__ uint2 e4m3x4_scaled_bf16(uint32_t w, float sc) {
   r.x = pack_bf16x2(a.x * sc, a.y * sc);
   r.y = pack_bf16x2(b.x * sc, b.y * sc);
   return r;
+}
+
+// Epilogue store of a 32-row x 32-column bf16 block held one row per lane
+// (w[16] = the row's 32 values as bf16 pairs) to rows rowp (per lane; NULL =
+// skip the row) at byte offset colb, of which the first ncols columns exist:
+// the block passes through the warp's 2 KB staging buffer (64 bytes per row,
+// 16-byte chunks XOR-swizzled so neither the row-wise writes nor the
+// column-wise reads conflict) and leaves as 8 rows x 64 contiguous bytes per
+// store instruction instead of 32 rows x 16 bytes.
+__device__ __forceinline__ void store_rows_staged(uint8_t* stg, const uint32_t (&w)[16], char* rowp, int64_t colb,
+                                                  int ncols, int lane) {
+  const int sw = (lane >> 1) & 3;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<uint4*>(stg + lane * 64 + ((j ^ sw) << 4)) =
+        make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  __syncwarp();
+#pragma unroll
+  for (int it = 0; it < 4; ++it) {
+    const int idx = it * 32 + lane;
+    const int rr = idx >> 2, cc = idx & 3;
+    char* rp = reinterpret_cast<char*>(__shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(rowp), rr));
+    const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 64 + ((cc ^ ((rr >> 1) & 3)) << 4));
+    if (rp && cc * 8 < ncols) *reinterpret_cast<uint4*>(rp + colb + cc * 16) = v;
+  }
+  __syncwarp();
 }
 
 // The two 128-row halves of a converter stage (gate and up rows, or the two
@@ -264,6 +295,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* s_pre = reinterpret_cast<int32_t*>(smem + Cfg::RING_BYTES + Cfg::BAR_BYTES);
   int32_t* s_offs = s_pre + 514;
+  uint8_t* epi_stage = smem + Cfg::EPI_OFF;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned tcode = kStatusTimeoutBase | (kKernGemmTc << 8);
@@ -285,7 +317,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull + b, 1);
-      mbar_init(tempty + b, 4);
+      mbar_init(tempty + b, Cfg::EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -420,8 +452,12 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
       drain_wait(drain, 0);
     }
     __syncwarp();
-  } else if (warp < 6) {
-    // ------------------------------------------------ epilogue (warps 2..5)
+  } else if (warp < 2 + Cfg::EPI_WARPS) {
+    // ------------------------------------------------ epilogue (warps 2 .. 2+EPI_WARPS-1)
+    // warp w reads TMEM lanes 32*(w%4) ..; with 8 warps the two warps of a lane
+    // quarter take the two halves of the tile's columns
+    constexpr int EG = Cfg::EPI_WARPS / 4;
+    const int eg = (warp - 2) / 4;
     const int q = warp & 3;
     const int row = q * 32 + lane;
     int acc = 0;
@@ -433,65 +469,46 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
       const uint32_t tb = tmem_base + acc * Cfg::ACC_COLS + ((uint32_t)(q * 32) << 16);
       const int64_t grow = t.row0 + row;
       const bool valid = t.m0 + row < t.rows && grow < p.rows_cap;
-      if (EPI == kTcSwiGLU) {
-        bf16* dst = p.H + grow * p.ldh;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t g[32], u[32];
-          tmem_ld32(tb + c * 32, g);
-          tmem_ld32(tb + BN + c * 32, u);
-          tmem_wait_regs(g);
-          tmem_wait_regs(u);
-          if (valid) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int n = t.n0 + c * 32 + v * 8;
-              if (n < t.N) {
-                uint4 o;
-                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                  const float g0 = __uint_as_float(g[v * 8 + 2 * e]), g1 = __uint_as_float(g[v * 8 + 2 * e + 1]);
-                  const float u0 = __uint_as_float(u[v * 8 + 2 * e]), u1 = __uint_as_float(u[v * 8 + 2 * e + 1]);
-                  ow[e] = pack_bf16x2(silu_f32(g0) * u0, silu_f32(g1) * u1);
-                }
-                *reinterpret_cast<uint4*>(dst + n) = o;
-              }
-            }
-          }
-        }
-      } else if (EPI == kTcSlotStore) {
-        int64_t dr = 0;
-        float w = 0.f;
+      if (EPI == kTcSwiGLU || EPI == kTcSlotStore || EPI == kTcStore) {
+        // destination row of this lane (NULL: nothing to write) and its scale
+        char* rowp = nullptr;
+        float w = 1.f;
         if (valid) {
-          dr = __ldg(p.row_dst + grow);
-          w = __ldg(p.row_w + grow);
-        }
-        bf16* dst = p.ys + dr * p.ldy;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t a[32];
-          tmem_ld32(tb + c * 32, a);
-          tmem_wait_regs(a);
-          if (valid && dr >= 0) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int n = t.n0 + c * 32 + v * 8;
-              if (n < t.N) {
-                uint4 o;
-                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  ow[e] = pack_bf16x2(w * __uint_as_float(a[v * 8 + 2 * e]), w * __uint_as_float(a[v * 8 + 2 * e + 1]));
-                *reinterpret_cast<uint4*>(dst + n) = o;
-              }
-            }
+          if (EPI == kTcSwiGLU) {
+            rowp = reinterpret_cast<char*>(p.H + grow * p.ldh);
+          } else if (EPI == kTcSlotStore) {
+            const int64_t dr = __ldg(p.row_dst + grow);
+            w = __ldg(p.row_w + grow);
+            if (dr >= 0) rowp = reinterpret_cast<char*>(p.ys + dr * p.ldy);
+          } else {
+            rowp = reinterpret_cast<char*>(p.out + grow * p.ldo);
           }
+        }
+        uint8_t* stg = epi_stage + (warp - 2) * 2048;
+        constexpr int CPW = (BN / 32) / EG;  // 32-column chunks per warp, contiguous
+#pragma unroll 1
+        for (int c = eg * CPW; c < (eg + 1) * CPW; ++c) {
+          uint32_t a[32], u[32];
+          tmem_ld32(tb + c * 32, a);
+          if (EPI == kTcSwiGLU) tmem_ld32(tb + BN + c * 32, u);
+          tmem_wait_regs(a);
+          if (EPI == kTcSwiGLU) tmem_wait_regs(u);
+          uint32_t o[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float x0 = __uint_as_float(a[2 * e]), x1 = __uint_as_float(a[2 * e + 1]);
+            if (EPI == kTcSwiGLU)
+              o[e] = pack_bf16x2(silu_f32(x0) * __uint_as_float(u[2 * e]), silu_f32(x1) * __uint_as_float(u[2 * e + 1]));
+            else
+              o[e] = pack_bf16x2(w * x0, w * x1);
+          }
+          const int n = t.n0 + c * 32;
+          store_rows_staged(stg, o, rowp, (int64_t)n * 2, t.N - n, lane);
         }
       } else if (EPI == kTcLogits) {
         float* dst = p.part + (int64_t)t.split * p.part_stride + grow * p.ldp;
 #pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
+        for (int c = eg; c < BN / 32; c += EG) {
           uint32_t a[32];
           tmem_ld32(tb + c * 32, a);
           tmem_wait_regs(a);
@@ -503,28 +520,6 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
                 *reinterpret_cast<float4*>(dst + n) =
                     make_float4(__uint_as_float(a[4 * v]), __uint_as_float(a[4 * v + 1]),
                                 __uint_as_float(a[4 * v + 2]), __uint_as_float(a[4 * v + 3]));
-            }
-          }
-        }
-      } else {
-        bf16* dst = p.out + grow * p.ldo;
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t a[32];
-          tmem_ld32(tb + c * 32, a);
-          tmem_wait_regs(a);
-          if (valid) {
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const int n = t.n0 + c * 32 + v * 8;
-              if (n < t.N) {
-                uint4 o;
-                uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                  ow[e] = pack_bf16x2(__uint_as_float(a[v * 8 + 2 * e]), __uint_as_float(a[v * 8 + 2 * e + 1]));
-                *reinterpret_cast<uint4*>(dst + n) = o;
-              }
             }
           }
         }

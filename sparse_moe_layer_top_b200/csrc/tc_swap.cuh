@@ -33,7 +33,8 @@ struct SwapCfg {
   static constexpr int STAGES = FP8 ? (DUAL ? 2 : 3) : (DUAL ? 5 : 8);
   static constexpr int RAW_STAGES = FP8 ? (DUAL ? 5 : 8) : 0;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES + RAW_STAGES * RAW_BYTES;
-  static constexpr int THREADS = FP8 ? 192 + NB : 192;
+  static constexpr int EPI_WARPS = FP8 ? 4 : 8;  // 8: two warps per TMEM lane quarter, one per token half
+  static constexpr int THREADS = FP8 ? 192 + NB : 64 + 32 * EPI_WARPS;
   static constexpr int ACC_COLS = (DUAL ? 2 : 1) * kNCH;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
   static constexpr int BAR_BYTES = (2 * STAGES + 2 * RAW_STAGES + 5) * 8 + 16;
@@ -111,7 +112,7 @@ __global__ void __launch_bounds__(SwapCfg<DUAL, FP8>::THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull + b, 1);
-      mbar_init(tempty + b, 4);
+      mbar_init(tempty + b, Cfg::EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -234,8 +235,10 @@ __global__ void __launch_bounds__(SwapCfg<DUAL, FP8>::THREADS, 1)
       drain_wait(drain, 0);
     }
     __syncwarp();
-  } else if (warp < 6) {
+  } else if (warp < 2 + Cfg::EPI_WARPS) {
     // ------------------------------------------------ epilogue: one thread per weight row
+    constexpr int EG = Cfg::EPI_WARPS / 4;
+    const int eg = (warp - 2) / 4;  // with 8 warps: which 32-token half this warp writes
     const int q = warp & 3;
     const int nl = q * 32 + lane;  // weight row within the tile = TMEM lane
     int acc = 0;
@@ -263,7 +266,7 @@ __global__ void __launch_bounds__(SwapCfg<DUAL, FP8>::THREADS, 1)
       const bool nvalid = n < t.N;
       const int jmax = min(kNCH, t.rows - t.c0);
 #pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
+      for (int half = eg; half < 2; half += EG) {
         uint32_t a[32], b[32];
         tmem_ld32(tb + half * 32, a);
         if (DUAL) tmem_ld32(tb + kNCH + half * 32, b);
