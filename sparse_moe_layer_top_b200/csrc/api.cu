@@ -17,6 +17,7 @@
 #include "simt.cuh"
 #include "tc_gemm.cuh"
 #include "tc_swap.cuh"
+#include "tc_swap8.cuh"
 
 using namespace moe;
 
@@ -143,9 +144,9 @@ static moe_status device_info(DeviceInfo** out) {
     CUDA_TRY(allow_smem(k_gemm_swap<true, kTcSwiGLU, false>, SwapCfg<true, false>::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_swap<false, kTcSlotStore, false>, SwapCfg<false, false>::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_swap<false, kTcStore, false>, SwapCfg<false, false>::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_swap<true, kTcSwiGLU, true>, SwapCfg<true, true>::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_swap<false, kTcSlotStore, true>, SwapCfg<false, true>::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_swap<false, kTcStore, true>, SwapCfg<false, true>::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap8<true, kTcSwiGLU>, Swap8Cfg<true>::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap8<false, kTcSlotStore>, Swap8Cfg<false>::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap8<false, kTcStore>, Swap8Cfg<false>::SMEM_BYTES));
     d.ready = true;
   }
   *out = &d;
@@ -173,20 +174,22 @@ static moe_status encode_fn(EncodeTiledFn* out) {
 }
 
 // Box {64 elements, box_rows} (x {1}); bf16 tiles are 128-byte swizzled for the
-// MMA, 1-byte E4M3 tiles are loaded plain for the converter warps.
+// MMA, 1-byte E4M3 tiles are loaded plain for the converter warps, or, `wide`,
+// as 128-code rows with 128-byte swizzling (the TMEM-operand kernels).
 // Out-of-range reads give zeros.
 static moe_status map_tile(CUtensorMap* m, const void* base, bool bytes, int rank, const uint64_t* dims,
-                           const uint64_t* strides_bytes, uint32_t box_rows) {
+                           const uint64_t* strides_bytes, uint32_t box_rows, bool wide = false) {
   EncodeTiledFn enc;
   moe_status s = encode_fn(&enc);
   if (s != MOE_OK) return s;
   cuuint64_t gd[3], gs[2];
-  cuuint32_t box[3] = {(cuuint32_t)kBK, box_rows, 1}, es[3] = {1, 1, 1};
+  const bool swz = !bytes || wide;
+  cuuint32_t box[3] = {(cuuint32_t)(wide ? kBK8 : kBK), box_rows, 1}, es[3] = {1, 1, 1};
   for (int i = 0; i < rank; ++i) gd[i] = dims[i] ? dims[i] : 1;
   for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
   CUresult r = enc(m, bytes ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank,
                    const_cast<void*>(base), gd, gs, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   bytes ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+                   swz ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(MOE_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) rank %d dims %llu x %llu", (int)r, rank,
@@ -194,16 +197,16 @@ static moe_status map_tile(CUtensorMap* m, const void* base, bool bytes, int ran
   return MOE_OK;
 }
 static moe_status map2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer, uint64_t stride_elems,
-                        uint32_t box_rows, bool bytes = false) {
+                        uint32_t box_rows, bool bytes = false, bool wide = false) {
   const uint64_t eb = bytes ? 1 : 2;
   uint64_t dims[2] = {inner, outer}, st[1] = {stride_elems * eb};
-  return map_tile(m, base, bytes, 2, dims, st, box_rows);
+  return map_tile(m, base, bytes, 2, dims, st, box_rows, wide);
 }
 static moe_status map3d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t outer,
-                        uint32_t box_rows, bool bytes = false) {
+                        uint32_t box_rows, bool bytes = false, bool wide = false) {
   const uint64_t eb = bytes ? 1 : 2;
   uint64_t dims[3] = {inner, mid, outer}, st[2] = {inner * eb, inner * mid * eb};
-  return map_tile(m, base, bytes, 3, dims, st, box_rows);
+  return map_tile(m, base, bytes, 3, dims, st, box_rows, wide);
 }
 
 // ============================================================== checks
@@ -614,8 +617,8 @@ template <bool FP8>
 static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
                                int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
                                DeviceInfo* dev) {
-  using C1 = SwapCfg<true, FP8>;
-  using C2 = SwapCfg<false, FP8>;
+  using C1 = SwapCfg<true, false>;
+  using C2 = SwapCfg<false, false>;
   const int64_t Rp = rows_total(p), ldh = ldh_of(p);
   const bool sh = p.I_s > 0;
   const float* sp[6];
@@ -624,13 +627,13 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
   CUtensorMap xR, xS, bR, bS, cR, cS;
   // gate/up + SwiGLU: weights [E, I, d] are the M operand, token rows the N operand
   if ((s = map2d(&xR, xp, p.d, Rp, p.d, kNCH)) != MOE_OK) return s;
-  if ((s = map3d(&bR, w.wg, p.d, p.I, p.E, 128, FP8)) != MOE_OK) return s;
-  if ((s = map3d(&cR, w.wu, p.d, p.I, p.E, 128, FP8)) != MOE_OK) return s;
+  if ((s = map3d(&bR, w.wg, p.d, p.I, p.E, 128, FP8, FP8)) != MOE_OK) return s;
+  if ((s = map3d(&cR, w.wu, p.d, p.I, p.E, 128, FP8, FP8)) != MOE_OK) return s;
   bS = bR;
   cS = cR;
   if (sh) {
-    if ((s = map2d(&bS, w.sg, p.d, p.I_s, p.d, 128, FP8)) != MOE_OK) return s;
-    if ((s = map2d(&cS, w.su, p.d, p.I_s, p.d, 128, FP8)) != MOE_OK) return s;
+    if ((s = map2d(&bS, w.sg, p.d, p.I_s, p.d, 128, FP8, FP8)) != MOE_OK) return s;
+    if ((s = map2d(&cS, w.su, p.d, p.I_s, p.d, 128, FP8, FP8)) != MOE_OK) return s;
   }
   TcGemmArgs a{};
   a.offs = offs;
@@ -650,15 +653,19 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
   a.sc_c_s = sp[4];
   a.status = dev->status;
   PROF_BEGIN("gemm_tc_swiglu", st);
-  k_gemm_swap<true, kTcSwiGLU, FP8><<<dev->sms, C1::THREADS, C1::SMEM_BYTES, st>>>(xR, xR, bR, bS, cR, cS, a);
+  if (FP8)
+    k_gemm_swap8<true, kTcSwiGLU><<<dev->sms, Swap8Cfg<true>::THREADS, Swap8Cfg<true>::SMEM_BYTES, st>>>(
+        xR, xR, bR, bS, cR, cS, a);
+  else
+    k_gemm_swap<true, kTcSwiGLU, false><<<dev->sms, C1::THREADS, C1::SMEM_BYTES, st>>>(xR, xR, bR, bS, cR, cS, a);
   LAUNCH_CHECK("gemm_tc_swiglu", st);
   // down: W_down [E, d, I] is the M operand, H rows the N operand
   if ((s = map2d(&xR, H, p.I, Rp, ldh, kNCH)) != MOE_OK) return s;
   xS = xR;
   if (sh && (s = map2d(&xS, H, p.I_s, Rp, ldh, kNCH)) != MOE_OK) return s;
-  if ((s = map3d(&bR, w.wd, p.I, p.d, p.E, 128, FP8)) != MOE_OK) return s;
+  if ((s = map3d(&bR, w.wd, p.I, p.d, p.E, 128, FP8, FP8)) != MOE_OK) return s;
   bS = bR;
-  if (sh && (s = map2d(&bS, w.sd, p.I_s, p.d, p.I_s, 128, FP8)) != MOE_OK) return s;
+  if (sh && (s = map2d(&bS, w.sd, p.I_s, p.d, p.I_s, 128, FP8, FP8)) != MOE_OK) return s;
   TcGemmArgs b{};
   b.offs = offs;
   b.prefix = pre_b;
@@ -678,13 +685,22 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
     PROF_BEGIN("gemm_tc_down", st);
-    k_gemm_swap<false, kTcSlotStore, FP8><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(xR, xS, bR, bS, bR, bS, b);
+    if (FP8)
+      k_gemm_swap8<false, kTcSlotStore><<<dev->sms, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st>>>(
+          xR, xS, bR, bS, bR, bS, b);
+    else
+      k_gemm_swap<false, kTcSlotStore, false><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(xR, xS, bR, bS, bR,
+                                                                                            bS, b);
     LAUNCH_CHECK("gemm_tc_down", st);
   } else {
     b.out = (bf16*)o.out;
     b.ldo = p.d;
     PROF_BEGIN("gemm_tc_store", st);
-    k_gemm_swap<false, kTcStore, FP8><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(xR, xS, bR, bS, bR, bS, b);
+    if (FP8)
+      k_gemm_swap8<false, kTcStore><<<dev->sms, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st>>>(
+          xR, xS, bR, bS, bR, bS, b);
+    else
+      k_gemm_swap<false, kTcStore, false><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(xR, xS, bR, bS, bR, bS, b);
     LAUNCH_CHECK("gemm_tc_store", st);
   }
   return MOE_OK;

@@ -71,6 +71,76 @@ __device__ __forceinline__ SwapTile decode_swap(const TcGemmArgs& p, const int32
   return t;
 }
 
+// Epilogue of a weight-row GEMM, run by EPI_WARPS warps numbered from 2: one
+// thread per weight row (= TMEM lane, output feature), walking the kNCH token
+// columns of each finished tile; with 8 warps two warps share a lane quarter
+// and take one 32-token half each.
+template <bool DUAL, int EPI, int EPI_WARPS>
+__device__ __forceinline__ void swap_epilogue(const TcGemmArgs& p, const int32_t* s_pre, const int32_t* s_offs,
+                                              int total, uint32_t tmem_base, uint64_t* tfull, uint64_t* tempty,
+                                              volatile int* abort_flag, unsigned tcode, int warp, int lane) {
+  constexpr int ACC_COLS = (DUAL ? 2 : 1) * kNCH;
+  constexpr int EG = EPI_WARPS / 4;
+  const int eg = (warp - 2) / 4;  // with 8 warps: which 32-token half this warp writes
+  const int q = warp & 3;
+  const int nl = q * 32 + lane;  // weight row within the tile = TMEM lane
+  int acc = 0;
+  uint32_t acc_phase = 0;
+  for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    const SwapTile t = decode_swap(p, s_pre, s_offs, tile);
+    // per-column data of the chunk: lane j holds token columns j and j + 32
+    int64_t dst_lo = -1, dst_hi = -1;
+    float w_lo = 0.f, w_hi = 0.f;
+    if (EPI == kTcSlotStore) {
+      const int64_t ra = t.row0 + lane, rb = t.row0 + 32 + lane;
+      if (t.c0 + lane < t.rows && ra < p.rows_cap) {
+        dst_lo = __ldg(p.row_dst + ra);
+        w_lo = __ldg(p.row_w + ra);
+      }
+      if (t.c0 + 32 + lane < t.rows && rb < p.rows_cap) {
+        dst_hi = __ldg(p.row_dst + rb);
+        w_hi = __ldg(p.row_w + rb);
+      }
+    }
+    if (!mbar_wait(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)) break;
+    tc_fence_after();
+    const uint32_t tb = tmem_base + acc * ACC_COLS + ((uint32_t)(q * 32) << 16);
+    const int n = t.n0 + nl;
+    const bool nvalid = n < t.N;
+    const int jmax = min(kNCH, t.rows - t.c0);
+#pragma unroll 1
+    for (int half = eg; half < 2; half += EG) {
+      uint32_t a[32], b[32];
+      tmem_ld32(tb + half * 32, a);
+      if (DUAL) tmem_ld32(tb + kNCH + half * 32, b);
+      tmem_wait_regs(a);
+      if (DUAL) tmem_wait_regs(b);
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int jj = half * 32 + j;
+        const int64_t row = t.row0 + jj;
+        if (EPI == kTcSwiGLU) {
+          if (nvalid && jj < jmax && row < p.rows_cap)
+            p.H[row * p.ldh + n] = __float2bfloat16_rn(silu_f32(__uint_as_float(a[j])) * __uint_as_float(b[j]));
+        } else if (EPI == kTcSlotStore) {
+          const int64_t dr = __shfl_sync(0xffffffffu, half ? dst_hi : dst_lo, j);
+          const float w = __shfl_sync(0xffffffffu, half ? w_hi : w_lo, j);
+          if (nvalid && jj < jmax && dr >= 0) p.ys[dr * p.ldy + n] = __float2bfloat16_rn(w * __uint_as_float(a[j]));
+        } else {
+          if (nvalid && jj < jmax && row < p.rows_cap) p.out[row * p.ldo + n] = __float2bfloat16_rn(__uint_as_float(a[j]));
+        }
+      }
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(tempty + acc);
+    if (++acc == 2) {
+      acc = 0;
+      acc_phase ^= 1;
+    }
+  }
+}
+
 // tmW*: weight maps (box 64 x 128 rows; gate / the single operand = B, up = C);
 // tmX*: token-row maps (box 64 x kNCH); _r routed groups, _s the shared group.
 template <bool DUAL, int EPI, bool FP8>
@@ -236,66 +306,8 @@ __global__ void __launch_bounds__(SwapCfg<DUAL, FP8>::THREADS, 1)
     }
     __syncwarp();
   } else if (warp < 2 + Cfg::EPI_WARPS) {
-    // ------------------------------------------------ epilogue: one thread per weight row
-    constexpr int EG = Cfg::EPI_WARPS / 4;
-    const int eg = (warp - 2) / 4;  // with 8 warps: which 32-token half this warp writes
-    const int q = warp & 3;
-    const int nl = q * 32 + lane;  // weight row within the tile = TMEM lane
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-      const SwapTile t = decode_swap(p, s_pre, s_offs, tile);
-      // per-column data of the chunk: lane j holds token columns j and j + 32
-      int64_t dst_lo = -1, dst_hi = -1;
-      float w_lo = 0.f, w_hi = 0.f;
-      if (EPI == kTcSlotStore) {
-        const int64_t ra = t.row0 + lane, rb = t.row0 + 32 + lane;
-        if (t.c0 + lane < t.rows && ra < p.rows_cap) {
-          dst_lo = __ldg(p.row_dst + ra);
-          w_lo = __ldg(p.row_w + ra);
-        }
-        if (t.c0 + 32 + lane < t.rows && rb < p.rows_cap) {
-          dst_hi = __ldg(p.row_dst + rb);
-          w_hi = __ldg(p.row_w + rb);
-        }
-      }
-      if (!mbar_wait(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)) break;
-      tc_fence_after();
-      const uint32_t tb = tmem_base + acc * Cfg::ACC_COLS + ((uint32_t)(q * 32) << 16);
-      const int n = t.n0 + nl;
-      const bool nvalid = n < t.N;
-      const int jmax = min(kNCH, t.rows - t.c0);
-#pragma unroll 1
-      for (int half = eg; half < 2; half += EG) {
-        uint32_t a[32], b[32];
-        tmem_ld32(tb + half * 32, a);
-        if (DUAL) tmem_ld32(tb + kNCH + half * 32, b);
-        tmem_wait_regs(a);
-        if (DUAL) tmem_wait_regs(b);
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int jj = half * 32 + j;
-          const int64_t row = t.row0 + jj;
-          if (EPI == kTcSwiGLU) {
-            if (nvalid && jj < jmax && row < p.rows_cap)
-              p.H[row * p.ldh + n] = __float2bfloat16_rn(silu_f32(__uint_as_float(a[j])) * __uint_as_float(b[j]));
-          } else if (EPI == kTcSlotStore) {
-            const int64_t dr = __shfl_sync(0xffffffffu, half ? dst_hi : dst_lo, j);
-            const float w = __shfl_sync(0xffffffffu, half ? w_hi : w_lo, j);
-            if (nvalid && jj < jmax && dr >= 0) p.ys[dr * p.ldy + n] = __float2bfloat16_rn(w * __uint_as_float(a[j]));
-          } else {
-            if (nvalid && jj < jmax && row < p.rows_cap) p.out[row * p.ldo + n] = __float2bfloat16_rn(__uint_as_float(a[j]));
-          }
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(tempty + acc);
-      if (++acc == 2) {
-        acc = 0;
-        acc_phase ^= 1;
-      }
-    }
+    swap_epilogue<DUAL, EPI, Cfg::EPI_WARPS>(p, s_pre, s_offs, total, tmem_base, tfull, tempty, abort_flag, tcode,
+                                            warp, lane);
   } else if (FP8) {
     // ------------------------------------------------ E4M3 -> bf16 converters
     const int ct = threadIdx.x - 192;

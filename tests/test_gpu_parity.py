@@ -184,6 +184,30 @@ def test_expert_ffn_matches_oracle(moe, sizes_kind, path):
             assert rel_l2(got[o[gi]:o[gi + 1]], ref[o[gi]:o[gi + 1]]) <= TOL["bf16"], "group %d" % gi
 
 
+@pytest.mark.parametrize("path", [0, 1, 2, 3])
+def test_expert_ffn_fp8_matches_oracle(moe, path):
+    """E4M3 weights with 128 x 128 block scales through the expert stage alone:
+    groups of 0, 1, 63, 64, 65 and 130 rows (token chunks of 64 split inside a
+    group), a shared group, d and I spanning several 128-wide scale blocks."""
+    E, d, I, I_s = 6, 384, 256, 128
+    sizes = [63, 0, 130, 1, 65, 64] + [97]
+    inp = moe_inputs.make_inputs(1, d, E, 1, I, I_s, act="bf16", w="fp8", seed=9)
+    x_perm, offs, T, R = _random_dispatch(E, sizes, d, "bf16", 13)
+    moe.set_path(path)
+    prob = moe.Problem.make(T, d, E, 1, I, I_s, "bf16", "fp8")
+    yp = moe.expert_ffn(prob, x_perm.cuda(), offs.cuda(), inp.wg.cuda(), inp.wu.cuda(), inp.wd.cuda(),
+                        inp.s_wg.cuda(), inp.s_wu.cuda(), inp.s_wd.cuda(), inp.scales.cuda())
+    torch.cuda.synchronize()
+    _no_device_errors(moe)
+    ref = oracle.expert_ffn(x_perm[:R], offs.numpy(), inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu, inp.s_wd,
+                            inp.scales)
+    got = yp[:R].float().cpu().numpy()
+    o = offs.numpy()
+    for gi in range(E + 1):
+        if o[gi + 1] > o[gi]:
+            assert rel_l2(got[o[gi]:o[gi + 1]], ref[o[gi]:o[gi + 1]]) <= TOL["fp8"], "group %d" % gi
+
+
 @pytest.mark.parametrize("act", ["f32", "bf16"])
 def test_combine_matches_oracle(moe, act):
     T, E, k, d = 93, 10, 3, 136
