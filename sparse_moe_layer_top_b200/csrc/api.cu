@@ -141,9 +141,9 @@ static moe_status device_info(DeviceInfo** out) {
     CUDA_TRY(allow_smem(k_gemm_tc<128, true, kFp8Stages, kTcSwiGLU, true>, Gemm1F8Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, kFp8Stages, kTcSlotStore, true>, Gemm2F8Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, kFp8Stages, kTcStore, true>, Gemm2F8Cfg::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_swap<true, kTcSwiGLU, false>, SwapCfg<true, false>::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_swap<false, kTcSlotStore, false>, SwapCfg<false, false>::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_swap<false, kTcStore, false>, SwapCfg<false, false>::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap<true, kTcSwiGLU>, SwapCfg<true>::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap<false, kTcSlotStore>, SwapCfg<false>::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap<false, kTcStore>, SwapCfg<false>::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_swap8<true, kTcSwiGLU>, Swap8Cfg<true>::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_swap8<false, kTcSlotStore>, Swap8Cfg<false>::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_swap8<false, kTcStore>, Swap8Cfg<false>::SMEM_BYTES));
@@ -617,8 +617,8 @@ template <bool FP8>
 static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
                                int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
                                DeviceInfo* dev) {
-  using C1 = SwapCfg<true, false>;
-  using C2 = SwapCfg<false, false>;
+  using C1 = SwapCfg<true>;
+  using C2 = SwapCfg<false>;
   const int64_t Rp = rows_total(p), ldh = ldh_of(p);
   const bool sh = p.I_s > 0;
   const float* sp[6];
@@ -657,7 +657,7 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
     k_gemm_swap8<true, kTcSwiGLU><<<dev->sms, Swap8Cfg<true>::THREADS, Swap8Cfg<true>::SMEM_BYTES, st>>>(
         xR, xR, bR, bS, cR, cS, a);
   else
-    k_gemm_swap<true, kTcSwiGLU, false><<<dev->sms, C1::THREADS, C1::SMEM_BYTES, st>>>(xR, xR, bR, bS, cR, cS, a);
+    k_gemm_swap<true, kTcSwiGLU><<<dev->sms, C1::THREADS, C1::SMEM_BYTES, st>>>(xR, xR, bR, bS, cR, cS, a);
   LAUNCH_CHECK("gemm_tc_swiglu", st);
   // down: W_down [E, d, I] is the M operand, H rows the N operand
   if ((s = map2d(&xR, H, p.I, Rp, ldh, kNCH)) != MOE_OK) return s;
@@ -689,7 +689,7 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
       k_gemm_swap8<false, kTcSlotStore><<<dev->sms, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st>>>(
           xR, xS, bR, bS, bR, bS, b);
     else
-      k_gemm_swap<false, kTcSlotStore, false><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(xR, xS, bR, bS, bR,
+      k_gemm_swap<false, kTcSlotStore><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(xR, xS, bR, bS, bR,
                                                                                             bS, b);
     LAUNCH_CHECK("gemm_tc_down", st);
   } else {
@@ -700,7 +700,7 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
       k_gemm_swap8<false, kTcStore><<<dev->sms, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st>>>(
           xR, xS, bR, bS, bR, bS, b);
     else
-      k_gemm_swap<false, kTcStore, false><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(xR, xS, bR, bS, bR, bS, b);
+      k_gemm_swap<false, kTcStore><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(xR, xS, bR, bS, bR, bS, b);
     LAUNCH_CHECK("gemm_tc_store", st);
   }
   return MOE_OK;

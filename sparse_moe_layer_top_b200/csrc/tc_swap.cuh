@@ -13,9 +13,9 @@
 //
 // Warp roles: warp 0 TMA producer; warp 1 TMEM owner + MMA issuer (dual:
 // gate and up accumulators side by side, two MMAs sharing the token tile);
-// warps 2..5 epilogue, one thread per weight row (output feature) walking the
-// token columns; FP8: warps 6.. convert E4M3 weight tiles to bf16 (the token
-// tile rides in the raw slot with the weights and is read by the MMA there).
+// warps 2..9 epilogue, one thread per weight row (output feature) walking the
+// token columns.  E4M3 weights take the kernel of tc_swap8.cuh, which shares
+// the tile list and the epilogue defined here.
 #pragma once
 #include "tc_gemm.cuh"
 
@@ -23,21 +23,19 @@ namespace moe {
 
 constexpr int kNCH = 64;  // token rows per tile: the MMA's N
 
-template <bool DUAL, bool FP8>
+template <bool DUAL>
 struct SwapCfg {
   static constexpr int NB = DUAL ? 256 : 128;  // weight rows per stage (gate then up, or one tile)
   static constexpr int W_BYTES = NB * 128;      // bf16 weight rows of 128 bytes
   static constexpr int X_BYTES = kNCH * 128;    // token rows of 128 bytes
-  static constexpr int STAGE_BYTES = FP8 ? W_BYTES : W_BYTES + X_BYTES;
-  static constexpr int RAW_BYTES = FP8 ? NB * kBK + X_BYTES : 0;  // raw E4M3 weights + token tile
-  static constexpr int STAGES = FP8 ? (DUAL ? 2 : 3) : (DUAL ? 5 : 8);
-  static constexpr int RAW_STAGES = FP8 ? (DUAL ? 5 : 8) : 0;
-  static constexpr int RING_BYTES = STAGES * STAGE_BYTES + RAW_STAGES * RAW_BYTES;
-  static constexpr int EPI_WARPS = FP8 ? 4 : 8;  // 8: two warps per TMEM lane quarter, one per token half
-  static constexpr int THREADS = FP8 ? 192 + NB : 64 + 32 * EPI_WARPS;
+  static constexpr int STAGE_BYTES = W_BYTES + X_BYTES;
+  static constexpr int STAGES = DUAL ? 5 : 8;
+  static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
+  static constexpr int EPI_WARPS = 8;  // two warps per TMEM lane quarter, one per token half
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int ACC_COLS = (DUAL ? 2 : 1) * kNCH;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
-  static constexpr int BAR_BYTES = (2 * STAGES + 2 * RAW_STAGES + 5) * 8 + 16;
+  static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8 + 16;
   static constexpr int SCHED_INTS = 2 * (512 + 2);
   static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + SCHED_INTS * 4;
   static_assert(TMEM_COLS == 128 || TMEM_COLS == 256, "TMEM columns");
@@ -75,7 +73,7 @@ __device__ __forceinline__ SwapTile decode_swap(const TcGemmArgs& p, const int32
 // thread per weight row (= TMEM lane, output feature), walking the kNCH token
 // columns of each finished tile; with 8 warps two warps share a lane quarter
 // and take one 32-token half each.
-template <bool DUAL, int EPI, int EPI_WARPS>
+template <bool DUAL, int EPI, int EPI_WARPS, int ACC_BUFS = 2>
 __device__ __forceinline__ void swap_epilogue(const TcGemmArgs& p, const int32_t* s_pre, const int32_t* s_offs,
                                               int total, uint32_t tmem_base, uint64_t* tfull, uint64_t* tempty,
                                               volatile int* abort_flag, unsigned tcode, int warp, int lane) {
@@ -109,7 +107,7 @@ __device__ __forceinline__ void swap_epilogue(const TcGemmArgs& p, const int32_t
     const bool nvalid = n < t.N;
     const int jmax = min(kNCH, t.rows - t.c0);
 #pragma unroll 1
-    for (int half = eg; half < 2; half += EG) {
+    for (int half = eg; half < 2 && half * 32 < jmax; half += EG) {  // (jmax is uniform per tile)
       uint32_t a[32], b[32];
       tmem_ld32(tb + half * 32, a);
       if (DUAL) tmem_ld32(tb + kNCH + half * 32, b);
@@ -134,7 +132,7 @@ __device__ __forceinline__ void swap_epilogue(const TcGemmArgs& p, const int32_t
     tc_fence_before();
     __syncwarp();
     if (lane == 0) mbar_arrive(tempty + acc);
-    if (++acc == 2) {
+    if (++acc == ACC_BUFS) {
       acc = 0;
       acc_phase ^= 1;
     }
@@ -143,24 +141,21 @@ __device__ __forceinline__ void swap_epilogue(const TcGemmArgs& p, const int32_t
 
 // tmW*: weight maps (box 64 x 128 rows; gate / the single operand = B, up = C);
 // tmX*: token-row maps (box 64 x kNCH); _r routed groups, _s the shared group.
-template <bool DUAL, int EPI, bool FP8>
-__global__ void __launch_bounds__(SwapCfg<DUAL, FP8>::THREADS, 1)
+template <bool DUAL, int EPI>
+__global__ void __launch_bounds__(SwapCfg<DUAL>::THREADS, 1)
     k_gemm_swap(const __grid_constant__ CUtensorMap tmX_r, const __grid_constant__ CUtensorMap tmX_s,
                 const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
                 const __grid_constant__ CUtensorMap tmC_r, const __grid_constant__ CUtensorMap tmC_s, TcGemmArgs p) {
-  using Cfg = SwapCfg<DUAL, FP8>;
-  constexpr int S = Cfg::STAGES, R = Cfg::RAW_STAGES;
+  using Cfg = SwapCfg<DUAL>;
+  constexpr int S = Cfg::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
-  uint8_t* raw_ring = smem + S * Cfg::STAGE_BYTES;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Cfg::RING_BYTES);
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint64_t* raw_full = drain + 1;
-  uint64_t* raw_empty = raw_full + R;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(raw_empty + R);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* s_pre = reinterpret_cast<int32_t*>(smem + Cfg::RING_BYTES + Cfg::BAR_BYTES);
   int32_t* s_offs = s_pre + 514;
@@ -173,12 +168,8 @@ __global__ void __launch_bounds__(SwapCfg<DUAL, FP8>::THREADS, 1)
   }
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      mbar_init(full + s, FP8 ? Cfg::NB / 32 : 1);  // FP8: one arrival per converter warp
+      mbar_init(full + s, 1);
       mbar_init(empty + s, 1);
-    }
-    for (int s = 0; s < R; ++s) {
-      mbar_init(raw_full + s, 1);
-      mbar_init(raw_empty + s, Cfg::NB / 32 + 1);  // converter warps + the MMA (token tile)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull + b, 1);
@@ -213,10 +204,6 @@ __global__ void __launch_bounds__(SwapCfg<DUAL, FP8>::THREADS, 1)
       // ------------------------------------------------ TMA producer
       const uint64_t pol_w = policy_evict_first();
       const uint64_t pol_x = policy_evict_last();
-      constexpr int RING = FP8 ? R : S;
-      uint64_t* land0 = FP8 ? raw_full : full;
-      uint64_t* free0 = FP8 ? raw_empty : empty;
-      constexpr uint32_t BYTES = FP8 ? Cfg::RAW_BYTES : Cfg::STAGE_BYTES;
       int stage = 0;
       uint32_t phase = 0, issued = 0, last_par = 0;
       bool ok = true;
@@ -224,57 +211,56 @@ __global__ void __launch_bounds__(SwapCfg<DUAL, FP8>::THREADS, 1)
         const SwapTile t = decode_swap(p, s_pre, s_offs, tile);
         const bool sh = t.g == p.E;
         for (int kb = 0; kb < t.kblocks; ++kb) {
-          if (!mbar_wait(free0 + stage, phase ^ 1, abort_flag, p.status, tcode | 1)) {
+          if (!mbar_wait(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 1)) {
             ok = false;
             break;
           }
-          uint64_t* land = land0 + stage;
-          uint8_t* base = FP8 ? raw_ring + stage * Cfg::RAW_BYTES : smem + stage * Cfg::STAGE_BYTES;
-          constexpr int WROW = FP8 ? kBK : 128;  // bytes per weight row in the destination
-          uint8_t* xdst = base + Cfg::NB * WROW;
-          mbar_arrive_expect_tx(land, BYTES);
+          uint64_t* land = full + stage;
+          uint8_t* base = smem + stage * Cfg::STAGE_BYTES;
+          uint8_t* xdst = base + Cfg::W_BYTES;
+          mbar_arrive_expect_tx(land, Cfg::STAGE_BYTES);
           if (sh) tma_load_2d(base, &tmB_s, land, kb * kBK, t.n0, pol_w);
           else tma_load_3d(base, &tmB_r, land, kb * kBK, t.n0, t.g, pol_w);
           if (DUAL) {
-            if (sh) tma_load_2d(base + 128 * WROW, &tmC_s, land, kb * kBK, t.n0, pol_w);
-            else tma_load_3d(base + 128 * WROW, &tmC_r, land, kb * kBK, t.n0, t.g, pol_w);
+            if (sh) tma_load_2d(base + 128 * 128, &tmC_s, land, kb * kBK, t.n0, pol_w);
+            else tma_load_3d(base + 128 * 128, &tmC_r, land, kb * kBK, t.n0, t.g, pol_w);
           }
           tma_load_2d(xdst, sh ? &tmX_s : &tmX_r, land, kb * kBK, (int)t.row0, pol_x);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == RING) {
+          if (++stage == S) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
       if (*abort_flag)
-        for (int s = 0; s < RING; ++s)
-          if (issued >> s & 1u) drain_wait(land0 + s, last_par >> s & 1u);
+        for (int s = 0; s < S; ++s)
+          if (issued >> s & 1u) drain_wait(full + s, last_par >> s & 1u);
     }
     __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer
-      constexpr uint32_t idesc = idesc_bf16(kBM, kNCH);
-      int stage = 0, rstage = 0, acc = 0;
-      uint32_t phase = 0, rphase = 0, acc_phase = 0;
+      int stage = 0, acc = 0;
+      uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const SwapTile t = decode_swap(p, s_pre, s_offs, tile);
+        // MMA N = the chunk's token rows rounded up to 16: columns past them are
+        // neither computed nor read back
+        const uint32_t idesc = idesc_bf16(kBM, min(kNCH, (t.rows - t.c0 + 15) & ~15));
         if (!mbar_wait(tempty + acc, acc_phase ^ 1, abort_flag, p.status, tcode | 2)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + acc * Cfg::ACC_COLS;
         for (int kb = 0; kb < t.kblocks; ++kb) {
-          // FP8: `full` is arrived by the converters after the raw slot (weights
-          // and token tile) has landed, so the token tile is there too.
           if (!mbar_wait(full + stage, phase, abort_flag, p.status, tcode | 3)) {
             ok = false;
             break;
           }
           tc_fence_after();
           const uint32_t sw = smem_u32(smem + stage * Cfg::STAGE_BYTES);
-          const uint32_t sx = FP8 ? smem_u32(raw_ring + rstage * Cfg::RAW_BYTES + Cfg::NB * kBK) : sw + Cfg::W_BYTES;
+          const uint32_t sx = sw + Cfg::W_BYTES;
 #pragma unroll
           for (int kk = 0; kk < kBK / 16; ++kk) {
             const uint64_t bd = sdesc_sw128(sx + kk * 32);
@@ -283,14 +269,9 @@ __global__ void __launch_bounds__(SwapCfg<DUAL, FP8>::THREADS, 1)
             if (DUAL) umma_f16(d0 + kNCH, sdesc_sw128(sw + 128 * 128 + kk * 32), bd, idesc, accum);
           }
           umma_commit(empty + stage);
-          if (FP8) umma_commit(raw_empty + rstage);
           if (++stage == S) {
             stage = 0;
             phase ^= 1;
-          }
-          if (FP8 && ++rstage == R) {
-            rstage = 0;
-            rphase ^= 1;
           }
         }
         if (!ok) break;
@@ -300,7 +281,6 @@ __global__ void __launch_bounds__(SwapCfg<DUAL, FP8>::THREADS, 1)
           acc_phase ^= 1;
         }
       }
-      (void)rphase;
       umma_commit(drain);
       drain_wait(drain, 0);
     }
@@ -308,45 +288,6 @@ __global__ void __launch_bounds__(SwapCfg<DUAL, FP8>::THREADS, 1)
   } else if (warp < 2 + Cfg::EPI_WARPS) {
     swap_epilogue<DUAL, EPI, Cfg::EPI_WARPS>(p, s_pre, s_offs, total, tmem_base, tfull, tempty, abort_flag, tcode,
                                             warp, lane);
-  } else if (FP8) {
-    // ------------------------------------------------ E4M3 -> bf16 converters
-    const int ct = threadIdx.x - 192;
-    int stage = 0, rstage = 0;
-    uint32_t phase = 0, rphase = 0;
-    bool stop = false;
-    for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
-      const SwapTile t = decode_swap(p, s_pre, s_offs, tile);
-      const bool sh = t.g == p.E;
-      ScaleStreams ss;
-      scale_rows(ss, DUAL, sh, t.g, t.n0, t.N, sh ? p.K_s : p.K_r, p.sc_b_r, p.sc_b_s, p.sc_c_r, p.sc_c_s,
-                 Cfg::NB);
-      ss.start(0);
-      for (int kb = 0; kb < t.kblocks; ++kb) {
-        ss.at(kb, 0);
-        const bool ok = mbar_wait(raw_full + rstage, rphase, abort_flag, p.status, tcode | 5) &&
-                        mbar_wait(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 7);
-        if (!__all_sync(0xffffffffu, ok)) {  // the warp goes on, or stops, as one
-          stop = true;
-          break;
-        }
-        convert_e4m3_rows<Cfg::NB>(raw_ring + rstage * Cfg::RAW_BYTES, smem + stage * Cfg::STAGE_BYTES, ct, ss.cur);
-        // raw weight bytes consumed; order these generic reads before the TMA's refill
-        fence_proxy_async_smem();
-        __syncwarp();  // the warp's writes and proxy fences, then one arrival per warp
-        if (lane == 0) {
-          mbar_arrive(full + stage);
-          mbar_arrive(raw_empty + rstage);
-        }
-        if (++stage == S) {
-          stage = 0;
-          phase ^= 1;
-        }
-        if (++rstage == R) {
-          rstage = 0;
-          rphase ^= 1;
-        }
-      }
-    }
   }
 
   tc_fence_before();

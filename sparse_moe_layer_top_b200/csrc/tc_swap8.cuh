@@ -37,13 +37,14 @@ struct Swap8Cfg {
   static constexpr int CONV_WARPS = NB / 32;
   static constexpr int THREADS = 64 + 32 * (EPI_WARPS + CONV_WARPS);
   static constexpr int ACC_COLS = (DUAL ? 2 : 1) * kNCH;
+  static constexpr int ACC_BUFS = 2;  // accumulator buffers (epilogue of tile i overlaps tile i + 1)
   static constexpr int A_COLS = (DUAL ? 2 : 1) * (kBK8 / 2);
   static constexpr int A_STAGES = DUAL ? 2 : 4;
   static constexpr int TMEM_COLS = 512;
   static constexpr int BAR_BYTES = (2 * RAW_STAGES + 2 * A_STAGES + 5) * 8 + 16;
   static constexpr int SCHED_INTS = 2 * (512 + 2);
   static constexpr int SMEM_BYTES = 1024 + RING_BYTES + BAR_BYTES + SCHED_INTS * 4;
-  static_assert(2 * ACC_COLS + A_STAGES * A_COLS <= TMEM_COLS, "TMEM columns");
+  static_assert(ACC_BUFS * ACC_COLS + A_STAGES * A_COLS <= TMEM_COLS, "TMEM columns");
   static_assert(RAW_BYTES % 1024 == 0 && (NB * kBK8) % 1024 == 0, "swizzled tiles need 1024-byte alignment");
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
@@ -87,7 +88,7 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
       mbar_init(a_full + s, Cfg::CONV_WARPS);
       mbar_init(a_empty + s, 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < Cfg::ACC_BUFS; ++b) {
       mbar_init(tfull + b, 1);
       mbar_init(tempty + b, Cfg::EPI_WARPS);
     }
@@ -162,12 +163,14 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------ MMA issuer (A from TMEM, B = token tile)
-      constexpr uint32_t idesc = idesc_bf16(kBM, kNCH);
       int rstage = 0, astage = 0, acc = 0;
       uint32_t aphase = 0, acc_phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         const SwapTile t = decode_swap(p, s_pre, s_offs, tile);
+        // MMA N = the chunk's token rows rounded up to 16: columns past them are
+        // neither computed nor read back
+        const uint32_t idesc = idesc_bf16(kBM, min(kNCH, (t.rows - t.c0 + 15) & ~15));
         const int nkb = (t.g == p.E ? p.K_s : p.K_r) / kBK8;
         if (!mbar_wait(tempty + acc, acc_phase ^ 1, abort_flag, p.status, tcode | 2)) break;
         tc_fence_after();
@@ -180,7 +183,7 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = tmem_base + 2 * Cfg::ACC_COLS + astage * Cfg::A_COLS;
+          const uint32_t a0 = tmem_base + Cfg::ACC_BUFS * Cfg::ACC_COLS + astage * Cfg::A_COLS;
           const uint32_t sx = smem_u32(smem + rstage * Cfg::RAW_BYTES + Cfg::NB * kBK8);
 #pragma unroll
           for (int kk = 0; kk < kBK8 / 16; ++kk) {
@@ -199,7 +202,7 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
         }
         if (!ok) break;
         umma_commit(tfull + acc);
-        if (++acc == 2) {
+        if (++acc == Cfg::ACC_BUFS) {
           acc = 0;
           acc_phase ^= 1;
         }
@@ -209,7 +212,7 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
     }
     __syncwarp();
   } else if (warp < 2 + Cfg::EPI_WARPS) {
-    swap_epilogue<DUAL, EPI, Cfg::EPI_WARPS>(p, s_pre, s_offs, total, tmem_base, tfull, tempty, abort_flag, tcode,
+    swap_epilogue<DUAL, EPI, Cfg::EPI_WARPS, Cfg::ACC_BUFS>(p, s_pre, s_offs, total, tmem_base, tfull, tempty, abort_flag, tcode,
                                             warp, lane);
   } else {
     // ------------------------------------------------ E4M3 -> bf16 converters, raw smem -> TMEM
@@ -223,8 +226,7 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
     for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
       const SwapTile t = decode_swap(p, s_pre, s_offs, tile);
       const bool sh = t.g == p.E;
-      const int K = sh ? p.K_s : p.K_r;
-      const int nkb = K / kBK8;
+      const int nkb = (sh ? p.K_s : p.K_r) / kBK8;
       // the tile's 128 rows are one scale row block: one fp32 scale per K block
       const float* sbase = mat == 0 ? (sh ? p.sc_b_s : p.sc_b_r) : (sh ? p.sc_c_s : p.sc_c_r);
       const float* srow = sbase + ((sh ? 0 : (int64_t)t.g * (t.N / 128)) + t.n0 / 128) * (int64_t)nkb;
@@ -239,31 +241,32 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
         }
         tc_fence_after();
         const uint8_t* src = smem + rstage * Cfg::RAW_BYTES + (mat * 128 + r) * kBK8;
-        const uint32_t ta = tmem_base + lane_off + 2 * Cfg::ACC_COLS + astage * Cfg::A_COLS + mat * (kBK8 / 2);
+        uint32_t o[64];
 #pragma unroll
         for (int h = 0; h < 2; ++h) {
           uint4 v[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j)  // 16-byte chunk c of the row sits at chunk c ^ (row & 7)
             v[j] = *reinterpret_cast<const uint4*>(src + (((h * 4 + j) ^ (r & 7)) << 4));
-          uint32_t o[32];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint2 a = e4m3x4_scaled_bf16(v[j].x, s_cur);
             const uint2 b = e4m3x4_scaled_bf16(v[j].y, s_cur);
             const uint2 c = e4m3x4_scaled_bf16(v[j].z, s_cur);
             const uint2 d = e4m3x4_scaled_bf16(v[j].w, s_cur);
-            o[8 * j + 0] = a.x;
-            o[8 * j + 1] = a.y;
-            o[8 * j + 2] = b.x;
-            o[8 * j + 3] = b.y;
-            o[8 * j + 4] = c.x;
-            o[8 * j + 5] = c.y;
-            o[8 * j + 6] = d.x;
-            o[8 * j + 7] = d.y;
+            uint32_t* w = o + 32 * h + 8 * j;
+            w[0] = a.x;
+            w[1] = a.y;
+            w[2] = b.x;
+            w[3] = b.y;
+            w[4] = c.x;
+            w[5] = c.y;
+            w[6] = d.x;
+            w[7] = d.y;
           }
-          tmem_st32(ta + h * 32, o);
         }
+        tmem_st64(tmem_base + lane_off + Cfg::ACC_BUFS * Cfg::ACC_COLS + astage * Cfg::A_COLS + mat * (kBK8 / 2),
+                  o);
         // raw weight bytes consumed: order these generic reads before the TMA's refill
         fence_proxy_async_smem();
         tmem_wait_st();
