@@ -368,10 +368,14 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
   if (!tc) {
     dim3 grid((unsigned)cdiv(p.T, 8));
     PROF_BEGIN("router_simt", st);
-    if (p.act_dtype == MOE_F32)
-      k_router_simt<float><<<grid, 256, 0, st>>>((const float*)x, (const float*)wr, bias, p.T, p.d, p.E, p.k, ids, tw);
-    else
-      k_router_simt<bf16><<<grid, 256, 0, st>>>((const bf16*)x, (const bf16*)wr, bias, p.T, p.d, p.E, p.k, ids, tw);
+    const int npl = select_npl(p.E);
+    if (p.act_dtype == MOE_F32) {
+      auto kf = npl == 4 ? k_router_simt<float, 4> : npl == 8 ? k_router_simt<float, 8> : k_router_simt<float, 16>;
+      kf<<<grid, 256, 0, st>>>((const float*)x, (const float*)wr, bias, p.T, p.d, p.E, p.k, ids, tw);
+    } else {
+      auto kb = npl == 4 ? k_router_simt<bf16, 4> : npl == 8 ? k_router_simt<bf16, 8> : k_router_simt<bf16, 16>;
+      kb<<<grid, 256, 0, st>>>((const bf16*)x, (const bf16*)wr, bias, p.T, p.d, p.E, p.k, ids, tw);
+    }
     LAUNCH_CHECK("router_simt", st);
     return MOE_OK;
   }
@@ -398,8 +402,10 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
   LAUNCH_CHECK("gemm_tc_router", st);
   if (counts) CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * p.E * 4, st));
   PROF_BEGIN("topk", st);
-  k_topk<<<(unsigned)cdiv(p.T, 8), 256, 0, st>>>(part, rs.ksplit, p.T * rs.ldp, rs.ldp, bias, p.T, p.E, p.k, ids, tw,
-                                                 counts);
+  const int npl = select_npl(p.E);
+  auto kt = npl == 4 ? k_topk<4> : npl == 8 ? k_topk<8> : k_topk<16>;
+  kt<<<(unsigned)cdiv(p.T, 8), 256, 0, st>>>(part, rs.ksplit, p.T * rs.ldp, rs.ldp, bias, p.T, p.E, p.k, ids, tw,
+                                             counts);
   LAUNCH_CHECK("topk", st);
   *counted = counts != nullptr;
   return MOE_OK;

@@ -11,6 +11,8 @@ namespace moe {
 using bf16 = __nv_bfloat16;
 using fp8 = __nv_fp8_storage_t;  // raw E4M3 code
 
+constexpr int kMaxK = 16;  // largest k (experts per token) the kernels support
+
 // Device status codes: high byte = which check, low bits = where.
 enum : unsigned {
   kStatusBadExpertId = 0x06000001u,  // a routing id outside [0, E)

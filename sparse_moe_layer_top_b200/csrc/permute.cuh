@@ -244,7 +244,8 @@ __global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ x, con
     if ((uint64_t)t >= (uint64_t)T) t = 0;  // cannot happen for valid routing
     const uint4* src = x + (int64_t)t * vec_per_row;
     uint4* dst = xp + r * vec_per_row;
-    for (int v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);
+#pragma unroll 4
+    for (int v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);  // (restrict: reads batch ahead)
   }
 }
 

@@ -17,28 +17,27 @@
 namespace moe {
 
 constexpr int kChunkTokens = 128;  // tokens per dispatch chunk (one k_topk / k_count block)
-constexpr int kMaxK = 16;          // largest k the selection supports
 
-// Warp-wide selection over one token's logits l[] (lane owns experts lane + 32 i).
-// Lane 0 writes the ids and weights; returns nothing.  `hist` (shared memory,
-// may be NULL) counts the selected experts.
-__device__ __forceinline__ void warp_select(float (&l)[16], int E, int k, int64_t t, int32_t* ids, float* tw,
-                                            int* hist) {
+// Warp-wide selection over one token's logits l[] (lane owns experts lane + 32 i;
+// NPL = 32-expert columns held, entries past E are -inf).  Each round takes the
+// warp arg-max (a strict > scan inside the lane keeps its lowest expert, the
+// shuffle tree prefers the lower expert on equal values) and sets the taken
+// entry to -inf.  Lanes < k write the ids and weights; `hist` (may be NULL)
+// counts the selected experts.
+template <int NPL>
+__device__ __forceinline__ void warp_select(float (&l)[NPL], int k, int64_t t, int32_t* ids, float* tw, int* hist) {
   const int lane = threadIdx.x & 31;
-  unsigned taken = 0;
   float v0 = 0.f, den = 0.f, my_v = 0.f;
   int my_e = 0;
   for (int s = 0; s < k; ++s) {
-    float bv = -INFINITY;
-    int be = 0x7fffffff;
+    float bv = l[0];
+    int be = lane;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !(taken >> i & 1u) && (l[i] > bv || be == 0x7fffffff)) {
+    for (int i = 1; i < NPL; ++i)
+      if (l[i] > bv) {
         bv = l[i];
-        be = e;
+        be = lane + 32 * i;
       }
-    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
       const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
@@ -48,7 +47,9 @@ __device__ __forceinline__ void warp_select(float (&l)[16], int E, int k, int64_
         be = oe;
       }
     }
-    if ((be & 31) == lane) taken |= 1u << (be >> 5);
+#pragma unroll
+    for (int i = 0; i < NPL; ++i)
+      if (be == lane + 32 * i) l[i] = -INFINITY;
     if (s == 0) v0 = bv;
     den += __expf(bv - v0);
     if (lane == s) {  // lane s keeps selection s (k <= 16 < 32)
@@ -64,7 +65,7 @@ __device__ __forceinline__ void warp_select(float (&l)[16], int E, int k, int64_
 }
 
 // fp32 path: one warp per token, logits by fp32 FMA.
-template <typename TA>
+template <typename TA, int NPL>
 __global__ void __launch_bounds__(256) k_router_simt(const TA* __restrict__ x, const TA* __restrict__ wr,
                                                      const float* __restrict__ bias, int64_t T, int d, int E, int k,
                                                      int32_t* __restrict__ ids, float* __restrict__ tw) {
@@ -72,9 +73,9 @@ __global__ void __launch_bounds__(256) k_router_simt(const TA* __restrict__ x, c
   const int64_t t = (int64_t)blockIdx.x * 8 + warp;
   if (t >= T) return;
   const TA* xt = x + t * d;
-  float l[16];
+  float l[NPL];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
+  for (int i = 0; i < NPL; ++i) {
     const int e = lane + 32 * i;
     float acc = -INFINITY;
     if (e < E) {
@@ -85,12 +86,13 @@ __global__ void __launch_bounds__(256) k_router_simt(const TA* __restrict__ x, c
     }
     l[i] = acc;
   }
-  warp_select(l, E, k, t, ids, tw, nullptr);
+  warp_select<NPL>(l, k, t, ids, tw, nullptr);
 }
 
 // Top-k from split logits, one warp per token.  When `counts` is given
 // (zeroed beforehand), the selected experts are also counted into the
 // per-chunk histograms counts[(t / kChunkTokens) * E + e] for the dispatch.
+template <int NPL>
 __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ part, int nsplit, int64_t split_stride,
                                               int64_t ldp, const float* __restrict__ bias, int64_t T, int E, int k,
                                               int32_t* __restrict__ ids, float* __restrict__ tw,
@@ -98,17 +100,20 @@ __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ part, in
   const int lane = threadIdx.x & 31;
   const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
-  float l[16];
+  float l[NPL];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) l[i] = (lane + 32 * i < E) ? (bias ? __ldg(bias + lane + 32 * i) : 0.f) : -INFINITY;
+  for (int i = 0; i < NPL; ++i) l[i] = (lane + 32 * i < E) ? (bias ? __ldg(bias + lane + 32 * i) : 0.f) : -INFINITY;
   const float* row = part + t * ldp;
 #pragma unroll 4
   for (int s = 0; s < nsplit; ++s) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < NPL; ++i)
       if (lane + 32 * i < E) l[i] += __ldg(row + s * split_stride + lane + 32 * i);
   }
-  warp_select(l, E, k, t, ids, tw, counts ? counts + (t / kChunkTokens) * E : nullptr);
+  warp_select<NPL>(l, k, t, ids, tw, counts ? counts + (t / kChunkTokens) * E : nullptr);
 }
+
+// Values per lane for E experts: the smallest of 4, 8, 16 with 32 * NPL >= E.
+inline int select_npl(int E) { return E <= 128 ? 4 : E <= 256 ? 8 : 16; }
 
 }  // namespace moe

@@ -168,20 +168,27 @@ __global__ void __launch_bounds__(256) k_slot_sum(const TA* __restrict__ ys, con
   if (has_shared) ok |= 1u << k;
   for (int c = threadIdx.x * 8; c < d; c += blockDim.x * 8) {
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-    for (int j = 0; j <= k; ++j) {
-      if (!(ok >> j & 1u)) continue;
-      const TA* row = src + (int64_t)j * d + c;
-      if (sizeof(TA) == 2) {
-        uint4 v = *reinterpret_cast<const uint4*>(row);
-        const bf16* h = reinterpret_cast<const bf16*>(&v);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] += to_f32(h[e]);
-      } else {
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] += to_f32(row[e]);
-      }
-    }
     if (sizeof(TA) == 2) {
+      // slot rows are read in batches of up to 9 (k = 8: all of them) issued
+      // before the batch's first addition; the additions keep slot order
+      constexpr int B = 9;
+      for (int j0 = 0; j0 <= k; j0 += B) {
+        uint4 v[B];
+#pragma unroll
+        for (int i = 0; i < B; ++i) {
+          const int j = j0 + i;
+          if (j <= k && (ok >> j & 1u)) v[i] = __ldg(reinterpret_cast<const uint4*>(src + (int64_t)j * d + c));
+        }
+#pragma unroll
+        for (int i = 0; i < B; ++i) {
+          const int j = j0 + i;
+          if (j <= k && (ok >> j & 1u)) {
+            const bf16* h = reinterpret_cast<const bf16*>(&v[i]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] += to_f32(h[e]);
+          }
+        }
+      }
       uint4 o;
       o.x = pack_bf16x2(acc[0], acc[1]);
       o.y = pack_bf16x2(acc[2], acc[3]);
@@ -189,6 +196,12 @@ __global__ void __launch_bounds__(256) k_slot_sum(const TA* __restrict__ ys, con
       o.w = pack_bf16x2(acc[6], acc[7]);
       *reinterpret_cast<uint4*>(y + t * d + c) = o;
     } else {
+      for (int j = 0; j <= k; ++j) {
+        if (!(ok >> j & 1u)) continue;
+        const TA* row = src + (int64_t)j * d + c;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += to_f32(row[e]);
+      }
 #pragma unroll
       for (int e = 0; e < 8; ++e) from_f32(acc[e], y + t * d + c + e);
     }
