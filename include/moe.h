@@ -169,11 +169,14 @@ MOE_API moe_status moe_router_topk_static(const moe_problem* p, const void* x, c
 /* Kernel-path selection for the calls above on the calling process:
  * 0 = automatic (tensor-core kernels where the types allow; for the expert
  *     GEMMs the weight-row form when T*k <= 64*E, i.e. when an expert sees at
- *     most one 64-token chunk on average, else the row-tiled form);
+ *     most one 64-token chunk on average, the form of 4 when bf16 experts
+ *     average 2048 rows or more (T*k >= 2048*E), else the row-tiled form);
  * 1 = SIMT CUDA kernels only (fp32 FMA; the path of fp32 problems);
  * 2 = tensor-core kernels required, row-tiled expert GEMMs;
- * 3 = tensor-core kernels required, weight-row expert GEMMs.
- * 2 and 3 return MOE_ERR_UNSUPPORTED when the types do not allow them. */
+ * 3 = tensor-core kernels required, weight-row expert GEMMs;
+ * 4 = tensor-core kernels required, row-tiled expert GEMMs on 2-CTA clusters
+ *     (256-row tiles, tcgen05 pair MMAs; E4M3 weights take the form of 2).
+ * 2, 3 and 4 return MOE_ERR_UNSUPPORTED when the types do not allow them. */
 MOE_API moe_status moe_set_path(int path);
 
 /* Synchronously read and clear the device status word of the current device

@@ -77,17 +77,17 @@ struct TileInfo {
 
 // s_pre / s_offs: the schedule's tile prefix and group offsets, cached in
 // shared memory at kernel start (grouped mode).
-template <int BN>
+template <int BN, int BM = kBM>
 __device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, const int32_t* s_pre, const int32_t* s_offs,
                                                 int tile) {
   TileInfo t;
   if (p.single_rows >= 0) {
     t.g = p.E;
     t.rows = p.single_rows;
-    const int mtc = (t.rows + kBM - 1) / kBM, ntc = (p.N_s + BN - 1) / BN;
+    const int mtc = (t.rows + BM - 1) / BM, ntc = (p.N_s + BN - 1) / BN;
     t.split = tile / (mtc * ntc);
     const int local = tile - t.split * mtc * ntc;
-    t.m0 = (local % mtc) * kBM;
+    t.m0 = (local % mtc) * BM;
     t.n0 = (local / mtc) * BN;
     t.row0 = t.m0;
     t.N = p.N_s;
@@ -106,10 +106,10 @@ __device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, const int32
   }
   const int r0 = s_offs[t.g];
   t.rows = s_offs[t.g + 1] - r0;
-  const int mtc = (t.rows + kBM - 1) / kBM;
+  const int mtc = (t.rows + BM - 1) / BM;
   const int local = tile - s_pre[t.g];
   const int mb = local % mtc, nb = local / mtc;
-  t.m0 = mb * kBM;
+  t.m0 = mb * BM;
   t.row0 = (int64_t)r0 + t.m0;
   t.n0 = nb * BN;
   const bool sh = t.g == p.E;
@@ -271,6 +271,50 @@ __device__ __forceinline__ void scale_rows(ScaleStreams& ss, bool dual, bool sh,
   } else {
     ss.row[0] = n0 < N ? base_b + (int64_t)(n0 / 128) * ss.kb128 : nullptr;
     ss.row[1] = (nrows > 128 && n0 + 128 < N) ? base_b + (int64_t)(n0 / 128 + 1) * ss.kb128 : nullptr;
+  }
+}
+
+// Epilogue of one row-tiled tile for the SwiGLU / SlotStore / Store modes, as
+// run by one warp: its 32 rows are the TMEM lanes addressed by `tb` (lane
+// offset included) and row `row` of the tile is this thread's; it converts the
+// 32-column chunks [c0, c1) and stores them through its 2 KB staging buffer.
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_rows(const TcGemmArgs& p, const TileInfo& t, uint32_t tb, int row, int c0,
+                                              int c1, uint8_t* stg, int lane) {
+  const int64_t grow = t.row0 + row;
+  const bool valid = t.m0 + row < t.rows && grow < p.rows_cap;
+  // destination row of this lane (NULL: nothing to write) and its scale
+  char* rowp = nullptr;
+  float w = 1.f;
+  if (valid) {
+    if (EPI == kTcSwiGLU) {
+      rowp = reinterpret_cast<char*>(p.H + grow * p.ldh);
+    } else if (EPI == kTcSlotStore) {
+      const int64_t dr = __ldg(p.row_dst + grow);
+      w = __ldg(p.row_w + grow);
+      if (dr >= 0) rowp = reinterpret_cast<char*>(p.ys + dr * p.ldy);
+    } else {
+      rowp = reinterpret_cast<char*>(p.out + grow * p.ldo);
+    }
+  }
+#pragma unroll 1
+  for (int c = c0; c < c1; ++c) {
+    uint32_t a[32], u[32];
+    tmem_ld32(tb + c * 32, a);
+    if (EPI == kTcSwiGLU) tmem_ld32(tb + BN + c * 32, u);
+    tmem_wait_regs(a);
+    if (EPI == kTcSwiGLU) tmem_wait_regs(u);
+    uint32_t o[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+      const float x0 = __uint_as_float(a[2 * e]), x1 = __uint_as_float(a[2 * e + 1]);
+      if (EPI == kTcSwiGLU)
+        o[e] = pack_bf16x2(silu_f32(x0) * __uint_as_float(u[2 * e]), silu_f32(x1) * __uint_as_float(u[2 * e + 1]));
+      else
+        o[e] = pack_bf16x2(w * x0, w * x1);
+    }
+    const int n = t.n0 + c * 32;
+    store_rows_staged(stg, o, rowp, (int64_t)n * 2, t.N - n, lane);
   }
 }
 
@@ -470,41 +514,8 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
       const int64_t grow = t.row0 + row;
       const bool valid = t.m0 + row < t.rows && grow < p.rows_cap;
       if (EPI == kTcSwiGLU || EPI == kTcSlotStore || EPI == kTcStore) {
-        // destination row of this lane (NULL: nothing to write) and its scale
-        char* rowp = nullptr;
-        float w = 1.f;
-        if (valid) {
-          if (EPI == kTcSwiGLU) {
-            rowp = reinterpret_cast<char*>(p.H + grow * p.ldh);
-          } else if (EPI == kTcSlotStore) {
-            const int64_t dr = __ldg(p.row_dst + grow);
-            w = __ldg(p.row_w + grow);
-            if (dr >= 0) rowp = reinterpret_cast<char*>(p.ys + dr * p.ldy);
-          } else {
-            rowp = reinterpret_cast<char*>(p.out + grow * p.ldo);
-          }
-        }
-        uint8_t* stg = epi_stage + (warp - 2) * 2048;
         constexpr int CPW = (BN / 32) / EG;  // 32-column chunks per warp, contiguous
-#pragma unroll 1
-        for (int c = eg * CPW; c < (eg + 1) * CPW; ++c) {
-          uint32_t a[32], u[32];
-          tmem_ld32(tb + c * 32, a);
-          if (EPI == kTcSwiGLU) tmem_ld32(tb + BN + c * 32, u);
-          tmem_wait_regs(a);
-          if (EPI == kTcSwiGLU) tmem_wait_regs(u);
-          uint32_t o[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x0 = __uint_as_float(a[2 * e]), x1 = __uint_as_float(a[2 * e + 1]);
-            if (EPI == kTcSwiGLU)
-              o[e] = pack_bf16x2(silu_f32(x0) * __uint_as_float(u[2 * e]), silu_f32(x1) * __uint_as_float(u[2 * e + 1]));
-            else
-              o[e] = pack_bf16x2(w * x0, w * x1);
-          }
-          const int n = t.n0 + c * 32;
-          store_rows_staged(stg, o, rowp, (int64_t)n * 2, t.N - n, lane);
-        }
+        epilogue_rows<BN, EPI>(p, t, tb, row, eg * CPW, (eg + 1) * CPW, epi_stage + (warp - 2) * 2048, lane);
       } else if (EPI == kTcLogits) {
         float* dst = p.part + (int64_t)t.split * p.part_stride + grow * p.ldp;
 #pragma unroll 1

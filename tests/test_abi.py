@@ -89,6 +89,6 @@ def test_host_rejects_before_any_launch():
 
 
 def test_set_path_validates():
-    assert moe.lib().moe_set_path(4) == 1
+    assert moe.lib().moe_set_path(5) == 1
     assert moe.lib().moe_set_path(-1) == 1
     assert moe.lib().moe_set_path(0) == 0
