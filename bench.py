@@ -36,7 +36,7 @@ DEFAULT_CONFIG = "qwen36_35b_a3b_bf16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
 KERNEL_SOURCES = ("api.cu", "common.cuh", "permute.cuh", "ptx.cuh", "router.cuh", "simt.cuh", "tc_gemm.cuh",
-                  "tc_swap.cuh")
+                  "tc_swap.cuh", "tc_swap8.cuh", "tc_pair.cuh")
 
 
 # ---------------------------------------------------------------- helpers
