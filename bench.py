@@ -35,15 +35,22 @@ UNIT = "tokens/s"
 DEFAULT_CONFIG = "qwen36_35b_a3b_bf16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
-KERNEL_SOURCES = ("api.cu", "common.cuh", "permute.cuh", "ptx.cuh", "router.cuh", "simt.cuh", "tc_gemm.cuh",
-                  "tc_swap.cuh", "tc_swap8.cuh", "tc_pair.cuh")
+# The files that define each timed kernel (its template, the PTX wrappers it
+# uses, its launch configuration): an ncu traffic figure stays valid while
+# their contents hash to the value recorded with it.
+KERNEL_SOURCES = {
+    "gemm_tc_swiglu": ("tc_gemm.cuh", "ptx.cuh", "common.cuh", "api.cu"),
+    "gemm_tc_down": ("tc_gemm.cuh", "ptx.cuh", "common.cuh", "api.cu"),
+}
+ALL_SOURCES = ("api.cu", "common.cuh", "permute.cuh", "ptx.cuh", "router.cuh", "simt.cuh", "tc_gemm.cuh",
+               "tc_swap.cuh", "tc_swap8.cuh", "tc_pair.cuh")
 
 
 # ---------------------------------------------------------------- helpers
-def kernel_source_sha():
+def kernel_source_sha(files=ALL_SOURCES):
     h = hashlib.sha256()
     d = os.path.join(ROOT, "sparse_moe_layer_top_b200", "csrc")
-    for f in KERNEL_SOURCES:
+    for f in files:
         with open(os.path.join(d, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -66,7 +73,8 @@ def load_traffic(kernel, workload):
         with open(p) as f:
             d = json.load(f)
         for e in d.get("entries", []):
-            if e["kernel"] == kernel and e["workload"] == workload and e["source_sha"] == kernel_source_sha():
+            files = tuple(e.get("sources", ALL_SOURCES))
+            if e["kernel"] == kernel and e["workload"] == workload and e["source_sha"] == kernel_source_sha(files):
                 return float(e["dram_bytes_per_launch"])
     except Exception:
         pass
