@@ -33,13 +33,17 @@ def lib():
         L.oracle_swiglu_expert.argtypes = [I64, I32, I32, I32, P, I64, I32, P, P, P, P, P, P, P]
         L.oracle_moe_forward.argtypes = [I64, I32, I32, I32, I32, I32, I32, I32,
                                          P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
+        L.oracle_block_forward.argtypes = [I64, I32, I32, I32, I32, I32, I32, I32, P, P, ctypes.c_double, P,
+                                           P, P, P, P, P, P, P, P, P, P, P, P, P, P, P]
+        L.oracle_rmsnorm.argtypes = [I64, I32, I32, P, P, ctypes.c_double, P]
         L.oracle_expert_ffn.argtypes = [I32, I32, I32, I32, I32, I32, P, P, P, P, P, P, P, P, P, P]
         L.oracle_combine.argtypes = [I64, I32, I32, I32, I32, P, P, P, P, P]
         L.oracle_param_count.argtypes = [I64, I64, I64, I64, I64, I32]
         L.oracle_param_count.restype = I64
         L.oracle_e4m3_decode.argtypes = [P, I64, P]
         for f in ("oracle_router", "oracle_permute", "oracle_swiglu_expert", "oracle_moe_forward",
-                  "oracle_expert_ffn", "oracle_combine", "oracle_e4m3_decode"):
+                  "oracle_block_forward", "oracle_rmsnorm", "oracle_expert_ffn", "oracle_combine",
+                  "oracle_e4m3_decode"):
             getattr(L, f).restype = I32
         L.oracle_num_threads.restype = I32
         _lib = L
@@ -176,6 +180,56 @@ def moe_forward(x, w_r, wg, wu, wd, s_wg, s_wu, s_wd, k, bias=None, scales=None,
                                   _p(y), _p(ids), _p(w), _p(probs))
     assert rc == 0
     return y, ids, w, probs
+
+
+def rmsnorm(x, gamma, eps=1e-6):
+    """Zero-centred RMSNorm of the rows of x [T, d]: x / sqrt(mean x^2 + eps) * (1 + gamma),
+    float64, not rounded (gamma [d] in x's type)."""
+    xa, adt = _np(x)
+    ga, gdt = _np(gamma)
+    assert gdt == adt
+    T, d = xa.shape
+    out = np.empty((T, d))
+    assert lib().oracle_rmsnorm(T, d, adt, _p(xa), _p(ga), float(eps), _p(out)) == 0
+    return out
+
+
+def block_forward(x, w_r, wg, wu, wd, s_wg, s_wu, s_wd, k, bias=None, scales=None, norm_weight=None,
+                  norm_eps=1e-6, shared_gate=None, force_ids=None, want_probs=True):
+    """The block with its optional neighbours -> (y, topk_ids, topk_w, probs, gate).
+
+    norm_weight [d] (x's type): zero-centred RMSNorm of x first, rounded to x's type;
+    shared_gate [d] (x's type): the shared expert weighted by sigmoid(x . shared_gate).
+    gate [T] is that weight (1 without a gate).  The rest as moe_forward.
+    """
+    xa, adt = _np(x)
+    ra, rdt = _np(w_r)
+    assert rdt == adt
+    ga, wdt = _np(wg)
+    ua, _ = _np(wu)
+    da, _ = _np(wd)
+    T, d = xa.shape
+    E, I = ga.shape[0], ga.shape[1]
+    if s_wg is None:
+        sga = sua = sda = None
+        I_s = 0
+    else:
+        sga, _ = _np(s_wg)
+        sua, _ = _np(s_wu)
+        sda, _ = _np(s_wd)
+        I_s = sga.shape[0]
+    na = None if norm_weight is None else _np(norm_weight)[0]
+    gwa = None if shared_gate is None else _np(shared_gate)[0]
+    b = _f32(bias)
+    sc = _f32(scales)
+    fi = None if force_ids is None else _i32(force_ids)
+    y = np.empty((T, d)); ids = np.empty((T, k), np.int32); w = np.empty((T, k)); gate = np.empty(T)
+    probs = np.empty((T, E)) if want_probs else None
+    rc = lib().oracle_block_forward(T, d, E, k, I, I_s, adt, wdt, _p(xa), _p(na), float(norm_eps), _p(gwa),
+                                    _p(ra), _p(b), _p(ga), _p(ua), _p(da), _p(sga), _p(sua), _p(sda), _p(sc),
+                                    _p(fi), _p(y), _p(ids), _p(w), _p(probs), _p(gate))
+    assert rc == 0
+    return y, ids, w, probs, gate
 
 
 def expert_ffn(x_perm, offs, wg, wu, wd, s_wg, s_wu, s_wd, scales=None):

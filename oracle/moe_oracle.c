@@ -30,6 +30,16 @@
  *                                               every input)
  *   output   y = sum_{e kept} w_e E_e(x) + S(x)
  *
+ * The block's neighbours (oracle_block_forward; both optional):
+ *   norm     x <- x / sqrt(mean_j x_j^2 + eps)   page 5: Qwen3-Next uses a
+ *            * (1 + gamma), rounded to the        "zero-centred" RMSNorm whose
+ *            activation type (the block's input)  parameters start at zero, so
+ *                                                 the applied scale is 1 + gamma;
+ *                                                 page 3 key rms_norm_eps = 1e-6
+ *   gate     S(x) weighted by sigmoid(x . w_sg)   not on the pages: an option
+ *                                                 some implementations carry;
+ *                                                 off (weight 1) by default
+ *
  * Every function below follows that definition literally, per token, in
  * float64, reading the caller's low-precision values (fp32, bf16 or E4M3 with
  * fp32 block scales) and converting each element as it is used.  There is no
@@ -98,6 +108,42 @@ static double welem(const void *w, int dt, const float *s, int64_t cols, int64_t
 }
 
 static double silu(double z) { return z / (1.0 + exp(-z)); }
+
+/* v rounded to the nearest value of the activation type (ties to even):
+ * bf16 keeps 8 significant bits (quantum 2^(e-8) for v = f 2^e, 1/2 <= |f| < 1;
+ * 2^-133 below the normal range); fp32 by the C conversion. */
+static double round_act(double v, int dt)
+{
+    if (dt == ODT_F32) return (double)(float)v;
+    if (v == 0.0 || !isfinite(v)) return v;
+    int e;
+    frexp(v, &e);
+    int qe = e - 8 < -133 ? -133 : e - 8;
+    double q = ldexp(1.0, qe);
+    return nearbyint(v / q) * q;
+}
+
+/* Zero-centred RMSNorm of one row of d values (read from x at row t):
+ * out_j = x_j / sqrt(mean x^2 + eps) * (1 + gamma_j), float64. */
+static void rmsnorm_row(int d, const void *x, int act_dt, int64_t t, const void *gamma, double eps, double *out)
+{
+    double ss = 0.0;
+    for (int j = 0; j < d; ++j) {
+        double v = elem(x, act_dt, t * d + j);
+        ss += v * v;
+    }
+    double r = 1.0 / sqrt(ss / d + eps);
+    for (int j = 0; j < d; ++j) out[j] = elem(x, act_dt, t * d + j) * r * (1.0 + elem(gamma, act_dt, j));
+}
+
+/* Zero-centred RMSNorm of T rows, float64 (not rounded). */
+int oracle_rmsnorm(int64_t T, int d, int act_dt, const void *x, const void *gamma, double eps, double *out)
+{
+    if (T < 0 || d <= 0 || !x || !gamma || !(eps >= 0.0)) return 1;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) rmsnorm_row(d, x, act_dt, t, gamma, eps, out + t * d);
+    return 0;
+}
 
 int oracle_num_threads(void)
 {
@@ -299,13 +345,19 @@ static void expert_ptrs(int d, int E, int I, int I_s, int w_dt, const void *wg, 
 /* The whole block, token by token.  force_ids [T,k] (may be NULL) replaces the
  * router's choice by a given set; the weights are still the renormalised
  * probabilities of that set.  probs [T,E] may be NULL. */
-int oracle_moe_forward(int64_t T, int d, int E, int k, int I, int I_s, int act_dt, int w_dt,
-                       const void *x, const void *w_r, const float *bias, const void *wg,
-                       const void *wu, const void *wd, const void *s_wg, const void *s_wu,
-                       const void *s_wd, const float *scales, const int32_t *force_ids, double *y,
-                       int32_t *topk_ids, double *topk_w, double *probs)
+/* The block with its optional neighbours: norm_w (NULL: none) applies the
+ * zero-centred RMSNorm to x first, its output rounded to the activation type;
+ * gate_w (NULL: none) weights the shared expert by sigmoid(x . gate_w), x being
+ * the (normalised) block input.  gate_out (may be NULL) receives that weight. */
+int oracle_block_forward(int64_t T, int d, int E, int k, int I, int I_s, int act_dt, int w_dt,
+                         const void *x, const void *norm_w, double eps, const void *gate_w,
+                         const void *w_r, const float *bias, const void *wg, const void *wu,
+                         const void *wd, const void *s_wg, const void *s_wu, const void *s_wd,
+                         const float *scales, const int32_t *force_ids, double *y,
+                         int32_t *topk_ids, double *topk_w, double *probs, double *gate_out)
 {
     if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || I <= 0 || I_s < 0) return 1;
+    if (norm_w && !(eps >= 0.0)) return 1;
     if (w_dt == ODT_E4M3 && !scales) return 1;
     if (force_ids)
         for (int64_t i = 0; i < T * k; ++i)
@@ -318,7 +370,19 @@ int oracle_moe_forward(int64_t T, int d, int E, int k, int I, int I_s, int act_d
         double *p = (double *)malloc(sizeof(double) * (size_t)E);
         double *h = (double *)malloc(sizeof(double) * (size_t)Imax);
         double *o = (double *)malloc(sizeof(double) * (size_t)d);
-        for (int j = 0; j < d; ++j) xt[j] = elem(x, act_dt, t * d + j);
+        if (norm_w) {
+            rmsnorm_row(d, x, act_dt, t, norm_w, eps, xt);
+            for (int j = 0; j < d; ++j) xt[j] = round_act(xt[j], act_dt);
+        } else {
+            for (int j = 0; j < d; ++j) xt[j] = elem(x, act_dt, t * d + j);
+        }
+        double sgate = 1.0;
+        if (gate_w) {
+            double z = 0.0;
+            for (int j = 0; j < d; ++j) z += xt[j] * elem(gate_w, act_dt, j);
+            sgate = 1.0 / (1.0 + exp(-z));
+        }
+        if (gate_out) gate_out[t] = sgate;
         for (int e = 0; e < E; ++e) {
             double acc = 0.0;
             for (int j = 0; j < d; ++j) acc += xt[j] * elem(w_r, act_dt, (int64_t)e * d + j);
@@ -330,7 +394,7 @@ int oracle_moe_forward(int64_t T, int d, int E, int k, int I, int I_s, int act_d
         for (int c = 0; c < d; ++c) y[t * d + c] = 0.0;
         for (int s = 0; s <= k; ++s) {
             int g = s < k ? topk_ids[t * k + s] : E;
-            double wgt = s < k ? topk_w[t * k + s] : 1.0;
+            double wgt = s < k ? topk_w[t * k + s] : sgate;
             const void *pp[3];
             const float *ss[3];
             int Ig;
@@ -346,6 +410,16 @@ int oracle_moe_forward(int64_t T, int d, int E, int k, int I, int I_s, int act_d
         free(o);
     }
     return 0;
+}
+
+int oracle_moe_forward(int64_t T, int d, int E, int k, int I, int I_s, int act_dt, int w_dt,
+                       const void *x, const void *w_r, const float *bias, const void *wg,
+                       const void *wu, const void *wd, const void *s_wg, const void *s_wu,
+                       const void *s_wd, const float *scales, const int32_t *force_ids, double *y,
+                       int32_t *topk_ids, double *topk_w, double *probs)
+{
+    return oracle_block_forward(T, d, E, k, I, I_s, act_dt, w_dt, x, NULL, 0.0, NULL, w_r, bias, wg, wu,
+                                wd, s_wg, s_wu, s_wd, scales, force_ids, y, topk_ids, topk_w, probs, NULL);
 }
 
 /* Expert stage on dispatched rows: group g's rows offs[g] .. offs[g+1]-1 of

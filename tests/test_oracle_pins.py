@@ -330,3 +330,64 @@ def test_fp8_packed_scale_layout_in_the_whole_block():
         ref = _np_expert(x[t:t + 1], deq(inp.wg[e], sg[e]), deq(inp.wu[e], su[e]), deq(inp.wd[e], sd[e]))
         ref += _np_expert(x[t:t + 1], deq(inp.s_wg, ssg), deq(inp.s_wu, ssu), deq(inp.s_wd, ssd))
         np.testing.assert_allclose(y[t], ref[0], rtol=1e-11, atol=1e-13)
+
+
+# --------------------------------------------------------------------------
+# The block's neighbours: zero-centred RMSNorm prologue, shared-expert gate.
+# --------------------------------------------------------------------------
+def test_rmsnorm_closed_form():
+    # mean of squares of (3, 4) is 25/2, so the row is divided by 5/sqrt(2)
+    out = oracle.rmsnorm(torch.tensor([[3.0, 4.0]]), torch.zeros(2), eps=0.0)
+    np.testing.assert_allclose(out[0], [3 * math.sqrt(2) / 5, 4 * math.sqrt(2) / 5], rtol=1e-15)
+
+
+def test_rmsnorm_zero_centred_scale():
+    # the applied scale is 1 + gamma: gamma = -1 silences a channel, gamma = 1 doubles it
+    x = torch.tensor([[3.0, 4.0, -12.0]])
+    base = oracle.rmsnorm(x, torch.zeros(3), eps=0.0)
+    out = oracle.rmsnorm(x, torch.tensor([-1.0, 1.0, 0.5]), eps=0.0)
+    np.testing.assert_allclose(out[0], [0.0, 2 * base[0, 1], 1.5 * base[0, 2]], rtol=1e-15)
+
+
+def test_rmsnorm_is_scale_invariant_and_unit_rms():
+    x = torch.randn(7, 64, generator=torch.Generator().manual_seed(3))
+    a = oracle.rmsnorm(x, torch.zeros(64), eps=0.0)
+    b = oracle.rmsnorm(x * 4.0, torch.zeros(64), eps=0.0)
+    np.testing.assert_allclose(a, b, rtol=1e-14)
+    np.testing.assert_allclose((a * a).mean(axis=1), 1.0, rtol=1e-13)
+    # eps keeps an all-zero row finite (and zero)
+    z = oracle.rmsnorm(torch.zeros(1, 8), torch.zeros(8), eps=1e-6)
+    assert np.all(z == 0.0)
+
+
+def test_block_with_norm_is_the_block_on_the_normalised_rounded_input():
+    inp = moe_inputs.make_inputs(9, 64, 6, 2, 32, 32, act="bf16", w="bf16", seed=4)
+    gamma = (torch.randn(64, generator=torch.Generator().manual_seed(5)) * 0.1).to(torch.bfloat16)
+    # numpy RMSNorm, rounded by torch's float -> bf16 conversion
+    x = inp.x.double().numpy()
+    xn = x / np.sqrt((x * x).mean(axis=1, keepdims=True) + 1e-6) * (1.0 + gamma.double().numpy())
+    xn_bf16 = torch.from_numpy(xn).float().to(torch.bfloat16)
+    y, ids, w, _, gate = oracle.block_forward(inp.x, inp.w_r, inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu,
+                                              inp.s_wd, inp.k, norm_weight=gamma, norm_eps=1e-6)
+    y2, ids2, w2, _ = oracle.moe_forward(xn_bf16, inp.w_r, inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu,
+                                         inp.s_wd, inp.k)
+    assert np.array_equal(ids, ids2)
+    np.testing.assert_allclose(y, y2, rtol=1e-12, atol=1e-14)
+    assert np.all(gate == 1.0)
+
+
+def test_shared_gate_weights_the_shared_expert_linearly():
+    inp = _tiny(T=8, d=8, E=5, k=2, I=4, I_s=3, seed=6)
+    gw = torch.randn(8, generator=torch.Generator().manual_seed(7)) * 0.3
+    y_full, ids, _, _ = _fwd(inp)
+    y_routed, ids0, _, _ = oracle.moe_forward(inp.x, inp.w_r, inp.wg, inp.wu, inp.wd, None, None, None, inp.k)
+    y, ids1, _, _, gate = oracle.block_forward(inp.x, inp.w_r, inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu,
+                                               inp.s_wd, inp.k, shared_gate=gw)
+    assert np.array_equal(ids, ids0) and np.array_equal(ids, ids1)
+    g = 1.0 / (1.0 + np.exp(-(inp.x.double().numpy() @ gw.double().numpy())))
+    np.testing.assert_allclose(gate, g, rtol=1e-14)
+    np.testing.assert_allclose(y, y_routed + g[:, None] * (y_full - y_routed), rtol=1e-11, atol=1e-12)
+    # a zero gate vector halves the shared expert
+    _, _, _, _, half = oracle.block_forward(inp.x, inp.w_r, inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu,
+                                            inp.s_wd, inp.k, shared_gate=torch.zeros(8))
+    assert np.all(half == 0.5)
