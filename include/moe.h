@@ -90,7 +90,7 @@ typedef struct {
 MOE_API moe_status moe_check_problem(const moe_problem* p);
 
 /* Bytes of device workspace the calls below need (0 for an invalid problem).
- * moe_workspace_size covers moe_layer_forward; moe_stage_workspace_size
+ * moe_workspace_size covers moe_layer_forward and moe_block_forward; moe_stage_workspace_size
  * covers moe_permute and moe_expert_ffn.  Pure host functions. */
 MOE_API size_t moe_workspace_size(const moe_problem* p);
 MOE_API size_t moe_stage_workspace_size(const moe_problem* p);
@@ -143,6 +143,42 @@ MOE_API moe_status moe_layer_forward(const moe_problem* p, const void* x, const 
                              const void* ws_down, const float* scales, void* y,
                              int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes,
                              void* stream);
+
+/* The block's neighbours on its input (Qwen3-Next story page: the models use
+ * a "zero-centred" RMSNorm whose parameters start at zero, so the applied
+ * scale is 1 + gamma; Architecture page, config.json: rms_norm_eps = 1e-6).
+ *   norm_weight  gamma [d] in the activation type, 16-byte aligned, or NULL:
+ *                x_n = x / sqrt(mean_j x_j^2 + norm_eps) * (1 + gamma), stored
+ *                in the activation type, is the input of the router and the
+ *                experts (sums in fp32);
+ *   norm_eps     >= 0 and finite (1e-6 for the Qwen3.x configs);
+ *   shared_gate  w [d] in the activation type, 16-byte aligned, or NULL: the
+ *                shared expert's output is weighted by sigmoid(x_n . w)
+ *                instead of 1.  The pages do not describe such a gate; some
+ *                implementations of this block carry one.  Ignored when
+ *                I_s == 0. */
+typedef struct {
+  const void* norm_weight;
+  float norm_eps;
+  const void* shared_gate;
+} moe_block_options;
+
+/* moe_layer_forward with the options above (opt NULL: exactly
+ * moe_layer_forward).  Same arguments and workspace otherwise; x is the
+ * block's input before the norm. */
+MOE_API moe_status moe_block_forward(const moe_problem* p, const moe_block_options* opt, const void* x,
+                             const void* w_router, const float* router_bias, const void* w_gate,
+                             const void* w_up, const void* w_down, const void* ws_gate,
+                             const void* ws_up, const void* ws_down, const float* scales, void* y,
+                             int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes,
+                             void* stream);
+
+/* The zero-centred RMSNorm of moe_block_options as a stage: x_out [T, d] =
+ * x / sqrt(mean_j x_j^2 + eps) * (1 + norm_weight), in the activation type
+ * (sums in fp32).  norm_weight [d] in the activation type; x, norm_weight and
+ * x_out 16-byte aligned; eps >= 0 and finite. */
+MOE_API moe_status moe_rmsnorm(const moe_problem* p, const void* x, const void* norm_weight, float eps,
+                       void* x_out, void* stream);
 
 /* moe_router_topk for callers that cannot allocate device memory: code that
  * runs where cudaMalloc is off limits (inside a host framework that owns every

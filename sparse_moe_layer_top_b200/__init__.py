@@ -15,7 +15,8 @@ import os
 
 import torch
 
-__all__ = ["MoEError", "Problem", "router_topk", "permute", "expert_ffn", "combine", "layer_forward",
+__all__ = ["MoEError", "Problem", "BlockOptions", "router_topk", "permute", "expert_ffn", "combine", "layer_forward",
+           "block_forward", "rmsnorm",
            "workspace_size", "stage_workspace_size", "set_path", "device_status", "last_launch_count",
            "profile_enable", "profile_read",
            "MoELayer", "lib_path", "F32", "BF16", "FP8_E4M3_B128"]
@@ -29,7 +30,7 @@ _STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "
 EXPORTS = ("moe_check_problem", "moe_workspace_size", "moe_stage_workspace_size", "moe_router_topk",
            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_set_path",
            "moe_device_status", "moe_last_launch_count", "moe_profile_enable", "moe_profile_read",
-           "moe_last_error_string", "moe_router_topk_static")
+           "moe_last_error_string", "moe_router_topk_static", "moe_block_forward", "moe_rmsnorm")
 
 
 class MoEError(RuntimeError):
@@ -47,6 +48,10 @@ class Problem(ctypes.Structure):
     def make(cls, T, d, E, k, I, I_s, act="bf16", w="bf16"):
         codes = {"f32": F32, "bf16": BF16, "fp8": FP8_E4M3_B128}
         return cls(int(T), int(d), int(E), int(k), int(I), int(I_s), codes[act], codes[w])
+
+
+class BlockOptions(ctypes.Structure):
+    _fields_ = [("norm_weight", ctypes.c_void_p), ("norm_eps", ctypes.c_float), ("shared_gate", ctypes.c_void_p)]
 
 
 _lib = None
@@ -71,6 +76,9 @@ def lib():
         L.moe_expert_ffn.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_combine.argtypes = [PP, P, P, P, P, P, P]
         L.moe_layer_forward.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.moe_block_forward.argtypes = [PP, ctypes.POINTER(BlockOptions), P, P, P, P, P, P, P, P, P, P, P, P, P,
+                                        P, ctypes.c_size_t, P]
+        L.moe_rmsnorm.argtypes = [PP, P, P, ctypes.c_float, P, P]
         L.moe_set_path.argtypes = [ctypes.c_int]
         L.moe_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32)]
         L.moe_last_launch_count.restype = ctypes.c_int
@@ -81,7 +89,7 @@ def lib():
         L.moe_profile_read.restype = ctypes.c_int
         L.moe_last_error_string.restype = ctypes.c_char_p
         for f in ("moe_check_problem", "moe_router_topk", "moe_router_topk_static", "moe_permute", "moe_expert_ffn", "moe_combine",
-                  "moe_layer_forward", "moe_set_path", "moe_device_status"):
+                  "moe_layer_forward", "moe_block_forward", "moe_rmsnorm", "moe_set_path", "moe_device_status"):
             getattr(L, f).restype = S
         _lib = L
     return _lib
@@ -225,13 +233,39 @@ def layer_forward(prob, x, w_router, bias, wg, wu, wd, s_wg=None, s_wu=None, s_w
     return y
 
 
+def block_forward(prob, x, w_router, bias, wg, wu, wd, s_wg=None, s_wu=None, s_wd=None, scales=None,
+                  norm_weight=None, norm_eps=1e-6, shared_gate=None, y=None, topk_ids=None, topk_w=None, ws=None,
+                  stream=None):
+    """layer_forward with the block's neighbours: zero-centred RMSNorm of x
+    (norm_weight [d]) and a sigmoid gate on the shared expert (shared_gate [d])."""
+    if y is None:
+        y = torch.empty((prob.T, prob.d), dtype=_act(prob), device=x.device)
+    ws = _ws(workspace_size(prob), x.device, ws)
+    opt = BlockOptions(_ptr(norm_weight), float(norm_eps), _ptr(shared_gate))
+    _check(lib().moe_block_forward(ctypes.byref(prob), ctypes.byref(opt), _ptr(x), _ptr(w_router), _ptr(bias),
+                                   _ptr(wg), _ptr(wu), _ptr(wd), _ptr(s_wg), _ptr(s_wu), _ptr(s_wd), _ptr(scales),
+                                   _ptr(y), _ptr(topk_ids), _ptr(topk_w), _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def rmsnorm(prob, x, norm_weight, eps=1e-6, out=None, stream=None):
+    """Zero-centred RMSNorm of the rows of x: x / sqrt(mean x^2 + eps) * (1 + norm_weight)."""
+    if out is None:
+        out = torch.empty_like(x)
+    _check(lib().moe_rmsnorm(ctypes.byref(prob), _ptr(x), _ptr(norm_weight), float(eps), _ptr(out),
+                             _stream(stream)))
+    return out
+
+
 class MoELayer:
     """One block's weights plus a workspace sized for up to `max_tokens` tokens."""
 
     def __init__(self, d, E, k, I, I_s, w_router, wg, wu, wd, s_wg=None, s_wu=None, s_wd=None, bias=None,
-                 scales=None, act="bf16", w="bf16", max_tokens=0):
+                 scales=None, act="bf16", w="bf16", max_tokens=0, norm_weight=None, norm_eps=1e-6,
+                 shared_gate=None):
         self.shape = (d, E, k, I, I_s, act, w)
         self.w = (w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales)
+        self.opts = (norm_weight, norm_eps, shared_gate)
         self.device = wg.device
         self.ws = None
         if max_tokens:
@@ -250,8 +284,13 @@ class MoELayer:
         prob = self.problem(x.shape[0])
         self._reserve(x.shape[0])
         w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales = self.w
-        return layer_forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, y=y,
-                             topk_ids=topk_ids, topk_w=topk_w, ws=self.ws, stream=stream)
+        norm_weight, norm_eps, shared_gate = self.opts
+        if norm_weight is None and shared_gate is None:
+            return layer_forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, y=y,
+                                 topk_ids=topk_ids, topk_w=topk_w, ws=self.ws, stream=stream)
+        return block_forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, norm_weight=norm_weight,
+                             norm_eps=norm_eps, shared_gate=shared_gate, y=y, topk_ids=topk_ids, topk_w=topk_w,
+                             ws=self.ws, stream=stream)
 
     @classmethod
     def from_inputs(cls, inp, max_tokens=0):

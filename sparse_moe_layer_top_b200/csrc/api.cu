@@ -13,6 +13,7 @@
 #include "../../include/moe.h"
 #include "common.cuh"
 #include "permute.cuh"
+#include "prologue.cuh"
 #include "router.cuh"
 #include "simt.cuh"
 #include "tc_gemm.cuh"
@@ -361,7 +362,7 @@ static RouterSplit router_split(const moe_problem& p) {
 
 struct Layout {
   size_t counts = 0, pre_a = 0, pre_b = 0, part = 0, ids = 0, tw = 0, offs = 0, row_tok = 0, row_w = 0, pos = 0,
-         row_dst = 0, xp = 0, h = 0, total = 0;
+         row_dst = 0, xp = 0, xn = 0, gate = 0, h = 0, total = 0;
 };
 
 static int64_t rows_total(const moe_problem& p) { return p.T * p.k + (p.I_s > 0 ? p.T : 0); }
@@ -398,6 +399,8 @@ static Layout layout(const moe_problem& p, bool forward) {
     L.pos = take(n * 4);
     L.row_dst = take(Rp * 4);
     L.xp = take(std::max(Rp, p.T * (p.k + 1)) * p.d * ab);
+    L.xn = take(p.T * p.d * ab);  // the normalised block input (moe_block_forward with a norm)
+    L.gate = take(p.T * 4);       // the shared expert's gate per token
   }
   L.h = take(Rp * ldh_of(p) * ab);
   L.total = o;
@@ -470,7 +473,7 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
 static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, const float* tw, bool counted,
                                   int32_t* offs, int32_t* row_tok, float* row_w, int32_t* pos, int32_t* row_dst,
                                   int32_t* counts, Schedule sa, int32_t* pre_a, Schedule sb, int32_t* pre_b,
-                                  cudaStream_t st, DeviceInfo* dev) {
+                                  cudaStream_t st, DeviceInfo* dev, const float* shared_gate = nullptr) {
   const int nch = (int)n_chunks(p);
   if (p.T == 0) {
     CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)p.E * 4, st));
@@ -481,7 +484,7 @@ static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, cons
   }
   PROF_BEGIN("dispatch", st);
   k_dispatch<<<nch, kScatterWarps * 32, 0, st>>>(ids, tw, p.T, p.k, p.E, counts, nch, p.I_s > 0, offs, sa, pre_a, sb,
-                                                 pre_b, row_tok, row_w, pos, row_dst);
+                                                 pre_b, row_tok, row_w, pos, row_dst, shared_gate);
   LAUNCH_CHECK("dispatch", st);
   return MOE_OK;
 }
@@ -1067,12 +1070,33 @@ moe_status moe_combine(const moe_problem* p, const void* y_perm, const int32_t* 
   return MOE_OK;
 }
 
-moe_status moe_layer_forward(const moe_problem* p, const void* x, const void* w_router, const float* router_bias,
-                             const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
-                             const void* ws_up, const void* ws_down, const float* scales, void* y,
-                             int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+// Launch the block's input prologue: x_out = zero-centred RMSNorm(x) when
+// gamma is given, gate_out[t] = sigmoid(x_n[t] . gate_w) when gate_w is given.
+static moe_status launch_prologue(const moe_problem& p, const void* x, const void* gamma, float eps,
+                                  const void* gate_w, void* x_out, float* gate_out, cudaStream_t st) {
+  const unsigned grid = (unsigned)cdiv(p.T, 8);
+  PROF_BEGIN("prologue", st);
+  if (p.act_dtype == MOE_F32)
+    k_prologue<float><<<grid, 256, 0, st>>>((const float*)x, (const float*)gamma, eps, (const float*)gate_w, p.T,
+                                            p.d, (float*)x_out, gate_out);
+  else
+    k_prologue<bf16><<<grid, 256, 0, st>>>((const bf16*)x, (const bf16*)gamma, eps, (const bf16*)gate_w, p.T, p.d,
+                                           (bf16*)x_out, gate_out);
+  LAUNCH_CHECK("prologue", st);
+  return MOE_OK;
+}
+
+static moe_status block_forward(const moe_problem* p, const moe_block_options* opt, const void* x,
+                                const void* w_router, const float* router_bias, const void* w_gate,
+                                const void* w_up, const void* w_down, const void* ws_gate, const void* ws_up,
+                                const void* ws_down, const float* scales, void* y, int32_t* topk_ids_out,
+                                float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
   moe_status s = check(p);
   if (s != MOE_OK) return s;
+  const void* norm_w = opt ? opt->norm_weight : nullptr;
+  const void* gate_w = opt ? opt->shared_gate : nullptr;
+  if (norm_w && !(opt->norm_eps >= 0.f && opt->norm_eps < 1e30f))
+    return fail(MOE_ERR_INVALID_ARG, "norm_eps must be finite and >= 0");
   if (p->T == 0) {
     g_launches = 0;
     return MOE_OK;
@@ -1083,6 +1107,8 @@ moe_status moe_layer_forward(const moe_problem* p, const void* x, const void* w_
   NEED(y);
   MAYBE(topk_ids_out);
   MAYBE(topk_w_out);
+  MAYBE(norm_w);
+  MAYBE(gate_w);
   NEED(ws);
   ExpertWeights w{w_gate, w_up, w_down, ws_gate, ws_up, ws_down, scales};
   if ((s = check_weights(*p, w)) != MOE_OK) return s;
@@ -1107,14 +1133,25 @@ moe_status moe_layer_forward(const moe_problem* p, const void* x, const void* w_
   int32_t* pre_a = (int32_t*)(wsp + L.pre_a);
   int32_t* pre_b = (int32_t*)(wsp + L.pre_b);
   void* xp = wsp + L.xp;
+  // the block's input: x, or its zero-centred RMSNorm; the shared expert's
+  // gate (only where there is a shared expert to weight)
+  const void* xin = x;
+  float* gate = (gate_w && p->I_s > 0) ? (float*)(wsp + L.gate) : nullptr;
+  if (norm_w || gate) {
+    if ((s = launch_prologue(*p, x, norm_w, norm_w ? opt->norm_eps : 0.f, gate ? gate_w : nullptr, wsp + L.xn, gate,
+                             st)) != MOE_OK)
+      return s;
+    if (norm_w) xin = wsp + L.xn;
+  }
   bool counted;
-  s = launch_router(*p, x, w_router, router_bias, ids, tw, (float*)(wsp + L.part), counts, &counted, st, dev);
+  s = launch_router(*p, xin, w_router, router_bias, ids, tw, (float*)(wsp + L.part), counts, &counted, st, dev);
   if (s != MOE_OK) return s;
   Schedule sa, sb;
   schedules(*p, form, &sa, &sb);
-  s = launch_dispatch(*p, ids, tw, counted, offs, row_tok, row_w, pos, row_dst, counts, sa, pre_a, sb, pre_b, st, dev);
+  s = launch_dispatch(*p, ids, tw, counted, offs, row_tok, row_w, pos, row_dst, counts, sa, pre_a, sb, pre_b, st, dev,
+                      gate);
   if (s != MOE_OK) return s;
-  if ((s = launch_gather(*p, x, row_tok, offs, xp, st, dev)) != MOE_OK) return s;
+  if ((s = launch_gather(*p, xin, row_tok, offs, xp, st, dev)) != MOE_OK) return s;
   DownOut o{xp, row_dst, row_w, nullptr};  // the slot rows reuse the dispatched-row buffer
   s = expert_gemms(*p, form, xp, offs, w, pre_a, pre_b, wsp + L.h, o, st, dev);
   if (s != MOE_OK) return s;
@@ -1124,6 +1161,42 @@ moe_status moe_layer_forward(const moe_problem* p, const void* x, const void* w_
   else
     k_slot_sum<bf16><<<(unsigned)p->T, 256, 0, st>>>((const bf16*)xp, pos, p->k, p->I_s > 0, p->d, (bf16*)y);
   LAUNCH_CHECK("slot_sum", st);
+  g_launches = g_launches_pending;
+  return MOE_OK;
+}
+
+moe_status moe_layer_forward(const moe_problem* p, const void* x, const void* w_router, const float* router_bias,
+                             const void* w_gate, const void* w_up, const void* w_down, const void* ws_gate,
+                             const void* ws_up, const void* ws_down, const float* scales, void* y,
+                             int32_t* topk_ids_out, float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  return block_forward(p, nullptr, x, w_router, router_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, scales, y,
+                       topk_ids_out, topk_w_out, ws, ws_bytes, stream);
+}
+
+moe_status moe_block_forward(const moe_problem* p, const moe_block_options* opt, const void* x,
+                             const void* w_router, const float* router_bias, const void* w_gate, const void* w_up,
+                             const void* w_down, const void* ws_gate, const void* ws_up, const void* ws_down,
+                             const float* scales, void* y, int32_t* topk_ids_out, float* topk_w_out, void* ws,
+                             size_t ws_bytes, void* stream) {
+  return block_forward(p, opt, x, w_router, router_bias, w_gate, w_up, w_down, ws_gate, ws_up, ws_down, scales, y,
+                       topk_ids_out, topk_w_out, ws, ws_bytes, stream);
+}
+
+moe_status moe_rmsnorm(const moe_problem* p, const void* x, const void* norm_weight, float eps, void* x_out,
+                       void* stream) {
+  moe_status s = check(p);
+  if (s != MOE_OK) return s;
+  if (!(eps >= 0.f && eps < 1e30f)) return fail(MOE_ERR_INVALID_ARG, "eps must be finite and >= 0");
+  if (p->T == 0) {
+    g_launches = 0;
+    return MOE_OK;
+  }
+  NEED(x);
+  NEED(norm_weight);
+  NEED(x_out);
+  g_launches_pending = 0;
+  if ((s = launch_prologue(*p, x, norm_weight, eps, nullptr, x_out, nullptr, (cudaStream_t)stream)) != MOE_OK)
+    return s;
   g_launches = g_launches_pending;
   return MOE_OK;
 }

@@ -114,7 +114,8 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
     const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int64_t T, int k, int E,
     const int32_t* __restrict__ counts, int nchunks, int has_shared, int32_t* __restrict__ offs, Schedule sa,
     int32_t* __restrict__ prefix_a, Schedule sb, int32_t* __restrict__ prefix_b, int32_t* __restrict__ row_tok,
-    float* __restrict__ row_w, int32_t* __restrict__ pos, int32_t* __restrict__ row_dst) {
+    float* __restrict__ row_w, int32_t* __restrict__ pos, int32_t* __restrict__ row_dst,
+    const float* __restrict__ shared_gate) {
   __shared__ int32_t wb[kScatterWarps][kMaxE];
   __shared__ int32_t s_base[kMaxE];
   __shared__ int sm_warp[32];
@@ -226,7 +227,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
     for (int64_t t = (int64_t)c * kChunkTokens + threadIdx.x; t < min(T, (int64_t)(c + 1) * kChunkTokens);
          t += blockDim.x) {
       row_tok[R + t] = (int32_t)t;
-      row_w[R + t] = 1.0f;
+      row_w[R + t] = shared_gate ? __ldg(shared_gate + t) : 1.0f;  // the shared expert's weight
       if (row_dst) row_dst[R + t] = (int32_t)(t * (k + 1) + k);
     }
   }

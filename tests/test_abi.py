@@ -92,3 +92,27 @@ def test_set_path_validates():
     assert moe.lib().moe_set_path(5) == 1
     assert moe.lib().moe_set_path(-1) == 1
     assert moe.lib().moe_set_path(0) == 0
+
+
+def _call_block(prob, norm=None, eps=1e-6, gate=None, x=16):
+    L = moe.lib()
+    v = lambda a: None if a is None else ctypes.c_void_p(a)
+    opt = moe.BlockOptions(norm, eps, gate)
+    return L.moe_block_forward(ctypes.byref(prob), ctypes.byref(opt), v(x), v(16), None, v(16), v(16), v(16),
+                               v(16), v(16), v(16), None, v(16), None, None, v(16), moe.workspace_size(prob), None)
+
+
+def test_block_options_rejected_before_any_launch():
+    prob = P()
+    # every case below fails on the host (fake addresses are never dereferenced)
+    assert _call_block(prob, norm=0x1008) == 3          # misaligned norm weight
+    assert _call_block(prob, gate=0x1008) == 3          # misaligned gate weight
+    assert _call_block(prob, norm=16, eps=-1.0) == 1    # negative eps
+    assert _call_block(prob, norm=16, eps=float("nan")) == 1
+    assert _call_block(prob, norm=16, x=None) == 1      # no input
+    L = moe.lib()
+    v = ctypes.c_void_p
+    assert L.moe_rmsnorm(ctypes.byref(prob), v(16), None, 1e-6, v(16), None) == 1
+    assert L.moe_rmsnorm(ctypes.byref(prob), v(16), v(16), -1.0, v(16), None) == 1
+    assert L.moe_rmsnorm(ctypes.byref(prob), v(16), v(0x1008), 1e-6, v(16), None) == 3
+    assert L.moe_rmsnorm(ctypes.byref(P(d=100)), v(16), v(16), 1e-6, v(16), None) == 3
