@@ -35,6 +35,7 @@ UNIT = "tokens/s"
 DEFAULT_CONFIG = "qwen36_35b_a3b_bf16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
+LONG_RUN_MS = 100.0  # timed regions at least this long use the sustained tensor peak
 # The files that define each timed kernel (its template, the PTX wrappers it
 # uses, its launch configuration): an ncu traffic figure stays valid while
 # their contents hash to the value recorded with it.
@@ -363,13 +364,22 @@ def run_ours(args):
             tc_t = wk["flops"] / (peaks["bf16_tflops"] * 1e12)
             if hbm_t >= tc_t:
                 roof = {"bound": "hbm", "achieved": wk["bytes"] / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+                which = ""
             else:
-                roof = {"bound": "tensor", "achieved": wk["flops"] / t_s / 1e12, "peak": peaks["bf16_tflops"],
-                        "unit": "TFLOP/s"}
+                # A tensor-bound kernel timed inside a long run of steps (the
+                # power cap engages within tens of milliseconds) is held to the
+                # sustained dense-GEMM figure, one timed alone to the burst figure;
+                # both fractions are reported.
+                long_run = step_ms * K >= LONG_RUN_MS
+                burst, sust = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+                ach = wk["flops"] / t_s / 1e12
+                roof = {"bound": "tensor", "achieved": ach, "peak": sust if long_run else burst, "unit": "TFLOP/s",
+                        "frac_burst": ach / burst, "frac_sustained": ach / sust}
+                which = " (sustained: %.0f ms timed)" % (step_ms * K) if long_run else " (burst)"
             roof["frac"] = roof["achieved"] / roof["peak"]
             roof["traffic"] = load_traffic(dom, args.config)
             roof.update({"kernel": dom, "kernel_ms": kern[dom], "algorithmic_bytes": wk["bytes"],
-                         "algorithmic_flops": wk["flops"], "peak_source": peak_src + " (burst)"})
+                         "algorithmic_flops": wk["flops"], "peak_source": peak_src + which})
         lw = work["layer"]
         st = step_ms / 1e3
         layer_roof = {"bytes": lw["bytes"], "flops": lw["flops"],
