@@ -1,0 +1,45 @@
+"""The fused forward inside a CUDA graph: the library's calls only enqueue
+work on the caller's stream (no synchronisation, no allocation), so one
+forward can be captured once and replayed; the replay must give the eager
+result bit for bit, on each expert-GEMM form."""
+import pytest
+import torch
+
+import moe_inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("path,w,E", [(2, "bf16", 20), (3, "bf16", 64), (4, "bf16", 2), (0, "fp8", 12)])
+def test_forward_replays_from_a_cuda_graph(path, w, E):
+    import sparse_moe_layer_top_b200 as moe
+    T, d, k, I, I_s = (2048, 256, 2, 256, 128) if E == 2 else (300, 384, 3, 256, 128)
+    inp = moe_inputs.make_inputs(T, d, E, k, I, I_s, act="bf16", w=w, seed=8, device="cuda")
+    moe.set_path(path)
+    try:
+        layer = moe.MoELayer.from_inputs(inp, max_tokens=T)
+        y_eager = layer(inp.x)
+        torch.cuda.synchronize()
+        x = inp.x.clone()
+        y = torch.empty_like(y_eager)
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            layer(x, y, stream=s)  # warm-up on the capture stream (device set-up, tensor maps)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            layer(x, y, stream=s)
+        y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, y_eager)
+        # a new input in the same buffer flows through the replay
+        x.copy_(inp.x.flip(0))
+        g.replay()
+        torch.cuda.synchronize()
+        assert torch.equal(y, layer(inp.x.flip(0).contiguous()))
+        status, detail = moe.device_status()
+        assert status == 0, hex(detail)
+    finally:
+        moe.set_path(0)
