@@ -92,6 +92,32 @@ static void prof_end(const char* name, cudaStream_t st) {
     ++g_launches_pending;                                                                    \
   } while (0)
 
+// Kernel launch.  Every launch of a library call after its first carries the
+// programmatic-serialisation attribute: the kernel may be scheduled while the
+// previous one finishes, runs its set-up, and waits for it (griddepcontrol.wait)
+// before touching its results -- every kernel of the library does.  The first
+// launch of a call (whose predecessor may be the caller's own kernel) and the
+// first after a memset go in plain stream order.
+static thread_local bool g_pdl_next = false;
+static void pdl_reset() { g_pdl_next = false; }
+
+template <typename... KArgs, typename... Args>
+static cudaError_t launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                          Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = g_pdl_next ? 1 : 0;
+  g_pdl_next = true;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // ============================================================== device state
 // The device status word: kernels record a rejected input or a wait that gave
 // up; moe_device_status() reads and clears it.
@@ -134,13 +160,16 @@ static cudaError_t launch_pair(K kernel, int ctas, int threads, int smem, cudaSt
   cfg.blockDim = dim3((unsigned)threads);
   cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = st;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 2;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = at;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = g_pdl_next ? 2 : 1;
+  g_pdl_next = true;
   return cudaLaunchKernelEx(&cfg, kernel, a0, a1, b0, b1, c0, c1, args);
 }
 
@@ -427,10 +456,10 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
     const int npl = select_npl(p.E);
     if (p.act_dtype == MOE_F32) {
       auto kf = npl == 4 ? k_router_simt<float, 4> : npl == 8 ? k_router_simt<float, 8> : k_router_simt<float, 16>;
-      kf<<<grid, 256, 0, st>>>((const float*)x, (const float*)wr, bias, p.T, p.d, p.E, p.k, ids, tw);
+      CUDA_TRY(launch(kf, grid, 256, 0, st, (const float*)x, (const float*)wr, bias, p.T, p.d, p.E, p.k, ids, tw));
     } else {
       auto kb = npl == 4 ? k_router_simt<bf16, 4> : npl == 8 ? k_router_simt<bf16, 8> : k_router_simt<bf16, 16>;
-      kb<<<grid, 256, 0, st>>>((const bf16*)x, (const bf16*)wr, bias, p.T, p.d, p.E, p.k, ids, tw);
+      CUDA_TRY(launch(kb, grid, 256, 0, st, (const bf16*)x, (const bf16*)wr, bias, p.T, p.d, p.E, p.k, ids, tw));
     }
     LAUNCH_CHECK("router_simt", st);
     return MOE_OK;
@@ -452,16 +481,19 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
   a.ldp = rs.ldp;
   a.part_stride = p.T * rs.ldp;
   a.status = dev->status;
+  if (counts) {  // the chunk histograms k_topk counts into
+    CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * p.E * 4, st));
+    pdl_reset();
+  }
   PROF_BEGIN("gemm_tc_router", st);
-  k_gemm_tc<kRouterBN, false, 4, kTcLogits>
-      <<<std::min(rs.tiles, dev->sms), Gemm2Cfg::THREADS, Gemm2Cfg::SMEM_BYTES, st>>>(ax, ax, bw, bw, bw, bw, a);
+  CUDA_TRY(launch(k_gemm_tc<kRouterBN, false, 4, kTcLogits>, std::min(rs.tiles, dev->sms), Gemm2Cfg::THREADS,
+                  Gemm2Cfg::SMEM_BYTES, st, ax, ax, bw, bw, bw, bw, a));
   LAUNCH_CHECK("gemm_tc_router", st);
-  if (counts) CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * p.E * 4, st));
   PROF_BEGIN("topk", st);
   const int npl = select_npl(p.E);
   auto kt = npl == 4 ? k_topk<4> : npl == 8 ? k_topk<8> : k_topk<16>;
-  kt<<<(unsigned)cdiv(p.T, 8), 256, 0, st>>>(part, rs.ksplit, p.T * rs.ldp, rs.ldp, bias, p.T, p.E, p.k, ids, tw,
-                                             counts);
+  CUDA_TRY(launch(kt, (unsigned)cdiv(p.T, 8), 256, 0, st, part, rs.ksplit, p.T * rs.ldp, rs.ldp, bias, p.T, p.E, p.k,
+                  ids, tw, counts));
   LAUNCH_CHECK("topk", st);
   *counted = counts != nullptr;
   return MOE_OK;
@@ -477,14 +509,15 @@ static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, cons
   const int nch = (int)n_chunks(p);
   if (p.T == 0) {
     CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)p.E * 4, st));
+    pdl_reset();
   } else if (!counted) {
     PROF_BEGIN("count", st);
-    k_count<<<nch, 256, 0, st>>>(ids, p.T, p.k, p.E, counts, dev->status);
+    CUDA_TRY(launch(k_count, nch, 256, 0, st, ids, p.T, p.k, p.E, counts, dev->status));
     LAUNCH_CHECK("count", st);
   }
   PROF_BEGIN("dispatch", st);
-  k_dispatch<<<nch, kScatterWarps * 32, 0, st>>>(ids, tw, p.T, p.k, p.E, counts, nch, p.I_s > 0, offs, sa, pre_a, sb,
-                                                 pre_b, row_tok, row_w, pos, row_dst, shared_gate);
+  CUDA_TRY(launch(k_dispatch, nch, kScatterWarps * 32, 0, st, ids, tw, p.T, p.k, p.E, counts, nch,
+                  p.I_s > 0, offs, sa, pre_a, sb, pre_b, row_tok, row_w, pos, row_dst, shared_gate));
   LAUNCH_CHECK("dispatch", st);
   return MOE_OK;
 }
@@ -496,7 +529,7 @@ static moe_status launch_gather(const moe_problem& p, const void* x, const int32
   if (rows == 0) return MOE_OK;
   unsigned grid = (unsigned)std::min<int64_t>(cdiv(rows, 8), (int64_t)dev->sms * 8);
   PROF_BEGIN("gather", st);
-  k_gather<<<grid, 256, 0, st>>>((const uint4*)x, row_tok, offs, p.E, p.T, vec, (uint4*)xp);
+  CUDA_TRY(launch(k_gather, grid, 256, 0, st, (const uint4*)x, row_tok, offs, p.E, p.T, vec, (uint4*)xp));
   LAUNCH_CHECK("gather", st);
   return MOE_OK;
 }
@@ -552,7 +585,7 @@ static moe_status simt_gemms(const moe_problem& p, const void* xp, const int32_t
   a.H = (TA*)H;
   a.ldh = ldh_of(p);
   PROF_BEGIN("gemm_simt_swiglu", st);
-  k_gemm_simt<TA, TW, kEpiSwiGLU><<<grid, 256, 0, st>>>(a);
+  CUDA_TRY(launch(k_gemm_simt<TA, TW, kEpiSwiGLU>, grid, 256, 0, st, a));
   LAUNCH_CHECK("gemm_simt_swiglu", st);
   // down: A = H [R', ldh], N = d, K = I (I_s)
   SimtGemmArgs<TA, TW> b{};
@@ -574,13 +607,13 @@ static moe_status simt_gemms(const moe_problem& p, const void* xp, const int32_t
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
     PROF_BEGIN("gemm_simt_slot", st);
-    k_gemm_simt<TA, TW, kEpiSlotStore><<<grid, 256, 0, st>>>(b);
+    CUDA_TRY(launch(k_gemm_simt<TA, TW, kEpiSlotStore>, grid, 256, 0, st, b));
     LAUNCH_CHECK("gemm_simt_slot", st);
   } else {
     b.out = (TA*)o.out;
     b.ldo = p.d;
     PROF_BEGIN("gemm_simt_store", st);
-    k_gemm_simt<TA, TW, kEpiStore><<<grid, 256, 0, st>>>(b);
+    CUDA_TRY(launch(k_gemm_simt<TA, TW, kEpiStore>, grid, 256, 0, st, b));
     LAUNCH_CHECK("gemm_simt_store", st);
   }
   return MOE_OK;
@@ -627,7 +660,8 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   a.sc_c_s = sp[4];
   a.status = dev->status;
   PROF_BEGIN("gemm_tc_swiglu", st);
-  k_gemm_tc<128, true, S, kTcSwiGLU, FP8><<<dev->sms, C1::THREADS, C1::SMEM_BYTES, st>>>(aR, aR, bR, bS, cR, cS, a);
+  CUDA_TRY(launch(k_gemm_tc<128, true, S, kTcSwiGLU, FP8>,
+                  dev->sms, C1::THREADS, C1::SMEM_BYTES, st, aR, aR, bR, bS, cR, cS, a));
   LAUNCH_CHECK("gemm_tc_swiglu", st);
   // down
   if ((s = map2d(&aR, H, p.I, Rp, ldh, kBM)) != MOE_OK) return s;
@@ -655,14 +689,15 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
     PROF_BEGIN("gemm_tc_down", st);
-    k_gemm_tc<256, false, S, kTcSlotStore, FP8>
-        <<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
+    CUDA_TRY(launch(k_gemm_tc<256, false, S, kTcSlotStore, FP8>,
+                    dev->sms, C2::THREADS, C2::SMEM_BYTES, st, aR, aS, bR, bS, bR, bS, b));
     LAUNCH_CHECK("gemm_tc_down", st);
   } else {
     b.out = (bf16*)o.out;
     b.ldo = p.d;
     PROF_BEGIN("gemm_tc_store", st);
-    k_gemm_tc<256, false, S, kTcStore, FP8><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(aR, aS, bR, bS, bR, bS, b);
+    CUDA_TRY(launch(k_gemm_tc<256, false, S, kTcStore, FP8>,
+                    dev->sms, C2::THREADS, C2::SMEM_BYTES, st, aR, aS, bR, bS, bR, bS, b));
     LAUNCH_CHECK("gemm_tc_store", st);
   }
   return MOE_OK;
@@ -716,10 +751,11 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
   a.status = dev->status;
   PROF_BEGIN("gemm_tc_swiglu", st);
   if (FP8)
-    k_gemm_swap8<true, kTcSwiGLU><<<dev->sms, Swap8Cfg<true>::THREADS, Swap8Cfg<true>::SMEM_BYTES, st>>>(
-        xR, xR, bR, bS, cR, cS, a);
+    CUDA_TRY(launch(k_gemm_swap8<true, kTcSwiGLU>,
+                    dev->sms, Swap8Cfg<true>::THREADS, Swap8Cfg<true>::SMEM_BYTES, st, xR, xR, bR, bS, cR, cS, a));
   else
-    k_gemm_swap<true, kTcSwiGLU><<<dev->sms, C1::THREADS, C1::SMEM_BYTES, st>>>(xR, xR, bR, bS, cR, cS, a);
+    CUDA_TRY(launch(k_gemm_swap<true, kTcSwiGLU>,
+                    dev->sms, C1::THREADS, C1::SMEM_BYTES, st, xR, xR, bR, bS, cR, cS, a));
   LAUNCH_CHECK("gemm_tc_swiglu", st);
   // down: W_down [E, d, I] is the M operand, H rows the N operand
   if ((s = map2d(&xR, H, p.I, Rp, ldh, kNCH)) != MOE_OK) return s;
@@ -748,21 +784,22 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
     b.row_w = o.row_w;
     PROF_BEGIN("gemm_tc_down", st);
     if (FP8)
-      k_gemm_swap8<false, kTcSlotStore><<<dev->sms, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st>>>(
-          xR, xS, bR, bS, bR, bS, b);
+      CUDA_TRY(launch(k_gemm_swap8<false, kTcSlotStore>,
+                      dev->sms, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
     else
-      k_gemm_swap<false, kTcSlotStore><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(xR, xS, bR, bS, bR,
-                                                                                            bS, b);
+      CUDA_TRY(launch(k_gemm_swap<false, kTcSlotStore>,
+                      dev->sms, C2::THREADS, C2::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
     LAUNCH_CHECK("gemm_tc_down", st);
   } else {
     b.out = (bf16*)o.out;
     b.ldo = p.d;
     PROF_BEGIN("gemm_tc_store", st);
     if (FP8)
-      k_gemm_swap8<false, kTcStore><<<dev->sms, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st>>>(
-          xR, xS, bR, bS, bR, bS, b);
+      CUDA_TRY(launch(k_gemm_swap8<false, kTcStore>,
+                      dev->sms, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
     else
-      k_gemm_swap<false, kTcStore><<<dev->sms, C2::THREADS, C2::SMEM_BYTES, st>>>(xR, xS, bR, bS, bR, bS, b);
+      CUDA_TRY(launch(k_gemm_swap<false, kTcStore>,
+                      dev->sms, C2::THREADS, C2::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
     LAUNCH_CHECK("gemm_tc_store", st);
   }
   return MOE_OK;
@@ -962,6 +999,7 @@ moe_status moe_router_topk(const moe_problem* p, const void* x, const void* w_ro
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != MOE_OK) return s;
   g_launches_pending = 0;
+  pdl_reset();
   bool counted;
   float* part = ws ? (float*)((char*)ws + L.part) : nullptr;
   s = launch_router(*p, x, w_router, router_bias, topk_ids, topk_w, part, nullptr, &counted, (cudaStream_t)stream,
@@ -992,6 +1030,7 @@ moe_status moe_permute(const moe_problem* p, const void* x, const int32_t* topk_
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != MOE_OK) return s;
   g_launches_pending = 0;
+  pdl_reset();
   cudaStream_t st = (cudaStream_t)stream;
   char* w = (char*)ws;
   s = launch_dispatch(*p, topk_ids, topk_w, false, offs, row_tok, row_w, pos, nullptr, (int32_t*)(w + L.counts),
@@ -1026,6 +1065,7 @@ moe_status moe_expert_ffn(const moe_problem* p, const void* x_perm, const int32_
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != MOE_OK) return s;
   g_launches_pending = 0;
+  pdl_reset();
   cudaStream_t st = (cudaStream_t)stream;
   char* wsp = (char*)ws;
   Schedule sa, sb;
@@ -1033,7 +1073,7 @@ moe_status moe_expert_ffn(const moe_problem* p, const void* x_perm, const int32_
   int32_t* pre_a = (int32_t*)(wsp + L.pre_a);
   int32_t* pre_b = (int32_t*)(wsp + L.pre_b);
   PROF_BEGIN("tile_prefix", st);
-  k_tile_prefix<<<1, 1024, 0, st>>>(offs, p->E, sa, pre_a, sb, pre_b);
+  CUDA_TRY(launch(k_tile_prefix, 1, 1024, 0, st, offs, p->E, sa, pre_a, sb, pre_b));
   LAUNCH_CHECK("tile_prefix", st);
   DownOut o{nullptr, nullptr, nullptr, y_perm};
   s = expert_gemms(*p, form, x_perm, offs, w, pre_a, pre_b, wsp + L.h, o, st, dev);
@@ -1057,14 +1097,15 @@ moe_status moe_combine(const moe_problem* p, const void* y_perm, const int32_t* 
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != MOE_OK) return s;
   g_launches_pending = 0;
+  pdl_reset();
   cudaStream_t st = (cudaStream_t)stream;
   PROF_BEGIN("combine", st);
   if (p->act_dtype == MOE_F32)
-    k_combine<float><<<(unsigned)p->T, 256, 0, st>>>((const float*)y_perm, pos, topk_w, offs, p->E, p->k, p->d, p->T,
-                                                     (float*)y);
+    CUDA_TRY(launch(k_combine<float>, (unsigned)p->T, 256, 0, st, (const float*)y_perm, pos, topk_w, offs, p->E,
+                    p->k, p->d, p->T, (float*)y));
   else
-    k_combine<bf16><<<(unsigned)p->T, 256, 0, st>>>((const bf16*)y_perm, pos, topk_w, offs, p->E, p->k, p->d, p->T,
-                                                    (bf16*)y);
+    CUDA_TRY(launch(k_combine<bf16>, (unsigned)p->T, 256, 0, st, (const bf16*)y_perm, pos, topk_w, offs, p->E,
+                    p->k, p->d, p->T, (bf16*)y));
   LAUNCH_CHECK("combine", st);
   g_launches = g_launches_pending;
   return MOE_OK;
@@ -1077,11 +1118,11 @@ static moe_status launch_prologue(const moe_problem& p, const void* x, const voi
   const unsigned grid = (unsigned)cdiv(p.T, 8);
   PROF_BEGIN("prologue", st);
   if (p.act_dtype == MOE_F32)
-    k_prologue<float><<<grid, 256, 0, st>>>((const float*)x, (const float*)gamma, eps, (const float*)gate_w, p.T,
-                                            p.d, (float*)x_out, gate_out);
+    CUDA_TRY(launch(k_prologue<float>, grid, 256, 0, st, (const float*)x, (const float*)gamma, eps,
+                    (const float*)gate_w, p.T, p.d, (float*)x_out, gate_out));
   else
-    k_prologue<bf16><<<grid, 256, 0, st>>>((const bf16*)x, (const bf16*)gamma, eps, (const bf16*)gate_w, p.T, p.d,
-                                           (bf16*)x_out, gate_out);
+    CUDA_TRY(launch(k_prologue<bf16>, grid, 256, 0, st, (const bf16*)x, (const bf16*)gamma, eps, (const bf16*)gate_w,
+                    p.T, p.d, (bf16*)x_out, gate_out));
   LAUNCH_CHECK("prologue", st);
   return MOE_OK;
 }
@@ -1120,6 +1161,7 @@ static moe_status block_forward(const moe_problem* p, const moe_block_options* o
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != MOE_OK) return s;
   g_launches_pending = 0;
+  pdl_reset();
   cudaStream_t st = (cudaStream_t)stream;
   char* wsp = (char*)ws;
   int32_t* ids = topk_ids_out ? topk_ids_out : (int32_t*)(wsp + L.ids);
@@ -1157,9 +1199,11 @@ static moe_status block_forward(const moe_problem* p, const moe_block_options* o
   if (s != MOE_OK) return s;
   PROF_BEGIN("slot_sum", st);
   if (p->act_dtype == MOE_F32)
-    k_slot_sum<float><<<(unsigned)p->T, 256, 0, st>>>((const float*)xp, pos, p->k, p->I_s > 0, p->d, (float*)y);
+    CUDA_TRY(launch(k_slot_sum<float>,
+                    (unsigned)p->T, 256, 0, st, (const float*)xp, pos, p->k, p->I_s > 0, p->d, (float*)y));
   else
-    k_slot_sum<bf16><<<(unsigned)p->T, 256, 0, st>>>((const bf16*)xp, pos, p->k, p->I_s > 0, p->d, (bf16*)y);
+    CUDA_TRY(launch(k_slot_sum<bf16>,
+                    (unsigned)p->T, 256, 0, st, (const bf16*)xp, pos, p->k, p->I_s > 0, p->d, (bf16*)y));
   LAUNCH_CHECK("slot_sum", st);
   g_launches = g_launches_pending;
   return MOE_OK;
@@ -1195,6 +1239,7 @@ moe_status moe_rmsnorm(const moe_problem* p, const void* x, const void* norm_wei
   NEED(norm_weight);
   NEED(x_out);
   g_launches_pending = 0;
+  pdl_reset();
   if ((s = launch_prologue(*p, x, norm_weight, eps, nullptr, x_out, nullptr, (cudaStream_t)stream)) != MOE_OK)
     return s;
   g_launches = g_launches_pending;
@@ -1249,13 +1294,15 @@ extern "C" moe_status moe_router_topk_static(const moe_problem* p, const void* x
     need = (size_t)rs.ksplit * p->T * rs.ldp * 4;
   }
   if (need > (size_t)MOE_ROUTER_STATIC_SCRATCH_BYTES)
-    return fail(MOE_ERR_UNSUPPORTED, "router needs %zu bytes of scratch; the built-in array holds %zu (use moe_router_topk with a workspace)",
+    return fail(MOE_ERR_UNSUPPORTED,
+                "router needs %zu bytes of scratch; the built-in array holds %zu (use moe_router_topk with a workspace)",
                 need, (size_t)MOE_ROUTER_STATIC_SCRATCH_BYTES);
   DeviceInfo* dev;
   if ((s = device_info(&dev)) != MOE_OK) return s;
   void* scratch = nullptr;
   if ((s = router_scratch(&scratch)) != MOE_OK) return s;
   g_launches_pending = 0;
+  pdl_reset();
   bool counted;
   s = launch_router(*p, x, w_router, router_bias, topk_ids, topk_w, (float*)scratch, nullptr, &counted,
                     (cudaStream_t)stream, dev);

@@ -25,6 +25,7 @@ constexpr int kMaxE = 512;
 
 __global__ void __launch_bounds__(256) k_count(const int32_t* __restrict__ ids, int64_t T, int k, int E,
                                                int32_t* __restrict__ counts, unsigned* status) {
+  pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   __shared__ int32_t h[kMaxE];
   for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
   __syncthreads();
@@ -79,6 +80,7 @@ __device__ __forceinline__ void write_tile_prefix(const Schedule& s, int E, int 
 __global__ void __launch_bounds__(1024) k_tile_prefix(const int32_t* __restrict__ offs, int E, Schedule sa,
                                                       int32_t* __restrict__ prefix_a, Schedule sb,
                                                       int32_t* __restrict__ prefix_b) {
+  pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   __shared__ int sm_warp[32];
   int g = threadIdx.x;
   int rows = g <= E ? offs[g + 1] - offs[g] : 0;
@@ -116,6 +118,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
     int32_t* __restrict__ prefix_a, Schedule sb, int32_t* __restrict__ prefix_b, int32_t* __restrict__ row_tok,
     float* __restrict__ row_w, int32_t* __restrict__ pos, int32_t* __restrict__ row_dst,
     const float* __restrict__ shared_gate) {
+  pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   __shared__ int32_t wb[kScatterWarps][kMaxE];
   __shared__ int32_t s_base[kMaxE];
   __shared__ int sm_warp[32];
@@ -237,6 +240,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
 __global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ x, const int32_t* __restrict__ row_tok,
                                                 const int32_t* __restrict__ offs, int E, int64_t T,
                                                 int vec_per_row, uint4* __restrict__ xp) {
+  pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   const int64_t rows = offs[E + 1];
   const int lane = threadIdx.x & 31;
   for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;

@@ -55,6 +55,7 @@ template <typename TA>
 __global__ void __launch_bounds__(256) k_prologue(const TA* __restrict__ x, const TA* __restrict__ gamma, float eps,
                                                   const TA* __restrict__ gate_w, int64_t T, int d,
                                                   TA* __restrict__ x_out, float* __restrict__ gate_out) {
+  pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   const int lane = threadIdx.x & 31;
   const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;

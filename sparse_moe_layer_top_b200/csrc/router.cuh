@@ -69,6 +69,7 @@ template <typename TA, int NPL>
 __global__ void __launch_bounds__(256) k_router_simt(const TA* __restrict__ x, const TA* __restrict__ wr,
                                                      const float* __restrict__ bias, int64_t T, int d, int E, int k,
                                                      int32_t* __restrict__ ids, float* __restrict__ tw) {
+  pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t = (int64_t)blockIdx.x * 8 + warp;
   if (t >= T) return;
@@ -97,6 +98,7 @@ __global__ void __launch_bounds__(256) k_topk(const float* __restrict__ part, in
                                               int64_t ldp, const float* __restrict__ bias, int64_t T, int E, int k,
                                               int32_t* __restrict__ ids, float* __restrict__ tw,
                                               int32_t* __restrict__ counts) {
+  pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   const int lane = threadIdx.x & 31;
   const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;

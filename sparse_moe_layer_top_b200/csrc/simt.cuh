@@ -61,6 +61,7 @@ __device__ __forceinline__ float weight_at(const WeightSet<TW>& ws, int g, int E
 
 template <typename TA, typename TW, int EPI>
 __global__ void __launch_bounds__(256) k_gemm_simt(SimtGemmArgs<TA, TW> p) {
+  pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   constexpr bool kDual = EPI == kEpiSwiGLU;
   __shared__ float As[16][64 + 4];
   __shared__ float Bs[16][64 + 4];
@@ -139,6 +140,7 @@ template <typename TA>
 __global__ void __launch_bounds__(256) k_combine(const TA* __restrict__ yp, const int32_t* __restrict__ pos,
                                                  const float* __restrict__ tw, const int32_t* __restrict__ offs,
                                                  int E, int k, int d, int64_t T, TA* __restrict__ y) {
+  pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   const int64_t t = blockIdx.x;
   const int64_t rs = offs[E], re = offs[E + 1];
   const bool shared = re > rs;
@@ -161,6 +163,7 @@ __global__ void __launch_bounds__(256) k_combine(const TA* __restrict__ yp, cons
 template <typename TA>
 __global__ void __launch_bounds__(256) k_slot_sum(const TA* __restrict__ ys, const int32_t* __restrict__ pos, int k,
                                                   int has_shared, int d, TA* __restrict__ y) {
+  pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   const int64_t t = blockIdx.x;
   const TA* src = ys + t * (int64_t)(k + 1) * d;
   unsigned ok = 0;

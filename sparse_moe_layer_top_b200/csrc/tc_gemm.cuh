@@ -343,12 +343,6 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned tcode = kStatusTimeoutBase | (kKernGemmTc << 8);
-  if (p.single_rows < 0)
-    for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) {
-      s_pre[i] = __ldg(p.prefix + i);
-      s_offs[i] = __ldg(p.offs + i);
-    }
-
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full + s, FP8 ? Cfg::NB / 32 : 1);  // FP8: one arrival per converter warp
@@ -381,6 +375,15 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
+  // the tile schedule comes from earlier kernels in the stream: read it once
+  // they are done (barrier set-up, tensor-map prefetch and TMEM allocation above
+  // overlap the previous kernel's tail under programmatic launch)
+  pdl_begin();
+  if (p.single_rows < 0)
+    for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) {
+      s_pre[i] = __ldg(p.prefix + i);
+      s_offs[i] = __ldg(p.offs + i);
+    }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();

@@ -84,10 +84,6 @@ __global__ void __launch_bounds__(PairCfg<BN, DUAL, STAGES>::THREADS, 1)
   const uint32_t rank = cluster_ctarank();
   const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const unsigned tcode = kStatusTimeoutBase | (kKernGemmTc << 8) | 0x80u;
-  for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) {
-    s_pre[i] = __ldg(p.prefix + i);
-    s_offs[i] = __ldg(p.offs + i);
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(full + s, 1);
@@ -115,6 +111,14 @@ __global__ void __launch_bounds__(PairCfg<BN, DUAL, STAGES>::THREADS, 1)
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, Cfg::TMEM_COLS);  // with the peer's warp 1
     tmem_relinquish_pair();
+  }
+  // the tile schedule comes from earlier kernels in the stream: read it once
+  // they are done (barrier set-up, tensor-map prefetch and TMEM allocation above
+  // overlap the previous kernel's tail under programmatic launch)
+  pdl_begin();
+  for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) {
+    s_pre[i] = __ldg(p.prefix + i);
+    s_offs[i] = __ldg(p.offs + i);
   }
   tc_fence_before();
   cluster_sync_all();

@@ -75,10 +75,6 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const unsigned tcode = kStatusTimeoutBase | (kKernGemmSwap << 8);
-  for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) {
-    s_pre[i] = __ldg(p.prefix + i);
-    s_offs[i] = __ldg(p.offs + i);
-  }
   if (threadIdx.x == 0) {
     for (int s = 0; s < R; ++s) {
       mbar_init(raw_full + s, 1);
@@ -109,6 +105,14 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
   if (warp == 1) {
     tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
     tmem_relinquish();
+  }
+  // the tile schedule comes from earlier kernels in the stream: read it once
+  // they are done (barrier set-up, tensor-map prefetch and TMEM allocation above
+  // overlap the previous kernel's tail under programmatic launch)
+  pdl_begin();
+  for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) {
+    s_pre[i] = __ldg(p.prefix + i);
+    s_offs[i] = __ldg(p.offs + i);
   }
   tc_fence_before();
   __syncthreads();
