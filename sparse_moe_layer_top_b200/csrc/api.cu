@@ -93,11 +93,11 @@ static void prof_end(const char* name, cudaStream_t st) {
   } while (0)
 
 // Kernel launch.  Every launch of a library call after its first carries the
-// programmatic-serialisation attribute: the kernel may be scheduled while the
-// previous one finishes, runs its set-up, and waits for it (griddepcontrol.wait)
-// before touching its results -- every kernel of the library does.  The first
-// launch of a call (whose predecessor may be the caller's own kernel) and the
-// first after a memset go in plain stream order.
+// programmatic-serialisation attribute: the kernel may be scheduled as the
+// previous one's blocks exit, runs its set-up, and waits for it
+// (griddepcontrol.wait) before touching its results -- every kernel of the
+// library does.  The first launch of a call (whose predecessor may be the
+// caller's own kernel) and the first after a memset go in plain stream order.
 static thread_local bool g_pdl_next = false;
 static void pdl_reset() { g_pdl_next = false; }
 
@@ -502,10 +502,14 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
 // Histogram (unless the router wrote it), then one kernel that scans it and
 // scatters: offs, row_tok, row_w, pos, row_dst (may be NULL), the shared rows,
 // and optionally the tile prefixes.
+// Dispatch: the stable sort of the (token, slot) pairs by expert and, when xp
+// is given, the copy of x's rows into their dispatched rows (and the shared
+// expert's rows), in one kernel.
 static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, const float* tw, bool counted,
                                   int32_t* offs, int32_t* row_tok, float* row_w, int32_t* pos, int32_t* row_dst,
                                   int32_t* counts, Schedule sa, int32_t* pre_a, Schedule sb, int32_t* pre_b,
-                                  cudaStream_t st, DeviceInfo* dev, const float* shared_gate = nullptr) {
+                                  const void* x, void* xp, cudaStream_t st, DeviceInfo* dev,
+                                  const float* shared_gate = nullptr) {
   const int nch = (int)n_chunks(p);
   if (p.T == 0) {
     CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)p.E * 4, st));
@@ -515,22 +519,12 @@ static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, cons
     CUDA_TRY(launch(k_count, nch, 256, 0, st, ids, p.T, p.k, p.E, counts, dev->status));
     LAUNCH_CHECK("count", st);
   }
-  PROF_BEGIN("dispatch", st);
-  CUDA_TRY(launch(k_dispatch, nch, kScatterWarps * 32, 0, st, ids, tw, p.T, p.k, p.E, counts, nch,
-                  p.I_s > 0, offs, sa, pre_a, sb, pre_b, row_tok, row_w, pos, row_dst, shared_gate));
-  LAUNCH_CHECK("dispatch", st);
-  return MOE_OK;
-}
-
-static moe_status launch_gather(const moe_problem& p, const void* x, const int32_t* row_tok, const int32_t* offs,
-                                void* xp, cudaStream_t st, DeviceInfo* dev) {
   const int vec = (int)(p.d * esize(p.act_dtype) / 16);
-  const int64_t rows = rows_total(p);
-  if (rows == 0) return MOE_OK;
-  unsigned grid = (unsigned)std::min<int64_t>(cdiv(rows, 8), (int64_t)dev->sms * 8);
-  PROF_BEGIN("gather", st);
-  CUDA_TRY(launch(k_gather, grid, 256, 0, st, (const uint4*)x, row_tok, offs, p.E, p.T, vec, (uint4*)xp));
-  LAUNCH_CHECK("gather", st);
+  PROF_BEGIN("dispatch", st);
+  CUDA_TRY(launch(k_dispatch, nch * kSubBlocks, kScatterWarps * 32, 0, st, ids, tw, p.T, p.k, p.E, counts, nch,
+                  p.I_s > 0, offs, sa, pre_a, sb, pre_b, row_tok, row_w, pos, row_dst, shared_gate,
+                  (const uint4*)x, vec, (uint4*)xp));
+  LAUNCH_CHECK("dispatch", st);
   return MOE_OK;
 }
 
@@ -1034,9 +1028,7 @@ moe_status moe_permute(const moe_problem* p, const void* x, const int32_t* topk_
   cudaStream_t st = (cudaStream_t)stream;
   char* w = (char*)ws;
   s = launch_dispatch(*p, topk_ids, topk_w, false, offs, row_tok, row_w, pos, nullptr, (int32_t*)(w + L.counts),
-                      Schedule{}, nullptr, Schedule{}, nullptr, st, dev);
-  if (s != MOE_OK) return s;
-  s = launch_gather(*p, x, row_tok, offs, x_perm, st, dev);
+                      Schedule{}, nullptr, Schedule{}, nullptr, x, x_perm, st, dev);
   if (s == MOE_OK) g_launches = g_launches_pending;
   return s;
 }
@@ -1190,10 +1182,9 @@ static moe_status block_forward(const moe_problem* p, const moe_block_options* o
   if (s != MOE_OK) return s;
   Schedule sa, sb;
   schedules(*p, form, &sa, &sb);
-  s = launch_dispatch(*p, ids, tw, counted, offs, row_tok, row_w, pos, row_dst, counts, sa, pre_a, sb, pre_b, st, dev,
-                      gate);
+  s = launch_dispatch(*p, ids, tw, counted, offs, row_tok, row_w, pos, row_dst, counts, sa, pre_a, sb, pre_b, xin, xp,
+                      st, dev, gate);
   if (s != MOE_OK) return s;
-  if ((s = launch_gather(*p, xin, row_tok, offs, xp, st, dev)) != MOE_OK) return s;
   DownOut o{xp, row_dst, row_w, nullptr};  // the slot rows reuse the dispatched-row buffer
   s = expert_gemms(*p, form, xp, offs, w, pre_a, pre_b, wsp + L.h, o, st, dev);
   if (s != MOE_OK) return s;

@@ -5,14 +5,14 @@
 // tokens (chunk c = the pairs of tokens c*kChunkTokens ...):
 //   counts      per-chunk histogram over the E experts (written by k_topk, or
 //               by k_count when the routing comes from elsewhere);
-//   k_dispatch  one block per chunk: column sums of the histograms give the
-//               group offsets offs[E+2] and the chunk's first row per expert
-//               (block 0 also writes the tile prefix sums of the GEMM
-//               schedules); within the chunk, warps take consecutive token
+//   k_dispatch  kSubBlocks blocks per chunk: column sums of the histograms
+//               give the group offsets offs[E+2] and each block's first row
+//               per expert (block 0 also writes the tile prefix sums of the
+//               GEMM schedules); within a block, warps take consecutive token
 //               ranges and rank equal experts by warp match masks, so row
-//               order = (token, slot) order; the chunk's shared-expert rows
-//               are written too;
-//   k_gather    copies x rows into the dispatched buffer (16-byte vectors).
+//               order = (token, slot) order; the shared-expert rows are
+//               written too, and each warp then copies its tokens' x rows into
+//               their dispatched rows (16-byte vectors).
 // Group E (the shared expert) is every token in order at rows offs[E] + t.
 #pragma once
 #include "common.cuh"
@@ -107,24 +107,32 @@ __device__ __forceinline__ int2 block256_scan2(int v0, int v1, int* sm_warp) {
   return make_int2(incl1 - v1, incl1);
 }
 
-// Scan and scatter in one kernel: block c (one chunk of kChunkTokens tokens)
-// sums the chunk histograms of every expert over all chunks and over the
-// chunks before its own, scans the totals into the group offsets, and then
-// places its own pairs in (token, slot) order.  Block 0 also writes offs and the
-// tile prefixes of the two GEMM schedules.  256 threads, E <= 512.
+// Scan, scatter and copy in one kernel.  Block b takes kBlockTokens tokens
+// of chunk c = b / kSubBlocks: it sums the chunk histograms of every expert over
+// all chunks and over the chunks before c, scans the totals into the group
+// offsets, adds the pairs of its chunk's earlier tokens, and then places its
+// own pairs in (token, slot) order.  Block 0 also writes offs and the tile
+// prefixes of the two GEMM schedules.  With xp given, each warp then copies its
+// tokens' rows of x to their k dispatched rows and their shared-expert row (a
+// row is read once and written k + 1 times).  256 threads, E <= 512.
+constexpr int kSubBlocks = 4;                              // blocks per histogram chunk
+constexpr int kBlockTokens = kChunkTokens / kSubBlocks;    // 32 tokens per block
+constexpr int kWarpTokens = kBlockTokens / kScatterWarps;  // 4 tokens per warp
 __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
     const int32_t* __restrict__ ids, const float* __restrict__ topk_w, int64_t T, int k, int E,
     const int32_t* __restrict__ counts, int nchunks, int has_shared, int32_t* __restrict__ offs, Schedule sa,
     int32_t* __restrict__ prefix_a, Schedule sb, int32_t* __restrict__ prefix_b, int32_t* __restrict__ row_tok,
     float* __restrict__ row_w, int32_t* __restrict__ pos, int32_t* __restrict__ row_dst,
-    const float* __restrict__ shared_gate) {
+    const float* __restrict__ shared_gate, const uint4* __restrict__ x, int vec_per_row, uint4* __restrict__ xp) {
   pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   __shared__ int32_t wb[kScatterWarps][kMaxE];
   __shared__ int32_t s_base[kMaxE];
+  __shared__ int32_t s_dst[kScatterWarps][kWarpTokens * kMaxK];  // dispatched row of each of a warp's pairs
   __shared__ int sm_warp[32];
   __shared__ int s_R, s_tot;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int c = blockIdx.x;
+  const int c = blockIdx.x / kSubBlocks, sub = blockIdx.x % kSubBlocks;
+  const int64_t t_blk = (int64_t)c * kChunkTokens + (int64_t)sub * kBlockTokens;  // first token of the block
   // 1. per expert: total over all chunks, and over the chunks before this one
   int tot[2] = {0, 0}, pre[2] = {0, 0};
 #pragma unroll
@@ -147,7 +155,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
   if (2 * threadIdx.x + 1 < E) s_base[2 * threadIdx.x + 1] = start1 + pre[1];
   __syncthreads();
   const int R = s_R;
-  if (c == 0) {
+  if (blockIdx.x == 0) {
     if (2 * threadIdx.x < E) offs[2 * threadIdx.x] = start0;
     if (2 * threadIdx.x + 1 < E) offs[2 * threadIdx.x + 1] = start1;
     if (threadIdx.x == 0) {
@@ -183,11 +191,16 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
       __syncthreads();
     }
   }
-  // 3. the chunk's pairs: per-warp histograms, their scan, then ranks by match masks
-  constexpr int kTokPerWarp = kChunkTokens / kScatterWarps;
+  // 3. pairs of the chunk's tokens before this block: they precede ours in every group
   const int64_t n = T * k;
-  const int64_t s0 = ((int64_t)c * kChunkTokens + (int64_t)warp * kTokPerWarp) * k;
-  const int64_t s1 = min(n, s0 + (int64_t)kTokPerWarp * k);
+  for (int64_t i = (int64_t)c * kChunkTokens * k + threadIdx.x; i < min(n, t_blk * k); i += blockDim.x) {
+    const int e = __ldg(ids + i);
+    if ((unsigned)e < (unsigned)E) atomicAdd(&s_base[e], 1);
+  }
+  __syncthreads();
+  // 4. the block's pairs: per-warp histograms, their scan, then ranks by match masks
+  const int64_t s0 = (t_blk + (int64_t)warp * kWarpTokens) * k;
+  const int64_t s1 = min(n, s0 + (int64_t)kWarpTokens * k);
   for (int e = lane; e < E; e += 32) wb[warp][e] = 0;
   __syncwarp();
   for (int64_t i = s0 + lane; i < s1; i += 32) {
@@ -225,32 +238,48 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
     } else if (act) {
       pos[i] = -1;
     }
+    if (act) s_dst[warp][i - s0] = ok ? r : -1;
   }
   if (has_shared) {
-    for (int64_t t = (int64_t)c * kChunkTokens + threadIdx.x; t < min(T, (int64_t)(c + 1) * kChunkTokens);
-         t += blockDim.x) {
+    for (int64_t t = t_blk + threadIdx.x; t < min(T, t_blk + kBlockTokens); t += blockDim.x) {
       row_tok[R + t] = (int32_t)t;
       row_w[R + t] = shared_gate ? __ldg(shared_gate + t) : 1.0f;  // the shared expert's weight
       if (row_dst) row_dst[R + t] = (int32_t)(t * (k + 1) + k);
     }
   }
-}
-
-// x_perm[r] = x[row_tok[r]], one warp per row, 16-byte vectors (row bytes % 16 == 0).
-__global__ void __launch_bounds__(256) k_gather(const uint4* __restrict__ x, const int32_t* __restrict__ row_tok,
-                                                const int32_t* __restrict__ offs, int E, int64_t T,
-                                                int vec_per_row, uint4* __restrict__ xp) {
-  pdl_begin();  // after the previous kernel in the stream (programmatic launch)
-  const int64_t rows = offs[E + 1];
-  const int lane = threadIdx.x & 31;
-  for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5; r < rows;
-       r += ((int64_t)gridDim.x * blockDim.x) >> 5) {
-    int t = __ldg(row_tok + r);
-    if ((uint64_t)t >= (uint64_t)T) t = 0;  // cannot happen for valid routing
-    const uint4* src = x + (int64_t)t * vec_per_row;
-    uint4* dst = xp + r * vec_per_row;
-#pragma unroll 4
-    for (int v = lane; v < vec_per_row; v += 32) dst[v] = __ldg(src + v);  // (restrict: reads batch ahead)
+  if (!xp) return;
+  // 5. each warp copies its tokens' rows: read once, written to the token's
+  //    dispatched rows and its shared-expert row, four 16-byte vectors per lane
+  //    in flight
+  __syncwarp();
+  for (int tt = 0; tt < kWarpTokens; ++tt) {
+    const int64_t t = t_blk + (int64_t)warp * kWarpTokens + tt;
+    if (t >= T) break;
+    const uint4* src = x + t * vec_per_row;
+    for (int v0 = 0; v0 < vec_per_row; v0 += 128) {
+      uint4 a[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int v = v0 + u * 32 + lane;
+        if (v < vec_per_row) a[u] = __ldg(src + v);
+      }
+      for (int j = 0; j <= k; ++j) {
+        int64_t r;
+        if (j < k) {
+          r = s_dst[warp][tt * k + j];
+          if (r < 0) continue;
+        } else {
+          if (!has_shared) break;
+          r = R + t;
+        }
+        uint4* dst = xp + r * vec_per_row;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int v = v0 + u * 32 + lane;
+          if (v < vec_per_row) dst[v] = a[u];
+        }
+      }
+    }
   }
 }
 

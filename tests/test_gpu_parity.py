@@ -301,4 +301,5 @@ def test_launch_count_reported(moe):
     g = to_device(inp, "cuda")
     moe.set_path(0)
     _gpu_forward(moe, g)
-    assert moe.last_launch_count() >= 7
+    # router GEMM, top-k, dispatch (with the row copy), gate/up GEMM, down GEMM, slot sum
+    assert moe.last_launch_count() == 6
