@@ -193,6 +193,7 @@ static moe_status device_info(DeviceInfo** out) {
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcSlotStore>, Gemm2Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcStore>, Gemm2Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcLogits>, Gemm2Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcTopK>, Gemm2Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<128, true, kFp8Stages, kTcSwiGLU, true>, Gemm1F8Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, kFp8Stages, kTcSlotStore, true>, Gemm2F8Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, kFp8Stages, kTcStore, true>, Gemm2F8Cfg::SMEM_BYTES));
@@ -372,6 +373,13 @@ static moe_status choose_form(const moe_problem& p, int* form) {
 constexpr int kRouterBN = 256;
 constexpr int kTargetTiles = 148;
 
+// The router with the selection in its epilogue (one 256-expert tile per
+// 128 tokens, no K split, no logit partials): when every expert fits one tile
+// and there are enough token tiles to spread over the GPU; otherwise the split-K
+// logits and k_topk.
+static_assert(kChunkTokens == kBM, "the fused router writes one histogram chunk per row tile");
+static bool router_fused(const moe_problem& p) { return p.E <= kRouterBN && cdiv(p.T, kBM) >= 16; }
+
 struct RouterSplit {
   int ksplit, kb_per, tiles;
   int64_t ldp;  // row stride of the logit partials (floats)
@@ -468,6 +476,34 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
   CUtensorMap ax, bw;
   if ((s = map2d(&ax, x, p.d, p.T, p.d, kBM)) != MOE_OK) return s;
   if ((s = map2d(&bw, wr, p.d, p.E, p.d, kRouterBN)) != MOE_OK) return s;
+  if (router_fused(p)) {
+    // every expert's logit of a token in one TMEM tile: select in the epilogue
+    if (counts) {
+      CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * p.E * 4, st));
+      pdl_reset();
+    }
+    TcGemmArgs a{};
+    a.E = 0;
+    a.N_s = p.E;
+    a.K_s = p.d;
+    a.rows_cap = p.T;
+    a.single_rows = (int)p.T;
+    a.single_tiles = (int)cdiv(p.T, kBM);
+    a.ksplit = 1;
+    a.kb_per_split = (int)cdiv(p.d, kBK);
+    a.topk = p.k;
+    a.ids = ids;
+    a.tw = tw;
+    a.bias = bias;
+    a.counts = counts;
+    a.status = dev->status;
+    PROF_BEGIN("gemm_tc_router", st);
+    CUDA_TRY(launch(k_gemm_tc<kRouterBN, false, 4, kTcTopK>, std::min(a.single_tiles, dev->sms), Gemm2Cfg::THREADS,
+                    Gemm2Cfg::SMEM_BYTES, st, ax, ax, bw, bw, bw, bw, a));
+    LAUNCH_CHECK("gemm_tc_router", st);
+    *counted = counts != nullptr;
+    return MOE_OK;
+  }
   TcGemmArgs a{};
   a.E = 0;
   a.N_s = p.E;

@@ -43,7 +43,7 @@ namespace moe {
 constexpr int kBM = 128;
 constexpr int kBK = 64;  // 64 bf16 = one 128-byte swizzle row
 
-enum { kTcSwiGLU = 0, kTcSlotStore = 1, kTcStore = 2, kTcLogits = 3 };
+enum { kTcSwiGLU = 0, kTcSlotStore = 1, kTcStore = 2, kTcLogits = 3, kTcTopK = 4 };
 
 struct TcGemmArgs {
   const int32_t* offs;    // [E+2] group row starts (grouped mode)
@@ -64,6 +64,14 @@ struct TcGemmArgs {
   int64_t ldo;
   float* part;            // Logits output [ksplit][rows, ldp]
   int64_t ldp, part_stride;
+  // TopK (router with selection, one N tile, no K split): topk_ids / topk_w
+  // [rows, topk] and the 128-row chunk histograms counts[rows / 128][N_s]
+  // (may be NULL); bias [N_s] fp32 (may be NULL) is added to the logits
+  int topk;
+  int32_t* ids;
+  float* tw;
+  const float* bias;
+  int32_t* counts;
   // E4M3 weights: fp32 scales per 128 x 128 block, [E][N/128][K/128] routed,
   // [N/128][K/128] shared; B = gate (or the single operand), C = up
   const float *sc_b_r, *sc_b_s, *sc_c_r, *sc_c_s;
@@ -148,7 +156,8 @@ struct TcGemmCfg {
   static constexpr int THREADS = FP8 ? 192 + NB + 32 : 64 + 32 * EPI_WARPS;
   static constexpr int ACC_COLS = DUAL ? 2 * BN : BN;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
-  static constexpr int BAR_BYTES = (3 * STAGES + 2 * RAW_STAGES + 5) * 8 + 16;
+  // + 4 + 4 handoff barriers of the router epilogue (one pair per lane quarter)
+  static constexpr int BAR_BYTES = (3 * STAGES + 2 * RAW_STAGES + 5 + 8) * 8 + 16;
   static constexpr int SCHED_INTS = 2 * (512 + 2);  // tile prefix + group offsets, E <= 512
   // epilogue staging: 32 rows x 64 bytes per epilogue warp
   static constexpr int EPI_OFF = (RING_BYTES + BAR_BYTES + SCHED_INTS * 4 + 127) / 128 * 128;
@@ -318,6 +327,104 @@ __device__ __forceinline__ void epilogue_rows(const TcGemmArgs& p, const TileInf
   }
 }
 
+// Push (v, e) into a list of KT (logit, expert) pairs sorted by logit, larger
+// first; the last pair drops out.  Empty slots hold (-inf, INT_MAX).
+// Candidates arrive in increasing expert order, so a strict comparison keeps
+// the lower expert first among equal logits (the selection order of the
+// router).  The list is sorted, so "v beats slot i" is monotone in i: every
+// slot is compared at once and shifted by selects, with one branch that skips
+// values below the last kept one.
+template <int KT>
+__device__ __forceinline__ void topk_push(float (&tv)[KT], int (&te)[KT], float v, int e) {
+  if (!(v > tv[KT - 1])) return;
+#pragma unroll
+  for (int i = KT - 1; i > 0; --i) {
+    const bool here = v > tv[i], above = v > tv[i - 1];
+    tv[i] = above ? tv[i - 1] : (here ? v : tv[i]);
+    te[i] = above ? te[i - 1] : (here ? e : te[i]);
+  }
+  if (v > tv[0]) {
+    tv[0] = v;
+    te[0] = e;
+  }
+}
+
+// Router epilogue: softmax top-k of each token's logits, read from TMEM.
+// With EG = 2 warps per lane quarter, warp eg scans columns [eg*BN/2,
+// (eg+1)*BN/2) of its 32 tokens; the second hands its KT best to the first
+// through shared memory (xv/xe, slot-major so lanes hit distinct banks) under
+// a bounded mbarrier handshake (hfull / hempty, 32 arrivals each), and the
+// first merges them -- all of them come from higher experts, which keeps the
+// order of equal logits -- then writes the top k, their softmax weights
+// renormalised over the kept experts and the chunk histogram.  Returns false
+// when a wait gave up (the caller stops).
+template <int BN, int EG, int KT>
+__device__ __forceinline__ bool topk_epilogue(const TcGemmArgs& p, const TileInfo& t, uint32_t tb, int eg,
+                                              int64_t grow, bool valid, float* xv, int* xe, uint64_t* hfull,
+                                              uint64_t* hempty, uint32_t hpar, volatile int* abort_flag,
+                                              unsigned where, int lane) {
+  float tv[KT];
+  int te[KT];
+#pragma unroll
+  for (int i = 0; i < KT; ++i) {
+    tv[i] = -INFINITY;
+    te[i] = 0x7fffffff;
+  }
+  constexpr int CW = BN / EG;  // columns per warp
+  const int c0 = eg * CW;
+  uint32_t a[8], nx[8];
+  tmem_ld8(tb + c0, a);
+  tmem_wait_regs(a);
+#pragma unroll 1
+  for (int c = c0; c < c0 + CW; c += 8) {
+    if (c + 8 < c0 + CW) tmem_ld8(tb + c + 8, nx);  // next 8 columns land while these are scanned
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = t.n0 + c + j;
+      const float v = e < t.N ? __uint_as_float(a[j]) + (p.bias ? __ldg(p.bias + e) : 0.f) : -INFINITY;
+      topk_push(tv, te, v, e);
+    }
+    if (c + 8 < c0 + CW) {
+      tmem_wait_regs(nx);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) a[j] = nx[j];
+    }
+  }
+  if (EG == 2) {
+    const bool ok = eg ? mbar_wait(hempty, hpar ^ 1, abort_flag, p.status, where)
+                       : mbar_wait(hfull, hpar, abort_flag, p.status, where);
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    if (eg) {
+#pragma unroll
+      for (int i = 0; i < KT; ++i) {
+        xv[i * 32 + lane] = tv[i];
+        xe[i * 32 + lane] = te[i];
+      }
+      mbar_arrive(hfull);
+      return true;
+    }
+#pragma unroll
+    for (int i = 0; i < KT; ++i) topk_push(tv, te, xv[i * 32 + lane], xe[i * 32 + lane]);
+    mbar_arrive(hempty);
+  }
+  if (valid) {
+    const float v0 = tv[0];
+    float den = 0.f;
+#pragma unroll
+    for (int i = 0; i < KT; ++i)
+      if (i < p.topk) den += __expf(tv[i] - v0);
+    int32_t* hist = p.counts ? p.counts + (grow / kBM) * t.N : nullptr;
+#pragma unroll
+    for (int i = 0; i < KT; ++i)
+      if (i < p.topk) {
+        p.ids[grow * p.topk + i] = te[i];
+        p.tw[grow * p.topk + i] = __expf(tv[i] - v0) / den;
+        if (hist) atomicAdd(hist + te[i], 1);
+      }
+  }
+  return true;
+}
+
 template <int BN, bool DUAL, int STAGES, int EPI, bool FP8 = false>
 __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
@@ -335,7 +442,9 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
   uint64_t* drain = tempty + 2;
   uint64_t* raw_full = drain + 1;        // FP8: raw weight tile landed
   uint64_t* raw_empty = raw_full + Cfg::RAW_STAGES;  // FP8: raw tile converted
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(raw_empty + Cfg::RAW_STAGES);
+  uint64_t* hfull = raw_empty + Cfg::RAW_STAGES;  // router epilogue: second warp's list written
+  uint64_t* hempty = hfull + 4;                    // router epilogue: list merged, slot free
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(hempty + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* s_pre = reinterpret_cast<int32_t*>(smem + Cfg::RING_BYTES + Cfg::BAR_BYTES);
   int32_t* s_offs = s_pre + 514;
@@ -358,6 +467,10 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
       mbar_init(tempty + b, Cfg::EPI_WARPS);
     }
     mbar_init(drain, 1);
+    for (int q = 0; q < 4; ++q) {
+      mbar_init(hfull + q, 32);
+      mbar_init(hempty + q, 32);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -508,10 +621,11 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
     const int q = warp & 3;
     const int row = q * 32 + lane;
     int acc = 0;
-    uint32_t acc_phase = 0;
+    uint32_t acc_phase = 0, hpar = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
       const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
-      if (!mbar_wait(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)))
+        break;  // the warp stops as one: its TMEM loads are warp-collective
       tc_fence_after();
       const uint32_t tb = tmem_base + acc * Cfg::ACC_COLS + ((uint32_t)(q * 32) << 16);
       const int64_t grow = t.row0 + row;
@@ -519,6 +633,16 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
       if (EPI == kTcSwiGLU || EPI == kTcSlotStore || EPI == kTcStore) {
         constexpr int CPW = (BN / 32) / EG;  // 32-column chunks per warp, contiguous
         epilogue_rows<BN, EPI>(p, t, tb, row, eg * CPW, (eg + 1) * CPW, epi_stage + (warp - 2) * 2048, lane);
+      } else if (EPI == kTcTopK) {
+        float* xv = reinterpret_cast<float*>(epi_stage + q * 4096);  // 16 KB: 4 quarters x 16 slots x 32 lanes x 8 B
+        int* xe = reinterpret_cast<int*>(epi_stage + q * 4096 + 2048);
+        const bool ok =
+            p.topk <= 8 ? topk_epilogue<BN, EG, 8>(p, t, tb, eg, grow, valid, xv, xe, hfull + q, hempty + q, hpar,
+                                                   abort_flag, tcode | 9, lane)
+                        : topk_epilogue<BN, EG, 16>(p, t, tb, eg, grow, valid, xv, xe, hfull + q, hempty + q, hpar,
+                                                    abort_flag, tcode | 9, lane);
+        hpar ^= 1;
+        if (!ok) break;
       } else if (EPI == kTcLogits) {
         float* dst = p.part + (int64_t)t.split * p.part_stride + grow * p.ldp;
 #pragma unroll 1

@@ -225,7 +225,8 @@ __global__ void __launch_bounds__(PairCfg<BN, DUAL, STAGES>::THREADS, 1)
     uint32_t acc_phase = 0;
     for (int tile = pair; tile < total; tile += npairs) {
       const TileInfo t = decode_tile<BN, kPairBM>(p, s_pre, s_offs, tile);
-      if (!mbar_wait_cluster(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait_cluster(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)))
+        break;  // the warp stops as one: its TMEM loads are warp-collective
       tc_fence_after();
       const uint32_t tb = tmem_base + acc * Cfg::ACC_COLS + ((uint32_t)(q * 32) << 16);
       epilogue_rows<BN, EPI>(p, t, tb, row, eg * CPW, (eg + 1) * CPW, epi_stage + (warp - 2) * 2048, lane);

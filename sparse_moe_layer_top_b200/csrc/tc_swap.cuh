@@ -100,7 +100,8 @@ __device__ __forceinline__ void swap_epilogue(const TcGemmArgs& p, const int32_t
         w_hi = __ldg(p.row_w + rb);
       }
     }
-    if (!mbar_wait(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)) break;
+    if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)))
+      break;  // the warp stops as one: its TMEM loads are warp-collective
     tc_fence_after();
     const uint32_t tb = tmem_base + acc * ACC_COLS + ((uint32_t)(q * 32) << 16);
     const int n = t.n0 + nl;

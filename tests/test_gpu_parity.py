@@ -55,13 +55,22 @@ FORWARD_CASES = {
     "bf16_long_ragged": (700, 384, 5, 2, 320, 192, "bf16", "bf16", None),
     # T*k >= 2048*E: the automatic choice takes the CTA-pair GEMMs
     "bf16_auto_pair": (2048, 256, 2, 2, 256, 128, "bf16", "bf16", None),
+    # E <= 256 and >= 16 row tiles: the router selects in its GEMM epilogue
+    # (E = 100: a partial expert tile; Zipf bias: the bias enters the selection)
+    "bf16_fused_router": (2304, 256, 100, 6, 128, 128, "bf16", "bf16", "zipf"),
     "fp8_small": (64, 256, 8, 2, 256, 128, "bf16", "fp8", None),
     "fp8_multi_tile": (300, 384, 12, 3, 384, 256, "bf16", "fp8", None),
 }
 
 
+ROUTER_ONLY = {
+    # the fused router at the 35B-shaped expert count, k = 8, ragged last tile
+    "bf16_fused_router_E256": (2100, 512, 256, 8, 64, 64, "bf16", "bf16", None),
+}
+
+
 def _make(case, seed=0):
-    T, d, E, k, I, I_s, act, w, bias = FORWARD_CASES[case]
+    T, d, E, k, I, I_s, act, w, bias = FORWARD_CASES[case] if case in FORWARD_CASES else ROUTER_ONLY[case]
     return moe_inputs.make_inputs(T, d, E, k, I, I_s, act=act, w=w, bias=bias, seed=seed,
                                   shared=I_s > 0)
 
@@ -104,7 +113,8 @@ def test_forward_matches_oracle(moe, case, path):
     assert err <= TOL[key], "rel-L2 %.3g > %.3g (near-tie tokens with another set: %d)" % (err, TOL[key], differ)
 
 
-@pytest.mark.parametrize("case", ["tiny_fp32", "bf16_multi_tile", "bf16_E512_k10", "bf16_zipf", "bf16_T1"])
+@pytest.mark.parametrize("case", ["tiny_fp32", "bf16_multi_tile", "bf16_E512_k10", "bf16_zipf", "bf16_T1",
+                                  "bf16_fused_router", "bf16_fused_router_E256"])
 def test_router_matches_oracle(moe, case):
     inp = _make(case)
     g = to_device(inp, "cuda")
