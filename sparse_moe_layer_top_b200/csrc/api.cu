@@ -143,6 +143,9 @@ static cudaError_t allow_smem(K kernel, int bytes) {
 // GEMM instantiations used by the library.
 using Gemm1Cfg = TcGemmCfg<128, true, 4>;
 using Gemm2Cfg = TcGemmCfg<256, false, 4>;
+// the router that selects in its epilogue: 64-expert column tiles, 8 stages
+constexpr int kTopkBN = 64, kTopkStages = 8;
+using TopkCfg = TcGemmCfg<kTopkBN, false, kTopkStages>;
 constexpr int kFp8Stages = 2;
 using Gemm1F8Cfg = TcGemmCfg<128, true, kFp8Stages, true>;
 using Gemm2F8Cfg = TcGemmCfg<256, false, kFp8Stages, true>;
@@ -193,7 +196,7 @@ static moe_status device_info(DeviceInfo** out) {
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcSlotStore>, Gemm2Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcStore>, Gemm2Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcLogits>, Gemm2Cfg::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcTopK>, Gemm2Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_tc<kTopkBN, false, kTopkStages, kTcTopK>, TopkCfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<128, true, kFp8Stages, kTcSwiGLU, true>, Gemm1F8Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, kFp8Stages, kTcSlotStore, true>, Gemm2F8Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, kFp8Stages, kTcStore, true>, Gemm2F8Cfg::SMEM_BYTES));
@@ -373,10 +376,10 @@ static moe_status choose_form(const moe_problem& p, int* form) {
 constexpr int kRouterBN = 256;
 constexpr int kTargetTiles = 148;
 
-// The router with the selection in its epilogue (one 256-expert tile per
-// 128 tokens, no K split, no logit partials): when every expert fits one tile
-// and there are enough token tiles to spread over the GPU; otherwise the split-K
-// logits and k_topk.
+// The router with the selection in its epilogue (128-token x 64-expert
+// tiles, no K split, no logit partials; the column tiles of a row tile merge
+// their candidate lists): for up to 256 experts and enough token tiles to
+// spread over the GPU; otherwise the split-K logits and k_topk.
 static_assert(kChunkTokens == kBM, "the fused router writes one histogram chunk per row tile");
 static bool router_fused(const moe_problem& p) { return p.E <= kRouterBN && cdiv(p.T, kBM) >= 16; }
 
@@ -395,6 +398,31 @@ static RouterSplit router_split(const moe_problem& p) {
   r.tiles = mn * r.ksplit;
   r.ldp = (int64_t)align_up(p.E, 32);
   return r;
+}
+
+// Router scratch: the split-K logit partials, or for the fused router the
+// per-(row tile, lane quarter) counters followed by the candidate lists.
+struct TopkScratch {
+  int64_t row_tiles;
+  int ntc;
+  size_t cnt_off, v_off, e_off, bytes;
+};
+static TopkScratch topk_scratch(const moe_problem& p) {
+  TopkScratch t;
+  t.row_tiles = cdiv(std::max<int64_t>(p.T, 1), kBM);
+  t.ntc = (int)cdiv(p.E, kTopkBN);
+  const size_t list = t.ntc > 1 ? (size_t)t.row_tiles * t.ntc * kMaxK * kBM * 4 : 0;
+  t.cnt_off = 0;
+  t.v_off = align_up((size_t)t.row_tiles * 4 * 4, 256);
+  t.e_off = t.v_off + align_up(list, 256);
+  t.bytes = t.e_off + list;
+  return t;
+}
+static size_t router_scratch_bytes(const moe_problem& p) {
+  if (p.act_dtype != MOE_BF16) return 0;
+  if (router_fused(p)) return topk_scratch(p).bytes;
+  const RouterSplit rs = router_split(p);
+  return (size_t)rs.ksplit * p.T * rs.ldp * 4;
 }
 
 struct Layout {
@@ -423,10 +451,7 @@ static Layout layout(const moe_problem& p, bool forward) {
   L.counts = take(n_chunks(p) * p.E * 4);
   L.pre_a = take((p.E + 2) * 4);
   L.pre_b = take((p.E + 2) * 4);
-  if (p.act_dtype == MOE_BF16) {
-    const RouterSplit rs = router_split(p);
-    L.part = take((size_t)rs.ksplit * p.T * rs.ldp * 4);
-  }
+  if (p.act_dtype == MOE_BF16) L.part = take(router_scratch_bytes(p));
   if (forward) {
     L.ids = take(n * 4);
     L.tw = take(n * 4);
@@ -477,7 +502,16 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
   if ((s = map2d(&ax, x, p.d, p.T, p.d, kBM)) != MOE_OK) return s;
   if ((s = map2d(&bw, wr, p.d, p.E, p.d, kRouterBN)) != MOE_OK) return s;
   if (router_fused(p)) {
-    // every expert's logit of a token in one TMEM tile: select in the epilogue
+    // every logit of a token in TMEM across the row tile's column tiles:
+    // select in the epilogue
+    const TopkScratch ts = topk_scratch(p);
+    CUtensorMap bw64;
+    if ((s = map2d(&bw64, wr, p.d, p.E, p.d, kTopkBN)) != MOE_OK) return s;
+    char* scratch = reinterpret_cast<char*>(part);
+    if (ts.ntc > 1) {
+      CUDA_TRY(cudaMemsetAsync(scratch + ts.cnt_off, 0, (size_t)ts.row_tiles * 4 * 4, st));
+      pdl_reset();
+    }
     if (counts) {
       CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * p.E * 4, st));
       pdl_reset();
@@ -488,7 +522,7 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
     a.K_s = p.d;
     a.rows_cap = p.T;
     a.single_rows = (int)p.T;
-    a.single_tiles = (int)cdiv(p.T, kBM);
+    a.single_tiles = (int)(ts.row_tiles * ts.ntc);
     a.ksplit = 1;
     a.kb_per_split = (int)cdiv(p.d, kBK);
     a.topk = p.k;
@@ -496,10 +530,13 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
     a.tw = tw;
     a.bias = bias;
     a.counts = counts;
+    a.cand_cnt = reinterpret_cast<int32_t*>(scratch + ts.cnt_off);
+    a.cand_v = reinterpret_cast<float*>(scratch + ts.v_off);
+    a.cand_e = reinterpret_cast<int32_t*>(scratch + ts.e_off);
     a.status = dev->status;
     PROF_BEGIN("gemm_tc_router", st);
-    CUDA_TRY(launch(k_gemm_tc<kRouterBN, false, 4, kTcTopK>, std::min(a.single_tiles, dev->sms), Gemm2Cfg::THREADS,
-                    Gemm2Cfg::SMEM_BYTES, st, ax, ax, bw, bw, bw, bw, a));
+    CUDA_TRY(launch(k_gemm_tc<kTopkBN, false, kTopkStages, kTcTopK>, std::min(a.single_tiles, dev->sms),
+                    TopkCfg::THREADS, TopkCfg::SMEM_BYTES, st, ax, ax, bw64, bw64, bw64, bw64, a));
     LAUNCH_CHECK("gemm_tc_router", st);
     *counted = counts != nullptr;
     return MOE_OK;
@@ -1315,11 +1352,7 @@ extern "C" moe_status moe_router_topk_static(const moe_problem* p, const void* x
   MAYBE(router_bias);
   NEED(topk_ids);
   NEED(topk_w);
-  size_t need = 0;
-  if (p->act_dtype == MOE_BF16) {
-    const RouterSplit rs = router_split(*p);
-    need = (size_t)rs.ksplit * p->T * rs.ldp * 4;
-  }
+  const size_t need = router_scratch_bytes(*p);
   if (need > (size_t)MOE_ROUTER_STATIC_SCRATCH_BYTES)
     return fail(MOE_ERR_UNSUPPORTED,
                 "router needs %zu bytes of scratch; the built-in array holds %zu (use moe_router_topk with a workspace)",

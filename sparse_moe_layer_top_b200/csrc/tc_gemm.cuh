@@ -11,18 +11,20 @@
 // one column block of a group are adjacent, so the CTAs that share a weight
 // tile run together and the second read of it comes from L2.
 //
-// Warp roles (6 warps):
+// Warp roles (10 warps):
 //   warp 0      TMA producer: A tile 128 x 64 and B tile(s) BN x 64 per stage,
 //               128-byte swizzled, into a STAGES-deep shared-memory ring;
 //   warp 1      TMEM owner and MMA issuer: tcgen05.mma M=128, N=BN, K=16,
 //               fp32 accumulators in TMEM, double-buffered across tiles;
-//   warps 2..5  epilogue: tcgen05.ld of the accumulator rows (warp w reads TMEM
-//               lanes 32*(w%4) ..), then one of
+//   warps 2..9  epilogue, two warps per TMEM lane quarter (warp w reads lanes
+//               32*(w%4) ..; the pair splits the columns): tcgen05.ld of the
+//               accumulator rows, then one of
 //                 SwiGLU    H[r, n] = SiLU(gate) * up -> bf16      (DUAL: two B)
 //                 SlotStore Y[dst(r), n] = w(r) * D -> bf16: the routing weight
 //                           applied and the row put back in (token, slot) order
 //                 Store     out[r, n] = D -> bf16
 //                 Logits    part[split][r, n] = D (+ nothing) -> fp32
+//                 TopK      the router's softmax top-k of D + bias per row
 // Rows of a tile past the end of its group are computed and discarded; rows
 // never mix in a GEMM, so those rows cannot disturb the kept ones.
 //
@@ -72,6 +74,13 @@ struct TcGemmArgs {
   float* tw;
   const float* bias;
   int32_t* counts;
+  // TopK over several column tiles: each tile's kept (logit, expert) pairs of a
+  // token go to cand_v / cand_e [row tile][column tile][kMaxK slots][kBM rows];
+  // cand_cnt [row tile][4 lane quarters] (zeroed before the launch) counts the
+  // tiles done, and the last one merges the lists and writes the outputs
+  float* cand_v;
+  int32_t* cand_e;
+  int32_t* cand_cnt;
   // E4M3 weights: fp32 scales per 128 x 128 block, [E][N/128][K/128] routed,
   // [N/128][K/128] shared; B = gate (or the single operand), C = up
   const float *sc_b_r, *sc_b_s, *sc_c_r, *sc_c_s;
@@ -349,17 +358,38 @@ __device__ __forceinline__ void topk_push(float (&tv)[KT], int (&te)[KT], float 
   }
 }
 
+// The same for candidates in any expert order: equal logits compare by
+// expert, lower first.
+template <int KT>
+__device__ __forceinline__ void topk_push_lex(float (&tv)[KT], int (&te)[KT], float v, int e) {
+#pragma unroll
+  for (int i = KT - 1; i > 0; --i) {
+    const bool here = v > tv[i] || (v == tv[i] && e < te[i]);
+    const bool above = v > tv[i - 1] || (v == tv[i - 1] && e < te[i - 1]);
+    tv[i] = above ? tv[i - 1] : (here ? v : tv[i]);
+    te[i] = above ? te[i - 1] : (here ? e : te[i]);
+  }
+  if (v > tv[0] || (v == tv[0] && e < te[0])) {
+    tv[0] = v;
+    te[0] = e;
+  }
+}
+
 // Router epilogue: softmax top-k of each token's logits, read from TMEM.
 // With EG = 2 warps per lane quarter, warp eg scans columns [eg*BN/2,
 // (eg+1)*BN/2) of its 32 tokens; the second hands its KT best to the first
 // through shared memory (xv/xe, slot-major so lanes hit distinct banks) under
 // a bounded mbarrier handshake (hfull / hempty, 32 arrivals each), and the
 // first merges them -- all of them come from higher experts, which keeps the
-// order of equal logits -- then writes the top k, their softmax weights
-// renormalised over the kept experts and the chunk histogram.  Returns false
-// when a wait gave up (the caller stops).
+// order of equal logits.  With the experts over several column tiles, the
+// first warp then stores its list (cand_v / cand_e) and counts itself in; the
+// warp that completes a row tile's count merges the other tiles' lists into
+// its own, comparing equal logits by expert -- a last-arriver merge, so no
+// warp waits for another CTA.  The merging warp writes the top k, their
+// softmax weights renormalised over the kept experts and the chunk histogram.
+// Returns false when a wait gave up (the caller stops).
 template <int BN, int EG, int KT>
-__device__ __forceinline__ bool topk_epilogue(const TcGemmArgs& p, const TileInfo& t, uint32_t tb, int eg,
+__device__ __forceinline__ bool topk_epilogue(const TcGemmArgs& p, const TileInfo& t, uint32_t tb, int eg, int row,
                                               int64_t grow, bool valid, float* xv, int* xe, uint64_t* hfull,
                                               uint64_t* hempty, uint32_t hpar, volatile int* abort_flag,
                                               unsigned where, int lane) {
@@ -406,6 +436,44 @@ __device__ __forceinline__ bool topk_epilogue(const TcGemmArgs& p, const TileInf
 #pragma unroll
     for (int i = 0; i < KT; ++i) topk_push(tv, te, xv[i * 32 + lane], xe[i * 32 + lane]);
     mbar_arrive(hempty);
+  }
+  const int ntc = (t.N + BN - 1) / BN;
+  if (ntc > 1) {
+    const int rt = t.m0 / kBM;
+    const int64_t tile_base = (int64_t)rt * ntc * (kMaxK * kBM) + row;
+    const int64_t mine = tile_base + (int64_t)(t.n0 / BN) * (kMaxK * kBM);
+#pragma unroll
+    for (int i = 0; i < KT; ++i) {
+      p.cand_v[mine + i * kBM] = tv[i];
+      p.cand_e[mine + i * kBM] = te[i];
+    }
+    __threadfence();  // the lists are visible before the count that publishes them
+    __syncwarp();
+    int last = 0;
+    if (lane == 0) last = atomicAdd(p.cand_cnt + rt * 4 + (row >> 5), 1) == ntc - 1;
+    if (!__shfl_sync(0xffffffffu, last, 0)) return true;
+    __threadfence();
+    // merge the other tiles' lists into this one's (lexicographic order, so
+    // any tile order gives the same list)
+    const int mine_c = t.n0 / BN;
+#pragma unroll 1
+    for (int c = 0; c < ntc; ++c) {
+      if (c == mine_c) continue;
+      const int64_t o = tile_base + (int64_t)c * (kMaxK * kBM);
+      float cv[KT];
+      int ce[KT];
+#pragma unroll
+      for (int i = 0; i < KT; ++i) {  // the whole list in flight at once
+        cv[i] = __ldcg(p.cand_v + o + i * kBM);
+        ce[i] = __ldcg(p.cand_e + o + i * kBM);
+      }
+      // a list is sorted: once no lane keeps an entry, none keeps a later one
+#pragma unroll
+      for (int i = 0; i < KT; ++i) {
+        if (!__any_sync(0xffffffffu, cv[i] > tv[KT - 1] || (cv[i] == tv[KT - 1] && ce[i] < te[KT - 1]))) break;
+        topk_push_lex(tv, te, cv[i], ce[i]);
+      }
+    }
   }
   if (valid) {
     const float v0 = tv[0];
@@ -637,9 +705,9 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
         float* xv = reinterpret_cast<float*>(epi_stage + q * 4096);  // 16 KB: 4 quarters x 16 slots x 32 lanes x 8 B
         int* xe = reinterpret_cast<int*>(epi_stage + q * 4096 + 2048);
         const bool ok =
-            p.topk <= 8 ? topk_epilogue<BN, EG, 8>(p, t, tb, eg, grow, valid, xv, xe, hfull + q, hempty + q, hpar,
+            p.topk <= 8 ? topk_epilogue<BN, EG, 8>(p, t, tb, eg, row, grow, valid, xv, xe, hfull + q, hempty + q, hpar,
                                                    abort_flag, tcode | 9, lane)
-                        : topk_epilogue<BN, EG, 16>(p, t, tb, eg, grow, valid, xv, xe, hfull + q, hempty + q, hpar,
+                        : topk_epilogue<BN, EG, 16>(p, t, tb, eg, row, grow, valid, xv, xe, hfull + q, hempty + q, hpar,
                                                     abort_flag, tcode | 9, lane);
         hpar ^= 1;
         if (!ok) break;

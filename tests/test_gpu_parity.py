@@ -125,6 +125,32 @@ def test_router_matches_oracle(moe, case):
     check_routing(ids.cpu().numpy(), tw.cpu().numpy(), probs, ids_or, TOL_W[precision_key(inp)])
 
 
+@pytest.mark.parametrize("E,k", [(256, 8), (200, 16), (130, 10), (64, 4)])
+def test_router_exact_ties_go_to_the_lower_expert(moe, E, k):
+    """Tokens with x = 0 have logits equal to the bias exactly (on both sides);
+    the bias repeats a few values on experts spread over every 64-expert column
+    tile, so the kept set and its order are decided by the lower-index rule
+    across tiles.  T = 2100: 17 row tiles (the router selects in its GEMM
+    epilogue) with a ragged last tile."""
+    T, d = 2100, 128
+    gen = torch.Generator().manual_seed(E * 31 + k)
+    x = torch.randn(T, d, generator=gen).to(torch.bfloat16)
+    zero = np.arange(0, T, 3)
+    x[torch.from_numpy(zero)] = 0
+    w_r = (torch.randn(E, d, generator=gen) * 0.02).to(torch.bfloat16)
+    bias = torch.randint(-4, 2, (E,), generator=gen).float() * 0.25
+    bias[torch.arange(5, E, 61)] = 2.0    # one or two per column tile
+    bias[torch.arange(1, E, 37)] = 1.0
+    prob = moe.Problem.make(T, d, E, k, 64, 64, "bf16", "bf16")
+    ids, tw = moe.router_topk(prob, x.cuda(), w_r.cuda(), bias.cuda())
+    torch.cuda.synchronize()
+    _no_device_errors(moe)
+    probs, ids_or, _ = oracle.router(x, w_r, k, bias=bias)
+    ids, tw = ids.cpu().numpy(), tw.cpu().numpy()
+    assert np.array_equal(ids[zero], np.asarray(ids_or)[zero])
+    check_routing(ids, tw, probs, ids_or, TOL_W["bf16"])
+
+
 @pytest.mark.parametrize("T,E,k,act", [(37, 9, 3, "f32"), (1000, 64, 8, "bf16"), (5000, 512, 10, "bf16"),
                                        (3, 600 // 2, 16, "bf16"), (1, 4, 4, "f32")])
 def test_permute_is_the_oracles_stable_sort(moe, T, E, k, act):
