@@ -180,6 +180,26 @@ MOE_API moe_status moe_block_forward(const moe_problem* p, const moe_block_optio
 MOE_API moe_status moe_rmsnorm(const moe_problem* p, const void* x, const void* norm_weight, float eps,
                        void* x_out, void* stream);
 
+/* Expert parallelism, receive side.  The block split over G ranks, rank g
+ * holding experts [g * E_local, (g + 1) * E_local) (the path's experts are
+ * independent, so they partition; the pages raise "how many GPUs for how many
+ * parameters" only as a chapter title, Fondations page, chapter 06).  A rank's
+ * dispatch leaves the rows bound for each rank contiguous and grouped by
+ * expert, so the rows a rank receives are blocks (source s, local expert e) in
+ * that order.  counts int32
+ * [G * E_local] (device): counts[s * E_local + e] = rows from source s for
+ * local expert e.  Writes ids int32 [R] (device): the local expert of each
+ * received row; R = the sum of the counts, known to the caller from the count
+ * exchange.  A k = 1 moe_permute on (received rows, ids) then groups the rows
+ * by expert for moe_expert_ffn.
+ * Errors: G or E_local < 1, G * E_local > 4096, R < 0 or > INT32_MAX ->
+ * MOE_ERR_INVALID_ARG; NULL or not 16-byte aligned pointers (R > 0) ->
+ * MOE_ERR_INVALID_ARG / MOE_ERR_ALIGNMENT, all before any launch.  A negative
+ * count, or fewer counted rows than R (those ids are written -1), sets
+ * MOE_ERR_DEVICE_CHECK in the device status. */
+MOE_API moe_status moe_ep_expand_ids(const int32_t* counts, int32_t G, int32_t E_local, int64_t R,
+                             int32_t* ids, void* stream);
+
 /* moe_router_topk for callers that cannot allocate device memory: code that
  * runs where cudaMalloc is off limits (inside a host framework that owns every
  * device allocation, or on a latency-critical thread that must not enter an
@@ -189,9 +209,11 @@ MOE_API moe_status moe_rmsnorm(const moe_problem* p, const void* x, const void* 
  * router's logit partials go to a file-scope __device__ array of
  * MOE_ROUTER_STATIC_SCRATCH_BYTES that every device that loads the library
  * keeps until the process exits.  Nothing is allocated or freed.
- *   - Problems whose partials need more than that (about
- *     splits * T * roundup(E, 32) * 4 bytes; e.g. T = 8192 with E = 512) are
- *     rejected with MOE_ERR_UNSUPPORTED before anything is launched.
+ *   - Problems whose scratch needs more than that are rejected with
+ *     MOE_ERR_UNSUPPORTED before anything is launched: about
+ *     splits * T * roundup(E, 32) * 4 bytes of split-K partials (e.g. T = 8192
+ *     with E = 512), or T * ceil(E / 64) * 128 bytes of candidate lists when
+ *     the router selects in its GEMM epilogue (E <= 256, T >= 1921).
  *   - The first call on a device looks up that device's copy of the array
  *     (a one-time set-up); make it before any stream capture.
  *   - Every call uses the same array and leaves its contents behind; calls

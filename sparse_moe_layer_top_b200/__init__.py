@@ -7,8 +7,10 @@ built in-tree (``python -m sparse_moe_layer_top_b200.build``) and loaded on
 first use; every call raises if it is missing -- there is no fallback.
 
 Entry points mirror ``include/moe.h``: ``router_topk``, ``permute``,
-``expert_ffn``, ``combine``, ``layer_forward``; ``MoELayer`` keeps a
-layer's weights and workspace together.
+``expert_ffn``, ``combine``, ``layer_forward``, ``block_forward``,
+``rmsnorm``, ``ep_expand_ids``; ``MoELayer`` keeps a layer's weights and
+workspace together; ``sparse_moe_layer_top_b200.ep`` splits the experts over
+several GPUs (expert parallelism).
 """
 import ctypes
 import os
@@ -16,7 +18,7 @@ import os
 import torch
 
 __all__ = ["MoEError", "Problem", "BlockOptions", "router_topk", "permute", "expert_ffn", "combine", "layer_forward",
-           "block_forward", "rmsnorm",
+           "block_forward", "rmsnorm", "ep_expand_ids",
            "workspace_size", "stage_workspace_size", "set_path", "device_status", "last_launch_count",
            "profile_enable", "profile_read",
            "MoELayer", "lib_path", "F32", "BF16", "FP8_E4M3_B128"]
@@ -30,7 +32,8 @@ _STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "
 EXPORTS = ("moe_check_problem", "moe_workspace_size", "moe_stage_workspace_size", "moe_router_topk",
            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_set_path",
            "moe_device_status", "moe_last_launch_count", "moe_profile_enable", "moe_profile_read",
-           "moe_last_error_string", "moe_router_topk_static", "moe_block_forward", "moe_rmsnorm")
+           "moe_last_error_string", "moe_router_topk_static", "moe_block_forward", "moe_rmsnorm",
+           "moe_ep_expand_ids")
 
 
 class MoEError(RuntimeError):
@@ -78,6 +81,7 @@ def lib():
         L.moe_layer_forward.argtypes = [PP, P, P, P, P, P, P, P, P, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.moe_block_forward.argtypes = [PP, ctypes.POINTER(BlockOptions), P, P, P, P, P, P, P, P, P, P, P, P, P,
                                         P, ctypes.c_size_t, P]
+        L.moe_ep_expand_ids.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, P, P]
         L.moe_rmsnorm.argtypes = [PP, P, P, ctypes.c_float, P, P]
         L.moe_set_path.argtypes = [ctypes.c_int]
         L.moe_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32)]
@@ -133,7 +137,7 @@ def check_problem(prob):
 
 def set_path(path):
     """0 automatic, 1 SIMT kernels only, 2 row-tiled tensor-core expert GEMMs,
-    3 weight-row tensor-core expert GEMMs."""
+    3 weight-row tensor-core expert GEMMs, 4 row-tiled on 2-CTA clusters."""
     _check(lib().moe_set_path(int(path)))
 
 
@@ -255,6 +259,16 @@ def rmsnorm(prob, x, norm_weight, eps=1e-6, out=None, stream=None):
     _check(lib().moe_rmsnorm(ctypes.byref(prob), _ptr(x), _ptr(norm_weight), float(eps), _ptr(out),
                              _stream(stream)))
     return out
+
+
+def ep_expand_ids(counts, G, E_local, R, ids=None, stream=None):
+    """Expert parallelism, receive side: the local expert (int32 [R]) of every
+    received row, rows arriving as blocks (source s, local expert e) in that
+    order with counts[s * E_local + e] rows each (int32, on the device)."""
+    if ids is None:
+        ids = torch.empty(max(int(R), 0), dtype=torch.int32, device=counts.device)
+    _check(lib().moe_ep_expand_ids(_ptr(counts), int(G), int(E_local), int(R), _ptr(ids), _stream(stream)))
+    return ids
 
 
 class MoELayer:

@@ -12,6 +12,7 @@
 
 #include "../../include/moe.h"
 #include "common.cuh"
+#include "ep.cuh"
 #include "permute.cuh"
 #include "prologue.cuh"
 #include "router.cuh"
@@ -1306,6 +1307,32 @@ moe_status moe_rmsnorm(const moe_problem* p, const void* x, const void* norm_wei
   pdl_reset();
   if ((s = launch_prologue(*p, x, norm_weight, eps, nullptr, x_out, nullptr, (cudaStream_t)stream)) != MOE_OK)
     return s;
+  g_launches = g_launches_pending;
+  return MOE_OK;
+}
+
+moe_status moe_ep_expand_ids(const int32_t* counts, int32_t G, int32_t E_local, int64_t R, int32_t* ids,
+                             void* stream) {
+  if (G < 1 || E_local < 1 || (int64_t)G * E_local > kEpMaxBlocks)
+    return fail(MOE_ERR_INVALID_ARG, "G = %d, E_local = %d: need G, E_local >= 1 and G * E_local <= %d", G, E_local,
+                kEpMaxBlocks);
+  if (R < 0 || R > INT32_MAX) return fail(MOE_ERR_INVALID_ARG, "R = %lld out of range", (long long)R);
+  if (R == 0) {
+    g_launches = 0;
+    return MOE_OK;
+  }
+  NEED(counts);
+  NEED(ids);
+  DeviceInfo* dev;
+  moe_status s;
+  if ((s = device_info(&dev)) != MOE_OK) return s;
+  g_launches_pending = 0;
+  pdl_reset();
+  cudaStream_t st = (cudaStream_t)stream;
+  const unsigned grid = (unsigned)std::min<int64_t>(cdiv(R, 256), 4 * (int64_t)dev->sms);
+  PROF_BEGIN("ep_expand_ids", st);
+  CUDA_TRY(launch(k_ep_expand_ids, grid, 256, 0, st, counts, G * E_local, (int)E_local, R, ids, dev->status));
+  LAUNCH_CHECK("ep_expand_ids", st);
   g_launches = g_launches_pending;
   return MOE_OK;
 }

@@ -16,6 +16,7 @@ constexpr int kMaxK = 16;  // largest k (experts per token) the kernels support
 // Device status codes: high byte = which check, low bits = where.
 enum : unsigned {
   kStatusBadExpertId = 0x06000001u,  // a routing id outside [0, E)
+  kStatusBadCount = 0x06000002u,     // expert parallelism: a negative or short row count
   kStatusTimeoutBase = 0x07000000u,  // | (kernel id << 8) | wait site
 };
 enum : unsigned { kKernRouterTc = 1, kKernGemmTc = 2, kKernGemmSwap = 3 };

@@ -116,3 +116,18 @@ def test_block_options_rejected_before_any_launch():
     assert L.moe_rmsnorm(ctypes.byref(prob), v(16), v(16), -1.0, v(16), None) == 1
     assert L.moe_rmsnorm(ctypes.byref(prob), v(16), v(0x1008), 1e-6, v(16), None) == 3
     assert L.moe_rmsnorm(ctypes.byref(P(d=100)), v(16), v(16), 1e-6, v(16), None) == 3
+
+
+def test_ep_expand_ids_rejected_before_any_launch():
+    L = moe.lib()
+    v = ctypes.c_void_p
+    # every case fails on the host (fake addresses are never dereferenced)
+    assert L.moe_ep_expand_ids(v(16), 0, 4, 10, v(16), None) == 1      # no ranks
+    assert L.moe_ep_expand_ids(v(16), 2, 0, 10, v(16), None) == 1      # no experts
+    assert L.moe_ep_expand_ids(v(16), 64, 65, 10, v(16), None) == 1    # 4160 blocks > 4096
+    assert L.moe_ep_expand_ids(v(16), 2, 4, -1, v(16), None) == 1      # negative row count
+    assert L.moe_ep_expand_ids(v(16), 2, 4, 1 << 31, v(16), None) == 1
+    assert L.moe_ep_expand_ids(None, 2, 4, 10, v(16), None) == 1       # no counts
+    assert L.moe_ep_expand_ids(v(16), 2, 4, 10, None, None) == 1       # no output
+    assert L.moe_ep_expand_ids(v(0x1008), 2, 4, 10, v(16), None) == 3  # misaligned
+    assert L.moe_ep_expand_ids(None, 2, 4, 0, None, None) == 0         # nothing to do
