@@ -144,15 +144,27 @@ def routing_counts(moe, layer, x):
     return cnt
 
 
+GATHER_MAX_BYTES = 32 << 20
+
+
+def gathers_rows(c, T):
+    """Whether the fused forward's gate/up GEMM reads its rows straight from the
+    token matrix (include/moe.h, moe_layer_forward: the row-tiled bf16 form,
+    i.e. 64*E < T*k < 2048*E on the automatic path, with T*d*2 <= 32 MiB)."""
+    k, E = c["k"], c["E"]
+    rows_form = 64 * E < T * k < 2048 * E
+    return rows_form and c["act"] == "bf16" and c["w"] == "bf16" and T * c["d"] * 2 <= GATHER_MAX_BYTES
+
+
 def work_model(c, counts, T):
     """Algorithmic bytes and flops of the block and of its two expert GEMMs.
 
     Weights are counted for the experts that received at least one row (and
     the shared expert); each kernel's activations once in and once out (the
-    gate/up GEMM reads the dispatched rows and writes H; the down GEMM reads H
-    and writes the weighted (token, slot) rows).  For the whole block only the
-    weights, W_r, x and y count: the dispatch copy, H and the slot rows are
-    overheads."""
+    gate/up GEMM reads the dispatched rows -- or, where it gathers them, the
+    token matrix itself -- and writes H; the down GEMM reads H and writes the
+    weighted (token, slot) rows).  For the whole block only the weights, W_r,
+    x and y count: the dispatch copy, H and the slot rows are overheads."""
     d, E, k, I, I_s = c["d"], c["E"], c["k"], c["I"], c["I_s"]
     ab = 4 if c["act"] == "f32" else 2
     wb = {"f32": 4, "bf16": 2, "fp8": 1}[c["w"]]
@@ -162,7 +174,8 @@ def work_model(c, counts, T):
     w_gu = (active * 2 * d * I + sh * 2 * d * I_s) * wb
     w_dn = (active * d * I + sh * d * I_s) * wb
     h_bytes = (R * I + sh * T * I_s) * ab
-    g1 = {"bytes": w_gu + (R + sh * T) * d * ab + h_bytes, "flops": 4 * d * (R * I + sh * T * I_s)}
+    a_in = (T if gathers_rows(c, T) else R + sh * T) * d * ab
+    g1 = {"bytes": w_gu + a_in + h_bytes, "flops": 4 * d * (R * I + sh * T * I_s)}
     g2 = {"bytes": w_dn + h_bytes + (R + sh * T) * d * ab, "flops": 2 * d * (R * I + sh * T * I_s)}
     layer = {"bytes": w_gu + w_dn + E * d * ab + 2 * T * d * ab,
              "flops": 2 * T * d * E + 6 * d * (R * I + sh * T * I_s)}

@@ -134,9 +134,13 @@ MOE_API moe_status moe_combine(const moe_problem* p, const void* y_perm, const i
                        const float* topk_w, const int32_t* offs, void* y, void* stream);
 
 /* The whole block, fused: router + top-k, dispatch, gate/up GEMM with SwiGLU,
- * down GEMM whose epilogue applies the routing weight and adds into y, plus
- * the shared expert.  y [T, d] in the activation type.  topk_ids_out and
- * topk_w_out ([T, k]) may be NULL.  ws: moe_workspace_size() bytes. */
+ * down GEMM whose epilogue applies the routing weight and stores each row in
+ * (token, slot) order, then one ordered fp32 sum per token of its k slot rows
+ * and its shared-expert row (reproducible: no atomics).  y [T, d] in the activation type.  topk_ids_out and
+ * topk_w_out ([T, k]) may be NULL.  ws: moe_workspace_size() bytes.
+ * On the row-tiled bf16 form (see moe_set_path) with T * d * 2 <= 32 MiB the
+ * gate/up GEMM reads each dispatched row straight from x (the rows stay in
+ * L2 while the weights stream), and the dispatch writes no copy of them. */
 MOE_API moe_status moe_layer_forward(const moe_problem* p, const void* x, const void* w_router,
                              const float* router_bias, const void* w_gate, const void* w_up,
                              const void* w_down, const void* ws_gate, const void* ws_up,

@@ -25,6 +25,10 @@
 //                 Store     out[r, n] = D -> bf16
 //                 Logits    part[split][r, n] = D (+ nothing) -> fp32
 //                 TopK      the router's softmax top-k of D + bias per row
+//   warps 10..13 (GATHER only) fetch the A rows straight from the token
+//               matrix by row index (cp.async, 128-byte swizzle written by
+//               hand): the gate/up GEMM of the fused forward needs no
+//               dispatched copy of its activation rows.
 // Rows of a tile past the end of its group are computed and discarded; rows
 // never mix in a GEMM, so those rows cannot disturb the kept ones.
 //
@@ -81,6 +85,11 @@ struct TcGemmArgs {
   float* cand_v;
   int32_t* cand_e;
   int32_t* cand_cnt;
+  // GATHER: A row r is x[row_tok[r]] (row stride ldx elements), gathered by
+  // the kernel instead of loaded from the dispatched-row matrix
+  const bf16* gx;
+  const int32_t* row_tok;
+  int64_t ldx;
   // E4M3 weights: fp32 scales per 128 x 128 block, [E][N/128][K/128] routed,
   // [N/128][K/128] shared; B = gate (or the single operand), C = up
   const float *sc_b_r, *sc_b_s, *sc_c_r, *sc_c_s;
@@ -148,8 +157,9 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
     if (clock64() - t0 > kWaitLimitCycles) break;
 }
 
-template <int BN, bool DUAL, int STAGES, bool FP8 = false>
+template <int BN, bool DUAL, int STAGES, bool FP8 = false, bool GATHER = false>
 struct TcGemmCfg {
+  static_assert(!(FP8 && GATHER), "the gathered A path is bf16 only");
   static constexpr int A_BYTES = kBM * kBK * 2;
   static constexpr int B_BYTES = BN * kBK * 2;
   static constexpr int NB = DUAL ? 2 * BN : BN;          // B rows per stage (gate rows, then up rows)
@@ -162,7 +172,8 @@ struct TcGemmCfg {
   // epilogue warps: 4 (one per TMEM lane quarter) with E4M3 weights, else 8
   // (two per quarter, splitting the accumulator columns) so stores drain faster
   static constexpr int EPI_WARPS = FP8 ? 4 : 8;
-  static constexpr int THREADS = FP8 ? 192 + NB + 32 : 64 + 32 * EPI_WARPS;
+  static constexpr int GATHER_WARPS = GATHER ? 4 : 0;  // A rows gathered from x with cp.async
+  static constexpr int THREADS = FP8 ? 192 + NB + 32 : 64 + 32 * (EPI_WARPS + GATHER_WARPS);
   static constexpr int ACC_COLS = DUAL ? 2 * BN : BN;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
   // + 4 + 4 handoff barriers of the router epilogue (one pair per lane quarter)
@@ -493,12 +504,12 @@ __device__ __forceinline__ bool topk_epilogue(const TcGemmArgs& p, const TileInf
   return true;
 }
 
-template <int BN, bool DUAL, int STAGES, int EPI, bool FP8 = false>
-__global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
+template <int BN, bool DUAL, int STAGES, int EPI, bool FP8 = false, bool GATHER = false>
+__global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
               const __grid_constant__ CUtensorMap tmB_r, const __grid_constant__ CUtensorMap tmB_s,
               const __grid_constant__ CUtensorMap tmC_r, const __grid_constant__ CUtensorMap tmC_s, TcGemmArgs p) {
-  using Cfg = TcGemmCfg<BN, DUAL, STAGES, FP8>;
+  using Cfg = TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint8_t* raw_ring = smem + STAGES * Cfg::STAGE_BYTES;       // FP8 only
@@ -522,7 +533,8 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
   const unsigned tcode = kStatusTimeoutBase | (kKernGemmTc << 8);
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(full + s, FP8 ? Cfg::NB / 32 : 1);  // FP8: one arrival per converter warp
+      // FP8: one arrival per converter warp; GATHER: the B loads plus one per gather warp
+      mbar_init(full + s, FP8 ? Cfg::NB / 32 : 1 + Cfg::GATHER_WARPS);
       mbar_init(empty + s, 1);
       mbar_init(a_full + s, 1);
     }
@@ -608,8 +620,8 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
           } else {
             uint8_t* sa = smem + stage * Cfg::STAGE_BYTES;
             uint8_t* sb = sa + Cfg::A_BYTES;
-            mbar_arrive_expect_tx(land, Cfg::STAGE_BYTES);
-            tma_load_2d(sa, sh ? &tmA_s : &tmA_r, land, kb * kBK, (int)t.row0, pol_a);
+            mbar_arrive_expect_tx(land, GATHER ? Cfg::STAGE_BYTES - Cfg::A_BYTES : Cfg::STAGE_BYTES);
+            if (!GATHER) tma_load_2d(sa, sh ? &tmA_s : &tmA_r, land, kb * kBK, (int)t.row0, pol_a);
             if (sh) tma_load_2d(sb, &tmB_s, land, kb * kBK, t.n0, pol_w);
             else tma_load_3d(sb, &tmB_r, land, kb * kBK, t.n0, t.g, pol_w);
             if (DUAL) {
@@ -737,6 +749,73 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8>::THREADS, 1)
         acc = 0;
         acc_phase ^= 1;
       }
+    }
+  } else if (GATHER) {
+    // ------------------------------------------------ A rows gathered from x (warps 10..13)
+    // Row r of a tile is x[row_tok[row0 + r]], zeros past the group or the
+    // buffer (and past K): thread gt copies 16-byte chunk gt % 8 of rows
+    // gt / 8 + RS i (RS = 4 * gather warps) into the 128-byte-swizzled A tile
+    // with cp.async, so 8 lanes read one row's 128 contiguous bytes.  A stage
+    // goes to the MMA warp (one arrival per gather warp on `full`, after the
+    // warp's copies have landed and the async proxy has been fenced) once the
+    // next stage's copies are issued (LAG = 1).  Holding stages longer ties up
+    // ring slots that the weight loads need: releasing STAGES - 1 stages late
+    // made the gate/up GEMM 30 % slower than 1 or 2 late (measured; 4 gather
+    // warps beat 2 by about 1 %).
+    constexpr int LAG = 1;
+    constexpr int RS = 4 * (Cfg::GATHER_WARPS > 0 ? Cfg::GATHER_WARPS : 1), RPT = kBM / RS;  // row stride, rows per thread
+    const int gt = threadIdx.x - 32 * (2 + Cfg::EPI_WARPS);
+    const int ch = gt & 7, rb = gt >> 3;
+    const uint32_t sw = (uint32_t)(ch ^ (rb & 7)) << 4;  // rows rb + RS i share their row-in-atom
+    const uint64_t pol_x = policy_evict_last();
+    int stage = 0, issued = 0, arrived = 0;
+    uint32_t phase = 0;
+    bool stop = false;
+    for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
+      const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
+      const bf16* src[RPT];
+      uint32_t live = 0;
+#pragma unroll
+      for (int i = 0; i < RPT; ++i) {
+        const int r = rb + RS * i;
+        const int64_t grow = t.row0 + r;
+        const bool in = t.m0 + r < t.rows && grow < p.rows_cap;
+        const int64_t tok = in ? (int64_t)__ldg(p.row_tok + grow) : 0;
+        src[i] = p.gx + tok * p.ldx + ch * 8;
+        live |= (uint32_t)in << i;
+      }
+      const int K = t.g == p.E ? p.K_s : p.K_r;
+      for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        if (!__all_sync(0xffffffffu, mbar_wait(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 10))) {
+          stop = true;  // the warp stops as one
+          break;
+        }
+        const uint32_t sa = smem_u32(smem + stage * Cfg::STAGE_BYTES) + sw;
+        const uint32_t kin = kb * kBK + ch * 8 < K ? 0xffffu : 0u;
+#pragma unroll
+        for (int i = 0; i < RPT; ++i)
+          cp_async_16(sa + (rb + RS * i) * 128, src[i] + kb * kBK, (live & kin) >> i & 1u ? 16u : 0u, pol_x);
+        cp_async_commit();
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+        if (issued - arrived > LAG) {
+          cp_async_wait<LAG>();
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(full + arrived % STAGES);
+          ++arrived;
+        }
+      }
+    }
+    cp_async_wait<0>();  // every copy lands before the CTA can exit
+    if (!stop) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      for (; arrived < issued; ++arrived)
+        if (lane == 0) mbar_arrive(full + arrived % STAGES);
     }
   } else if (FP8 && warp < 6 + Cfg::NB / 32) {
     // ------------------------------------------------ E4M3 -> bf16 converters
