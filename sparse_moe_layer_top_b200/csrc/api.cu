@@ -452,8 +452,8 @@ static Layout layout(const moe_problem& p, bool forward) {
   const int64_t n = p.T * p.k, Rp = rows_total(p);
   const size_t ab = esize(p.act_dtype);
   L.counts = take(n_chunks(p) * p.E * 4);
-  L.pre_a = take((p.E + 2) * 4);
-  L.pre_b = take((p.E + 2) * 4);
+  L.pre_a = take((p.E + 3) * 4);  // tile prefix [E+2] + the GEMM's tile-claim counter
+  L.pre_b = take((p.E + 3) * 4);
   if (p.act_dtype == MOE_BF16) L.part = take(router_scratch_bytes(p));
   if (forward) {
     L.ids = take(n * 4);
@@ -739,6 +739,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   a.sc_c_r = sp[1];
   a.sc_c_s = sp[4];
   a.status = dev->status;
+  if (!FP8) a.sched = pre_a + p.E + 2;  // tiles claimed in order (the prefix writer zeroed it)
   PROF_BEGIN("gemm_tc_swiglu", st);
   if (!FP8 && g.x) {
     a.gx = (const bf16*)g.x;
@@ -771,6 +772,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   b.sc_b_r = sp[2];
   b.sc_b_s = sp[5];
   b.status = dev->status;
+  if (!FP8) b.sched = pre_b + p.E + 2;
   if (o.ys) {
     b.ys = (bf16*)o.ys;
     b.ldy = p.d;

@@ -67,13 +67,17 @@ __device__ __forceinline__ int block_incl_scan(int v, int* sm_warp) {
 }
 
 // Tile prefix of one schedule from the group sizes (E+1 groups, one thread each).
+// prefix[E + 2] is the GEMM's tile-claim counter, zeroed here (see TcGemmArgs::sched).
 __device__ __forceinline__ void write_tile_prefix(const Schedule& s, int E, int rows_g, int32_t* prefix,
                                                   int* sm_warp) {
   int g = threadIdx.x;
   int tiles = (g <= E) ? sched_tiles(s, g, E, rows_g) : 0;
   int incl = block_incl_scan(tiles, sm_warp);
   if (g <= E) prefix[g] = incl - tiles;
-  if (g == E) prefix[E + 1] = incl;
+  if (g == E) {
+    prefix[E + 1] = incl;
+    prefix[E + 2] = 0;
+  }
 }
 
 // Tile prefixes from caller-supplied group offsets (the expert stage alone).
@@ -187,6 +191,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
           pf[E] = s_tot;
           pf[E + 1] = s_tot + sched_tiles(sc, E, E, has_shared ? (int)T : 0);
         }
+        pf[E + 2] = 0;  // the GEMM's tile-claim counter
       }
       __syncthreads();
     }

@@ -85,6 +85,10 @@ struct TcGemmArgs {
   float* cand_v;
   int32_t* cand_e;
   int32_t* cand_cnt;
+  // Tile order (bf16 kernels): NULL = CTA c takes tiles c, c + grid, ...;
+  // else a counter (zeroed by whoever wrote `prefix`) from which a CTA claims
+  // each tile after its first, so CTAs that draw cheap tiles draw more.
+  int* sched;
   // GATHER: A row r is x[row_tok[r]] (row stride ldx elements), gathered by
   // the kernel instead of loaded from the dispatched-row matrix
   const bf16* gx;
@@ -177,7 +181,8 @@ struct TcGemmCfg {
   static constexpr int ACC_COLS = DUAL ? 2 * BN : BN;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
   // + 4 + 4 handoff barriers of the router epilogue (one pair per lane quarter)
-  static constexpr int BAR_BYTES = (3 * STAGES + 2 * RAW_STAGES + 5 + 8) * 8 + 16;
+  // + 4 + 4 barriers and 4 ints of the tile queue
+  static constexpr int BAR_BYTES = (3 * STAGES + 2 * RAW_STAGES + 5 + 8 + 8) * 8 + 16 + 16;
   static constexpr int SCHED_INTS = 2 * (512 + 2);  // tile prefix + group offsets, E <= 512
   // epilogue staging: 32 rows x 64 bytes per epilogue warp
   static constexpr int EPI_OFF = (RING_BYTES + BAR_BYTES + SCHED_INTS * 4 + 127) / 128 * 128;
@@ -504,6 +509,46 @@ __device__ __forceinline__ bool topk_epilogue(const TcGemmArgs& p, const TileInf
   return true;
 }
 
+// A CTA's tile sequence (bf16 kernels), handed from the producer thread to the
+// other roles through a 4-slot ring in shared memory: the producer puts each
+// tile (a value >= total ends the sequence); every consumer role takes them in
+// order, one arrival per warp on `empty`.  Waits are bounded; on abort, take()
+// returns -1.
+struct TileQueue {
+  int* id;
+  uint64_t* full;
+  uint64_t* empty;
+  int slot;
+  uint32_t phase;
+  __device__ __forceinline__ TileQueue(int* i, uint64_t* f, uint64_t* e) : id(i), full(f), empty(e), slot(0), phase(0) {}
+  __device__ __forceinline__ void advance() {
+    if (++slot == 4) {
+      slot = 0;
+      phase ^= 1;
+    }
+  }
+  // producer thread
+  __device__ __forceinline__ bool put(int tile, volatile int* abort_flag, unsigned* status, unsigned where) {
+    if (!mbar_wait(empty + slot, phase ^ 1, abort_flag, status, where)) return false;
+    id[slot] = tile;
+    mbar_arrive(full + slot);
+    advance();
+    return true;
+  }
+  // a whole warp (every lane gets the tile), or one thread (warp_wide false)
+  __device__ __forceinline__ int take(bool warp_wide, int lane, volatile int* abort_flag, unsigned* status,
+                                      unsigned where) {
+    bool ok = mbar_wait(full + slot, phase, abort_flag, status, where);
+    if (warp_wide) ok = __all_sync(0xffffffffu, ok);
+    if (!ok) return -1;
+    const int t = id[slot];
+    if (warp_wide) __syncwarp();
+    if (!warp_wide || lane == 0) mbar_arrive(empty + slot);
+    advance();
+    return t;
+  }
+};
+
 template <int BN, bool DUAL, int STAGES, int EPI, bool FP8 = false, bool GATHER = false>
 __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THREADS, 1)
     k_gemm_tc(const __grid_constant__ CUtensorMap tmA_r, const __grid_constant__ CUtensorMap tmA_s,
@@ -523,7 +568,10 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
   uint64_t* raw_empty = raw_full + Cfg::RAW_STAGES;  // FP8: raw tile converted
   uint64_t* hfull = raw_empty + Cfg::RAW_STAGES;  // router epilogue: second warp's list written
   uint64_t* hempty = hfull + 4;                    // router epilogue: list merged, slot free
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(hempty + 4);
+  uint64_t* tq_full = hempty + 4;                  // tile queue (bf16 kernels)
+  uint64_t* tq_empty = tq_full + 4;
+  int* tq_id = reinterpret_cast<int*>(tq_empty + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq_id + 4);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* s_pre = reinterpret_cast<int32_t*>(smem + Cfg::RING_BYTES + Cfg::BAR_BYTES);
   int32_t* s_offs = s_pre + 514;
@@ -550,6 +598,8 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
     for (int q = 0; q < 4; ++q) {
       mbar_init(hfull + q, 32);
       mbar_init(hempty + q, 32);
+      mbar_init(tq_full + q, 1);
+      mbar_init(tq_empty + q, 1 + Cfg::EPI_WARPS + Cfg::GATHER_WARPS);  // MMA thread + each consumer warp
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -596,7 +646,10 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
       uint64_t* free0 = FP8 ? raw_empty : empty;
       int stage = 0;
       uint32_t phase = 0, issued = 0, last_par = 0;
-      for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      TileQueue tq(tq_id, tq_full, tq_empty);
+      for (int tile = blockIdx.x;;) {
+        if (!FP8 && !tq.put(min(tile, total), abort_flag, p.status, tcode | 11)) break;
+        if (tile >= total) break;
         const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
         const bool sh = t.g == p.E;
         bool ok = true;
@@ -638,6 +691,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
           }
         }
         if (!ok) break;
+        tile = (!FP8 && p.sched) ? (int)gridDim.x + atomicAdd(p.sched, 1) : tile + (int)gridDim.x;
       }
       if (*abort_flag)  // copies in flight must land before the CTA exits
         for (int s = 0; s < RING; ++s)
@@ -654,7 +708,10 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
       int stage = 0, acc = 0;
       uint32_t phase = 0, acc_phase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      TileQueue tq(tq_id, tq_full, tq_empty);
+      for (int tile = FP8 ? (int)blockIdx.x : tq.take(false, lane, abort_flag, p.status, tcode | 12);
+           tile >= 0 && tile < total && ok;
+           tile = FP8 ? tile + (int)gridDim.x : tq.take(false, lane, abort_flag, p.status, tcode | 12)) {
         const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
         if (!mbar_wait(tempty + acc, acc_phase ^ 1, abort_flag, p.status, tcode | 2)) break;
         tc_fence_after();
@@ -702,7 +759,10 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
     const int row = q * 32 + lane;
     int acc = 0;
     uint32_t acc_phase = 0, hpar = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    TileQueue tq(tq_id, tq_full, tq_empty);
+    for (int tile = FP8 ? (int)blockIdx.x : tq.take(true, lane, abort_flag, p.status, tcode | 13);
+         tile >= 0 && tile < total;
+         tile = FP8 ? tile + (int)gridDim.x : tq.take(true, lane, abort_flag, p.status, tcode | 13)) {
       const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
       if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)))
         break;  // the warp stops as one: its TMEM loads are warp-collective
@@ -771,7 +831,9 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
     int stage = 0, issued = 0, arrived = 0;
     uint32_t phase = 0;
     bool stop = false;
-    for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
+    TileQueue tq(tq_id, tq_full, tq_empty);
+    for (int tile = tq.take(true, lane, abort_flag, p.status, tcode | 14); tile >= 0 && tile < total && !stop;
+         tile = tq.take(true, lane, abort_flag, p.status, tcode | 14)) {
       const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
       const bf16* src[RPT];
       uint32_t live = 0;
