@@ -251,6 +251,9 @@ def barrier(world, device=None):
         dist.barrier()
 
 
+E2E_MIN_STEPS = 50
+
+
 def e2e_pipelined(layer, x, y, K, dev):
     import torch
     xh = [x.cpu().pin_memory() for _ in range(2)]
@@ -358,7 +361,10 @@ def run_ours(args):
     # streams with two buffers each, as a serving loop would run them: the
     # host->device copy of step i+1 and the device->host copy of step i-1
     # overlap the forward of step i.  Per-step time = whole timed region / K.
-    e2e_ms = e2e_pipelined(layer, x, y, K, dev)
+    # at least E2E_MIN_STEPS steps, so that filling and draining the pipeline
+    # (one step's copy in, one step's copy out) is spread as in a serving loop
+    K_e2e = max(K, E2E_MIN_STEPS)
+    e2e_ms = e2e_pipelined(layer, x, y, K_e2e, dev)
     e2e_max, _ = aggregate(e2e_ms, T, world, dev)
     s, detail = moe.device_status()
     if s != 0:
@@ -415,7 +421,7 @@ def run_ours(args):
             "roofline": roof, "layer_roofline": layer_roof, "cpu_baseline": cpu,
             "e2e": {"value": tokens_all / (e2e_max / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": x.numel() * x.element_size(),
-                    "d2h_bytes_per_step": y.numel() * y.element_size(), "ms_per_step": e2e_max,
+                    "d2h_bytes_per_step": y.numel() * y.element_size(), "ms_per_step": e2e_max, "steps": K_e2e,
                     "pipelining": "host->device copy of step i+1 and device->host copy of step i-1 "
                                   "overlap the forward of step i (3 streams, 2 buffers)"},
             "gpu_launches": launches_per_step * K, "launches_per_step": launches_per_step,
