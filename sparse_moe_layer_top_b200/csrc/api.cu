@@ -451,7 +451,8 @@ static Layout layout(const moe_problem& p, bool forward) {
   };
   const int64_t n = p.T * p.k, Rp = rows_total(p);
   const size_t ab = esize(p.act_dtype);
-  L.counts = take(n_chunks(p) * p.E * 4);
+  // chunk histograms, then the fused router's row-tile counters (one memset clears both)
+  L.counts = take(n_chunks(p) * p.E * 4 + n_chunks(p) * 4 * 4);
   L.pre_a = take((p.E + 3) * 4);  // tile prefix [E+2] + the GEMM's tile-claim counter
   L.pre_b = take((p.E + 3) * 4);
   if (p.act_dtype == MOE_BF16) L.part = take(router_scratch_bytes(p));
@@ -511,12 +512,15 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
     CUtensorMap bw64;
     if ((s = map2d(&bw64, wr, p.d, p.E, p.d, kTopkBN)) != MOE_OK) return s;
     char* scratch = reinterpret_cast<char*>(part);
-    if (ts.ntc > 1) {
-      CUDA_TRY(cudaMemsetAsync(scratch + ts.cnt_off, 0, (size_t)ts.row_tiles * 4 * 4, st));
-      pdl_reset();
-    }
+    // the row-tile counters: after the chunk histograms when there are some
+    // (one memset for both; kChunkTokens == kBM, so there is one counter
+    // quadruple per chunk), else in the scratch
+    int32_t* cnt = counts ? counts + n_chunks(p) * p.E : reinterpret_cast<int32_t*>(scratch + ts.cnt_off);
     if (counts) {
-      CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * p.E * 4, st));
+      CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * (p.E + 4) * 4, st));
+      pdl_reset();
+    } else if (ts.ntc > 1) {
+      CUDA_TRY(cudaMemsetAsync(cnt, 0, (size_t)ts.row_tiles * 4 * 4, st));
       pdl_reset();
     }
     TcGemmArgs a{};
@@ -533,7 +537,7 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
     a.tw = tw;
     a.bias = bias;
     a.counts = counts;
-    a.cand_cnt = reinterpret_cast<int32_t*>(scratch + ts.cnt_off);
+    a.cand_cnt = cnt;
     a.cand_v = reinterpret_cast<float*>(scratch + ts.v_off);
     a.cand_e = reinterpret_cast<int32_t*>(scratch + ts.e_off);
     a.status = dev->status;
