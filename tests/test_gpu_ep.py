@@ -110,7 +110,8 @@ def _check_rank(inp, lo, hi, y, state):
     assert err <= TOL[key], "rel-L2 %.3g > %.3g" % (err, TOL[key])
 
 
-@pytest.mark.parametrize("G,tokens,I_s", [(2, [300, 212], 128), (4, [150, 0, 333, 117], 128), (4, [64, 64, 1, 9], 0)])
+@pytest.mark.parametrize("G,tokens,I_s", [(2, [300, 212], 128), (4, [150, 0, 333, 117], 128), (4, [64, 64, 1, 9], 0),
+                                          (8, [40, 0, 17, 1, 64, 5, 33, 2], 128)])
 def test_expert_parallel_ranks_emulated_on_one_gpu_match_the_oracle(moe, G, tokens, I_s):
     d, E, k, I = 256, 32, 4, 128
     inp = moe_inputs.make_inputs(sum(tokens), d, E, k, I, I_s, act="bf16", w="bf16", seed=11, shared=I_s > 0)
