@@ -213,9 +213,18 @@ __device__ __forceinline__ uint2 e4m3x4_scaled_bf16(uint32_t w, float sc) {
 // the block passes through the warp's 2 KB staging buffer (64 bytes per row,
 // 16-byte chunks XOR-swizzled so neither the row-wise writes nor the
 // column-wise reads conflict) and leaves as 8 rows x 64 contiguous bytes per
-// store instruction instead of 32 rows x 16 bytes.
+// store instruction instead of 32 rows x 16 bytes.  The stores carry an L2
+// evict-last hint: what the epilogues write (H, the weighted slot rows) is
+// read back by the next kernel, while the weights stream past evict-first
+// (measured: down GEMM 138 -> 135 us at the 35B shape).
+__device__ __forceinline__ void st_global_evict_last(void* p, uint4 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w), "l"(pol)
+               : "memory");
+}
 __device__ __forceinline__ void store_rows_staged(uint8_t* stg, const uint32_t (&w)[16], char* rowp, int64_t colb,
                                                   int ncols, int lane) {
+  const uint64_t pol = policy_evict_last();
   const int sw = (lane >> 1) & 3;
 #pragma unroll
   for (int j = 0; j < 4; ++j)
@@ -228,7 +237,7 @@ __device__ __forceinline__ void store_rows_staged(uint8_t* stg, const uint32_t (
     const int rr = idx >> 2, cc = idx & 3;
     char* rp = reinterpret_cast<char*>(__shfl_sync(0xffffffffu, reinterpret_cast<uintptr_t>(rowp), rr));
     const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 64 + ((cc ^ ((rr >> 1) & 3)) << 4));
-    if (rp && cc * 8 < ncols) *reinterpret_cast<uint4*>(rp + colb + cc * 16) = v;
+    if (rp && cc * 8 < ncols) st_global_evict_last(rp + colb + cc * 16, v, pol);
   }
   __syncwarp();
 }
