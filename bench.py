@@ -144,16 +144,12 @@ def routing_counts(moe, layer, x):
     return cnt
 
 
-GATHER_MAX_BYTES = 32 << 20
-
-
 def gathers_rows(c, T):
     """Whether the fused forward's gate/up GEMM reads its rows straight from the
-    token matrix (include/moe.h, moe_layer_forward: the row-tiled bf16 form,
-    i.e. 64*E < T*k < 2048*E on the automatic path, with T*d*2 <= 32 MiB)."""
-    k, E = c["k"], c["E"]
-    rows_form = 64 * E < T * k < 2048 * E
-    return rows_form and c["act"] == "bf16" and c["w"] == "bf16" and T * c["d"] * 2 <= GATHER_MAX_BYTES
+    token matrix, as the library decides it (moe_forward_plan, host only)."""
+    import sparse_moe_layer_top_b200 as moe
+    prob = moe.Problem.make(T, c["d"], c["E"], c["k"], c["I"], c["I_s"], c["act"], c["w"])
+    return moe.forward_plan(prob)["gathered"]
 
 
 def work_model(c, counts, T):

@@ -228,6 +228,19 @@ MOE_API moe_status moe_router_topk_static(const moe_problem* p, const void* x, c
                                   const float* router_bias, int32_t* topk_ids, float* topk_w,
                                   void* stream);
 
+/* What moe_layer_forward / moe_block_forward launch for problem p under the
+ * current moe_set_path, decided on the host (no CUDA call, no device needed):
+ * expert_form: 0 SIMT kernels, 1 row-tiled tensor-core GEMMs, 2 weight-row
+ * (swap-AB) GEMMs, 3 row-tiled GEMMs on CTA pairs; router_selects: 1 when the
+ * router's GEMM selects the top k in its epilogue (bf16, E <= 256, at least
+ * 16 tiles of 128 tokens), 0 for the split-K GEMM + top-k kernel or the SIMT
+ * router; gathered: 1 when the gate/up GEMM reads its rows straight from x.
+ * Any output pointer may be NULL.  Errors: those of moe_check_problem, and
+ * MOE_ERR_UNSUPPORTED where moe_set_path asks for a form the types do not
+ * allow. */
+MOE_API moe_status moe_forward_plan(const moe_problem* p, int32_t* expert_form, int32_t* router_selects,
+                            int32_t* gathered);
+
 /* Kernel-path selection for the calls above on the calling process:
  * 0 = automatic (tensor-core kernels where the types allow; for the expert
  *     GEMMs the weight-row form when T*k <= 64*E, i.e. when an expert sees at

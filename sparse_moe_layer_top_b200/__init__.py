@@ -18,7 +18,7 @@ import os
 import torch
 
 __all__ = ["MoEError", "Problem", "BlockOptions", "router_topk", "permute", "expert_ffn", "combine", "layer_forward",
-           "block_forward", "rmsnorm", "ep_expand_ids",
+           "block_forward", "rmsnorm", "ep_expand_ids", "forward_plan",
            "workspace_size", "stage_workspace_size", "set_path", "device_status", "last_launch_count",
            "profile_enable", "profile_read",
            "MoELayer", "lib_path", "F32", "BF16", "FP8_E4M3_B128"]
@@ -33,7 +33,7 @@ EXPORTS = ("moe_check_problem", "moe_workspace_size", "moe_stage_workspace_size"
            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_set_path",
            "moe_device_status", "moe_last_launch_count", "moe_profile_enable", "moe_profile_read",
            "moe_last_error_string", "moe_router_topk_static", "moe_block_forward", "moe_rmsnorm",
-           "moe_ep_expand_ids")
+           "moe_ep_expand_ids", "moe_forward_plan")
 
 
 class MoEError(RuntimeError):
@@ -82,6 +82,8 @@ def lib():
         L.moe_block_forward.argtypes = [PP, ctypes.POINTER(BlockOptions), P, P, P, P, P, P, P, P, P, P, P, P, P,
                                         P, ctypes.c_size_t, P]
         L.moe_ep_expand_ids.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, P, P]
+        I32P = ctypes.POINTER(ctypes.c_int32)
+        L.moe_forward_plan.argtypes = [PP, I32P, I32P, I32P]
         L.moe_rmsnorm.argtypes = [PP, P, P, ctypes.c_float, P, P]
         L.moe_set_path.argtypes = [ctypes.c_int]
         L.moe_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32)]
@@ -259,6 +261,17 @@ def rmsnorm(prob, x, norm_weight, eps=1e-6, out=None, stream=None):
     _check(lib().moe_rmsnorm(ctypes.byref(prob), _ptr(x), _ptr(norm_weight), float(eps), _ptr(out),
                              _stream(stream)))
     return out
+
+
+EXPERT_FORMS = ("simt", "rows", "weight_rows", "cta_pairs")
+
+
+def forward_plan(prob):
+    """What the fused forward launches for `prob` under the current path,
+    decided on the host: dict(expert_form, router_selects, gathered)."""
+    f, r, g = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(lib().moe_forward_plan(ctypes.byref(prob), ctypes.byref(f), ctypes.byref(r), ctypes.byref(g)))
+    return {"expert_form": EXPERT_FORMS[f.value], "router_selects": bool(r.value), "gathered": bool(g.value)}
 
 
 def ep_expand_ids(counts, G, E_local, R, ids=None, stream=None):

@@ -631,6 +631,13 @@ static void scale_parts(const moe_problem& p, const float* sc, const float* part
 // Largest token matrix the gate/up GEMM gathers from (a quarter of the 126 MB L2).
 constexpr int64_t kGatherMaxBytes = 32ll << 20;
 
+// Whether the fused forward's gate/up GEMM gathers its rows from the block's
+// input: the row-tiled bf16 form, with the token matrix small enough to stay
+// L2-resident while the weights stream past (every row is read k + 1 times).
+static bool gathers_rows(const moe_problem& p, int form) {
+  return form == kFormRows && p.w_dtype == MOE_BF16 && p.T * p.d * 2 <= kGatherMaxBytes;
+}
+
 // The gate/up GEMM's activation rows taken straight from the token matrix
 // (row r = x[row_tok[r]]) instead of from the dispatched rows; x NULL: not.
 struct GatherSrc {
@@ -1283,13 +1290,11 @@ static moe_status block_forward(const moe_problem* p, const moe_block_options* o
   Schedule sa, sb;
   schedules(*p, form, &sa, &sb);
   // the row-tiled bf16 gate/up GEMM gathers its rows from the block's input
-  // when that stays L2-resident while the weights stream past (every row is
-  // read k + 1 times): the dispatch then writes no copy of them.  Measured:
-  // 35B shape (x 16 MB) 0.524 -> 0.484 ms; the prefill shape (x 128 MB, larger
-  // than L2) 7 % slower gathered, so it keeps the copy.
+  // when that stays L2-resident: the dispatch then writes no copy of them.
+  // Measured: 35B shape (x 16 MB) 0.524 -> 0.484 ms; the prefill shape (x
+  // 128 MB, larger than L2) 7 % slower gathered, so it keeps the copy.
   GatherSrc gs;
-  if (form == kFormRows && p->w_dtype == MOE_BF16 && p->T * p->d * 2 <= kGatherMaxBytes)
-    gs = GatherSrc{xin, row_tok};
+  if (gathers_rows(*p, form)) gs = GatherSrc{xin, row_tok};
   s = launch_dispatch(*p, ids, tw, counted, offs, row_tok, row_w, pos, row_dst, counts, sa, pre_a, sb, pre_b, xin,
                       gs.x ? nullptr : xp, st, dev, gate);
   if (s != MOE_OK) return s;
@@ -1342,6 +1347,20 @@ moe_status moe_rmsnorm(const moe_problem* p, const void* x, const void* norm_wei
   if ((s = launch_prologue(*p, x, norm_weight, eps, nullptr, x_out, nullptr, (cudaStream_t)stream)) != MOE_OK)
     return s;
   g_launches = g_launches_pending;
+  return MOE_OK;
+}
+
+moe_status moe_forward_plan(const moe_problem* p, int32_t* expert_form, int32_t* router_selects,
+                            int32_t* gathered) {
+  moe_status s = check(p);
+  if (s != MOE_OK) return s;
+  int form;
+  if ((s = choose_form(*p, &form)) != MOE_OK) return s;
+  bool router_tc;
+  if ((s = choose(p->act_dtype == MOE_BF16, &router_tc)) != MOE_OK) return s;
+  if (expert_form) *expert_form = form;
+  if (router_selects) *router_selects = router_tc && router_fused(*p) ? 1 : 0;
+  if (gathered) *gathered = gathers_rows(*p, form) ? 1 : 0;
   return MOE_OK;
 }
 

@@ -131,3 +131,31 @@ def test_ep_expand_ids_rejected_before_any_launch():
     assert L.moe_ep_expand_ids(v(16), 2, 4, 10, None, None) == 1       # no output
     assert L.moe_ep_expand_ids(v(0x1008), 2, 4, 10, v(16), None) == 3  # misaligned
     assert L.moe_ep_expand_ids(None, 2, 4, 0, None, None) == 0         # nothing to do
+
+
+def test_forward_plan_on_the_host():
+    # the bench workloads' plans (host only: no device needed)
+    plan = lambda *a: moe.forward_plan(moe.Problem.make(*a))  # noqa: E731
+    assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16") == \
+        {"expert_form": "rows", "router_selects": True, "gathered": True}
+    assert plan(8192, 8192, 512, 10, 2048, 2048, "bf16", "bf16") == \
+        {"expert_form": "rows", "router_selects": False, "gathered": False}      # 512 experts; x > 32 MiB
+    assert plan(64, 8192, 512, 10, 2048, 2048, "bf16", "bf16")["expert_form"] == "weight_rows"
+    assert plan(2048, 8192, 512, 10, 2048, 2048, "bf16", "fp8")["expert_form"] == "weight_rows"
+    assert plan(32, 128, 16, 2, 64, 64, "f32", "f32") == \
+        {"expert_form": "simt", "router_selects": False, "gathered": False}
+    # the router selects in its epilogue from 16 token tiles on; the gather stops above 32 MiB of x
+    assert not plan(1920, 256, 64, 4, 128, 128, "bf16", "bf16")["router_selects"]
+    assert plan(1921, 256, 64, 4, 128, 128, "bf16", "bf16")["router_selects"]
+    assert plan(2048, 8192, 64, 8, 256, 256, "bf16", "bf16")["gathered"]        # exactly 32 MiB
+    assert not plan(2049, 8192, 64, 8, 256, 256, "bf16", "bf16")["gathered"]
+    # the path setting moves the form
+    try:
+        moe.set_path(4)
+        assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16")["expert_form"] == "cta_pairs"
+        moe.set_path(1)
+        assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16") == \
+            {"expert_form": "simt", "router_selects": False, "gathered": False}
+    finally:
+        moe.set_path(0)
+    assert moe.lib().moe_forward_plan(ctypes.byref(P(T=-1)), None, None, None) == 1
