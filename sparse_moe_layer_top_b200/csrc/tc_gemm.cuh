@@ -529,7 +529,8 @@ struct TileQueue {
   uint64_t* empty;
   int slot;
   uint32_t phase;
-  __device__ __forceinline__ TileQueue(int* i, uint64_t* f, uint64_t* e) : id(i), full(f), empty(e), slot(0), phase(0) {}
+  __device__ __forceinline__ TileQueue(int* i, uint64_t* f, uint64_t* e)
+      : id(i), full(f), empty(e), slot(0), phase(0) {}
   __device__ __forceinline__ void advance() {
     if (++slot == 4) {
       slot = 0;
@@ -832,7 +833,8 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
     // made the gate/up GEMM 30 % slower than 1 or 2 late (measured; 4 gather
     // warps beat 2 by about 1 %).
     constexpr int LAG = 1;
-    constexpr int RS = 4 * (Cfg::GATHER_WARPS > 0 ? Cfg::GATHER_WARPS : 1), RPT = kBM / RS;  // row stride, rows per thread
+    // row stride and rows per thread
+    constexpr int RS = 4 * (Cfg::GATHER_WARPS > 0 ? Cfg::GATHER_WARPS : 1), RPT = kBM / RS;
     const int gt = threadIdx.x - 32 * (2 + Cfg::EPI_WARPS);
     const int ch = gt & 7, rb = gt >> 3;
     const uint32_t sw = (uint32_t)(ch ^ (rb & 7)) << 4;  // rows rb + RS i share their row-in-atom
