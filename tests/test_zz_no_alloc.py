@@ -72,3 +72,24 @@ def test_static_router_rejects_what_does_not_fit():
     torch.cuda.synchronize()
     assert rc == 2
     assert b"scratch" in L.moe_last_error_string()
+
+
+def test_static_router_rejects_candidate_lists_that_do_not_fit():
+    import sparse_moe_layer_top_b200 as moe
+    # E <= 256: the router selects in its GEMM epilogue, and its scratch is the
+    # candidate lists, 64 KB per 128-token tile (4 expert tiles x 16 slots x
+    # 128 rows x (logit, expert)): 512 tiles fill the 32 MiB array exactly, and
+    # the row-tile counters come on top.  Real buffers, as above.
+    T, d, E, k = 65536, 256, 256, 8
+    x = torch.zeros((T, d), dtype=torch.bfloat16, device="cuda")
+    w_r = torch.zeros((E, d), dtype=torch.bfloat16, device="cuda")
+    ids = torch.empty((T, k), dtype=torch.int32, device="cuda")
+    tw = torch.empty((T, k), dtype=torch.float32, device="cuda")
+    prob = moe.Problem.make(T, d, E, k, 128, 128, "bf16", "bf16")
+    assert moe.forward_plan(prob)["router_selects"]
+    L = moe.lib()
+    rc = L.moe_router_topk_static(ctypes.byref(prob), _p(x), _p(w_r), None, _p(ids), _p(tw),
+                                  ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert rc == 2
+    assert b"scratch" in L.moe_last_error_string()
