@@ -5,6 +5,10 @@ kernels.  Tensors are CUDA torch tensors (contiguous, row-major); the calls
 enqueue on the current torch stream and never synchronise.  The library is
 built in-tree (``python -m sparse_moe_layer_top_b200.build``) and loaded on
 first use; every call raises if it is missing -- there is no fallback.
+The C ABI sees only pointers, so every call first checks its tensors' element
+types and sizes against the problem and raises ValueError, before any pointer
+is taken, when a buffer is of the wrong type or too small for what the call
+reads or writes.
 
 Entry points mirror ``include/moe.h``: ``router_topk``, ``permute``,
 ``expert_ffn``, ``combine``, ``layer_forward``, ``block_forward``,
@@ -106,6 +110,44 @@ def _check(status):
         raise MoEError(status, lib().moe_last_error_string().decode())
 
 
+_F32, _I32 = (torch.float32,), (torch.int32,)
+_ACT_TYPES = {F32: (torch.float32,), BF16: (torch.bfloat16,)}
+_W_TYPES = {F32: (torch.float32,), BF16: (torch.bfloat16,), FP8_E4M3_B128: (torch.float8_e4m3fn, torch.uint8)}
+
+
+def _need(t, name, n, dtypes, row=None):
+    """t (if given) holds at least n elements of one of dtypes (None: the
+    problem's type code is invalid, which the library itself reports) and, if
+    it has two or more dimensions, rows of `row` elements."""
+    if t is None:
+        return
+    if dtypes is not None and t.dtype not in dtypes:
+        raise ValueError("%s: element type %s, expected %s" % (name, t.dtype, " or ".join(map(str, dtypes))))
+    if t.numel() < n:
+        raise ValueError("%s: %d elements, the problem needs %d" % (name, t.numel(), n))
+    if row is not None and t.dim() >= 2 and t.shape[-1] != row:
+        raise ValueError("%s: rows of %d elements, expected %d" % (name, t.shape[-1], row))
+
+
+def _need_weights(prob, wg, wu, wd, s_wg, s_wu, s_wd, scales):
+    d, E, I, I_s = prob.d, prob.E, prob.I, prob.I_s
+    wt = _W_TYPES.get(prob.w_dtype)
+    _need(wg, "w_gate", E * I * d, wt, d)
+    _need(wu, "w_up", E * I * d, wt, d)
+    _need(wd, "w_down", E * d * I, wt, I)
+    if I_s > 0:
+        _need(s_wg, "ws_gate", I_s * d, wt, d)
+        _need(s_wu, "ws_up", I_s * d, wt, d)
+        _need(s_wd, "ws_down", d * I_s, wt, I_s)
+    if prob.w_dtype == FP8_E4M3_B128:
+        blocks = 3 * E * (I // 128) * (d // 128) + (3 * (I_s // 128) * (d // 128) if I_s > 0 else 0)
+        _need(scales, "scales", blocks, _F32)
+
+
+def _nbytes(t):
+    return t.numel() * t.element_size()
+
+
 def _ptr(t):
     if t is None:
         return None
@@ -177,13 +219,19 @@ def _ws(nbytes, device, ws):
 
 def router_topk(prob, x, w_router, bias=None, topk_ids=None, topk_w=None, ws=None, stream=None):
     T, k = prob.T, prob.k
+    a = _ACT_TYPES.get(prob.act_dtype)
+    _need(x, "x", T * prob.d, a, prob.d)
+    _need(w_router, "w_router", prob.E * prob.d, a, prob.d)
+    _need(bias, "router_bias", prob.E, _F32)
+    _need(topk_ids, "topk_ids", T * k, _I32, k)
+    _need(topk_w, "topk_w", T * k, _F32, k)
     if topk_ids is None:
         topk_ids = torch.empty((T, k), dtype=torch.int32, device=x.device)
     if topk_w is None:
         topk_w = torch.empty((T, k), dtype=torch.float32, device=x.device)
     ws = _ws(stage_workspace_size(prob), x.device, ws)
     _check(lib().moe_router_topk(ctypes.byref(prob), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(topk_ids),
-                                 _ptr(topk_w), _ptr(ws), ws.numel(), _stream(stream)))
+                                 _ptr(topk_w), _ptr(ws), _nbytes(ws), _stream(stream)))
     return topk_ids, topk_w
 
 
@@ -193,6 +241,9 @@ def rows_total(prob):
 
 def permute(prob, x, topk_ids, topk_w, ws=None, stream=None):
     """-> dict(x_perm, row_tok, row_w, pos, offs)."""
+    _need(x, "x", prob.T * prob.d, _ACT_TYPES.get(prob.act_dtype), prob.d)
+    _need(topk_ids, "topk_ids", prob.T * prob.k, _I32, prob.k)
+    _need(topk_w, "topk_w", prob.T * prob.k, _F32, prob.k)
     dev = x.device
     Rp = rows_total(prob)
     out = dict(x_perm=torch.empty((Rp, prob.d), dtype=_act(prob), device=dev),
@@ -204,23 +255,34 @@ def permute(prob, x, topk_ids, topk_w, ws=None, stream=None):
     ws = _ws(nbytes, dev, ws)
     _check(lib().moe_permute(ctypes.byref(prob), _ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(out["x_perm"]),
                              _ptr(out["row_tok"]), _ptr(out["row_w"]), _ptr(out["pos"]), _ptr(out["offs"]),
-                             _ptr(ws), ws.numel(), _stream(stream)))
+                             _ptr(ws), _nbytes(ws), _stream(stream)))
     return out
 
 
 def expert_ffn(prob, x_perm, offs, wg, wu, wd, s_wg=None, s_wu=None, s_wd=None, scales=None, y_perm=None,
                ws=None, stream=None):
+    a, Rp = _ACT_TYPES.get(prob.act_dtype), rows_total(prob)
+    _need(x_perm, "x_perm", Rp * prob.d, a, prob.d)
+    _need(offs, "offs", prob.E + 2, _I32)
+    _need_weights(prob, wg, wu, wd, s_wg, s_wu, s_wd, scales)
+    _need(y_perm, "y_perm", Rp * prob.d, a, prob.d)
     dev = x_perm.device
     if y_perm is None:
         y_perm = torch.empty((x_perm.shape[0], prob.d), dtype=_act(prob), device=dev)
     ws = _ws(stage_workspace_size(prob), dev, ws)
     _check(lib().moe_expert_ffn(ctypes.byref(prob), _ptr(x_perm), _ptr(offs), _ptr(wg), _ptr(wu), _ptr(wd),
-                                _ptr(s_wg), _ptr(s_wu), _ptr(s_wd), _ptr(scales), _ptr(y_perm), _ptr(ws), ws.numel(),
+                                _ptr(s_wg), _ptr(s_wu), _ptr(s_wd), _ptr(scales), _ptr(y_perm), _ptr(ws), _nbytes(ws),
                                 _stream(stream)))
     return y_perm
 
 
 def combine(prob, y_perm, pos, topk_w, offs, y=None, stream=None):
+    a = _ACT_TYPES.get(prob.act_dtype)
+    _need(y_perm, "y_perm", rows_total(prob) * prob.d, a, prob.d)
+    _need(pos, "pos", prob.T * prob.k, _I32, prob.k)
+    _need(topk_w, "topk_w", prob.T * prob.k, _F32, prob.k)
+    _need(offs, "offs", prob.E + 2, _I32)
+    _need(y, "y", prob.T * prob.d, a, prob.d)
     if y is None:
         y = torch.empty((prob.T, prob.d), dtype=_act(prob), device=y_perm.device)
     _check(lib().moe_combine(ctypes.byref(prob), _ptr(y_perm), _ptr(pos), _ptr(topk_w), _ptr(offs), _ptr(y),
@@ -228,14 +290,27 @@ def combine(prob, y_perm, pos, topk_w, offs, y=None, stream=None):
     return y
 
 
+def _need_forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, y, topk_ids, topk_w):
+    T, d, k = prob.T, prob.d, prob.k
+    a = _ACT_TYPES.get(prob.act_dtype)
+    _need(x, "x", T * d, a, d)
+    _need(w_router, "w_router", prob.E * d, a, d)
+    _need(bias, "router_bias", prob.E, _F32)
+    _need_weights(prob, wg, wu, wd, s_wg, s_wu, s_wd, scales)
+    _need(y, "y", T * d, a, d)
+    _need(topk_ids, "topk_ids", T * k, _I32, k)
+    _need(topk_w, "topk_w", T * k, _F32, k)
+
+
 def layer_forward(prob, x, w_router, bias, wg, wu, wd, s_wg=None, s_wu=None, s_wd=None, scales=None, y=None,
                   topk_ids=None, topk_w=None, ws=None, stream=None):
+    _need_forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, y, topk_ids, topk_w)
     if y is None:
         y = torch.empty((prob.T, prob.d), dtype=_act(prob), device=x.device)
     ws = _ws(workspace_size(prob), x.device, ws)
     _check(lib().moe_layer_forward(ctypes.byref(prob), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(wg), _ptr(wu),
                                    _ptr(wd), _ptr(s_wg), _ptr(s_wu), _ptr(s_wd), _ptr(scales), _ptr(y),
-                                   _ptr(topk_ids), _ptr(topk_w), _ptr(ws), ws.numel(), _stream(stream)))
+                                   _ptr(topk_ids), _ptr(topk_w), _ptr(ws), _nbytes(ws), _stream(stream)))
     return y
 
 
@@ -244,18 +319,26 @@ def block_forward(prob, x, w_router, bias, wg, wu, wd, s_wg=None, s_wu=None, s_w
                   stream=None):
     """layer_forward with the block's neighbours: zero-centred RMSNorm of x
     (norm_weight [d]) and a sigmoid gate on the shared expert (shared_gate [d])."""
+    _need_forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, y, topk_ids, topk_w)
+    a = _ACT_TYPES.get(prob.act_dtype)
+    _need(norm_weight, "norm_weight", prob.d, a)
+    _need(shared_gate, "shared_gate", prob.d, a)
     if y is None:
         y = torch.empty((prob.T, prob.d), dtype=_act(prob), device=x.device)
     ws = _ws(workspace_size(prob), x.device, ws)
     opt = BlockOptions(_ptr(norm_weight), float(norm_eps), _ptr(shared_gate))
     _check(lib().moe_block_forward(ctypes.byref(prob), ctypes.byref(opt), _ptr(x), _ptr(w_router), _ptr(bias),
                                    _ptr(wg), _ptr(wu), _ptr(wd), _ptr(s_wg), _ptr(s_wu), _ptr(s_wd), _ptr(scales),
-                                   _ptr(y), _ptr(topk_ids), _ptr(topk_w), _ptr(ws), ws.numel(), _stream(stream)))
+                                   _ptr(y), _ptr(topk_ids), _ptr(topk_w), _ptr(ws), _nbytes(ws), _stream(stream)))
     return y
 
 
 def rmsnorm(prob, x, norm_weight, eps=1e-6, out=None, stream=None):
     """Zero-centred RMSNorm of the rows of x: x / sqrt(mean x^2 + eps) * (1 + norm_weight)."""
+    a = _ACT_TYPES.get(prob.act_dtype)
+    _need(x, "x", prob.T * prob.d, a, prob.d)
+    _need(norm_weight, "norm_weight", prob.d, a)
+    _need(out, "out", prob.T * prob.d, a, prob.d)
     if out is None:
         out = torch.empty_like(x)
     _check(lib().moe_rmsnorm(ctypes.byref(prob), _ptr(x), _ptr(norm_weight), float(eps), _ptr(out),
@@ -278,6 +361,8 @@ def ep_expand_ids(counts, G, E_local, R, ids=None, stream=None):
     """Expert parallelism, receive side: the local expert (int32 [R]) of every
     received row, rows arriving as blocks (source s, local expert e) in that
     order with counts[s * E_local + e] rows each (int32, on the device)."""
+    _need(counts, "counts", int(G) * int(E_local), _I32)
+    _need(ids, "ids", int(R), _I32)
     if ids is None:
         ids = torch.empty(max(int(R), 0), dtype=torch.int32, device=counts.device)
     _check(lib().moe_ep_expand_ids(_ptr(counts), int(G), int(E_local), int(R), _ptr(ids), _stream(stream)))
