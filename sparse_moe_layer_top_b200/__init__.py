@@ -290,28 +290,51 @@ def combine(prob, y_perm, pos, topk_w, offs, y=None, stream=None):
     return y
 
 
-def _need_forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, y, topk_ids, topk_w):
+def _need_params(prob, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, norm_weight=None, shared_gate=None):
+    """The block's parameters (independent of the token count)."""
+    a = _ACT_TYPES.get(prob.act_dtype)
+    _need(w_router, "w_router", prob.E * prob.d, a, prob.d)
+    _need(bias, "router_bias", prob.E, _F32)
+    _need_weights(prob, wg, wu, wd, s_wg, s_wu, s_wd, scales)
+    _need(norm_weight, "norm_weight", prob.d, a)
+    _need(shared_gate, "shared_gate", prob.d, a)
+
+
+def _need_tokens(prob, x, y, topk_ids, topk_w):
+    """One call's token buffers."""
     T, d, k = prob.T, prob.d, prob.k
     a = _ACT_TYPES.get(prob.act_dtype)
     _need(x, "x", T * d, a, d)
-    _need(w_router, "w_router", prob.E * d, a, d)
-    _need(bias, "router_bias", prob.E, _F32)
-    _need_weights(prob, wg, wu, wd, s_wg, s_wu, s_wd, scales)
     _need(y, "y", T * d, a, d)
     _need(topk_ids, "topk_ids", T * k, _I32, k)
     _need(topk_w, "topk_w", T * k, _F32, k)
 
 
-def layer_forward(prob, x, w_router, bias, wg, wu, wd, s_wg=None, s_wu=None, s_wd=None, scales=None, y=None,
-                  topk_ids=None, topk_w=None, ws=None, stream=None):
-    _need_forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, y, topk_ids, topk_w)
+def _forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, norm_weight, norm_eps, shared_gate, y,
+             topk_ids, topk_w, ws, stream, block):
+    """The fused forward on checked arguments (moe_block_forward when `block`)."""
     if y is None:
         y = torch.empty((prob.T, prob.d), dtype=_act(prob), device=x.device)
     ws = _ws(workspace_size(prob), x.device, ws)
-    _check(lib().moe_layer_forward(ctypes.byref(prob), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(wg), _ptr(wu),
-                                   _ptr(wd), _ptr(s_wg), _ptr(s_wu), _ptr(s_wd), _ptr(scales), _ptr(y),
-                                   _ptr(topk_ids), _ptr(topk_w), _ptr(ws), _nbytes(ws), _stream(stream)))
+    if block:
+        opt = BlockOptions(_ptr(norm_weight), float(norm_eps), _ptr(shared_gate))
+        _check(lib().moe_block_forward(ctypes.byref(prob), ctypes.byref(opt), _ptr(x), _ptr(w_router), _ptr(bias),
+                                       _ptr(wg), _ptr(wu), _ptr(wd), _ptr(s_wg), _ptr(s_wu), _ptr(s_wd),
+                                       _ptr(scales), _ptr(y), _ptr(topk_ids), _ptr(topk_w), _ptr(ws), _nbytes(ws),
+                                       _stream(stream)))
+    else:
+        _check(lib().moe_layer_forward(ctypes.byref(prob), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(wg), _ptr(wu),
+                                       _ptr(wd), _ptr(s_wg), _ptr(s_wu), _ptr(s_wd), _ptr(scales), _ptr(y),
+                                       _ptr(topk_ids), _ptr(topk_w), _ptr(ws), _nbytes(ws), _stream(stream)))
     return y
+
+
+def layer_forward(prob, x, w_router, bias, wg, wu, wd, s_wg=None, s_wu=None, s_wd=None, scales=None, y=None,
+                  topk_ids=None, topk_w=None, ws=None, stream=None):
+    _need_params(prob, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales)
+    _need_tokens(prob, x, y, topk_ids, topk_w)
+    return _forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, None, 0.0, None, y, topk_ids,
+                    topk_w, ws, stream, block=False)
 
 
 def block_forward(prob, x, w_router, bias, wg, wu, wd, s_wg=None, s_wu=None, s_wd=None, scales=None,
@@ -319,18 +342,10 @@ def block_forward(prob, x, w_router, bias, wg, wu, wd, s_wg=None, s_wu=None, s_w
                   stream=None):
     """layer_forward with the block's neighbours: zero-centred RMSNorm of x
     (norm_weight [d]) and a sigmoid gate on the shared expert (shared_gate [d])."""
-    _need_forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, y, topk_ids, topk_w)
-    a = _ACT_TYPES.get(prob.act_dtype)
-    _need(norm_weight, "norm_weight", prob.d, a)
-    _need(shared_gate, "shared_gate", prob.d, a)
-    if y is None:
-        y = torch.empty((prob.T, prob.d), dtype=_act(prob), device=x.device)
-    ws = _ws(workspace_size(prob), x.device, ws)
-    opt = BlockOptions(_ptr(norm_weight), float(norm_eps), _ptr(shared_gate))
-    _check(lib().moe_block_forward(ctypes.byref(prob), ctypes.byref(opt), _ptr(x), _ptr(w_router), _ptr(bias),
-                                   _ptr(wg), _ptr(wu), _ptr(wd), _ptr(s_wg), _ptr(s_wu), _ptr(s_wd), _ptr(scales),
-                                   _ptr(y), _ptr(topk_ids), _ptr(topk_w), _ptr(ws), _nbytes(ws), _stream(stream)))
-    return y
+    _need_params(prob, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, norm_weight, shared_gate)
+    _need_tokens(prob, x, y, topk_ids, topk_w)
+    return _forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, norm_weight, norm_eps,
+                    shared_gate, y, topk_ids, topk_w, ws, stream, block=True)
 
 
 def rmsnorm(prob, x, norm_weight, eps=1e-6, out=None, stream=None):
@@ -378,6 +393,9 @@ class MoELayer:
         self.shape = (d, E, k, I, I_s, act, w)
         self.w = (w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales)
         self.opts = (norm_weight, norm_eps, shared_gate)
+        # the parameters are checked once here; each call checks its token buffers
+        _need_params(self.problem(0), w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, norm_weight,
+                     shared_gate)
         self.device = wg.device
         self.ws = None
         if max_tokens:
@@ -394,15 +412,13 @@ class MoELayer:
 
     def __call__(self, x, y=None, topk_ids=None, topk_w=None, stream=None):
         prob = self.problem(x.shape[0])
+        _need_tokens(prob, x, y, topk_ids, topk_w)
         self._reserve(x.shape[0])
         w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales = self.w
         norm_weight, norm_eps, shared_gate = self.opts
-        if norm_weight is None and shared_gate is None:
-            return layer_forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, y=y,
-                                 topk_ids=topk_ids, topk_w=topk_w, ws=self.ws, stream=stream)
-        return block_forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, norm_weight=norm_weight,
-                             norm_eps=norm_eps, shared_gate=shared_gate, y=y, topk_ids=topk_ids, topk_w=topk_w,
-                             ws=self.ws, stream=stream)
+        block = norm_weight is not None or shared_gate is not None
+        return _forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, norm_weight, norm_eps,
+                        shared_gate, y, topk_ids, topk_w, self.ws, stream, block)
 
     @classmethod
     def from_inputs(cls, inp, max_tokens=0):

@@ -148,3 +148,21 @@ def test_expert_parallel_receive_side_checks_its_buffers():
         moe.ep_expand_ids(torch.zeros(8, dtype=torch.int32), 2, 4, 10, ids=torch.zeros(9, dtype=torch.int32))
     with pytest.raises(ValueError, match=ON_DEVICE):
         moe.ep_expand_ids(torch.zeros(8, dtype=torch.int32), 2, 4, 10)
+
+
+def test_layer_object_checks_its_weights_once_and_its_tokens_every_call():
+    a = _forward_args("bf16", "fp8")
+    p = a["prob"]
+    args = (p.d, p.E, p.k, p.I, p.I_s, a["w_router"], a["wg"], a["wu"], a["wd"], a["s_wg"], a["s_wu"], a["s_wd"])
+    with pytest.raises(ValueError, match="scales:"):
+        moe.MoELayer(*args, bias=a["bias"], scales=a["scales"][:3], act="bf16", w="fp8")
+    with pytest.raises(ValueError, match="shared_gate:"):
+        moe.MoELayer(*args, bias=a["bias"], scales=a["scales"], act="bf16", w="fp8",
+                     shared_gate=torch.zeros(p.d - 8, dtype=torch.bfloat16))
+    layer = moe.MoELayer(*args, bias=a["bias"], scales=a["scales"], act="bf16", w="fp8")
+    with pytest.raises(ValueError, match="x: element type"):
+        layer(a["x"].float())
+    with pytest.raises(ValueError, match="y:"):
+        layer(a["x"], y=a["y"][:-1])
+    with pytest.raises(ValueError, match=ON_DEVICE):
+        layer(a["x"], y=a["y"], topk_ids=a["topk_ids"], topk_w=a["topk_w"])
