@@ -73,17 +73,17 @@ class EPMoELayer:
     """One rank's share of an expert-parallel MoE block.
 
     w_router [E, d] and the shared expert are full replicas; wg, wu [E_l, I, d]
-    and wd [E_l, d, I] are this rank's experts, E_l = E / world.  ``ops`` is the
-    namespace of stage calls (default: this package)."""
+    and wd [E_l, d, I] are this rank's experts, E_l = E / world.  With E4M3
+    weights (w="fp8"), ``scales`` is this rank's packed block-scale buffer
+    (``split_scales``).  ``ops`` is the namespace of stage calls (default: this
+    package)."""
 
     def __init__(self, rank, world, d, E, k, I, I_s, w_router, wg, wu, wd, s_wg=None, s_wu=None, s_wd=None,
-                 bias=None, act="bf16", w="bf16", ops=None):
+                 bias=None, act="bf16", w="bf16", ops=None, scales=None):
         if world < 1 or not 0 <= rank < world:
             raise ValueError("rank %d of %d" % (rank, world))
         if E % world:
             raise ValueError("E = %d experts do not split over %d ranks" % (E, world))
-        if w == "fp8":
-            raise ValueError("expert parallelism takes bf16 or fp32 weights")
         if ops is None:
             import sparse_moe_layer_top_b200 as ops
         self.ops = ops
@@ -92,6 +92,13 @@ class EPMoELayer:
         self.E_l = E // world
         if wg.shape[0] != self.E_l or wu.shape[0] != self.E_l or wd.shape[0] != self.E_l:
             raise ValueError("rank weights must hold E / world = %d experts" % self.E_l)
+        if w == "fp8":
+            n = _scale_blocks(self.E_l, d, I, I_s)
+            if scales is None or scales.numel() != n:
+                raise ValueError("E4M3 weights need this rank's %d block scales (split_scales)" % n)
+        elif scales is not None:
+            raise ValueError("block scales are for E4M3 weights only")
+        self.scales = scales
         self.w_router, self.bias = w_router, bias
         self.wg, self.wu, self.wd = wg, wu, wd
         self.s_wg, self.s_wu, self.s_wd = s_wg, s_wu, s_wd
@@ -133,7 +140,8 @@ class EPMoELayer:
         ones = torch.ones((R_recv, 1), dtype=torch.float32, device=x_recv.device)
         prob = self._prob(R_recv, self.E_l, 1, 0)
         perm = self.ops.permute(prob, x_recv, ids, ones)
-        y_perm = self.ops.expert_ffn(prob, perm["x_perm"], perm["offs"], self.wg, self.wu, self.wd)
+        y_perm = self.ops.expert_ffn(prob, perm["x_perm"], perm["offs"], self.wg, self.wu, self.wd,
+                                     scales=self.scales)
         return self.ops.combine(prob, y_perm, perm["pos"], ones, perm["offs"])
 
     # -------------------------------------------------------------- step 4
@@ -150,7 +158,7 @@ class EPMoELayer:
         offs = torch.tensor([T] * (self.E_l + 1) + [2 * T], dtype=torch.int32, device=st.x_perm.device)
         prob = self._prob(T, self.E_l, 1, self.I_s)
         self.ops.expert_ffn(prob, st.x_perm[R - T:R + T], offs, self.wg, self.wu, self.wd, self.s_wg, self.s_wu,
-                            self.s_wd, y_perm=st.y_full[R - T:R + T])
+                            self.s_wd, scales=self.scales, y_perm=st.y_full[R - T:R + T])
 
     # -------------------------------------------------------------- step 5
     def combine(self, st):
@@ -184,3 +192,25 @@ def split_experts(rank, world, wg, wu, wd):
     E_l = E // world
     sl = slice(rank * E_l, (rank + 1) * E_l)
     return wg[sl].contiguous(), wu[sl].contiguous(), wd[sl].contiguous()
+
+
+def _scale_blocks(E, d, I, I_s):
+    """Length of the packed E4M3 scale buffer: gate, up and down of E experts,
+    then the shared expert's three, one scale per 128 x 128 block each."""
+    per = (I // 128) * (d // 128)
+    return 3 * E * per + (3 * (I_s // 128) * (d // 128) if I_s > 0 else 0)
+
+
+def split_scales(rank, world, E, d, I, I_s, scales):
+    """This rank's packed E4M3 block scales from the whole block's buffer: the
+    gate, up and down scales of its experts, then the shared expert's
+    (replicated), in the same packed order as the whole buffer."""
+    if scales.numel() != _scale_blocks(E, d, I, I_s):
+        raise ValueError("scales hold %d values, not the %d of the whole block"
+                         % (scales.numel(), _scale_blocks(E, d, I, I_s)))
+    E_l = E // world
+    per = (I // 128) * (d // 128)
+    lo, hi = rank * E_l * per, (rank + 1) * E_l * per
+    flat = scales.reshape(-1)
+    parts = [flat[m * E * per:(m + 1) * E * per][lo:hi] for m in range(3)] + [flat[3 * E * per:]]
+    return torch.cat(parts).contiguous()

@@ -101,11 +101,11 @@ def _check_rank(inp, lo, hi, y, state):
     x = inp.x[lo:hi].contiguous()
     key = precision_key(inp)
     y_or, ids_or, _, probs = oracle.moe_forward(x, inp.w_r, inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu, inp.s_wd,
-                                                inp.k, bias=inp.bias)
+                                                inp.k, bias=inp.bias, scales=inp.scales)
     use, differ = check_routing(state.ids.cpu().numpy(), state.tw.cpu().numpy(), probs, ids_or, TOL_W[key])
     if differ:
         y_or, *_ = oracle.moe_forward(x, inp.w_r, inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu, inp.s_wd, inp.k,
-                                      bias=inp.bias, force_ids=use)
+                                      bias=inp.bias, scales=inp.scales, force_ids=use)
     err = rel_l2(y.float().cpu().numpy(), y_or)
     assert err <= TOL[key], "rel-L2 %.3g > %.3g" % (err, TOL[key])
 
@@ -122,6 +122,27 @@ def test_expert_parallel_ranks_emulated_on_one_gpu_match_the_oracle(moe, G, toke
     for r in range(G):
         wg, wu, wd = ep.split_experts(r, G, g["wg"], g["wu"], g["wd"])
         layers.append(ep.EPMoELayer(r, G, d, E, k, I, I_s, g["w_r"], wg, wu, wd, g["s_wg"], g["s_wu"], g["s_wd"]))
+        xs.append(g["x"][bounds[r]:bounds[r + 1]].contiguous())
+    ys, st = _emulate(layers, xs)
+    torch.cuda.synchronize()
+    _no_device_errors(moe)
+    for r in range(G):
+        _check_rank(inp, bounds[r], bounds[r + 1], ys[r], st[r])
+
+
+@pytest.mark.parametrize("G,tokens,I_s", [(2, [300, 212], 128), (4, [64, 0, 130, 9], 0)])
+def test_expert_parallel_e4m3_ranks_emulated_on_one_gpu_match_the_oracle(moe, G, tokens, I_s):
+    d, E, k, I = 256, 16, 4, 128
+    inp = moe_inputs.make_inputs(sum(tokens), d, E, k, I, I_s, act="bf16", w="fp8", seed=13, shared=I_s > 0)
+    g = {n: (getattr(inp, n).cuda() if getattr(inp, n) is not None else None)
+         for n in ("x", "w_r", "wg", "wu", "wd", "s_wg", "s_wu", "s_wd", "scales")}
+    bounds = np.concatenate([[0], np.cumsum(tokens)]).tolist()
+    layers, xs = [], []
+    for r in range(G):
+        wg, wu, wd = ep.split_experts(r, G, g["wg"], g["wu"], g["wd"])
+        sc = ep.split_scales(r, G, E, d, I, I_s, g["scales"])
+        layers.append(ep.EPMoELayer(r, G, d, E, k, I, I_s, g["w_r"], wg, wu, wd, g["s_wg"], g["s_wu"], g["s_wd"],
+                                    w="fp8", scales=sc))
         xs.append(g["x"][bounds[r]:bounds[r + 1]].contiguous())
     ys, st = _emulate(layers, xs)
     torch.cuda.synchronize()
