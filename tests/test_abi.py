@@ -159,3 +159,42 @@ def test_forward_plan_on_the_host():
     finally:
         moe.set_path(0)
     assert moe.lib().moe_forward_plan(ctypes.byref(P(T=-1)), None, None, None) == 1
+
+
+def _c_kind(decl):
+    """Kind of one C parameter declaration: pointer, i64, i32, size or f32."""
+    decl = decl.strip()
+    if "*" in decl:
+        return "pointer"
+    t = decl.rsplit(None, 1)[0].replace("const", "").strip()
+    return {"int64_t": "i64", "int32_t": "i32", "int": "i32", "size_t": "size", "float": "f32"}[t]
+
+
+def _ctypes_kind(t):
+    if t is ctypes.c_void_p or t is ctypes.c_char_p or hasattr(t, "_type_") and isinstance(t._type_, type):
+        return "pointer"
+    if t is ctypes.c_size_t:
+        return "size"
+    if t is ctypes.c_float:
+        return "f32"
+    return {8: "i64", 4: "i32"}[ctypes.sizeof(t)]
+
+
+def test_binding_argument_types_follow_the_header():
+    """Every declared entry point's parameters, one by one, against the ctypes
+    signature the binding gives it: a mismatch would pass a value where the
+    library reads a pointer (or a 32-bit value where it reads 64 bits)."""
+    src = re.sub(r"/\*.*?\*/", "", open(os.path.join(ROOT, "include", "moe.h")).read(), flags=re.S)
+    L = moe.lib()
+    seen = 0
+    for m in re.finditer(r"MOE_API\s+([\w\s\*]+?)\b(moe_\w+)\s*\(([^)]*)\)\s*;", src):
+        ret, name, params = m.group(1).strip(), m.group(2), m.group(3).strip()
+        decls = [] if params in ("", "void") else params.split(",")
+        f = getattr(L, name)
+        got = [] if f.argtypes is None else [_ctypes_kind(t) for t in f.argtypes]
+        assert got == [_c_kind(p) for p in decls], name
+        want_ret = {"moe_status": ctypes.c_int, "int": ctypes.c_int, "size_t": ctypes.c_size_t,
+                    "const char*": ctypes.c_char_p}[ret.replace(" *", "*")]
+        assert f.restype is want_ret, name
+        seen += 1
+    assert seen == len(moe.EXPORTS)
