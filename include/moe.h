@@ -136,8 +136,13 @@ MOE_API moe_status moe_combine(const moe_problem* p, const void* y_perm, const i
 /* The whole block, fused: router + top-k, dispatch, gate/up GEMM with SwiGLU,
  * down GEMM whose epilogue applies the routing weight and stores each row in
  * (token, slot) order, then one ordered fp32 sum per token of its k slot rows
- * and its shared-expert row (reproducible: no atomics).  y [T, d] in the activation type.  topk_ids_out and
- * topk_w_out ([T, k]) may be NULL.  ws: moe_workspace_size() bytes.
+ * and its shared-expert row (reproducible: the order of the additions is
+ * fixed).  On the row-tiled form that sum runs in the down GEMM's epilogue:
+ * the warp that stores a token's last slot row over a column span adds the
+ * token's rows there (counters in the workspace say which is last); the other
+ * forms run it as a separate pass.  Both give the same bits.  y [T, d] in the
+ * activation type.  topk_ids_out and topk_w_out ([T, k]) may be NULL.  ws:
+ * moe_workspace_size() bytes.
  * On the row-tiled bf16 form (see moe_set_path) with T * d * 2 <= 32 MiB the
  * gate/up GEMM reads each dispatched row straight from x (the rows stay in
  * L2 while the weights stream), and the dispatch writes no copy of them. */
