@@ -883,9 +883,6 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
       if (EPI == kTcSwiGLU || EPI == kTcSlotStore || EPI == kTcStore) {
         constexpr int CPW = (BN / 32) / EG;  // 32-column chunks per warp, contiguous
         epilogue_rows<BN, EPI>(p, t, tb, row, eg * CPW, (eg + 1) * CPW, epi_stage + (warp - 2) * 2048, lane);
-        if constexpr (EPI == kTcSlotStore) {
-          if (p.y != nullptr) slot_sum_fused<CPW>(p, t, row, t.n0 + eg * CPW * 32, lane);
-        }
       } else if (EPI == kTcTopK) {
         float* xv = reinterpret_cast<float*>(epi_stage + q * 4096);  // 16 KB: 4 quarters x 16 slots x 32 lanes x 8 B
         int* xe = reinterpret_cast<int*>(epi_stage + q * 4096 + 2048);
@@ -918,6 +915,12 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + acc);
+      if constexpr (EPI == kTcSlotStore) {
+        // the slot sum reads global memory only: it runs after the accumulator
+        // has gone back to the MMA warp, alongside the next tile's MMAs
+        constexpr int CPW = (BN / 32) / EG;
+        if (p.y != nullptr) slot_sum_fused<CPW>(p, t, row, t.n0 + eg * CPW * 32, lane);
+      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;
