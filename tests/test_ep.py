@@ -48,7 +48,7 @@ def _single_process(ops, prob, x, inp):
     return ops.combine(prob, yp, pm["pos"], tw, pm["offs"])
 
 
-def _rank(rank, world, port, tokens, I_s, q, w="f32"):
+def _rank(rank, world, port, tokens, I_s, q, w="f32", bias=None):
     import datetime
     import torch.distributed as dist
     import ep_cpu_ops
@@ -60,17 +60,17 @@ def _rank(rank, world, port, tokens, I_s, q, w="f32"):
         act = "bf16" if w == "fp8" else w
         T = _rank_tokens(rank, tokens)
         inp = moe_inputs.make_inputs(max(T, 1), c["d"], c["E"], c["k"], c["I"], c["I_s"], act=act, w=w,
-                                     seed=3, x_seed=100 + rank, shared=I_s > 0)
+                                     bias=bias, seed=3, x_seed=100 + rank, shared=I_s > 0)
         x = inp.x[:T].contiguous()
         wg, wu, wd = ep.split_experts(rank, world, inp.wg, inp.wu, inp.wd)
         sc = None if w != "fp8" else ep.split_scales(rank, world, c["E"], c["d"], c["I"], c["I_s"], inp.scales)
         layer = ep.EPMoELayer(rank, world, c["d"], c["E"], c["k"], c["I"], c["I_s"], inp.w_r, wg, wu, wd,
-                              inp.s_wg, inp.s_wu, inp.s_wd, act=act, w=w, ops=ep_cpu_ops, scales=sc)
+                              inp.s_wg, inp.s_wu, inp.s_wd, bias=inp.bias, act=act, w=w, ops=ep_cpu_ops, scales=sc)
         y = layer.forward(x, ep.TorchExchange())
         same = True
         if T:
             ref, _, _, _ = oracle.moe_forward(x, inp.w_r, inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu, inp.s_wd,
-                                              c["k"], scales=inp.scales, want_probs=False)
+                                              c["k"], bias=inp.bias, scales=inp.scales, want_probs=False)
             err = float(np.linalg.norm(y.double().numpy() - ref) / max(np.linalg.norm(ref), 1e-30))
             prob = ep_cpu_ops.Problem.make(T, c["d"], c["E"], c["k"], c["I"], c["I_s"], act, w)
             same = torch.equal(y, _single_process(ep_cpu_ops, prob, x, inp))
@@ -83,11 +83,11 @@ def _rank(rank, world, port, tokens, I_s, q, w="f32"):
         dist.destroy_process_group()
 
 
-def _run(world, tokens, I_s=32, w="f32", tol=2e-6):
+def _run(world, tokens, I_s=32, w="f32", tol=2e-6, bias=None):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank, args=(r, world, port, tokens, I_s, q, w)) for r in range(world)]
+    procs = [ctx.Process(target=_rank, args=(r, world, port, tokens, I_s, q, w, bias)) for r in range(world)]
     for p in procs:
         p.start()
     got = sorted(q.get(timeout=240) for _ in procs)
@@ -108,6 +108,12 @@ def test_expert_parallel_ranks_match_the_whole_block(world, tokens):
 
 def test_expert_parallel_rank_without_tokens_and_no_shared_expert():
     _run(2, [0, 41], I_s=0)
+
+
+def test_expert_parallel_with_a_skewed_router_bias():
+    # the replicated router adds the Zipf bias on every rank: most rows go to
+    # the low experts, all held by rank 0
+    _run(2, [44, 29], bias="zipf")
 
 
 @pytest.mark.parametrize("world,tokens,I_s", [(2, [30, 45], 128), (4, [12, 0, 25, 7], 0)])

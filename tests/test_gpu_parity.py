@@ -48,6 +48,8 @@ FORWARD_CASES = {
     "bf16_zipf": (200, 256, 64, 6, 128, 128, "bf16", "bf16", "zipf"),
     "bf16_no_shared": (150, 192, 12, 2, 96, 0, "bf16", "bf16", None),
     "bf16_T1": (1, 256, 40, 5, 128, 64, "bf16", "bf16", None),
+    # k = 16, the largest the boundary takes: 17 slot rows per token
+    "bf16_k16": (190, 256, 48, 16, 128, 128, "bf16", "bf16", None),
     "bf16_I_ne_Is": (129, 256, 16, 3, 136, 264, "bf16", "bf16", None),
     # groups of several 256-row tiles with ragged tails; d = 384 leaves half of
     # the last 256-row weight block of the down projection outside d
