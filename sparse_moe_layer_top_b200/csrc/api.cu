@@ -596,7 +596,7 @@ static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, cons
                                   int32_t* offs, int32_t* row_tok, float* row_w, int32_t* pos, int32_t* row_dst,
                                   int32_t* counts, Schedule sa, int32_t* pre_a, Schedule sb, int32_t* pre_b,
                                   const void* x, void* xp, cudaStream_t st, DeviceInfo* dev,
-                                  const float* shared_gate = nullptr) {
+                                  const float* shared_gate = nullptr, void* y0 = nullptr) {
   const int nch = (int)n_chunks(p);
   if (p.T == 0) {
     CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)p.E * 4, st));
@@ -610,7 +610,7 @@ static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, cons
   PROF_BEGIN("dispatch", st);
   CUDA_TRY(launch(k_dispatch, nch * kSubBlocks, kScatterWarps * 32, 0, st, ids, tw, p.T, p.k, p.E, counts, nch,
                   p.I_s > 0, offs, sa, pre_a, sb, pre_b, row_tok, row_w, pos, row_dst, shared_gate,
-                  (const uint4*)x, vec, (uint4*)xp));
+                  (const uint4*)x, vec, (uint4*)xp, (uint4*)y0));
   LAUNCH_CHECK("dispatch", st);
   return MOE_OK;
 }
@@ -1321,7 +1321,7 @@ static moe_status block_forward(const moe_problem* p, const moe_block_options* o
   GatherSrc gs;
   if (gathers_rows(*p, form)) gs = GatherSrc{xin, row_tok};
   s = launch_dispatch(*p, ids, tw, counted, offs, row_tok, row_w, pos, row_dst, counts, sa, pre_a, sb, pre_b, xin,
-                      gs.x ? nullptr : xp, st, dev, gate);
+                      gs.x ? nullptr : xp, st, dev, gate, fuse_sum ? y : nullptr);
   if (s != MOE_OK) return s;
   DownOut o{xp, row_dst, row_w, nullptr};  // the slot rows reuse the dispatched-row buffer
   if (fuse_sum) {
