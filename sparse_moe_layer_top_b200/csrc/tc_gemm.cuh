@@ -376,7 +376,8 @@ __device__ __forceinline__ void epilogue_rows(const TcGemmArgs& p, const TileInf
 // columns from n0c.  Release: every lane fences its own stores, the warp
 // syncs, then each lane counts its row in sum_cnt[token][span].  Acquire: the
 // lane whose count completes the token's (all valid slot rows of that span
-// landed, from any CTA) is found by ballot, every lane fences, and the warp
+// landed, from any CTA) is found by ballot, every lane fences, the warp syncs,
+// and the warp
 // adds that token's slot rows through L2 (lane l: columns n0c + VEC l ..
 // + VEC - 1), slots 0..k in order, in fp32 from zero -- the arithmetic of the
 // separate slot-sum pass, so y is the same bit for bit.
@@ -403,7 +404,10 @@ __device__ __forceinline__ void slot_sum_fused(const TcGemmArgs& p, const TileIn
   }
   unsigned m = __ballot_sync(0xffffffffu, last);
   if (m == 0) return;
+  // the completing lane's fence, then a warp barrier (which orders memory
+  // among the warp's lanes, unlike the ballot) before any lane's loads
   __threadfence();
+  __syncwarp();
   const int c = n0c + lane * VEC;
   const bool cin = c < t.N;  // N % 8 == 0: a lane's columns are all in or all out
   while (m) {
