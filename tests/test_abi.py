@@ -198,3 +198,16 @@ def test_binding_argument_types_follow_the_header():
         assert f.restype is want_ret, name
         seen += 1
     assert seen == len(moe.EXPORTS)
+
+
+def test_a_missing_library_fails_loudly(monkeypatch, tmp_path):
+    """No fallback: without libmoe.so every call raises, on the host, before
+    anything could run elsewhere."""
+    import torch
+    monkeypatch.setattr(moe, "lib_path", str(tmp_path / "libmoe.so"))
+    monkeypatch.setattr(moe, "_lib", None)
+    with pytest.raises(ImportError, match="not built"):
+        moe.workspace_size(P())
+    a = torch.zeros((64, 256), dtype=torch.bfloat16)
+    with pytest.raises(ImportError, match="not built"):
+        moe.router_topk(P(), a, torch.zeros((16, 256), dtype=torch.bfloat16))

@@ -12,6 +12,8 @@ import math
 import os
 
 import numpy as np
+from hypothesis import given, settings
+from hypothesis import strategies as st
 import pytest
 import torch
 
@@ -391,3 +393,31 @@ def test_shared_gate_weights_the_shared_expert_linearly():
     _, _, _, _, half = oracle.block_forward(inp.x, inp.w_r, inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu,
                                             inp.s_wd, inp.k, shared_gate=torch.zeros(8))
     assert np.all(half == 0.5)
+
+
+@settings(max_examples=300, deadline=None)
+@given(st.integers(2, 9).flatmap(lambda E: st.tuples(
+    st.just(E), st.integers(1, E), st.lists(st.integers(-3, 2), min_size=E, max_size=E))))
+def test_topk_with_exact_ties_against_brute_force(case):
+    """x = 0, so the logits are exactly the bias; a bias drawn from six values
+    makes exact ties common.  The kept set maximises the summed probability,
+    ties to the lexicographically smallest index set; the ids come out by
+    descending probability, equal ones by ascending index."""
+    E, k, levels = case
+    bias = torch.tensor([0.5 * v for v in levels], dtype=torch.float32)
+    x = _f32(np.zeros((2, 1)))
+    w_r = _f32(np.ones((E, 1)))
+    probs, ids, w = oracle.router(x, w_r, k, bias=bias)
+    b = bias.double().numpy()
+    p = np.exp(b - b.max())
+    p /= p.sum()
+    best, best_key = None, None
+    for S in itertools.combinations(range(E), k):
+        key = (round(float(p[list(S)].sum()), 12), tuple(-s for s in S))
+        if best_key is None or key > best_key:
+            best, best_key = S, key
+    for t in range(2):
+        got = ids[t].tolist()
+        assert sorted(got) == list(best)
+        assert got == sorted(got, key=lambda e: (-p[e], e))
+        np.testing.assert_allclose(w[t], p[got] / p[got].sum(), rtol=1e-12)
