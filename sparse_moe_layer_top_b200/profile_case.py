@@ -13,15 +13,7 @@ import os
 import sys
 
 
-def main(argv=None):
-    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    if root not in sys.path:
-        sys.path.insert(0, root)
-    import torch
-
-    import moe_inputs
-    import sparse_moe_layer_top_b200 as moe
-
+def arg_parser():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--T", type=int, default=256)
     ap.add_argument("--d", type=int, default=8192)
@@ -33,7 +25,19 @@ def main(argv=None):
     ap.add_argument("--bias", choices=("none", "zipf"), default="none")
     ap.add_argument("--path", type=int, default=0)
     ap.add_argument("--reps", type=int, default=2)
-    a = ap.parse_args(argv)
+    return ap
+
+
+def main(argv=None):
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    if root not in sys.path:
+        sys.path.insert(0, root)
+    import torch
+
+    import moe_inputs
+    import sparse_moe_layer_top_b200 as moe
+
+    a = arg_parser().parse_args(argv)
     torch.cuda.set_device(0)
     inp = moe_inputs.make_inputs(a.T, a.d, a.E, a.k, a.I, a.Is, act="bf16", w=a.w,
                                  bias=None if a.bias == "none" else a.bias, seed=0, device="cuda")

@@ -109,3 +109,30 @@ def test_warmup_below_three_is_refused():
     out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--warmup", "2"], capture_output=True,
                          text=True, timeout=300, cwd=ROOT)
     assert out.returncode != 0 and "warmup" in out.stderr
+
+
+def _profile_commands(target):
+    """The argument lists given to `target` in the commands of profiles/*.md."""
+    import glob
+    import re
+    import shlex
+    out = []
+    for f in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.md"))):
+        text = open(f).read().replace("\\\n", " ")
+        for line in text.splitlines():
+            for m in re.finditer(re.escape(target) + r"((?:\s+--?[\w-]+(?:\s+(?!-)[^\s>&|]+)?)*)", line):
+                out.append((os.path.basename(f), shlex.split(m.group(1))))
+    return out
+
+
+def test_profile_commands_match_the_current_command_lines():
+    """Every command a committed ncu summary gives for bench.py or the
+    profiler target still parses: the summaries can be re-run as written."""
+    from sparse_moe_layer_top_b200 import profile_case
+    bench_cmds = _profile_commands("bench.py")
+    case_cmds = _profile_commands("sparse_moe_layer_top_b200.profile_case")
+    assert bench_cmds and case_cmds
+    for name, args in bench_cmds:
+        bench.arg_parser().parse_args(args)
+    for name, args in case_cmds:
+        profile_case.arg_parser().parse_args(args)
