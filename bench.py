@@ -161,7 +161,7 @@ def gathers_rows(c, T):
 def down_sums_slots(c, T):
     """Whether the down GEMM also sums each token's slot rows into y (the
     row-tiled form), so that y is written by it."""
-    return forward_plan(c, T)["expert_form"] == "rows"
+    return forward_plan(c, T)["slot_sum_in_down"]
 
 
 def work_model(c, counts, T):

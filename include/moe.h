@@ -239,12 +239,14 @@ MOE_API moe_status moe_router_topk_static(const moe_problem* p, const void* x, c
  * (swap-AB) GEMMs, 3 row-tiled GEMMs on CTA pairs; router_selects: 1 when the
  * router's GEMM selects the top k in its epilogue (bf16, E <= 256, at least
  * 16 tiles of 128 tokens), 0 for the split-K GEMM + top-k kernel or the SIMT
- * router; gathered: 1 when the gate/up GEMM reads its rows straight from x.
+ * router; gathered: 1 when the gate/up GEMM reads its rows straight from x;
+ * slot_sum_in_down: 1 when the down GEMM's epilogue sums each token's slot
+ * rows into y (the row-tiled form), 0 when a separate pass does.
  * Any output pointer may be NULL.  Errors: those of moe_check_problem, and
  * MOE_ERR_UNSUPPORTED where moe_set_path asks for a form the types do not
  * allow. */
 MOE_API moe_status moe_forward_plan(const moe_problem* p, int32_t* expert_form, int32_t* router_selects,
-                            int32_t* gathered);
+                            int32_t* gathered, int32_t* slot_sum_in_down);
 
 /* Kernel-path selection for the calls above on the calling process:
  * 0 = automatic (tensor-core kernels where the types allow; for the expert

@@ -357,6 +357,9 @@ static moe_status choose(bool tc_possible, bool* use_tc) {
 // rows per expert, even at 1024, slower on prefill-sized Zipf-skewed groups);
 // else the row-tiled form.
 enum { kFormSimt = 0, kFormRows = 1, kFormSwap = 2, kFormPair = 3 };
+// The row-tiled down GEMM sums each token's slot rows in its epilogue; the
+// other forms leave that to k_slot_sum.
+static bool sums_in_down(int form) { return form == kFormRows; }
 constexpr int kPairRowsPerExpert = 2048;
 static moe_status choose_form(const moe_problem& p, int* form) {
   bool tc;
@@ -1308,7 +1311,7 @@ static moe_status block_forward(const moe_problem* p, const moe_block_options* o
   bool counted;
   // the row-tiled down GEMM sums each token's slot rows itself (its counters
   // follow the router's, zeroed by the router's memset)
-  const bool fuse_sum = form == kFormRows;
+  const bool fuse_sum = sums_in_down(form);
   s = launch_router(*p, xin, w_router, router_bias, ids, tw, (float*)(wsp + L.part), counts, &counted, st, dev,
                     fuse_sum ? (size_t)p->T * sum_cnt_ld(*p) * 4 : 0);
   if (s != MOE_OK) return s;
@@ -1386,7 +1389,7 @@ moe_status moe_rmsnorm(const moe_problem* p, const void* x, const void* norm_wei
 }
 
 moe_status moe_forward_plan(const moe_problem* p, int32_t* expert_form, int32_t* router_selects,
-                            int32_t* gathered) {
+                            int32_t* gathered, int32_t* slot_sum_in_down) {
   moe_status s = check(p);
   if (s != MOE_OK) return s;
   int form;
@@ -1396,6 +1399,7 @@ moe_status moe_forward_plan(const moe_problem* p, int32_t* expert_form, int32_t*
   if (expert_form) *expert_form = form;
   if (router_selects) *router_selects = router_tc && router_fused(*p) ? 1 : 0;
   if (gathered) *gathered = gathers_rows(*p, form) ? 1 : 0;
+  if (slot_sum_in_down) *slot_sum_in_down = sums_in_down(form) ? 1 : 0;
   return MOE_OK;
 }
 
