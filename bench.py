@@ -32,10 +32,17 @@ if ROOT not in sys.path:
 
 METRIC = "MoE-layer tokens/s at 1 B200; % HBM roofline (decode) / % bf16 TC peak (prefill)"
 UNIT = "tokens/s"
-DEFAULT_CONFIG = "qwen36_35b_a3b_bf16"
+DEFAULT_CONFIG = "qwen38max_prefill_zipf_bf16"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 FLUSH_BYTES = 256 << 20
-LONG_RUN_MS = 100.0  # timed regions at least this long use the sustained tensor peak
+# Expert weights the oracle may receive on the host for the CPU baseline; a
+# workload whose weights exceed it is timed on a token sample whose experts fit.
+HOST_WEIGHT_BUDGET = 12 << 30
+# A workload whose weights are those of another (same shapes and seed) also
+# times that one in the same run, on the same resident weights: the metric's
+# two regimes of the 3.8-Max-shaped block, prefill (tensor-bound) and decode
+# (weight-streaming).
+COMPANION = {"qwen38max_prefill_zipf_bf16": "qwen38max_decode_bf16"}
 # The files that define each timed kernel (its template, the PTX wrappers it
 # uses, its launch configuration): an ncu traffic figure stays valid while
 # their contents hash to the value recorded with it.
@@ -134,14 +141,15 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def routing_counts(moe, layer, x):
-    """Rows per group from the block's own router (outside the timed region)."""
+def routing(moe, layer, x):
+    """(topk_ids [T,k] on the device, rows per expert) from the block's own
+    router, outside the timed region."""
     import torch
     prob = layer.problem(x.shape[0])
     w_router, bias = layer.w[0], layer.w[1]
     ids, _ = moe.router_topk(prob, x, w_router, bias)
     cnt = torch.bincount(ids.reshape(-1).long(), minlength=prob.E).cpu().tolist()
-    return cnt
+    return ids, cnt
 
 
 def forward_plan(c, T):
@@ -215,14 +223,109 @@ def host_copy(inp):
     return out
 
 
-def cpu_baseline(inp, target_s=15.0):
+def weight_bytes(inp):
+    return sum(getattr(inp, n).numel() * getattr(inp, n).element_size()
+               for n in ("wg", "wu", "wd") if getattr(inp, n) is not None)
+
+
+def sample_tokens(ids, T, n_max):
+    """Token order of a sample: a token of the hottest expert, one of the
+    coldest active expert, then tokens spread evenly over the batch (so that
+    every 128-token tile of it is represented once n is large enough)."""
+    import torch
+    flat = ids.reshape(-1).long()
+    cnt = torch.bincount(flat)
+    hot = int(cnt.argmax())
+    act = torch.nonzero(cnt > 0).flatten()
+    cold = int(act[cnt[act].argmin()])
+    first = [int(torch.nonzero((ids == hot).any(1)).flatten()[0]),
+             int(torch.nonzero((ids == cold).any(1)).flatten()[-1])]
+    n = min(T, n_max)
+    spread = [(i * T) // n + (T // n) // 2 for i in range(n)]
+    out = []
+    for t in first + spread:
+        if t not in out:
+            out.append(t)
+    return out
+
+
+def compact_experts(inp, experts):
+    """Host copies of only the given routed experts (E4M3 as raw codes), and
+    the packed E4M3 scales restricted to them."""
+    import torch
+    sel = torch.as_tensor(experts, device=inp.wg.device, dtype=torch.long)
+
+    def pick(t):
+        if t.dtype == torch.float8_e4m3fn:
+            t = t.view(torch.uint8)
+        return t[sel].cpu()
+
+    out = {"wg": pick(inp.wg), "wu": pick(inp.wu), "wd": pick(inp.wd), "scales": None}
+    if inp.w == "fp8":
+        E, gd, gi = inp.E, inp.d // 128, inp.I // 128
+        n = E * gi * gd
+        sc = inp.scales
+        parts = [sc[:n].view(E, -1)[sel], sc[n:2 * n].view(E, -1)[sel], sc[2 * n:3 * n].view(E, -1)[sel], sc[3 * n:]]
+        out["scales"] = torch.cat([p.reshape(-1) for p in parts]).cpu()
+    return out
+
+
+def cpu_baseline_compact(inp, ids, target_s=15.0, n_max=256, budget=HOST_WEIGHT_BUDGET):
+    """The oracle on a token sample of a batch whose weights do not fit the
+    host budget: the sample's tokens (hottest and coldest experts' first) are
+    added while the experts they use fit the budget; the oracle gets host
+    copies of those experts only.  Timed: its router over all E experts, then
+    the block over the compact expert list with each token's experts forced
+    to the ones the device's router chose (the renormalised weights over a
+    token's kept experts do not depend on the other experts)."""
+    import numpy as np
+    import oracle
+    T, k = inp.T, inp.k
+    per_expert = weight_bytes(inp) // inp.E
+    max_experts = max(k, budget // max(per_expert, 1))
+    ids_h = ids.cpu()
+    toks, used = [], set()
+    for t in sample_tokens(ids, T, n_max):
+        s = set(ids_h[t].tolist())
+        if len(used | s) > max_experts:
+            continue
+        toks.append(t)
+        used |= s
+        if len(toks) == n_max:
+            break
+    experts = sorted(used)
+    remap = {e: i for i, e in enumerate(experts)}
+    w = compact_experts(inp, experts)
+    x_all = inp.x[toks].cpu()
+    w_r = inp.w_r.cpu()
+    bias = inp.bias.cpu() if inp.bias is not None else None
+    force = np.vectorize(remap.get)(ids_h[toks].numpy()).astype(np.int32)
+    sh = [None if t is None else t.cpu() for t in (inp.s_wg, inp.s_wu, inp.s_wd)]
+
+    def run(n):
+        t0 = time.perf_counter()
+        oracle.router(x_all[:n], w_r, k, bias=bias)
+        oracle.moe_forward(x_all[:n], w_r[experts], w["wg"], w["wu"], w["wd"], sh[0], sh[1], sh[2], k,
+                           bias=None if bias is None else bias[experts], scales=w["scales"],
+                           force_ids=force[:n], want_probs=False)
+        return time.perf_counter() - t0
+
+    probe = min(4, len(toks))
+    t_probe = run(probe)
+    n = int(min(len(toks), max(probe, target_s * probe / max(t_probe, 1e-6))))
+    t = run(n)
+    return {"value": n / t, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": "%d of %d tokens of the batch (a token of the hottest and of the coldest active expert, then "
+                      "tokens spread over the batch), float64 router over all %d experts and the block on host "
+                      "copies of the %d experts those tokens use (%.1f GB), %.1f s"
+                      % (n, T, inp.E, len(experts), len(experts) * per_expert / 1e9, t)}
+
+
+def cpu_baseline(inp, ids, target_s=15.0):
     """The oracle, as it stands, on a bounded token sample of the batch."""
     import oracle
-    wbytes = sum(getattr(inp, n).numel() * getattr(inp, n).element_size()
-                 for n in ("wg", "wu", "wd") if getattr(inp, n) is not None)
-    if wbytes > (8 << 30):
-        return {"value": None, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
-                "sample": "not run: weights too large to copy to the host here"}
+    if weight_bytes(inp) > (8 << 30):
+        return cpu_baseline_compact(inp, ids, target_s)
     host = host_copy(inp)
     probe = 16
     t_probe = oracle_sample_time(lambda: host, probe)
@@ -308,6 +411,116 @@ def e2e_pipelined(layer, x, y, K, dev):
 
 
 # ---------------------------------------------------------------- our arm
+def check_status(moe, when):
+    s, detail = moe.device_status()
+    if s != 0:
+        raise RuntimeError("device status %d (0x%08x) %s" % (s, detail & 0xffffffff, when))
+
+
+def time_steps(moe, layer, x, y, K, W, flush, world, dev, clocks=None):
+    """W warm-up forwards, then K timed ones (CUDA events on the launching
+    stream, L2 flushed before each outside the events) -> (mean step ms, mean
+    ms per tensor-core GEMM kernel, launches per step, clock record)."""
+    import torch
+    for _ in range(W):
+        layer(x, y)
+    torch.cuda.synchronize()
+    check_status(moe, "after warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    barrier(world, dev)
+    torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.start()
+    moe.profile_enable(2)  # events around the tensor-core GEMMs only
+    for i in range(K):
+        flush.zero_()
+        ev[i][0].record()
+        layer(x, y)
+        ev[i][1].record()
+    torch.cuda.synchronize()
+    barrier(world, dev)
+    launches_per_step = moe.last_launch_count()
+    prof = moe.profile_read()
+    moe.profile_enable(0)
+    clk = clocks.stop() if clocks is not None else None
+    check_status(moe, "after the timed steps")
+    per = {}
+    for name, ms in prof:
+        per.setdefault(name, []).append(ms)
+    kern = {n: statistics.mean(v) for n, v in per.items()}
+    return statistics.mean(a.elapsed_time(b) for a, b in ev), kern, launches_per_step, clk
+
+
+def kernel_roofline(work, kern, peaks, peak_src, workload):
+    """Roofline of the dominant expert GEMM: its algorithmic bytes or flops
+    over its live CUDA-event time, against the measured copy bandwidth (HBM
+    bound) or the measured dense bf16 GEMM burst figure (tensor bound; the
+    fraction of the sustained figure is given beside it)."""
+    gemms = {"gemm_tc_swiglu": work["gemm_gate_up"], "gemm_tc_down": work["gemm_down"]}
+    dom = max((n for n in gemms if n in kern), key=lambda n: kern[n], default=None)
+    if dom is None:
+        return None
+    wk = gemms[dom]
+    t_s = kern[dom] / 1e3
+    hbm_t = wk["bytes"] / (peaks["hbm_gbs"] * 1e9)
+    tc_t = wk["flops"] / (peaks["bf16_tflops"] * 1e12)
+    if hbm_t >= tc_t:
+        roof = {"bound": "hbm", "achieved": wk["bytes"] / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
+        which = " copy bandwidth"
+    else:
+        burst, sust = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+        ach = wk["flops"] / t_s / 1e12
+        roof = {"bound": "tensor", "achieved": ach, "peak": burst, "unit": "TFLOP/s", "frac_sustained": ach / sust}
+        which = " bf16 dense GEMM, burst"
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = load_traffic(dom, workload)
+    roof.update({"kernel": dom, "kernel_ms": kern[dom], "algorithmic_bytes": wk["bytes"],
+                 "algorithmic_flops": wk["flops"], "peak_source": peak_src + which})
+    return roof
+
+
+def layer_roofline(work, step_ms, peaks, peak_src):
+    lw = work["layer"]
+    st = step_ms / 1e3
+    return {"bytes": lw["bytes"], "flops": lw["flops"],
+            "hbm_frac": lw["bytes"] / st / 1e9 / peaks["hbm_gbs"],
+            "tc_frac": lw["flops"] / st / 1e12 / peaks["bf16_tflops"],
+            "achieved_gbs": lw["bytes"] / st / 1e9, "achieved_tflops": lw["flops"] / st / 1e12,
+            "active_experts": work["active_experts"], "peak_source": peak_src + " (tensor: burst)"}
+
+
+def run_companion(args, moe, inp, flush, world, rank, dev, peaks, peak_src):
+    """The companion workload on the same resident weights (its own tokens,
+    its own router bias): step time, roofline and CPU baseline."""
+    import moe_inputs
+    import torch
+    name = COMPANION[args.config]
+    c = dict(moe_inputs.CONFIGS[name])
+    T = c["T"]
+    x = moe_inputs.randn((T, c["d"]), dev, rank, moe_inputs.X, 1.0, inp.x.dtype)
+    bias = moe_inputs.zipf_bias(c["E"], dev) if c["bias"] == "zipf" else None
+    layer = moe.MoELayer(inp.d, inp.E, inp.k, inp.I, inp.I_s, inp.w_r, inp.wg, inp.wu, inp.wd, inp.s_wg, inp.s_wu,
+                         inp.s_wd, bias=bias, scales=inp.scales, act=inp.act, w=inp.w, max_tokens=T)
+    y = torch.empty((T, c["d"]), dtype=x.dtype, device=dev)
+    ids, counts = routing(moe, layer, x)
+    work = work_model(c, counts, T)
+    step_ms, kern, lps, _ = time_steps(moe, layer, x, y, args.steps, args.warmup, flush, world, dev)
+    ms_max, tokens_all = aggregate(step_ms, T, world, dev)
+    if rank != 0:
+        return None
+    out = {"workload": name, "value": tokens_all / (ms_max / 1e3), "unit": UNIT, "ms_per_step": ms_max,
+           "T": T, "router_bias": c["bias"], "roofline": kernel_roofline(work, kern, peaks, peak_src, name),
+           "layer_roofline": layer_roofline(work, ms_max, peaks, peak_src), "kernel_ms": kern,
+           "launches_per_step": lps, "cpu_baseline": None}
+    if world == 1 and not args.no_cpu_baseline:
+        import moe_inputs as mi
+        sub = mi.MoEInputs(T, inp.d, inp.E, inp.k, inp.I, inp.I_s, inp.act, inp.w, x=x, w_r=inp.w_r, bias=bias,
+                           wg=inp.wg, wu=inp.wu, wd=inp.wd, s_wg=inp.s_wg, s_wu=inp.s_wu, s_wd=inp.s_wd,
+                           scales=inp.scales)
+        out["cpu_baseline"] = cpu_baseline(sub, ids, args.cpu_seconds)
+    return out
+
+
 def run_ours(args):
     import torch
     import torch.distributed as dist
@@ -328,96 +541,41 @@ def run_ours(args):
     x = inp.x
     y = torch.empty((T, inp.d), dtype=x.dtype, device=dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    counts = routing_counts(moe, layer, x)
+    ids, counts = routing(moe, layer, x)
     work = work_model(cfg, counts, T)
 
-    for _ in range(args.warmup):
-        layer(x, y)
-    torch.cuda.synchronize()
-    s, detail = moe.device_status()
-    if s != 0:
-        raise RuntimeError("device status %d (0x%08x) after warm-up" % (s, detail & 0xffffffff))
-
     K = args.steps
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     clocks = ClockSampler(local)
-    barrier(world, dev)
-    torch.cuda.synchronize()
-    clocks.start()
-    moe.profile_enable(2)  # events around the tensor-core GEMMs only
-    for i in range(K):
-        flush.zero_()
-        ev[i][0].record()
-        layer(x, y)
-        ev[i][1].record()
-    torch.cuda.synchronize()
-    barrier(world, dev)
-    launches_per_step = moe.last_launch_count()
-    prof = moe.profile_read()
-    moe.profile_enable(0)
-    clk = clocks.stop()
-    step_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    step_ms, kern, launches_per_step, clk = time_steps(moe, layer, x, y, K, args.warmup, flush, world, dev, clocks)
     ms_max, tokens_all = aggregate(step_ms, T, world, dev)
-
-    # per-kernel durations of the GEMMs (CUDA events on the launching stream, timed region)
-    per = {}
-    for name, ms in prof:
-        per.setdefault(name, []).append(ms)
-    kern = {n: statistics.mean(v) for n, v in per.items()}
 
     # End to end through the public API: every step copies its batch from
     # pinned host memory and its result back.  Steps are pipelined over three
     # streams with two buffers each, as a serving loop would run them: the
     # host->device copy of step i+1 and the device->host copy of step i-1
-    # overlap the forward of step i.  Per-step time = whole timed region / K.
-    # at least E2E_MIN_STEPS steps, so that filling and draining the pipeline
-    # (one step's copy in, one step's copy out) is spread as in a serving loop
+    # overlap the forward of step i.  Per-step time = whole timed region / K,
+    # over at least E2E_MIN_STEPS steps, so that filling and draining the
+    # pipeline (one step's copy in, one step's copy out) is spread as in a
+    # serving loop.  Steps run back to back, with no L2 flush between them.
     K_e2e = max(K, E2E_MIN_STEPS)
     e2e_ms = e2e_pipelined(layer, x, y, K_e2e, dev)
     e2e_max, _ = aggregate(e2e_ms, T, world, dev)
-    s, detail = moe.device_status()
-    if s != 0:
-        raise RuntimeError("device status %d (0x%08x) after the timed steps" % (s, detail & 0xffffffff))
+    check_status(moe, "after the end-to-end steps")
 
     peaks, peak_src = load_peaks()
+    regimes = {}
+    if args.config in COMPANION and not args.no_companion:
+        comp = run_companion(args, moe, inp, flush, world, rank, dev, peaks, peak_src)
+        if comp is not None:
+            regimes[comp["workload"]] = comp
     line = None
     if rank == 0:
-        gemms = {"gemm_tc_swiglu": work["gemm_gate_up"], "gemm_tc_down": work["gemm_down"]}
-        dom = max((n for n in gemms if n in kern), key=lambda n: kern[n], default=None)
-        roof = None
-        if dom is not None:
-            wk = gemms[dom]
-            t_s = kern[dom] / 1e3
-            hbm_t = wk["bytes"] / (peaks["hbm_gbs"] * 1e9)
-            tc_t = wk["flops"] / (peaks["bf16_tflops"] * 1e12)
-            if hbm_t >= tc_t:
-                roof = {"bound": "hbm", "achieved": wk["bytes"] / t_s / 1e9, "peak": peaks["hbm_gbs"], "unit": "GB/s"}
-                which = ""
-            else:
-                # A tensor-bound kernel timed inside a long run of steps (the
-                # power cap engages within tens of milliseconds) is held to the
-                # sustained dense-GEMM figure, one timed alone to the burst figure;
-                # both fractions are reported.
-                long_run = step_ms * K >= LONG_RUN_MS
-                burst, sust = peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
-                ach = wk["flops"] / t_s / 1e12
-                roof = {"bound": "tensor", "achieved": ach, "peak": sust if long_run else burst, "unit": "TFLOP/s",
-                        "frac_burst": ach / burst, "frac_sustained": ach / sust}
-                which = " (sustained: %.0f ms timed)" % (step_ms * K) if long_run else " (burst)"
-            roof["frac"] = roof["achieved"] / roof["peak"]
-            roof["traffic"] = load_traffic(dom, args.config)
-            roof.update({"kernel": dom, "kernel_ms": kern[dom], "algorithmic_bytes": wk["bytes"],
-                         "algorithmic_flops": wk["flops"], "peak_source": peak_src + which})
-        lw = work["layer"]
-        st = step_ms / 1e3
-        layer_roof = {"bytes": lw["bytes"], "flops": lw["flops"],
-                      "hbm_frac": lw["bytes"] / st / 1e9 / peaks["hbm_gbs"],
-                      "tc_frac": lw["flops"] / st / 1e12 / peaks["bf16_tflops"],
-                      "achieved_gbs": lw["bytes"] / st / 1e9, "achieved_tflops": lw["flops"] / st / 1e12,
-                      "active_experts": work["active_experts"], "peak_source": peak_src}
+        roof = kernel_roofline(work, kern, peaks, peak_src, args.config)
+        layer_roof = layer_roofline(work, ms_max, peaks, peak_src)
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
-            cpu = cpu_baseline(inp, args.cpu_seconds)
+            cpu = cpu_baseline(inp, ids, args.cpu_seconds)
+        resident = x.numel() * x.element_size() + y.numel() * y.element_size() + weight_bytes(inp)
         line = {
             "metric": METRIC, "value": tokens_all / (ms_max / 1e3), "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
@@ -432,10 +590,14 @@ def run_ours(args):
                     "h2d_bytes_per_step": x.numel() * x.element_size(),
                     "d2h_bytes_per_step": y.numel() * y.element_size(), "ms_per_step": e2e_max, "steps": K_e2e,
                     "pipelining": "host->device copy of step i+1 and device->host copy of step i-1 "
-                                  "overlap the forward of step i (3 streams, 2 buffers)"},
+                                  "overlap the forward of step i (3 streams, 2 buffers)",
+                    "l2": "no flush between steps; the step reads %.1f GB (tokens, result, weights) against "
+                          "126 MB of L2" % (resident / 1e9)},
             "gpu_launches": launches_per_step * K, "launches_per_step": launches_per_step,
             "kernel_ms": kern, "clocks": clk, "impl": "ours",
         }
+        if regimes:
+            line["regimes"] = regimes
     if world > 1:
         dist.destroy_process_group()
     if line is not None:
@@ -443,8 +605,47 @@ def run_ours(args):
 
 
 # ---------------------------------------------------------------- reference arm
+def oracle_routed_time(inp, toks, w_r, bias, budget=HOST_WEIGHT_BUDGET):
+    """Seconds the oracle takes for the block on tokens `toks` of a batch
+    whose weights stay on the device: its router over all E experts picks
+    each token's experts, host copies of only those experts are made
+    (untimed), and the block runs on them with the router's choice forced.
+    Tokens whose experts would pass the host budget go in further batches."""
+    import numpy as np
+    import oracle
+    x = inp.x[toks].cpu()
+    k = inp.k
+    t0 = time.perf_counter()
+    _, ids, _ = oracle.router(x, w_r, k, bias=bias)
+    secs = time.perf_counter() - t0
+    per_expert = weight_bytes(inp) // inp.E
+    max_experts = max(k, budget // max(per_expert, 1))
+    sh = [None if t is None else t.cpu() for t in (inp.s_wg, inp.s_wu, inp.s_wd)]
+    i = 0
+    while i < len(toks):
+        used, j = set(), i
+        while j < len(toks) and (j == i or len(used | set(ids[j].tolist())) <= max_experts):
+            used |= set(ids[j].tolist())
+            j += 1
+        experts = sorted(used)
+        remap = {e: n for n, e in enumerate(experts)}
+        w = compact_experts(inp, experts)
+        force = np.vectorize(remap.get)(ids[i:j]).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.moe_forward(x[i:j], w_r[experts], w["wg"], w["wu"], w["wd"], sh[0], sh[1], sh[2], k,
+                           bias=None if bias is None else bias[experts], scales=w["scales"], force_ids=force,
+                           want_probs=False)
+        secs += time.perf_counter() - t0
+        del w
+        i = j
+    return secs
+
+
 def run_reference(args):
-    """The float64 oracle on the host cores, on a bounded sample per step."""
+    """The float64 oracle on the host cores, on a bounded sample per step.
+    Workloads whose weights pass the host budget keep them on the device and
+    give the oracle host copies of the experts each step's tokens use, chosen
+    by the oracle's own router."""
     world, rank, local = dist_env()
     if rank != 0:
         return
@@ -456,33 +657,38 @@ def run_reference(args):
     cfg = dict(moe_inputs.CONFIGS[args.config])
     dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
     inp = moe_inputs.make_config(args.config, seed=0, device=dev)
-    wbytes = sum(getattr(inp, n).numel() * getattr(inp, n).element_size() for n in ("wg", "wu", "wd"))
-    if wbytes > (8 << 30):
-        print(json.dumps({"impl": "reference", "unavailable": "the float64 oracle needs the full weights on the "
-                          "host; %.1f GB is beyond this arm's host-memory budget" % (wbytes / 1e9)}))
-        return
-    host = host_copy(inp)
+    big = weight_bytes(inp) > (8 << 30)
+    host = None if big else host_copy(inp)
+    w_r = inp.w_r.cpu()
+    bias = inp.bias.cpu() if inp.bias is not None else None
     per_step = args.ref_tokens
     samples = []
     for i in range(args.warmup + args.steps):
         lo = (i * per_step) % max(inp.T - per_step + 1, 1)
-        x = host["x"][lo:lo + per_step]
-        t0 = time.perf_counter()
-        oracle.moe_forward(x, host["w_r"], host["wg"], host["wu"], host["wd"], host["s_wg"], host["s_wu"],
-                           host["s_wd"], host["k"], bias=host["bias"], scales=host["scales"], want_probs=False)
-        dt = time.perf_counter() - t0
+        if big:
+            dt = oracle_routed_time(inp, list(range(lo, min(inp.T, lo + per_step))), w_r, bias)
+        else:
+            x = host["x"][lo:lo + per_step]
+            t0 = time.perf_counter()
+            oracle.moe_forward(x, host["w_r"], host["wg"], host["wu"], host["wd"], host["s_wg"], host["s_wu"],
+                               host["s_wd"], host["k"], bias=host["bias"], scales=host["scales"], want_probs=False)
+            dt = time.perf_counter() - t0
         if i >= args.warmup:
             samples.append(dt)
     ms = statistics.mean(samples) * 1e3
-    value = per_step / (ms / 1e3)
-    sample = "%d tokens of the %d-token batch per step, full block in float64" % (per_step, inp.T)
+    n_step = min(per_step, inp.T)
+    value = n_step / (ms / 1e3)
+    sample = "%d tokens of the %d-token batch per step, full block in float64" % (n_step, inp.T)
+    if big:
+        sample += (" (router over all %d experts; the block on host copies of the experts those tokens use, "
+                   "copied outside the timed region)" % inp.E)
     print(json.dumps({
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1) tokens, N(0,0.02^2) weights)",
         "config": {"workload": args.config, "T": inp.T, "d": cfg["d"], "E": cfg["E"], "k": cfg["k"],
                    "I": cfg["I"], "I_s": cfg["I_s"], "act": cfg["act"], "weights": cfg["w"],
-                   "tokens_per_step": per_step},
+                   "router_bias": cfg["bias"], "tokens_per_step": n_step},
         "impl": "reference",
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": sample},
@@ -499,6 +705,8 @@ def arg_parser():
     import moe_inputs
     ap.add_argument("--config", choices=sorted(moe_inputs.CONFIGS), default=DEFAULT_CONFIG)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-companion", action="store_true",
+                    help="do not also time the workload that shares this one's weights (decode beside prefill)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--ref-tokens", type=int, default=32)
     return ap

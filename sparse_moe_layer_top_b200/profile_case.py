@@ -4,6 +4,9 @@ Meant as the target of profiler runs (ncu) on sizes smaller than the
 benchmark workloads:
 
     python -m sparse_moe_layer_top_b200.profile_case --T 64 --d 8192 --E 32 --k 10 --I 2048 --w bf16
+    python -m sparse_moe_layer_top_b200.profile_case --config qwen38max_prefill_zipf_bf16 --reps 3
+
+(--config runs a named benchmark workload at its full size instead.)
 
 Inputs come from moe_inputs (seeded).  Exits non-zero if the device status
 word reports a fault.
@@ -25,6 +28,7 @@ def arg_parser():
     ap.add_argument("--bias", choices=("none", "zipf"), default="none")
     ap.add_argument("--path", type=int, default=0)
     ap.add_argument("--reps", type=int, default=2)
+    ap.add_argument("--config", default=None, help="a named workload of moe_inputs.CONFIGS, at its full size")
     return ap
 
 
@@ -39,10 +43,13 @@ def main(argv=None):
 
     a = arg_parser().parse_args(argv)
     torch.cuda.set_device(0)
-    inp = moe_inputs.make_inputs(a.T, a.d, a.E, a.k, a.I, a.Is, act="bf16", w=a.w,
-                                 bias=None if a.bias == "none" else a.bias, seed=0, device="cuda")
+    if a.config:
+        inp = moe_inputs.make_config(a.config, seed=0, device="cuda")
+    else:
+        inp = moe_inputs.make_inputs(a.T, a.d, a.E, a.k, a.I, a.Is, act="bf16", w=a.w,
+                                     bias=None if a.bias == "none" else a.bias, seed=0, device="cuda")
     moe.set_path(a.path)
-    layer = moe.MoELayer.from_inputs(inp, max_tokens=a.T)
+    layer = moe.MoELayer.from_inputs(inp, max_tokens=inp.T)
     for _ in range(a.reps):
         y = layer(inp.x)
     torch.cuda.synchronize()

@@ -136,3 +136,40 @@ def test_profile_commands_match_the_current_command_lines():
         bench.arg_parser().parse_args(args)
     for name, args in case_cmds:
         profile_case.arg_parser().parse_args(args)
+
+
+def _small_inputs():
+    import moe_inputs
+    return moe_inputs.make_inputs(48, 128, 16, 2, 64, 64, act="bf16", w="bf16", seed=0)
+
+
+def test_cpu_baseline_compact_sample_fits_the_host_budget():
+    """The CPU baseline of a workload too large for the host times the oracle
+    on a token sample whose experts fit the budget, hottest expert first."""
+    import torch
+
+    import oracle
+    inp = _small_inputs()
+    _, ids, _ = oracle.router(inp.x, inp.w_r, inp.k)
+    ids = torch.as_tensor(ids)
+    per_expert = bench.weight_bytes(inp) // inp.E
+    d = bench.cpu_baseline_compact(inp, ids, target_s=0.05, n_max=16, budget=5 * per_expert)
+    assert d["value"] > 0 and d["kind"] == "oracle"
+    assert "hottest" in d["sample"]
+    n_exp = int(d["sample"].split("copies of the ")[1].split()[0])
+    assert inp.k <= n_exp <= 5
+    toks = bench.sample_tokens(ids, inp.T, 16)
+    cnt = torch.bincount(ids.reshape(-1).long())
+    assert int(cnt.argmax()) in ids[toks[0]].tolist()
+    assert len(set(toks)) == len(toks) and all(0 <= t < inp.T for t in toks)
+
+
+def test_oracle_routed_time_splits_a_step_over_the_budget():
+    import oracle
+    inp = _small_inputs()
+    per_expert = bench.weight_bytes(inp) // inp.E
+    t = bench.oracle_routed_time(inp, list(range(12)), inp.w_r, None, budget=3 * per_expert)
+    assert t > 0
+    # a budget below k experts still runs each token on its own
+    t = bench.oracle_routed_time(inp, [0, 5], inp.w_r, None, budget=1)
+    assert t > 0
