@@ -128,12 +128,23 @@ MOE_API moe_status moe_expert_ffn(const moe_problem* p, const void* x_perm, cons
                           const float* scales, void* y_perm, void* ws, size_t ws_bytes,
                           void* stream);
 
-/* Combine stage: y[t] = sum_j topk_w[t, j] * y_perm[pos[t, j]] + y_perm[offs[E] + t]
- * (the last term when I_s > 0).  y [T, d] in the activation type. */
+/* Combine stage (steps 3 and 5: the token's output is the kept experts'
+ * outputs weighted by their renormalised router probabilities -- Qwen3.6
+ * explainer, router paragraphs -- plus the always-on shared expert's output
+ * with weight 1 -- Qwen3.6 explainer, shared-expert paragraph; Qwen3-Next
+ * story, the shared expert that treats every input):
+ *   y[t] = sum_j topk_w[t, j] * y_perm[pos[t, j]] + y_perm[offs[E] + t]
+ * (the last term when I_s > 0); pairs with pos < 0 (dropped by moe_permute)
+ * add nothing.  Sums in fp32 in slot order, rounded once.  y [T, d] in the
+ * activation type. */
 MOE_API moe_status moe_combine(const moe_problem* p, const void* y_perm, const int32_t* pos,
                        const float* topk_w, const int32_t* offs, void* y, void* stream);
 
-/* The whole block, fused: router + top-k, dispatch, gate/up GEMM with SwiGLU,
+/* The whole block, fused (steps 1-5 above: the router and softmax top-k of the
+ * Qwen3.6 explainer's router paragraphs, the SwiGLU experts of the
+ * Architecture page's config.json, the shared expert of the explainer's
+ * shared-expert paragraph, summed as y = sum_{e kept} w_e E_e(x) + S(x)):
+ * router + top-k, dispatch, gate/up GEMM with SwiGLU,
  * down GEMM whose epilogue applies the routing weight and stores each row in
  * (token, slot) order, then one ordered fp32 sum per token of its k slot rows
  * and its shared-expert row (reproducible: the order of the additions is
@@ -265,6 +276,19 @@ MOE_API moe_status moe_set_path(int path);
  * (MOE_OK, MOE_ERR_DEVICE_CHECK or MOE_ERR_TIMEOUT); *detail receives the
  * raw code (which kernel and which wait), or 0.  Synchronises the device. */
 MOE_API moe_status moe_device_status(int32_t* detail);
+
+/* The bound, in SM clock cycles, of every pipeline wait in the library's
+ * kernels on the current device (cycles <= 0: the default, 4e9 cycles, about
+ * 2 s at B200 clocks).  A wait that passes it gives up: the kernel records
+ * MOE_ERR_TIMEOUT with the kernel and the wait in the device status word,
+ * drains the copies it issued (always with the default bound), releases its
+ * tensor memory and returns, leaving its outputs incomplete.  A short bound
+ * lets a test make waits give up on purpose and check that the kernels come
+ * back and the device stays usable.  Takes effect for kernels that start
+ * after the call returns; call it with no library work in flight on the
+ * device (the write is a synchronous copy to device memory).  MOE_ERR_CUDA if
+ * that copy fails. */
+MOE_API moe_status moe_set_wait_limit(int64_t cycles);
 
 /* Number of kernels the last successful call on this thread launched. */
 MOE_API int moe_last_launch_count(void);

@@ -8,7 +8,9 @@ first use; every call raises if it is missing -- there is no fallback.
 The C ABI sees only pointers, so every call first checks its tensors' element
 types and sizes against the problem and raises ValueError, before any pointer
 is taken, when a buffer is of the wrong type or too small for what the call
-reads or writes.
+reads or writes.  The library launches on the current CUDA device and its
+current stream: every call also requires all its tensors (and a stream it is
+given) to be on one device, and runs with that device current.
 
 Entry points mirror ``include/moe.h``: ``router_topk``, ``permute``,
 ``expert_ffn``, ``combine``, ``layer_forward``, ``block_forward``,
@@ -16,6 +18,7 @@ Entry points mirror ``include/moe.h``: ``router_topk``, ``permute``,
 workspace together; ``sparse_moe_layer_top_b200.ep`` splits the experts over
 several GPUs (expert parallelism).
 """
+import contextlib
 import ctypes
 import os
 
@@ -23,7 +26,8 @@ import torch
 
 __all__ = ["MoEError", "Problem", "BlockOptions", "router_topk", "permute", "expert_ffn", "combine", "layer_forward",
            "block_forward", "rmsnorm", "ep_expand_ids", "forward_plan",
-           "workspace_size", "stage_workspace_size", "set_path", "device_status", "last_launch_count",
+           "workspace_size", "stage_workspace_size", "set_path", "set_wait_limit", "device_status",
+           "last_launch_count",
            "profile_enable", "profile_read",
            "MoELayer", "lib_path", "F32", "BF16", "FP8_E4M3_B128"]
 
@@ -37,7 +41,7 @@ EXPORTS = ("moe_check_problem", "moe_workspace_size", "moe_stage_workspace_size"
            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_set_path",
            "moe_device_status", "moe_last_launch_count", "moe_profile_enable", "moe_profile_read",
            "moe_last_error_string", "moe_router_topk_static", "moe_block_forward", "moe_rmsnorm",
-           "moe_ep_expand_ids", "moe_forward_plan")
+           "moe_ep_expand_ids", "moe_forward_plan", "moe_set_wait_limit")
 
 
 class MoEError(RuntimeError):
@@ -90,6 +94,7 @@ def lib():
         L.moe_forward_plan.argtypes = [PP, I32P, I32P, I32P, I32P]
         L.moe_rmsnorm.argtypes = [PP, P, P, ctypes.c_float, P, P]
         L.moe_set_path.argtypes = [ctypes.c_int]
+        L.moe_set_wait_limit.argtypes = [ctypes.c_int64]
         L.moe_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32)]
         L.moe_last_launch_count.restype = ctypes.c_int
         L.moe_profile_enable.argtypes = [ctypes.c_int]
@@ -99,7 +104,8 @@ def lib():
         L.moe_profile_read.restype = ctypes.c_int
         L.moe_last_error_string.restype = ctypes.c_char_p
         for f in ("moe_check_problem", "moe_router_topk", "moe_router_topk_static", "moe_permute", "moe_expert_ffn", "moe_combine",
-                  "moe_layer_forward", "moe_block_forward", "moe_rmsnorm", "moe_set_path", "moe_device_status"):
+                  "moe_layer_forward", "moe_block_forward", "moe_rmsnorm", "moe_set_path", "moe_device_status",
+                  "moe_set_wait_limit"):
             getattr(L, f).restype = S
         _lib = L
     return _lib
@@ -158,6 +164,32 @@ def _ptr(t):
     return ctypes.c_void_p(t.data_ptr())
 
 
+def _device(stream=None, **tensors):
+    """The one device all given tensors are on (None if none is given); a
+    given stream must belong to it.  Raises ValueError naming the tensors
+    otherwise -- the library would launch on the current device with
+    another device's pointers."""
+    devs = {}
+    for name, t in tensors.items():
+        if t is not None:
+            devs.setdefault(t.device, []).append(name)
+    if len(devs) > 1:
+        raise ValueError("tensors on different devices: " +
+                         "; ".join("%s on %s" % (", ".join(n), d) for d, n in devs.items()))
+    dev = next(iter(devs), None)
+    if stream is not None and dev is not None and dev.type == "cuda" and stream.device != dev:
+        raise ValueError("stream on %s, tensors on %s" % (stream.device, dev))
+    return dev
+
+
+def _current(dev):
+    """A context in which `dev` is the current CUDA device (nothing to do
+    for a non-CUDA device: the pointer step rejects its tensors)."""
+    if dev is not None and dev.type == "cuda":
+        return torch.cuda.device(dev)
+    return contextlib.nullcontext()
+
+
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
@@ -183,6 +215,13 @@ def set_path(path):
     """0 automatic, 1 SIMT kernels only, 2 row-tiled tensor-core expert GEMMs,
     3 weight-row tensor-core expert GEMMs, 4 row-tiled on 2-CTA clusters."""
     _check(lib().moe_set_path(int(path)))
+
+
+def set_wait_limit(cycles=0):
+    """Bound, in SM cycles, of the kernels' pipeline waits on the current
+    device (0: the default, about 2 s).  Synchronous; call it with no library
+    work in flight."""
+    _check(lib().moe_set_wait_limit(int(cycles)))
 
 
 def device_status():
@@ -225,13 +264,15 @@ def router_topk(prob, x, w_router, bias=None, topk_ids=None, topk_w=None, ws=Non
     _need(bias, "router_bias", prob.E, _F32)
     _need(topk_ids, "topk_ids", T * k, _I32, k)
     _need(topk_w, "topk_w", T * k, _F32, k)
+    dev = _device(stream, x=x, w_router=w_router, router_bias=bias, topk_ids=topk_ids, topk_w=topk_w, ws=ws)
     if topk_ids is None:
         topk_ids = torch.empty((T, k), dtype=torch.int32, device=x.device)
     if topk_w is None:
         topk_w = torch.empty((T, k), dtype=torch.float32, device=x.device)
     ws = _ws(stage_workspace_size(prob), x.device, ws)
-    _check(lib().moe_router_topk(ctypes.byref(prob), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(topk_ids),
-                                 _ptr(topk_w), _ptr(ws), _nbytes(ws), _stream(stream)))
+    with _current(dev):
+        _check(lib().moe_router_topk(ctypes.byref(prob), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(topk_ids),
+                                     _ptr(topk_w), _ptr(ws), _nbytes(ws), _stream(stream)))
     return topk_ids, topk_w
 
 
@@ -244,6 +285,7 @@ def permute(prob, x, topk_ids, topk_w, ws=None, stream=None):
     _need(x, "x", prob.T * prob.d, _ACT_TYPES.get(prob.act_dtype), prob.d)
     _need(topk_ids, "topk_ids", prob.T * prob.k, _I32, prob.k)
     _need(topk_w, "topk_w", prob.T * prob.k, _F32, prob.k)
+    cur = _device(stream, x=x, topk_ids=topk_ids, topk_w=topk_w, ws=ws)
     dev = x.device
     Rp = rows_total(prob)
     out = dict(x_perm=torch.empty((Rp, prob.d), dtype=_act(prob), device=dev),
@@ -253,9 +295,10 @@ def permute(prob, x, topk_ids, topk_w, ws=None, stream=None):
                offs=torch.empty(prob.E + 2, dtype=torch.int32, device=dev))
     nbytes = stage_workspace_size(prob)
     ws = _ws(nbytes, dev, ws)
-    _check(lib().moe_permute(ctypes.byref(prob), _ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(out["x_perm"]),
-                             _ptr(out["row_tok"]), _ptr(out["row_w"]), _ptr(out["pos"]), _ptr(out["offs"]),
-                             _ptr(ws), _nbytes(ws), _stream(stream)))
+    with _current(cur):
+        _check(lib().moe_permute(ctypes.byref(prob), _ptr(x), _ptr(topk_ids), _ptr(topk_w), _ptr(out["x_perm"]),
+                                 _ptr(out["row_tok"]), _ptr(out["row_w"]), _ptr(out["pos"]), _ptr(out["offs"]),
+                                 _ptr(ws), _nbytes(ws), _stream(stream)))
     return out
 
 
@@ -266,13 +309,16 @@ def expert_ffn(prob, x_perm, offs, wg, wu, wd, s_wg=None, s_wu=None, s_wd=None, 
     _need(offs, "offs", prob.E + 2, _I32)
     _need_weights(prob, wg, wu, wd, s_wg, s_wu, s_wd, scales)
     _need(y_perm, "y_perm", Rp * prob.d, a, prob.d)
+    cur = _device(stream, x_perm=x_perm, offs=offs, w_gate=wg, w_up=wu, w_down=wd, ws_gate=s_wg, ws_up=s_wu,
+                  ws_down=s_wd, scales=scales, y_perm=y_perm, ws=ws)
     dev = x_perm.device
     if y_perm is None:
         y_perm = torch.empty((x_perm.shape[0], prob.d), dtype=_act(prob), device=dev)
     ws = _ws(stage_workspace_size(prob), dev, ws)
-    _check(lib().moe_expert_ffn(ctypes.byref(prob), _ptr(x_perm), _ptr(offs), _ptr(wg), _ptr(wu), _ptr(wd),
-                                _ptr(s_wg), _ptr(s_wu), _ptr(s_wd), _ptr(scales), _ptr(y_perm), _ptr(ws), _nbytes(ws),
-                                _stream(stream)))
+    with _current(cur):
+        _check(lib().moe_expert_ffn(ctypes.byref(prob), _ptr(x_perm), _ptr(offs), _ptr(wg), _ptr(wu), _ptr(wd),
+                                    _ptr(s_wg), _ptr(s_wu), _ptr(s_wd), _ptr(scales), _ptr(y_perm), _ptr(ws),
+                                    _nbytes(ws), _stream(stream)))
     return y_perm
 
 
@@ -283,10 +329,12 @@ def combine(prob, y_perm, pos, topk_w, offs, y=None, stream=None):
     _need(topk_w, "topk_w", prob.T * prob.k, _F32, prob.k)
     _need(offs, "offs", prob.E + 2, _I32)
     _need(y, "y", prob.T * prob.d, a, prob.d)
+    cur = _device(stream, y_perm=y_perm, pos=pos, topk_w=topk_w, offs=offs, y=y)
     if y is None:
         y = torch.empty((prob.T, prob.d), dtype=_act(prob), device=y_perm.device)
-    _check(lib().moe_combine(ctypes.byref(prob), _ptr(y_perm), _ptr(pos), _ptr(topk_w), _ptr(offs), _ptr(y),
-                             _stream(stream)))
+    with _current(cur):
+        _check(lib().moe_combine(ctypes.byref(prob), _ptr(y_perm), _ptr(pos), _ptr(topk_w), _ptr(offs), _ptr(y),
+                                 _stream(stream)))
     return y
 
 
@@ -313,9 +361,20 @@ def _need_tokens(prob, x, y, topk_ids, topk_w):
 def _forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, norm_weight, norm_eps, shared_gate, y,
              topk_ids, topk_w, ws, stream, block):
     """The fused forward on checked arguments (moe_block_forward when `block`)."""
+    cur = _device(stream, x=x, w_router=w_router, router_bias=bias, w_gate=wg, w_up=wu, w_down=wd, ws_gate=s_wg,
+                  ws_up=s_wu, ws_down=s_wd, scales=scales, norm_weight=norm_weight, shared_gate=shared_gate, y=y,
+                  topk_ids=topk_ids, topk_w=topk_w, ws=ws)
     if y is None:
         y = torch.empty((prob.T, prob.d), dtype=_act(prob), device=x.device)
     ws = _ws(workspace_size(prob), x.device, ws)
+    with _current(cur):
+        _forward_call(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, norm_weight, norm_eps,
+                      shared_gate, y, topk_ids, topk_w, ws, stream, block)
+    return y
+
+
+def _forward_call(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, norm_weight, norm_eps, shared_gate,
+                  y, topk_ids, topk_w, ws, stream, block):
     if block:
         opt = BlockOptions(_ptr(norm_weight), float(norm_eps), _ptr(shared_gate))
         _check(lib().moe_block_forward(ctypes.byref(prob), ctypes.byref(opt), _ptr(x), _ptr(w_router), _ptr(bias),
@@ -326,7 +385,6 @@ def _forward(prob, x, w_router, bias, wg, wu, wd, s_wg, s_wu, s_wd, scales, norm
         _check(lib().moe_layer_forward(ctypes.byref(prob), _ptr(x), _ptr(w_router), _ptr(bias), _ptr(wg), _ptr(wu),
                                        _ptr(wd), _ptr(s_wg), _ptr(s_wu), _ptr(s_wd), _ptr(scales), _ptr(y),
                                        _ptr(topk_ids), _ptr(topk_w), _ptr(ws), _nbytes(ws), _stream(stream)))
-    return y
 
 
 def layer_forward(prob, x, w_router, bias, wg, wu, wd, s_wg=None, s_wu=None, s_wd=None, scales=None, y=None,
@@ -354,10 +412,12 @@ def rmsnorm(prob, x, norm_weight, eps=1e-6, out=None, stream=None):
     _need(x, "x", prob.T * prob.d, a, prob.d)
     _need(norm_weight, "norm_weight", prob.d, a)
     _need(out, "out", prob.T * prob.d, a, prob.d)
+    cur = _device(stream, x=x, norm_weight=norm_weight, out=out)
     if out is None:
         out = torch.empty_like(x)
-    _check(lib().moe_rmsnorm(ctypes.byref(prob), _ptr(x), _ptr(norm_weight), float(eps), _ptr(out),
-                             _stream(stream)))
+    with _current(cur):
+        _check(lib().moe_rmsnorm(ctypes.byref(prob), _ptr(x), _ptr(norm_weight), float(eps), _ptr(out),
+                                 _stream(stream)))
     return out
 
 
@@ -381,9 +441,11 @@ def ep_expand_ids(counts, G, E_local, R, ids=None, stream=None):
     order with counts[s * E_local + e] rows each (int32, on the device)."""
     _need(counts, "counts", int(G) * int(E_local), _I32)
     _need(ids, "ids", int(R), _I32)
+    cur = _device(stream, counts=counts, ids=ids)
     if ids is None:
         ids = torch.empty(max(int(R), 0), dtype=torch.int32, device=counts.device)
-    _check(lib().moe_ep_expand_ids(_ptr(counts), int(G), int(E_local), int(R), _ptr(ids), _stream(stream)))
+    with _current(cur):
+        _check(lib().moe_ep_expand_ids(_ptr(counts), int(G), int(E_local), int(R), _ptr(ids), _stream(stream)))
     return ids
 
 

@@ -460,8 +460,9 @@ static Layout layout(const moe_problem& p, bool forward) {
   // chunk histograms, then the fused router's row-tile counters, then (in the
   // forward) the fused slot sum's counters: one memset clears them all
   L.counts = take(n_chunks(p) * p.E * 4 + n_chunks(p) * 4 * 4 + (forward ? p.T * sum_cnt_ld(p) * 4 : 0));
-  L.pre_a = take((p.E + 3) * 4);  // tile prefix [E+2] + the GEMM's tile-claim counter
-  L.pre_b = take((p.E + 3) * 4);
+  // tile prefix [E+2], the GEMM's tile-claim counter, the small groups' prefix [E+2]
+  L.pre_a = take((2 * p.E + 5) * 4);
+  L.pre_b = take((2 * p.E + 5) * 4);
   if (p.act_dtype == MOE_BF16) L.part = take(router_scratch_bytes(p));
   if (forward) {
     L.ids = take(n * 4);
@@ -481,8 +482,16 @@ static Layout layout(const moe_problem& p, bool forward) {
 }
 
 // ============================================================== launch pieces
-static Schedule sched_simt(int n_r, int n_s) { return Schedule{64, 64, n_r, n_s, 0}; }
-static Schedule sched_tc(int bn, int n_r, int n_s) { return Schedule{kBM, bn, n_r, n_s, 0}; }
+static Schedule sched_simt(int n_r, int n_s) { return Schedule{64, 64, n_r, n_s, 0, 0}; }
+static Schedule sched_tc(int bn, int n_r, int n_s, int small_rows = 0) {
+  return Schedule{kBM, bn, n_r, n_s, 0, small_rows};
+}
+// The row-tiled bf16 GEMMs (tiles claimed in order) spread the tiles of
+// groups with one row tile among the others; the E4M3 form (tiles dealt in a
+// fixed order) keeps the plain group order.
+static int small_rows_of(const moe_problem& p, int form) {
+  return form == kFormRows && p.w_dtype != MOE_FP8_E4M3_B128 ? kBM : 0;
+}
 
 // Router and top-k.  `counts` (may be NULL) receives the per-chunk histograms
 // for the dispatch when the tensor-core path is taken; *counted says so.  The
@@ -767,6 +776,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   a.sc_c_s = sp[4];
   a.status = dev->status;
   if (!FP8) a.sched = pre_a + p.E + 2;  // tiles claimed in order (the prefix writer zeroed it)
+  if (small_rows_of(p, kFormRows) > 0) a.prefix_small = pre_a + p.E + 3;
   PROF_BEGIN("gemm_tc_swiglu", st);
   if (!FP8 && g.x) {
     a.gx = (const bf16*)g.x;
@@ -800,6 +810,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   b.sc_b_s = sp[5];
   b.status = dev->status;
   if (!FP8) b.sched = pre_b + p.E + 2;
+  if (small_rows_of(p, kFormRows) > 0) b.prefix_small = pre_b + p.E + 3;
   if (o.ys) {
     b.ys = (bf16*)o.ys;
     b.ldy = p.d;
@@ -1020,14 +1031,14 @@ static moe_status expert_gemms(const moe_problem& p, int form, const void* xp, c
 
 static void schedules(const moe_problem& p, int form, Schedule* sa, Schedule* sb) {
   if (form == kFormRows) {
-    *sa = sched_tc(128, p.I, p.I_s);
-    *sb = sched_tc(256, p.d, p.d);
+    *sa = sched_tc(128, p.I, p.I_s, small_rows_of(p, form));
+    *sb = sched_tc(256, p.d, p.d, small_rows_of(p, form));
   } else if (form == kFormPair) {  // 256-row tiles of CTA pairs
-    *sa = Schedule{kPairBM, 128, p.I, p.I_s, 0};
-    *sb = Schedule{kPairBM, 256, p.d, p.d, 0};
+    *sa = Schedule{kPairBM, 128, p.I, p.I_s, 0, 0};
+    *sb = Schedule{kPairBM, 256, p.d, p.d, 0, 0};
   } else if (form == kFormSwap) {  // (token chunk, 128 weight rows) tiles
-    *sa = Schedule{kNCH, 128, p.I, p.I_s, 0};
-    *sb = Schedule{kNCH, 128, p.d, p.d, 0};
+    *sa = Schedule{kNCH, 128, p.I, p.I_s, 0, 0};
+    *sb = Schedule{kNCH, 128, p.d, p.d, 0, 0};
   } else {
     *sa = sched_simt(p.I, p.I_s);
     *sb = sched_simt(p.d, p.d);
@@ -1058,6 +1069,15 @@ size_t moe_stage_workspace_size(const moe_problem* p) { return check(p) == MOE_O
 moe_status moe_set_path(int path) {
   if (path < 0 || path > 4) return fail(MOE_ERR_INVALID_ARG, "path %d is not 0, 1, 2, 3 or 4", path);
   g_path = path;
+  return MOE_OK;
+}
+
+moe_status moe_set_wait_limit(int64_t cycles) {
+  DeviceInfo* dev;
+  moe_status s = device_info(&dev);
+  if (s != MOE_OK) return s;
+  const long long v = cycles > 0 ? (long long)cycles : kWaitLimitCycles;
+  CUDA_TRY(cudaMemcpyToSymbol(g_wait_limit, &v, sizeof v));
   return MOE_OK;
 }
 

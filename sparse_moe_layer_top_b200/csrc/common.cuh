@@ -63,9 +63,18 @@ __device__ __forceinline__ int find_group(const int32_t* prefix, int ngroups, in
 // tiles of group g = m_tiles(rows_g) * ceil(N_g / bn), with
 // m_tiles = ceil(rows / bm) for the row-tiled kernels, and 0 or 1 for the
 // weight-row (swap) kernels whose N covers every row of a group.
+// Tiles of a grouped GEMM: ceil(rows / bm) x ceil(n / bn) per group (one
+// row tile per group when swap).  With small_rows > 0 the groups of at most
+// small_rows rows (one row tile: each of their tiles streams its weight block
+// from HBM for few rows) are counted in a prefix of their own, so that the
+// GEMM can spread their tiles evenly among the others (see decode_tile).
 struct Schedule {
-  int bm, bn, n_routed, n_shared, swap;
+  int bm, bn, n_routed, n_shared, swap, small_rows;
 };
+
+__host__ __device__ __forceinline__ bool sched_small(const Schedule& s, int rows) {
+  return s.small_rows > 0 && rows > 0 && rows <= s.small_rows;
+}
 
 __device__ __forceinline__ int sched_tiles(const Schedule& s, int g, int E, int rows) {
   int n = g < E ? s.n_routed : s.n_shared;

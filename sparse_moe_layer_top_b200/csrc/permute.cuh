@@ -68,16 +68,22 @@ __device__ __forceinline__ int block_incl_scan(int v, int* sm_warp) {
 
 // Tile prefix of one schedule from the group sizes (E+1 groups, one thread each).
 // prefix[E + 2] is the GEMM's tile-claim counter, zeroed here (see TcGemmArgs::sched).
+// A schedule that splits off its small groups (Schedule::small_rows) has
+// prefix[0 .. E+1] over the other groups and prefix[E+3 .. 2E+4] over the
+// small ones (each counting only its own groups' tiles).
 __device__ __forceinline__ void write_tile_prefix(const Schedule& s, int E, int rows_g, int32_t* prefix,
                                                   int* sm_warp) {
-  int g = threadIdx.x;
-  int tiles = (g <= E) ? sched_tiles(s, g, E, rows_g) : 0;
-  int incl = block_incl_scan(tiles, sm_warp);
-  if (g <= E) prefix[g] = incl - tiles;
-  if (g == E) {
-    prefix[E + 1] = incl;
-    prefix[E + 2] = 0;
+  const int g = threadIdx.x;
+  const int tiles = (g <= E) ? sched_tiles(s, g, E, rows_g) : 0;
+  const bool small = g <= E && sched_small(s, rows_g);
+  for (int part = 0; part < (s.small_rows > 0 ? 2 : 1); ++part) {
+    int32_t* q = part ? prefix + E + 3 : prefix;
+    const int mine = small == (part == 1) ? tiles : 0;
+    const int incl = block_incl_scan(mine, sm_warp);
+    if (g <= E) q[g] = incl - mine;
+    if (g == E) q[E + 1] = incl;
   }
+  if (g == E) prefix[E + 2] = 0;
 }
 
 // Tile prefixes from caller-supplied group offsets (the expert stage alone).
@@ -169,32 +175,39 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
     }
     // tile prefixes over the E+1 groups (group E: the shared expert); with
     // E == 512 the shared group is one past the 512 the block scans
+    // (a schedule that splits off its small groups gets a second prefix over
+    // them at pf + E + 3, as write_tile_prefix lays it out)
     for (int which = 0; which < 2; ++which) {
       const Schedule& sc = which ? sb : sa;
       int32_t* pf = which ? prefix_b : prefix_a;
       if (!pf) continue;
-      int tl[2];
+      for (int part = 0; part < (sc.small_rows > 0 ? 2 : 1); ++part) {
+        int32_t* q = part ? pf + E + 3 : pf;
+        int tl[2];
 #pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int g = 2 * threadIdx.x + h;
-        const int rows = g < E ? tot[h] : (has_shared ? (int)T : 0);
-        tl[h] = g <= E ? sched_tiles(sc, g, E, rows) : 0;
-      }
-      const int2 ti = block256_scan2(tl[0], tl[1], sm_warp);
-      if (2 * threadIdx.x <= E) pf[2 * threadIdx.x] = ti.x - tl[0];
-      if (2 * threadIdx.x + 1 <= E) pf[2 * threadIdx.x + 1] = ti.y - tl[1];
-      if (threadIdx.x == blockDim.x - 1) s_tot = ti.y;
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        if (E < kMaxE) {
-          pf[E + 1] = s_tot;
-        } else {
-          pf[E] = s_tot;
-          pf[E + 1] = s_tot + sched_tiles(sc, E, E, has_shared ? (int)T : 0);
+        for (int h = 0; h < 2; ++h) {
+          const int g = 2 * threadIdx.x + h;
+          const int rows = g < E ? tot[h] : (has_shared ? (int)T : 0);
+          const int n = g <= E ? sched_tiles(sc, g, E, rows) : 0;
+          tl[h] = sched_small(sc, rows) == (part == 1) ? n : 0;
         }
-        pf[E + 2] = 0;  // the GEMM's tile-claim counter
+        const int2 ti = block256_scan2(tl[0], tl[1], sm_warp);
+        if (2 * threadIdx.x <= E) q[2 * threadIdx.x] = ti.x - tl[0];
+        if (2 * threadIdx.x + 1 <= E) q[2 * threadIdx.x + 1] = ti.y - tl[1];
+        if (threadIdx.x == blockDim.x - 1) s_tot = ti.y;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+          if (E < kMaxE) {
+            q[E + 1] = s_tot;
+          } else {
+            const int sh_rows = has_shared ? (int)T : 0;
+            q[E] = s_tot;
+            q[E + 1] = s_tot + (sched_small(sc, sh_rows) == (part == 1) ? sched_tiles(sc, E, E, sh_rows) : 0);
+          }
+          if (part == 0) pf[E + 2] = 0;  // the GEMM's tile-claim counter
+        }
+        __syncthreads();
       }
-      __syncthreads();
     }
   }
   // 3. pairs of the chunk's tokens before this block: they precede ours in every group

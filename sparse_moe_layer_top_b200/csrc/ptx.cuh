@@ -47,25 +47,35 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Every wait in the library is bounded: after about kWaitLimitCycles SM
-// cycles without progress (about 2 s at B200 clocks; longer at lower clocks,
-// bounded all the same) the waiter records `where` in the device status word,
-// raises the CTA's abort flag and returns false; any other waiter of the CTA
-// that sees the abort flag returns false at once.  Kernels then skip their
-// remaining work, drain what they issued and release TMEM before exiting.
-// The bound is kept off the fast path: the cycle counter and the abort flag
-// are read once every 256 polls.
+// Every wait in the library is bounded: after about g_wait_limit SM cycles
+// without progress (by default kWaitLimitCycles, about 2 s at B200 clocks;
+// longer at lower clocks, bounded all the same) the waiter records `where` in
+// the device status word, raises the CTA's abort flag and returns false; any
+// other waiter of the CTA that sees the abort flag returns false at once.
+// Kernels then skip their remaining work, drain what they issued and release
+// TMEM before exiting; those drains always allow kWaitLimitCycles, whatever
+// g_wait_limit says, so a copy in flight lands before its CTA exits.
+// moe_set_wait_limit changes g_wait_limit (a short limit makes a test's waits
+// give up on purpose).  The bound is kept off the fast path: at the default
+// limit the cycle counter and the abort flag are read once every 256 polls; a
+// limit under kShortWaitLimit is checked on every poll, so that it holds.
 constexpr long long kWaitLimitCycles = 4000000000ll;
+constexpr long long kShortWaitLimit = 1ll << 24;
+static __device__ long long g_wait_limit = kWaitLimitCycles;
+
+__device__ __forceinline__ long long wait_limit() { return *reinterpret_cast<volatile long long*>(&g_wait_limit); }
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                           unsigned* status, unsigned where) {
   if (mbar_try_wait(bar, parity)) return true;
+  const long long lim = wait_limit();
+  const uint32_t mask = lim < kShortWaitLimit ? 0u : 255u;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0) {
+    if ((i & mask) == 0) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > lim) {
         *abort_flag = 1;
         atomicCAS(status, 0u, where);
         return false;
@@ -286,12 +296,14 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t pa
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                                   unsigned* status, unsigned where) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
+  const long long lim = wait_limit();
+  const uint32_t mask = lim < kShortWaitLimit ? 0u : 255u;
   const long long t0 = clock64();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
-    if ((i & 255u) == 0) {
+    if ((i & mask) == 0) {
       if (*abort_flag) return false;
-      if (clock64() - t0 > kWaitLimitCycles) {
+      if (clock64() - t0 > lim) {
         *abort_flag = 1;
         atomicCAS(status, 0u, where);
         return false;

@@ -166,3 +166,25 @@ def test_layer_object_checks_its_weights_once_and_its_tokens_every_call():
         layer(a["x"], y=a["y"][:-1])
     with pytest.raises(ValueError, match=ON_DEVICE):
         layer(a["x"], y=a["y"], topk_ids=a["topk_ids"], topk_w=a["topk_w"])
+
+
+def test_tensors_on_different_devices_are_rejected_before_any_pointer():
+    """The library launches on the current device with the pointers it is
+    given, so one call's tensors must share a device: a mix is refused,
+    naming the tensors, before the pointer step (here a CPU tensor beside a
+    meta tensor stands for cuda:0 beside cuda:1)."""
+    a = _forward_args()
+    a["w_router"] = a["w_router"].to("meta")
+    with pytest.raises(ValueError, match="different devices.*w_router on meta"):
+        _forward(a)
+    a = _forward_args()
+    p = a["prob"]
+    with pytest.raises(ValueError, match="different devices"):
+        moe.router_topk(p, a["x"], a["w_router"], None, topk_ids=a["topk_ids"].to("meta"))
+    with pytest.raises(ValueError, match="different devices"):
+        moe.combine(p, torch.zeros((p.T * (p.k + 1), p.d), dtype=torch.bfloat16), a["topk_ids"], a["topk_w"],
+                    torch.zeros(p.E + 2, dtype=torch.int32), y=a["y"].to("meta"))
+    layer = moe.MoELayer(p.d, p.E, p.k, 128, 128, a["w_router"], a["wg"], a["wu"], a["wd"], a["s_wg"], a["s_wu"],
+                         a["s_wd"])
+    with pytest.raises(ValueError, match="different devices"):
+        layer(a["x"].to("meta"))

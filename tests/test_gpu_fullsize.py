@@ -1,13 +1,14 @@
 """Parity at the full workload sizes, in the launch configuration the
 benchmark times (MoELayer over the whole batch).
 
-The oracle cannot redo a whole batch at these sizes, so it recomputes a few
-sampled tokens -- the first and last, a token of the hottest and of the
-coldest active expert, and two more -- from host copies of only the experts
-those tokens use (the renormalised weights over a token's kept set do not
-depend on which other experts exist, so a compact expert list with the set
-forced gives the same result).  Properties that hold at any size are checked
-on every token.
+The oracle cannot redo a whole batch at these sizes, so it recomputes sampled
+tokens -- the first and last, a token of the hottest and of the coldest active
+expert, and one token in each 128-token row tile (the router's and the
+row-tiled GEMMs' tiles), while the experts they use fit a host budget -- from
+host copies of only those experts (the renormalised weights over a token's
+kept set do not depend on which other experts exist, so a compact expert list
+with the set forced gives the same result).  Properties that hold at any size
+are checked on every token.
 """
 import gc
 
@@ -43,7 +44,14 @@ def _pick(t, sel):
     return t[sel].cpu()
 
 
-def _sample_tokens(ids, T):
+HOST_BUDGET = 16 << 30  # bytes of expert weights copied to the host for the oracle
+
+
+def _sample_tokens(ids, T, per_expert_bytes):
+    """First, last, hottest- and coldest-expert tokens, then one token at a
+    seeded offset in every 128-token row tile, then up to 32 seeded ones, in
+    that order, each kept while the union of the kept tokens' experts fits
+    HOST_BUDGET (96 tokens at most)."""
     flat = ids.reshape(-1).long()
     cnt = torch.bincount(flat, minlength=int(flat.max()) + 1)
     hot = int(cnt.argmax())
@@ -52,8 +60,18 @@ def _sample_tokens(ids, T):
     tok_hot = int(torch.nonzero((ids == hot).any(1)).flatten()[0])
     tok_cold = int(torch.nonzero((ids == cold).any(1)).flatten()[-1])
     g = torch.Generator().manual_seed(1)
-    extra = torch.randint(0, T, (2,), generator=g).tolist()
-    return sorted(set([0, T - 1, tok_hot, tok_cold] + extra))
+    tiles = [min(T - 1, r0 + int(torch.randint(0, 128, (1,), generator=g))) for r0 in range(0, T, 128)]
+    more = torch.randperm(T, generator=g)[:32].tolist()  # a batch of a tile or two: more of its tokens
+    ids_h = ids.cpu()
+    max_experts = HOST_BUDGET // per_expert_bytes
+    keep, used = [], set()
+    for t in [0, T - 1, tok_hot, tok_cold] + tiles + more:
+        s = set(ids_h[t].tolist())
+        if t in keep or len(used | s) > max_experts or len(keep) == 96:
+            continue
+        keep.append(t)
+        used |= s
+    return sorted(keep)
 
 
 @pytest.mark.parametrize("name", WORKLOADS)
@@ -79,7 +97,10 @@ def test_full_size_sampled_tokens(name):
     assert (tw[:, :-1] >= tw[:, 1:] - 1e-7).all(), "weights not in descending order"
 
     # sampled tokens against the oracle
-    toks = _sample_tokens(ids, T)
+    per_expert = sum(t[0].numel() * t.element_size() for t in (inp.wg, inp.wu, inp.wd))
+    toks = _sample_tokens(ids, T, per_expert)
+    # every row tile is represented unless the host budget stopped it
+    assert len(toks) >= min(T // 128 + 2, 12), toks
     key = precision_key(inp)
     x_s = inp.x[toks].cpu()
     w_r = inp.w_r.cpu()

@@ -328,13 +328,21 @@ def test_out_of_range_expert_id_sets_device_status(moe):
     assert moe.device_status()[0] == 0  # reading clears it
 
 
-def test_repeat_calls_are_deterministic_in_routing_and_close_in_output(moe):
-    inp = _make("bf16_multi_tile", seed=4)
+@pytest.mark.parametrize("path", [0, 1, 2, 3, 4])
+@pytest.mark.parametrize("case", ["bf16_multi_tile", "bf16_fused_router", "bf16_auto_pair", "fp8_multi_tile"])
+def test_repeat_calls_are_bit_identical(moe, case, path):
+    """No floating-point atomics anywhere in the forward: the router sums its
+    K splits in order, every output element comes from one tile with a fixed K
+    order (whatever tile a CTA claims), and each token's slot rows are summed
+    in slot order -- so two calls give the same bits."""
+    inp = _make(case, seed=4)
     g = to_device(inp, "cuda")
+    moe.set_path(path)
     y1, ids1, tw1 = _gpu_forward(moe, g)
     y2, ids2, tw2 = _gpu_forward(moe, g)
+    _no_device_errors(moe)
     assert np.array_equal(ids1, ids2) and np.array_equal(tw1, tw2)
-    assert rel_l2(y1, y2) <= 1e-3  # only the order of the fp32 reductions may differ
+    assert np.array_equal(y1, y2)
 
 
 def test_launch_count_reported(moe):
