@@ -152,24 +152,12 @@ def routing(moe, layer, x):
     return ids, cnt
 
 
-def forward_plan(c, T):
-    """The fused forward's kernel choices, as the library decides them
-    (moe_forward_plan, host only)."""
-    import sparse_moe_layer_top_b200 as moe
-    prob = moe.Problem.make(T, c["d"], c["E"], c["k"], c["I"], c["I_s"], c["act"], c["w"])
-    return moe.forward_plan(prob)
-
-
 def gathers_rows(c, T):
     """Whether the fused forward's gate/up GEMM reads its rows straight from the
-    token matrix."""
-    return forward_plan(c, T)["gathered"]
-
-
-def down_sums_slots(c, T):
-    """Whether the down GEMM also sums each token's slot rows into y (the
-    row-tiled form), so that y is written by it."""
-    return forward_plan(c, T)["slot_sum_in_down"]
+    token matrix, as the library decides it (moe_forward_plan, host only)."""
+    import sparse_moe_layer_top_b200 as moe
+    prob = moe.Problem.make(T, c["d"], c["E"], c["k"], c["I"], c["I_s"], c["act"], c["w"])
+    return moe.forward_plan(prob)["gathered"]
 
 
 def work_model(c, counts, T):
@@ -179,7 +167,7 @@ def work_model(c, counts, T):
     the shared expert); each kernel's activations once in and once out (the
     gate/up GEMM reads the dispatched rows -- or, where it gathers them, the
     token matrix itself -- and writes H; the down GEMM reads H and writes the
-    weighted (token, slot) rows, and y where it sums them itself).  For the whole block only the weights, W_r,
+    weighted (token, slot) rows).  For the whole block only the weights, W_r,
     x and y count: the dispatch copy, H and the slot rows are overheads."""
     d, E, k, I, I_s = c["d"], c["E"], c["k"], c["I"], c["I_s"]
     ab = 4 if c["act"] == "f32" else 2
@@ -192,8 +180,7 @@ def work_model(c, counts, T):
     h_bytes = (R * I + sh * T * I_s) * ab
     a_in = (T if gathers_rows(c, T) else R + sh * T) * d * ab
     g1 = {"bytes": w_gu + a_in + h_bytes, "flops": 4 * d * (R * I + sh * T * I_s)}
-    y_out = T * d * ab if down_sums_slots(c, T) else 0
-    g2 = {"bytes": w_dn + h_bytes + (R + sh * T) * d * ab + y_out, "flops": 2 * d * (R * I + sh * T * I_s)}
+    g2 = {"bytes": w_dn + h_bytes + (R + sh * T) * d * ab, "flops": 2 * d * (R * I + sh * T * I_s)}
     layer = {"bytes": w_gu + w_dn + E * d * ab + 2 * T * d * ab,
              "flops": 2 * T * d * E + 6 * d * (R * I + sh * T * I_s)}
     if c["w"] == "fp8":

@@ -147,13 +147,8 @@ MOE_API moe_status moe_combine(const moe_problem* p, const void* y_perm, const i
  * router + top-k, dispatch, gate/up GEMM with SwiGLU,
  * down GEMM whose epilogue applies the routing weight and stores each row in
  * (token, slot) order, then one ordered fp32 sum per token of its k slot rows
- * and its shared-expert row (reproducible: the order of the additions is
- * fixed).  On the row-tiled form that sum runs in the down GEMM's epilogue:
- * the warp that stores a token's last slot row over a column span adds the
- * token's rows there (counters in the workspace say which is last); the other
- * forms run it as a separate pass.  Both give the same bits.  y [T, d] in the
- * activation type.  topk_ids_out and topk_w_out ([T, k]) may be NULL.  ws:
- * moe_workspace_size() bytes.
+ * and its shared-expert row (reproducible: no atomics).  y [T, d] in the activation type.  topk_ids_out and
+ * topk_w_out ([T, k]) may be NULL.  ws: moe_workspace_size() bytes.
  * On the row-tiled bf16 form (see moe_set_path) with T * d * 2 <= 32 MiB the
  * gate/up GEMM reads each dispatched row straight from x (the rows stay in
  * L2 while the weights stream), and the dispatch writes no copy of them. */
@@ -250,14 +245,12 @@ MOE_API moe_status moe_router_topk_static(const moe_problem* p, const void* x, c
  * (swap-AB) GEMMs, 3 row-tiled GEMMs on CTA pairs; router_selects: 1 when the
  * router's GEMM selects the top k in its epilogue (bf16, E <= 256, at least
  * 16 tiles of 128 tokens), 0 for the split-K GEMM + top-k kernel or the SIMT
- * router; gathered: 1 when the gate/up GEMM reads its rows straight from x;
- * slot_sum_in_down: 1 when the down GEMM's epilogue sums each token's slot
- * rows into y (the row-tiled form), 0 when a separate pass does.
+ * router; gathered: 1 when the gate/up GEMM reads its rows straight from x.
  * Any output pointer may be NULL.  Errors: those of moe_check_problem, and
  * MOE_ERR_UNSUPPORTED where moe_set_path asks for a form the types do not
  * allow. */
 MOE_API moe_status moe_forward_plan(const moe_problem* p, int32_t* expert_form, int32_t* router_selects,
-                            int32_t* gathered, int32_t* slot_sum_in_down);
+                            int32_t* gathered);
 
 /* Kernel-path selection for the calls above on the calling process:
  * 0 = automatic (tensor-core kernels where the types allow; for the expert

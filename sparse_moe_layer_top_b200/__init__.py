@@ -91,7 +91,7 @@ def lib():
                                         P, ctypes.c_size_t, P]
         L.moe_ep_expand_ids.argtypes = [P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int64, P, P]
         I32P = ctypes.POINTER(ctypes.c_int32)
-        L.moe_forward_plan.argtypes = [PP, I32P, I32P, I32P, I32P]
+        L.moe_forward_plan.argtypes = [PP, I32P, I32P, I32P]
         L.moe_rmsnorm.argtypes = [PP, P, P, ctypes.c_float, P, P]
         L.moe_set_path.argtypes = [ctypes.c_int]
         L.moe_set_wait_limit.argtypes = [ctypes.c_int64]
@@ -426,13 +426,10 @@ EXPERT_FORMS = ("simt", "rows", "weight_rows", "cta_pairs")
 
 def forward_plan(prob):
     """What the fused forward launches for `prob` under the current path,
-    decided on the host: dict(expert_form, router_selects, gathered,
-    slot_sum_in_down)."""
-    f, r, g, ss = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
-    _check(lib().moe_forward_plan(ctypes.byref(prob), ctypes.byref(f), ctypes.byref(r), ctypes.byref(g),
-                                  ctypes.byref(ss)))
-    return {"expert_form": EXPERT_FORMS[f.value], "router_selects": bool(r.value), "gathered": bool(g.value),
-            "slot_sum_in_down": bool(ss.value)}
+    decided on the host: dict(expert_form, router_selects, gathered)."""
+    f, r, g = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    _check(lib().moe_forward_plan(ctypes.byref(prob), ctypes.byref(f), ctypes.byref(r), ctypes.byref(g)))
+    return {"expert_form": EXPERT_FORMS[f.value], "router_selects": bool(r.value), "gathered": bool(g.value)}
 
 
 def ep_expand_ids(counts, G, E_local, R, ids=None, stream=None):

@@ -357,9 +357,6 @@ static moe_status choose(bool tc_possible, bool* use_tc) {
 // rows per expert, even at 1024, slower on prefill-sized Zipf-skewed groups);
 // else the row-tiled form.
 enum { kFormSimt = 0, kFormRows = 1, kFormSwap = 2, kFormPair = 3 };
-// The row-tiled down GEMM sums each token's slot rows in its epilogue; the
-// other forms leave that to k_slot_sum.
-static bool sums_in_down(int form) { return form == kFormRows; }
 constexpr int kPairRowsPerExpert = 2048;
 static moe_status choose_form(const moe_problem& p, int* form) {
   bool tc;
@@ -439,9 +436,6 @@ struct Layout {
 static int64_t rows_total(const moe_problem& p) { return p.T * p.k + (p.I_s > 0 ? p.T : 0); }
 static int64_t n_chunks(const moe_problem& p) { return std::max<int64_t>(1, cdiv(p.T, kChunkTokens)); }
 static int64_t ldh_of(const moe_problem& p) { return std::max(p.I, p.I_s); }
-// counters per token of the fused slot sum: one per 128 columns of y (an
-// epilogue warp's span: 128 columns, or 256 with E4M3 weights)
-static int64_t sum_cnt_ld(const moe_problem& p) { return cdiv(p.d, 128); }
 
 // Workspace of moe_layer_forward (forward) or of the stage calls.  In the
 // forward, the dispatched rows x_perm and the weighted (token, slot) rows of
@@ -457,9 +451,8 @@ static Layout layout(const moe_problem& p, bool forward) {
   };
   const int64_t n = p.T * p.k, Rp = rows_total(p);
   const size_t ab = esize(p.act_dtype);
-  // chunk histograms, then the fused router's row-tile counters, then (in the
-  // forward) the fused slot sum's counters: one memset clears them all
-  L.counts = take(n_chunks(p) * p.E * 4 + n_chunks(p) * 4 * 4 + (forward ? p.T * sum_cnt_ld(p) * 4 : 0));
+  // chunk histograms, then the fused router's row-tile counters (one memset clears both)
+  L.counts = take(n_chunks(p) * p.E * 4 + n_chunks(p) * 4 * 4);
   // tile prefix [E+2], the GEMM's tile-claim counter, the small groups' prefix [E+2]
   L.pre_a = take((2 * p.E + 5) * 4);
   L.pre_b = take((2 * p.E + 5) * 4);
@@ -494,12 +487,10 @@ static int small_rows_of(const moe_problem& p, int form) {
 }
 
 // Router and top-k.  `counts` (may be NULL) receives the per-chunk histograms
-// for the dispatch when the tensor-core path is taken; *counted says so.  The
-// memset that zeroes them also zeroes the zero_extra bytes that follow the
-// router's row-tile counters (the forward's slot-sum counters).
+// for the dispatch when the tensor-core path is taken; *counted says so.
 static moe_status launch_router(const moe_problem& p, const void* x, const void* wr, const float* bias,
                                 int32_t* ids, float* tw, float* part, int32_t* counts, bool* counted,
-                                cudaStream_t st, DeviceInfo* dev, size_t zero_extra = 0) {
+                                cudaStream_t st, DeviceInfo* dev) {
   *counted = false;
   if (p.T == 0) return MOE_OK;
   bool tc;
@@ -535,7 +526,7 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
     // quadruple per chunk), else in the scratch
     int32_t* cnt = counts ? counts + n_chunks(p) * p.E : reinterpret_cast<int32_t*>(scratch + ts.cnt_off);
     if (counts) {
-      CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * (p.E + 4) * 4 + zero_extra, st));
+      CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * (p.E + 4) * 4, st));
       pdl_reset();
     } else if (ts.ntc > 1) {
       CUDA_TRY(cudaMemsetAsync(cnt, 0, (size_t)ts.row_tiles * 4 * 4, st));
@@ -580,8 +571,7 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
   a.part_stride = p.T * rs.ldp;
   a.status = dev->status;
   if (counts) {  // the chunk histograms k_topk counts into
-    const size_t hist = (size_t)n_chunks(p) * p.E * 4;
-    CUDA_TRY(cudaMemsetAsync(counts, 0, zero_extra ? hist + (size_t)n_chunks(p) * 16 + zero_extra : hist, st));
+    CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * p.E * 4, st));
     pdl_reset();
   }
   PROF_BEGIN("gemm_tc_router", st);
@@ -608,7 +598,7 @@ static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, cons
                                   int32_t* offs, int32_t* row_tok, float* row_w, int32_t* pos, int32_t* row_dst,
                                   int32_t* counts, Schedule sa, int32_t* pre_a, Schedule sb, int32_t* pre_b,
                                   const void* x, void* xp, cudaStream_t st, DeviceInfo* dev,
-                                  const float* shared_gate = nullptr, void* y0 = nullptr) {
+                                  const float* shared_gate = nullptr) {
   const int nch = (int)n_chunks(p);
   if (p.T == 0) {
     CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)p.E * 4, st));
@@ -622,7 +612,7 @@ static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, cons
   PROF_BEGIN("dispatch", st);
   CUDA_TRY(launch(k_dispatch, nch * kSubBlocks, kScatterWarps * 32, 0, st, ids, tw, p.T, p.k, p.E, counts, nch,
                   p.I_s > 0, offs, sa, pre_a, sb, pre_b, row_tok, row_w, pos, row_dst, shared_gate,
-                  (const uint4*)x, vec, (uint4*)xp, (uint4*)y0));
+                  (const uint4*)x, vec, (uint4*)xp));
   LAUNCH_CHECK("dispatch", st);
   return MOE_OK;
 }
@@ -669,12 +659,6 @@ struct DownOut {
   const int32_t* row_dst;
   const float* row_w;
   void* out;              // dispatch layout [R', d], or NULL
-  // the row-tiled tensor-core down GEMM also sums the slot rows into y when
-  // y is set (counters sum_cnt [T, cnt_ld], zeroed before the launch)
-  void* y;
-  const int32_t* pos;
-  unsigned* sum_cnt;
-  int cnt_ld;
 };
 
 template <typename TA, typename TW>
@@ -816,14 +800,6 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
     b.ldy = p.d;
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
-    if (o.y) {
-      b.y = (bf16*)o.y;
-      b.pos = o.pos;
-      b.sum_cnt = o.sum_cnt;
-      b.k_slots = p.k;
-      b.has_shared = sh ? 1 : 0;
-      b.cnt_ld = o.cnt_ld;
-    }
     PROF_BEGIN("gemm_tc_down", st);
     CUDA_TRY(launch(k_gemm_tc<256, false, S, kTcSlotStore, FP8>,
                     dev->sms, C2::THREADS, C2::SMEM_BYTES, st, aR, aS, bR, bS, bR, bS, b));
@@ -1329,11 +1305,7 @@ static moe_status block_forward(const moe_problem* p, const moe_block_options* o
     if (norm_w) xin = wsp + L.xn;
   }
   bool counted;
-  // the row-tiled down GEMM sums each token's slot rows itself (its counters
-  // follow the router's, zeroed by the router's memset)
-  const bool fuse_sum = sums_in_down(form);
-  s = launch_router(*p, xin, w_router, router_bias, ids, tw, (float*)(wsp + L.part), counts, &counted, st, dev,
-                    fuse_sum ? (size_t)p->T * sum_cnt_ld(*p) * 4 : 0);
+  s = launch_router(*p, xin, w_router, router_bias, ids, tw, (float*)(wsp + L.part), counts, &counted, st, dev);
   if (s != MOE_OK) return s;
   Schedule sa, sb;
   schedules(*p, form, &sa, &sb);
@@ -1344,21 +1316,11 @@ static moe_status block_forward(const moe_problem* p, const moe_block_options* o
   GatherSrc gs;
   if (gathers_rows(*p, form)) gs = GatherSrc{xin, row_tok};
   s = launch_dispatch(*p, ids, tw, counted, offs, row_tok, row_w, pos, row_dst, counts, sa, pre_a, sb, pre_b, xin,
-                      gs.x ? nullptr : xp, st, dev, gate, fuse_sum ? y : nullptr);
+                      gs.x ? nullptr : xp, st, dev, gate);
   if (s != MOE_OK) return s;
   DownOut o{xp, row_dst, row_w, nullptr};  // the slot rows reuse the dispatched-row buffer
-  if (fuse_sum) {
-    o.y = y;
-    o.pos = pos;
-    o.sum_cnt = reinterpret_cast<unsigned*>(counts + n_chunks(*p) * (p->E + 4));
-    o.cnt_ld = (int)sum_cnt_ld(*p);
-  }
   s = expert_gemms(*p, form, xp, offs, w, pre_a, pre_b, wsp + L.h, o, st, dev, gs);
   if (s != MOE_OK) return s;
-  if (fuse_sum) {
-    g_launches = g_launches_pending;
-    return MOE_OK;
-  }
   PROF_BEGIN("slot_sum", st);
   if (p->act_dtype == MOE_F32)
     CUDA_TRY(launch(k_slot_sum<float>,
@@ -1409,7 +1371,7 @@ moe_status moe_rmsnorm(const moe_problem* p, const void* x, const void* norm_wei
 }
 
 moe_status moe_forward_plan(const moe_problem* p, int32_t* expert_form, int32_t* router_selects,
-                            int32_t* gathered, int32_t* slot_sum_in_down) {
+                            int32_t* gathered) {
   moe_status s = check(p);
   if (s != MOE_OK) return s;
   int form;
@@ -1419,7 +1381,6 @@ moe_status moe_forward_plan(const moe_problem* p, int32_t* expert_form, int32_t*
   if (expert_form) *expert_form = form;
   if (router_selects) *router_selects = router_tc && router_fused(*p) ? 1 : 0;
   if (gathered) *gathered = gathers_rows(*p, form) ? 1 : 0;
-  if (slot_sum_in_down) *slot_sum_in_down = sums_in_down(form) ? 1 : 0;
   return MOE_OK;
 }
 

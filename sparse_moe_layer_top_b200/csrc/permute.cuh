@@ -133,8 +133,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
     const int32_t* __restrict__ counts, int nchunks, int has_shared, int32_t* __restrict__ offs, Schedule sa,
     int32_t* __restrict__ prefix_a, Schedule sb, int32_t* __restrict__ prefix_b, int32_t* __restrict__ row_tok,
     float* __restrict__ row_w, int32_t* __restrict__ pos, int32_t* __restrict__ row_dst,
-    const float* __restrict__ shared_gate, const uint4* __restrict__ x, int vec_per_row, uint4* __restrict__ xp,
-    uint4* __restrict__ y0) {
+    const float* __restrict__ shared_gate, const uint4* __restrict__ x, int vec_per_row, uint4* __restrict__ xp) {
   pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   __shared__ int32_t wb[kScatterWarps][kMaxE];
   __shared__ int32_t s_base[kMaxE];
@@ -264,21 +263,6 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
       row_tok[R + t] = (int32_t)t;
       row_w[R + t] = shared_gate ? __ldg(shared_gate + t) : 1.0f;  // the shared expert's weight
       if (row_dst) row_dst[R + t] = (int32_t)(t * (k + 1) + k);
-    }
-  }
-  // y0 (the down GEMM sums the slot rows itself, so it never reaches a token
-  // without any): a token none of whose pairs is valid, with no shared
-  // expert, has no slot row; its row of y is zeroed here, as the separate
-  // slot-sum pass leaves it
-  if (y0 && !has_shared) {
-    __syncwarp();
-    for (int tt = 0; tt < kWarpTokens; ++tt) {
-      const int64_t t = t_blk + (int64_t)warp * kWarpTokens + tt;
-      if (t >= T) break;
-      bool any = false;
-      for (int j = lane; j < k; j += 32) any |= s_dst[warp][tt * k + j] >= 0;
-      if (__any_sync(0xffffffffu, any)) continue;
-      for (int v = lane; v < vec_per_row; v += 32) y0[t * vec_per_row + v] = make_uint4(0u, 0u, 0u, 0u);
     }
   }
   if (!xp) return;

@@ -69,16 +69,6 @@ struct TcGemmArgs {
   int64_t ldy;
   const int32_t* row_dst; // SlotStore: destination row of each dispatched row
   const float* row_w;     // SlotStore: routing weight of each dispatched row
-  // SlotStore with the slot sum fused (y != NULL): once an epilogue warp has
-  // stored its rows over its column span, each of them counts once in
-  // sum_cnt[token][span] (zeroed before the launch); the row that completes a
-  // token's count (its valid slots, pos[t][j] >= 0, plus the shared row when
-  // has_shared) has the warp add the token's slot rows over that span in slot
-  // order, in fp32, and write y[token] -- what a separate slot-sum pass does.
-  bf16* y;                // [T, d]
-  const int32_t* pos;     // [T, k_slots]
-  unsigned* sum_cnt;      // [T, cnt_ld]
-  int k_slots, has_shared, cnt_ld;
   bf16* out;              // Store output [rows, ldo]
   int64_t ldo;
   float* part;            // Logits output [ksplit][rows, ldp]
@@ -387,100 +377,6 @@ __device__ __forceinline__ void epilogue_rows(const TcGemmArgs& p, const TileInf
     }
     const int n = t.n0 + c * 32;
     store_rows_staged(stg, o, rowp, (int64_t)n * 2, t.N - n, lane);
-  }
-}
-
-// Slot sum fused into the down GEMM (SlotStore with p.y set), run by one
-// epilogue warp right after it has stored its 32 rows over the 32 * VEC
-// columns from n0c.  Release: every lane fences its own stores, the warp
-// syncs, then each lane counts its row in sum_cnt[token][span].  Acquire: the
-// lane whose count completes the token's (all valid slot rows of that span
-// landed, from any CTA) is found by ballot, every lane fences, the warp syncs,
-// and the warp
-// adds that token's slot rows through L2 (lane l: columns n0c + VEC l ..
-// + VEC - 1), slots 0..k in order, in fp32 from zero -- the arithmetic of the
-// separate slot-sum pass, so y is the same bit for bit.
-template <int VEC>
-__device__ __forceinline__ void slot_sum_fused(const TcGemmArgs& p, const TileInfo& t, int row, int n0c, int lane) {
-  static_assert(VEC == 4 || VEC == 8, "a lane sums 8 or 16 bytes of each slot row");
-  // a span wholly past the last column (d not a multiple of 256) stores
-  // nothing and has no counter: sum_cnt holds cdiv(d, 128) per token
-  if (n0c >= t.N) return;
-  const int64_t grow = t.row0 + row;
-  const bool valid = t.m0 + row < t.rows && grow < p.rows_cap;
-  const int ks = p.k_slots + 1;  // slot rows per token (the last one the shared expert's)
-  const int64_t dr = valid ? (int64_t)__ldg(p.row_dst + grow) : -1;
-  __threadfence();
-  __syncwarp();
-  int tok = -1;
-  bool last = false;
-  if (dr >= 0) {
-    tok = (int)(dr / ks);
-    unsigned need = p.has_shared ? 1u : 0u;
-    for (int j = 0; j < p.k_slots; ++j) need += __ldg(p.pos + (int64_t)tok * p.k_slots + j) >= 0 ? 1u : 0u;
-    const unsigned old = atomicAdd(p.sum_cnt + (int64_t)tok * p.cnt_ld + n0c / (32 * VEC), 1u);
-    last = old + 1 == need;
-  }
-  unsigned m = __ballot_sync(0xffffffffu, last);
-  if (m == 0) return;
-  // the completing lane's fence, then a warp barrier (which orders memory
-  // among the warp's lanes, unlike the ballot) before any lane's loads
-  __threadfence();
-  __syncwarp();
-  const int c = n0c + lane * VEC;
-  const bool cin = c < t.N;  // N % 8 == 0: a lane's columns are all in or all out
-  while (m) {
-    const int src = __ffs(m) - 1;
-    m &= m - 1;
-    const int tk = __shfl_sync(0xffffffffu, tok, src);
-    const int pj = lane < p.k_slots ? __ldg(p.pos + (int64_t)tk * p.k_slots + lane) : -1;
-    unsigned ok = __ballot_sync(0xffffffffu, pj >= 0);
-    if (p.has_shared) ok |= 1u << p.k_slots;
-    if (!cin) continue;
-    const bf16* base = p.ys + (int64_t)tk * ks * p.ldy + c;
-    float acc[VEC];
-#pragma unroll
-    for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-    constexpr int B = 9;  // slot rows in flight before a batch's additions
-    for (int j0 = 0; j0 < ks; j0 += B) {
-      uint32_t v[B][VEC / 2];
-#pragma unroll
-      for (int i = 0; i < B; ++i) {
-        const int j = j0 + i;
-        if (j < ks && (ok >> j & 1u)) {
-          const bf16* rp = base + (int64_t)j * p.ldy;
-          if constexpr (VEC == 4) {
-            const uint2 q = __ldcg(reinterpret_cast<const uint2*>(rp));
-            v[i][0] = q.x;
-            v[i][1] = q.y;
-          } else {
-            const uint4 q = __ldcg(reinterpret_cast<const uint4*>(rp));
-            v[i][0] = q.x;
-            v[i][1] = q.y;
-            v[i][2] = q.z;
-            v[i][3] = q.w;
-          }
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < B; ++i) {
-        const int j = j0 + i;
-        if (j < ks && (ok >> j & 1u)) {
-#pragma unroll
-          for (int e = 0; e < VEC / 2; ++e) {
-            acc[2 * e] += __uint_as_float(v[i][e] << 16);
-            acc[2 * e + 1] += __uint_as_float(v[i][e] & 0xffff0000u);
-          }
-        }
-      }
-    }
-    bf16* yp = p.y + (int64_t)tk * p.ldy + c;  // y [T, d] has the slot rows' row length
-    if constexpr (VEC == 4) {
-      *reinterpret_cast<uint2*>(yp) = make_uint2(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]));
-    } else {
-      *reinterpret_cast<uint4*>(yp) = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
-                                                 pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
-    }
   }
 }
 
@@ -940,12 +836,6 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(tempty + acc);
-      if constexpr (EPI == kTcSlotStore) {
-        // the slot sum reads global memory only: it runs after the accumulator
-        // has gone back to the MMA warp, alongside the next tile's MMAs
-        constexpr int CPW = (BN / 32) / EG;
-        if (p.y != nullptr) slot_sum_fused<CPW>(p, t, row, t.n0 + eg * CPW * 32, lane);
-      }
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;

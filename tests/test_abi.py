@@ -137,15 +137,13 @@ def test_forward_plan_on_the_host():
     # the bench workloads' plans (host only: no device needed)
     plan = lambda *a: moe.forward_plan(moe.Problem.make(*a))  # noqa: E731
     assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16") == \
-        {"expert_form": "rows", "router_selects": True, "gathered": True, "slot_sum_in_down": True}
+        {"expert_form": "rows", "router_selects": True, "gathered": True}
     assert plan(8192, 8192, 512, 10, 2048, 2048, "bf16", "bf16") == \
-        {"expert_form": "rows", "router_selects": False, "gathered": False,
-         "slot_sum_in_down": True}                                              # 512 experts; x > 32 MiB
+        {"expert_form": "rows", "router_selects": False, "gathered": False}      # 512 experts; x > 32 MiB
     assert plan(64, 8192, 512, 10, 2048, 2048, "bf16", "bf16")["expert_form"] == "weight_rows"
-    fp8 = plan(2048, 8192, 512, 10, 2048, 2048, "bf16", "fp8")
-    assert fp8["expert_form"] == "weight_rows" and not fp8["slot_sum_in_down"]
+    assert plan(2048, 8192, 512, 10, 2048, 2048, "bf16", "fp8")["expert_form"] == "weight_rows"
     assert plan(32, 128, 16, 2, 64, 64, "f32", "f32") == \
-        {"expert_form": "simt", "router_selects": False, "gathered": False, "slot_sum_in_down": False}
+        {"expert_form": "simt", "router_selects": False, "gathered": False}
     # the router selects in its epilogue from 16 token tiles on; the gather stops above 32 MiB of x
     assert not plan(1920, 256, 64, 4, 128, 128, "bf16", "bf16")["router_selects"]
     assert plan(1921, 256, 64, 4, 128, 128, "bf16", "bf16")["router_selects"]
@@ -154,14 +152,13 @@ def test_forward_plan_on_the_host():
     # the path setting moves the form
     try:
         moe.set_path(4)
-        pair = plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16")
-        assert pair["expert_form"] == "cta_pairs" and not pair["slot_sum_in_down"]
+        assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16")["expert_form"] == "cta_pairs"
         moe.set_path(1)
         assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16") == \
-            {"expert_form": "simt", "router_selects": False, "gathered": False, "slot_sum_in_down": False}
+            {"expert_form": "simt", "router_selects": False, "gathered": False}
     finally:
         moe.set_path(0)
-    assert moe.lib().moe_forward_plan(ctypes.byref(P(T=-1)), None, None, None, None) == 1
+    assert moe.lib().moe_forward_plan(ctypes.byref(P(T=-1)), None, None, None) == 1
 
 
 def _c_kind(decl):

@@ -55,8 +55,8 @@ FORWARD_CASES = {
     # the last 256-row weight block of the down projection outside d
     "bf16_long_groups": (700, 512, 6, 2, 256, 256, "bf16", "bf16", None),
     "bf16_long_ragged": (700, 384, 5, 2, 320, 192, "bf16", "bf16", None),
-    # d = 136: the down GEMM's last 128-column span holds 8 columns, and the
-    # span after it none (the fused slot sum counts and sums only real ones)
+    # d = 136: the down GEMM's last 256-column tile holds 136 columns, and
+    # the last epilogue warp's 128-column span 8 of them
     "bf16_d136": (300, 136, 10, 3, 128, 64, "bf16", "bf16", None),
     # T*k >= 2048*E: the automatic choice takes the CTA-pair GEMMs
     "bf16_auto_pair": (2048, 256, 2, 2, 256, 128, "bf16", "bf16", None),
