@@ -434,7 +434,9 @@ def time_steps(moe, layer, x, y, K, W, flush, world, dev, clocks=None):
     per = {}
     for name, ms in prof:
         per.setdefault(name, []).append(ms)
-    kern = {n: statistics.mean(v) for n, v in per.items()}
+    # per step: a stage may run as more than one launch (the split form runs
+    # each projection as a pair-tile and a weight-row launch)
+    kern = {n: sum(v) / K for n, v in per.items()}
     return statistics.mean(a.elapsed_time(b) for a, b in ev), kern, launches_per_step, clk
 
 
@@ -524,6 +526,7 @@ def run_ours(args):
     cfg = dict(moe_inputs.CONFIGS[args.config])
     inp = moe_inputs.make_config(args.config, seed=0, device=dev, x_seed=rank)
     T = inp.T
+    moe.set_path(args.path)
     layer = moe.MoELayer.from_inputs(inp, max_tokens=T)
     x = inp.x
     y = torch.empty((T, inp.d), dtype=x.dtype, device=dev)
@@ -581,7 +584,7 @@ def run_ours(args):
                     "l2": "no flush between steps; the step reads %.1f GB (tokens, result, weights) against "
                           "126 MB of L2" % (resident / 1e9)},
             "gpu_launches": launches_per_step * K, "launches_per_step": launches_per_step,
-            "kernel_ms": kern, "clocks": clk, "impl": "ours",
+            "kernel_ms": kern, "expert_form": forward_plan(cfg, T)["expert_form"], "clocks": clk, "impl": "ours",
         }
         if regimes:
             line["regimes"] = regimes
@@ -691,6 +694,9 @@ def arg_parser():
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     import moe_inputs
     ap.add_argument("--config", choices=sorted(moe_inputs.CONFIGS), default=DEFAULT_CONFIG)
+    ap.add_argument("--path", type=int, default=0,
+                    help="expert-GEMM form (moe_set_path): 0 automatic, 2 row-tiled, 3 weight-row, 4 CTA pairs, "
+                         "5 split")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-companion", action="store_true",
                     help="do not also time the workload that shares this one's weights (decode beside prefill)")

@@ -242,7 +242,8 @@ MOE_API moe_status moe_router_topk_static(const moe_problem* p, const void* x, c
 /* What moe_layer_forward / moe_block_forward launch for problem p under the
  * current moe_set_path, decided on the host (no CUDA call, no device needed):
  * expert_form: 0 SIMT kernels, 1 row-tiled tensor-core GEMMs, 2 weight-row
- * (swap-AB) GEMMs, 3 row-tiled GEMMs on CTA pairs; router_selects: 1 when the
+ * (swap-AB) GEMMs, 3 row-tiled GEMMs on CTA pairs, 4 split (CTA pairs for the
+ * groups of 256 rows or more, weight-row GEMMs for the others); router_selects: 1 when the
  * router's GEMM selects the top k in its epilogue (bf16, E <= 256, at least
  * 16 tiles of 128 tokens), 0 for the split-K GEMM + top-k kernel or the SIMT
  * router; gathered: 1 when the gate/up GEMM reads its rows straight from x.
@@ -256,13 +257,19 @@ MOE_API moe_status moe_forward_plan(const moe_problem* p, int32_t* expert_form, 
  * 0 = automatic (tensor-core kernels where the types allow; for the expert
  *     GEMMs the weight-row form when T*k <= 64*E, i.e. when an expert sees at
  *     most one 64-token chunk on average, the form of 4 when bf16 experts
- *     average 2048 rows or more (T*k >= 2048*E), else the row-tiled form);
+ *     average 2048 rows or more (T*k >= 2048*E), the form of 5 when they
+ *     average 144 rows or more, else the row-tiled form);
  * 1 = SIMT CUDA kernels only (fp32 FMA; the path of fp32 problems);
  * 2 = tensor-core kernels required, row-tiled expert GEMMs;
  * 3 = tensor-core kernels required, weight-row expert GEMMs;
  * 4 = tensor-core kernels required, row-tiled expert GEMMs on 2-CTA clusters
- *     (256-row tiles, tcgen05 pair MMAs; E4M3 weights take the form of 2).
- * 2, 3 and 4 return MOE_ERR_UNSUPPORTED when the types do not allow them. */
+ *     (256-row tiles, tcgen05 pair MMAs; E4M3 weights take the form of 2);
+ * 5 = tensor-core kernels required, split expert GEMMs: the groups of 256
+ *     rows or more as in 4, the others as in 3, one launch each per
+ *     projection (E4M3 weights take the form of 2).  Automatic for bf16
+ *     weights when experts average 144 to 2047 rows (a large batch, where
+ *     skewed routing leaves some experts thousands of rows and many a few).
+ * 2 to 5 return MOE_ERR_UNSUPPORTED when the types do not allow them. */
 MOE_API moe_status moe_set_path(int path);
 
 /* Synchronously read and clear the device status word of the current device

@@ -213,7 +213,9 @@ def check_problem(prob):
 
 def set_path(path):
     """0 automatic, 1 SIMT kernels only, 2 row-tiled tensor-core expert GEMMs,
-    3 weight-row tensor-core expert GEMMs, 4 row-tiled on 2-CTA clusters."""
+    3 weight-row tensor-core expert GEMMs, 4 row-tiled on 2-CTA clusters,
+    5 split: groups of 256 rows or more on 2-CTA clusters, the others in
+    weight-row form."""
     _check(lib().moe_set_path(int(path)))
 
 
@@ -421,7 +423,7 @@ def rmsnorm(prob, x, norm_weight, eps=1e-6, out=None, stream=None):
     return out
 
 
-EXPERT_FORMS = ("simt", "rows", "weight_rows", "cta_pairs")
+EXPERT_FORMS = ("simt", "rows", "weight_rows", "cta_pairs", "split")
 
 
 def forward_plan(prob):

@@ -355,9 +355,17 @@ static moe_status choose(bool tc_possible, bool* use_tc) {
 // weights) when experts average kPairRowsPerExpert rows or more, where its
 // 256-row tiles waste little on group tails (measured: 12-15 % faster at 4096
 // rows per expert, even at 1024, slower on prefill-sized Zipf-skewed groups);
+// between, when experts average kSplitAvgRows rows or more (bf16 weights),
+// the split form: the groups of kSplitRows rows or more on CTA pairs, the
+// others in weight-row form, two launches per projection (a large batch whose
+// routing is skewed gives a few experts thousands of rows and many experts a
+// handful: the first want the pair tiles' operand economy, the second would
+// spend a 128-row tile's MMAs on a few rows while their weights stream);
 // else the row-tiled form.
-enum { kFormSimt = 0, kFormRows = 1, kFormSwap = 2, kFormPair = 3 };
+enum { kFormSimt = 0, kFormRows = 1, kFormSwap = 2, kFormPair = 3, kFormSplit = 4 };
 constexpr int kPairRowsPerExpert = 2048;
+constexpr int kSplitAvgRows = 144;
+constexpr int kSplitRows = 256;
 static moe_status choose_form(const moe_problem& p, int* form) {
   bool tc;
   moe_status s = choose(tc_shapes(p), &tc);
@@ -366,8 +374,10 @@ static moe_status choose_form(const moe_problem& p, int* form) {
   else if (g_path == 2) *form = kFormRows;
   else if (g_path == 3) *form = kFormSwap;
   else if (g_path == 4) *form = p.w_dtype == MOE_BF16 ? kFormPair : kFormRows;
+  else if (g_path == 5) *form = p.w_dtype == MOE_BF16 ? kFormSplit : kFormRows;
   else if (p.T * (int64_t)p.k <= (int64_t)kNCH * p.E) *form = kFormSwap;
   else if (p.w_dtype == MOE_BF16 && p.T * (int64_t)p.k >= (int64_t)kPairRowsPerExpert * p.E) *form = kFormPair;
+  else if (p.w_dtype == MOE_BF16 && p.T * (int64_t)p.k >= (int64_t)kSplitAvgRows * p.E) *form = kFormSplit;
   else *form = kFormRows;
   return MOE_OK;
 }
@@ -475,9 +485,9 @@ static Layout layout(const moe_problem& p, bool forward) {
 }
 
 // ============================================================== launch pieces
-static Schedule sched_simt(int n_r, int n_s) { return Schedule{64, 64, n_r, n_s, 0, 0}; }
+static Schedule sched_simt(int n_r, int n_s) { return Schedule{64, 64, n_r, n_s, 0, 0, 0, 0}; }
 static Schedule sched_tc(int bn, int n_r, int n_s, int small_rows = 0) {
-  return Schedule{kBM, bn, n_r, n_s, 0, small_rows};
+  return Schedule{kBM, bn, n_r, n_s, 0, small_rows, 0, 0};
 }
 // The row-tiled bf16 GEMMs (tiles claimed in order) spread the tiles of
 // groups with one row tile among the others; the E4M3 form (tiles dealt in a
@@ -1000,6 +1010,14 @@ static moe_status expert_gemms(const moe_problem& p, int form, const void* xp, c
   }
   if (form == kFormRows) return tc_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, g);
   if (form == kFormPair) return pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
+  if (form == kFormSplit) {
+    // the large groups' tiles are counted in pre_a / pre_b, the others' in
+    // the second prefix of each (pre + E + 3): each kernel walks its own list
+    // and writes its own rows of H and of the slot rows
+    moe_status s = pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
+    if (s != MOE_OK) return s;
+    return swap_gemms_t<false>(p, xp, offs, w, pre_a + p.E + 3, pre_b + p.E + 3, H, o, st, dev);
+  }
   if (p.act_dtype == MOE_F32) return simt_gemms<float, float>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
   if (p.w_dtype == MOE_BF16) return simt_gemms<bf16, bf16>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
   return simt_gemms<bf16, uint8_t>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
@@ -1010,11 +1028,14 @@ static void schedules(const moe_problem& p, int form, Schedule* sa, Schedule* sb
     *sa = sched_tc(128, p.I, p.I_s, small_rows_of(p, form));
     *sb = sched_tc(256, p.d, p.d, small_rows_of(p, form));
   } else if (form == kFormPair) {  // 256-row tiles of CTA pairs
-    *sa = Schedule{kPairBM, 128, p.I, p.I_s, 0, 0};
-    *sb = Schedule{kPairBM, 256, p.d, p.d, 0, 0};
+    *sa = Schedule{kPairBM, 128, p.I, p.I_s, 0, 0, 0, 0};
+    *sb = Schedule{kPairBM, 256, p.d, p.d, 0, 0, 0, 0};
   } else if (form == kFormSwap) {  // (token chunk, 128 weight rows) tiles
-    *sa = Schedule{kNCH, 128, p.I, p.I_s, 0, 0};
-    *sb = Schedule{kNCH, 128, p.d, p.d, 0, 0};
+    *sa = Schedule{kNCH, 128, p.I, p.I_s, 0, 0, 0, 0};
+    *sb = Schedule{kNCH, 128, p.d, p.d, 0, 0, 0, 0};
+  } else if (form == kFormSplit) {  // pair tiles for the large groups, weight-row tiles for the rest
+    *sa = Schedule{kPairBM, 128, p.I, p.I_s, 0, kSplitRows - 1, kNCH, 128};
+    *sb = Schedule{kPairBM, 256, p.d, p.d, 0, kSplitRows - 1, kNCH, 128};
   } else {
     *sa = sched_simt(p.I, p.I_s);
     *sb = sched_simt(p.d, p.d);
@@ -1043,7 +1064,7 @@ size_t moe_workspace_size(const moe_problem* p) { return check(p) == MOE_OK ? la
 size_t moe_stage_workspace_size(const moe_problem* p) { return check(p) == MOE_OK ? layout(*p, false).total : 0; }
 
 moe_status moe_set_path(int path) {
-  if (path < 0 || path > 4) return fail(MOE_ERR_INVALID_ARG, "path %d is not 0, 1, 2, 3 or 4", path);
+  if (path < 0 || path > 5) return fail(MOE_ERR_INVALID_ARG, "path %d is not 0, 1, 2, 3, 4 or 5", path);
   g_path = path;
   return MOE_OK;
 }

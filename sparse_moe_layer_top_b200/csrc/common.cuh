@@ -65,11 +65,14 @@ __device__ __forceinline__ int find_group(const int32_t* prefix, int ngroups, in
 // weight-row (swap) kernels whose N covers every row of a group.
 // Tiles of a grouped GEMM: ceil(rows / bm) x ceil(n / bn) per group (one
 // row tile per group when swap).  With small_rows > 0 the groups of at most
-// small_rows rows (one row tile: each of their tiles streams its weight block
-// from HBM for few rows) are counted in a prefix of their own, so that the
-// GEMM can spread their tiles evenly among the others (see decode_tile).
+// small_rows rows are counted in a prefix of their own, with tiles of
+// bm_small x bn_small (0: bm, bn).  Two uses: the row-tiled GEMM spreads the
+// tiles of its one-row-tile groups (each streams its weight block from HBM for
+// few rows) evenly among the others (see decode_tile); the split form runs
+// the large groups on CTA pairs and the small ones in weight-row form, each
+// kernel walking its own prefix.
 struct Schedule {
-  int bm, bn, n_routed, n_shared, swap, small_rows;
+  int bm, bn, n_routed, n_shared, swap, small_rows, bm_small, bn_small;
 };
 
 __host__ __device__ __forceinline__ bool sched_small(const Schedule& s, int rows) {
@@ -79,8 +82,11 @@ __host__ __device__ __forceinline__ bool sched_small(const Schedule& s, int rows
 __device__ __forceinline__ int sched_tiles(const Schedule& s, int g, int E, int rows) {
   int n = g < E ? s.n_routed : s.n_shared;
   if (rows <= 0 || n <= 0) return 0;
-  int mt = s.swap ? 1 : (int)cdiv(rows, s.bm);
-  return mt * (int)cdiv(n, s.bn);
+  const bool small = sched_small(s, rows);
+  const int bm = small && s.bm_small > 0 ? s.bm_small : s.bm;
+  const int bn = small && s.bn_small > 0 ? s.bn_small : s.bn;
+  int mt = s.swap ? 1 : (int)cdiv(rows, bm);
+  return mt * (int)cdiv(n, bn);
 }
 
 }  // namespace moe

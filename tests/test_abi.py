@@ -89,7 +89,8 @@ def test_host_rejects_before_any_launch():
 
 
 def test_set_path_validates():
-    assert moe.lib().moe_set_path(5) == 1
+    assert moe.lib().moe_set_path(6) == 1
+    assert moe.lib().moe_set_path(5) == 0
     assert moe.lib().moe_set_path(-1) == 1
     assert moe.lib().moe_set_path(0) == 0
 
@@ -139,7 +140,12 @@ def test_forward_plan_on_the_host():
     assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16") == \
         {"expert_form": "rows", "router_selects": True, "gathered": True}
     assert plan(8192, 8192, 512, 10, 2048, 2048, "bf16", "bf16") == \
-        {"expert_form": "rows", "router_selects": False, "gathered": False}      # 512 experts; x > 32 MiB
+        {"expert_form": "split", "router_selects": False, "gathered": False}     # 512 experts; 160 rows each
+    # the split form from 144 rows per expert on average, the pair form from 2048
+    assert plan(7372, 8192, 512, 10, 2048, 2048, "bf16", "bf16")["expert_form"] == "rows"
+    assert plan(7373, 8192, 512, 10, 2048, 2048, "bf16", "bf16")["expert_form"] == "split"
+    assert plan(7373, 8192, 512, 10, 2048, 2048, "bf16", "fp8")["expert_form"] == "rows"
+    assert plan(4096, 256, 2, 1, 256, 256, "bf16", "bf16")["expert_form"] == "cta_pairs"
     assert plan(64, 8192, 512, 10, 2048, 2048, "bf16", "bf16")["expert_form"] == "weight_rows"
     assert plan(2048, 8192, 512, 10, 2048, 2048, "bf16", "fp8")["expert_form"] == "weight_rows"
     assert plan(32, 128, 16, 2, 64, 64, "f32", "f32") == \
@@ -147,12 +153,15 @@ def test_forward_plan_on_the_host():
     # the router selects in its epilogue from 16 token tiles on; the gather stops above 32 MiB of x
     assert not plan(1920, 256, 64, 4, 128, 128, "bf16", "bf16")["router_selects"]
     assert plan(1921, 256, 64, 4, 128, 128, "bf16", "bf16")["router_selects"]
-    assert plan(2048, 8192, 64, 8, 256, 256, "bf16", "bf16")["gathered"]        # exactly 32 MiB
-    assert not plan(2049, 8192, 64, 8, 256, 256, "bf16", "bf16")["gathered"]
+    assert plan(2048, 8192, 128, 8, 256, 256, "bf16", "bf16")["gathered"]       # exactly 32 MiB
+    assert not plan(2049, 8192, 128, 8, 256, 256, "bf16", "bf16")["gathered"]
     # the path setting moves the form
     try:
         moe.set_path(4)
         assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16")["expert_form"] == "cta_pairs"
+        moe.set_path(5)
+        assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16")["expert_form"] == "split"
+        assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "fp8")["expert_form"] == "rows"
         moe.set_path(1)
         assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16") == \
             {"expert_form": "simt", "router_selects": False, "gathered": False}

@@ -1,8 +1,10 @@
 """Failure detection on the device: a pipeline wait that runs out.
 
-Every wait in the kernels is bounded.  Here the bound is set far below any
-real wait's length (moe_set_wait_limit), so the kernels' waits give up on
-purpose -- no fault, no hang: each waiter records the timeout in the device
+Every wait in the kernels is bounded.  Here the bound is set far below the
+length of the kernels' longer waits (moe_set_wait_limit), so those waits give
+up on purpose -- no fault, no hang (a wait that one poll of the barrier
+outlasts is not checked against the bound, so the problems are sized for
+waits of many microseconds): each waiter records the timeout in the device
 status word, raises its CTA's abort flag, and the kernel drains the copies
 and tensor-core work it issued (with the default bound), frees its tensor
 memory and returns.  The test checks that the call comes back, that
@@ -71,8 +73,10 @@ def test_expert_gemm_waits_that_run_out_report_timeout_and_the_device_stays_usab
 
 
 def test_router_waits_that_run_out_report_timeout_and_the_device_stays_usable(moe):
-    # E <= 256 with 18 row tiles: the router GEMM selects the top k in its epilogue
-    inp = moe_inputs.make_inputs(2304, 256, 100, 6, 128, 128, act="bf16", w="bf16", bias="zipf", seed=3)
+    # E <= 256 with 18 row tiles: the router GEMM selects the top k in its
+    # epilogue; d = 8192 makes each tile's main loop (128 K-blocks) far longer
+    # than one poll of a wait, so the epilogue's wait for the accumulator runs out
+    inp = moe_inputs.make_inputs(2304, 8192, 100, 6, 128, 128, act="bf16", w="bf16", bias="zipf", seed=3)
     g = to_device(inp, "cuda")
     prob = moe.Problem.make(inp.T, inp.d, inp.E, inp.k, inp.I, inp.I_s, "bf16", "bf16")
     ids_ok, w_ok = moe.router_topk(prob, g.x, g.w_r, g.bias)
