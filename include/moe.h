@@ -290,6 +290,19 @@ MOE_API moe_status moe_device_status(int32_t* detail);
  * that copy fails. */
 MOE_API moe_status moe_set_wait_limit(int64_t cycles);
 
+/* 1 in the bounds-checking build of the library (libmoe_checks.so, compiled
+ * with -DMOE_CHECKS), 0 otherwise.  That build checks, on the device, the
+ * indices the kernels compute or read before they address memory with them:
+ * the row a (token, slot) pair is dispatched to and the rows the dispatch
+ * copies into, the token row a gathering GEMM reads, the (token, slot) row a
+ * down GEMM's epilogue stores, and the dispatched rows moe_combine reads for
+ * the caller's pos (and the shared row offs[E] + t).  An index out of range
+ * skips that access and records MOE_ERR_DEVICE_CHECK with code
+ * 0x08000000 | site (1 dispatched row, 2 copied row, 3 gathered token row,
+ * 4 slot row, 5 combined row) in the device status word.  The normal build
+ * compiles these checks away. */
+MOE_API int moe_bounds_checked(void);
+
 /* Number of kernels the last successful call on this thread launched. */
 MOE_API int moe_last_launch_count(void);
 

@@ -27,12 +27,15 @@ import torch
 __all__ = ["MoEError", "Problem", "BlockOptions", "router_topk", "permute", "expert_ffn", "combine", "layer_forward",
            "block_forward", "rmsnorm", "ep_expand_ids", "forward_plan",
            "workspace_size", "stage_workspace_size", "set_path", "set_wait_limit", "device_status",
-           "last_launch_count",
+           "last_launch_count", "bounds_checked",
            "profile_enable", "profile_read",
            "MoELayer", "lib_path", "F32", "BF16", "FP8_E4M3_B128"]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-lib_path = os.path.join(HERE, "libmoe.so")
+# MOE_CHECKS=1 loads the bounds-checking build (python -m
+# sparse_moe_layer_top_b200.build --checks), whose kernels check their
+# computed indices on the device (moe_bounds_checked in include/moe.h)
+lib_path = os.path.join(HERE, "libmoe_checks.so" if os.environ.get("MOE_CHECKS") == "1" else "libmoe.so")
 
 F32, BF16, FP8_E4M3_B128 = 0, 1, 2
 _STATUS = {0: "MOE_OK", 1: "MOE_ERR_INVALID_ARG", 2: "MOE_ERR_UNSUPPORTED", 3: "MOE_ERR_ALIGNMENT",
@@ -41,7 +44,7 @@ EXPORTS = ("moe_check_problem", "moe_workspace_size", "moe_stage_workspace_size"
            "moe_permute", "moe_expert_ffn", "moe_combine", "moe_layer_forward", "moe_set_path",
            "moe_device_status", "moe_last_launch_count", "moe_profile_enable", "moe_profile_read",
            "moe_last_error_string", "moe_router_topk_static", "moe_block_forward", "moe_rmsnorm",
-           "moe_ep_expand_ids", "moe_forward_plan", "moe_set_wait_limit")
+           "moe_ep_expand_ids", "moe_forward_plan", "moe_set_wait_limit", "moe_bounds_checked")
 
 
 class MoEError(RuntimeError):
@@ -97,6 +100,7 @@ def lib():
         L.moe_set_wait_limit.argtypes = [ctypes.c_int64]
         L.moe_device_status.argtypes = [ctypes.POINTER(ctypes.c_int32)]
         L.moe_last_launch_count.restype = ctypes.c_int
+        L.moe_bounds_checked.restype = ctypes.c_int
         L.moe_profile_enable.argtypes = [ctypes.c_int]
         L.moe_profile_enable.restype = ctypes.c_int
         L.moe_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_float),
@@ -231,6 +235,11 @@ def device_status():
     d = ctypes.c_int32(0)
     s = lib().moe_device_status(ctypes.byref(d))
     return s, d.value
+
+
+def bounds_checked():
+    """True when the loaded library is the bounds-checking build."""
+    return bool(lib().moe_bounds_checked())
 
 
 def last_launch_count():

@@ -622,7 +622,7 @@ static moe_status launch_dispatch(const moe_problem& p, const int32_t* ids, cons
   PROF_BEGIN("dispatch", st);
   CUDA_TRY(launch(k_dispatch, nch * kSubBlocks, kScatterWarps * 32, 0, st, ids, tw, p.T, p.k, p.E, counts, nch,
                   p.I_s > 0, offs, sa, pre_a, sb, pre_b, row_tok, row_w, pos, row_dst, shared_gate,
-                  (const uint4*)x, vec, (uint4*)xp));
+                  (const uint4*)x, vec, (uint4*)xp, dev->status));
   LAUNCH_CHECK("dispatch", st);
   return MOE_OK;
 }
@@ -713,6 +713,8 @@ static moe_status simt_gemms(const moe_problem& p, const void* xp, const int32_t
   b.b2 = b.b1;
   if (o.ys) {
     b.ys = (TA*)o.ys;
+    b.ys_rows = p.T * (p.k + 1);
+    b.status = dev->status;
     b.ldy = p.d;
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
@@ -774,6 +776,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   PROF_BEGIN("gemm_tc_swiglu", st);
   if (!FP8 && g.x) {
     a.gx = (const bf16*)g.x;
+    a.gx_rows = p.T;
     a.row_tok = g.row_tok;
     a.ldx = p.d;
     CUDA_TRY(launch(k_gemm_tc<128, true, 4, kTcSwiGLU, false, true>, dev->sms, Gemm1GCfg::THREADS,
@@ -807,6 +810,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   if (small_rows_of(p, kFormRows) > 0) b.prefix_small = pre_b + p.E + 3;
   if (o.ys) {
     b.ys = (bf16*)o.ys;
+    b.ys_rows = p.T * (p.k + 1);
     b.ldy = p.d;
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
@@ -832,10 +836,15 @@ static moe_status tc_gemms(const moe_problem& p, const void* xp, const int32_t* 
   return tc_gemms_t<false>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, g);
 }
 
+// Which projections a launcher enqueues: the split form runs both gate/up
+// launches before either down launch, since a down GEMM stores its slot rows
+// into the buffer the other gate/up GEMM reads its dispatched rows from.
+enum { kPhaseGateUp = 1, kPhaseDown = 2, kPhaseBoth = 3 };
+
 template <bool FP8>
 static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
                                int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
-                               DeviceInfo* dev) {
+                               DeviceInfo* dev, int phases = kPhaseBoth) {
   using C1 = SwapCfg<true>;
   using C2 = SwapCfg<false>;
   const int64_t Rp = rows_total(p), ldh = ldh_of(p);
@@ -845,40 +854,43 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
   moe_status s;
   CUtensorMap xR, xS, bR, bS, cR, cS;
   // gate/up + SwiGLU: weights [E, I, d] are the M operand, token rows the N operand
-  if ((s = map2d(&xR, xp, p.d, Rp, p.d, kNCH)) != MOE_OK) return s;
-  if ((s = map3d(&bR, w.wg, p.d, p.I, p.E, 128, FP8, FP8)) != MOE_OK) return s;
-  if ((s = map3d(&cR, w.wu, p.d, p.I, p.E, 128, FP8, FP8)) != MOE_OK) return s;
-  bS = bR;
-  cS = cR;
-  if (sh) {
-    if ((s = map2d(&bS, w.sg, p.d, p.I_s, p.d, 128, FP8, FP8)) != MOE_OK) return s;
-    if ((s = map2d(&cS, w.su, p.d, p.I_s, p.d, 128, FP8, FP8)) != MOE_OK) return s;
+  if (phases & kPhaseGateUp) {
+    if ((s = map2d(&xR, xp, p.d, Rp, p.d, kNCH)) != MOE_OK) return s;
+    if ((s = map3d(&bR, w.wg, p.d, p.I, p.E, 128, FP8, FP8)) != MOE_OK) return s;
+    if ((s = map3d(&cR, w.wu, p.d, p.I, p.E, 128, FP8, FP8)) != MOE_OK) return s;
+    bS = bR;
+    cS = cR;
+    if (sh) {
+      if ((s = map2d(&bS, w.sg, p.d, p.I_s, p.d, 128, FP8, FP8)) != MOE_OK) return s;
+      if ((s = map2d(&cS, w.su, p.d, p.I_s, p.d, 128, FP8, FP8)) != MOE_OK) return s;
+    }
+    TcGemmArgs a{};
+    a.offs = offs;
+    a.prefix = pre_a;
+    a.E = p.E;
+    a.rows_cap = Rp;
+    a.single_rows = -1;
+    a.N_r = p.I;
+    a.N_s = p.I_s;
+    a.K_r = p.d;
+    a.K_s = p.d;
+    a.H = (bf16*)H;
+    a.ldh = ldh;
+    a.sc_b_r = sp[0];
+    a.sc_b_s = sp[3];
+    a.sc_c_r = sp[1];
+    a.sc_c_s = sp[4];
+    a.status = dev->status;
+    PROF_BEGIN("gemm_tc_swiglu", st);
+    if (FP8)
+      CUDA_TRY(launch(k_gemm_swap8<true, kTcSwiGLU>,
+                      dev->sms, Swap8Cfg<true>::THREADS, Swap8Cfg<true>::SMEM_BYTES, st, xR, xR, bR, bS, cR, cS, a));
+    else
+      CUDA_TRY(launch(k_gemm_swap<true, kTcSwiGLU>,
+                      dev->sms, C1::THREADS, C1::SMEM_BYTES, st, xR, xR, bR, bS, cR, cS, a));
+    LAUNCH_CHECK("gemm_tc_swiglu", st);
   }
-  TcGemmArgs a{};
-  a.offs = offs;
-  a.prefix = pre_a;
-  a.E = p.E;
-  a.rows_cap = Rp;
-  a.single_rows = -1;
-  a.N_r = p.I;
-  a.N_s = p.I_s;
-  a.K_r = p.d;
-  a.K_s = p.d;
-  a.H = (bf16*)H;
-  a.ldh = ldh;
-  a.sc_b_r = sp[0];
-  a.sc_b_s = sp[3];
-  a.sc_c_r = sp[1];
-  a.sc_c_s = sp[4];
-  a.status = dev->status;
-  PROF_BEGIN("gemm_tc_swiglu", st);
-  if (FP8)
-    CUDA_TRY(launch(k_gemm_swap8<true, kTcSwiGLU>,
-                    dev->sms, Swap8Cfg<true>::THREADS, Swap8Cfg<true>::SMEM_BYTES, st, xR, xR, bR, bS, cR, cS, a));
-  else
-    CUDA_TRY(launch(k_gemm_swap<true, kTcSwiGLU>,
-                    dev->sms, C1::THREADS, C1::SMEM_BYTES, st, xR, xR, bR, bS, cR, cS, a));
-  LAUNCH_CHECK("gemm_tc_swiglu", st);
+  if (!(phases & kPhaseDown)) return MOE_OK;
   // down: W_down [E, d, I] is the M operand, H rows the N operand
   if ((s = map2d(&xR, H, p.I, Rp, ldh, kNCH)) != MOE_OK) return s;
   xS = xR;
@@ -901,6 +913,7 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
   b.status = dev->status;
   if (o.ys) {
     b.ys = (bf16*)o.ys;
+    b.ys_rows = p.T * (p.k + 1);
     b.ldy = p.d;
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
@@ -931,38 +944,41 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
 // loading 128 activation rows and a 128-row half of the weight tile.
 static moe_status pair_gemms(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
                              int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
-                             DeviceInfo* dev) {
+                             DeviceInfo* dev, int phases = kPhaseBoth) {
   const int64_t Rp = rows_total(p), ldh = ldh_of(p);
   const bool sh = p.I_s > 0;
   moe_status s;
   CUtensorMap aR, aS, bR, bS, cR, cS;
   // gate/up + SwiGLU: rank 0 streams gate rows, rank 1 up rows
-  if ((s = map2d(&aR, xp, p.d, Rp, p.d, kBM)) != MOE_OK) return s;
-  if ((s = map3d(&bR, w.wg, p.d, p.I, p.E, 128)) != MOE_OK) return s;
-  if ((s = map3d(&cR, w.wu, p.d, p.I, p.E, 128)) != MOE_OK) return s;
-  bS = bR;
-  cS = cR;
-  if (sh) {
-    if ((s = map2d(&bS, w.sg, p.d, p.I_s, p.d, 128)) != MOE_OK) return s;
-    if ((s = map2d(&cS, w.su, p.d, p.I_s, p.d, 128)) != MOE_OK) return s;
+  if (phases & kPhaseGateUp) {
+    if ((s = map2d(&aR, xp, p.d, Rp, p.d, kBM)) != MOE_OK) return s;
+    if ((s = map3d(&bR, w.wg, p.d, p.I, p.E, 128)) != MOE_OK) return s;
+    if ((s = map3d(&cR, w.wu, p.d, p.I, p.E, 128)) != MOE_OK) return s;
+    bS = bR;
+    cS = cR;
+    if (sh) {
+      if ((s = map2d(&bS, w.sg, p.d, p.I_s, p.d, 128)) != MOE_OK) return s;
+      if ((s = map2d(&cS, w.su, p.d, p.I_s, p.d, 128)) != MOE_OK) return s;
+    }
+    TcGemmArgs a{};
+    a.offs = offs;
+    a.prefix = pre_a;
+    a.E = p.E;
+    a.rows_cap = Rp;
+    a.single_rows = -1;
+    a.N_r = p.I;
+    a.N_s = p.I_s;
+    a.K_r = p.d;
+    a.K_s = p.d;
+    a.H = (bf16*)H;
+    a.ldh = ldh;
+    a.status = dev->status;
+    PROF_BEGIN("gemm_tc_swiglu", st);
+    CUDA_TRY(launch_pair(k_gemm_pair<128, true, kPairStages, kTcSwiGLU>, dev->pair_ctas, Pair1Cfg::THREADS,
+                         Pair1Cfg::SMEM_BYTES, st, aR, aR, bR, bS, cR, cS, a));
+    LAUNCH_CHECK("gemm_tc_swiglu", st);
   }
-  TcGemmArgs a{};
-  a.offs = offs;
-  a.prefix = pre_a;
-  a.E = p.E;
-  a.rows_cap = Rp;
-  a.single_rows = -1;
-  a.N_r = p.I;
-  a.N_s = p.I_s;
-  a.K_r = p.d;
-  a.K_s = p.d;
-  a.H = (bf16*)H;
-  a.ldh = ldh;
-  a.status = dev->status;
-  PROF_BEGIN("gemm_tc_swiglu", st);
-  CUDA_TRY(launch_pair(k_gemm_pair<128, true, kPairStages, kTcSwiGLU>, dev->pair_ctas, Pair1Cfg::THREADS,
-                       Pair1Cfg::SMEM_BYTES, st, aR, aR, bR, bS, cR, cS, a));
-  LAUNCH_CHECK("gemm_tc_swiglu", st);
+  if (!(phases & kPhaseDown)) return MOE_OK;
   // down: the two 128-row halves of each 256-row weight block
   if ((s = map2d(&aR, H, p.I, Rp, ldh, kBM)) != MOE_OK) return s;
   aS = aR;
@@ -983,6 +999,7 @@ static moe_status pair_gemms(const moe_problem& p, const void* xp, const int32_t
   b.status = dev->status;
   if (o.ys) {
     b.ys = (bf16*)o.ys;
+    b.ys_rows = p.T * (p.k + 1);
     b.ldy = p.d;
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
@@ -1013,10 +1030,15 @@ static moe_status expert_gemms(const moe_problem& p, int form, const void* xp, c
   if (form == kFormSplit) {
     // the large groups' tiles are counted in pre_a / pre_b, the others' in
     // the second prefix of each (pre + E + 3): each kernel walks its own list
-    // and writes its own rows of H and of the slot rows
-    moe_status s = pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
-    if (s != MOE_OK) return s;
-    return swap_gemms_t<false>(p, xp, offs, w, pre_a + p.E + 3, pre_b + p.E + 3, H, o, st, dev);
+    // and writes its own rows of H and of the slot rows; both gate/up GEMMs
+    // read the dispatched rows before either down GEMM overwrites them
+    int32_t* sa = pre_a + p.E + 3;
+    int32_t* sb = pre_b + p.E + 3;
+    moe_status s;
+    if ((s = pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, kPhaseGateUp)) != MOE_OK) return s;
+    if ((s = swap_gemms_t<false>(p, xp, offs, w, sa, sb, H, o, st, dev, kPhaseGateUp)) != MOE_OK) return s;
+    if ((s = pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, kPhaseDown)) != MOE_OK) return s;
+    return swap_gemms_t<false>(p, xp, offs, w, sa, sb, H, o, st, dev, kPhaseDown);
   }
   if (p.act_dtype == MOE_F32) return simt_gemms<float, float>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
   if (p.w_dtype == MOE_BF16) return simt_gemms<bf16, bf16>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
@@ -1079,6 +1101,14 @@ moe_status moe_set_wait_limit(int64_t cycles) {
 }
 
 int moe_last_launch_count(void) { return g_launches; }
+
+int moe_bounds_checked(void) {
+#ifdef MOE_CHECKS
+  return 1;
+#else
+  return 0;
+#endif
+}
 
 moe_status moe_profile_enable(int on) {
   if (on < 0 || on > 2) return fail(MOE_ERR_INVALID_ARG, "profile mode %d is not 0, 1 or 2", on);
@@ -1242,10 +1272,10 @@ moe_status moe_combine(const moe_problem* p, const void* y_perm, const int32_t* 
   PROF_BEGIN("combine", st);
   if (p->act_dtype == MOE_F32)
     CUDA_TRY(launch(k_combine<float>, (unsigned)p->T, 256, 0, st, (const float*)y_perm, pos, topk_w, offs, p->E,
-                    p->k, p->d, p->T, (float*)y));
+                    p->k, p->d, p->T, (float*)y, rows_total(*p), dev->status));
   else
     CUDA_TRY(launch(k_combine<bf16>, (unsigned)p->T, 256, 0, st, (const bf16*)y_perm, pos, topk_w, offs, p->E,
-                    p->k, p->d, p->T, (bf16*)y));
+                    p->k, p->d, p->T, (bf16*)y, rows_total(*p), dev->status));
   LAUNCH_CHECK("combine", st);
   g_launches = g_launches_pending;
   return MOE_OK;

@@ -18,8 +18,39 @@ enum : unsigned {
   kStatusBadExpertId = 0x06000001u,  // a routing id outside [0, E)
   kStatusBadCount = 0x06000002u,     // expert parallelism: a negative or short row count
   kStatusTimeoutBase = 0x07000000u,  // | (kernel id << 8) | wait site
+  kStatusBoundsBase = 0x08000000u,   // bounds-checking build: | index site (kSite*)
 };
 enum : unsigned { kKernRouterTc = 1, kKernGemmTc = 2, kKernGemmSwap = 3 };
+
+// Index sites the bounds-checking build (-DMOE_CHECKS) verifies: the row a
+// pair is dispatched to, the rows the dispatch copies into, the token row a
+// gathering GEMM reads, the (token, slot) row a down-GEMM epilogue stores, and
+// the dispatched row moe_combine reads for a pair (a caller's input there).
+enum : unsigned {
+  kSiteDispatchRow = 1,
+  kSiteCopyRow = 2,
+  kSiteGatherToken = 3,
+  kSiteSlotRow = 4,
+  kSiteCombineRow = 5,
+};
+
+// True when 0 <= i < cap.  In the bounds-checking build an index outside that
+// range records kStatusBoundsBase | site in the device status word (the first
+// fault wins) and the caller skips the access; the normal build assumes the
+// index is in range and the check compiles away.
+__device__ __forceinline__ bool in_range(int64_t i, int64_t cap, unsigned* status, unsigned site) {
+#ifdef MOE_CHECKS
+  if (i >= 0 && i < cap) return true;
+  if (status) atomicCAS(status, 0u, kStatusBoundsBase | site);
+  return false;
+#else
+  (void)i;
+  (void)cap;
+  (void)status;
+  (void)site;
+  return true;
+#endif
+}
 
 // Programmatic dependent launch.  Each kernel calls pdl_begin() before it
 // touches what the previous kernel in the stream wrote (or overwrites what that

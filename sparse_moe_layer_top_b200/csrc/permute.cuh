@@ -133,7 +133,8 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
     const int32_t* __restrict__ counts, int nchunks, int has_shared, int32_t* __restrict__ offs, Schedule sa,
     int32_t* __restrict__ prefix_a, Schedule sb, int32_t* __restrict__ prefix_b, int32_t* __restrict__ row_tok,
     float* __restrict__ row_w, int32_t* __restrict__ pos, int32_t* __restrict__ row_dst,
-    const float* __restrict__ shared_gate, const uint4* __restrict__ x, int vec_per_row, uint4* __restrict__ xp) {
+    const float* __restrict__ shared_gate, const uint4* __restrict__ x, int vec_per_row, uint4* __restrict__ xp,
+    unsigned* status) {
   pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   __shared__ int32_t wb[kScatterWarps][kMaxE];
   __shared__ int32_t s_base[kMaxE];
@@ -240,13 +241,14 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
     const int64_t i = b + lane;
     const bool act = i < s1;
     const int e = act ? __ldg(ids + i) : -1;
-    const bool ok = act && (unsigned)e < (unsigned)E;
+    bool ok = act && (unsigned)e < (unsigned)E;
     const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
     int r = 0;
     if (ok) r = wb[warp][e] + __popc(peers & lt);
     __syncwarp();
     if (ok && (peers & lt) == 0) wb[warp][e] += __popc(peers);
     __syncwarp();
+    if (ok && !in_range(r, R, status, kSiteDispatchRow)) ok = false;  // (checking build) the pair is dropped
     if (ok) {
       const int64_t t = i / k;
       row_tok[r] = (int32_t)t;
@@ -290,6 +292,7 @@ __global__ void __launch_bounds__(kScatterWarps * 32) k_dispatch(
           if (!has_shared) break;
           r = R + t;
         }
+        if (!in_range(r, R + (has_shared ? T : 0), status, kSiteCopyRow)) continue;
         uint4* dst = xp + r * vec_per_row;
 #pragma unroll
         for (int u = 0; u < 4; ++u) {

@@ -36,6 +36,8 @@ struct SimtGemmArgs {
   int64_t ldh;
   TA* ys;                 // kEpiSlotStore: [T*(k+1), ldy], row_w-weighted, (token, slot) order
   int64_t ldy;
+  int64_t ys_rows;        // rows of ys (checked in the bounds-checking build)
+  unsigned* status;
   const int32_t* row_dst;
   const float* row_w;
   TA* out;                // kEpiStore: [rows, ldo]
@@ -124,7 +126,8 @@ __global__ void __launch_bounds__(256) k_gemm_simt(SimtGemmArgs<TA, TW> p) {
           from_f32(silu_f32(acc[i][j]) * acc2[i][j], p.H + r * p.ldh + n);
         } else if (EPI == kEpiSlotStore) {
           int64_t dr = __ldg(p.row_dst + r);
-          if (dr >= 0) from_f32(__ldg(p.row_w + r) * acc[i][j], p.ys + dr * p.ldy + n);
+          if (dr >= 0 && in_range(dr, p.ys_rows, p.status, kSiteSlotRow))
+            from_f32(__ldg(p.row_w + r) * acc[i][j], p.ys + dr * p.ldy + n);
         } else {
           from_f32(acc[i][j], p.out + r * p.ldo + n);
         }
@@ -139,16 +142,18 @@ __global__ void __launch_bounds__(256) k_gemm_simt(SimtGemmArgs<TA, TW> p) {
 template <typename TA>
 __global__ void __launch_bounds__(256) k_combine(const TA* __restrict__ yp, const int32_t* __restrict__ pos,
                                                  const float* __restrict__ tw, const int32_t* __restrict__ offs,
-                                                 int E, int k, int d, int64_t T, TA* __restrict__ y) {
+                                                 int E, int k, int d, int64_t T, TA* __restrict__ y,
+                                                 int64_t rows, unsigned* status) {
   pdl_begin();  // after the previous kernel in the stream (programmatic launch)
   const int64_t t = blockIdx.x;
   const int64_t rs = offs[E], re = offs[E + 1];
-  const bool shared = re > rs;
+  const bool shared = re > rs && in_range(rs + t, rows, status, kSiteCombineRow);
   for (int c = threadIdx.x; c < d; c += blockDim.x) {
     float acc = 0.f;
     for (int j = 0; j < k; ++j) {
       int r = __ldg(pos + t * k + j);
-      if (r >= 0) acc = fmaf(__ldg(tw + t * k + j), to_f32(yp[(int64_t)r * d + c]), acc);
+      if (r >= 0 && in_range(r, rows, status, kSiteCombineRow))
+        acc = fmaf(__ldg(tw + t * k + j), to_f32(yp[(int64_t)r * d + c]), acc);
     }
     if (shared) acc += to_f32(yp[(rs + t) * d + c]);
     from_f32(acc, y + t * d + c);

@@ -67,6 +67,7 @@ struct TcGemmArgs {
   int64_t ldh;
   bf16* ys;               // SlotStore output [T*(k+1), ldy]
   int64_t ldy;
+  int64_t ys_rows;        // SlotStore: rows of ys (checked in the bounds-checking build)
   const int32_t* row_dst; // SlotStore: destination row of each dispatched row
   const float* row_w;     // SlotStore: routing weight of each dispatched row
   bf16* out;              // Store output [rows, ldo]
@@ -97,6 +98,7 @@ struct TcGemmArgs {
   const bf16* gx;
   const int32_t* row_tok;
   int64_t ldx;
+  int64_t gx_rows;        // rows of the token matrix (checked in the bounds-checking build)
   // E4M3 weights: fp32 scales per 128 x 128 block, [E][N/128][K/128] routed,
   // [N/128][K/128] shared; B = gate (or the single operand), C = up
   const float *sc_b_r, *sc_b_s, *sc_c_r, *sc_c_s;
@@ -354,7 +356,8 @@ __device__ __forceinline__ void epilogue_rows(const TcGemmArgs& p, const TileInf
     } else if (EPI == kTcSlotStore) {
       const int64_t dr = __ldg(p.row_dst + grow);
       w = __ldg(p.row_w + grow);
-      if (dr >= 0) rowp = reinterpret_cast<char*>(p.ys + dr * p.ldy);
+      if (dr >= 0 && in_range(dr, p.ys_rows, p.status, kSiteSlotRow))
+        rowp = reinterpret_cast<char*>(p.ys + dr * p.ldy);
     } else {
       rowp = reinterpret_cast<char*>(p.out + grow * p.ldo);
     }
@@ -874,9 +877,11 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
         const int r = rb + RS * i;
         const int64_t grow = t.row0 + r;
         const bool in = t.m0 + r < t.rows && grow < p.rows_cap;
-        const int64_t tok = in ? (int64_t)__ldg(p.row_tok + grow) : 0;
+        int64_t tok = in ? (int64_t)__ldg(p.row_tok + grow) : 0;
+        const bool tin = !in || in_range(tok, p.gx_rows, p.status, kSiteGatherToken);
+        if (!tin) tok = 0;  // (checking build) the row reads zeros instead
         src[i] = p.gx + tok * p.ldx + ch * 8;
-        live |= (uint32_t)in << i;
+        live |= (uint32_t)(in && tin) << i;
       }
       const int K = t.g == p.E ? p.K_s : p.K_r;
       for (int kb = t.kb0; kb < t.kb1; ++kb) {

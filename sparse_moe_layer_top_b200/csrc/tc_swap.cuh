@@ -94,10 +94,12 @@ __device__ __forceinline__ void swap_epilogue(const TcGemmArgs& p, const int32_t
       if (t.c0 + lane < t.rows && ra < p.rows_cap) {
         dst_lo = __ldg(p.row_dst + ra);
         w_lo = __ldg(p.row_w + ra);
+        if (dst_lo >= 0 && !in_range(dst_lo, p.ys_rows, p.status, kSiteSlotRow)) dst_lo = -1;
       }
       if (t.c0 + 32 + lane < t.rows && rb < p.rows_cap) {
         dst_hi = __ldg(p.row_dst + rb);
         w_hi = __ldg(p.row_w + rb);
+        if (dst_hi >= 0 && !in_range(dst_hi, p.ys_rows, p.status, kSiteSlotRow)) dst_hi = -1;
       }
     }
     if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)))

@@ -30,6 +30,18 @@ def test_library_exports_every_declared_symbol():
     assert set(_declared()) == set(moe.EXPORTS)
 
 
+def test_bounds_checking_build_exports_the_same_symbols():
+    """libmoe_checks.so (-DMOE_CHECKS) is the same boundary with device index
+    checks compiled in; it says so through moe_bounds_checked."""
+    path = os.path.join(os.path.dirname(moe.lib_path), "libmoe_checks.so")
+    assert os.path.exists(path), "python -m sparse_moe_layer_top_b200.build --checks"
+    L = ctypes.CDLL(path)
+    for name in _declared():
+        assert hasattr(L, name), name
+    assert L.moe_bounds_checked() == 1
+    assert ctypes.CDLL(os.path.join(os.path.dirname(moe.lib_path), "libmoe.so")).moe_bounds_checked() == 0
+
+
 def P(**kw):
     base = dict(T=64, d=256, E=16, k=2, I=128, I_s=64, act="bf16", w="bf16")
     base.update(kw)
