@@ -152,12 +152,18 @@ def routing(moe, layer, x):
     return ids, cnt
 
 
-def gathers_rows(c, T):
-    """Whether the fused forward's gate/up GEMM reads its rows straight from the
-    token matrix, as the library decides it (moe_forward_plan, host only)."""
+def forward_plan(c, T):
+    """The fused forward's kernel choices for workload c under the current
+    path, as the library decides them (moe_forward_plan, host only)."""
     import sparse_moe_layer_top_b200 as moe
     prob = moe.Problem.make(T, c["d"], c["E"], c["k"], c["I"], c["I_s"], c["act"], c["w"])
-    return moe.forward_plan(prob)["gathered"]
+    return moe.forward_plan(prob)
+
+
+def gathers_rows(c, T):
+    """Whether the fused forward's gate/up GEMM reads its rows straight from the
+    token matrix."""
+    return forward_plan(c, T)["gathered"]
 
 
 def work_model(c, counts, T):
