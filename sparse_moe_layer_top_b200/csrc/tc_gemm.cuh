@@ -157,14 +157,28 @@ __device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, const int32
   }
   const int r0 = s_offs[t.g];
   t.rows = s_offs[t.g + 1] - r0;
-  const int mtc = (t.rows + BM - 1) / BM;
+  const bool sh = t.g == p.E;
+  t.N = sh ? p.N_s : p.N_r;
+  const int mtc = (t.rows + BM - 1) / BM, ntc = (t.N + BN - 1) / BN;
   const int local = tile - pre[t.g];
-  const int mb = local % mtc, nb = local / mtc;
+  // Order of a group's tiles.  Column-block-major (its row tiles adjacent)
+  // while the group's activation rows are the smaller operand: the CTAs that
+  // run together share one weight block through L2, and the rows stay there
+  // from one block to the next.  Row-block-major once its rows outnumber its
+  // output columns (a Zipf-hot expert: 8192 rows x 8192 x 2 bytes = 134 MB,
+  // past L2): each activation tile is then read from HBM once, its column
+  // blocks adjacent, while the expert's weights stay in L2.
+  int mb, nb;
+  if (t.rows > t.N) {
+    mb = local / ntc;
+    nb = local - mb * ntc;
+  } else {
+    mb = local % mtc;
+    nb = local / mtc;
+  }
   t.m0 = mb * BM;
   t.row0 = (int64_t)r0 + t.m0;
   t.n0 = nb * BN;
-  const bool sh = t.g == p.E;
-  t.N = sh ? p.N_s : p.N_r;
   t.kb0 = 0;
   t.kb1 = ((sh ? p.K_s : p.K_r) + kBK - 1) / kBK;
   t.split = 0;
