@@ -731,6 +731,11 @@ static moe_status simt_gemms(const moe_problem& p, const void* xp, const int32_t
   return MOE_OK;
 }
 
+// Epilogue outputs of up to this many bytes are stored with an L2
+// evict-last hint (the next kernel reads them back); larger ones evict-first.
+constexpr int64_t kKeepOutBytes = 160ll << 20;
+static int keep_out(int64_t bytes) { return bytes <= kKeepOutBytes ? 1 : 0; }
+
 template <bool FP8>
 static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
                              int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
@@ -766,6 +771,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   a.K_s = p.d;
   a.H = (bf16*)H;
   a.ldh = ldh;
+  a.out_keep = keep_out(Rp * ldh * 2);
   a.sc_b_r = sp[0];
   a.sc_b_s = sp[3];
   a.sc_c_r = sp[1];
@@ -806,6 +812,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   b.sc_b_r = sp[2];
   b.sc_b_s = sp[5];
   b.status = dev->status;
+  b.out_keep = keep_out((o.ys ? p.T * (p.k + 1) : Rp) * p.d * 2);
   if (!FP8) b.sched = pre_b + p.E + 2;
   if (small_rows_of(p, kFormRows) > 0) b.prefix_small = pre_b + p.E + 3;
   if (o.ys) {
@@ -972,6 +979,7 @@ static moe_status pair_gemms(const moe_problem& p, const void* xp, const int32_t
     a.K_s = p.d;
     a.H = (bf16*)H;
     a.ldh = ldh;
+    a.out_keep = keep_out(Rp * ldh * 2);
     a.status = dev->status;
     PROF_BEGIN("gemm_tc_swiglu", st);
     CUDA_TRY(launch_pair(k_gemm_pair<128, true, kPairStages, kTcSwiGLU>, dev->pair_ctas, Pair1Cfg::THREADS,
@@ -997,6 +1005,7 @@ static moe_status pair_gemms(const moe_problem& p, const void* xp, const int32_t
   b.K_r = p.I;
   b.K_s = p.I_s;
   b.status = dev->status;
+  b.out_keep = keep_out((o.ys ? p.T * (p.k + 1) : Rp) * p.d * 2);
   if (o.ys) {
     b.ys = (bf16*)o.ys;
     b.ys_rows = p.T * (p.k + 1);

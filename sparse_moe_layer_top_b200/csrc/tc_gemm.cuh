@@ -60,6 +60,7 @@ struct TcGemmArgs {
   int E;
   int N_r, N_s, K_r, K_s;
   int64_t rows_cap;       // rows of the activation/output buffers; no row at or past it is written
+  int out_keep;           // epilogue stores (H, slot rows, out): 1 L2 evict-last, 0 evict-first
   // single-group mode (single_rows >= 0): one group of single_rows rows that
   // uses the "shared" maps, split along K into ksplit parts
   int single_rows, single_tiles, ksplit, kb_per_split;
@@ -108,7 +109,21 @@ struct TcGemmArgs {
 struct TileInfo {
   int g, rows, m0, n0, kb0, kb1, N, split;
   int64_t row0;
+  bool rowmajor;  // the group's tiles run row-block-major (see decode_tile)
 };
+
+// L2 hints of a tile's loads.  Column-block-major: the weight block serves the
+// row tiles running beside it and is done (evict-first), while each
+// activation tile comes back for the next column block (evict-last).
+// Row-block-major: the other way round -- an activation tile serves its column
+// blocks back to back, the expert's weight blocks come back for every row
+// block.
+struct LoadPolicy {
+  uint64_t w, a;
+};
+__device__ __forceinline__ LoadPolicy load_policy(const TileInfo& t, uint64_t keep, uint64_t stream) {
+  return t.rowmajor ? LoadPolicy{keep, stream} : LoadPolicy{stream, keep};
+}
 
 // s_pre / s_offs: the schedule's tile prefix and group offsets, cached in
 // shared memory at kernel start (grouped mode).  s_pre_s (or NULL): the
@@ -134,6 +149,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, const int32
     const int kbt = (p.K_s + kBK - 1) / kBK;
     t.kb0 = t.split * p.kb_per_split;
     t.kb1 = min(kbt, t.kb0 + p.kb_per_split);
+    t.rowmajor = false;
     return t;
   }
   const int32_t* pre = s_pre;
@@ -169,7 +185,8 @@ __device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, const int32
   // past L2): each activation tile is then read from HBM once, its column
   // blocks adjacent, while the expert's weights stay in L2.
   int mb, nb;
-  if (t.rows > t.N) {
+  t.rowmajor = t.rows > t.N;
+  if (t.rowmajor) {
     mb = local / ntc;
     nb = local - mb * ntc;
   } else {
@@ -249,17 +266,17 @@ __device__ __forceinline__ uint2 e4m3x4_scaled_bf16(uint32_t w, float sc) {
 // 16-byte chunks XOR-swizzled so neither the row-wise writes nor the
 // column-wise reads conflict) and leaves as 8 rows x 64 contiguous bytes per
 // store instruction instead of 32 rows x 16 bytes.  The stores carry an L2
-// evict-last hint: what the epilogues write (H, the weighted slot rows) is
-// read back by the next kernel, while the weights stream past evict-first
-// (measured: down GEMM 138 -> 135 us at the 35B shape).
+// hint: evict-last when what the epilogue writes (H, the weighted slot rows)
+// is small enough for the next kernel to find it in L2 (measured: down GEMM
+// 138 -> 135 us at the 35B shape), evict-first when it is far larger than L2
+// and would only push out the operands still in use (TcGemmArgs::out_keep).
 __device__ __forceinline__ void st_global_evict_last(void* p, uint4 v, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
                "r"(v.w), "l"(pol)
                : "memory");
 }
 __device__ __forceinline__ void store_rows_staged(uint8_t* stg, const uint32_t (&w)[16], char* rowp, int64_t colb,
-                                                  int ncols, int lane) {
-  const uint64_t pol = policy_evict_last();
+                                                  int ncols, int lane, uint64_t pol) {
   const int sw = (lane >> 1) & 3;
 #pragma unroll
   for (int j = 0; j < 4; ++j)
@@ -361,6 +378,8 @@ __device__ __forceinline__ void epilogue_rows(const TcGemmArgs& p, const TileInf
                                               int c1, uint8_t* stg, int lane) {
   const int64_t grow = t.row0 + row;
   const bool valid = t.m0 + row < t.rows && grow < p.rows_cap;
+  // outputs the next kernel will find in L2 are stored evict-last, larger ones evict-first
+  const uint64_t pol = p.out_keep ? policy_evict_last() : policy_evict_first();
   // destination row of this lane (NULL: nothing to write) and its scale
   char* rowp = nullptr;
   float w = 1.f;
@@ -393,7 +412,7 @@ __device__ __forceinline__ void epilogue_rows(const TcGemmArgs& p, const TileInf
         o[e] = pack_bf16x2(w * x0, w * x1);
     }
     const int n = t.n0 + c * 32;
-    store_rows_staged(stg, o, rowp, (int64_t)n * 2, t.N - n, lane);
+    store_rows_staged(stg, o, rowp, (int64_t)n * 2, t.N - n, lane, pol);
   }
 }
 
@@ -687,8 +706,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
       // bf16: A and B tiles into the stage ring.  FP8: raw weight tiles into
       // the raw ring, running ahead of the stage ring, plus an L2 prefetch of
       // the A tile that the A warp will load for the same K-block.
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_a = policy_evict_last();
+      const uint64_t pol_keep = policy_evict_last(), pol_stream = policy_evict_first();
       constexpr int RING = FP8 ? Cfg::RAW_STAGES : STAGES;
       uint64_t* land0 = FP8 ? raw_full : full;
       uint64_t* free0 = FP8 ? raw_empty : empty;
@@ -700,6 +718,8 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
         if (tile >= total) break;
         const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile, s_pre_s);
         const bool sh = t.g == p.E;
+        const LoadPolicy lp = load_policy(t, pol_keep, pol_stream);
+        const uint64_t pol_w = lp.w, pol_a = lp.a;
         bool ok = true;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(free0 + stage, phase ^ 1, abort_flag, p.status, tcode | 1)) {

@@ -129,8 +129,7 @@ __global__ void __launch_bounds__(PairCfg<BN, DUAL, STAGES>::THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer (both ranks, own tiles only)
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_a = policy_evict_last();
+      const uint64_t pol_keep = policy_evict_last(), pol_stream = policy_evict_first();
       const uint32_t full0 = mapa_rank(full, 0);
       int stage = 0;
       uint32_t phase = 0, issued = 0, last_par = 0;
@@ -138,6 +137,8 @@ __global__ void __launch_bounds__(PairCfg<BN, DUAL, STAGES>::THREADS, 1)
       for (int tile = pair; tile < total && ok; tile += npairs) {
         const TileInfo t = decode_tile<BN, kPairBM>(p, s_pre, s_offs, tile);
         const bool sh = t.g == p.E;
+        const LoadPolicy lp = load_policy(t, pol_keep, pol_stream);
+        const uint64_t pol_w = lp.w, pol_a = lp.a;
         const int arow = (int)t.row0 + (int)rank * 128;
         // gate/up: rank 0 loads the gate rows, rank 1 the up rows; down: the two row halves
         const CUtensorMap* wmap = DUAL ? (rank ? (sh ? &tmC_s : &tmC_r) : (sh ? &tmB_s : &tmB_r))
