@@ -443,6 +443,10 @@ def time_steps(moe, layer, x, y, K, W, flush, world, dev, clocks=None):
     # per step: a stage may run as more than one launch (the split form runs
     # each projection as a pair-tile and a weight-row launch)
     kern = {n: sum(v) / K for n, v in per.items()}
+    # and per launch of a step, in launch order (every step launches the same sequence)
+    n = len(prof) // K if K else 0
+    if n and n * K == len(prof):
+        kern["launches"] = [[prof[j][0], statistics.mean(prof[i * n + j][1] for i in range(K))] for j in range(n)]
     return statistics.mean(a.elapsed_time(b) for a, b in ev), kern, launches_per_step, clk
 
 

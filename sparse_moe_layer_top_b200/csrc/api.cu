@@ -731,6 +731,13 @@ static moe_status simt_gemms(const moe_problem& p, const void* xp, const int32_t
   return MOE_OK;
 }
 
+// Tile order of the grouped tensor-core GEMMs: panels of column blocks whose
+// weight blocks take about kPanelBytes together (decode_tile).
+constexpr int64_t kPanelBytes = 32ll << 20;
+static int panel_of(int64_t weight_tile_bytes) {
+  return (int)std::max<int64_t>(1, std::min<int64_t>(64, kPanelBytes / std::max<int64_t>(weight_tile_bytes, 1)));
+}
+
 // Epilogue outputs of up to this many bytes are stored with an L2
 // evict-last hint (the next kernel reads them back); larger ones evict-first.
 constexpr int64_t kKeepOutBytes = 160ll << 20;
@@ -772,6 +779,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   a.H = (bf16*)H;
   a.ldh = ldh;
   a.out_keep = keep_out(Rp * ldh * 2);
+  a.panel = panel_of(2 * 128 * (int64_t)p.d * (FP8 ? 1 : 2));  // gate and up rows of a 128-column block
   a.sc_b_r = sp[0];
   a.sc_b_s = sp[3];
   a.sc_c_r = sp[1];
@@ -813,6 +821,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   b.sc_b_s = sp[5];
   b.status = dev->status;
   b.out_keep = keep_out((o.ys ? p.T * (p.k + 1) : Rp) * p.d * 2);
+  b.panel = panel_of(256 * (int64_t)std::max(p.I, p.I_s) * (FP8 ? 1 : 2));
   if (!FP8) b.sched = pre_b + p.E + 2;
   if (small_rows_of(p, kFormRows) > 0) b.prefix_small = pre_b + p.E + 3;
   if (o.ys) {
@@ -980,6 +989,7 @@ static moe_status pair_gemms(const moe_problem& p, const void* xp, const int32_t
     a.H = (bf16*)H;
     a.ldh = ldh;
     a.out_keep = keep_out(Rp * ldh * 2);
+    a.panel = panel_of(2 * 128 * (int64_t)p.d * 2);
     a.status = dev->status;
     PROF_BEGIN("gemm_tc_swiglu", st);
     CUDA_TRY(launch_pair(k_gemm_pair<128, true, kPairStages, kTcSwiGLU>, dev->pair_ctas, Pair1Cfg::THREADS,
@@ -1006,6 +1016,7 @@ static moe_status pair_gemms(const moe_problem& p, const void* xp, const int32_t
   b.K_s = p.I_s;
   b.status = dev->status;
   b.out_keep = keep_out((o.ys ? p.T * (p.k + 1) : Rp) * p.d * 2);
+  b.panel = panel_of(256 * (int64_t)std::max(p.I, p.I_s) * 2);
   if (o.ys) {
     b.ys = (bf16*)o.ys;
     b.ys_rows = p.T * (p.k + 1);

@@ -61,6 +61,7 @@ struct TcGemmArgs {
   int N_r, N_s, K_r, K_s;
   int64_t rows_cap;       // rows of the activation/output buffers; no row at or past it is written
   int out_keep;           // epilogue stores (H, slot rows, out): 1 L2 evict-last, 0 evict-first
+  int panel;              // grouped mode: column blocks per panel of the tile order (decode_tile)
   // single-group mode (single_rows >= 0): one group of single_rows rows that
   // uses the "shared" maps, split along K into ksplit parts
   int single_rows, single_tiles, ksplit, kb_per_split;
@@ -109,15 +110,14 @@ struct TcGemmArgs {
 struct TileInfo {
   int g, rows, m0, n0, kb0, kb1, N, split;
   int64_t row0;
-  bool rowmajor;  // the group's tiles run row-block-major (see decode_tile)
+  bool rowmajor;  // the group's weight blocks serve several row blocks (see decode_tile)
 };
 
-// L2 hints of a tile's loads.  Column-block-major: the weight block serves the
-// row tiles running beside it and is done (evict-first), while each
-// activation tile comes back for the next column block (evict-last).
-// Row-block-major: the other way round -- an activation tile serves its column
-// blocks back to back, the expert's weight blocks come back for every row
-// block.
+// L2 hints of a tile's loads.  A group of one row tile: its weight blocks are
+// used once (evict-first) and its activation tile by every column block
+// (evict-last).  Larger groups, in panel order: the other way round -- an
+// activation tile serves the panel's column blocks back to back, the panel's
+// weight blocks come back for every row block.
 struct LoadPolicy {
   uint64_t w, a;
 };
@@ -177,22 +177,21 @@ __device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, const int32
   t.N = sh ? p.N_s : p.N_r;
   const int mtc = (t.rows + BM - 1) / BM, ntc = (t.N + BN - 1) / BN;
   const int local = tile - pre[t.g];
-  // Order of a group's tiles.  Column-block-major (its row tiles adjacent)
-  // while the group's activation rows are the smaller operand: the CTAs that
-  // run together share one weight block through L2, and the rows stay there
-  // from one block to the next.  Row-block-major once its rows outnumber its
-  // output columns (a Zipf-hot expert: 8192 rows x 8192 x 2 bytes = 134 MB,
-  // past L2): each activation tile is then read from HBM once, its column
-  // blocks adjacent, while the expert's weights stay in L2.
-  int mb, nb;
-  t.rowmajor = t.rows > t.N;
-  if (t.rowmajor) {
-    mb = local / ntc;
-    nb = local - mb * ntc;
-  } else {
-    mb = local % mtc;
-    nb = local / mtc;
-  }
+  // Order of a group's tiles: panels of p.panel column blocks, each swept row
+  // block by row block (the panel's column blocks adjacent).  The panel's
+  // weight blocks (about 32 MB) stay in L2 while the activation tiles stream
+  // past, each read from HBM once per panel and shared by the CTAs that run
+  // its column blocks together.  Pure column-block-major order re-reads a large
+  // group's activation rows for every column block, pure row-block-major its
+  // whole weight slice for every row block, and for data that all SMs read
+  // B200's L2 holds about half its 126 MB (one copy per die): at the prefill
+  // shape a Zipf-hot expert has 134 MB of rows and 64 MB of gate/up weights.
+  const int P = min(max(p.panel, 1), ntc);
+  const int pan = local / (mtc * P);
+  const int p0 = pan * P, cw = min(P, ntc - p0);
+  const int i = local - pan * mtc * P;
+  const int mb = i / cw, nb = p0 + i % cw;
+  t.rowmajor = mtc > 1;  // weight blocks reused across row blocks
   t.m0 = mb * BM;
   t.row0 = (int64_t)r0 + t.m0;
   t.n0 = nb * BN;
