@@ -59,9 +59,11 @@ struct Profiler {
 };
 static thread_local Profiler g_prof;
 
-// Mode 2 records only the tensor-core GEMM launches (names "gemm_tc_*").
+// Mode 2 records only the tensor-core GEMMs (names "gemm_*": "gemm_tc_*" the
+// launches, or the spans of a stage run as concurrent launches, "gemm_pair_*" /
+// "gemm_swap_*" those launches).
 static bool prof_wants(const char* name) {
-  return g_prof.mode == 1 || (g_prof.mode == 2 && strncmp(name, "gemm_tc", 7) == 0);
+  return g_prof.mode == 1 || (g_prof.mode == 2 && strncmp(name, "gemm_", 5) == 0);
 }
 static void prof_begin(const char* name, cudaStream_t st) {
   Profiler& P = g_prof;
@@ -82,6 +84,20 @@ static void prof_end(const char* name, cudaStream_t st) {
   P.ev[P.used].name = name;
   cudaEventRecord(P.ev[P.used].end, st);
   ++P.used;
+}
+// A span over several launches (one stage run as concurrent kernels on two
+// streams): its begin and end are recorded on the caller's stream around the
+// whole stage.  Returns the span's entry, or -1.
+static int prof_open(const char* name, cudaStream_t st) {
+  prof_begin(name, st);
+  Profiler& P = g_prof;
+  if (!P.pending) return -1;
+  P.pending = false;
+  P.ev[P.used].name = name;
+  return P.used++;
+}
+static void prof_close(int idx, cudaStream_t st) {
+  if (idx >= 0) cudaEventRecord(g_prof.ev[idx].end, st);
 }
 
 #define PROF_BEGIN(name, st) prof_begin(name, st)
@@ -134,6 +150,16 @@ struct DeviceInfo {
 };
 static DeviceInfo g_dev[kMaxDevices];
 static std::mutex g_dev_mu;
+
+// A second stream per device and calling thread, with its events: the split
+// form runs its weight-row GEMMs there, beside the CTA-pair GEMMs on the
+// caller's stream.  Created on first use (so a first call should come before
+// any stream capture), kept until the process exits.
+struct SideStream {
+  cudaStream_t st = nullptr;
+  cudaEvent_t fork = nullptr, pair_gu = nullptr, swap_gu = nullptr, join = nullptr;
+};
+static thread_local SideStream g_side[kMaxDevices];
 static int g_path = 0;
 
 template <typename K>
@@ -176,6 +202,20 @@ static cudaError_t launch_pair(K kernel, int ctas, int threads, int smem, cudaSt
   cfg.numAttrs = g_pdl_next ? 2 : 1;
   g_pdl_next = true;
   return cudaLaunchKernelEx(&cfg, kernel, a0, a1, b0, b1, c0, c1, args);
+}
+
+static moe_status side_stream(SideStream** out) {
+  int dev = 0;
+  CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_CUDA, "device ordinal %d out of range", dev);
+  SideStream& s = g_side[dev];
+  if (!s.st) {
+    CUDA_TRY(cudaStreamCreateWithFlags(&s.st, cudaStreamNonBlocking));
+    for (cudaEvent_t* e : {&s.fork, &s.pair_gu, &s.swap_gu, &s.join})
+      CUDA_TRY(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
+  }
+  *out = &s;
+  return MOE_OK;
 }
 
 static moe_status device_info(DeviceInfo** out) {
@@ -860,8 +900,13 @@ enum { kPhaseGateUp = 1, kPhaseDown = 2, kPhaseBoth = 3 };
 template <bool FP8>
 static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
                                int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
-                               DeviceInfo* dev, int phases = kPhaseBoth) {
+                               DeviceInfo* dev, int phases = kPhaseBoth, int ctas = 0) {
   using C1 = SwapCfg<true>;
+  const int grid = ctas > 0 ? ctas : dev->sms;
+  // run beside the pair GEMMs (ctas given), the launches carry names of their own
+  const char* nm_gu = ctas > 0 ? "gemm_swap_swiglu" : "gemm_tc_swiglu";
+  const char* nm_dn = ctas > 0 ? "gemm_swap_down" : "gemm_tc_down";
+  const char* nm_st = ctas > 0 ? "gemm_swap_store" : "gemm_tc_store";
   using C2 = SwapCfg<false>;
   const int64_t Rp = rows_total(p), ldh = ldh_of(p);
   const bool sh = p.I_s > 0;
@@ -897,14 +942,14 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
     a.sc_c_r = sp[1];
     a.sc_c_s = sp[4];
     a.status = dev->status;
-    PROF_BEGIN("gemm_tc_swiglu", st);
+    PROF_BEGIN(nm_gu, st);
     if (FP8)
       CUDA_TRY(launch(k_gemm_swap8<true, kTcSwiGLU>,
-                      dev->sms, Swap8Cfg<true>::THREADS, Swap8Cfg<true>::SMEM_BYTES, st, xR, xR, bR, bS, cR, cS, a));
+                      grid, Swap8Cfg<true>::THREADS, Swap8Cfg<true>::SMEM_BYTES, st, xR, xR, bR, bS, cR, cS, a));
     else
       CUDA_TRY(launch(k_gemm_swap<true, kTcSwiGLU>,
-                      dev->sms, C1::THREADS, C1::SMEM_BYTES, st, xR, xR, bR, bS, cR, cS, a));
-    LAUNCH_CHECK("gemm_tc_swiglu", st);
+                      grid, C1::THREADS, C1::SMEM_BYTES, st, xR, xR, bR, bS, cR, cS, a));
+    LAUNCH_CHECK(nm_gu, st);
   }
   if (!(phases & kPhaseDown)) return MOE_OK;
   // down: W_down [E, d, I] is the M operand, H rows the N operand
@@ -933,25 +978,25 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
     b.ldy = p.d;
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
-    PROF_BEGIN("gemm_tc_down", st);
+    PROF_BEGIN(nm_dn, st);
     if (FP8)
       CUDA_TRY(launch(k_gemm_swap8<false, kTcSlotStore>,
-                      dev->sms, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
+                      grid, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
     else
       CUDA_TRY(launch(k_gemm_swap<false, kTcSlotStore>,
-                      dev->sms, C2::THREADS, C2::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
-    LAUNCH_CHECK("gemm_tc_down", st);
+                      grid, C2::THREADS, C2::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
+    LAUNCH_CHECK(nm_dn, st);
   } else {
     b.out = (bf16*)o.out;
     b.ldo = p.d;
-    PROF_BEGIN("gemm_tc_store", st);
+    PROF_BEGIN(nm_st, st);
     if (FP8)
       CUDA_TRY(launch(k_gemm_swap8<false, kTcStore>,
-                      dev->sms, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
+                      grid, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
     else
       CUDA_TRY(launch(k_gemm_swap<false, kTcStore>,
-                      dev->sms, C2::THREADS, C2::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
-    LAUNCH_CHECK("gemm_tc_store", st);
+                      grid, C2::THREADS, C2::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
+    LAUNCH_CHECK(nm_st, st);
   }
   return MOE_OK;
 }
@@ -960,7 +1005,12 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
 // loading 128 activation rows and a 128-row half of the weight tile.
 static moe_status pair_gemms(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
                              int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
-                             DeviceInfo* dev, int phases = kPhaseBoth) {
+                             DeviceInfo* dev, int phases = kPhaseBoth, int ctas = 0) {
+  const int grid = ctas > 0 ? ctas : dev->pair_ctas;
+  // run beside the weight-row GEMMs (ctas given), the launches carry names of their own
+  const char* nm_gu = ctas > 0 ? "gemm_pair_swiglu" : "gemm_tc_swiglu";
+  const char* nm_dn = ctas > 0 ? "gemm_pair_down" : "gemm_tc_down";
+  const char* nm_st = ctas > 0 ? "gemm_pair_store" : "gemm_tc_store";
   const int64_t Rp = rows_total(p), ldh = ldh_of(p);
   const bool sh = p.I_s > 0;
   moe_status s;
@@ -991,10 +1041,10 @@ static moe_status pair_gemms(const moe_problem& p, const void* xp, const int32_t
     a.out_keep = keep_out(Rp * ldh * 2);
     a.panel = panel_of(2 * 128 * (int64_t)p.d * 2);
     a.status = dev->status;
-    PROF_BEGIN("gemm_tc_swiglu", st);
-    CUDA_TRY(launch_pair(k_gemm_pair<128, true, kPairStages, kTcSwiGLU>, dev->pair_ctas, Pair1Cfg::THREADS,
+    PROF_BEGIN(nm_gu, st);
+    CUDA_TRY(launch_pair(k_gemm_pair<128, true, kPairStages, kTcSwiGLU>, grid, Pair1Cfg::THREADS,
                          Pair1Cfg::SMEM_BYTES, st, aR, aR, bR, bS, cR, cS, a));
-    LAUNCH_CHECK("gemm_tc_swiglu", st);
+    LAUNCH_CHECK(nm_gu, st);
   }
   if (!(phases & kPhaseDown)) return MOE_OK;
   // down: the two 128-row halves of each 256-row weight block
@@ -1023,18 +1073,62 @@ static moe_status pair_gemms(const moe_problem& p, const void* xp, const int32_t
     b.ldy = p.d;
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
-    PROF_BEGIN("gemm_tc_down", st);
-    CUDA_TRY(launch_pair(k_gemm_pair<256, false, kPairStages, kTcSlotStore>, dev->pair_ctas, Pair2Cfg::THREADS,
+    PROF_BEGIN(nm_dn, st);
+    CUDA_TRY(launch_pair(k_gemm_pair<256, false, kPairStages, kTcSlotStore>, grid, Pair2Cfg::THREADS,
                          Pair2Cfg::SMEM_BYTES, st, aR, aS, bR, bS, bR, bS, b));
-    LAUNCH_CHECK("gemm_tc_down", st);
+    LAUNCH_CHECK(nm_dn, st);
   } else {
     b.out = (bf16*)o.out;
     b.ldo = p.d;
-    PROF_BEGIN("gemm_tc_store", st);
-    CUDA_TRY(launch_pair(k_gemm_pair<256, false, kPairStages, kTcStore>, dev->pair_ctas, Pair2Cfg::THREADS,
+    PROF_BEGIN(nm_st, st);
+    CUDA_TRY(launch_pair(k_gemm_pair<256, false, kPairStages, kTcStore>, grid, Pair2Cfg::THREADS,
                          Pair2Cfg::SMEM_BYTES, st, aR, aS, bR, bS, bR, bS, b));
-    LAUNCH_CHECK("gemm_tc_store", st);
+    LAUNCH_CHECK(nm_st, st);
   }
+  return MOE_OK;
+}
+
+// The split form: the large groups' tiles are counted in pre_a / pre_b, the
+// others' in the second prefix of each (pre + E + 3).  The CTA-pair GEMMs run
+// on the caller's stream with all SMs but kSplitSwapSMs, the weight-row GEMMs
+// on the side stream with those: the weight-row tiles stream their weights
+// from HBM while the pair tiles keep the tensor cores busy.  Each kernel walks
+// its own list and writes its own rows of H and of the slot rows.  A down
+// GEMM stores its slot rows over the dispatched rows that both gate/up GEMMs
+// read, so each down GEMM also waits for the other side's gate/up GEMM.
+constexpr int kSplitSwapSMs = 20;
+static moe_status split_gemms(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
+                              int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
+                              DeviceInfo* dev) {
+  int32_t* sa = pre_a + p.E + 3;
+  int32_t* sb = pre_b + p.E + 3;
+  SideStream* side;
+  moe_status s;
+  if ((s = side_stream(&side)) != MOE_OK) return s;
+  const int swap_ctas = std::min(kSplitSwapSMs, dev->sms / 2);
+  const int pair_ctas = std::max(2, std::min(dev->pair_ctas, (dev->sms - swap_ctas) & ~1));
+  const int span_gu = prof_open("gemm_tc_swiglu", st);
+  CUDA_TRY(cudaEventRecord(side->fork, st));
+  CUDA_TRY(cudaStreamWaitEvent(side->st, side->fork, 0));
+  if ((s = pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, kPhaseGateUp, pair_ctas)) != MOE_OK) return s;
+  CUDA_TRY(cudaEventRecord(side->pair_gu, st));
+  pdl_reset();
+  if ((s = swap_gemms_t<false>(p, xp, offs, w, sa, sb, H, o, side->st, dev, kPhaseGateUp, swap_ctas)) != MOE_OK)
+    return s;
+  CUDA_TRY(cudaEventRecord(side->swap_gu, side->st));
+  CUDA_TRY(cudaStreamWaitEvent(st, side->swap_gu, 0));
+  prof_close(span_gu, st);
+  pdl_reset();
+  const int span_dn = prof_open(o.ys ? "gemm_tc_down" : "gemm_tc_store", st);
+  if ((s = pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, kPhaseDown, pair_ctas)) != MOE_OK) return s;
+  CUDA_TRY(cudaStreamWaitEvent(side->st, side->pair_gu, 0));
+  pdl_reset();
+  if ((s = swap_gemms_t<false>(p, xp, offs, w, sa, sb, H, o, side->st, dev, kPhaseDown, swap_ctas)) != MOE_OK)
+    return s;
+  CUDA_TRY(cudaEventRecord(side->join, side->st));
+  CUDA_TRY(cudaStreamWaitEvent(st, side->join, 0));
+  prof_close(span_dn, st);
+  pdl_reset();
   return MOE_OK;
 }
 
@@ -1047,19 +1141,7 @@ static moe_status expert_gemms(const moe_problem& p, int form, const void* xp, c
   }
   if (form == kFormRows) return tc_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, g);
   if (form == kFormPair) return pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
-  if (form == kFormSplit) {
-    // the large groups' tiles are counted in pre_a / pre_b, the others' in
-    // the second prefix of each (pre + E + 3): each kernel walks its own list
-    // and writes its own rows of H and of the slot rows; both gate/up GEMMs
-    // read the dispatched rows before either down GEMM overwrites them
-    int32_t* sa = pre_a + p.E + 3;
-    int32_t* sb = pre_b + p.E + 3;
-    moe_status s;
-    if ((s = pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, kPhaseGateUp)) != MOE_OK) return s;
-    if ((s = swap_gemms_t<false>(p, xp, offs, w, sa, sb, H, o, st, dev, kPhaseGateUp)) != MOE_OK) return s;
-    if ((s = pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, kPhaseDown)) != MOE_OK) return s;
-    return swap_gemms_t<false>(p, xp, offs, w, sa, sb, H, o, st, dev, kPhaseDown);
-  }
+  if (form == kFormSplit) return split_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
   if (p.act_dtype == MOE_F32) return simt_gemms<float, float>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
   if (p.w_dtype == MOE_BF16) return simt_gemms<bf16, bf16>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
   return simt_gemms<bf16, uint8_t>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);

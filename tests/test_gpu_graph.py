@@ -10,11 +10,15 @@ import moe_inputs
 pytestmark = pytest.mark.gpu
 
 
-@pytest.mark.parametrize("path,w,E", [(2, "bf16", 20), (3, "bf16", 64), (4, "bf16", 2), (0, "fp8", 12)])
-def test_forward_replays_from_a_cuda_graph(path, w, E):
+# (path, weights, E, T, bias); path 5 (split) on Zipf-skewed groups runs its
+# CTA-pair and weight-row GEMMs on two streams: the capture forks and joins
+@pytest.mark.parametrize("path,w,E,T,bias", [(2, "bf16", 20, 300, None), (3, "bf16", 64, 300, None),
+                                             (4, "bf16", 2, 2048, None), (0, "fp8", 12, 300, None),
+                                             (5, "bf16", 24, 1536, "zipf")])
+def test_forward_replays_from_a_cuda_graph(path, w, E, T, bias):
     import sparse_moe_layer_top_b200 as moe
-    T, d, k, I, I_s = (2048, 256, 2, 256, 128) if E == 2 else (300, 384, 3, 256, 128)
-    inp = moe_inputs.make_inputs(T, d, E, k, I, I_s, act="bf16", w=w, seed=8, device="cuda")
+    d, k, I, I_s = (256, 2, 256, 128) if E == 2 else (384, 3, 256, 128)
+    inp = moe_inputs.make_inputs(T, d, E, k, I, I_s, act="bf16", w=w, bias=bias, seed=8, device="cuda")
     moe.set_path(path)
     try:
         layer = moe.MoELayer.from_inputs(inp, max_tokens=T)
