@@ -257,8 +257,7 @@ MOE_API moe_status moe_forward_plan(const moe_problem* p, int32_t* expert_form, 
  * 0 = automatic (tensor-core kernels where the types allow; for the expert
  *     GEMMs the weight-row form when T*k <= 64*E, i.e. when an expert sees at
  *     most one 64-token chunk on average, the form of 4 when bf16 experts
- *     average 2048 rows or more (T*k >= 2048*E), the form of 5 when they
- *     average 144 rows or more, else the row-tiled form);
+ *     average 2048 rows or more (T*k >= 2048*E), else the row-tiled form);
  * 1 = SIMT CUDA kernels only (fp32 FMA; the path of fp32 problems);
  * 2 = tensor-core kernels required, row-tiled expert GEMMs;
  * 3 = tensor-core kernels required, weight-row expert GEMMs;
@@ -266,9 +265,9 @@ MOE_API moe_status moe_forward_plan(const moe_problem* p, int32_t* expert_form, 
  *     (256-row tiles, tcgen05 pair MMAs; E4M3 weights take the form of 2);
  * 5 = tensor-core kernels required, split expert GEMMs: the groups of 256
  *     rows or more as in 4, the others as in 3, one launch each per
- *     projection (E4M3 weights take the form of 2).  Automatic for bf16
- *     weights when experts average 144 to 2047 rows (a large batch, where
- *     skewed routing leaves some experts thousands of rows and many a few).
+ *     projection (E4M3 weights take the form of 2).  Never chosen
+ *     automatically: on skewed prefill batches the row-tiled form of 2 was
+ *     faster, since it runs the small groups' tiles among the large ones.
  * 2 to 5 return MOE_ERR_UNSUPPORTED when the types do not allow them. */
 MOE_API moe_status moe_set_path(int path);
 

@@ -219,7 +219,7 @@ def set_path(path):
     """0 automatic, 1 SIMT kernels only, 2 row-tiled tensor-core expert GEMMs,
     3 weight-row tensor-core expert GEMMs, 4 row-tiled on 2-CTA clusters,
     5 split: groups of 256 rows or more on 2-CTA clusters, the others in
-    weight-row form."""
+    weight-row form (on request only)."""
     _check(lib().moe_set_path(int(path)))
 
 

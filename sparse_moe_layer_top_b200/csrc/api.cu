@@ -59,11 +59,9 @@ struct Profiler {
 };
 static thread_local Profiler g_prof;
 
-// Mode 2 records only the tensor-core GEMMs (names "gemm_*": "gemm_tc_*" the
-// launches, or the spans of a stage run as concurrent launches, "gemm_pair_*" /
-// "gemm_swap_*" those launches).
+// Mode 2 records only the tensor-core GEMM launches (names "gemm_tc_*").
 static bool prof_wants(const char* name) {
-  return g_prof.mode == 1 || (g_prof.mode == 2 && strncmp(name, "gemm_", 5) == 0);
+  return g_prof.mode == 1 || (g_prof.mode == 2 && strncmp(name, "gemm_tc", 7) == 0);
 }
 static void prof_begin(const char* name, cudaStream_t st) {
   Profiler& P = g_prof;
@@ -84,20 +82,6 @@ static void prof_end(const char* name, cudaStream_t st) {
   P.ev[P.used].name = name;
   cudaEventRecord(P.ev[P.used].end, st);
   ++P.used;
-}
-// A span over several launches (one stage run as concurrent kernels on two
-// streams): its begin and end are recorded on the caller's stream around the
-// whole stage.  Returns the span's entry, or -1.
-static int prof_open(const char* name, cudaStream_t st) {
-  prof_begin(name, st);
-  Profiler& P = g_prof;
-  if (!P.pending) return -1;
-  P.pending = false;
-  P.ev[P.used].name = name;
-  return P.used++;
-}
-static void prof_close(int idx, cudaStream_t st) {
-  if (idx >= 0) cudaEventRecord(g_prof.ev[idx].end, st);
 }
 
 #define PROF_BEGIN(name, st) prof_begin(name, st)
@@ -150,16 +134,6 @@ struct DeviceInfo {
 };
 static DeviceInfo g_dev[kMaxDevices];
 static std::mutex g_dev_mu;
-
-// A second stream per device and calling thread, with its events: the split
-// form runs its weight-row GEMMs there, beside the CTA-pair GEMMs on the
-// caller's stream.  Created on first use (so a first call should come before
-// any stream capture), kept until the process exits.
-struct SideStream {
-  cudaStream_t st = nullptr;
-  cudaEvent_t fork = nullptr, pair_gu = nullptr, swap_gu = nullptr, join = nullptr;
-};
-static thread_local SideStream g_side[kMaxDevices];
 static int g_path = 0;
 
 template <typename K>
@@ -202,20 +176,6 @@ static cudaError_t launch_pair(K kernel, int ctas, int threads, int smem, cudaSt
   cfg.numAttrs = g_pdl_next ? 2 : 1;
   g_pdl_next = true;
   return cudaLaunchKernelEx(&cfg, kernel, a0, a1, b0, b1, c0, c1, args);
-}
-
-static moe_status side_stream(SideStream** out) {
-  int dev = 0;
-  CUDA_TRY(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_CUDA, "device ordinal %d out of range", dev);
-  SideStream& s = g_side[dev];
-  if (!s.st) {
-    CUDA_TRY(cudaStreamCreateWithFlags(&s.st, cudaStreamNonBlocking));
-    for (cudaEvent_t* e : {&s.fork, &s.pair_gu, &s.swap_gu, &s.join})
-      CUDA_TRY(cudaEventCreateWithFlags(e, cudaEventDisableTiming));
-  }
-  *out = &s;
-  return MOE_OK;
 }
 
 static moe_status device_info(DeviceInfo** out) {
@@ -389,22 +349,20 @@ static moe_status choose(bool tc_possible, bool* use_tc) {
 }
 
 // Expert GEMM form: 0 SIMT, 1 row-tiled tensor core, 2 weight-row (swap)
-// tensor core, 3 row-tiled on CTA pairs.  Automatic choice: the weight-row
+// tensor core, 3 row-tiled on CTA pairs, 4 split (CTA pairs for the groups of
+// kSplitRows rows or more, weight-row tiles for the others, one launch each
+// per projection; chosen with moe_set_path(5) only: on the Zipf prefill
+// workload it measured 10.9 ms against 10.5-10.6 for the row-tiled form, whose
+// interleaved tile order already runs the small groups' weight streaming
+// beside the large groups' tensor work).  Automatic choice: the weight-row
 // form when an expert sees at most one token chunk on average (T*k <= 64*E),
 // where a 128-row activation tile would be mostly empty; the pair form (bf16
 // weights) when experts average kPairRowsPerExpert rows or more, where its
 // 256-row tiles waste little on group tails (measured: 12-15 % faster at 4096
 // rows per expert, even at 1024, slower on prefill-sized Zipf-skewed groups);
-// between, when experts average kSplitAvgRows rows or more (bf16 weights),
-// the split form: the groups of kSplitRows rows or more on CTA pairs, the
-// others in weight-row form, two launches per projection (a large batch whose
-// routing is skewed gives a few experts thousands of rows and many experts a
-// handful: the first want the pair tiles' operand economy, the second would
-// spend a 128-row tile's MMAs on a few rows while their weights stream);
 // else the row-tiled form.
 enum { kFormSimt = 0, kFormRows = 1, kFormSwap = 2, kFormPair = 3, kFormSplit = 4 };
 constexpr int kPairRowsPerExpert = 2048;
-constexpr int kSplitAvgRows = 144;
 constexpr int kSplitRows = 256;
 static moe_status choose_form(const moe_problem& p, int* form) {
   bool tc;
@@ -417,7 +375,6 @@ static moe_status choose_form(const moe_problem& p, int* form) {
   else if (g_path == 5) *form = p.w_dtype == MOE_BF16 ? kFormSplit : kFormRows;
   else if (p.T * (int64_t)p.k <= (int64_t)kNCH * p.E) *form = kFormSwap;
   else if (p.w_dtype == MOE_BF16 && p.T * (int64_t)p.k >= (int64_t)kPairRowsPerExpert * p.E) *form = kFormPair;
-  else if (p.w_dtype == MOE_BF16 && p.T * (int64_t)p.k >= (int64_t)kSplitAvgRows * p.E) *form = kFormSplit;
   else *form = kFormRows;
   return MOE_OK;
 }
@@ -772,9 +729,14 @@ static moe_status simt_gemms(const moe_problem& p, const void* xp, const int32_t
 }
 
 // Tile order of the grouped tensor-core GEMMs: panels of column blocks whose
-// weight blocks take about kPanelBytes together (decode_tile).
-constexpr int64_t kPanelBytes = 32ll << 20;
-static int panel_of(int64_t weight_tile_bytes) {
+// weight blocks take about kPanelBytes together (decode_tile); column-block-
+// major (a panel of one) when a group's whole weight slice is at most
+// kSmallSliceBytes, where a group's rows are few and everything stays in L2
+// (the 35B shapes: 4 and 2 MB per expert; measured there, panels of every
+// column block made the gate/up GEMM 231 -> 252 us).
+constexpr int64_t kPanelBytes = 32ll << 20, kSmallSliceBytes = 16ll << 20;
+static int panel_of(int64_t weight_tile_bytes, int64_t column_blocks) {
+  if (weight_tile_bytes * column_blocks <= kSmallSliceBytes) return 1;
   return (int)std::max<int64_t>(1, std::min<int64_t>(64, kPanelBytes / std::max<int64_t>(weight_tile_bytes, 1)));
 }
 
@@ -819,7 +781,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   a.H = (bf16*)H;
   a.ldh = ldh;
   a.out_keep = keep_out(Rp * ldh * 2);
-  a.panel = panel_of(2 * 128 * (int64_t)p.d * (FP8 ? 1 : 2));  // gate and up rows of a 128-column block
+  a.panel = panel_of(2 * 128 * (int64_t)p.d * (FP8 ? 1 : 2), cdiv(p.I, 128));  // gate and up rows, 128 columns
   a.sc_b_r = sp[0];
   a.sc_b_s = sp[3];
   a.sc_c_r = sp[1];
@@ -861,7 +823,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   b.sc_b_s = sp[5];
   b.status = dev->status;
   b.out_keep = keep_out((o.ys ? p.T * (p.k + 1) : Rp) * p.d * 2);
-  b.panel = panel_of(256 * (int64_t)std::max(p.I, p.I_s) * (FP8 ? 1 : 2));
+  b.panel = panel_of(256 * (int64_t)std::max(p.I, p.I_s) * (FP8 ? 1 : 2), cdiv(p.d, 256));
   if (!FP8) b.sched = pre_b + p.E + 2;
   if (small_rows_of(p, kFormRows) > 0) b.prefix_small = pre_b + p.E + 3;
   if (o.ys) {
@@ -900,13 +862,9 @@ enum { kPhaseGateUp = 1, kPhaseDown = 2, kPhaseBoth = 3 };
 template <bool FP8>
 static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
                                int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
-                               DeviceInfo* dev, int phases = kPhaseBoth, int ctas = 0) {
+                               DeviceInfo* dev, int phases = kPhaseBoth) {
   using C1 = SwapCfg<true>;
-  const int grid = ctas > 0 ? ctas : dev->sms;
-  // run beside the pair GEMMs (ctas given), the launches carry names of their own
-  const char* nm_gu = ctas > 0 ? "gemm_swap_swiglu" : "gemm_tc_swiglu";
-  const char* nm_dn = ctas > 0 ? "gemm_swap_down" : "gemm_tc_down";
-  const char* nm_st = ctas > 0 ? "gemm_swap_store" : "gemm_tc_store";
+  const int grid = dev->sms;
   using C2 = SwapCfg<false>;
   const int64_t Rp = rows_total(p), ldh = ldh_of(p);
   const bool sh = p.I_s > 0;
@@ -942,14 +900,14 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
     a.sc_c_r = sp[1];
     a.sc_c_s = sp[4];
     a.status = dev->status;
-    PROF_BEGIN(nm_gu, st);
+    PROF_BEGIN("gemm_tc_swiglu", st);
     if (FP8)
       CUDA_TRY(launch(k_gemm_swap8<true, kTcSwiGLU>,
                       grid, Swap8Cfg<true>::THREADS, Swap8Cfg<true>::SMEM_BYTES, st, xR, xR, bR, bS, cR, cS, a));
     else
       CUDA_TRY(launch(k_gemm_swap<true, kTcSwiGLU>,
                       grid, C1::THREADS, C1::SMEM_BYTES, st, xR, xR, bR, bS, cR, cS, a));
-    LAUNCH_CHECK(nm_gu, st);
+    LAUNCH_CHECK("gemm_tc_swiglu", st);
   }
   if (!(phases & kPhaseDown)) return MOE_OK;
   // down: W_down [E, d, I] is the M operand, H rows the N operand
@@ -978,25 +936,25 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
     b.ldy = p.d;
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
-    PROF_BEGIN(nm_dn, st);
+    PROF_BEGIN("gemm_tc_down", st);
     if (FP8)
       CUDA_TRY(launch(k_gemm_swap8<false, kTcSlotStore>,
                       grid, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
     else
       CUDA_TRY(launch(k_gemm_swap<false, kTcSlotStore>,
                       grid, C2::THREADS, C2::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
-    LAUNCH_CHECK(nm_dn, st);
+    LAUNCH_CHECK("gemm_tc_down", st);
   } else {
     b.out = (bf16*)o.out;
     b.ldo = p.d;
-    PROF_BEGIN(nm_st, st);
+    PROF_BEGIN("gemm_tc_store", st);
     if (FP8)
       CUDA_TRY(launch(k_gemm_swap8<false, kTcStore>,
                       grid, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
     else
       CUDA_TRY(launch(k_gemm_swap<false, kTcStore>,
                       grid, C2::THREADS, C2::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
-    LAUNCH_CHECK(nm_st, st);
+    LAUNCH_CHECK("gemm_tc_store", st);
   }
   return MOE_OK;
 }
@@ -1005,12 +963,8 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
 // loading 128 activation rows and a 128-row half of the weight tile.
 static moe_status pair_gemms(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
                              int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
-                             DeviceInfo* dev, int phases = kPhaseBoth, int ctas = 0) {
-  const int grid = ctas > 0 ? ctas : dev->pair_ctas;
-  // run beside the weight-row GEMMs (ctas given), the launches carry names of their own
-  const char* nm_gu = ctas > 0 ? "gemm_pair_swiglu" : "gemm_tc_swiglu";
-  const char* nm_dn = ctas > 0 ? "gemm_pair_down" : "gemm_tc_down";
-  const char* nm_st = ctas > 0 ? "gemm_pair_store" : "gemm_tc_store";
+                             DeviceInfo* dev, int phases = kPhaseBoth) {
+  const int grid = dev->pair_ctas;
   const int64_t Rp = rows_total(p), ldh = ldh_of(p);
   const bool sh = p.I_s > 0;
   moe_status s;
@@ -1039,12 +993,12 @@ static moe_status pair_gemms(const moe_problem& p, const void* xp, const int32_t
     a.H = (bf16*)H;
     a.ldh = ldh;
     a.out_keep = keep_out(Rp * ldh * 2);
-    a.panel = panel_of(2 * 128 * (int64_t)p.d * 2);
+    a.panel = panel_of(2 * 128 * (int64_t)p.d * 2, cdiv(p.I, 128));
     a.status = dev->status;
-    PROF_BEGIN(nm_gu, st);
+    PROF_BEGIN("gemm_tc_swiglu", st);
     CUDA_TRY(launch_pair(k_gemm_pair<128, true, kPairStages, kTcSwiGLU>, grid, Pair1Cfg::THREADS,
                          Pair1Cfg::SMEM_BYTES, st, aR, aR, bR, bS, cR, cS, a));
-    LAUNCH_CHECK(nm_gu, st);
+    LAUNCH_CHECK("gemm_tc_swiglu", st);
   }
   if (!(phases & kPhaseDown)) return MOE_OK;
   // down: the two 128-row halves of each 256-row weight block
@@ -1066,70 +1020,43 @@ static moe_status pair_gemms(const moe_problem& p, const void* xp, const int32_t
   b.K_s = p.I_s;
   b.status = dev->status;
   b.out_keep = keep_out((o.ys ? p.T * (p.k + 1) : Rp) * p.d * 2);
-  b.panel = panel_of(256 * (int64_t)std::max(p.I, p.I_s) * 2);
+  b.panel = panel_of(256 * (int64_t)std::max(p.I, p.I_s) * 2, cdiv(p.d, 256));
   if (o.ys) {
     b.ys = (bf16*)o.ys;
     b.ys_rows = p.T * (p.k + 1);
     b.ldy = p.d;
     b.row_dst = o.row_dst;
     b.row_w = o.row_w;
-    PROF_BEGIN(nm_dn, st);
+    PROF_BEGIN("gemm_tc_down", st);
     CUDA_TRY(launch_pair(k_gemm_pair<256, false, kPairStages, kTcSlotStore>, grid, Pair2Cfg::THREADS,
                          Pair2Cfg::SMEM_BYTES, st, aR, aS, bR, bS, bR, bS, b));
-    LAUNCH_CHECK(nm_dn, st);
+    LAUNCH_CHECK("gemm_tc_down", st);
   } else {
     b.out = (bf16*)o.out;
     b.ldo = p.d;
-    PROF_BEGIN(nm_st, st);
+    PROF_BEGIN("gemm_tc_store", st);
     CUDA_TRY(launch_pair(k_gemm_pair<256, false, kPairStages, kTcStore>, grid, Pair2Cfg::THREADS,
                          Pair2Cfg::SMEM_BYTES, st, aR, aS, bR, bS, bR, bS, b));
-    LAUNCH_CHECK(nm_st, st);
+    LAUNCH_CHECK("gemm_tc_store", st);
   }
   return MOE_OK;
 }
 
 // The split form: the large groups' tiles are counted in pre_a / pre_b, the
-// others' in the second prefix of each (pre + E + 3).  The CTA-pair GEMMs run
-// on the caller's stream with all SMs but kSplitSwapSMs, the weight-row GEMMs
-// on the side stream with those: the weight-row tiles stream their weights
-// from HBM while the pair tiles keep the tensor cores busy.  Each kernel walks
-// its own list and writes its own rows of H and of the slot rows.  A down
-// GEMM stores its slot rows over the dispatched rows that both gate/up GEMMs
-// read, so each down GEMM also waits for the other side's gate/up GEMM.
-constexpr int kSplitSwapSMs = 20;
+// others' in the second prefix of each (pre + E + 3); each kernel walks its
+// own list and writes its own rows of H and of the slot rows.  A down GEMM
+// stores its slot rows over the dispatched rows that both gate/up GEMMs read,
+// so both gate/up GEMMs run before either down GEMM.
 static moe_status split_gemms(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
                               int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
                               DeviceInfo* dev) {
   int32_t* sa = pre_a + p.E + 3;
   int32_t* sb = pre_b + p.E + 3;
-  SideStream* side;
   moe_status s;
-  if ((s = side_stream(&side)) != MOE_OK) return s;
-  const int swap_ctas = std::min(kSplitSwapSMs, dev->sms / 2);
-  const int pair_ctas = std::max(2, std::min(dev->pair_ctas, (dev->sms - swap_ctas) & ~1));
-  const int span_gu = prof_open("gemm_tc_swiglu", st);
-  CUDA_TRY(cudaEventRecord(side->fork, st));
-  CUDA_TRY(cudaStreamWaitEvent(side->st, side->fork, 0));
-  if ((s = pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, kPhaseGateUp, pair_ctas)) != MOE_OK) return s;
-  CUDA_TRY(cudaEventRecord(side->pair_gu, st));
-  pdl_reset();
-  if ((s = swap_gemms_t<false>(p, xp, offs, w, sa, sb, H, o, side->st, dev, kPhaseGateUp, swap_ctas)) != MOE_OK)
-    return s;
-  CUDA_TRY(cudaEventRecord(side->swap_gu, side->st));
-  CUDA_TRY(cudaStreamWaitEvent(st, side->swap_gu, 0));
-  prof_close(span_gu, st);
-  pdl_reset();
-  const int span_dn = prof_open(o.ys ? "gemm_tc_down" : "gemm_tc_store", st);
-  if ((s = pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, kPhaseDown, pair_ctas)) != MOE_OK) return s;
-  CUDA_TRY(cudaStreamWaitEvent(side->st, side->pair_gu, 0));
-  pdl_reset();
-  if ((s = swap_gemms_t<false>(p, xp, offs, w, sa, sb, H, o, side->st, dev, kPhaseDown, swap_ctas)) != MOE_OK)
-    return s;
-  CUDA_TRY(cudaEventRecord(side->join, side->st));
-  CUDA_TRY(cudaStreamWaitEvent(st, side->join, 0));
-  prof_close(span_dn, st);
-  pdl_reset();
-  return MOE_OK;
+  if ((s = pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, kPhaseGateUp)) != MOE_OK) return s;
+  if ((s = swap_gemms_t<false>(p, xp, offs, w, sa, sb, H, o, st, dev, kPhaseGateUp)) != MOE_OK) return s;
+  if ((s = pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, kPhaseDown)) != MOE_OK) return s;
+  return swap_gemms_t<false>(p, xp, offs, w, sa, sb, H, o, st, dev, kPhaseDown);
 }
 
 static moe_status expert_gemms(const moe_problem& p, int form, const void* xp, const int32_t* offs,

@@ -113,11 +113,12 @@ struct TileInfo {
   bool rowmajor;  // the group's weight blocks serve several row blocks (see decode_tile)
 };
 
-// L2 hints of a tile's loads.  A group of one row tile: its weight blocks are
-// used once (evict-first) and its activation tile by every column block
-// (evict-last).  Larger groups, in panel order: the other way round -- an
-// activation tile serves the panel's column blocks back to back, the panel's
-// weight blocks come back for every row block.
+// L2 hints of a tile's loads.  In column-block-major order (and in a group of
+// one row tile) a weight block serves the row tiles running beside it and is
+// done (evict-first), while the activation tiles come back for the next column
+// block (evict-last).  In panels of several column blocks the other way round:
+// an activation tile serves the panel's column blocks back to back, the
+// panel's weight blocks come back for every row block.
 struct LoadPolicy {
   uint64_t w, a;
 };
@@ -191,7 +192,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, const int32
   const int p0 = pan * P, cw = min(P, ntc - p0);
   const int i = local - pan * mtc * P;
   const int mb = i / cw, nb = p0 + i % cw;
-  t.rowmajor = mtc > 1;  // weight blocks reused across row blocks
+  t.rowmajor = P > 1 && mtc > 1;  // weight blocks reused across row blocks
   t.m0 = mb * BM;
   t.row0 = (int64_t)r0 + t.m0;
   t.n0 = nb * BN;

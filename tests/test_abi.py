@@ -152,11 +152,9 @@ def test_forward_plan_on_the_host():
     assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16") == \
         {"expert_form": "rows", "router_selects": True, "gathered": True}
     assert plan(8192, 8192, 512, 10, 2048, 2048, "bf16", "bf16") == \
-        {"expert_form": "split", "router_selects": False, "gathered": False}     # 512 experts; 160 rows each
-    # the split form from 144 rows per expert on average, the pair form from 2048
-    assert plan(7372, 8192, 512, 10, 2048, 2048, "bf16", "bf16")["expert_form"] == "rows"
-    assert plan(7373, 8192, 512, 10, 2048, 2048, "bf16", "bf16")["expert_form"] == "split"
-    assert plan(7373, 8192, 512, 10, 2048, 2048, "bf16", "fp8")["expert_form"] == "rows"
+        {"expert_form": "rows", "router_selects": False, "gathered": False}      # 512 experts; x > 32 MiB
+    # the pair form from 2048 rows per expert on average; the split form only on request
+    assert plan(4095, 256, 2, 1, 256, 256, "bf16", "bf16")["expert_form"] == "rows"
     assert plan(4096, 256, 2, 1, 256, 256, "bf16", "bf16")["expert_form"] == "cta_pairs"
     assert plan(64, 8192, 512, 10, 2048, 2048, "bf16", "bf16")["expert_form"] == "weight_rows"
     assert plan(2048, 8192, 512, 10, 2048, 2048, "bf16", "fp8")["expert_form"] == "weight_rows"

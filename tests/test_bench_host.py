@@ -73,7 +73,7 @@ def test_gate_up_input_is_the_token_matrix_where_the_gemm_gathers_it():
     assert not bench.gathers_rows(pre, 8192)        # x = 128 MiB, larger than L2
     assert not bench.gathers_rows(pre, 64)          # decode: the weight-row form
     assert not bench.gathers_rows(dict(c35, w="fp8"), 4096)
-    assert bench.forward_plan(pre, 8192)["expert_form"] == "split"   # the line reports it
+    assert bench.forward_plan(pre, 8192)["expert_form"] == "rows"   # the line reports it
     counts = [128] * 256
     T = 4096
     w = bench.work_model(c35, counts, T)
