@@ -483,15 +483,7 @@ static Layout layout(const moe_problem& p, bool forward) {
 
 // ============================================================== launch pieces
 static Schedule sched_simt(int n_r, int n_s) { return Schedule{64, 64, n_r, n_s, 0, 0, 0, 0}; }
-static Schedule sched_tc(int bn, int n_r, int n_s, int small_rows = 0) {
-  return Schedule{kBM, bn, n_r, n_s, 0, small_rows, 0, 0};
-}
-// The row-tiled bf16 GEMMs (tiles claimed in order) spread the tiles of
-// groups with one row tile among the others; the E4M3 form (tiles dealt in a
-// fixed order) keeps the plain group order.
-static int small_rows_of(const moe_problem& p, int form) {
-  return form == kFormRows && p.w_dtype != MOE_FP8_E4M3_B128 ? kBM : 0;
-}
+static Schedule sched_tc(int bn, int n_r, int n_s) { return Schedule{kBM, bn, n_r, n_s, 0, 0, 0, 0}; }
 
 // Router and top-k.  `counts` (may be NULL) receives the per-chunk histograms
 // for the dispatch when the tensor-core path is taken; *counted says so.
@@ -788,7 +780,6 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   a.sc_c_s = sp[4];
   a.status = dev->status;
   if (!FP8) a.sched = pre_a + p.E + 2;  // tiles claimed in order (the prefix writer zeroed it)
-  if (small_rows_of(p, kFormRows) > 0) a.prefix_small = pre_a + p.E + 3;
   PROF_BEGIN("gemm_tc_swiglu", st);
   if (!FP8 && g.x) {
     a.gx = (const bf16*)g.x;
@@ -825,7 +816,6 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   b.out_keep = keep_out((o.ys ? p.T * (p.k + 1) : Rp) * p.d * 2);
   b.panel = panel_of(256 * (int64_t)std::max(p.I, p.I_s) * (FP8 ? 1 : 2), cdiv(p.d, 256));
   if (!FP8) b.sched = pre_b + p.E + 2;
-  if (small_rows_of(p, kFormRows) > 0) b.prefix_small = pre_b + p.E + 3;
   if (o.ys) {
     b.ys = (bf16*)o.ys;
     b.ys_rows = p.T * (p.k + 1);
@@ -1076,8 +1066,8 @@ static moe_status expert_gemms(const moe_problem& p, int form, const void* xp, c
 
 static void schedules(const moe_problem& p, int form, Schedule* sa, Schedule* sb) {
   if (form == kFormRows) {
-    *sa = sched_tc(128, p.I, p.I_s, small_rows_of(p, form));
-    *sb = sched_tc(256, p.d, p.d, small_rows_of(p, form));
+    *sa = sched_tc(128, p.I, p.I_s);
+    *sb = sched_tc(256, p.d, p.d);
   } else if (form == kFormPair) {  // 256-row tiles of CTA pairs
     *sa = Schedule{kPairBM, 128, p.I, p.I_s, 0, 0, 0, 0};
     *sb = Schedule{kPairBM, 256, p.d, p.d, 0, 0, 0, 0};

@@ -95,13 +95,10 @@ __device__ __forceinline__ int find_group(const int32_t* prefix, int ngroups, in
 // m_tiles = ceil(rows / bm) for the row-tiled kernels, and 0 or 1 for the
 // weight-row (swap) kernels whose N covers every row of a group.
 // Tiles of a grouped GEMM: ceil(rows / bm) x ceil(n / bn) per group (one
-// row tile per group when swap).  With small_rows > 0 the groups of at most
-// small_rows rows are counted in a prefix of their own, with tiles of
-// bm_small x bn_small (0: bm, bn).  Two uses: the row-tiled GEMM spreads the
-// tiles of its one-row-tile groups (each streams its weight block from HBM for
-// few rows) evenly among the others (see decode_tile); the split form runs
-// the large groups on CTA pairs and the small ones in weight-row form, each
-// kernel walking its own prefix.
+// row tile per group when swap).  With small_rows > 0 (the split form) the
+// groups of at most small_rows rows are counted in a prefix of their own, with
+// tiles of bm_small x bn_small (0: bm, bn): the large groups run on CTA pairs
+// and the small ones in weight-row form, each kernel walking its own prefix.
 struct Schedule {
   int bm, bn, n_routed, n_shared, swap, small_rows, bm_small, bn_small;
 };

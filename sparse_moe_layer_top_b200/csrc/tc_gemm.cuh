@@ -54,9 +54,6 @@ enum { kTcSwiGLU = 0, kTcSlotStore = 1, kTcStore = 2, kTcLogits = 3, kTcTopK = 4
 struct TcGemmArgs {
   const int32_t* offs;    // [E+2] group row starts (grouped mode)
   const int32_t* prefix;  // [E+2] tile prefix of this schedule (grouped mode)
-  // [E+2] tile prefix of the schedule's small groups (Schedule::small_rows),
-  // or NULL: their tiles are spread evenly among the others (decode_tile)
-  const int32_t* prefix_small;
   int E;
   int N_r, N_s, K_r, K_s;
   int64_t rows_cap;       // rows of the activation/output buffers; no row at or past it is written
@@ -127,15 +124,10 @@ __device__ __forceinline__ LoadPolicy load_policy(const TileInfo& t, uint64_t ke
 }
 
 // s_pre / s_offs: the schedule's tile prefix and group offsets, cached in
-// shared memory at kernel start (grouped mode).  s_pre_s (or NULL): the
-// prefix of the small groups, whose ns tiles are spread over the nb + ns tile
-// indices: index i is the small tile floor(i ns / (nb + ns)) when that count
-// grows at i + 1, else big tile i - floor(i ns / (nb + ns)).  Claimed in index
-// order, the weight-streaming tiles of groups with few rows then run beside
-// the tensor-bound tiles of large groups instead of all at once.
+// shared memory at kernel start (grouped mode).
 template <int BN, int BM = kBM>
 __device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, const int32_t* s_pre, const int32_t* s_offs,
-                                                int tile, const int32_t* s_pre_s = nullptr) {
+                                                int tile) {
   TileInfo t;
   if (p.single_rows >= 0) {
     t.g = p.E;
@@ -154,16 +146,6 @@ __device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, const int32
     return t;
   }
   const int32_t* pre = s_pre;
-  if (s_pre_s) {
-    const int64_t ns = s_pre_s[p.E + 1], n = (int64_t)s_pre[p.E + 1] + ns;
-    const int before = (int)((int64_t)tile * ns / n);
-    if ((int)((int64_t)(tile + 1) * ns / n) > before) {
-      pre = s_pre_s;
-      tile = before;
-    } else {
-      tile -= before;
-    }
-  }
   {
     int lo = 0, hi = p.E + 1;  // pre[lo] <= tile < pre[hi]
     while (hi - lo > 1) {
@@ -235,7 +217,7 @@ struct TcGemmCfg {
   // + 4 + 4 handoff barriers of the router epilogue (one pair per lane quarter)
   // + 4 + 4 barriers and 4 ints of the tile queue
   static constexpr int BAR_BYTES = (3 * STAGES + 2 * RAW_STAGES + 5 + 8 + 8) * 8 + 16 + 16;
-  static constexpr int SCHED_INTS = 3 * (512 + 2);  // tile prefixes (all/small) + group offsets, E <= 512
+  static constexpr int SCHED_INTS = 2 * (512 + 2);  // tile prefix + group offsets, E <= 512
   // epilogue staging: 32 rows x 64 bytes per epilogue warp
   static constexpr int EPI_OFF = (RING_BYTES + BAR_BYTES + SCHED_INTS * 4 + 127) / 128 * 128;
   static constexpr int SMEM_BYTES = 1024 + EPI_OFF + EPI_WARPS * 2048;
@@ -640,7 +622,6 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int32_t* s_pre = reinterpret_cast<int32_t*>(smem + Cfg::RING_BYTES + Cfg::BAR_BYTES);
   int32_t* s_offs = s_pre + 514;
-  int32_t* s_pre_s = p.prefix_small ? s_offs + 514 : nullptr;
   uint8_t* epi_stage = smem + Cfg::EPI_OFF;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -692,13 +673,12 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
     for (int i = threadIdx.x; i < p.E + 2; i += blockDim.x) {
       s_pre[i] = __ldg(p.prefix + i);
       s_offs[i] = __ldg(p.offs + i);
-      if (s_pre_s) s_pre_s[i] = __ldg(p.prefix_small + i);
     }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = p.single_rows >= 0 ? p.single_tiles : s_pre[p.E + 1] + (s_pre_s ? s_pre_s[p.E + 1] : 0);
+  const int total = p.single_rows >= 0 ? p.single_tiles : s_pre[p.E + 1];
 
   if (warp == 0) {
     if (lane == 0) {
@@ -716,7 +696,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
       for (int tile = blockIdx.x;;) {
         if (!FP8 && !tq.put(min(tile, total), abort_flag, p.status, tcode | 11)) break;
         if (tile >= total) break;
-        const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile, s_pre_s);
+        const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
         const bool sh = t.g == p.E;
         const LoadPolicy lp = load_policy(t, pol_keep, pol_stream);
         const uint64_t pol_w = lp.w, pol_a = lp.a;
@@ -780,7 +760,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
       for (int tile = FP8 ? (int)blockIdx.x : tq.take(false, lane, abort_flag, p.status, tcode | 12);
            tile >= 0 && tile < total && ok;
            tile = FP8 ? tile + (int)gridDim.x : tq.take(false, lane, abort_flag, p.status, tcode | 12)) {
-        const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile, s_pre_s);
+        const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
         if (!mbar_wait(tempty + acc, acc_phase ^ 1, abort_flag, p.status, tcode | 2)) break;
         tc_fence_after();
         const uint32_t d0 = tmem_base + acc * Cfg::ACC_COLS;
@@ -831,7 +811,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
     for (int tile = FP8 ? (int)blockIdx.x : tq.take(true, lane, abort_flag, p.status, tcode | 13);
          tile >= 0 && tile < total;
          tile = FP8 ? tile + (int)gridDim.x : tq.take(true, lane, abort_flag, p.status, tcode | 13)) {
-      const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile, s_pre_s);
+      const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
       if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)))
         break;  // the warp stops as one: its TMEM loads are warp-collective
       tc_fence_after();
@@ -903,7 +883,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
     TileQueue tq(tq_id, tq_full, tq_empty);
     for (int tile = tq.take(true, lane, abort_flag, p.status, tcode | 14); tile >= 0 && tile < total && !stop;
          tile = tq.take(true, lane, abort_flag, p.status, tcode | 14)) {
-      const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile, s_pre_s);
+      const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
       const bf16* src[RPT];
       uint32_t live = 0;
 #pragma unroll
@@ -958,7 +938,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
     uint32_t phase = 0, rphase = 0;
     bool stop = false;
     for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
-      const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile, s_pre_s);
+      const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
       const bool sh = t.g == p.E;
       ScaleStreams ss;
       scale_rows(ss, DUAL, sh, t.g, t.n0, t.N, sh ? p.K_s : p.K_r, p.sc_b_r, p.sc_b_s, p.sc_c_r, p.sc_c_s,
@@ -1001,7 +981,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
       uint32_t phase = 0, issued = 0, last_par = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile, s_pre_s);
+        const TileInfo t = decode_tile<BN>(p, s_pre, s_offs, tile);
         const bool sh = t.g == p.E;
         for (int kb = t.kb0; kb < t.kb1; ++kb) {
           if (!mbar_wait(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 8)) {
