@@ -152,7 +152,7 @@ def test_forward_plan_on_the_host():
     assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16") == \
         {"expert_form": "rows", "router_selects": True, "gathered": True}
     assert plan(8192, 8192, 512, 10, 2048, 2048, "bf16", "bf16") == \
-        {"expert_form": "rows", "router_selects": False, "gathered": False}      # 512 experts; x > 32 MiB
+        {"expert_form": "rows", "router_selects": False, "gathered": True}       # 512 experts; x = 128 MiB
     # the pair form from 2048 rows per expert on average; the split form only on request
     assert plan(4095, 256, 2, 1, 256, 256, "bf16", "bf16")["expert_form"] == "rows"
     assert plan(4096, 256, 2, 1, 256, 256, "bf16", "bf16")["expert_form"] == "cta_pairs"
@@ -160,11 +160,11 @@ def test_forward_plan_on_the_host():
     assert plan(2048, 8192, 512, 10, 2048, 2048, "bf16", "fp8")["expert_form"] == "weight_rows"
     assert plan(32, 128, 16, 2, 64, 64, "f32", "f32") == \
         {"expert_form": "simt", "router_selects": False, "gathered": False}
-    # the router selects in its epilogue from 16 token tiles on; the gather stops above 32 MiB of x
+    # the router selects in its epilogue from 16 token tiles on; the gather stops above 256 MiB of x
     assert not plan(1920, 256, 64, 4, 128, 128, "bf16", "bf16")["router_selects"]
     assert plan(1921, 256, 64, 4, 128, 128, "bf16", "bf16")["router_selects"]
-    assert plan(2048, 8192, 128, 8, 256, 256, "bf16", "bf16")["gathered"]       # exactly 32 MiB
-    assert not plan(2049, 8192, 128, 8, 256, 256, "bf16", "bf16")["gathered"]
+    assert plan(16384, 8192, 128, 8, 256, 256, "bf16", "bf16")["gathered"]      # exactly 256 MiB
+    assert not plan(16385, 8192, 128, 8, 256, 256, "bf16", "bf16")["gathered"]
     # the path setting moves the form
     try:
         moe.set_path(4)

@@ -70,7 +70,7 @@ def test_gate_up_input_is_the_token_matrix_where_the_gemm_gathers_it():
     c35 = dict(d=2048, E=256, k=8, I=512, I_s=512, act="bf16", w="bf16")
     pre = dict(d=8192, E=512, k=10, I=2048, I_s=2048, act="bf16", w="bf16")
     assert bench.gathers_rows(c35, 4096)            # x = 16 MiB: rows gathered
-    assert not bench.gathers_rows(pre, 8192)        # x = 128 MiB, larger than L2
+    assert bench.gathers_rows(pre, 8192)            # x = 128 MiB: gathered too (up to 256 MiB)
     assert not bench.gathers_rows(pre, 64)          # decode: the weight-row form
     assert not bench.gathers_rows(dict(c35, w="fp8"), 4096)
     assert bench.forward_plan(pre, 8192)["expert_form"] == "rows"   # the line reports it
@@ -80,13 +80,16 @@ def test_gate_up_input_is_the_token_matrix_where_the_gemm_gathers_it():
     weights = (256 * 2 * 2048 * 512 + 2 * 2048 * 512) * 2
     h = (128 * 256 * 512 + T * 512) * 2
     assert w["gemm_gate_up"]["bytes"] == weights + T * 2048 * 2 + h
-    # without the gather (prefill shape) the dispatched rows are the input
+    # prefill shape, gathered: the token matrix is the input
     counts = [160] * 512
     T = 8192
     w = bench.work_model(pre, counts, T)
     weights = (512 * 2 * 8192 * 2048 + 2 * 8192 * 2048) * 2
     h = (160 * 512 * 2048 + T * 2048) * 2
-    assert w["gemm_gate_up"]["bytes"] == weights + (160 * 512 + T) * 8192 * 2 + h
+    assert w["gemm_gate_up"]["bytes"] == weights + T * 8192 * 2 + h
+    # without the gather (E4M3 weights, row-tiled) the dispatched rows are the input
+    pre8 = dict(pre, w="fp8")
+    assert not bench.gathers_rows(pre8, 8192)
 
 
 def test_reference_arm_prints_one_json_line():
