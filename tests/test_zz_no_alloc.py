@@ -93,3 +93,51 @@ def test_static_router_rejects_candidate_lists_that_do_not_fit():
     torch.cuda.synchronize()
     assert rc == 2
     assert b"scratch" in L.moe_last_error_string()
+
+
+def _router_inputs(moe, T, d, E, k, seed):
+    x = moe_inputs.randn((T, d), "cuda", seed, moe_inputs.X, 1.0, torch.bfloat16)
+    w_r = moe_inputs.randn((E, d), "cuda", seed, moe_inputs.W_R, 0.02, torch.bfloat16)
+    return moe.Problem.make(T, d, E, k, 64, 64, "bf16", "bf16"), x, w_r
+
+
+def test_static_router_leaves_no_state_between_problems_and_allocates_nothing():
+    """The built-in array keeps what the last call left: a large problem whose
+    epilogue-selecting router fills many row-tile counters and candidate lists,
+    then a smaller one of the same router form, must still match the workspace
+    router.  Around the later calls neither the device's free memory nor the
+    caching allocator's reservation moves: the entry point allocates nothing."""
+    import sparse_moe_layer_top_b200 as moe
+    torch.cuda.set_device(0)
+    L = moe.lib()
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    big = _router_inputs(moe, 4096, 2048, 256, 8, 11)
+    small = _router_inputs(moe, 1921, 512, 200, 6, 12)
+    assert moe.forward_plan(big[0])["router_selects"] and moe.forward_plan(small[0])["router_selects"]
+    out = {}
+    for name, (prob, x, w_r) in (("big", big), ("small", small)):
+        ids = torch.empty((prob.T, prob.k), dtype=torch.int32, device="cuda")
+        tw = torch.empty((prob.T, prob.k), dtype=torch.float32, device="cuda")
+        ref = moe.router_topk(prob, x, w_r)
+        out[name] = (prob, x, w_r, ids, tw, ref)
+    torch.cuda.synchronize()
+    # a first call of each problem: kernel modules, the array's address
+    for prob, x, w_r, ids, tw, _ in out.values():
+        assert L.moe_router_topk_static(ctypes.byref(prob), _p(x), _p(w_r), None, _p(ids), _p(tw), stream) == 0
+    torch.cuda.synchronize()
+    for name in ("big", "small", "big", "small"):
+        prob, x, w_r, ids, tw, (ids_ref, w_ref) = out[name]
+        ids.fill_(-7)
+        tw.fill_(-1.0)
+        torch.cuda.synchronize()
+        free0, _ = torch.cuda.mem_get_info()
+        reserved0 = torch.cuda.memory_reserved()
+        rc = L.moe_router_topk_static(ctypes.byref(prob), _p(x), _p(w_r), None, _p(ids), _p(tw), stream)
+        assert rc == 0, L.moe_last_error_string()
+        torch.cuda.synchronize()
+        free1, _ = torch.cuda.mem_get_info()
+        assert torch.cuda.memory_reserved() == reserved0, name
+        assert free1 == free0, "%s: device free memory moved by %d bytes" % (name, free0 - free1)
+        assert moe.device_status()[0] == 0
+        assert torch.equal(ids, ids_ref), name
+        assert (tw - w_ref).abs().max().item() <= TOL_W["bf16"], name
