@@ -192,7 +192,11 @@ def work_model(c, counts, T):
     if c["w"] == "fp8":
         n_sc = (E * 3 * (I // 128) * (d // 128) + sh * 3 * (I_s // 128) * (d // 128)) * 4
         layer["bytes"] += n_sc * active // max(E, 1)
-    return {"active_experts": active, "rows": R, "gemm_gate_up": g1, "gemm_down": g2, "layer": layer}
+    loads = sorted(n for n in counts if n > 0)
+    load = {"max": loads[-1] if loads else 0, "median": loads[len(loads) // 2] if loads else 0,
+            "min": loads[0] if loads else 0}
+    return {"active_experts": active, "rows": R, "expert_rows": load, "gemm_gate_up": g1, "gemm_down": g2,
+            "layer": layer}
 
 
 # ---------------------------------------------------------------- CPU oracle timing
@@ -490,7 +494,8 @@ def layer_roofline(work, step_ms, peaks, peak_src):
             "hbm_frac": lw["bytes"] / st / 1e9 / peaks["hbm_gbs"],
             "tc_frac": lw["flops"] / st / 1e12 / peaks["bf16_tflops"],
             "achieved_gbs": lw["bytes"] / st / 1e9, "achieved_tflops": lw["flops"] / st / 1e12,
-            "active_experts": work["active_experts"], "peak_source": peak_src + " (tensor: burst)"}
+            "active_experts": work["active_experts"], "expert_rows": work["expert_rows"],
+            "peak_source": peak_src + " (tensor: burst)"}
 
 
 def run_companion(args, moe, inp, flush, world, rank, dev, peaks, peak_src):

@@ -309,7 +309,11 @@ MOE_API int moe_last_launch_count(void);
  * launches through this library is bracketed by two CUDA events recorded on
  * its stream; on = 2: only the tensor-core GEMM launches; on = 0: off.
  * Events are created once and reused; at most 4096 launches are recorded
- * until the next read.  Every call clears the record. */
+ * until the next read.  Every call clears the record.  A thread starts in the
+ * mode the environment variable MOE_PROFILE gives (1 or 2), else off.
+ * Independently of this, every entry point and every stage of the fused
+ * forward (moe.router, moe.dispatch, moe.expert_gemms, moe.slot_sum) is an
+ * NVTX range on the host, for nsys and for ncu's NVTX filters. */
 MOE_API moe_status moe_profile_enable(int on);
 
 /* Copy up to `max` recorded launches, in launch order, into ms[] (device

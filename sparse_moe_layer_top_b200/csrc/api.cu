@@ -3,10 +3,12 @@
 // One translation unit: the kernels are included from the headers beside it.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -44,6 +46,27 @@ static moe_status fail(moe_status s, const char* fmt, ...) {
     if (e_ != cudaSuccess) return fail(MOE_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
   } while (0)
 
+// NVTX ranges on the host around every entry point and every stage of the
+// fused forward, for nsys and ncu's NVTX filters (header-only NVTX 3: without
+// a tool attached a range costs a branch).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+  NvtxRange(const NvtxRange&) = delete;
+  NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
+// The profiling mode a thread starts in: MOE_PROFILE=1 (every launch) or 2
+// (the tensor-core GEMMs) in the environment, else off (moe_profile_enable).
+static int env_profile_mode() {
+  static const int m = [] {
+    const char* e = getenv("MOE_PROFILE");
+    const int v = e ? atoi(e) : 0;
+    return v == 1 || v == 2 ? v : 0;
+  }();
+  return m;
+}
+
 // Optional per-launch timing: when enabled, every kernel launch of the
 // calling thread is bracketed by two CUDA events recorded on its stream.
 struct LaunchEvent {
@@ -51,8 +74,8 @@ struct LaunchEvent {
   cudaEvent_t begin, end;
 };
 struct Profiler {
-  bool on = false, pending = false;
-  int mode = 0;
+  bool on = env_profile_mode() != 0, pending = false;
+  int mode = env_profile_mode();
   int used = 0;
   LaunchEvent ev[kProfileCapacity];
   int created = 0;
@@ -1176,6 +1199,7 @@ moe_status moe_device_status(int32_t* detail) {
 
 moe_status moe_router_topk(const moe_problem* p, const void* x, const void* w_router, const float* router_bias,
                            int32_t* topk_ids, float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("moe_router_topk");
   moe_status s = check(p);
   if (s != MOE_OK) return s;
   if (p->T == 0) {
@@ -1208,6 +1232,7 @@ moe_status moe_router_topk(const moe_problem* p, const void* x, const void* w_ro
 moe_status moe_permute(const moe_problem* p, const void* x, const int32_t* topk_ids, const float* topk_w,
                        void* x_perm, int32_t* row_tok, float* row_w, int32_t* pos, int32_t* offs, void* ws,
                        size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("moe_permute");
   moe_status s = check(p);
   if (s != MOE_OK) return s;
   NEED(offs);
@@ -1240,6 +1265,7 @@ moe_status moe_expert_ffn(const moe_problem* p, const void* x_perm, const int32_
                           const void* w_up, const void* w_down, const void* ws_gate, const void* ws_up,
                           const void* ws_down, const float* scales, void* y_perm, void* ws, size_t ws_bytes,
                           void* stream) {
+  NvtxRange nvtx_("moe_expert_ffn");
   moe_status s = check(p);
   if (s != MOE_OK) return s;
   if (p->T == 0) {
@@ -1278,6 +1304,7 @@ moe_status moe_expert_ffn(const moe_problem* p, const void* x_perm, const int32_
 
 moe_status moe_combine(const moe_problem* p, const void* y_perm, const int32_t* pos, const float* topk_w,
                        const int32_t* offs, void* y, void* stream) {
+  NvtxRange nvtx_("moe_combine");
   moe_status s = check(p);
   if (s != MOE_OK) return s;
   if (p->T == 0) {
@@ -1327,6 +1354,7 @@ static moe_status block_forward(const moe_problem* p, const moe_block_options* o
                                 const void* w_up, const void* w_down, const void* ws_gate, const void* ws_up,
                                 const void* ws_down, const float* scales, void* y, int32_t* topk_ids_out,
                                 float* topk_w_out, void* ws, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx_("moe_layer_forward");
   moe_status s = check(p);
   if (s != MOE_OK) return s;
   const void* norm_w = opt ? opt->norm_weight : nullptr;
@@ -1381,22 +1409,32 @@ static moe_status block_forward(const moe_problem* p, const moe_block_options* o
     if (norm_w) xin = wsp + L.xn;
   }
   bool counted;
-  s = launch_router(*p, xin, w_router, router_bias, ids, tw, (float*)(wsp + L.part), counts, &counted, st, dev);
+  {
+    NvtxRange r_("moe.router");
+    s = launch_router(*p, xin, w_router, router_bias, ids, tw, (float*)(wsp + L.part), counts, &counted, st, dev);
+  }
   if (s != MOE_OK) return s;
   Schedule sa, sb;
   schedules(*p, form, &sa, &sb);
   // the row-tiled bf16 gate/up GEMM gathers its rows from the block's input
-  // when that stays L2-resident: the dispatch then writes no copy of them.
-  // Measured: 35B shape (x 16 MB) 0.524 -> 0.484 ms; the prefill shape (x
-  // 128 MB, larger than L2) 7 % slower gathered, so it keeps the copy.
+  // (up to kGatherMaxBytes of it): the dispatch then writes no copy of them.
+  // Measured: 35B shape (x 16 MB) 0.524 -> 0.484 ms; prefill (x 128 MB, in
+  // the panel tile order) 10.80 -> 10.62 ms.
   GatherSrc gs;
   if (gathers_rows(*p, form)) gs = GatherSrc{xin, row_tok};
-  s = launch_dispatch(*p, ids, tw, counted, offs, row_tok, row_w, pos, row_dst, counts, sa, pre_a, sb, pre_b, xin,
-                      gs.x ? nullptr : xp, st, dev, gate);
+  {
+    NvtxRange r_("moe.dispatch");
+    s = launch_dispatch(*p, ids, tw, counted, offs, row_tok, row_w, pos, row_dst, counts, sa, pre_a, sb, pre_b, xin,
+                        gs.x ? nullptr : xp, st, dev, gate);
+  }
   if (s != MOE_OK) return s;
   DownOut o{xp, row_dst, row_w, nullptr};  // the slot rows reuse the dispatched-row buffer
-  s = expert_gemms(*p, form, xp, offs, w, pre_a, pre_b, wsp + L.h, o, st, dev, gs);
+  {
+    NvtxRange r_("moe.expert_gemms");
+    s = expert_gemms(*p, form, xp, offs, w, pre_a, pre_b, wsp + L.h, o, st, dev, gs);
+  }
   if (s != MOE_OK) return s;
+  NvtxRange r_sum_("moe.slot_sum");
   PROF_BEGIN("slot_sum", st);
   if (p->act_dtype == MOE_F32)
     CUDA_TRY(launch(k_slot_sum<float>,
@@ -1428,6 +1466,7 @@ moe_status moe_block_forward(const moe_problem* p, const moe_block_options* opt,
 
 moe_status moe_rmsnorm(const moe_problem* p, const void* x, const void* norm_weight, float eps, void* x_out,
                        void* stream) {
+  NvtxRange nvtx_("moe_rmsnorm");
   moe_status s = check(p);
   if (s != MOE_OK) return s;
   if (!(eps >= 0.f && eps < 1e30f)) return fail(MOE_ERR_INVALID_ARG, "eps must be finite and >= 0");
@@ -1462,6 +1501,7 @@ moe_status moe_forward_plan(const moe_problem* p, int32_t* expert_form, int32_t*
 
 moe_status moe_ep_expand_ids(const int32_t* counts, int32_t G, int32_t E_local, int64_t R, int32_t* ids,
                              void* stream) {
+  NvtxRange nvtx_("moe_ep_expand_ids");
   if (G < 1 || E_local < 1 || (int64_t)G * E_local > kEpMaxBlocks)
     return fail(MOE_ERR_INVALID_ARG, "G = %d, E_local = %d: need G, E_local >= 1 and G * E_local <= %d", G, E_local,
                 kEpMaxBlocks);
@@ -1517,6 +1557,7 @@ static moe_status router_scratch(void** out) {
 extern "C" moe_status moe_router_topk_static(const moe_problem* p, const void* x, const void* w_router,
                                              const float* router_bias, int32_t* topk_ids, float* topk_w,
                                              void* stream) {
+  NvtxRange nvtx_("moe_router_topk_static");
   moe_status s = check(p);
   if (s != MOE_OK) return s;
   if (p->T == 0) {

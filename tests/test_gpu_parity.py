@@ -355,3 +355,27 @@ def test_launch_count_reported(moe):
     _gpu_forward(moe, g)
     # router GEMM, top-k, dispatch (with the row copy), gate/up GEMM, down GEMM, slot sum
     assert moe.last_launch_count() == 6
+
+
+def test_profile_environment_variable_times_every_launch():
+    """MOE_PROFILE=1 starts a thread with per-launch event timing on: the
+    forward's launches come back from moe_profile_read by name, in order."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    child = (
+        "import sys, torch\n"
+        "sys.path.insert(0, sys.argv[1])\n"
+        "import moe_inputs, sparse_moe_layer_top_b200 as moe\n"
+        "inp = moe_inputs.make_inputs(300, 256, 20, 4, 192, 128, seed=1, device='cuda')\n"
+        "moe.MoELayer.from_inputs(inp, max_tokens=300)(inp.x)\n"
+        "names = [n for n, ms in moe.profile_read() if ms >= 0]\n"
+        "print(','.join(names))\n")
+    out = subprocess.run([sys.executable, "-c", child, root], capture_output=True, text=True, timeout=300,
+                         env=dict(os.environ, MOE_PROFILE="1"))
+    assert out.returncode == 0, out.stderr[-3000:]
+    names = out.stdout.strip().splitlines()[-1].split(",")
+    assert names[0].startswith("gemm_tc_router") or names[0] == "router_topk", names
+    assert "dispatch" in names and "gemm_tc_swiglu" in names and "gemm_tc_down" in names, names
+    assert names[-1] == "slot_sum", names
