@@ -803,6 +803,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   a.ldh = ldh;
   a.out_keep = keep_out(Rp * ldh * 2);
   a.panel = panel_of(2 * 128 * (int64_t)p.d * (FP8 ? 1 : 2), cdiv(p.I, 128));  // gate and up rows, 128 columns
+  a.swap_small = FP8 ? 0 : 1;  // tiles of at most 64 rows run with the MMA roles swapped
   a.sc_b_r = sp[0];
   a.sc_b_s = sp[3];
   a.sc_c_r = sp[1];
@@ -844,6 +845,7 @@ static moe_status tc_gemms_t(const moe_problem& p, const void* xp, const int32_t
   b.status = dev->status;
   b.out_keep = keep_out((o.ys ? p.T * (p.k + 1) : Rp) * p.d * 2);
   b.panel = panel_of(256 * (int64_t)std::max(p.I, p.I_s) * (FP8 ? 1 : 2), cdiv(p.d, 256));
+  b.swap_small = FP8 ? 0 : 1;
   if (!FP8) b.sched = pre_b + p.E + 2;
   if (o.ys) {
     b.ys = (bf16*)o.ys;

@@ -59,6 +59,7 @@ struct TcGemmArgs {
   int64_t rows_cap;       // rows of the activation/output buffers; no row at or past it is written
   int out_keep;           // epilogue stores (H, slot rows, out): 1 L2 evict-last, 0 evict-first
   int panel;              // grouped mode: column blocks per panel of the tile order (decode_tile)
+  int swap_small;         // grouped bf16 SwiGLU / SlotStore / Store: tiles of at most kSwapRows rows swap roles
   // single-group mode (single_rows >= 0): one group of single_rows rows that
   // uses the "shared" maps, split along K into ksplit parts
   int single_rows, single_tiles, ksplit, kb_per_split;
@@ -108,7 +109,19 @@ struct TileInfo {
   int g, rows, m0, n0, kb0, kb1, N, split;
   int64_t row0;
   bool rowmajor;  // the group's weight blocks serve several row blocks (see decode_tile)
+  int swap_n;     // 0, or the MMA N of a tile run with swapped roles (see decode_tile)
 };
+
+// A tile with at most kSwapRows rows of its group (the groups of a few rows a
+// skewed batch gives most experts, and the last rows of larger groups) runs
+// with the MMA's roles swapped on the same shared-memory stage: the weight
+// rows are the M = 128 operand and the tile's activation rows the N operand,
+// N = its rows rounded up to 16, so the tensor core does not compute 128 rows
+// for a handful.  The accumulator then holds one weight row (output feature)
+// per TMEM lane and one token per column, and the epilogue writes it
+// transposed.  Which tiles swap depends only on the row counts, so results
+// stay reproducible.
+constexpr int kSwapRows = 64;
 
 // L2 hints of a tile's loads.  In column-block-major order (and in a group of
 // one row tile) a weight block serves the row tiles running beside it and is
@@ -143,6 +156,7 @@ __device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, const int32
     t.kb0 = t.split * p.kb_per_split;
     t.kb1 = min(kbt, t.kb0 + p.kb_per_split);
     t.rowmajor = false;
+    t.swap_n = 0;
     return t;
   }
   const int32_t* pre = s_pre;
@@ -178,6 +192,8 @@ __device__ __forceinline__ TileInfo decode_tile(const TcGemmArgs& p, const int32
   t.m0 = mb * BM;
   t.row0 = (int64_t)r0 + t.m0;
   t.n0 = nb * BN;
+  const int here = min(BM, t.rows - t.m0);
+  t.swap_n = p.swap_small && here <= kSwapRows ? (here + 15) & ~15 : 0;
   t.kb0 = 0;
   t.kb1 = ((sh ? p.K_s : p.K_r) + kBK - 1) / kBK;
   t.split = 0;
@@ -395,6 +411,74 @@ __device__ __forceinline__ void epilogue_rows(const TcGemmArgs& p, const TileInf
     }
     const int n = t.n0 + c * 32;
     store_rows_staged(stg, o, rowp, (int64_t)n * 2, t.N - n, lane, pol);
+  }
+}
+
+// Epilogue of a tile run with swapped roles (TileInfo::swap_n), as run by one
+// epilogue warp of lane quarter q and column group eg (EG = 2): TMEM lane =
+// weight row, column = the tile's token j.  SwiGLU: gate rows at columns
+// [0, N), up rows at [BN, BN + N); warp eg takes tokens 32 eg ..; the lane's
+// output feature is n0 + 32 q + lane.  SlotStore / Store: the two 128-row
+// halves of the 256-row weight tile at columns [0, N) and [128, 128 + N);
+// warp eg takes half eg, every token.  Each token's row is written 32
+// features (64 bytes) per warp.
+template <int BN, int EPI>
+__device__ __forceinline__ void epilogue_swapped(const TcGemmArgs& p, const TileInfo& t, uint32_t tb, int q, int eg,
+                                                 int lane) {
+  const int here = min(kBM, t.rows - t.m0);
+  const uint64_t pol = p.out_keep ? policy_evict_last() : policy_evict_first();
+  if (EPI == kTcSwiGLU) {
+    const int j0 = eg * 32;
+    if (j0 >= here) return;  // uniform over the warp
+    uint32_t a[32], u[32];
+    tmem_ld32(tb + j0, a);
+    tmem_ld32(tb + BN + j0, u);
+    tmem_wait_regs(a);
+    tmem_wait_regs(u);
+    const int n = t.n0 + q * 32 + lane;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int64_t grow = t.row0 + j0 + j;
+      if (j0 + j < here && grow < p.rows_cap && n < t.N) {
+        const float h = silu_f32(__uint_as_float(a[j])) * __uint_as_float(u[j]);
+        asm volatile("st.global.L2::cache_hint.b16 [%0], %1, %2;" ::"l"(p.H + grow * p.ldh + n),
+                     "h"(__bfloat16_as_ushort(__float2bfloat16_rn(h))), "l"(pol)
+                     : "memory");
+      }
+    }
+  } else {
+    const int n = t.n0 + eg * 128 + q * 32 + lane;
+#pragma unroll 1
+    for (int j0 = 0; j0 < here; j0 += 32) {
+      uint32_t a[32];
+      tmem_ld32(tb + eg * 128 + j0, a);
+      tmem_wait_regs(a);
+      // lane j's token: its destination row and routing weight, then broadcast
+      const int64_t gl = t.row0 + j0 + lane;
+      const bool lin = j0 + lane < here && gl < p.rows_cap;
+      int64_t dst = -1;
+      float w = 1.f;
+      if (lin) {
+        if (EPI == kTcSlotStore) {
+          dst = __ldg(p.row_dst + gl);
+          w = __ldg(p.row_w + gl);
+          if (dst >= 0 && !in_range(dst, p.ys_rows, p.status, kSiteSlotRow)) dst = -1;
+        } else {
+          dst = gl;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        const int64_t dr = __shfl_sync(0xffffffffu, dst, j);
+        const float wj = __shfl_sync(0xffffffffu, w, j);
+        if (dr >= 0 && n < t.N) {
+          bf16* op = EPI == kTcSlotStore ? p.ys + dr * p.ldy + n : p.out + dr * p.ldo + n;
+          asm volatile("st.global.L2::cache_hint.b16 [%0], %1, %2;" ::"l"(op),
+                       "h"(__bfloat16_as_ushort(__float2bfloat16_rn(wj * __uint_as_float(a[j])))), "l"(pol)
+                       : "memory");
+        }
+      }
+    }
   }
 }
 
@@ -773,11 +857,27 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
           tc_fence_after();
           const uint32_t sa = smem_u32(smem + stage * Cfg::STAGE_BYTES);
           const uint32_t sb = sa + Cfg::A_BYTES;
+          if (t.swap_n) {
+            // swapped roles: 128 weight rows x the tile's first swap_n
+            // activation rows; gate / up (or the two 128-row halves of the
+            // weight tile) into columns [0, N) and [BN or 128, + N)
+            const uint32_t idesc_s = idesc_bf16(kBM, t.swap_n);
+            constexpr uint32_t half_off = DUAL ? Cfg::B_BYTES : 128 * 128;
+            constexpr uint32_t col_off = DUAL ? BN : 128;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(sa + kk * 32);
-            const uint32_t accum = (kb != t.kb0 || kk != 0);
-            umma_f16(d0, ad, sdesc_sw128(sb + kk * 32), idesc, accum);
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t xd = sdesc_sw128(sa + kk * 32);
+              const uint32_t accum = (kb != t.kb0 || kk != 0);
+              umma_f16(d0, sdesc_sw128(sb + kk * 32), xd, idesc_s, accum);
+              if (DUAL || BN > 128) umma_f16(d0 + col_off, sdesc_sw128(sb + half_off + kk * 32), xd, idesc_s, accum);
+            }
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < kBK / 16; ++kk) {
+              const uint64_t ad = sdesc_sw128(sa + kk * 32);
+              const uint32_t accum = (kb != t.kb0 || kk != 0);
+              umma_f16(d0, ad, sdesc_sw128(sb + kk * 32), idesc, accum);
+            }
           }
           umma_commit(empty + stage);
           if (++stage == STAGES) {
@@ -820,7 +920,10 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
       const bool valid = t.m0 + row < t.rows && grow < p.rows_cap;
       if (EPI == kTcSwiGLU || EPI == kTcSlotStore || EPI == kTcStore) {
         constexpr int CPW = (BN / 32) / EG;  // 32-column chunks per warp, contiguous
-        epilogue_rows<BN, EPI>(p, t, tb, row, eg * CPW, (eg + 1) * CPW, epi_stage + (warp - 2) * 2048, lane);
+        if (t.swap_n)
+          epilogue_swapped<BN, EPI>(p, t, tb, q, eg, lane);
+        else
+          epilogue_rows<BN, EPI>(p, t, tb, row, eg * CPW, (eg + 1) * CPW, epi_stage + (warp - 2) * 2048, lane);
       } else if (EPI == kTcTopK) {
         float* xv = reinterpret_cast<float*>(epi_stage + q * 4096);  // 16 KB: 4 quarters x 16 slots x 32 lanes x 8 B
         int* xe = reinterpret_cast<int*>(epi_stage + q * 4096 + 2048);
