@@ -250,8 +250,8 @@ static moe_status device_info(DeviceInfo** out) {
       d.pair_ctas = 2 * std::max(1, std::min(clusters, d.sms / 2));
     }
     CUDA_TRY(allow_smem(k_gemm_swap8<true, kTcSwiGLU>, Swap8Cfg<true>::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_swap8<false, kTcSlotStore>, Swap8Cfg<false>::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_swap8<false, kTcStore>, Swap8Cfg<false>::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap8<true, kTcSlotStore>, Swap8Cfg<true>::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_swap8<true, kTcStore>, Swap8Cfg<true>::SMEM_BYTES));
     d.ready = true;
   }
   *out = &d;
@@ -950,6 +950,8 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
   b.K_s = p.I_s;
   b.sc_b_r = sp[2];
   b.sc_b_s = sp[5];
+  b.sc_c_r = sp[2];  // E4M3: the second 128-row half of each 256-row tile, same matrix
+  b.sc_c_s = sp[5];
   b.status = dev->status;
   if (o.ys) {
     b.ys = (bf16*)o.ys;
@@ -959,8 +961,8 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
     b.row_w = o.row_w;
     PROF_BEGIN("gemm_tc_down", st);
     if (FP8)
-      CUDA_TRY(launch(k_gemm_swap8<false, kTcSlotStore>,
-                      grid, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
+      CUDA_TRY(launch(k_gemm_swap8<true, kTcSlotStore>,
+                      grid, Swap8Cfg<true>::THREADS, Swap8Cfg<true>::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
     else
       CUDA_TRY(launch(k_gemm_swap<false, kTcSlotStore>,
                       grid, C2::THREADS, C2::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
@@ -970,8 +972,8 @@ static moe_status swap_gemms_t(const moe_problem& p, const void* xp, const int32
     b.ldo = p.d;
     PROF_BEGIN("gemm_tc_store", st);
     if (FP8)
-      CUDA_TRY(launch(k_gemm_swap8<false, kTcStore>,
-                      grid, Swap8Cfg<false>::THREADS, Swap8Cfg<false>::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
+      CUDA_TRY(launch(k_gemm_swap8<true, kTcStore>,
+                      grid, Swap8Cfg<true>::THREADS, Swap8Cfg<true>::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
     else
       CUDA_TRY(launch(k_gemm_swap<false, kTcStore>,
                       grid, C2::THREADS, C2::SMEM_BYTES, st, xR, xS, bR, bS, bR, bS, b));
@@ -1102,9 +1104,9 @@ static void schedules(const moe_problem& p, int form, Schedule* sa, Schedule* sb
   } else if (form == kFormPair) {  // 256-row tiles of CTA pairs
     *sa = Schedule{kPairBM, 128, p.I, p.I_s, 0, 0, 0, 0};
     *sb = Schedule{kPairBM, 256, p.d, p.d, 0, 0, 0, 0};
-  } else if (form == kFormSwap) {  // (token chunk, 128 weight rows) tiles
+  } else if (form == kFormSwap) {  // (token chunk, 128 weight rows) tiles; E4M3 down: 256 rows
     *sa = Schedule{kNCH, 128, p.I, p.I_s, 0, 0, 0, 0};
-    *sb = Schedule{kNCH, 128, p.d, p.d, 0, 0, 0, 0};
+    *sb = Schedule{kNCH, p.w_dtype == MOE_FP8_E4M3_B128 ? 256 : 128, p.d, p.d, 0, 0, 0, 0};
   } else if (form == kFormSplit) {  // pair tiles for the large groups, weight-row tiles for the rest
     *sa = Schedule{kPairBM, 128, p.I, p.I_s, 0, kSplitRows - 1, kNCH, 128};
     *sb = Schedule{kPairBM, 256, p.d, p.d, 0, kSplitRows - 1, kNCH, 128};

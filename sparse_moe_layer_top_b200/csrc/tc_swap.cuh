@@ -47,6 +47,9 @@ struct SwapTile {
   int64_t row0;
 };
 
+// TILE_ROWS: weight rows per tile (128; 256 for the E4M3 down GEMM, whose
+// tile is two 128-row halves sharing the token chunk).
+template <int TILE_ROWS = 128>
 __device__ __forceinline__ SwapTile decode_swap(const TcGemmArgs& p, const int32_t* s_pre, const int32_t* s_offs,
                                                 int tile) {
   SwapTile t;
@@ -61,7 +64,7 @@ __device__ __forceinline__ SwapTile decode_swap(const TcGemmArgs& p, const int32
   const int chc = (t.rows + kNCH - 1) / kNCH;
   const int local = tile - s_pre[t.g];
   t.c0 = (local % chc) * kNCH;
-  t.n0 = (local / chc) * 128;
+  t.n0 = (local / chc) * TILE_ROWS;
   t.row0 = (int64_t)r0 + t.c0;
   const bool sh = t.g == p.E;
   t.N = sh ? p.N_s : p.N_r;
@@ -73,11 +76,16 @@ __device__ __forceinline__ SwapTile decode_swap(const TcGemmArgs& p, const int32
 // thread per weight row (= TMEM lane, output feature), walking the kNCH token
 // columns of each finished tile; with 8 warps two warps share a lane quarter
 // and take one 32-token half each.
+// DUAL with SwiGLU: gate and up accumulators of one 128-row weight tile;
+// DUAL with SlotStore / Store: the accumulators of the two 128-row halves of a
+// 256-row weight tile (output features n0 .. n0 + 255).
 template <bool DUAL, int EPI, int EPI_WARPS, int ACC_BUFS = 2>
 __device__ __forceinline__ void swap_epilogue(const TcGemmArgs& p, const int32_t* s_pre, const int32_t* s_offs,
                                               int total, uint32_t tmem_base, uint64_t* tfull, uint64_t* tempty,
                                               volatile int* abort_flag, unsigned tcode, int warp, int lane) {
   constexpr int ACC_COLS = (DUAL ? 2 : 1) * kNCH;
+  constexpr bool HALVES = DUAL && EPI != kTcSwiGLU;
+  constexpr int TILE_ROWS = HALVES ? 256 : 128;
   constexpr int EG = EPI_WARPS / 4;
   const int eg = (warp - 2) / 4;  // with 8 warps: which 32-token half this warp writes
   const int q = warp & 3;
@@ -85,7 +93,7 @@ __device__ __forceinline__ void swap_epilogue(const TcGemmArgs& p, const int32_t
   int acc = 0;
   uint32_t acc_phase = 0;
   for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
-    const SwapTile t = decode_swap(p, s_pre, s_offs, tile);
+    const SwapTile t = decode_swap<TILE_ROWS>(p, s_pre, s_offs, tile);
     // per-column data of the chunk: lane j holds token columns j and j + 32
     int64_t dst_lo = -1, dst_hi = -1;
     float w_lo = 0.f, w_hi = 0.f;
@@ -105,17 +113,19 @@ __device__ __forceinline__ void swap_epilogue(const TcGemmArgs& p, const int32_t
     if (!__all_sync(0xffffffffu, mbar_wait(tfull + acc, acc_phase, abort_flag, p.status, tcode | 4)))
       break;  // the warp stops as one: its TMEM loads are warp-collective
     tc_fence_after();
-    const uint32_t tb = tmem_base + acc * ACC_COLS + ((uint32_t)(q * 32) << 16);
-    const int n = t.n0 + nl;
-    const bool nvalid = n < t.N;
     const int jmax = min(kNCH, t.rows - t.c0);
 #pragma unroll 1
+    for (int m = 0; m < (HALVES ? 2 : 1); ++m)
+#pragma unroll 1
     for (int half = eg; half < 2 && half * 32 < jmax; half += EG) {  // (jmax is uniform per tile)
+      const uint32_t tb = tmem_base + acc * ACC_COLS + ((uint32_t)(q * 32) << 16) + m * kNCH;
+      const int n = t.n0 + m * 128 + nl;
+      const bool nvalid = n < t.N;
       uint32_t a[32], b[32];
       tmem_ld32(tb + half * 32, a);
-      if (DUAL) tmem_ld32(tb + kNCH + half * 32, b);
+      if (DUAL && !HALVES) tmem_ld32(tb + kNCH + half * 32, b);
       tmem_wait_regs(a);
-      if (DUAL) tmem_wait_regs(b);
+      if (DUAL && !HALVES) tmem_wait_regs(b);
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         const int jj = half * 32 + j;

@@ -59,6 +59,13 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
                  const __grid_constant__ CUtensorMap tmC_r, const __grid_constant__ CUtensorMap tmC_s, TcGemmArgs p) {
   using Cfg = Swap8Cfg<DUAL>;
   constexpr int R = Cfg::RAW_STAGES, A = Cfg::A_STAGES;
+  // DUAL with a SlotStore / Store epilogue (the down GEMM): the two matrices
+  // are the two 128-row halves of a 256-row weight tile of one matrix, so each
+  // K block's handoffs carry twice the weight bytes; the second half's rows
+  // and scales start 128 rows further
+  constexpr bool HALVES = DUAL && EPI != kTcSwiGLU;
+  constexpr int TILE_ROWS = HALVES ? 256 : 128;
+  constexpr int C_ROW = HALVES ? 128 : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   uint64_t* raw_full = reinterpret_cast<uint64_t*>(smem + Cfg::RING_BYTES);
@@ -129,7 +136,7 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
       uint32_t phase = 0, issued = 0, last_par = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const SwapTile t = decode_swap(p, s_pre, s_offs, tile);
+        const SwapTile t = decode_swap<TILE_ROWS>(p, s_pre, s_offs, tile);
         const bool sh = t.g == p.E;
         const int nkb = (sh ? p.K_s : p.K_r) / kBK8;
         for (int kb = 0; kb < nkb; ++kb) {
@@ -145,8 +152,8 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
           if (sh) tma_load_2d(base, &tmB_s, land, k0, t.n0, pol_w);
           else tma_load_3d(base, &tmB_r, land, k0, t.n0, t.g, pol_w);
           if (DUAL) {
-            if (sh) tma_load_2d(base + 128 * kBK8, &tmC_s, land, k0, t.n0, pol_w);
-            else tma_load_3d(base + 128 * kBK8, &tmC_r, land, k0, t.n0, t.g, pol_w);
+            if (sh) tma_load_2d(base + 128 * kBK8, &tmC_s, land, k0, t.n0 + C_ROW, pol_w);
+            else tma_load_3d(base + 128 * kBK8, &tmC_r, land, k0, t.n0 + C_ROW, t.g, pol_w);
           }
           const CUtensorMap* tx = sh ? &tmX_s : &tmX_r;
           tma_load_2d(xdst, tx, land, k0, (int)t.row0, pol_x);
@@ -171,7 +178,7 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
       uint32_t aphase = 0, acc_phase = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const SwapTile t = decode_swap(p, s_pre, s_offs, tile);
+        const SwapTile t = decode_swap<TILE_ROWS>(p, s_pre, s_offs, tile);
         // MMA N = the chunk's token rows rounded up to 16: columns past them are
         // neither computed nor read back
         const uint32_t idesc = idesc_bf16(kBM, min(kNCH, (t.rows - t.c0 + 15) & ~15));
@@ -228,14 +235,17 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
     uint32_t rphase = 0, aphase = 0;
     bool stop = false;
     for (int tile = blockIdx.x; tile < total && !stop; tile += gridDim.x) {
-      const SwapTile t = decode_swap(p, s_pre, s_offs, tile);
+      const SwapTile t = decode_swap<TILE_ROWS>(p, s_pre, s_offs, tile);
       const bool sh = t.g == p.E;
       const int nkb = (sh ? p.K_s : p.K_r) / kBK8;
       // the tile's 128 rows are one scale row block: one fp32 scale per K block
+      // (a second half past the matrix's last row reads zeros and no scale)
       const float* sbase = mat == 0 ? (sh ? p.sc_b_s : p.sc_b_r) : (sh ? p.sc_c_s : p.sc_c_r);
-      const float* srow = sbase + ((sh ? 0 : (int64_t)t.g * (t.N / 128)) + t.n0 / 128) * (int64_t)nkb;
-      float s_cur = __ldg(srow);
-      float s_nxt = nkb > 1 ? __ldg(srow + 1) : 0.f;
+      const int rb0 = t.n0 + mat * C_ROW;
+      const bool rin = rb0 < t.N;
+      const float* srow = sbase + ((sh ? 0 : (int64_t)t.g * (t.N / 128)) + rb0 / 128) * (int64_t)nkb;
+      float s_cur = rin ? __ldg(srow) : 0.f;
+      float s_nxt = rin && nkb > 1 ? __ldg(srow + 1) : 0.f;
       for (int kb = 0; kb < nkb; ++kb) {
         const bool ok = mbar_wait(raw_full + rstage, rphase, abort_flag, p.status, tcode | 5) &&
                         mbar_wait(a_empty + astage, aphase ^ 1, abort_flag, p.status, tcode | 7);
@@ -281,7 +291,7 @@ __global__ void __launch_bounds__(Swap8Cfg<DUAL>::THREADS, 1)
           mbar_arrive(raw_empty + rstage);
         }
         s_cur = s_nxt;
-        s_nxt = kb + 2 < nkb ? __ldg(srow + kb + 2) : 0.f;
+        s_nxt = rin && kb + 2 < nkb ? __ldg(srow + kb + 2) : 0.f;
         if (++astage == A) {
           astage = 0;
           aphase ^= 1;
