@@ -243,7 +243,8 @@ MOE_API moe_status moe_router_topk_static(const moe_problem* p, const void* x, c
  * current moe_set_path, decided on the host (no CUDA call, no device needed):
  * expert_form: 0 SIMT kernels, 1 row-tiled tensor-core GEMMs, 2 weight-row
  * (swap-AB) GEMMs, 3 row-tiled GEMMs on CTA pairs, 4 split (CTA pairs for the
- * groups of 256 rows or more, weight-row GEMMs for the others); router_selects: 1 when the
+ * groups of 256 rows or more, weight-row GEMMs for the others), 5 GEMMs on CTA
+ * pairs with the tokens as the MMA's N; router_selects: 1 when the
  * router's GEMM selects the top k in its epilogue (bf16, E <= 256, at least
  * 16 tiles of 128 tokens), 0 for the split-K GEMM + top-k kernel or the SIMT
  * router; gathered: 1 when the gate/up GEMM reads its rows straight from x.
@@ -267,8 +268,13 @@ MOE_API moe_status moe_forward_plan(const moe_problem* p, int32_t* expert_form, 
  *     rows or more as in 4, the others as in 3, one launch each per
  *     projection (E4M3 weights take the form of 2).  Never chosen
  *     automatically: on skewed prefill batches the row-tiled form of 2 was
- *     faster, since it runs the small groups' tiles among the large ones.
- * 2 to 5 return MOE_ERR_UNSUPPORTED when the types do not allow them. */
+ *     faster, since it runs the small groups' tiles among the large ones;
+ * 6 = tensor-core kernels required, expert GEMMs on 2-CTA clusters with the
+ *     weights as the pair MMA's M = 256 operand and a tile's tokens (up to
+ *     256, the count rounded up to 16) as its N (E4M3 weights take the form
+ *     of 2).  Never chosen automatically: it measured no faster than 2 on
+ *     the skewed prefill batch and than 4 on long groups.
+ * 2 to 6 return MOE_ERR_UNSUPPORTED when the types do not allow them. */
 MOE_API moe_status moe_set_path(int path);
 
 /* Synchronously read and clear the device status word of the current device

@@ -219,7 +219,8 @@ def set_path(path):
     """0 automatic, 1 SIMT kernels only, 2 row-tiled tensor-core expert GEMMs,
     3 weight-row tensor-core expert GEMMs, 4 row-tiled on 2-CTA clusters,
     5 split: groups of 256 rows or more on 2-CTA clusters, the others in
-    weight-row form (on request only)."""
+    weight-row form (on request only), 6 on 2-CTA clusters with the tokens as
+    the MMA's N (tiles of up to 256 rows, padded to 16)."""
     _check(lib().moe_set_path(int(path)))
 
 
@@ -432,7 +433,7 @@ def rmsnorm(prob, x, norm_weight, eps=1e-6, out=None, stream=None):
     return out
 
 
-EXPERT_FORMS = ("simt", "rows", "weight_rows", "cta_pairs", "split")
+EXPERT_FORMS = ("simt", "rows", "weight_rows", "cta_pairs", "split", "cta_pairs_tokens_n")
 
 
 def forward_plan(prob):

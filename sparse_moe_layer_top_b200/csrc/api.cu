@@ -23,6 +23,7 @@
 #include "tc_swap.cuh"
 #include "tc_swap8.cuh"
 #include "tc_pair.cuh"
+#include "tc_pairt.cuh"
 
 using namespace moe;
 
@@ -153,6 +154,7 @@ struct DeviceInfo {
   unsigned* status = nullptr;
   int sms = 0;
   int pair_ctas = 0;  // CTAs of the pair GEMMs: 2 x the 2-CTA clusters that fit at once
+  int pairt_ctas = 0;  // the same for the token-N pair GEMMs
   bool attr_set = false;
 };
 static DeviceInfo g_dev[kMaxDevices];
@@ -177,6 +179,10 @@ using Gemm2F8Cfg = TcGemmCfg<256, false, kFp8Stages, true>;
 constexpr int kPairStages = 6;
 using Pair1Cfg = PairCfg<128, true, kPairStages>;
 using Pair2Cfg = PairCfg<256, false, kPairStages>;
+constexpr int kPairTStages = 6;
+static_assert(kPairTRows == kPairBM, "the token-N pair form shares the pair form's tile schedule");
+using PairT1Cfg = PairTCfg<true, kPairTStages>;
+using PairT2Cfg = PairTCfg<false, kPairTStages>;
 
 // Launch a pair GEMM as 2-CTA clusters.
 template <typename K>
@@ -199,6 +205,28 @@ static cudaError_t launch_pair(K kernel, int ctas, int threads, int smem, cudaSt
   cfg.numAttrs = g_pdl_next ? 2 : 1;
   g_pdl_next = true;
   return cudaLaunchKernelEx(&cfg, kernel, a0, a1, b0, b1, c0, c1, args);
+}
+
+// Launch a token-N pair GEMM as 2-CTA clusters (eight tensor maps).
+template <typename K>
+static cudaError_t launch_pairt(K kernel, int ctas, int threads, int smem, cudaStream_t st, const CUtensorMap* m,
+                                const TcGemmArgs& args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ctas);
+  cfg.blockDim = dim3((unsigned)threads);
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = g_pdl_next ? 2 : 1;
+  g_pdl_next = true;
+  return cudaLaunchKernelEx(&cfg, kernel, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], args);
 }
 
 static moe_status device_info(DeviceInfo** out) {
@@ -248,6 +276,25 @@ static moe_status device_info(DeviceInfo** out) {
       int clusters = 0;
       CUDA_TRY(cudaOccupancyMaxActiveClusters(&clusters, k_gemm_pair<256, false, kPairStages, kTcSlotStore>, &cfg));
       d.pair_ctas = 2 * std::max(1, std::min(clusters, d.sms / 2));
+    }
+    CUDA_TRY(allow_smem(k_gemm_pairt<true, kPairTStages, kTcSwiGLU>, PairT1Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_pairt<false, kPairTStages, kTcSlotStore>, PairT2Cfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_gemm_pairt<false, kPairTStages, kTcStore>, PairT2Cfg::SMEM_BYTES));
+    {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)(d.sms & ~1));
+      cfg.blockDim = dim3((unsigned)PairT1Cfg::THREADS);
+      cfg.dynamicSmemBytes = (size_t)std::max(PairT1Cfg::SMEM_BYTES, PairT2Cfg::SMEM_BYTES);
+      cudaLaunchAttribute at[1];
+      at[0].id = cudaLaunchAttributeClusterDimension;
+      at[0].val.clusterDim.x = 2;
+      at[0].val.clusterDim.y = 1;
+      at[0].val.clusterDim.z = 1;
+      cfg.attrs = at;
+      cfg.numAttrs = 1;
+      int clusters = 0;
+      CUDA_TRY(cudaOccupancyMaxActiveClusters(&clusters, k_gemm_pairt<true, kPairTStages, kTcSwiGLU>, &cfg));
+      d.pairt_ctas = 2 * std::max(1, std::min(clusters, d.sms / 2));
     }
     CUDA_TRY(allow_smem(k_gemm_swap8<true, kTcSwiGLU>, Swap8Cfg<true>::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_swap8<true, kTcSlotStore>, Swap8Cfg<true>::SMEM_BYTES));
@@ -384,7 +431,7 @@ static moe_status choose(bool tc_possible, bool* use_tc) {
 // 256-row tiles waste little on group tails (measured: 12-15 % faster at 4096
 // rows per expert, even at 1024, slower on prefill-sized Zipf-skewed groups);
 // else the row-tiled form.
-enum { kFormSimt = 0, kFormRows = 1, kFormSwap = 2, kFormPair = 3, kFormSplit = 4 };
+enum { kFormSimt = 0, kFormRows = 1, kFormSwap = 2, kFormPair = 3, kFormSplit = 4, kFormPairT = 5 };
 constexpr int kPairRowsPerExpert = 2048;
 constexpr int kSplitRows = 256;
 static moe_status choose_form(const moe_problem& p, int* form) {
@@ -396,6 +443,7 @@ static moe_status choose_form(const moe_problem& p, int* form) {
   else if (g_path == 3) *form = kFormSwap;
   else if (g_path == 4) *form = p.w_dtype == MOE_BF16 ? kFormPair : kFormRows;
   else if (g_path == 5) *form = p.w_dtype == MOE_BF16 ? kFormSplit : kFormRows;
+  else if (g_path == 6) *form = p.w_dtype == MOE_BF16 ? kFormPairT : kFormRows;
   else if (p.T * (int64_t)p.k <= (int64_t)kNCH * p.E) *form = kFormSwap;
   else if (p.w_dtype == MOE_BF16 && p.T * (int64_t)p.k >= (int64_t)kPairRowsPerExpert * p.E) *form = kFormPair;
   else *form = kFormRows;
@@ -1065,6 +1113,97 @@ static moe_status pair_gemms(const moe_problem& p, const void* xp, const int32_t
   return MOE_OK;
 }
 
+// Expert GEMMs on CTA pairs with the tokens as the MMA's N (bf16 weights):
+// tiles of up to 256 dispatched rows, the MMA's N their count rounded up to
+// 16; each CTA loads 128 weight rows and half of the tile's token rows.
+static moe_status pairt_gemms(const moe_problem& p, const void* xp, const int32_t* offs, const ExpertWeights& w,
+                              int32_t* pre_a, int32_t* pre_b, void* H, const DownOut& o, cudaStream_t st,
+                              DeviceInfo* dev) {
+  const int grid = dev->pairt_ctas;
+  const int64_t Rp = rows_total(p), ldh = ldh_of(p);
+  const bool sh = p.I_s > 0;
+  moe_status s;
+  // maps: tokens (small boxes, routed / shared K), tokens (wide boxes), B, C
+  CUtensorMap m[8];
+  CUtensorMap &tR = m[0], &tS = m[1], &uR = m[2], &uS = m[3], &bR = m[4], &bS = m[5], &cR = m[6], &cS = m[7];
+  // gate/up + SwiGLU: each CTA streams 64 gate and 64 up rows of its features
+  if ((s = map2d(&tR, xp, p.d, Rp, p.d, kTokBox)) != MOE_OK) return s;
+  if ((s = map2d(&uR, xp, p.d, Rp, p.d, kTokBoxWide)) != MOE_OK) return s;
+  tS = tR;
+  uS = uR;
+  if ((s = map3d(&bR, w.wg, p.d, p.I, p.E, 64)) != MOE_OK) return s;
+  if ((s = map3d(&cR, w.wu, p.d, p.I, p.E, 64)) != MOE_OK) return s;
+  bS = bR;
+  cS = cR;
+  if (sh) {
+    if ((s = map2d(&bS, w.sg, p.d, p.I_s, p.d, 64)) != MOE_OK) return s;
+    if ((s = map2d(&cS, w.su, p.d, p.I_s, p.d, 64)) != MOE_OK) return s;
+  }
+  TcGemmArgs a{};
+  a.offs = offs;
+  a.prefix = pre_a;
+  a.E = p.E;
+  a.rows_cap = Rp;
+  a.single_rows = -1;
+  a.N_r = p.I;
+  a.N_s = p.I_s;
+  a.K_r = p.d;
+  a.K_s = p.d;
+  a.H = (bf16*)H;
+  a.ldh = ldh;
+  a.out_keep = keep_out(Rp * ldh * 2);
+  a.panel = panel_of(2 * 128 * (int64_t)p.d * 2, cdiv(p.I, 128));
+  a.status = dev->status;
+  PROF_BEGIN("gemm_tc_swiglu", st);
+  CUDA_TRY(launch_pairt(k_gemm_pairt<true, kPairTStages, kTcSwiGLU>, grid, PairT1Cfg::THREADS, PairT1Cfg::SMEM_BYTES,
+                        st, m, a));
+  LAUNCH_CHECK("gemm_tc_swiglu", st);
+  // down: each CTA streams 128 rows of a 256-row weight block
+  if ((s = map2d(&tR, H, p.I, Rp, ldh, kTokBox)) != MOE_OK) return s;
+  if ((s = map2d(&uR, H, p.I, Rp, ldh, kTokBoxWide)) != MOE_OK) return s;
+  tS = tR;
+  uS = uR;
+  if (sh && (s = map2d(&tS, H, p.I_s, Rp, ldh, kTokBox)) != MOE_OK) return s;
+  if (sh && (s = map2d(&uS, H, p.I_s, Rp, ldh, kTokBoxWide)) != MOE_OK) return s;
+  if ((s = map3d(&bR, w.wd, p.I, p.d, p.E, 128)) != MOE_OK) return s;
+  bS = bR;
+  if (sh && (s = map2d(&bS, w.sd, p.I_s, p.d, p.I_s, 128)) != MOE_OK) return s;
+  cR = bR;
+  cS = bS;
+  TcGemmArgs b{};
+  b.offs = offs;
+  b.prefix = pre_b;
+  b.E = p.E;
+  b.rows_cap = Rp;
+  b.single_rows = -1;
+  b.N_r = p.d;
+  b.N_s = p.d;
+  b.K_r = p.I;
+  b.K_s = p.I_s;
+  b.status = dev->status;
+  b.out_keep = keep_out((o.ys ? p.T * (p.k + 1) : Rp) * p.d * 2);
+  b.panel = panel_of(256 * (int64_t)std::max(p.I, p.I_s) * 2, cdiv(p.d, 256));
+  if (o.ys) {
+    b.ys = (bf16*)o.ys;
+    b.ys_rows = p.T * (p.k + 1);
+    b.ldy = p.d;
+    b.row_dst = o.row_dst;
+    b.row_w = o.row_w;
+    PROF_BEGIN("gemm_tc_down", st);
+    CUDA_TRY(launch_pairt(k_gemm_pairt<false, kPairTStages, kTcSlotStore>, grid, PairT2Cfg::THREADS,
+                          PairT2Cfg::SMEM_BYTES, st, m, b));
+    LAUNCH_CHECK("gemm_tc_down", st);
+  } else {
+    b.out = (bf16*)o.out;
+    b.ldo = p.d;
+    PROF_BEGIN("gemm_tc_store", st);
+    CUDA_TRY(launch_pairt(k_gemm_pairt<false, kPairTStages, kTcStore>, grid, PairT2Cfg::THREADS,
+                          PairT2Cfg::SMEM_BYTES, st, m, b));
+    LAUNCH_CHECK("gemm_tc_store", st);
+  }
+  return MOE_OK;
+}
+
 // The split form: the large groups' tiles are counted in pre_a / pre_b, the
 // others' in the second prefix of each (pre + E + 3); each kernel walks its
 // own list and writes its own rows of H and of the slot rows.  A down GEMM
@@ -1092,6 +1231,7 @@ static moe_status expert_gemms(const moe_problem& p, int form, const void* xp, c
   if (form == kFormRows) return tc_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev, g);
   if (form == kFormPair) return pair_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
   if (form == kFormSplit) return split_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
+  if (form == kFormPairT) return pairt_gemms(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
   if (p.act_dtype == MOE_F32) return simt_gemms<float, float>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
   if (p.w_dtype == MOE_BF16) return simt_gemms<bf16, bf16>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
   return simt_gemms<bf16, uint8_t>(p, xp, offs, w, pre_a, pre_b, H, o, st, dev);
@@ -1101,7 +1241,7 @@ static void schedules(const moe_problem& p, int form, Schedule* sa, Schedule* sb
   if (form == kFormRows) {
     *sa = sched_tc(128, p.I, p.I_s);
     *sb = sched_tc(256, p.d, p.d);
-  } else if (form == kFormPair) {  // 256-row tiles of CTA pairs
+  } else if (form == kFormPair || form == kFormPairT) {  // 256-row tiles of CTA pairs
     *sa = Schedule{kPairBM, 128, p.I, p.I_s, 0, 0, 0, 0};
     *sb = Schedule{kPairBM, 256, p.d, p.d, 0, 0, 0, 0};
   } else if (form == kFormSwap) {  // (token chunk, 128 weight rows) tiles; E4M3 down: 256 rows
@@ -1138,7 +1278,7 @@ size_t moe_workspace_size(const moe_problem* p) { return check(p) == MOE_OK ? la
 size_t moe_stage_workspace_size(const moe_problem* p) { return check(p) == MOE_OK ? layout(*p, false).total : 0; }
 
 moe_status moe_set_path(int path) {
-  if (path < 0 || path > 5) return fail(MOE_ERR_INVALID_ARG, "path %d is not 0, 1, 2, 3, 4 or 5", path);
+  if (path < 0 || path > 6) return fail(MOE_ERR_INVALID_ARG, "path %d is not 0, 1, 2, 3, 4, 5 or 6", path);
   g_path = path;
   return MOE_OK;
 }

@@ -276,9 +276,14 @@ __device__ __forceinline__ uint32_t mapa_rank(const void* p, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
   return r;
 }
-// Arrive on an mbarrier of another CTA of the cluster (release, cluster scope).
-__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+// Arrive on an mbarrier of this CTA or of the peer (a shared::cluster address)
+// with release at CTA scope: enough for an epilogue warp handing an
+// accumulator back to the MMA issuer -- its TMEM reads are complete
+// (tcgen05.wait::ld) and fenced (tcgen05.fence::before_thread_sync) -- and,
+// unlike a cluster-scope release, it does not wait for the warp's global
+// stores to complete.
+__device__ __forceinline__ void mbar_arrive_cta_scope(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
 __device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
   uint32_t ok;

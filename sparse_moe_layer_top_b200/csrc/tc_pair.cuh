@@ -233,7 +233,7 @@ __global__ void __launch_bounds__(PairCfg<BN, DUAL, STAGES>::THREADS, 1)
       epilogue_rows<BN, EPI>(p, t, tb, row, eg * CPW, (eg + 1) * CPW, epi_stage + (warp - 2) * 2048, lane);
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tempty0 + acc * 8);
+      if (lane == 0) mbar_arrive_cta_scope(tempty0 + acc * 8);
       if (++acc == 2) {
         acc = 0;
         acc_phase ^= 1;

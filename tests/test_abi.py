@@ -101,7 +101,7 @@ def test_host_rejects_before_any_launch():
 
 
 def test_set_path_validates():
-    assert moe.lib().moe_set_path(6) == 1
+    assert moe.lib().moe_set_path(7) == 1
     assert moe.lib().moe_set_path(5) == 0
     assert moe.lib().moe_set_path(-1) == 1
     assert moe.lib().moe_set_path(0) == 0
@@ -171,6 +171,10 @@ def test_forward_plan_on_the_host():
         assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16")["expert_form"] == "cta_pairs"
         moe.set_path(5)
         assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16")["expert_form"] == "split"
+        assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "fp8")["expert_form"] == "rows"
+        moe.set_path(6)
+        assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16") == \
+            {"expert_form": "cta_pairs_tokens_n", "router_selects": True, "gathered": False}
         assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "fp8")["expert_form"] == "rows"
         moe.set_path(1)
         assert plan(4096, 2048, 256, 8, 512, 512, "bf16", "bf16") == \

@@ -66,7 +66,7 @@ CASES = {
 
 
 @pytest.mark.parametrize("opts", ["norm", "gate", "norm_gate"])
-@pytest.mark.parametrize("path", [0, 1, 2, 3, 4, 5])
+@pytest.mark.parametrize("path", [0, 1, 2, 3, 4, 5, 6])
 @pytest.mark.parametrize("case", list(CASES))
 def test_block_with_options_matches_oracle(moe, case, path, opts):
     T, d, E, k, I, I_s, act, w, bias = CASES[case]

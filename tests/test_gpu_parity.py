@@ -100,7 +100,7 @@ def _gpu_forward(moe, g):
 
 # 0 automatic, 1 SIMT kernels, 2 row-tiled tensor-core GEMMs, 3 weight-row tensor-core GEMMs,
 # 4 row-tiled GEMMs on CTA pairs (256-row tiles; E4M3 weights take the row-tiled form)
-@pytest.mark.parametrize("path", [0, 1, 2, 3, 4, 5])
+@pytest.mark.parametrize("path", [0, 1, 2, 3, 4, 5, 6])
 @pytest.mark.parametrize("case", list(FORWARD_CASES))
 def test_forward_matches_oracle(moe, case, path):
     inp = _make(case)
@@ -207,7 +207,7 @@ def _random_dispatch(E, sizes, d, act, seed):
     return x_perm, offs, T, R
 
 
-@pytest.mark.parametrize("path", [0, 1, 2, 3, 4, 5])
+@pytest.mark.parametrize("path", [0, 1, 2, 3, 4, 5, 6])
 @pytest.mark.parametrize("sizes_kind", ["ragged", "one_hot_expert", "empty_shared"])
 def test_expert_ffn_matches_oracle(moe, sizes_kind, path):
     E, d, I, I_s = 12, 256, 192, 128
@@ -235,7 +235,7 @@ def test_expert_ffn_matches_oracle(moe, sizes_kind, path):
             assert rel_l2(got[o[gi]:o[gi + 1]], ref[o[gi]:o[gi + 1]]) <= TOL["bf16"], "group %d" % gi
 
 
-@pytest.mark.parametrize("path", [0, 1, 2, 3, 4, 5])
+@pytest.mark.parametrize("path", [0, 1, 2, 3, 4, 5, 6])
 def test_expert_ffn_fp8_matches_oracle(moe, path):
     """E4M3 weights with 128 x 128 block scales through the expert stage alone:
     groups of 0, 1, 63, 64, 65 and 130 rows (token chunks of 64 split inside a
@@ -295,7 +295,7 @@ def test_paths_agree(moe, w):
     inp = moe_inputs.make_inputs(200, 512, 24, 4, 256, 256, act="bf16", w=w, seed=2)
     g = to_device(inp, "cuda")
     out = []
-    for path in (1, 2, 3, 4, 5):
+    for path in (1, 2, 3, 4, 5, 6):
         moe.set_path(path)
         y, ids, tw = _gpu_forward(moe, g)
         out.append((y, ids))
@@ -310,7 +310,7 @@ def test_paths_agree_35b_shape(moe):
     inp = _make("bf16_35b_shape_T256", seed=1)
     g = to_device(inp, "cuda")
     out = []
-    for path in (1, 2, 3, 4, 5):
+    for path in (1, 2, 3, 4, 5, 6):
         moe.set_path(path)
         y, ids, tw = _gpu_forward(moe, g)
         out.append(y)
@@ -331,7 +331,7 @@ def test_out_of_range_expert_id_sets_device_status(moe):
     assert moe.device_status()[0] == 0  # reading clears it
 
 
-@pytest.mark.parametrize("path", [0, 1, 2, 3, 4, 5])
+@pytest.mark.parametrize("path", [0, 1, 2, 3, 4, 5, 6])
 @pytest.mark.parametrize("case", ["bf16_multi_tile", "bf16_fused_router", "bf16_auto_pair", "fp8_multi_tile"])
 def test_repeat_calls_are_bit_identical(moe, case, path):
     """No floating-point atomics anywhere in the forward: the router sums its
