@@ -48,7 +48,9 @@ struct PairTCfg {
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int RING_BYTES = STAGES * STAGE_BYTES;
   static constexpr int EPI_WARPS = 8;
-  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  // two TMA producer warps (0 and the last one), taking alternate K blocks
+  static constexpr int PRODUCER2_WARP = 2 + EPI_WARPS;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS + 32;
   static constexpr int ACC_COLS = kPairTRows;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
   static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8 + 16;
@@ -280,13 +282,18 @@ __global__ void __launch_bounds__(PairTCfg<DUAL, STAGES>::THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total = s_pre[p.E + 1];
 
-  if (warp == 0) {
+  if (warp == 0 || warp == Cfg::PRODUCER2_WARP) {
     if (lane == 0) {
-      // ------------------------------------------------ TMA producer (both ranks, own tiles only)
+      // ------------------------------------------------ TMA producers (both ranks, own tiles only)
+      // producer `which` takes the K blocks whose running index over the
+      // pair's tiles is `which` modulo 2 (ring stages of one parity): a single
+      // issuing thread completes a TMA box only every few hundred ns
+      const unsigned which = warp == 0 ? 0u : 1u;
       const uint64_t pol_keep = policy_evict_last(), pol_stream = policy_evict_first();
       const uint32_t full0 = mapa_rank(full, 0);
       int stage = 0;
       uint32_t phase = 0, issued = 0, last_par = 0;
+      unsigned g = 0;  // running K-block index
       bool ok = true;
       for (int tile = pair; tile < total && ok; tile += npairs) {
         const TileInfo t = decode_tile<BN, kPairTRows>(p, s_pre, s_offs, tile);
@@ -300,7 +307,10 @@ __global__ void __launch_bounds__(PairTCfg<DUAL, STAGES>::THREADS, 1)
         const int trow = (int)t.row0 + (int)rank * s.nh;  // this CTA's first token row
         const int wrow = t.n0 + (int)rank * (DUAL ? 64 : 128);
         const uint32_t tx = 2u * (uint32_t)(Cfg::A_BYTES + s.boxes * s.box_rows * kBK * 2);
-        for (int kb = t.kb0; kb < t.kb1; ++kb) {
+        for (int kb = t.kb0; kb < t.kb1; ++kb, ++g) {
+          if ((g & 1u) != which) continue;
+          stage = (int)(g % STAGES);
+          phase = (g / STAGES) & 1u;
           if (!mbar_wait_cluster(empty + stage, phase ^ 1, abort_flag, p.status, tcode | 1)) {
             ok = false;
             break;
@@ -325,10 +335,6 @@ __global__ void __launch_bounds__(PairTCfg<DUAL, STAGES>::THREADS, 1)
             tma_load_2d_pair(sb + b * s.box_rows * kBK * 2, tok, land, kb * kBK, trow + b * s.box_rows, lp.a);
           issued |= 1u << stage;
           last_par = (last_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
-            stage = 0;
-            phase ^= 1;
-          }
         }
       }
       // copies in flight must land before the CTA exits (see k_gemm_pair)
