@@ -24,6 +24,7 @@
 #include "tc_swap8.cuh"
 #include "tc_pair.cuh"
 #include "tc_pairt.cuh"
+#include "router_kc.cuh"
 
 using namespace moe;
 
@@ -171,8 +172,9 @@ using Gemm1Cfg = TcGemmCfg<128, true, 4>;
 using Gemm1GCfg = TcGemmCfg<128, true, 4, false, true>;  // A rows gathered from the token matrix
 using Gemm2Cfg = TcGemmCfg<256, false, 4>;
 // the router that selects in its epilogue: 64-expert column tiles, 8 stages
-constexpr int kTopkBN = 64, kTopkStages = 8;
-using TopkCfg = TcGemmCfg<kTopkBN, false, kTopkStages>;
+// the router with the selection in its epilogue: experts in column tiles of 64
+// (one per CTA of the K-split router's cluster)
+constexpr int kTopkBN = 64;
 constexpr int kFp8Stages = 2;
 using Gemm1F8Cfg = TcGemmCfg<128, true, kFp8Stages, true>;
 using Gemm2F8Cfg = TcGemmCfg<256, false, kFp8Stages, true>;
@@ -229,6 +231,28 @@ static cudaError_t launch_pairt(K kernel, int ctas, int threads, int smem, cudaS
   return cudaLaunchKernelEx(&cfg, kernel, m[0], m[1], m[2], m[3], m[4], m[5], m[6], m[7], args);
 }
 
+// Launch the K-split router as 4-CTA clusters.
+template <typename K>
+static cudaError_t launch_router_kc(K kernel, int ctas, cudaStream_t st, const CUtensorMap& x, const CUtensorMap& w,
+                                    const TcGemmArgs& args, int npad) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)ctas);
+  cfg.blockDim = dim3((unsigned)RouterKcCfg::THREADS);
+  cfg.dynamicSmemBytes = (size_t)RouterKcCfg::SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute at[2];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = kRouterKcCtas;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = g_pdl_next ? 2 : 1;
+  g_pdl_next = true;
+  return cudaLaunchKernelEx(&cfg, kernel, x, w, args, npad);
+}
+
 static moe_status device_info(DeviceInfo** out) {
   int dev = 0;
   CUDA_TRY(cudaGetDevice(&dev));
@@ -250,7 +274,6 @@ static moe_status device_info(DeviceInfo** out) {
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcSlotStore>, Gemm2Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcStore>, Gemm2Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, 4, kTcLogits>, Gemm2Cfg::SMEM_BYTES));
-    CUDA_TRY(allow_smem(k_gemm_tc<kTopkBN, false, kTopkStages, kTcTopK>, TopkCfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<128, true, kFp8Stages, kTcSwiGLU, true>, Gemm1F8Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, kFp8Stages, kTcSlotStore, true>, Gemm2F8Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_tc<256, false, kFp8Stages, kTcStore, true>, Gemm2F8Cfg::SMEM_BYTES));
@@ -277,6 +300,8 @@ static moe_status device_info(DeviceInfo** out) {
       CUDA_TRY(cudaOccupancyMaxActiveClusters(&clusters, k_gemm_pair<256, false, kPairStages, kTcSlotStore>, &cfg));
       d.pair_ctas = 2 * std::max(1, std::min(clusters, d.sms / 2));
     }
+    CUDA_TRY(allow_smem(k_router_kc<8>, RouterKcCfg::SMEM_BYTES));
+    CUDA_TRY(allow_smem(k_router_kc<16>, RouterKcCfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_pairt<true, kPairTStages, kTcSwiGLU>, PairT1Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_pairt<false, kPairTStages, kTcSlotStore>, PairT2Cfg::SMEM_BYTES));
     CUDA_TRY(allow_smem(k_gemm_pairt<false, kPairTStages, kTcStore>, PairT2Cfg::SMEM_BYTES));
@@ -588,8 +613,9 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
     // every logit of a token in TMEM across the row tile's column tiles:
     // select in the epilogue
     const TopkScratch ts = topk_scratch(p);
-    CUtensorMap bw64;
-    if ((s = map2d(&bw64, wr, p.d, p.E, p.d, kTopkBN)) != MOE_OK) return s;
+    const int npad = std::max(16, (int)align_up((size_t)p.E, 16));  // the MMA's N: every expert
+    CUtensorMap bwn;
+    if ((s = map2d(&bwn, wr, p.d, p.E, p.d, (uint32_t)npad)) != MOE_OK) return s;
     char* scratch = reinterpret_cast<char*>(part);
     // the row-tile counters: after the chunk histograms when there are some
     // (one memset for both; kChunkTokens == kBM, so there is one counter
@@ -621,8 +647,9 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
     a.cand_e = reinterpret_cast<int32_t*>(scratch + ts.e_off);
     a.status = dev->status;
     PROF_BEGIN("gemm_tc_router", st);
-    CUDA_TRY(launch(k_gemm_tc<kTopkBN, false, kTopkStages, kTcTopK>, std::min(a.single_tiles, dev->sms),
-                    TopkCfg::THREADS, TopkCfg::SMEM_BYTES, st, ax, ax, bw64, bw64, bw64, bw64, a));
+    const int ctas = (int)ts.row_tiles * kRouterKcCtas;
+    if (p.k <= 8) CUDA_TRY(launch_router_kc(k_router_kc<8>, ctas, st, ax, bwn, a, npad));
+    else CUDA_TRY(launch_router_kc(k_router_kc<16>, ctas, st, ax, bwn, a, npad));
     LAUNCH_CHECK("gemm_tc_router", st);
     *counted = counts != nullptr;
     return MOE_OK;

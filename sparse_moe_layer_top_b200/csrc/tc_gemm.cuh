@@ -24,7 +24,8 @@
 //                           applied and the row put back in (token, slot) order
 //                 Store     out[r, n] = D -> bf16
 //                 Logits    part[split][r, n] = D (+ nothing) -> fp32
-//                 TopK      the router's softmax top-k of D + bias per row
+//               (the router's top-k selection from TMEM, topk_epilogue below,
+//               runs in the K-split router of router_kc.cuh)
 //   warps 10..13 (GATHER only) fetch the A rows straight from the token
 //               matrix by row index (cp.async, 128-byte swizzle written by
 //               hand): the gate/up GEMM of the fused forward needs no
@@ -74,15 +75,15 @@ struct TcGemmArgs {
   int64_t ldo;
   float* part;            // Logits output [ksplit][rows, ldp]
   int64_t ldp, part_stride;
-  // TopK (router with selection, one N tile, no K split): topk_ids / topk_w
-  // [rows, topk] and the 128-row chunk histograms counts[rows / 128][N_s]
-  // (may be NULL); bias [N_s] fp32 (may be NULL) is added to the logits
+  // top-k selection (topk_epilogue): topk_ids / topk_w [rows, topk] and the
+  // 128-row chunk histograms counts[rows / 128][N_s] (may be NULL); bias [N_s]
+  // fp32 (may be NULL) is added to the logits
   int topk;
   int32_t* ids;
   float* tw;
   const float* bias;
   int32_t* counts;
-  // TopK over several column tiles: each tile's kept (logit, expert) pairs of a
+  // selection over several column tiles: each tile's kept (logit, expert) pairs of a
   // token go to cand_v / cand_e [row tile][column tile][kMaxK slots][kBM rows];
   // cand_cnt [row tile][4 lane quarters] (zeroed before the launch) counts the
   // tiles done, and the last one merges the lists and writes the outputs
@@ -906,7 +907,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
     const int q = warp & 3;
     const int row = q * 32 + lane;
     int acc = 0;
-    uint32_t acc_phase = 0, hpar = 0;
+    uint32_t acc_phase = 0;
     TileQueue tq(tq_id, tq_full, tq_empty);
     for (int tile = FP8 ? (int)blockIdx.x : tq.take(true, lane, abort_flag, p.status, tcode | 13);
          tile >= 0 && tile < total;
@@ -924,16 +925,6 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
           epilogue_swapped<BN, EPI>(p, t, tb, q, eg, lane);
         else
           epilogue_rows<BN, EPI>(p, t, tb, row, eg * CPW, (eg + 1) * CPW, epi_stage + (warp - 2) * 2048, lane);
-      } else if (EPI == kTcTopK) {
-        float* xv = reinterpret_cast<float*>(epi_stage + q * 4096);  // 16 KB: 4 quarters x 16 slots x 32 lanes x 8 B
-        int* xe = reinterpret_cast<int*>(epi_stage + q * 4096 + 2048);
-        const bool ok =
-            p.topk <= 8 ? topk_epilogue<BN, EG, 8>(p, t, tb, eg, row, grow, valid, xv, xe, hfull + q, hempty + q, hpar,
-                                                   abort_flag, tcode | 9, lane)
-                        : topk_epilogue<BN, EG, 16>(p, t, tb, eg, row, grow, valid, xv, xe, hfull + q, hempty + q, hpar,
-                                                    abort_flag, tcode | 9, lane);
-        hpar ^= 1;
-        if (!ok) break;
       } else if (EPI == kTcLogits) {
         float* dst = p.part + (int64_t)t.split * p.part_stride + grow * p.ldp;
 #pragma unroll 1

@@ -62,11 +62,6 @@ struct PairTCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory");
 };
 
-// Named barrier of `threads` threads (ids 1..15; 0 is __syncthreads).
-__device__ __forceinline__ void named_bar_sync(int id, int threads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
-}
-
 // Token rows of a tile: `here` real ones, the MMA's N (here rounded up to
 // 16), and the rows each CTA holds (N / 2), loaded in kTokBox-row boxes, or
 // in one kTokBoxWide-row box when there are more than 96 (fewer TMA issues).
