@@ -227,8 +227,8 @@ MOE_API moe_status moe_ep_expand_ids(const int32_t* counts, int32_t G, int32_t E
  *   - Problems whose scratch needs more than that are rejected with
  *     MOE_ERR_UNSUPPORTED before anything is launched: about
  *     splits * T * roundup(E, 32) * 4 bytes of split-K partials (e.g. T = 8192
- *     with E = 512), or T * ceil(E / 64) * 128 bytes of candidate lists when
- *     the router selects in its GEMM epilogue (E <= 256, T >= 1921).
+ *     with E = 512).  The router that selects in its GEMM epilogue (E <= 256,
+ *     T >= 1921) uses no scratch, so it takes any T.
  *   - The first call on a device looks up that device's copy of the array
  *     (a one-time set-up); make it before any stream capture.
  *   - Every call uses the same array and leaves its contents behind; calls

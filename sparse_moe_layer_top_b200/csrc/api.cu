@@ -172,9 +172,6 @@ using Gemm1Cfg = TcGemmCfg<128, true, 4>;
 using Gemm1GCfg = TcGemmCfg<128, true, 4, false, true>;  // A rows gathered from the token matrix
 using Gemm2Cfg = TcGemmCfg<256, false, 4>;
 // the router that selects in its epilogue: 64-expert column tiles, 8 stages
-// the router with the selection in its epilogue: experts in column tiles of 64
-// (one per CTA of the K-split router's cluster)
-constexpr int kTopkBN = 64;
 constexpr int kFp8Stages = 2;
 using Gemm1F8Cfg = TcGemmCfg<128, true, kFp8Stages, true>;
 using Gemm2F8Cfg = TcGemmCfg<256, false, kFp8Stages, true>;
@@ -508,25 +505,9 @@ static RouterSplit router_split(const moe_problem& p) {
 
 // Router scratch: the split-K logit partials, or for the fused router the
 // per-(row tile, lane quarter) counters followed by the candidate lists.
-struct TopkScratch {
-  int64_t row_tiles;
-  int ntc;
-  size_t cnt_off, v_off, e_off, bytes;
-};
-static TopkScratch topk_scratch(const moe_problem& p) {
-  TopkScratch t;
-  t.row_tiles = cdiv(std::max<int64_t>(p.T, 1), kBM);
-  t.ntc = (int)cdiv(p.E, kTopkBN);
-  const size_t list = t.ntc > 1 ? (size_t)t.row_tiles * t.ntc * kMaxK * kBM * 4 : 0;
-  t.cnt_off = 0;
-  t.v_off = align_up((size_t)t.row_tiles * 4 * 4, 256);
-  t.e_off = t.v_off + align_up(list, 256);
-  t.bytes = t.e_off + list;
-  return t;
-}
 static size_t router_scratch_bytes(const moe_problem& p) {
   if (p.act_dtype != MOE_BF16) return 0;
-  if (router_fused(p)) return topk_scratch(p).bytes;
+  if (router_fused(p)) return 0;
   const RouterSplit rs = router_split(p);
   return (size_t)rs.ksplit * p.T * rs.ldp * 4;
 }
@@ -555,7 +536,7 @@ static Layout layout(const moe_problem& p, bool forward) {
   const int64_t n = p.T * p.k, Rp = rows_total(p);
   const size_t ab = esize(p.act_dtype);
   // chunk histograms, then the fused router's row-tile counters (one memset clears both)
-  L.counts = take(n_chunks(p) * p.E * 4 + n_chunks(p) * 4 * 4);
+  L.counts = take(n_chunks(p) * p.E * 4);
   // tile prefix [E+2], the GEMM's tile-claim counter, the small groups' prefix [E+2]
   L.pre_a = take((2 * p.E + 5) * 4);
   L.pre_b = take((2 * p.E + 5) * 4);
@@ -610,22 +591,15 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
   if ((s = map2d(&ax, x, p.d, p.T, p.d, kBM)) != MOE_OK) return s;
   if ((s = map2d(&bw, wr, p.d, p.E, p.d, kRouterBN)) != MOE_OK) return s;
   if (router_fused(p)) {
-    // every logit of a token in TMEM across the row tile's column tiles:
-    // select in the epilogue
-    const TopkScratch ts = topk_scratch(p);
+    // every logit of a row tile in one 4-CTA cluster: select in the epilogue
+    // (no scratch: the partials and lists move through the cluster's shared
+    // memory); the chunk histograms are counted with atomics
+    const int64_t row_tiles = cdiv(p.T, kBM);
     const int npad = std::max(16, (int)align_up((size_t)p.E, 16));  // the MMA's N: every expert
     CUtensorMap bwn;
     if ((s = map2d(&bwn, wr, p.d, p.E, p.d, (uint32_t)npad)) != MOE_OK) return s;
-    char* scratch = reinterpret_cast<char*>(part);
-    // the row-tile counters: after the chunk histograms when there are some
-    // (one memset for both; kChunkTokens == kBM, so there is one counter
-    // quadruple per chunk), else in the scratch
-    int32_t* cnt = counts ? counts + n_chunks(p) * p.E : reinterpret_cast<int32_t*>(scratch + ts.cnt_off);
     if (counts) {
-      CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * (p.E + 4) * 4, st));
-      pdl_reset();
-    } else if (ts.ntc > 1) {
-      CUDA_TRY(cudaMemsetAsync(cnt, 0, (size_t)ts.row_tiles * 4 * 4, st));
+      CUDA_TRY(cudaMemsetAsync(counts, 0, (size_t)n_chunks(p) * p.E * 4, st));
       pdl_reset();
     }
     TcGemmArgs a{};
@@ -633,21 +607,14 @@ static moe_status launch_router(const moe_problem& p, const void* x, const void*
     a.N_s = p.E;
     a.K_s = p.d;
     a.rows_cap = p.T;
-    a.single_rows = (int)p.T;
-    a.single_tiles = (int)(ts.row_tiles * ts.ntc);
-    a.ksplit = 1;
-    a.kb_per_split = (int)cdiv(p.d, kBK);
     a.topk = p.k;
     a.ids = ids;
     a.tw = tw;
     a.bias = bias;
     a.counts = counts;
-    a.cand_cnt = cnt;
-    a.cand_v = reinterpret_cast<float*>(scratch + ts.v_off);
-    a.cand_e = reinterpret_cast<int32_t*>(scratch + ts.e_off);
     a.status = dev->status;
     PROF_BEGIN("gemm_tc_router", st);
-    const int ctas = (int)ts.row_tiles * kRouterKcCtas;
+    const int ctas = (int)row_tiles * kRouterKcCtas;
     if (p.k <= 8) CUDA_TRY(launch_router_kc(k_router_kc<8>, ctas, st, ax, bwn, a, npad));
     else CUDA_TRY(launch_router_kc(k_router_kc<16>, ctas, st, ax, bwn, a, npad));
     LAUNCH_CHECK("gemm_tc_router", st);

@@ -84,6 +84,40 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// The same bounded wait, polling with the non-blocking test_wait, for a
+// barrier whose phase is completed by bulk copies from another CTA of the
+// cluster: a thread suspended in try_wait on such a barrier was seen to resume
+// about 12 us after the copies had landed.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ bool mbar_wait_poll(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                               unsigned* status, unsigned where) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const long long lim = wait_limit();
+  const uint32_t mask = lim < kShortWaitLimit ? 0u : 255u;
+  const long long t0 = clock64();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((i & mask) == 0) {
+      if (*abort_flag) return false;
+      if (clock64() - t0 > lim) {
+        *abort_flag = 1;
+        atomicCAS(status, 0u, where);
+        return false;
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------- cp.async
 // 16 bytes global -> shared, L1 bypassed; bytes = 16 copies, 0 writes zeros
 // (and reads nothing).  The copy is a generic-proxy write: fence the async

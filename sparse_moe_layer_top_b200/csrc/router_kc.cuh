@@ -14,15 +14,16 @@
 // completing on the owner's mbarrier (the ring, idle after the main loop,
 // holds both); storing the partials into the peers' shared memory thread by
 // thread was slower (8 us for the exchange at the 35B shape, against 5).  c sums
-// the four K quarters in a fixed order, writes the sums back to TMEM and runs
-// the row-tiled router's top-k epilogue (topk_epilogue, tc_gemm.cuh) as
-// column tile c: the last of a row tile's owners to finish merges the lists
-// and writes ids, weights and the chunk histogram.
+// the four K quarters in a fixed order and selects the best KT (expert, logit)
+// pairs of each token among its experts; the owners' lists go to the row
+// tile's first CTA by bulk copies, which merges them (equal logits by expert)
+// and writes ids, softmax weights renormalised over the kept experts and the
+// chunk histogram.
 //
-// Every thread of every CTA passes the cluster barrier at the main loop's end,
-// also after a wait gave up, so no CTA waits on a peer that left; all
-// mbarrier waits are bounded, and a CTA leaves only once its own bulk copies
-// and those into it have completed.
+// Every thread of every CTA passes the cluster barriers (after the main loop,
+// after the owners' sums, before leaving -- once every CTA's bulk copies have
+// completed), also after a wait gave up, so no CTA waits on a peer that left
+// and no copy lands in a CTA that left; all mbarrier waits are bounded.
 //
 // Warps: 0 TMA producer; 1 TMEM owner and MMA issuer; 2..9 exchange and
 // top-k epilogue (two warps per TMEM lane quarter, splitting the columns).
@@ -43,7 +44,7 @@ struct RouterKcCfg {
   static constexpr int RING_BYTES = kRouterKcStages * kRouterKcStageBytes;
   static constexpr int BUF_BYTES =
       RING_BYTES > kRouterKcRecvBytes + kRouterKcSendBytes ? RING_BYTES : kRouterKcRecvBytes + kRouterKcSendBytes;
-  static constexpr int BAR_BYTES = (2 * kRouterKcStages + 2 + 8) * 8 + 16;
+  static constexpr int BAR_BYTES = (2 * kRouterKcStages + 2 + 4 + 2) * 8 + 16;
   static constexpr int SMEM_BYTES = 1024 + BUF_BYTES + BAR_BYTES;
   static constexpr int EPI_WARPS = 8;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
@@ -55,6 +56,60 @@ struct RouterKcCfg {
 // A 128 x 64 fp32 block, row r's 16-byte chunk j at chunk j ^ (r & 7): the
 // row-per-thread writes and reads of 8 consecutive rows hit distinct banks.
 __device__ __forceinline__ int kc_chunk(int r, int j) { return r * 16 + (j ^ (r & 7)); }
+
+// Sorting networks on (logit, expert) pairs held in registers, best first:
+// a pair is better with the larger logit, or the lower expert on equal logits
+// (the router's order).  Fixed, branch-free compare-exchanges: the inserts of
+// a sorted-list push are a dependent chain, which measured about 0.4 us per
+// pushed candidate per warp when merging lists.
+__device__ __forceinline__ bool kc_better(float av, int ae, float bv, int be) {
+  return av > bv || (av == bv && ae < be);
+}
+// after the call, slot a holds the better of the two
+__device__ __forceinline__ void kc_cmpx(float& av, int& ae, float& bv, int& be) {
+  const bool sw = kc_better(bv, be, av, ae);
+  const float tv = sw ? bv : av;
+  const int te = sw ? be : ae;
+  bv = sw ? av : bv;
+  be = sw ? ae : be;
+  av = tv;
+  ae = te;
+}
+// bitonic sort of N (a power of two) pairs, best first
+template <int N>
+__device__ __forceinline__ void kc_sort(float (&v)[N], int (&e)[N]) {
+#pragma unroll
+  for (int size = 2; size <= N; size <<= 1)
+#pragma unroll
+    for (int stride = size >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+      for (int i = 0; i < N; ++i) {
+        const int j = i ^ stride;
+        if (j > i) {
+          if ((i & size) == 0 || size == N) kc_cmpx(v[i], e[i], v[j], e[j]);
+          else kc_cmpx(v[j], e[j], v[i], e[i]);
+        }
+      }
+}
+// a (sorted, best first) <- the best N of a and b (sorted, best first): the
+// better of a[i] and b[N-1-i] are the best N, in a bitonic order that one
+// bitonic merge sorts
+template <int N>
+__device__ __forceinline__ void kc_merge(float (&av)[N], int (&ae)[N], const float (&bv)[N], const int (&be)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i)
+    if (kc_better(bv[N - 1 - i], be[N - 1 - i], av[i], ae[i])) {
+      av[i] = bv[N - 1 - i];
+      ae[i] = be[N - 1 - i];
+    }
+#pragma unroll
+  for (int stride = N >> 1; stride > 0; stride >>= 1)
+#pragma unroll
+    for (int i = 0; i < N; ++i) {
+      const int j = i ^ stride;
+      if (j > i) kc_cmpx(av[i], ae[i], av[j], ae[j]);
+    }
+}
 
 // tmX: the token matrix (box 64 x 128); tmW: W_r (box 64 x npad rows, npad =
 // E rounded up to 16).  p: N_s = E, K_s = d, rows_cap = T, and the TopK fields
@@ -72,9 +127,10 @@ __global__ void __launch_bounds__(RouterKcCfg::THREADS, 1)
   uint64_t* empty = full + S;
   uint64_t* tfull = empty + S;
   uint64_t* recv_full = tfull + 1;  // the three other K quarters of this CTA's experts have landed
-  uint64_t* hfull = recv_full + 1;  // [4] top-k hand-over, one pair per lane quarter
-  uint64_t* hempty = hfull + 4;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(hempty + 4);
+  uint64_t* hfull = recv_full + 1;  // [4] top-k hand-over, one per lane quarter
+  uint64_t* lst_ready = hfull + 4;  // this owner's token lists are staged (one arrival per list warp)
+  uint64_t* lists_full = lst_ready + 1;  // (rank 0) the other owners' token lists have landed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(lists_full + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   // after the main loop: recv [source rank] and send [owner slot] blocks, then
   // the hand-over lists over the send blocks
@@ -97,10 +153,9 @@ __global__ void __launch_bounds__(RouterKcCfg::THREADS, 1)
     }
     mbar_init(tfull, 1);
     mbar_init(recv_full, 1);
-    for (int q = 0; q < 4; ++q) {
-      mbar_init(hfull + q, 32);
-      mbar_init(hempty + q, 32);
-    }
+    for (int q = 0; q < 4; ++q) mbar_init(hfull + q, 32);
+    mbar_init(lst_ready, 4);
+    mbar_init(lists_full, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -227,12 +282,14 @@ __global__ void __launch_bounds__(RouterKcCfg::THREADS, 1)
     }
     named_bar_sync(1, 32 * Cfg::EPI_WARPS);
   }
+  // ---- owners: the four K quarters of this CTA's 64 experts, summed in rank
+  // order; warp eg holds columns 32 eg .. 32 eg + 31 of its 32 tokens
+  uint32_t v[32];
+  bool sel = false;  // (warp-uniform) this warp selects
   if (warp >= 2 && owner) {
-    const bool got = __all_sync(0xffffffffu, mbar_wait(recv_full, 0, abort_flag, p.status, tcode | 5));
-    if (got && acc_ok && !*abort_flag) {
-      // the four K quarters of this CTA's experts, summed in rank order; warp
-      // eg takes columns 32 eg .. 32 eg + 31, writes them to TMEM and selects
-      uint32_t v[32];
+    const bool got = __all_sync(0xffffffffu, mbar_wait_poll(recv_full, 0, abort_flag, p.status, tcode | 5));
+    sel = got && acc_ok && !*abort_flag;
+    if (sel) {
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
         float4 s = recv[kc_chunk(row, eg * 8 + j)];
@@ -249,28 +306,110 @@ __global__ void __launch_bounds__(RouterKcCfg::THREADS, 1)
         v[4 * j + 2] = __float_as_uint(s.z);
         v[4 * j + 3] = __float_as_uint(s.w);
       }
-      tmem_st32(tmem_base + lane_off + eg * 32, v);
-      tmem_wait_st();
-      TileInfo t{};
-      t.g = 0;
-      t.rows = (int)p.rows_cap;
-      t.m0 = rt * kBM;
-      t.row0 = t.m0;
-      t.n0 = (int)rank * 64;
-      t.N = p.N_s;
-      t.kb0 = 0;
-      t.kb1 = nkb;
-      const int64_t grow = t.row0 + row;
-      float* xv = reinterpret_cast<float*>(hand + q * 4096);
-      int* xe = reinterpret_cast<int*>(hand + q * 4096 + 2048);
-      topk_epilogue<64, 2, KT>(p, t, tmem_base + lane_off, eg, row, grow, grow < p.rows_cap, xv, xe, hfull + q,
-                               hempty + q, 0u, abort_flag, tcode | 9, lane);
     }
   }
-  if (warp == 2 && lane == 0) {
-    bulk_wait_all();                     // no copy of this CTA is in flight when it exits,
-    if (owner) drain_wait(recv_full, 0);  // nor one into it (bounded, also after a wait gave up)
+  // (C) every owner has read its receive blocks: rank 0's become the list buffer
+  cluster_sync_all();
+  const int list_bytes = KT * kBM * 8;  // an owner's lists: KT logits, then KT experts, per token
+  float* lst_v = reinterpret_cast<float*>(send) + 4096;  // staging, past the hand-over (send blocks are read)
+  int* lst_e = reinterpret_cast<int*>(lst_v + KT * kBM);
+  if (sel) {
+    // best KT of this warp's 32 experts (bias added; experts past E at -inf):
+    // groups of KT sorted, then merged
+    const int e0 = (int)rank * 64 + eg * 32;
+    float tv[KT], bv[KT];
+    int te[KT], be[KT];
+#pragma unroll
+    for (int gbase = 0; gbase < 32; gbase += KT) {
+      float* gv = gbase == 0 ? tv : bv;
+      int* ge = gbase == 0 ? te : be;
+#pragma unroll
+      for (int i = 0; i < KT; ++i) {
+        const int e = e0 + gbase + i;
+        ge[i] = e < p.N_s ? e : 0x7fffffff;
+        gv[i] = e < p.N_s ? __uint_as_float(v[gbase + i]) + (p.bias ? __ldg(p.bias + e) : 0.f) : -INFINITY;
+      }
+      if (gbase == 0) {
+        kc_sort<KT>(tv, te);
+      } else {
+        kc_sort<KT>(bv, be);
+        kc_merge<KT>(tv, te, bv, be);
+      }
+    }
+    // the second warp of a lane quarter hands its list to the first (its
+    // experts are all higher, which keeps the order of equal logits)
+    float* xv = reinterpret_cast<float*>(hand + q * 4096);
+    int* xe = reinterpret_cast<int*>(hand + q * 4096 + 2048);
+    if (eg) {
+#pragma unroll
+      for (int i = 0; i < KT; ++i) {
+        xv[i * 32 + lane] = tv[i];
+        xe[i * 32 + lane] = te[i];
+      }
+      mbar_arrive(hfull + q);
+    } else if (__all_sync(0xffffffffu, mbar_wait_poll(hfull + q, 0, abort_flag, p.status, tcode | 9))) {
+#pragma unroll
+      for (int i = 0; i < KT; ++i) {
+        bv[i] = xv[i * 32 + lane];
+        be[i] = xe[i * 32 + lane];
+      }
+      kc_merge<KT>(tv, te, bv, be);
+      if (rank != 0) {
+        // the owner's list of this token to rank 0's list buffer
+#pragma unroll
+        for (int i = 0; i < KT; ++i) {
+          lst_v[i * kBM + row] = tv[i];
+          lst_e[i * kBM + row] = te[i];
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(lst_ready);
+        if (warp == 2 && lane == 0 &&
+            mbar_wait_poll(lst_ready, 0, abort_flag, p.status, tcode | 10))
+          bulk_copy_to_cta(mapa_rank(reinterpret_cast<float*>(recv) + (int)rank * (KT * kBM * 2), 0u), lst_v,
+                           (uint32_t)list_bytes, mapa_rank(lists_full, 0u));
+      } else {
+        // rank 0: merge the other owners' lists (higher experts) and write
+        if (warp == 2 && lane == 0 && owners > 1)
+          mbar_arrive_expect_tx(lists_full, (uint32_t)((owners - 1) * list_bytes));
+        const bool have = owners == 1 ||
+                          __all_sync(0xffffffffu, mbar_wait_poll(lists_full, 0, abort_flag, p.status, tcode | 11));
+        if (have) {
+          const float* rv = reinterpret_cast<const float*>(recv);
+          for (int o = 1; o < owners; ++o) {
+            const float* ov = rv + o * (KT * kBM * 2);
+            const int* oe = reinterpret_cast<const int*>(ov + KT * kBM);
+#pragma unroll
+            for (int i = 0; i < KT; ++i) {
+              bv[i] = ov[i * kBM + row];
+              be[i] = oe[i * kBM + row];
+            }
+            kc_merge<KT>(tv, te, bv, be);
+          }
+          const int64_t grow = (int64_t)rt * kBM + row;
+          if (grow < p.rows_cap) {
+            const float m = tv[0];
+            float den = 0.f;
+#pragma unroll
+            for (int i = 0; i < KT; ++i)
+              if (i < p.topk) den += __expf(tv[i] - m);
+            int32_t* hist = p.counts ? p.counts + (grow / kBM) * p.N_s : nullptr;
+#pragma unroll
+            for (int i = 0; i < KT; ++i)
+              if (i < p.topk) {
+                p.ids[grow * p.topk + i] = te[i];
+                p.tw[grow * p.topk + i] = __expf(tv[i] - m) / den;
+                if (hist) atomicAdd(hist + te[i], 1);
+              }
+          }
+        }
+      }
+    }
   }
+  // (D) every CTA's bulk copies have completed: none is in flight into a CTA
+  // that leaves
+  if (warp == 2 && lane == 0) bulk_wait_all();
+  cluster_sync_all();
 
   tc_fence_before();
   __syncthreads();

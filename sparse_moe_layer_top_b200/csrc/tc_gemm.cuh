@@ -24,8 +24,8 @@
 //                           applied and the row put back in (token, slot) order
 //                 Store     out[r, n] = D -> bf16
 //                 Logits    part[split][r, n] = D (+ nothing) -> fp32
-//               (the router's top-k selection from TMEM, topk_epilogue below,
-//               runs in the K-split router of router_kc.cuh)
+//               (the router that selects its top k in the epilogue is the
+//               K-split kernel of router_kc.cuh)
 //   warps 10..13 (GATHER only) fetch the A rows straight from the token
 //               matrix by row index (cp.async, 128-byte swizzle written by
 //               hand): the gate/up GEMM of the fused forward needs no
@@ -50,7 +50,7 @@ namespace moe {
 constexpr int kBM = 128;
 constexpr int kBK = 64;  // 64 bf16 = one 128-byte swizzle row
 
-enum { kTcSwiGLU = 0, kTcSlotStore = 1, kTcStore = 2, kTcLogits = 3, kTcTopK = 4 };
+enum { kTcSwiGLU = 0, kTcSlotStore = 1, kTcStore = 2, kTcLogits = 3 };
 
 struct TcGemmArgs {
   const int32_t* offs;    // [E+2] group row starts (grouped mode)
@@ -75,21 +75,15 @@ struct TcGemmArgs {
   int64_t ldo;
   float* part;            // Logits output [ksplit][rows, ldp]
   int64_t ldp, part_stride;
-  // top-k selection (topk_epilogue): topk_ids / topk_w [rows, topk] and the
-  // 128-row chunk histograms counts[rows / 128][N_s] (may be NULL); bias [N_s]
-  // fp32 (may be NULL) is added to the logits
+  // the router's top-k selection (router_kc.cuh): topk_ids / topk_w [rows,
+  // topk] and the 128-row chunk histograms counts[rows / 128][N_s] (may be
+  // NULL; zeroed before the launch); bias [N_s] fp32 (may be NULL) is added to
+  // the logits
   int topk;
   int32_t* ids;
   float* tw;
   const float* bias;
   int32_t* counts;
-  // selection over several column tiles: each tile's kept (logit, expert) pairs of a
-  // token go to cand_v / cand_e [row tile][column tile][kMaxK slots][kBM rows];
-  // cand_cnt [row tile][4 lane quarters] (zeroed before the launch) counts the
-  // tiles done, and the last one merges the lists and writes the outputs
-  float* cand_v;
-  int32_t* cand_e;
-  int32_t* cand_cnt;
   // Tile order (bf16 kernels): NULL = CTA c takes tiles c, c + grid, ...;
   // else a counter (zeroed by whoever wrote `prefix`) from which a CTA claims
   // each tile after its first, so CTAs that draw cheap tiles draw more.
@@ -231,9 +225,8 @@ struct TcGemmCfg {
   static constexpr int THREADS = FP8 ? 192 + NB + 32 : 64 + 32 * (EPI_WARPS + GATHER_WARPS);
   static constexpr int ACC_COLS = DUAL ? 2 * BN : BN;
   static constexpr int TMEM_COLS = 2 * ACC_COLS;
-  // + 4 + 4 handoff barriers of the router epilogue (one pair per lane quarter)
   // + 4 + 4 barriers and 4 ints of the tile queue
-  static constexpr int BAR_BYTES = (3 * STAGES + 2 * RAW_STAGES + 5 + 8 + 8) * 8 + 16 + 16;
+  static constexpr int BAR_BYTES = (3 * STAGES + 2 * RAW_STAGES + 5 + 8) * 8 + 16 + 16;
   static constexpr int SCHED_INTS = 2 * (512 + 2);  // tile prefix + group offsets, E <= 512
   // epilogue staging: 32 rows x 64 bytes per epilogue warp
   static constexpr int EPI_OFF = (RING_BYTES + BAR_BYTES + SCHED_INTS * 4 + 127) / 128 * 128;
@@ -483,163 +476,6 @@ __device__ __forceinline__ void epilogue_swapped(const TcGemmArgs& p, const Tile
   }
 }
 
-// Push (v, e) into a list of KT (logit, expert) pairs sorted by logit, larger
-// first; the last pair drops out.  Empty slots hold (-inf, INT_MAX).
-// Candidates arrive in increasing expert order, so a strict comparison keeps
-// the lower expert first among equal logits (the selection order of the
-// router).  The list is sorted, so "v beats slot i" is monotone in i: every
-// slot is compared at once and shifted by selects, with one branch that skips
-// values below the last kept one.
-template <int KT>
-__device__ __forceinline__ void topk_push(float (&tv)[KT], int (&te)[KT], float v, int e) {
-  if (!(v > tv[KT - 1])) return;
-#pragma unroll
-  for (int i = KT - 1; i > 0; --i) {
-    const bool here = v > tv[i], above = v > tv[i - 1];
-    tv[i] = above ? tv[i - 1] : (here ? v : tv[i]);
-    te[i] = above ? te[i - 1] : (here ? e : te[i]);
-  }
-  if (v > tv[0]) {
-    tv[0] = v;
-    te[0] = e;
-  }
-}
-
-// The same for candidates in any expert order: equal logits compare by
-// expert, lower first.
-template <int KT>
-__device__ __forceinline__ void topk_push_lex(float (&tv)[KT], int (&te)[KT], float v, int e) {
-#pragma unroll
-  for (int i = KT - 1; i > 0; --i) {
-    const bool here = v > tv[i] || (v == tv[i] && e < te[i]);
-    const bool above = v > tv[i - 1] || (v == tv[i - 1] && e < te[i - 1]);
-    tv[i] = above ? tv[i - 1] : (here ? v : tv[i]);
-    te[i] = above ? te[i - 1] : (here ? e : te[i]);
-  }
-  if (v > tv[0] || (v == tv[0] && e < te[0])) {
-    tv[0] = v;
-    te[0] = e;
-  }
-}
-
-// Router epilogue: softmax top-k of each token's logits, read from TMEM.
-// With EG = 2 warps per lane quarter, warp eg scans columns [eg*BN/2,
-// (eg+1)*BN/2) of its 32 tokens; the second hands its KT best to the first
-// through shared memory (xv/xe, slot-major so lanes hit distinct banks) under
-// a bounded mbarrier handshake (hfull / hempty, 32 arrivals each), and the
-// first merges them -- all of them come from higher experts, which keeps the
-// order of equal logits.  With the experts over several column tiles, the
-// first warp then stores its list (cand_v / cand_e) and counts itself in; the
-// warp that completes a row tile's count merges the other tiles' lists into
-// its own, comparing equal logits by expert -- a last-arriver merge, so no
-// warp waits for another CTA.  The merging warp writes the top k, their
-// softmax weights renormalised over the kept experts and the chunk histogram.
-// Returns false when a wait gave up (the caller stops).
-template <int BN, int EG, int KT>
-__device__ __forceinline__ bool topk_epilogue(const TcGemmArgs& p, const TileInfo& t, uint32_t tb, int eg, int row,
-                                              int64_t grow, bool valid, float* xv, int* xe, uint64_t* hfull,
-                                              uint64_t* hempty, uint32_t hpar, volatile int* abort_flag,
-                                              unsigned where, int lane) {
-  float tv[KT];
-  int te[KT];
-#pragma unroll
-  for (int i = 0; i < KT; ++i) {
-    tv[i] = -INFINITY;
-    te[i] = 0x7fffffff;
-  }
-  constexpr int CW = BN / EG;  // columns per warp
-  const int c0 = eg * CW;
-  uint32_t a[8], nx[8];
-  tmem_ld8(tb + c0, a);
-  tmem_wait_regs(a);
-#pragma unroll 1
-  for (int c = c0; c < c0 + CW; c += 8) {
-    if (c + 8 < c0 + CW) tmem_ld8(tb + c + 8, nx);  // next 8 columns land while these are scanned
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = t.n0 + c + j;
-      const float v = e < t.N ? __uint_as_float(a[j]) + (p.bias ? __ldg(p.bias + e) : 0.f) : -INFINITY;
-      topk_push(tv, te, v, e);
-    }
-    if (c + 8 < c0 + CW) {
-      tmem_wait_regs(nx);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) a[j] = nx[j];
-    }
-  }
-  if (EG == 2) {
-    const bool ok = eg ? mbar_wait(hempty, hpar ^ 1, abort_flag, p.status, where)
-                       : mbar_wait(hfull, hpar, abort_flag, p.status, where);
-    if (!__all_sync(0xffffffffu, ok)) return false;
-    if (eg) {
-#pragma unroll
-      for (int i = 0; i < KT; ++i) {
-        xv[i * 32 + lane] = tv[i];
-        xe[i * 32 + lane] = te[i];
-      }
-      mbar_arrive(hfull);
-      return true;
-    }
-#pragma unroll
-    for (int i = 0; i < KT; ++i) topk_push(tv, te, xv[i * 32 + lane], xe[i * 32 + lane]);
-    mbar_arrive(hempty);
-  }
-  const int ntc = (t.N + BN - 1) / BN;
-  if (ntc > 1) {
-    const int rt = t.m0 / kBM;
-    const int64_t tile_base = (int64_t)rt * ntc * (kMaxK * kBM) + row;
-    const int64_t mine = tile_base + (int64_t)(t.n0 / BN) * (kMaxK * kBM);
-#pragma unroll
-    for (int i = 0; i < KT; ++i) {
-      p.cand_v[mine + i * kBM] = tv[i];
-      p.cand_e[mine + i * kBM] = te[i];
-    }
-    __threadfence();  // the lists are visible before the count that publishes them
-    __syncwarp();
-    int last = 0;
-    if (lane == 0) last = atomicAdd(p.cand_cnt + rt * 4 + (row >> 5), 1) == ntc - 1;
-    if (!__shfl_sync(0xffffffffu, last, 0)) return true;
-    __threadfence();
-    // merge the other tiles' lists into this one's (lexicographic order, so
-    // any tile order gives the same list)
-    const int mine_c = t.n0 / BN;
-#pragma unroll 1
-    for (int c = 0; c < ntc; ++c) {
-      if (c == mine_c) continue;
-      const int64_t o = tile_base + (int64_t)c * (kMaxK * kBM);
-      float cv[KT];
-      int ce[KT];
-#pragma unroll
-      for (int i = 0; i < KT; ++i) {  // the whole list in flight at once
-        cv[i] = __ldcg(p.cand_v + o + i * kBM);
-        ce[i] = __ldcg(p.cand_e + o + i * kBM);
-      }
-      // a list is sorted: once no lane keeps an entry, none keeps a later one
-#pragma unroll
-      for (int i = 0; i < KT; ++i) {
-        if (!__any_sync(0xffffffffu, cv[i] > tv[KT - 1] || (cv[i] == tv[KT - 1] && ce[i] < te[KT - 1]))) break;
-        topk_push_lex(tv, te, cv[i], ce[i]);
-      }
-    }
-  }
-  if (valid) {
-    const float v0 = tv[0];
-    float den = 0.f;
-#pragma unroll
-    for (int i = 0; i < KT; ++i)
-      if (i < p.topk) den += __expf(tv[i] - v0);
-    int32_t* hist = p.counts ? p.counts + (grow / kBM) * t.N : nullptr;
-#pragma unroll
-    for (int i = 0; i < KT; ++i)
-      if (i < p.topk) {
-        p.ids[grow * p.topk + i] = te[i];
-        p.tw[grow * p.topk + i] = __expf(tv[i] - v0) / den;
-        if (hist) atomicAdd(hist + te[i], 1);
-      }
-  }
-  return true;
-}
-
 // A CTA's tile sequence (bf16 kernels), handed from the producer thread to the
 // other roles through a 4-slot ring in shared memory: the producer puts each
 // tile (a value >= total ends the sequence); every consumer role takes them in
@@ -698,9 +534,7 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
   uint64_t* drain = tempty + 2;
   uint64_t* raw_full = drain + 1;        // FP8: raw weight tile landed
   uint64_t* raw_empty = raw_full + Cfg::RAW_STAGES;  // FP8: raw tile converted
-  uint64_t* hfull = raw_empty + Cfg::RAW_STAGES;  // router epilogue: second warp's list written
-  uint64_t* hempty = hfull + 4;                    // router epilogue: list merged, slot free
-  uint64_t* tq_full = hempty + 4;                  // tile queue (bf16 kernels)
+  uint64_t* tq_full = raw_empty + Cfg::RAW_STAGES;  // tile queue (bf16 kernels)
   uint64_t* tq_empty = tq_full + 4;
   int* tq_id = reinterpret_cast<int*>(tq_empty + 4);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tq_id + 4);
@@ -728,8 +562,6 @@ __global__ void __launch_bounds__(TcGemmCfg<BN, DUAL, STAGES, FP8, GATHER>::THRE
     }
     mbar_init(drain, 1);
     for (int q = 0; q < 4; ++q) {
-      mbar_init(hfull + q, 32);
-      mbar_init(hempty + q, 32);
       mbar_init(tq_full + q, 1);
       mbar_init(tq_empty + q, 1 + Cfg::EPI_WARPS + Cfg::GATHER_WARPS);  // MMA thread + each consumer warp
     }
