@@ -74,6 +74,11 @@ FORWARD_CASES = {
 ROUTER_ONLY = {
     # the fused router at the 35B-shaped expert count, k = 8, ragged last tile
     "bf16_fused_router_E256": (2100, 512, 256, 8, 64, 64, "bf16", "bf16", None),
+    # 16-slot lists (k = 12), three expert owners of the last one partial, and a
+    # K of 2048 split four ways (8 K blocks per CTA of the cluster)
+    "bf16_fused_router_k12": (2048, 2048, 160, 12, 64, 64, "bf16", "bf16", "zipf"),
+    # E <= 64: one owner, no list exchange
+    "bf16_fused_router_E48": (1921, 1024, 48, 5, 64, 64, "bf16", "bf16", None),
 }
 
 
@@ -122,7 +127,8 @@ def test_forward_matches_oracle(moe, case, path):
 
 
 @pytest.mark.parametrize("case", ["tiny_fp32", "bf16_multi_tile", "bf16_E512_k10", "bf16_zipf", "bf16_T1",
-                                  "bf16_fused_router", "bf16_fused_router_E256"])
+                                  "bf16_fused_router", "bf16_fused_router_E256", "bf16_fused_router_k12",
+                                  "bf16_fused_router_E48"])
 def test_router_matches_oracle(moe, case):
     inp = _make(case)
     g = to_device(inp, "cuda")
