@@ -63,7 +63,7 @@ extern "C" {
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1,          /* a size, pointer or type is not allowed */
-  MOE_ERR_UNSUPPORTED = 2,          /* a valid combination this build does not implement */
+  MOE_ERR_UNSUPPORTED = 2,          /* a valid combination the library does not implement */
   MOE_ERR_ALIGNMENT = 3,            /* a pointer or a row stride is not 16-byte aligned */
   MOE_ERR_WORKSPACE_TOO_SMALL = 4,  /* ws_bytes below the *_workspace_size() figure */
   MOE_ERR_CUDA = 5,                 /* a CUDA runtime call or a launch failed */
