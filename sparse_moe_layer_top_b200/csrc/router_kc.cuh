@@ -177,7 +177,10 @@ __global__ void __launch_bounds__(RouterKcCfg::THREADS, 1)
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------ TMA producer: this CTA's K quarter
-      const uint64_t pol_x = policy_evict_first(), pol_w = policy_evict_last();
+      // both stay in L2: W_r serves every row tile, and the gate/up GEMM that
+      // follows gathers its rows from x (evict-first here made it about 3 %
+      // slower at the 35B shape)
+      const uint64_t pol_x = policy_evict_last(), pol_w = policy_evict_last();
       const uint32_t tx = (uint32_t)(kBM * kBK * 2 + npad * kBK * 2);
       int stage = 0;
       uint32_t phase = 0, issued = 0, last_par = 0;
