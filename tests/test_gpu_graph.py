@@ -10,11 +10,14 @@ import moe_inputs
 pytestmark = pytest.mark.gpu
 
 
-# (path, weights, E, T, bias); path 5 (split) on Zipf-skewed groups runs its
-# CTA-pair and weight-row GEMMs on two streams: the capture forks and joins
+# (path, weights, E, T, bias); path 5 (split) on Zipf-skewed groups launches
+# a CTA-pair and a weight-row GEMM per projection; path 6 the token-N CTA-pair
+# GEMMs; T = 2048 with E = 24 takes the router that selects in its epilogue
+# (4-CTA clusters exchanging partials by bulk copies)
 @pytest.mark.parametrize("path,w,E,T,bias", [(2, "bf16", 20, 300, None), (3, "bf16", 64, 300, None),
                                              (4, "bf16", 2, 2048, None), (0, "fp8", 12, 300, None),
-                                             (5, "bf16", 24, 1536, "zipf")])
+                                             (5, "bf16", 24, 1536, "zipf"), (6, "bf16", 24, 1536, "zipf"),
+                                             (0, "bf16", 24, 2048, "zipf")])
 def test_forward_replays_from_a_cuda_graph(path, w, E, T, bias):
     import sparse_moe_layer_top_b200 as moe
     d, k, I, I_s = (256, 2, 256, 128) if E == 2 else (384, 3, 256, 128)
